@@ -1,0 +1,227 @@
+// C ABI of libgenrank: host-side argument checks and dispatch to the kernels.
+// Declarations and argument documentation live in include/genrank.h.
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace gr;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int elem_size(int dtype) { return dtype == GENRANK_BF16 ? 2 : (dtype == GENRANK_F32 ? 4 : 0); }
+
+bool fill_attn(AttnArgs& a, int B, int64_t T, const int32_t* off, const int32_t* hl,
+               int max_seqlen, const void* q, const void* k, const void* v, int64_t tok_stride,
+               int H, int dh, const int32_t* pos, const int64_t* ts, const float* sp,
+               const float* st, float scale, int dtype, int64_t o_stride, int32_t* err) {
+  memset(&a, 0, sizeof(a));
+  a.B = B;
+  a.T = T;
+  a.off = off;
+  a.hist_len = hl;
+  a.max_seqlen = max_seqlen;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.tok_stride = tok_stride;
+  a.H = H;
+  a.dh = dh;
+  a.pos = pos;
+  a.ts = ts;
+  for (int h = 0; h < H; ++h) {
+    a.slope_pos[h] = sp[h];
+    a.slope_time[h] = st[h];
+  }
+  a.scale = scale;
+  a.dtype = dtype;
+  a.o_stride = o_stride;
+  a.err = err;
+  return true;
+}
+
+int check_attn_common(int B, int64_t T, const int32_t* off, const int32_t* hl, int max_seqlen,
+                      const void* q, const void* k, const void* v, int64_t tok_stride, int H,
+                      int dh, const int32_t* pos, const int64_t* ts, const float* sp,
+                      const float* st, float scale, int dtype, int64_t o_stride,
+                      int32_t* err) {
+  if (B < 1 || T < 0 || max_seqlen < 0 || H < 1 || dh < 1 || !off || !hl || !pos || !ts ||
+      !sp || !st || !err || !(scale > 0.f) || !isfinite(scale))
+    return GENRANK_ERR_INVALID_ARG;
+  if (T > 0 && (!q || !k || !v)) return GENRANK_ERR_INVALID_ARG;
+  if (H > kMaxHeads) return GENRANK_ERR_UNSUPPORTED;
+  const int es = elem_size(dtype);
+  if (!es) return GENRANK_ERR_INVALID_ARG;
+  if (tok_stride < (int64_t)H * dh || o_stride < (int64_t)H * dh) return GENRANK_ERR_INVALID_ARG;
+  if ((tok_stride * es) % 16 || (o_stride * es) % 16 || (dh * es) % 16)
+    return GENRANK_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return GENRANK_ERR_INVALID_ARG;
+  for (int h = 0; h < H; ++h)
+    if (!isfinite(sp[h]) || !isfinite(st[h]) || sp[h] < 0.f || st[h] < 0.f)
+      return GENRANK_ERR_INVALID_ARG;
+  return GENRANK_OK;
+}
+
+bool use_tc(int dtype, int dh) { return dtype == GENRANK_BF16 && dh == 64; }
+
+}  // namespace
+
+extern "C" {
+
+const char* genrank_status_string(int code) {
+  switch (code) {
+    case GENRANK_OK: return "ok";
+    case GENRANK_ERR_INVALID_ARG: return "invalid argument";
+    case GENRANK_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case GENRANK_ERR_WORKSPACE: return "workspace missing or too small";
+    case GENRANK_ERR_LAUNCH: return "kernel launch failed";
+    case GENRANK_ERR_CUDA: return "CUDA call failed";
+    default: return "unknown status";
+  }
+}
+
+const char* genrank_device_error_string(int bit) {
+  switch (bit) {
+    case 0: return "clean";
+    case GENRANK_DERR_LAYOUT: return "device: bad seq_offsets/hist_len layout";
+    case GENRANK_DERR_ITEM_ID: return "device: item id out of range";
+    case GENRANK_DERR_ACTION_ID: return "device: action id out of range";
+    case GENRANK_DERR_TS_ORDER: return "device: timestamps out of order";
+    case GENRANK_DERR_POS_RANGE: return "device: position beyond the position table";
+    case GENRANK_DERR_INDEX: return "device: metadata index out of range";
+    case GENRANK_DERR_TIMEOUT: return "device: bounded wait timed out";
+    default: return "several or unknown device error bits";
+  }
+}
+
+int genrank_check_error(const int32_t* dev_err, genrank_stream_t stream) {
+  if (!dev_err) return -GENRANK_ERR_INVALID_ARG;
+  int32_t h = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, dev_err, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return -GENRANK_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return -GENRANK_ERR_CUDA;
+  return h;
+}
+
+int genrank_alibi_slopes(int H, float* slope_pos, float* slope_time) {
+  if (H < 1 || !slope_pos || !slope_time) return GENRANK_ERR_INVALID_ARG;
+  for (int h = 0; h < H; ++h) {
+    const double m = exp2(-8.0 * (h + 1) / (double)H);
+    slope_pos[h] = (float)m;
+    slope_time[h] = (float)(m / 3600.0);
+  }
+  return GENRANK_OK;
+}
+
+int genrank_embed_assemble(int B, int64_t T, const int32_t* seq_offsets, const int32_t* hist_len,
+                           const int32_t* item_ids, const int32_t* action_ids, const int64_t* ts,
+                           const void* item_tab, int64_t n_item, const void* action_tab,
+                           int n_action, const void* pos_tab, int n_pos, const void* ri_tab,
+                           int n_ri, const void* rt_tab, int n_rt, int d, int dtype, void* E,
+                           int32_t* pos, int32_t* req_idx, int32_t* rt_bucket, int32_t* dev_err,
+                           genrank_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (B < 1 || T < 0 || !seq_offsets || !hist_len || !dev_err || !es || d < 1)
+    return GENRANK_ERR_INVALID_ARG;
+  if (n_item < 1 || n_action < 1 || n_pos < 2 || n_ri < 2 || n_rt < 2)
+    return GENRANK_ERR_INVALID_ARG;
+  if (n_rt > 65) return GENRANK_ERR_UNSUPPORTED;
+  if (((int64_t)d * es) % 16) return GENRANK_ERR_INVALID_ARG;
+  if (T > 0 && (!item_ids || !action_ids || !ts || !item_tab || !action_tab || !pos_tab ||
+                !ri_tab || !rt_tab || !E || !pos || !req_idx || !rt_bucket))
+    return GENRANK_ERR_INVALID_ARG;
+  if (!aligned16(item_tab) || !aligned16(action_tab) || !aligned16(pos_tab) ||
+      !aligned16(ri_tab) || !aligned16(rt_tab) || !aligned16(E))
+    return GENRANK_ERR_INVALID_ARG;
+  EmbedFwdArgs a{B, T, seq_offsets, hist_len, item_ids, action_ids, ts, item_tab, n_item,
+                 action_tab, n_action, pos_tab, n_pos, ri_tab, n_ri, rt_tab, n_rt, d, dtype,
+                 E, pos, req_idx, rt_bucket, dev_err};
+  return launch_embed_fwd(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int genrank_embed_assemble_bwd(int B, int64_t T, const int32_t* seq_offsets,
+                               const int32_t* hist_len, const int32_t* item_ids,
+                               const int32_t* action_ids, const int32_t* pos,
+                               const int32_t* req_idx, const int32_t* rt_bucket, const void* dE,
+                               int d, int dtype, float* d_item, int64_t n_item, float* d_action,
+                               int n_action, float* d_pos, int n_pos, float* d_ri, int n_ri,
+                               float* d_rt, int n_rt, int32_t* dev_err, genrank_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (B < 1 || T < 0 || !seq_offsets || !hist_len || !dev_err || !es || d < 2 || (d & 1))
+    return GENRANK_ERR_INVALID_ARG;
+  if (n_item < 1 || n_action < 1 || n_pos < 1 || n_ri < 1 || n_rt < 1)
+    return GENRANK_ERR_INVALID_ARG;
+  if (T > 0 && (!item_ids || !action_ids || !pos || !req_idx || !rt_bucket || !dE || !d_item ||
+                !d_action || !d_pos || !d_ri || !d_rt))
+    return GENRANK_ERR_INVALID_ARG;
+  EmbedBwdArgs a{B, T, seq_offsets, hist_len, item_ids, action_ids, pos, req_idx, rt_bucket, dE,
+                 d, dtype, d_item, n_item, d_action, n_action, d_pos, n_pos, d_ri, n_ri, d_rt,
+                 n_rt, dev_err};
+  return launch_embed_bwd(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t genrank_attn_workspace_size(int B, int64_t T, int H, int dh, int max_seqlen, int is_bwd) {
+  if (B < 1 || T < 0 || H < 1 || dh < 1 || max_seqlen < 0) return 0;
+  if (is_bwd) return attn_bwd_simt_workspace(B, T, H, dh, max_seqlen);
+  return attn_fwd_tc_workspace(B, T, H, max_seqlen);
+}
+
+int genrank_attn_fwd(int B, int64_t T, const int32_t* seq_offsets, const int32_t* hist_len,
+                     int max_seqlen, const void* q, const void* k, const void* v,
+                     int64_t tok_stride, int H, int dh, const int32_t* pos, const int64_t* ts,
+                     const float* slope_pos, const float* slope_time, float scale, int dtype,
+                     void* o, int64_t o_stride, float* lse, void* ws, size_t ws_bytes,
+                     int32_t* dev_err, genrank_stream_t stream) {
+  int rc = check_attn_common(B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh,
+                             pos, ts, slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  if (rc) return rc;
+  if (T > 0 && (!o || !aligned16(o))) return GENRANK_ERR_INVALID_ARG;
+  if (!use_tc(dtype, dh) && dh != 32 && dh != 64) return GENRANK_ERR_UNSUPPORTED;
+  const size_t need = genrank_attn_workspace_size(B, T, H, dh, max_seqlen, 0);
+  if (use_tc(dtype, dh) && (!ws || ws_bytes < need || !aligned16(ws))) return GENRANK_ERR_WORKSPACE;
+  if (T == 0) return GENRANK_OK;
+  AttnArgs a;
+  fill_attn(a, B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts,
+            slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  a.o = o;
+  a.lse = lse;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return use_tc(dtype, dh) ? launch_attn_fwd_tc(a, s) : launch_attn_fwd_simt(a, s);
+}
+
+int genrank_attn_bwd(int B, int64_t T, const int32_t* seq_offsets, const int32_t* hist_len,
+                     int max_seqlen, const void* q, const void* k, const void* v,
+                     int64_t tok_stride, int H, int dh, const int32_t* pos, const int64_t* ts,
+                     const float* slope_pos, const float* slope_time, float scale, int dtype,
+                     const void* o, const void* dO, int64_t o_stride, const float* lse, void* dq,
+                     void* dk, void* dv, void* ws, size_t ws_bytes, int32_t* dev_err,
+                     genrank_stream_t stream) {
+  int rc = check_attn_common(B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh,
+                             pos, ts, slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  if (rc) return rc;
+  if (T > 0 && (!o || !dO || !lse || !dq || !dk || !dv)) return GENRANK_ERR_INVALID_ARG;
+  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return GENRANK_ERR_INVALID_ARG;
+  if (dh != 32 && dh != 64) return GENRANK_ERR_UNSUPPORTED;
+  const size_t need = genrank_attn_workspace_size(B, T, H, dh, max_seqlen, 1);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return GENRANK_ERR_WORKSPACE;
+  if (T == 0) return GENRANK_OK;
+  AttnArgs a;
+  fill_attn(a, B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts,
+            slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  a.o = const_cast<void*>(o);
+  a.dO = dO;
+  a.lse_in = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  return launch_attn_bwd_simt(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,382 @@
+// Action-oriented input assembly: per-token metadata and the five-way embedding
+// gather-sum (forward), and its scatter-add backward.
+//
+// "GenRank [2025]" chapter notes (huaxiaozhuan.com), §1.4.1 and §1.4.2: a token
+// is psi(x_i) + phi(a_i) (candidates: psi(x_j) + m, the mask action), plus the
+// position embedding (candidates of one request share position n + 1), the
+// request-index embedding |{t_1..t_i}| and the pre-request time embedding
+// bucket(t_i - max_{t_j < t_i} t_j).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gr {
+
+// ------------------------------------------------------------------------------------------
+// block scans (inclusive) over blockDim.x <= 1024 threads
+// ------------------------------------------------------------------------------------------
+template <bool kMax>
+__device__ int block_scan(int v, int* sh /* >= 32 ints */) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int x = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v = kMax ? max(v, x) : v + x;
+  }
+  if (lane == 31) sh[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? sh[lane] : (kMax ? -2147483647 : 0);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int x = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w = kMax ? max(w, x) : w + x;
+    }
+    sh[lane] = w;
+  }
+  __syncthreads();
+  if (warp > 0) v = kMax ? max(v, sh[warp - 1]) : v + sh[warp - 1];
+  __syncthreads();
+  return v;
+}
+
+// One block per user.  History tokens are scanned in chunks of blockDim.x with
+// the request count and the current group start carried across chunks.
+__global__ void __launch_bounds__(256) k_token_meta(
+    int B, long long T, const int32_t* __restrict__ off, const int32_t* __restrict__ hist_len,
+    const int64_t* __restrict__ ts, int n_pos, int n_ri, int n_rt, int32_t* __restrict__ pos,
+    int32_t* __restrict__ req_idx, int32_t* __restrict__ rt_bucket, int32_t* err) {
+  __shared__ int sh[32];
+  __shared__ int carry_cnt, carry_gs;
+  const int u = blockIdx.x;
+  long long s = off[u], e = off[u + 1];
+  int n = hist_len[u];
+  if (s < 0 || e < s || e > T) {
+    if (threadIdx.x == 0) flag(err, GENRANK_DERR_LAYOUT);
+    return;
+  }
+  const int L = (int)(e - s);
+  if (n < 0 || n > L) {
+    if (threadIdx.x == 0) flag(err, GENRANK_DERR_LAYOUT);
+    n = max(0, min(n, L));
+  }
+  if (threadIdx.x == 0) {
+    carry_cnt = 0;
+    carry_gs = 0;
+  }
+  __syncthreads();
+  for (int c0 = 0; c0 < n; c0 += blockDim.x) {
+    const int i = c0 + threadIdx.x;
+    const bool valid = i < n;
+    long long t = valid ? ts[s + i] : 0;
+    long long tp = (valid && i > 0) ? ts[s + i - 1] : t;
+    int is_new = valid && (i == 0 || t != tp);
+    if (valid && i > 0 && t < tp) flag(err, GENRANK_DERR_TS_ORDER);
+    const int cc = carry_cnt, cg = carry_gs;
+    int cnt = block_scan<false>(is_new, sh) + cc;
+    int gs = max(block_scan<true>(is_new ? i : 0, sh), cg);
+    if (valid) {
+      int p = i + 1;
+      if (p >= n_pos) {
+        flag(err, GENRANK_DERR_POS_RANGE);
+        p = n_pos - 1;
+      }
+      pos[s + i] = p;
+      req_idx[s + i] = min(cnt, n_ri - 1);
+      rt_bucket[s + i] = gs > 0 ? time_bucket(t - ts[s + gs - 1], n_rt) : 0;
+    }
+    const int last = min(c0 + (int)blockDim.x, n) - 1;
+    if (i == last) {
+      carry_cnt = cnt;
+      carry_gs = gs;
+    }
+    __syncthreads();
+  }
+  if (L > n) {
+    const long long t_req = ts[s + n];
+    const long long tl = n > 0 ? ts[s + n - 1] : t_req;
+    if (threadIdx.x == 0 && n > 0 && t_req < tl) flag(err, GENRANK_DERR_TS_ORDER);
+    const bool new_req = (n == 0) || (t_req > tl);
+    const int cnt = carry_cnt + (new_req ? 1 : 0);
+    const int gs = new_req ? n : carry_gs;
+    const int b = gs > 0 ? time_bucket(t_req - ts[s + gs - 1], n_rt) : 0;
+    int p = n + 1;
+    if (p >= n_pos) {
+      if (threadIdx.x == 0) flag(err, GENRANK_DERR_POS_RANGE);
+      p = n_pos - 1;
+    }
+    for (int i = n + threadIdx.x; i < L; i += blockDim.x) {
+      if (ts[s + i] != t_req) flag(err, GENRANK_DERR_TS_ORDER);
+      pos[s + i] = p;
+      req_idx[s + i] = min(cnt, n_ri - 1);
+      rt_bucket[s + i] = b;
+    }
+  }
+}
+
+// Warp-per-token gather-sum.  Each warp owns a contiguous run of tokens, finds
+// the user of its first token with a 32-way search of seq_offsets, then walks
+// forward.  Rows are moved as 16-byte vectors; the five rows are summed in fp32
+// and rounded once.
+template <typename T>
+__global__ void __launch_bounds__(256) k_embed_fwd(
+    int B, long long Ttok, const int32_t* __restrict__ off, const int32_t* __restrict__ hist_len,
+    const int32_t* __restrict__ item_ids, const int32_t* __restrict__ action_ids,
+    const T* __restrict__ item_tab, long long n_item, const T* __restrict__ action_tab,
+    int n_action, const T* __restrict__ pos_tab, const T* __restrict__ ri_tab,
+    const T* __restrict__ rt_tab, int d, int n_pos, int n_ri, int n_rt,
+    const int32_t* __restrict__ pos, const int32_t* __restrict__ req_idx,
+    const int32_t* __restrict__ rt_bucket, T* __restrict__ E, int tokens_per_warp, int32_t* err) {
+  constexpr int V = Elem<T>::kPerVec;
+  const int lane = threadIdx.x & 31;
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  long long t0 = warp * tokens_per_warp;
+  const long long tend = min(Ttok, (long long)off[B]);
+  if (t0 >= tend) return;
+  const long long t1 = min(tend, t0 + tokens_per_warp);
+  const int nv = d / V;
+  int u = warp_find_user(off, B, t0);
+  long long u_end = off[u + 1];
+  long long u_beg = off[u];
+  int n = hist_len[u];
+  for (long long t = t0; t < t1; ++t) {
+    while (t >= u_end && u < B - 1) {
+      ++u;
+      u_beg = u_end;
+      u_end = off[u + 1];
+      n = hist_len[u];
+    }
+    const bool cand = (t - u_beg) >= n;
+    long long it = item_ids[t];
+    if (it < 0 || it >= n_item) {
+      if (lane == 0) flag(err, GENRANK_DERR_ITEM_ID);
+      it = it < 0 ? 0 : n_item - 1;
+    }
+    int a = n_action;  // the mask-action row M
+    if (!cand) {
+      a = action_ids[t];
+      if (a < 0 || a >= n_action) {
+        if (lane == 0) flag(err, GENRANK_DERR_ACTION_ID);
+        a = a < 0 ? 0 : n_action - 1;
+      }
+    }
+    int p = pos[t], r = req_idx[t], b = rt_bucket[t];
+    if (p < 0 || p >= n_pos || r < 0 || r >= n_ri || b < 0 || b >= n_rt) {
+      // only reachable when the metadata pass rejected this user's layout
+      if (lane == 0) flag(err, GENRANK_DERR_INDEX);
+      p = min(max(p, 0), n_pos - 1);
+      r = min(max(r, 0), n_ri - 1);
+      b = min(max(b, 0), n_rt - 1);
+    }
+    const uint4* r0 = reinterpret_cast<const uint4*>(item_tab + it * d);
+    const uint4* r1 = reinterpret_cast<const uint4*>(action_tab + (long long)a * d);
+    const uint4* r2 = reinterpret_cast<const uint4*>(pos_tab + (long long)p * d);
+    const uint4* r3 = reinterpret_cast<const uint4*>(ri_tab + (long long)r * d);
+    const uint4* r4 = reinterpret_cast<const uint4*>(rt_tab + (long long)b * d);
+    uint4* out = reinterpret_cast<uint4*>(E + t * d);
+    for (int v = lane; v < nv; v += 32) {
+      uint4 x0 = __ldg(r0 + v), x1 = __ldg(r1 + v), x2 = __ldg(r2 + v), x3 = __ldg(r3 + v),
+            x4 = __ldg(r4 + v);
+      float f[V], g[V];
+      Elem<T>::unpack(x0, f);
+      Elem<T>::unpack(x1, g);
+#pragma unroll
+      for (int k = 0; k < V; ++k) f[k] += g[k];
+      Elem<T>::unpack(x2, g);
+#pragma unroll
+      for (int k = 0; k < V; ++k) f[k] += g[k];
+      Elem<T>::unpack(x3, g);
+#pragma unroll
+      for (int k = 0; k < V; ++k) f[k] += g[k];
+      Elem<T>::unpack(x4, g);
+#pragma unroll
+      for (int k = 0; k < V; ++k) f[k] += g[k];
+      out[v] = Elem<T>::pack(f);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// backward: scatter-add dE into the five fp32 gradient tables
+// ------------------------------------------------------------------------------------------
+// Grid (token chunks, column slices of kCols).  The small tables (action, pos,
+// ri, rt) are accumulated for the CTA's column slice in shared memory and added
+// to global memory once at the end; item rows go straight to global memory with
+// vector reductions.  Without room in shared memory every table goes straight
+// to global memory.
+constexpr int kBwdCols = 64;
+
+GR_DEVICE void red_add_v2(float* p, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+}
+
+template <typename T, bool kSmem>
+__global__ void __launch_bounds__(1024) k_embed_bwd(
+    int B, long long Ttok, const int32_t* __restrict__ off, const int32_t* __restrict__ hist_len,
+    const int32_t* __restrict__ item_ids, const int32_t* __restrict__ action_ids,
+    const int32_t* __restrict__ pos, const int32_t* __restrict__ req_idx,
+    const int32_t* __restrict__ rt_bucket, const T* __restrict__ dE, int d,
+    float* __restrict__ g_item, long long n_item, float* __restrict__ g_action, int n_action,
+    float* __restrict__ g_pos, int n_pos, float* __restrict__ g_ri, int n_ri,
+    float* __restrict__ g_rt, int n_rt, int tokens_per_warp, int32_t* err) {
+  extern __shared__ float acc[];  // [rows_small][kBwdCols] when kSmem
+  const int n_act_rows = n_action + 1;
+  const int rows_small = n_act_rows + n_pos + n_ri + n_rt;
+  float* s_action = acc;
+  float* s_pos = s_action + n_act_rows * kBwdCols;
+  float* s_ri = s_pos + n_pos * kBwdCols;
+  float* s_rt = s_ri + n_ri * kBwdCols;
+  if (kSmem) {
+    for (int i = threadIdx.x; i < rows_small * kBwdCols; i += blockDim.x) acc[i] = 0.f;
+    __syncthreads();
+  }
+  const int lane = threadIdx.x & 31;
+  const int c0 = blockIdx.y * kBwdCols;
+  const int col = c0 + 2 * lane;  // each lane owns two adjacent columns
+  const bool col_ok = col < d;
+  const long long tend = min(Ttok, (long long)off[B]);
+  const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const long long t0 = warp * tokens_per_warp;
+  if (t0 < tend) {
+    const long long t1 = min(tend, t0 + tokens_per_warp);
+    int u = warp_find_user(off, B, t0);
+    long long u_beg = off[u], u_end = off[u + 1];
+    int n = hist_len[u];
+    for (long long t = t0; t < t1; ++t) {
+      while (t >= u_end && u < B - 1) {
+        ++u;
+        u_beg = u_end;
+        u_end = off[u + 1];
+        n = hist_len[u];
+      }
+      const bool cand = (t - u_beg) >= n;
+      long long it = item_ids[t];
+      int a = cand ? n_action : action_ids[t];
+      int p = pos[t], r = req_idx[t], b = rt_bucket[t];
+      bool bad = it < 0 || it >= n_item || a < 0 || a > n_action || p < 0 || p >= n_pos ||
+                 r < 0 || r >= n_ri || b < 0 || b >= n_rt;
+      if (bad) {
+        if (lane == 0) flag(err, GENRANK_DERR_INDEX);
+        continue;
+      }
+      if (!col_ok) continue;
+      float g0, g1;
+      if (sizeof(T) == 2) {
+        uint32_t w = *reinterpret_cast<const uint32_t*>(dE + t * d + col);
+        g0 = bf16_lo(w);
+        g1 = bf16_hi(w);
+      } else {
+        float2 w = *reinterpret_cast<const float2*>(dE + t * d + col);
+        g0 = w.x;
+        g1 = w.y;
+      }
+      red_add_v2(g_item + it * d + col, g0, g1);
+      if (kSmem) {
+        const int cl = 2 * lane;
+        atomicAdd(s_action + a * kBwdCols + cl, g0);
+        atomicAdd(s_action + a * kBwdCols + cl + 1, g1);
+        atomicAdd(s_pos + p * kBwdCols + cl, g0);
+        atomicAdd(s_pos + p * kBwdCols + cl + 1, g1);
+        atomicAdd(s_ri + r * kBwdCols + cl, g0);
+        atomicAdd(s_ri + r * kBwdCols + cl + 1, g1);
+        atomicAdd(s_rt + b * kBwdCols + cl, g0);
+        atomicAdd(s_rt + b * kBwdCols + cl + 1, g1);
+      } else {
+        red_add_v2(g_action + (long long)a * d + col, g0, g1);
+        red_add_v2(g_pos + (long long)p * d + col, g0, g1);
+        red_add_v2(g_ri + (long long)r * d + col, g0, g1);
+        red_add_v2(g_rt + (long long)b * d + col, g0, g1);
+      }
+    }
+  }
+  if (kSmem) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < rows_small * kBwdCols; i += blockDim.x) {
+      const float v = acc[i];
+      const int row = i / kBwdCols, c = c0 + i % kBwdCols;
+      if (v == 0.f || c >= d) continue;
+      float* dst;
+      if (row < n_act_rows) dst = g_action + (long long)row * d;
+      else if (row < n_act_rows + n_pos) dst = g_pos + (long long)(row - n_act_rows) * d;
+      else if (row < n_act_rows + n_pos + n_ri) dst = g_ri + (long long)(row - n_act_rows - n_pos) * d;
+      else dst = g_rt + (long long)(row - n_act_rows - n_pos - n_ri) * d;
+      atomicAdd(dst + c, v);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// host launchers
+// ------------------------------------------------------------------------------------------
+static int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+int launch_embed_fwd(const EmbedFwdArgs& a, cudaStream_t st) {
+  k_token_meta<<<a.B, 256, 0, st>>>(a.B, a.T, a.off, a.hist_len, a.ts, a.n_pos, a.n_ri, a.n_rt,
+                                    a.pos, a.req_idx, a.rt_bucket, a.err);
+  if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
+  if (a.T == 0) return GENRANK_OK;
+  // enough warps for ~16 resident 256-thread blocks per SM, a few tokens each
+  const long long warps_target = (long long)sm_count() * 64 * 4;
+  int tpw = (int)max(1LL, (a.T + warps_target - 1) / warps_target);
+  long long warps = (a.T + tpw - 1) / tpw;
+  long long blocks = (warps + 7) / 8;
+  if (a.dtype == GENRANK_BF16) {
+    using T = __nv_bfloat16;
+    k_embed_fwd<T><<<(unsigned)blocks, 256, 0, st>>>(
+        a.B, a.T, a.off, a.hist_len, a.item_ids, a.action_ids, (const T*)a.item_tab, a.n_item,
+        (const T*)a.action_tab, a.n_action, (const T*)a.pos_tab, (const T*)a.ri_tab,
+        (const T*)a.rt_tab, a.d, a.n_pos, a.n_ri, a.n_rt, a.pos, a.req_idx, a.rt_bucket, (T*)a.E,
+        tpw, a.err);
+  } else {
+    using T = float;
+    k_embed_fwd<T><<<(unsigned)blocks, 256, 0, st>>>(
+        a.B, a.T, a.off, a.hist_len, a.item_ids, a.action_ids, (const T*)a.item_tab, a.n_item,
+        (const T*)a.action_tab, a.n_action, (const T*)a.pos_tab, (const T*)a.ri_tab,
+        (const T*)a.rt_tab, a.d, a.n_pos, a.n_ri, a.n_rt, a.pos, a.req_idx, a.rt_bucket, (T*)a.E,
+        tpw, a.err);
+  }
+  return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
+}
+
+template <typename T, bool kSmem>
+static int launch_bwd_t(const EmbedBwdArgs& a, cudaStream_t st) {
+  const int rows_small = a.n_action + 1 + a.n_pos + a.n_ri + a.n_rt;
+  const size_t smem = kSmem ? (size_t)rows_small * kBwdCols * sizeof(float) : 0;
+  if (kSmem) {
+    if (cudaFuncSetAttribute(k_embed_bwd<T, kSmem>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return GENRANK_ERR_CUDA;
+  }
+  const int slices = (a.d + kBwdCols - 1) / kBwdCols;
+  // about two waves of one 1024-thread CTA per SM over all slices
+  const long long ctas_per_slice = max(1LL, (long long)(2 * sm_count() + slices - 1) / slices);
+  const long long warps = ctas_per_slice * 32;
+  const int tpw = (int)max(1LL, (a.T + warps - 1) / warps);
+  const long long chunks = max(1LL, ((a.T + tpw - 1) / tpw + 31) / 32);
+  dim3 grid((unsigned)chunks, (unsigned)slices);
+  k_embed_bwd<T, kSmem><<<grid, 1024, smem, st>>>(
+      a.B, a.T, a.off, a.hist_len, a.item_ids, a.action_ids, a.pos, a.req_idx, a.rt_bucket,
+      (const T*)a.dE, a.d, a.g_item, a.n_item, a.g_action, a.n_action, a.g_pos, a.n_pos, a.g_ri,
+      a.n_ri, a.g_rt, a.n_rt, tpw, a.err);
+  return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
+}
+
+int launch_embed_bwd(const EmbedBwdArgs& a, cudaStream_t st) {
+  if (a.T == 0) return GENRANK_OK;
+  const size_t rows_small = (size_t)a.n_action + 1 + a.n_pos + a.n_ri + a.n_rt;
+  const bool smem_ok = rows_small * kBwdCols * sizeof(float) <= 224 * 1024;
+  if (a.dtype == GENRANK_BF16)
+    return smem_ok ? launch_bwd_t<__nv_bfloat16, true>(a, st)
+                   : launch_bwd_t<__nv_bfloat16, false>(a, st);
+  return smem_ok ? launch_bwd_t<float, true>(a, st) : launch_bwd_t<float, false>(a, st);
+}
+
+}  // namespace gr

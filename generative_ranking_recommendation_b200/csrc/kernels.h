@@ -1,0 +1,110 @@
+// Internal launch interfaces between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gr {
+
+struct EmbedFwdArgs {
+  int B;
+  long long T;
+  const int32_t* off;
+  const int32_t* hist_len;
+  const int32_t* item_ids;
+  const int32_t* action_ids;
+  const int64_t* ts;
+  const void* item_tab;
+  long long n_item;
+  const void* action_tab;
+  int n_action;
+  const void* pos_tab;
+  int n_pos;
+  const void* ri_tab;
+  int n_ri;
+  const void* rt_tab;
+  int n_rt;
+  int d;
+  int dtype;
+  void* E;
+  int32_t* pos;
+  int32_t* req_idx;
+  int32_t* rt_bucket;
+  int32_t* err;
+};
+
+struct EmbedBwdArgs {
+  int B;
+  long long T;
+  const int32_t* off;
+  const int32_t* hist_len;
+  const int32_t* item_ids;
+  const int32_t* action_ids;
+  const int32_t* pos;
+  const int32_t* req_idx;
+  const int32_t* rt_bucket;
+  const void* dE;
+  int d;
+  int dtype;
+  float* g_item;
+  long long n_item;
+  float* g_action;
+  int n_action;
+  float* g_pos;
+  int n_pos;
+  float* g_ri;
+  int n_ri;
+  float* g_rt;
+  int n_rt;
+  int32_t* err;
+};
+
+constexpr int kMaxHeads = 64;
+
+// Everything an attention launch needs; slopes are copied by value.
+struct AttnArgs {
+  int B;
+  long long T;
+  const int32_t* off;
+  const int32_t* hist_len;
+  int max_seqlen;
+  const void* q;
+  const void* k;
+  const void* v;
+  long long tok_stride;  // elements
+  int H;
+  int dh;
+  const int32_t* pos;
+  const int64_t* ts;
+  float slope_pos[kMaxHeads];
+  float slope_time[kMaxHeads];
+  float scale;
+  int dtype;
+  void* o;
+  long long o_stride;  // elements
+  float* lse;          // [H, T] or null
+  // backward only
+  const void* dO;
+  void* dq;
+  void* dk;
+  void* dv;
+  const float* lse_in;
+  void* ws;
+  size_t ws_bytes;
+  int32_t* err;
+};
+
+int launch_embed_fwd(const EmbedFwdArgs& a, cudaStream_t st);
+int launch_embed_bwd(const EmbedBwdArgs& a, cudaStream_t st);
+
+// CUDA-core attention (fp32 storage, or bf16 with dh != 64)
+int launch_attn_fwd_simt(const AttnArgs& a, cudaStream_t st);
+int launch_attn_bwd_simt(const AttnArgs& a, cudaStream_t st);
+size_t attn_bwd_simt_workspace(int B, long long T, int H, int dh, int max_seqlen);
+
+// tcgen05 / TMEM / TMA attention forward (bf16, dh = 64)
+int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st);
+size_t attn_fwd_tc_workspace(int B, long long T, int H, int max_seqlen);
+
+}  // namespace gr

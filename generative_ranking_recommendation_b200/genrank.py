@@ -1,0 +1,193 @@
+"""Thin Python binding of libgenrank (include/genrank.h), by the same names.
+
+Argument marshalling only: torch tensors supply device pointers and the
+current CUDA stream; every step of the computation runs in the library's
+kernels.  There is no fallback: if the shared library is missing or the call
+fails, an exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgenrank.so")
+
+F32, BF16 = 0, 1
+DERR = {
+    "LAYOUT": 1 << 0, "ITEM_ID": 1 << 1, "ACTION_ID": 1 << 2, "TS_ORDER": 1 << 3,
+    "POS_RANGE": 1 << 4, "INDEX": 1 << 5, "TIMEOUT": 1 << 6,
+}
+
+# every entry point declared in include/genrank.h
+EXPORTS = (
+    "genrank_status_string", "genrank_device_error_string", "genrank_check_error",
+    "genrank_alibi_slopes", "genrank_embed_assemble", "genrank_embed_assemble_bwd",
+    "genrank_attn_fwd", "genrank_attn_bwd", "genrank_attn_workspace_size",
+)
+
+
+class GenRankError(RuntimeError):
+    pass
+
+
+_lib = None
+_P, _I, _L, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+
+def lib():
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise GenRankError(
+                f"{LIB_PATH} is missing; build it with "
+                "`python -m generative_ranking_recommendation_b200.csrc.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.genrank_status_string.restype = ctypes.c_char_p
+        L.genrank_status_string.argtypes = [_I]
+        L.genrank_device_error_string.restype = ctypes.c_char_p
+        L.genrank_device_error_string.argtypes = [_I]
+        L.genrank_check_error.restype = _I
+        L.genrank_check_error.argtypes = [_P, _P]
+        L.genrank_alibi_slopes.restype = _I
+        L.genrank_alibi_slopes.argtypes = [_I, _P, _P]
+        L.genrank_embed_assemble.restype = _I
+        L.genrank_embed_assemble.argtypes = [
+            _I, _L, _P, _P, _P, _P, _P, _P, _L, _P, _I, _P, _I, _P, _I, _P, _I, _I, _I,
+            _P, _P, _P, _P, _P, _P]
+        L.genrank_embed_assemble_bwd.restype = _I
+        L.genrank_embed_assemble_bwd.argtypes = [
+            _I, _L, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _L, _P, _I, _P, _I, _P, _I,
+            _P, _I, _P, _P]
+        L.genrank_attn_fwd.restype = _I
+        L.genrank_attn_fwd.argtypes = [
+            _I, _L, _P, _P, _I, _P, _P, _P, _L, _I, _I, _P, _P, _P, _P, _F, _I, _P, _L, _P,
+            _P, _Z, _P, _P]
+        L.genrank_attn_bwd.restype = _I
+        L.genrank_attn_bwd.argtypes = [
+            _I, _L, _P, _P, _I, _P, _P, _P, _L, _I, _I, _P, _P, _P, _P, _F, _I, _P, _P, _L,
+            _P, _P, _P, _P, _P, _Z, _P, _P]
+        L.genrank_attn_workspace_size.restype = _Z
+        L.genrank_attn_workspace_size.argtypes = [_I, _L, _I, _I, _I, _I]
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        msg = lib().genrank_status_string(rc).decode()
+        raise GenRankError(f"{what}: {msg} (code {rc})")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise GenRankError(f"unsupported dtype {t.dtype}")
+
+
+def status_string(code: int) -> str:
+    return lib().genrank_status_string(int(code)).decode()
+
+
+def device_error_string(bit: int) -> str:
+    return lib().genrank_device_error_string(int(bit)).decode()
+
+
+def alibi_slopes(H: int):
+    """(slope_pos, slope_time) as Python float lists, from the library."""
+    sp = (ctypes.c_float * H)()
+    st = (ctypes.c_float * H)()
+    _check(lib().genrank_alibi_slopes(H, ctypes.cast(sp, _P), ctypes.cast(st, _P)),
+           "genrank_alibi_slopes")
+    return list(sp), list(st)
+
+
+def check_error(dev_err: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream and returns the device error word (0 = clean)."""
+    rc = lib().genrank_check_error(_ptr(dev_err), _stream(stream))
+    if rc < 0:
+        _check(-rc, "genrank_check_error")
+    return rc
+
+
+def embed_assemble(seq_offsets, hist_len, item_ids, action_ids, ts, item_tab, action_tab,
+                   pos_tab, ri_tab, rt_tab, E, pos, req_idx, rt_bucket, dev_err, stream=None):
+    """genrank_embed_assemble on torch tensors (all on one CUDA device)."""
+    B = hist_len.numel()
+    T = item_ids.numel()
+    d = item_tab.shape[1]
+    rc = lib().genrank_embed_assemble(
+        B, T, _ptr(seq_offsets), _ptr(hist_len), _ptr(item_ids), _ptr(action_ids), _ptr(ts),
+        _ptr(item_tab), item_tab.shape[0], _ptr(action_tab), action_tab.shape[0] - 1,
+        _ptr(pos_tab), pos_tab.shape[0], _ptr(ri_tab), ri_tab.shape[0], _ptr(rt_tab),
+        rt_tab.shape[0], d, _dtype_code(item_tab), _ptr(E), _ptr(pos), _ptr(req_idx),
+        _ptr(rt_bucket), _ptr(dev_err), _stream(stream))
+    _check(rc, "genrank_embed_assemble")
+
+
+def embed_assemble_bwd(seq_offsets, hist_len, item_ids, action_ids, pos, req_idx, rt_bucket, dE,
+                       d_item, d_action, d_pos, d_ri, d_rt, dev_err, stream=None):
+    """genrank_embed_assemble_bwd: accumulates into the fp32 gradient tables."""
+    B = hist_len.numel()
+    T = item_ids.numel()
+    rc = lib().genrank_embed_assemble_bwd(
+        B, T, _ptr(seq_offsets), _ptr(hist_len), _ptr(item_ids), _ptr(action_ids), _ptr(pos),
+        _ptr(req_idx), _ptr(rt_bucket), _ptr(dE), dE.shape[1], _dtype_code(dE), _ptr(d_item),
+        d_item.shape[0], _ptr(d_action), d_action.shape[0] - 1, _ptr(d_pos), d_pos.shape[0],
+        _ptr(d_ri), d_ri.shape[0], _ptr(d_rt), d_rt.shape[0], _ptr(dev_err), _stream(stream))
+    _check(rc, "genrank_embed_assemble_bwd")
+
+
+def attn_workspace_size(B, T, H, dh, max_seqlen, is_bwd=False) -> int:
+    return int(lib().genrank_attn_workspace_size(B, T, H, dh, max_seqlen, int(bool(is_bwd))))
+
+
+def _host_floats(xs):
+    arr = (ctypes.c_float * len(xs))(*[float(x) for x in xs])
+    return arr
+
+
+def attn_fwd(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts, slope_pos,
+             slope_time, scale, o, o_stride, lse, ws, dev_err, T=None, stream=None):
+    """genrank_attn_fwd.  q/k/v are tensors whose data_ptr is the first element of
+    head 0 of token 0 (views into a fused QKV buffer are fine); slopes are host lists."""
+    B = hist_len.numel()
+    T = o.shape[0] if T is None else T
+    sp, st = _host_floats(slope_pos), _host_floats(slope_time)
+    rc = lib().genrank_attn_fwd(
+        B, T, _ptr(seq_offsets), _ptr(hist_len), int(max_seqlen), _ptr(q), _ptr(k), _ptr(v),
+        int(tok_stride), H, dh, _ptr(pos), _ptr(ts), ctypes.cast(sp, _P), ctypes.cast(st, _P),
+        float(scale), _dtype_code(q), _ptr(o), int(o_stride), _ptr(lse), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream))
+    _check(rc, "genrank_attn_fwd")
+
+
+def attn_bwd(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts, slope_pos,
+             slope_time, scale, o, dO, o_stride, lse, dq, dk, dv, ws, dev_err, T=None,
+             stream=None):
+    """genrank_attn_bwd; dq/dk/dv share the layout (tok_stride) of q/k/v."""
+    B = hist_len.numel()
+    T = o.shape[0] if T is None else T
+    sp, st = _host_floats(slope_pos), _host_floats(slope_time)
+    rc = lib().genrank_attn_bwd(
+        B, T, _ptr(seq_offsets), _ptr(hist_len), int(max_seqlen), _ptr(q), _ptr(k), _ptr(v),
+        int(tok_stride), H, dh, _ptr(pos), _ptr(ts), ctypes.cast(sp, _P), ctypes.cast(st, _P),
+        float(scale), _dtype_code(q), _ptr(o), _ptr(dO), int(o_stride), _ptr(lse), _ptr(dq),
+        _ptr(dk), _ptr(dv), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _ptr(dev_err), _stream(stream))
+    _check(rc, "genrank_attn_bwd")

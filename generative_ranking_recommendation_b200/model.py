@@ -1,0 +1,209 @@
+"""The GenRank scoring and training step built on libgenrank.
+
+The hot path (metadata + embedding assembly, masked ALiBi attention forward
+and backward, embedding backward) runs in the library's kernels.  The blocks
+around it are torch ops: the fused QKV projection, the output projection and
+residual, pre-RMSNorm (eps 1e-6, unit gain) and the 4d SiLU FFN of the 4-layer
+workloads, the final RMSNorm and the candidate head (a dot with w_head at
+candidate rows only, as the loss lives only at candidate positions:
+"GenRank [2025]" chapter notes §1.3.1).  The residual stream is kept in fp32;
+projections run in the storage dtype with fp32 accumulation.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import genrank as G
+
+RMS_EPS = 1e-6
+
+
+@dataclass
+class DeviceBatch:
+    B: int
+    T: int
+    max_seqlen: int
+    seq_offsets: torch.Tensor  # int32 [B+1]
+    hist_len: torch.Tensor  # int32 [B]
+    item_ids: torch.Tensor  # int32 [T]
+    action_ids: torch.Tensor  # int32 [T]
+    ts: torch.Tensor  # int64 [T]
+    cand_rows: torch.Tensor  # int64 [sum m]
+    labels: torch.Tensor | None  # float32 [sum m]
+
+    @staticmethod
+    def host_arrays(batch):
+        """The per-step input arrays of a generated batch, in upload order."""
+        cand = np.concatenate([np.arange(batch.seq_offsets[u] + batch.hist_len[u],
+                                         batch.seq_offsets[u + 1]) for u in range(batch.B)])
+        arrs = [batch.seq_offsets, batch.hist_len, batch.item_ids, batch.action_ids, batch.ts,
+                cand.astype(np.int64)]
+        if batch.labels is not None:
+            arrs.append(batch.labels)
+        return arrs
+
+    @classmethod
+    def from_tensors(cls, batch, tensors):
+        t = list(tensors)
+        labels = t[6] if len(t) > 6 else None
+        return cls(batch.B, batch.T, int(np.max(np.diff(batch.seq_offsets))) if batch.B else 0,
+                   t[0], t[1], t[2], t[3], t[4], t[5], labels)
+
+    @classmethod
+    def from_batch(cls, batch, device):
+        arrs = cls.host_arrays(batch)
+        return cls.from_tensors(batch, [torch.from_numpy(np.ascontiguousarray(a)).to(device)
+                                        for a in arrs])
+
+
+def _tt(x, dtype, device):
+    return torch.from_numpy(np.ascontiguousarray(x)).to(device=device, dtype=dtype)
+
+
+class GenRankModel:
+    """Device-resident tables and weights of one workload configuration."""
+
+    def __init__(self, cfg, model, device="cuda", item_tab: torch.Tensor | None = None):
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.dtype = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+        dt, dev = self.dtype, self.device
+        if item_tab is None:
+            from gen import item_table_torch  # seeded input generator (data only)
+            item_tab = item_table_torch(cfg.seed, cfg.n_item, cfg.d, cfg.dtype, dev)
+        self.item_tab = item_tab
+        self.action_tab = _tt(model.action_tab, dt, dev)
+        self.pos_tab = _tt(model.pos_tab, dt, dev)
+        self.ri_tab = _tt(model.ri_tab, dt, dev)
+        self.rt_tab = _tt(model.rt_tab, dt, dev)
+        self.layers = []
+        for L in model.layers:
+            W = {"Wqkv": _tt(np.concatenate([L["Wq"], L["Wk"], L["Wv"]], axis=1), dt, dev),
+                 "Wo": _tt(L["Wo"], dt, dev)}
+            if cfg.ffn:
+                W["W1"] = _tt(L["W1"], dt, dev)
+                W["W2"] = _tt(L["W2"], dt, dev)
+            self.layers.append(W)
+        self.w_head = _tt(model.w_head, torch.float32, dev)
+        self.H, self.dh, self.d = cfg.H, cfg.dh, cfg.d
+        self.slope_pos, self.slope_time = G.alibi_slopes(cfg.H)
+        self.scale = 1.0 / math.sqrt(cfg.dh)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self._ws = {}
+
+    # -------------------------------------------------------------------------------------
+    def workspace(self, db: DeviceBatch, bwd: bool) -> torch.Tensor:
+        n = G.attn_workspace_size(db.B, db.T, self.H, self.dh, db.max_seqlen, bwd)
+        key = bool(bwd)
+        w = self._ws.get(key)
+        if w is None or w.numel() < n:
+            w = torch.empty(max(n, 256), dtype=torch.uint8, device=self.device)
+            self._ws[key] = w
+        return w
+
+    def embed(self, db: DeviceBatch):
+        T, dev = db.T, self.device
+        E = torch.empty((T, self.d), dtype=self.dtype, device=dev)
+        pos = torch.empty(T, dtype=torch.int32, device=dev)
+        req = torch.empty(T, dtype=torch.int32, device=dev)
+        rtb = torch.empty(T, dtype=torch.int32, device=dev)
+        G.embed_assemble(db.seq_offsets, db.hist_len, db.item_ids, db.action_ids, db.ts,
+                         self.item_tab, self.action_tab, self.pos_tab, self.ri_tab, self.rt_tab,
+                         E, pos, req, rtb, self.err)
+        return E, (pos, req, rtb)
+
+    def attention(self, db: DeviceBatch, qkv: torch.Tensor, pos: torch.Tensor, need_lse=False):
+        d = self.d
+        o = torch.empty((db.T, d), dtype=qkv.dtype, device=self.device)
+        lse = torch.empty((self.H, db.T), dtype=torch.float32, device=self.device) if need_lse else None
+        G.attn_fwd(db.seq_offsets, db.hist_len, db.max_seqlen, qkv, qkv[:, d:], qkv[:, 2 * d:],
+                   3 * d, self.H, self.dh, pos, db.ts, self.slope_pos, self.slope_time,
+                   self.scale, o, d, lse, self.workspace(db, False), self.err, T=db.T)
+        return o, lse
+
+    def attention_bwd(self, db, qkv, pos, o, lse, do):
+        d = self.d
+        dqkv = torch.empty_like(qkv)
+        G.attn_bwd(db.seq_offsets, db.hist_len, db.max_seqlen, qkv, qkv[:, d:], qkv[:, 2 * d:],
+                   3 * d, self.H, self.dh, pos, db.ts, self.slope_pos, self.slope_time,
+                   self.scale, o, do.contiguous(), d, lse, dqkv, dqkv[:, d:], dqkv[:, 2 * d:],
+                   self.workspace(db, True), self.err, T=db.T)
+        return dqkv
+
+    @staticmethod
+    def rms(x):
+        return x * torch.rsqrt((x * x).mean(dim=-1, keepdim=True) + RMS_EPS)
+
+    # -------------------------------------------------------------------------------------
+    @torch.no_grad()
+    def forward(self, db: DeviceBatch) -> torch.Tensor:
+        """Candidate logits (fp32 [sum m]) for one batch."""
+        E, (pos, _, _) = self.embed(db)
+        ffn = self.cfg.ffn
+        x = E.float()
+        for W in self.layers:
+            a = (self.rms(x) if ffn else x).to(self.dtype)
+            qkv = a @ W["Wqkv"]
+            o, _ = self.attention(db, qkv, pos)
+            x = x + (o @ W["Wo"]).float()
+            if ffn:
+                f = self.rms(x).to(self.dtype)
+                x = x + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"]).float()
+        if ffn:
+            x = self.rms(x)
+        return x.index_select(0, db.cand_rows) @ self.w_head
+
+    # -------------------------------------------------------------------------------------
+    def train_step(self, db: DeviceBatch):
+        """Mean BCE over candidates, and the five fp32 table gradients.
+
+        The attention backward and the embedding backward run in the library;
+        torch autograd carries the gradient through the blocks around them.
+        """
+        E, (pos, req, rtb) = self.embed(db)
+        Eg = E.detach().requires_grad_(True)
+        model = self
+
+        class _Attn(torch.autograd.Function):
+            @staticmethod
+            def forward(ctx, qkv):
+                o, lse = model.attention(db, qkv, pos, need_lse=True)
+                ctx.save_for_backward(qkv, o, lse)
+                return o
+
+            @staticmethod
+            def backward(ctx, do):
+                qkv, o, lse = ctx.saved_tensors
+                return model.attention_bwd(db, qkv, pos, o, lse, do)
+
+        ffn = self.cfg.ffn
+        x = Eg.float()
+        for W in self.layers:
+            a = (self.rms(x) if ffn else x).to(self.dtype)
+            qkv = a @ W["Wqkv"]
+            o = _Attn.apply(qkv)
+            x = x + (o @ W["Wo"]).float()
+            if ffn:
+                f = self.rms(x).to(self.dtype)
+                x = x + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"]).float()
+        if ffn:
+            x = self.rms(x)
+        z = x.index_select(0, db.cand_rows) @ self.w_head
+        loss = torch.nn.functional.binary_cross_entropy_with_logits(z, db.labels)
+        loss.backward()
+        dE = Eg.grad.to(self.dtype).contiguous()
+        f32 = dict(dtype=torch.float32, device=self.device)
+        grads = {"item": torch.zeros(self.item_tab.shape, **f32),
+                 "action": torch.zeros(self.action_tab.shape, **f32),
+                 "pos": torch.zeros(self.pos_tab.shape, **f32),
+                 "ri": torch.zeros(self.ri_tab.shape, **f32),
+                 "rt": torch.zeros(self.rt_tab.shape, **f32)}
+        G.embed_assemble_bwd(db.seq_offsets, db.hist_len, db.item_ids, db.action_ids, pos, req,
+                             rtb, dE, grads["item"], grads["action"], grads["pos"], grads["ri"],
+                             grads["rt"], self.err)
+        return loss.detach(), z.detach(), grads

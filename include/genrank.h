@@ -1,0 +1,196 @@
+/*
+ * genrank.h — C ABI of the GenRank hot-path library (libgenrank.so, sm_100a).
+ *
+ * The operations follow the GenRank pages ("Towards Large-scale Generative
+ * Ranking"):
+ *   - huaxiaozhuan.com chapter notes "GenRank [2025]", §1.4.1 Item-Action
+ *     Organization (token = item embedding + action embedding, candidates carry
+ *     the mask action, candidate mask) and §1.4.2 Position & Time Biases (the
+ *     position, request-index and pre-request time embeddings, the five-way
+ *     input sum, ALiBi fused into the attention score, slopes 2^(-8(h+1)/H));
+ *   - wln20.github.io "生成式排序 —— 小红书 GenRank 精读笔记" (the candidate mask
+ *     makes batched scoring equal to appending each candidate alone);
+ *   - fun-rec mdbook "The Overall Generative Ranking Paradigm", §7.2.1 and
+ *     §7.2.2 (history causal, candidates see all history and not each other;
+ *     ALiBi over position and time).
+ *
+ * Conventions shared by every entry point:
+ *   - Every array argument is a DEVICE pointer owned by the caller, unless it is
+ *     documented as a host pointer.  The library allocates no memory and keeps
+ *     no state between calls; scratch space is the caller's workspace.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream).  Nothing inside synchronises except genrank_check_error.
+ *   - The return value is GENRANK_OK or a host-detected GENRANK_ERR_* code; on
+ *     such an error nothing was launched.  Errors found in the data on the device
+ *     (ids out of range, unsorted timestamps, ...) are OR-ed as GENRANK_DERR_*
+ *     bits into *dev_err (one caller-zeroed device int32); the kernels clamp the
+ *     offending index and keep going, so no call traps or hangs the GPU.  Every
+ *     wait inside a kernel is bounded and reports GENRANK_DERR_TIMEOUT.
+ *   - Token layout ("jagged"): users are contiguous; user u owns tokens
+ *     [seq_offsets[u], seq_offsets[u+1]), history first (hist_len[u] tokens,
+ *     oldest first), then its candidates.  Every call also takes T, a HOST
+ *     value: the row count of every per-token array (normally seq_offsets[B]).
+ *     Kernels never touch rows at or beyond T; offsets that point past it raise
+ *     GENRANK_DERR_LAYOUT.
+ *   - dtype is GENRANK_F32 or GENRANK_BF16 and applies to every floating-point
+ *     tensor of the call unless stated otherwise; accumulation is fp32.
+ */
+#ifndef GENRANK_H_
+#define GENRANK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *genrank_stream_t; /* the same handle as cudaStream_t */
+
+enum { GENRANK_F32 = 0, GENRANK_BF16 = 1 };
+
+/* host-detected status codes (return values) */
+enum {
+  GENRANK_OK = 0,
+  GENRANK_ERR_INVALID_ARG = 1,  /* null pointer, bad size or stride */
+  GENRANK_ERR_UNSUPPORTED = 2,  /* a valid but unsupported shape or dtype */
+  GENRANK_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+  GENRANK_ERR_LAUNCH = 4,       /* a kernel launch failed (cudaGetLastError) */
+  GENRANK_ERR_CUDA = 5          /* another CUDA runtime/driver call failed */
+};
+
+/* device-detected data errors (bits of *dev_err) */
+enum {
+  GENRANK_DERR_LAYOUT = 1 << 0,     /* bad seq_offsets / hist_len, or offsets beyond T */
+  GENRANK_DERR_ITEM_ID = 1 << 1,    /* item id outside [0, n_item) (clamped) */
+  GENRANK_DERR_ACTION_ID = 1 << 2,  /* history action id outside [0, n_action) (clamped) */
+  GENRANK_DERR_TS_ORDER = 1 << 3,   /* history timestamps decrease, candidate times differ,
+                                       or the request time precedes the last history time */
+  GENRANK_DERR_POS_RANGE = 1 << 4,  /* position >= n_pos (clamped) */
+  GENRANK_DERR_INDEX = 1 << 5,      /* a metadata index outside its table (backward) */
+  GENRANK_DERR_TIMEOUT = 1 << 6     /* a bounded in-kernel wait gave up */
+};
+
+/* Human-readable name of a GENRANK_OK / GENRANK_ERR_* return code. */
+const char *genrank_status_string(int code);
+
+/* Human-readable name of one GENRANK_DERR_* bit (or "clean" for 0). */
+const char *genrank_device_error_string(int bit);
+
+/* Synchronises `stream`, reads *dev_err and returns it (0 when clean); returns
+ * -GENRANK_ERR_CUDA if the copy or the synchronisation failed. */
+int genrank_check_error(const int32_t *dev_err, genrank_stream_t stream);
+
+/* ALiBi slopes, written to HOST arrays of H floats:
+ *   slope_pos[h]  = 2^(-8(h+1)/H)                (per unit of position)
+ *   slope_time[h] = slope_pos[h] / 3600          (per second of |t_i - t_j|)
+ * huaxiaozhuan "GenRank [2025]" §1.4.2 gives the slope formula and the H = 8
+ * example (1/2 ... 1/256); the per-second time slope is the linear time bias of
+ * the workloads this library serves.  Returns GENRANK_ERR_INVALID_ARG for H < 1. */
+int genrank_alibi_slopes(int H, float *slope_pos, float *slope_time);
+
+/* ---------------------------------------------------------------------------
+ * Step a1 + a2: per-token metadata and the five-way embedding sum.
+ *   E_i = item[x_i] + action[a_i, or M for candidates] + pos_tab[pos_i]
+ *         + ri_tab[req_idx_i] + rt_tab[rt_bucket_i]
+ * (huaxiaozhuan "GenRank [2025]" §1.4.1 token sum, §1.4.2 input
+ * representation), summed in fp32 and rounded once to dtype.
+ *   pos_i       = 1-based index for history tokens; n_u + 1 for every candidate
+ *                 (§1.4.2 Position Embeddings: candidates of one request share it)
+ *   req_idx_i   = |{t_1..t_i}|, distinct timestamps so far, clamped to n_ri - 1
+ *                 (§1.4.2 Request Index Embeddings)
+ *   rt_bucket_i = 0 if no earlier request, else 1 + min(n_rt - 2,
+ *                 floor(4 log2(gap + 1))), gap = t_i - max{t_j : t_j < t_i}
+ *                 (§1.4.2 Pre-Request Time Embeddings; the bucket form is this
+ *                 library's reading); a candidate's values are those of the
+ *                 token made by appending it alone at time t_req.
+ * Arguments:
+ *   B            number of users (>= 1); seq_offsets [B+1] int32, hist_len [B] int32
+ *   item_ids     [T] int32, rows of item_tab
+ *   action_ids   [T] int32 in [0, n_action); ignored at candidate slots
+ *   ts           [T] int64 seconds; history non-decreasing; every candidate slot
+ *                holds the request time t_req >= the last history time
+ *   item_tab     [n_item, d]; action_tab [n_action + 1, d] whose LAST row is the
+ *                mask action M; pos_tab [n_pos, d] (row 0 unused); ri_tab [n_ri, d];
+ *                rt_tab [n_rt, d] with 2 <= n_rt <= 65.  Row-major, dtype, 16-byte
+ *                aligned rows (d * sizeof(dtype) a multiple of 16).
+ *   E            [T, d] output (dtype); pos, req_idx, rt_bucket: [T] int32 outputs
+ * Two kernels on `stream`: the per-user metadata scan, then the row gather-sum. */
+int genrank_embed_assemble(int B, int64_t T, const int32_t *seq_offsets, const int32_t *hist_len,
+                           const int32_t *item_ids, const int32_t *action_ids, const int64_t *ts,
+                           const void *item_tab, int64_t n_item, const void *action_tab,
+                           int n_action, const void *pos_tab, int n_pos, const void *ri_tab,
+                           int n_ri, const void *rt_tab, int n_rt, int d, int dtype,
+                           void *E, int32_t *pos, int32_t *req_idx, int32_t *rt_bucket,
+                           int32_t *dev_err, genrank_stream_t stream);
+
+/* Step a5: table gradients of the embedding sum (training).  Each token's dE_i
+ * is added to the five rows it read: d_item[x_i], d_action[a_i or M],
+ * d_pos[pos_i], d_ri[req_idx_i], d_rt[rt_bucket_i].  pos/req_idx/rt_bucket are
+ * the metadata written by genrank_embed_assemble.  dE is [T, d] in dtype; the
+ * five gradient tables are fp32, caller-zeroed (the call accumulates into them),
+ * with the row counts of the forward tables (d_action has n_action + 1 rows).
+ * Float atomics make the summation order, and so the last bits, vary from run
+ * to run. */
+int genrank_embed_assemble_bwd(int B, int64_t T, const int32_t *seq_offsets, const int32_t *hist_len,
+                               const int32_t *item_ids, const int32_t *action_ids,
+                               const int32_t *pos, const int32_t *req_idx,
+                               const int32_t *rt_bucket, const void *dE, int d, int dtype,
+                               float *d_item, int64_t n_item, float *d_action, int n_action,
+                               float *d_pos, int n_pos, float *d_ri, int n_ri, float *d_rt,
+                               int n_rt, int32_t *dev_err, genrank_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Step a3: masked multi-head attention with on-the-fly ALiBi position and time
+ * biases (huaxiaozhuan "GenRank [2025]" §1.4.2 score formula; §1.4.1 candidate
+ * mask; fun-rec §7.2.2 bias over position and time).  For user u, head h, local
+ * rows i and keys j:
+ *   s_ij = scale * q_i.k_j - slope_pos[h] |p_i - p_j| - slope_time[h] |t_i - t_j|
+ *   visible(i, j) = j <= i                 for history rows (i < n_u)
+ *                 = j < n_u  or  j == i    for candidate rows
+ *   O_i = sum_j softmax_j(s_ij) v_j over visible j;  LSE_i = log sum_j exp(s_ij)
+ * p = pos from genrank_embed_assemble, t = ts.  No N x N bias is ever stored.
+ * Arguments:
+ *   max_seqlen   an upper bound of seq_offsets[u+1] - seq_offsets[u] (host value)
+ *   q, k, v      [T] rows of H * dh values; head h of token t starts at
+ *                ptr + t * tok_stride + h * dh (elements).  A fused [T, 3, H, dh]
+ *                projection output passes q = base, k = base + H*dh, v = base + 2*H*dh,
+ *                tok_stride = 3*H*dh.  tok_stride * sizeof(dtype) % 16 == 0 and
+ *                16-byte aligned bases are required.
+ *   pos [T] int32, ts [T] int64 (device); slope_pos, slope_time: HOST arrays [H]
+ *   scale        > 0, normally 1/sqrt(dh)
+ *   o            [T, H * dh] output, row stride o_stride elements (dtype)
+ *   lse          [H, T] fp32 natural-log LSE output, or NULL to skip
+ *   ws, ws_bytes caller scratch of at least genrank_attn_workspace_size(..., 0) bytes
+ * Supported: bf16 with dh = 64 runs the tcgen05/TMEM/TMA kernel; fp32 (any
+ * dtype) with dh in {32, 64, 128} runs the CUDA-core kernel.  H <= 64. */
+int genrank_attn_fwd(int B, int64_t T, const int32_t *seq_offsets, const int32_t *hist_len, int max_seqlen,
+                     const void *q, const void *k, const void *v, int64_t tok_stride, int H,
+                     int dh, const int32_t *pos, const int64_t *ts, const float *slope_pos,
+                     const float *slope_time, float scale, int dtype, void *o, int64_t o_stride,
+                     float *lse, void *ws, size_t ws_bytes, int32_t *dev_err,
+                     genrank_stream_t stream);
+
+/* Step a4: gradients of step a3 (training).  Given dO [T, H*dh] (row stride
+ * o_stride, like o), the forward's o and lse, writes dq, dk, dv with the layout
+ * of q, k, v (tok_stride).  The biases have no parameters, so there is no bias
+ * gradient.  With P = softmax(S): dV = P^T dO, dP = dO V^T,
+ * dS = P * (dP - rowsum(dO * O)), dQ = scale dS K, dK = scale dS^T Q.
+ * Every token row of dq/dk/dv is written (no accumulation into them). */
+int genrank_attn_bwd(int B, int64_t T, const int32_t *seq_offsets, const int32_t *hist_len, int max_seqlen,
+                     const void *q, const void *k, const void *v, int64_t tok_stride, int H,
+                     int dh, const int32_t *pos, const int64_t *ts, const float *slope_pos,
+                     const float *slope_time, float scale, int dtype, const void *o,
+                     const void *dO, int64_t o_stride, const float *lse, void *dq, void *dk,
+                     void *dv, void *ws, size_t ws_bytes, int32_t *dev_err,
+                     genrank_stream_t stream);
+
+/* Bytes of workspace genrank_attn_fwd (is_bwd = 0) or genrank_attn_bwd
+ * (is_bwd = 1) need for these sizes.  Returns 0 for invalid sizes. */
+size_t genrank_attn_workspace_size(int B, int64_t T, int H, int dh, int max_seqlen, int is_bwd);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GENRANK_H_ */

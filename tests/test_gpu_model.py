@@ -1,0 +1,75 @@
+"""End-to-end parity of the scoring and training steps (library kernels + torch
+blocks) against the float64 oracle on the same seeded inputs."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ref
+from gen import CONFIGS, make_batch, make_model
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def M():
+    from generative_ranking_recommendation_b200 import model as M
+    from generative_ranking_recommendation_b200.csrc import build
+
+    build.build()
+    return M
+
+
+@pytest.mark.parametrize("name,users", [("c0", None), ("c1", 32), ("c2", 6), ("c4_m256", 6)])
+def test_logits_parity(M, name, users):
+    cfg = CONFIGS[name]
+    batch = make_batch(cfg)
+    model = make_model(cfg)
+    gm = M.GenRankModel(cfg, model, "cuda")
+    db = M.DeviceBatch.from_batch(batch, "cuda")
+    z = gm.forward(db).cpu().numpy().astype(np.float64)
+    from generative_ranking_recommendation_b200 import genrank as G
+
+    assert G.check_error(gm.err) == 0
+    sel = list(range(batch.B)) if users is None else sorted(
+        np.random.default_rng(3).choice(cfg.B, users, replace=False).tolist())
+    zr = ref.model_logits(batch, model, sel)
+    cr_all = ref.cand_rows(batch)
+    where = {r: k for k, r in enumerate(cr_all)}
+    zg = z[[where[r] for r in ref.cand_rows(batch, sel)]]
+    if cfg.dtype == "f32":
+        assert np.max(np.abs(zg - zr)) <= 1e-4
+    else:
+        assert ref.rel_to_max(zg, zr) <= 2e-2
+
+
+def test_train_step_parity(M):
+    cfg = CONFIGS["c3"].with_(B=6, n_item=100_000)
+    batch = make_batch(cfg)
+    model = make_model(cfg)
+    gm = M.GenRankModel(cfg, model, "cuda")
+    db = M.DeviceBatch.from_batch(batch, "cuda")
+    loss, z, grads = gm.train_step(db)
+    from generative_ranking_recommendation_b200 import genrank as G
+
+    assert G.check_error(gm.err) == 0
+    # oracle: forward, BCE, analytic backward, scatter into the tables
+    item, ids = ref.compact_items(batch, model)
+    mr = ref.meta(batch)
+    E = oracle.embed_assemble(batch.seq_offsets, batch.hist_len, ids, batch.action_ids, mr, item,
+                              model.action_tab, model.pos_tab, model.ri_tab, model.rt_tab)
+    zr, cache = oracle.block_forward(E, model.layers, model.w_head, batch.seq_offsets,
+                                     batch.hist_len, mr[0], batch.ts, cfg.H, cfg.ffn)
+    assert ref.rel_to_max(z.cpu().numpy(), zr) <= 2e-2
+    lr = oracle.bce_loss(zr, batch.labels)
+    assert abs(float(loss) - lr) <= 2e-2 * abs(lr)
+    dE = oracle.block_backward(zr, batch.labels, cache, model.layers, model.w_head,
+                               batch.seq_offsets, batch.hist_len, mr[0], batch.ts, cfg.H, cfg.ffn)
+    uniq = np.unique(batch.item_ids)
+    gr = oracle.embed_assemble_bwd(dE, batch.seq_offsets, batch.hist_len, ids, batch.action_ids,
+                                   mr, len(uniq), 9, cfg.n_pos, cfg.n_ri, cfg.n_rt)
+    got = {k: v.cpu().numpy().astype(np.float64) for k, v in grads.items()}
+    assert ref.rel_to_max(got["item"][uniq], gr["item"]) <= 2e-2
+    for k in ("action", "pos", "ri", "rt"):
+        assert ref.rel_to_max(got[k], gr[k]) <= 2e-2, k

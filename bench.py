@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark of the GenRank hot path on B200.
+
+Workload (default): inference scoring, 256 users, history lengths U[32,480],
+128 candidates each, d = 256 (4 heads x 64), 1 layer, bf16 with fp32
+accumulation, item table 1M rows, Zipf(1.1) ids, synthetic seeded data.
+One step = embedding assembly (metadata + five-way gather-sum) -> fused QKV
+projection -> candidate-masked ALiBi attention -> output projection and
+residual -> candidate head.  Metric: candidates scored per second (whole job),
+with the attention kernel's algorithmic TFLOP/s against the bf16 peak in
+``roofline``.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Multi-GPU: one process per GPU (torchrun), each rank scores its own shard of
+users (weak scaling, no collective on the data path); the step time is the max
+over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "candidates scored/sec and attention TFLOP/s (% of B200 bf16 tensor peak)"
+UNIT = "candidates/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_tc_traffic.json")
+ATTN_SRC = os.path.join(ROOT, "generative_ranking_recommendation_b200", "csrc", "attn_tc.cu")
+L2_FLUSH_BYTES = 256 << 20  # larger than the 126 MB L2
+
+
+# ------------------------------------------------------------------------------------------
+# workload arithmetic
+# ------------------------------------------------------------------------------------------
+def attn_pairs(seq_offsets, hist_len) -> int:
+    """Visible (query, key) pairs: n(n+1)/2 causal history + m n candidates x history + m self."""
+    n = np.asarray(hist_len, np.int64)
+    m = np.diff(np.asarray(seq_offsets, np.int64)) - n
+    return int(np.sum(n * (n + 1) // 2 + m * n + m))
+
+
+def attn_flops(seq_offsets, hist_len, d) -> float:
+    return 4.0 * d * attn_pairs(seq_offsets, hist_len)
+
+
+def embed_bytes(T, d, elem) -> float:
+    """Item row read + E row written + ids/ts read + 3 int32 metadata written, per token."""
+    return float(T) * (2 * d * elem + 4 + 4 + 8 + 12)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    with open(ATTN_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from an ncu capture, if it was
+    taken on the current kernel source; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("source_sha256_16") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k] == "Active"})
+        loaded = [x for x in sm if x > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------------
+# CPU baseline: the float64 oracle on the host cores (process pool over users)
+# ------------------------------------------------------------------------------------------
+def _oracle_user(args):
+    """Oracle logits of one user (independent of the others): metadata, embedding
+    sum, the block and the head, in float64."""
+    name, u = args
+    import oracle
+    from gen import CONFIGS, make_batch, make_model
+
+    cfg = CONFIGS[name]
+    b = make_batch(cfg, users=[u])
+    mdl = make_model(cfg)
+    uniq, ids = np.unique(b.item_ids, return_inverse=True)
+    meta = oracle.token_metadata(b.seq_offsets, b.hist_len, b.ts, cfg.n_ri, cfg.n_rt)
+    E = oracle.embed_assemble(b.seq_offsets, b.hist_len, ids, b.action_ids, meta,
+                              mdl.item_rows(uniq), mdl.action_tab, mdl.pos_tab, mdl.ri_tab,
+                              mdl.rt_tab)
+    z, _ = oracle.block_forward(E, mdl.layers, mdl.w_head, b.seq_offsets, b.hist_len, meta[0],
+                                b.ts, cfg.H, cfg.ffn)
+    return len(z)
+
+
+def _pool(cores):
+    """Spawned workers, one BLAS thread each (one user per task)."""
+    import multiprocessing as mp
+
+    for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[k] = "1"
+    return mp.get_context("spawn").Pool(cores)
+
+
+def cpu_baseline(name: str, B: int, target_s: float = 15.0):
+    cores = max(1, len(os.sched_getaffinity(0)))
+    t0 = time.perf_counter()
+    _oracle_user((name, 0))
+    per_user = time.perf_counter() - t0
+    n_users = int(min(B, max(cores, round(target_s * cores / max(per_user, 1e-3)))))
+    users = [(name, u) for u in range(n_users)]
+    with _pool(cores) as pool:
+        pool.map(_oracle_user, users[:cores])  # import warm-up in every worker
+        t0 = time.perf_counter()
+        cands = sum(pool.map(_oracle_user, users))
+        dt = time.perf_counter() - t0
+    return {"value": cands / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_users} of the {B} users of the workload (all their {cands} candidates), "
+                      f"float64 numpy oracle, one user per task in a {cores}-process pool",
+            "seconds": dt}
+
+
+# ------------------------------------------------------------------------------------------
+# arms
+# ------------------------------------------------------------------------------------------
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def config_block(cfg, world, extra=None):
+    c = {"workload": f"inference scoring ({cfg.name}): {cfg.B} users/GPU, history "
+                     f"U[{cfg.hist[1]},{cfg.hist[2]}], {cfg.m} candidates, d={cfg.d} "
+                     f"({cfg.H}x{cfg.dh}), {cfg.layers} layer, item table {cfg.n_item} rows",
+         "global_batch_users": cfg.B * world, "candidates_per_step": cfg.B * cfg.m * world,
+         "parallelism": f"users sharded over {world} GPU(s), no collective on the data path",
+         "l2": "flushed (256 MB write) before every timed step"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def run_reference(args, cfg, world, rank):
+    """The oracle as the reference arm: each step scores a bounded sample of users."""
+    if rank != 0:
+        return
+    cores = max(1, len(os.sched_getaffinity(0)))
+    users_per_step = cores
+    with _pool(cores) as pool:
+        times = []
+        cands = 0
+        for k in range(args.warmup + args.steps):
+            batch_users = [(cfg.name, (k * users_per_step + j) % cfg.B) for j in range(users_per_step)]
+            t0 = time.perf_counter()
+            c = sum(pool.map(_oracle_user, batch_users))
+            dt = time.perf_counter() - t0
+            if k >= args.warmup:
+                times.append(dt)
+                cands += c
+    total = sum(times)
+    value = cands / total
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded generator shaped like the pages' workloads)",
+           "config": config_block(cfg, 1, {"reference_sample": f"{users_per_step} users per step"}),
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                            "sample": f"{users_per_step} users of the workload per step, "
+                                      f"float64 numpy oracle, {cores}-process pool"},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def run_native(args, cfg, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    from gen import make_batch, make_model
+    from generative_ranking_recommendation_b200 import genrank as G
+    from generative_ranking_recommendation_b200.model import DeviceBatch, GenRankModel
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+
+    users = list(range(rank * cfg.B, (rank + 1) * cfg.B))
+    batches = [make_batch(cfg, users=users, seed=cfg.seed + 1000 * k) for k in range(2)]
+    mdl = make_model(cfg)
+    gm = GenRankModel(cfg, mdl, dev)
+    dbs = [DeviceBatch.from_batch(b, dev) for b in batches]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def sync_all():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for k in range(args.warmup):
+        gm.forward(dbs[k % 2])
+    torch.cuda.synchronize()
+    assert G.check_error(gm.err) == 0, "device error flags raised during warm-up"
+
+    # ---- device-resident inputs, CUDA events per step, L2 flushed between steps
+    sampler = ClockSampler(local)
+    sync_all()
+    sampler.start()
+    ev = []
+    attn_ev = []
+    for k in range(args.steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        gm.forward(dbs[k % 2], attn_events=attn_ev)
+        e.record()
+        ev.append((s, e))
+    sync_all()
+    clocks = sampler.stop()
+    step_ms = [s.elapsed_time(e) for s, e in ev]
+    total_ms = sum(step_ms)
+    attn_ms = [s.elapsed_time(e) for s, e in attn_ev]
+
+    # ---- end to end through the public API: pinned host inputs -> device -> logits -> host
+    host = [DeviceBatch.host_arrays(b) for b in batches]
+    pinned = [[torch.from_numpy(np.ascontiguousarray(a)).pin_memory() for a in h] for h in host]
+    dev_bufs = [[torch.empty(p.shape, dtype=p.dtype, device=dev) for p in ps] for ps in pinned]
+    n_cand = int(sum(b.cand_count.sum() for b in batches[:1]))
+    out_host = torch.empty(n_cand, dtype=torch.float32).pin_memory()
+    h2d = sum(p.numel() * p.element_size() for p in pinned[0])
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step(k):
+        i = k % 2
+        for p, d in zip(pinned[i], dev_bufs[i]):
+            d.copy_(p, non_blocking=True)
+        db = DeviceBatch.from_tensors(batches[i], dev_bufs[i])
+        z = gm.forward(db)
+        out_host.copy_(z, non_blocking=True)
+
+    for k in range(2):
+        e2e_step(k)
+    sync_all()
+    ev2 = []
+    for k in range(args.steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        e2e_step(k)
+        e.record()
+        ev2.append((s, e))
+    sync_all()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in ev2)
+    assert G.check_error(gm.err) == 0, "device error flags raised during the timed region"
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    cands_per_step = cfg.B * cfg.m * world
+    value = cands_per_step / (total_ms / args.steps / 1e3)
+    peaks, src = load_peaks()
+    flops = np.mean([attn_flops(b.seq_offsets, b.hist_len, cfg.d) for b in batches])
+    attn_avg_ms = float(np.mean(attn_ms))
+    achieved = flops / (attn_avg_ms / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generator shaped like the pages' workloads; random-init "
+                "tables and weights)",
+        "config": config_block(cfg, world),
+        "attention_tflops": achieved,
+        "attention_pct_of_bf16_peak": 100.0 * achieved / peak,
+        "roofline": {"bound": "tensor", "kernel": "k_attn_fwd_tc", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{src} bf16 (burst, cuBLAS 8192^3)",
+                     "traffic": measured_traffic(cfg.name),
+                     "algorithmic_flops_per_launch": flops,
+                     "avg_launch_ms": attn_avg_ms},
+        "e2e": {"value": cands_per_step / (e2e_ms / args.steps / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 4 * args.steps * cfg.layers,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(cfg.name, cfg.B)
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--config", default="c1")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from gen import CONFIGS
+
+    cfg = CONFIGS[args.config]
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, cfg, world, rank)
+    else:
+        run_native(args, cfg, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+"""Per-kernel benchmark of the hot path on one workload configuration.
+
+    python -m generative_ranking_recommendation_b200.kbench --config c2 \
+        [--kernels embed_fwd,attn_fwd,attn_bwd,embed_bwd] [--iters 20] [--warmup 3]
+
+Times each library call with CUDA events (inputs resident in HBM, L2 flushed
+before every timed launch) and prints one JSON line per kernel with its
+algorithmic throughput: GB/s for the embedding kernels, TFLOP/s for attention
+(4 d flops per visible pair forward, 10 d backward; masked pairs and padding
+not counted).  Attention operands are unit-scale random bf16 values.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import sys
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from gen import CONFIGS, item_table_torch, make_batch, make_model  # noqa: E402
+
+from . import genrank as G  # noqa: E402
+
+
+def visible_pairs(off, hl):
+    n = np.asarray(hl, np.int64)
+    m = np.diff(np.asarray(off, np.int64)) - n
+    return int(np.sum(n * (n + 1) // 2 + m * n + m))
+
+
+def positions(batch):
+    pos = np.zeros(batch.T, np.int32)
+    for u in range(batch.B):
+        s, e, n = batch.seq_offsets[u], batch.seq_offsets[u + 1], batch.hist_len[u]
+        pos[s:s + n] = np.arange(1, n + 1)
+        pos[s + n:e] = n + 1
+    return pos
+
+
+def timed(fn, iters, warmup, flush):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(iters):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        ts.append((s, e))
+    torch.cuda.synchronize()
+    return float(np.median([s.elapsed_time(e) for s, e in ts]))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--config", default="c1")
+    ap.add_argument("--kernels", default="embed_fwd,attn_fwd,attn_bwd,embed_bwd")
+    ap.add_argument("--iters", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    args = ap.parse_args(argv)
+    cfg = CONFIGS[args.config]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    batch = make_batch(cfg)
+    T, H, dh, d = batch.T, cfg.H, cfg.dh, cfg.d
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    es = 2 if cfg.dtype == "bf16" else 4
+    off = torch.from_numpy(batch.seq_offsets).to(dev)
+    hl = torch.from_numpy(batch.hist_len).to(dev)
+    ids = torch.from_numpy(batch.item_ids).to(dev)
+    acts = torch.from_numpy(batch.action_ids).to(dev)
+    ts = torch.from_numpy(batch.ts).to(dev)
+    pos = torch.from_numpy(positions(batch)).to(dev)
+    msl = int(np.max(np.diff(batch.seq_offsets)))
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sp, st = G.alibi_slopes(H)
+    scale = 1.0 / math.sqrt(dh)
+    kernels = args.kernels.split(",")
+    base = {"config": cfg.name, "T": T, "B": batch.B, "H": H, "dh": dh}
+    pairs = visible_pairs(batch.seq_offsets, batch.hist_len)
+
+    if "embed_fwd" in kernels or "embed_bwd" in kernels:
+        mdl = make_model(cfg)
+        item = item_table_torch(cfg.seed, cfg.n_item, d, cfg.dtype, dev)
+        tabs = [item] + [torch.from_numpy(x).to(dev, tdt)
+                         for x in (mdl.action_tab, mdl.pos_tab, mdl.ri_tab, mdl.rt_tab)]
+        E = torch.empty((T, d), dtype=tdt, device=dev)
+        meta = [torch.empty(T, dtype=torch.int32, device=dev) for _ in range(3)]
+
+        def fe():
+            G.embed_assemble(off, hl, ids, acts, ts, *tabs, E, *meta, err)
+
+        if "embed_fwd" in kernels:
+            ms = timed(fe, args.iters, args.warmup, flush)
+            nbytes = T * (2 * d * es + 28)
+            print(json.dumps({**base, "kernel": "embed_fwd", "ms": ms,
+                              "GB_per_s": nbytes / ms / 1e6, "algorithmic_bytes": nbytes}),
+                  flush=True)
+        if "embed_bwd" in kernels:
+            fe()
+            dE = torch.randn((T, d), device=dev).to(tdt)
+            f32 = dict(dtype=torch.float32, device=dev)
+            grads = [torch.zeros(t.shape, **f32) for t in tabs]
+
+            def fb():
+                G.embed_assemble_bwd(off, hl, ids, acts, *meta, dE, *grads, err)
+
+            ms = timed(fb, args.iters, args.warmup, flush)
+            nbytes = T * (d * es + 4 * d + 28)  # dE read, item-row reduction, ids and metadata
+            print(json.dumps({**base, "kernel": "embed_bwd", "ms": ms,
+                              "GB_per_s": nbytes / ms / 1e6, "algorithmic_bytes": nbytes}),
+                  flush=True)
+
+    if "attn_fwd" in kernels or "attn_bwd" in kernels:
+        g = torch.Generator(device=dev)
+        g.manual_seed(cfg.seed)
+        qkv = torch.randn((T, 3 * d), device=dev, generator=g).to(tdt)
+        o = torch.empty((T, d), dtype=tdt, device=dev)
+        lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(G.attn_workspace_size(batch.B, T, H, dh, msl, False),
+                             G.attn_workspace_size(batch.B, T, H, dh, msl, True)),
+                         dtype=torch.uint8, device=dev)
+
+        def fa():
+            G.attn_fwd(off, hl, msl, qkv, qkv[:, d:], qkv[:, 2 * d:], 3 * d, H, dh, pos, ts, sp,
+                       st, scale, o, d, lse, ws, err, T=T)
+
+        if "attn_fwd" in kernels:
+            ms = timed(fa, args.iters, args.warmup, flush)
+            fl = 4.0 * d * pairs
+            print(json.dumps({**base, "kernel": "attn_fwd", "ms": ms, "TFLOP_per_s": fl / ms / 1e9,
+                              "algorithmic_flops": fl, "visible_pairs": pairs}), flush=True)
+        if "attn_bwd" in kernels:
+            fa()
+            do = torch.randn((T, d), device=dev, generator=g).to(tdt)
+            dqkv = torch.empty_like(qkv)
+
+            def fb():
+                G.attn_bwd(off, hl, msl, qkv, qkv[:, d:], qkv[:, 2 * d:], 3 * d, H, dh, pos, ts,
+                           sp, st, scale, o, do, d, lse, dqkv, dqkv[:, d:], dqkv[:, 2 * d:], ws,
+                           err, T=T)
+
+            ms = timed(fb, args.iters, args.warmup, flush)
+            fl = 10.0 * d * pairs
+            print(json.dumps({**base, "kernel": "attn_bwd", "ms": ms, "TFLOP_per_s": fl / ms / 1e9,
+                              "algorithmic_flops": fl, "visible_pairs": pairs}), flush=True)
+    code = G.check_error(err)
+    if code:
+        raise SystemExit(f"device error flags: {code}")
+
+
+if __name__ == "__main__":
+    main()

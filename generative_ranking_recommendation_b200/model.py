@@ -141,15 +141,25 @@ class GenRankModel:
 
     # -------------------------------------------------------------------------------------
     @torch.no_grad()
-    def forward(self, db: DeviceBatch) -> torch.Tensor:
-        """Candidate logits (fp32 [sum m]) for one batch."""
+    def forward(self, db: DeviceBatch, attn_events=None) -> torch.Tensor:
+        """Candidate logits (fp32 [sum m]) for one batch.
+
+        ``attn_events``: optional list; a (start, end) pair of CUDA events recorded
+        on the current stream around each attention launch is appended to it.
+        """
         E, (pos, _, _) = self.embed(db)
         ffn = self.cfg.ffn
         x = E.float()
         for W in self.layers:
             a = (self.rms(x) if ffn else x).to(self.dtype)
             qkv = a @ W["Wqkv"]
+            if attn_events is not None:
+                ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                ev[0].record()
             o, _ = self.attention(db, qkv, pos)
+            if attn_events is not None:
+                ev[1].record()
+                attn_events.append(ev)
             x = x + (o @ W["Wo"]).float()
             if ffn:
                 f = self.rms(x).to(self.dtype)

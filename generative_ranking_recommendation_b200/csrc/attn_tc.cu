@@ -6,24 +6,28 @@
 //   candidate rows see all history and themselves.
 //
 // Design (bf16 inputs, head dim 64, fp32 accumulation):
-//   * Work items are (user, 128-row query tile, head).  A one-block scheduling
-//     kernel lists the (user, tile) pairs sorted by the number of 128-key tiles
-//     they visit (longest first); a persistent grid of one CTA per SM walks the
-//     list round-robin.  Key tiles a query tile never sees are never visited:
-//     history tile t visits key tiles 0..t, candidate rows visit the history only.
-//   * Warp 4 loads Q, K, V tiles with TMA (128B swizzle, no multicast) into a
-//     two-stage ring and writes the per-key bias column for the stage.
-//   * Warp 5 issues tcgen05.mma: S = Q K^T (128x128, fp32 in TMEM, two buffers)
-//     and O_part = P V (128x64, fp32 in TMEM, two buffers).
-//   * Warps 0-3 (one thread per query row, one TMEM lane each) run the online
-//     softmax on S, write P in bf16 to shared memory in the UMMA K-major
-//     swizzled layout, and fold each O_part into a register-resident O.
-//   * On visible pairs p_i >= p_j and t_i >= t_j, so the bias splits into a row
-//     term that cancels in the softmax and a column term c_j = m p_j + m_t (t_j - t_0);
-//     only c_j is added per element.  The literal LSE is recovered in the epilogue.
+//   * A prologue kernel lists (user, 128-row query tile) work records sorted by the
+//     number of 128-key tiles they visit (longest first), and writes the ALiBi
+//     column term c_j = log2(e) (m_h p_j + m_t,h (t_j - t_0)) for every token and
+//     head into a 16-byte aligned scratch layout.  On visible pairs p_i >= p_j and
+//     t_i >= t_j, so the bias is c_j - c_i; c_i cancels in the softmax and only c_j
+//     is added per element; the literal LSE subtracts c_i in the epilogue.
+//   * Persistent grid, two CTAs per SM; each CTA walks the records round-robin
+//     (one head per work item).  Key tiles a query tile never sees are never
+//     visited: history tile t visits key tiles 0..t, candidate rows the history only.
+//   * Warp 4 issues TMA loads (Q; K, V two-stage ring; 128B swizzle, no multicast)
+//     and a bulk copy of the key tile's column terms.
+//   * Warp 5 (one thread) issues tcgen05.mma: S = Q K^T (128 x 128, fp32 in TMEM)
+//     from shared memory, then O += P V (128 x 64, fp32 in TMEM) with P read from
+//     tensor memory, where the softmax left it in place of S (bf16 pairs).
+//   * Warps 0-3 (one query row per thread, one TMEM lane each) load S, add the
+//     column term, mask only tiles that straddle a row's last visible key, and run
+//     the online softmax with a lazily updated offset: O in TMEM is rescaled only
+//     when a row's maximum grows by more than 2^8, so most tiles touch O not at all.
+//   * The other CTA on the SM hides each CTA's per-item latencies (work-record
+//     loads, the epilogue's global loads and stores).
 //   * A candidate's own key lies outside the tiles it visits; its score (bias 0)
 //     is merged into the softmax state in the epilogue on CUDA cores.
-//   * Masks are evaluated only on tiles that straddle a row's last visible key.
 // Every mbarrier wait is bounded in time; a timeout sets GENRANK_DERR_TIMEOUT,
 // every role drains out of its loop and the CTA frees its tensor memory.
 #include <cuda.h>
@@ -38,124 +42,136 @@ namespace tc {
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
 constexpr int DH = 64;   // head dim
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;  // warps 0-3 softmax, warp 4 TMA, warp 5 MMA
 constexpr uint32_t kTileBytes = BM * DH * 2;  // one Q, K or V tile (16 KB)
-constexpr uint32_t kPBytes = BM * BN * 2;     // one P tile (32 KB)
+constexpr uint32_t kCBBytes = BN * 4;         // column terms of one key tile
+constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 // dynamic shared memory layout (offsets from a 1024-byte aligned base)
-constexpr uint32_t kOffQ = 0;                          // 2 x 16 KB
-constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;     // 2 x 16 KB
+constexpr uint32_t kOffQ = 0;                          // 16 KB
+constexpr uint32_t kOffK = kOffQ + kTileBytes;         // 2 x 16 KB
 constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;     // 2 x 16 KB
-constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;     // 2 x 32 KB
-constexpr uint32_t kOffCB = kOffP + 2 * kPBytes;       // 2 x 128 floats
-constexpr uint32_t kOffBar = kOffCB + 2 * BN * 4;      // barriers
-constexpr uint32_t kNumBars = 18;
+constexpr uint32_t kOffCB = kOffV + 2 * kTileBytes;    // 2 x 512 B
+constexpr uint32_t kOffBar = kOffCB + 2 * kCBBytes;    // barriers
+constexpr uint32_t kNumBars = 12;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
 
-// TMEM columns
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;    // S buffers at 0 and 128
-constexpr uint32_t kColO = 256;  // O_part buffers at 256 and 320
+// TMEM columns (per CTA; two CTAs share an SM's 512)
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0;    // S (fp32, 128 columns); P (bf16 pairs) in its first 64
+constexpr uint32_t kColO = 128;  // O (fp32, 64 columns)
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);   // Q K-major, K K-major
-constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, DH, 0, 1);  // P K-major, V MN-major
+constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, DH, 0, 1);  // P K-major (TMEM), V MN-major
 
-constexpr int kItemTileBits = 10;  // item = (user << 10) | query tile
+// scratch layout
+constexpr size_t kHeaderBytes = 256;
+constexpr int kRecInts = 8;  // s, L, n, q0, nk, spad, u, unused
 
 struct Params {
   CUtensorMap tq, tk, tv;
   AttnArgs a;
-  const int32_t* items;  // [count] sorted (user, tile) pairs
-  const int32_t* count;
+  const int4* recs;      // [count][2] work records
+  const int32_t* count;  // number of records
+  const float* cbias;    // [H][Tp] column terms (log2 units)
+  long long Tp;
 };
 
-enum Bar {
-  kQFull = 0, kQEmpty = 2, kKFull = 4, kVFull = 6, kKVEmpty = 8, kCBFull = 10, kSFull = 12,
-  kPFull = 14, kPVFull = 16
-};
+enum Bar { kQFull = 0, kQEmpty = 1, kKFull = 2, kVFull = 4, kKVEmpty = 6, kSFull = 8,
+           kPFull = 9, kPVFull = 10 };
 
 struct Item {
-  long long s;  // first token of the user
-  int L, n;     // tokens, history tokens
-  int q0;       // first query row (local)
-  int nk;       // key tiles visited
-  int h;
-  bool ok;
+  int s, L, n, q0, nk, spad, h;
 };
 
 GR_DEVICE Item load_item(const Params& P, int w) {
-  const AttnArgs& a = P.a;
+  const int pair = w / P.a.H;
+  const int4 r0 = P.recs[2 * pair];
+  const int4 r1 = P.recs[2 * pair + 1];
   Item it;
-  const int pair = w / a.H;
-  it.h = w - pair * a.H;
-  const int rec = P.items[pair];
-  const int u = rec >> kItemTileBits;
-  const int t = rec & ((1 << kItemTileBits) - 1);
-  it.s = a.off[u];
-  const long long e = a.off[u + 1];
-  it.ok = !(it.s < 0 || e < it.s || e > a.T);
-  it.L = it.ok ? (int)(e - it.s) : 0;
-  it.n = max(0, min(a.hist_len[u], it.L));
-  it.q0 = t * BM;
-  const int kmax = min(it.q0 + BM, it.n);  // keys [0, kmax) are visited
-  it.nk = (it.ok && kmax > 0) ? (kmax + BN - 1) / BN : 0;
+  it.h = w - pair * P.a.H;
+  it.s = r0.x;
+  it.L = r0.y;
+  it.n = r0.z;
+  it.q0 = r0.w;
+  it.nk = r1.x;
+  it.spad = r1.y;
   return it;
 }
 
+// Start of user u's segment in the column-term scratch: 16-byte aligned and
+// disjoint from the previous user's (4 ceil(s/4) + 4u grows by at least L + 1).
+__host__ __device__ inline long long seg_start(long long s, int u) {
+  return 4 * ((s + 3) / 4) + 4LL * u;
+}
+__host__ __device__ inline long long scratch_tp(long long T, int B) {
+  return ((T + 4LL * B + 4 + BN) + 3) / 4 * 4;
+}
+
 // ------------------------------------------------------------------------------------------
-// scheduling: (user, query tile) pairs sorted by visited key tiles, longest first
+// prologue: work records (block B) and column terms (blocks 0..B-1)
 // ------------------------------------------------------------------------------------------
 constexpr int kMaxNkBuckets = 257;
 
-__global__ void __launch_bounds__(1024) k_schedule(int B, long long T, const int32_t* off,
-                                                   const int32_t* hist_len, int max_tiles,
-                                                   int32_t* items, int32_t* count,
-                                                   int32_t* err) {
+__global__ void __launch_bounds__(256) k_prologue(const __grid_constant__ AttnArgs a,
+                                                  int max_tiles, int4* recs, int32_t* count,
+                                                  float* cbias, long long Tp) {
+  const int b = blockIdx.x;
+  if (b < a.B) {
+    const long long s = a.off[b], e = a.off[b + 1];
+    if (s < 0 || e < s || e > a.T) return;  // flagged by the schedule block
+    const int L = (int)(e - s);
+    const long long base = seg_start(s, b);
+    const long long t0 = L > 0 ? a.ts[s] : 0;
+    for (int i = threadIdx.x; i < L; i += blockDim.x) {
+      const float p = (float)a.pos[s + i];
+      const float dt = (float)(a.ts[s + i] - t0);
+      for (int h = 0; h < a.H; ++h)
+        cbias[(long long)h * Tp + base + i] = kLog2e * (a.slope_pos[h] * p + a.slope_time[h] * dt);
+    }
+    return;
+  }
+  // schedule: histogram of visited key tiles, then a scatter longest first
   __shared__ int hist[kMaxNkBuckets];
   __shared__ int cursor[kMaxNkBuckets];
   for (int i = threadIdx.x; i < kMaxNkBuckets; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  // pass 1: histogram of visited key tiles
-  for (int u = threadIdx.x; u < B; u += blockDim.x) {
-    const long long s = off[u], e = off[u + 1];
-    if (s < 0 || e < s || e > T) {
-      flag(err, GENRANK_DERR_LAYOUT);
-      continue;
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int u = threadIdx.x; u < a.B; u += blockDim.x) {
+      const long long s = a.off[u], e = a.off[u + 1];
+      if (s < 0 || e < s || e > a.T) {
+        if (pass == 0) flag(a.err, GENRANK_DERR_LAYOUT);
+        continue;
+      }
+      const int L = (int)(e - s);
+      const int n = max(0, min(a.hist_len[u], L));
+      const int tiles_all = (L + BM - 1) / BM;
+      if (pass == 0 && tiles_all > max_tiles) flag(a.err, GENRANK_DERR_LAYOUT);
+      const int tiles = min(tiles_all, max_tiles);
+      for (int t = 0; t < tiles; ++t) {
+        const int kmax = min(t * BM + BM, n);
+        const int nk = kmax > 0 ? (kmax + BN - 1) / BN : 0;
+        const int bucket = min(nk, kMaxNkBuckets - 1);
+        if (pass == 0) {
+          atomicAdd(&hist[bucket], 1);
+        } else {
+          const int slot = atomicAdd(&cursor[bucket], 1);
+          recs[2 * slot] = make_int4((int)s, L, n, t * BM);
+          recs[2 * slot + 1] = make_int4(nk, (int)seg_start(s, u), u, 0);
+        }
+      }
     }
-    const int L = (int)(e - s);
-    const int n = max(0, min(hist_len[u], L));
-    const int tiles = min((L + BM - 1) / BM, max_tiles);
-    if ((L + BM - 1) / BM > max_tiles) flag(err, GENRANK_DERR_LAYOUT);
-    for (int t = 0; t < tiles; ++t) {
-      const int kmax = min(t * BM + BM, n);
-      const int nk = min(kmax > 0 ? (kmax + BN - 1) / BN : 0, kMaxNkBuckets - 1);
-      atomicAdd(&hist[nk], 1);
+    __syncthreads();
+    if (pass == 0 && threadIdx.x == 0) {
+      int acc = 0;
+      for (int q = kMaxNkBuckets - 1; q >= 0; --q) {
+        cursor[q] = acc;
+        acc += hist[q];
+      }
+      *count = acc;
     }
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int b = kMaxNkBuckets - 1; b >= 0; --b) {
-      cursor[b] = acc;
-      acc += hist[b];
-    }
-    *count = acc;
-  }
-  __syncthreads();
-  // pass 2: scatter
-  for (int u = threadIdx.x; u < B; u += blockDim.x) {
-    const long long s = off[u], e = off[u + 1];
-    if (s < 0 || e < s || e > T) continue;
-    const int L = (int)(e - s);
-    const int n = max(0, min(hist_len[u], L));
-    const int tiles = min((L + BM - 1) / BM, max_tiles);
-    for (int t = 0; t < tiles; ++t) {
-      const int kmax = min(t * BM + BM, n);
-      const int nk = min(kmax > 0 ? (kmax + BN - 1) / BN : 0, kMaxNkBuckets - 1);
-      const int slot = atomicAdd(&cursor[nk], 1);
-      items[slot] = (u << kItemTileBits) | t;
-    }
+    __syncthreads();
   }
 }
 
@@ -171,7 +187,7 @@ GR_DEVICE bool wait_warp(uint64_t* bar, uint32_t par, volatile int* abort_flag, 
   return __all_sync(0xffffffffu, ok);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_constant__ Params P) {
+__global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_constant__ Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -179,21 +195,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  float* sCB = reinterpret_cast<float*>(smem + kOffCB);
+  const float* sCB = reinterpret_cast<const float*>(smem + kOffCB);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    mbar_init(&bars[kQFull], 1);
+    mbar_init(&bars[kQEmpty], 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars[kQFull + i], 1);
-      mbar_init(&bars[kQEmpty + i], 1);
       mbar_init(&bars[kKFull + i], 1);
       mbar_init(&bars[kVFull + i], 1);
       mbar_init(&bars[kKVEmpty + i], 1);
-      mbar_init(&bars[kCBFull + i], 32);
-      mbar_init(&bars[kSFull + i], 1);
-      mbar_init(&bars[kPFull + i], 128);
-      mbar_init(&bars[kPVFull + i], 1);
     }
+    mbar_init(&bars[kSFull], 1);
+    mbar_init(&bars[kPFull], 128);
+    mbar_init(&bars[kPVFull], 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -210,7 +225,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
   const int total = *P.count * a.H;
 
   if (warp == 4) {
@@ -220,15 +234,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const Item it = load_item(P, w);
       if (it.nk == 0) continue;
-      const int qb = qi & 1;
-      if (!wait_warp(&bars[kQEmpty + qb], parity(qi >> 1) ^ 1u, abort_flag, a.err)) break;
+      if (!wait_warp(&bars[kQEmpty], parity(qi) ^ 1u, abort_flag, a.err)) break;
       if (lane == 0) {
-        mbar_expect_tx(&bars[kQFull + qb], kTileBytes);
-        tma_load_3d(smem + kOffQ + qb * kTileBytes, &P.tq, &bars[kQFull + qb], 0, it.h,
-                    (int)(it.s + it.q0));
+        mbar_expect_tx(&bars[kQFull], kTileBytes);
+        tma_load_3d(smem + kOffQ, &P.tq, &bars[kQFull], 0, it.h, it.s + it.q0);
       }
-      const float spos = a.slope_pos[it.h] * kLog2e, stime = a.slope_time[it.h] * kLog2e;
-      const long long t0 = a.ts[it.s];
+      const float* cb_src = P.cbias + (long long)it.h * P.Tp + it.spad;
       bool ok = true;
       for (int j = 0; j < it.nk; ++j, ++g) {
         const int st = g & 1;
@@ -236,26 +247,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
           ok = false;
           break;
         }
-        const int kv0 = j * BN;
         if (lane == 0) {
-          mbar_expect_tx(&bars[kKFull + st], kTileBytes);
+          const int kv0 = j * BN;
+          mbar_expect_tx(&bars[kKFull + st], kTileBytes + kCBBytes);
           tma_load_3d(smem + kOffK + st * kTileBytes, &P.tk, &bars[kKFull + st], 0, it.h,
-                      (int)(it.s + kv0));
+                      it.s + kv0);
+          bulk_load(smem + kOffCB + st * kCBBytes, cb_src + kv0, kCBBytes, &bars[kKFull + st]);
           mbar_expect_tx(&bars[kVFull + st], kTileBytes);
           tma_load_3d(smem + kOffV + st * kTileBytes, &P.tv, &bars[kVFull + st], 0, it.h,
-                      (int)(it.s + kv0));
+                      it.s + kv0);
         }
-        // bias column of this key tile, in log2 units: c_j = log2e (m p_j + m_t (t_j - t_0))
-        for (int c = lane; c < BN; c += 32) {
-          const int key = kv0 + c;
-          float cb = 0.f;
-          if (key < it.n) {
-            const long long tk = a.ts[it.s + key];
-            cb = spos * (float)a.pos[it.s + key] + stime * (float)(tk - t0);
-          }
-          sCB[st * BN + c] = cb;
-        }
-        mbar_arrive(&bars[kCBFull + st]);
       }
       if (!ok) break;
       ++qi;
@@ -264,188 +265,195 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
     // ---------------------------------------------------------------- MMA issuer (one thread)
     int qi = 0, g = 0;
     const uint32_t sQ = smem_u32(smem + kOffQ), sK = smem_u32(smem + kOffK),
-                   sV = smem_u32(smem + kOffV), sPb = smem_u32(smem + kOffP);
-    for (int w = blockIdx.x; w < total && !*abort_flag; w += gridDim.x) {
+                   sV = smem_u32(smem + kOffV);
+    bool ok = true;
+    for (int w = blockIdx.x; w < total && ok && !*abort_flag; w += gridDim.x) {
       const Item it = load_item(P, w);
       if (it.nk == 0) continue;
-      const int qb = qi & 1;
-      if (!mbar_wait(&bars[kQFull + qb], parity(qi >> 1), abort_flag, a.err)) break;
-      tc_fence_after();
-      bool ok = true;
-      auto issue_s = [&](int gg) -> bool {
-        const int st = gg & 1;
-        if (!mbar_wait(&bars[kKFull + st], parity(gg >> 1), abort_flag, a.err)) return false;
+      if (!mbar_wait(&bars[kQFull], parity(qi), abort_flag, a.err)) break;
+      for (int j = 0; j < it.nk; ++j, ++g) {
+        const int st = g & 1;
+        // K landed, and the previous P V finished (S overwrites that P)
+        if (!mbar_wait(&bars[kKFull + st], parity(g >> 1), abort_flag, a.err) ||
+            (g > 0 && !mbar_wait(&bars[kPVFull], parity(g - 1), abort_flag, a.err))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d = tmem + kColS + (uint32_t)(gg & 1) * BN;
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k) {
-          const uint64_t ad = smem_desc_sw128(sQ + qb * kTileBytes + k * 32, 16, 1024);
+          const uint64_t ad = smem_desc_sw128(sQ + k * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(sK + st * kTileBytes + k * 32, 16, 1024);
-          mma_bf16_ss(d, ad, bd, kIdescS, k > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + kColS, ad, bd, kIdescS, k > 0 ? 1u : 0u);
         }
-        mma_commit(&bars[kSFull + (gg & 1)]);
-        return true;
-      };
-      if (!issue_s(g)) break;
-      for (int j = 0; j < it.nk; ++j) {
-        const int gj = g + j;
-        if (j + 1 < it.nk && !issue_s(gj + 1)) {
-          ok = false;
-          break;
-        }
-        const int b = gj & 1;
-        if (!mbar_wait(&bars[kPFull + b], parity(gj >> 1), abort_flag, a.err) ||
-            !mbar_wait(&bars[kVFull + b], parity(gj >> 1), abort_flag, a.err)) {
+        mma_commit(&bars[kSFull]);
+        if (j == it.nk - 1) mma_commit(&bars[kQEmpty]);
+        if (!mbar_wait(&bars[kPFull], parity(g), abort_flag, a.err) ||
+            !mbar_wait(&bars[kVFull + st], parity(g >> 1), abort_flag, a.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + kColO + (uint32_t)b * DH;
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k) {
-          const uint64_t ad =
-              smem_desc_sw128(sPb + b * kPBytes + (k >> 2) * (BM * 128) + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sV + b * kTileBytes + k * 16 * 128, kTileBytes, 1024);
-          mma_bf16_ss(d, ad, bd, kIdescPV, k > 0 ? 1u : 0u);
+          const uint64_t bd = smem_desc_sw128(sV + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
+          mma_bf16_ts(tmem + kColO, tmem + kColS + k * 8, bd, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
         }
-        mma_commit(&bars[kPVFull + b]);
-        mma_commit(&bars[kKVEmpty + b]);
+        mma_commit(&bars[kPVFull]);
+        mma_commit(&bars[kKVEmpty + st]);
       }
-      if (!ok) break;
-      mma_commit(&bars[kQEmpty + qb]);
-      g += it.nk;
       ++qi;
     }
   } else if (warp < 4) {
     // ---------------------------------------------------------------- softmax warps 0-3
     const int r = threadIdx.x;  // query row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    uint8_t* sPbase = smem + kOffP;
     const float scale_log2 = a.scale * kLog2e;
+    const __nv_bfloat16* Qg = (const __nv_bfloat16*)a.q;
+    const __nv_bfloat16* Kg = (const __nv_bfloat16*)a.k;
+    const __nv_bfloat16* Vg = (const __nv_bfloat16*)a.v;
     int g = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
       __syncwarp();
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const Item it = load_item(P, w);
-      if (!it.ok) continue;
       const int i = it.q0 + r;
       const bool row = i < it.L;
+      const long long tok = (long long)it.s + i;
+      const bool cand = row && i >= it.n;
+      float rowcb = 0.f;
+      if (row) rowcb = P.cbias[(long long)it.h * P.Tp + it.spad + i];
+      if (cand) {  // warm L2 for the epilogue's self-term rows
+        prefetch_l2(Qg + tok * a.tok_stride + it.h * DH);
+        prefetch_l2(Kg + tok * a.tok_stride + it.h * DH);
+        prefetch_l2(Vg + tok * a.tok_stride + it.h * DH);
+      }
       const int lim = min(i, it.n - 1);
-      const int mask_from = min(it.q0, it.n - 1);  // tiles with kv0 + 127 > this need masks
-      float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
-      float o[DH];
-#pragma unroll
-      for (int c = 0; c < DH; ++c) o[c] = 0.f;
+      const int mask_from = min(it.q0, it.n - 1);  // a tile needs masks if kv0 + 127 > this
+      float m = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < it.nk; ++j) {
-        const int gj = g + j, b = gj & 1;
+      for (int j = 0; j < it.nk; ++j, ++g) {
+        const int st = g & 1;
         const int kv0 = j * BN;
-        if (!wait_warp(&bars[kCBFull + b], parity(gj >> 1), abort_flag, a.err) ||
-            !wait_warp(&bars[kSFull + b], parity(gj >> 1), abort_flag, a.err)) {
+        if (!wait_warp(&bars[kSFull], parity(g), abort_flag, a.err) ||
+            !wait_warp(&bars[kKFull + st], parity(g >> 1), abort_flag, a.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        float x[BN];
-        tmem_ld128(tmem + lane_base + kColS + b * BN, x);
-        const float* cb = sCB + b * BN;
+        const float* cb = sCB + st * BN;
+        const bool masked = kv0 + BN - 1 > mask_from;
+        // pass 1: row maximum of the biased scores, 32 columns at a time
         float mx = -INFINITY;
-        if (kv0 + BN - 1 > mask_from) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          float x[32];
+          tmem_ld32(tmem + lane_base + kColS + c0, x);
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const float v = fmaf(x[c], scale_log2, cb[c]);
-            x[c] = (kv0 + c <= lim) ? v : -INFINITY;
-            mx = fmaxf(mx, x[c]);
-          }
-        } else {
+          for (int c = 0; c < 32; c += 4) {
+            const float4 b4 = *reinterpret_cast<const float4*>(cb + c0 + c);
+            const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            x[c] = fmaf(x[c], scale_log2, cb[c]);
-            mx = fmaxf(mx, x[c]);
+            for (int e = 0; e < 4; ++e) {
+              float v = fmaf(x[c + e], scale_log2, bb[e]);
+              if (masked && kv0 + c0 + c + e > lim) v = -INFINITY;
+              mx = fmaxf(mx, v);
+            }
           }
         }
-        const float m_new = fmaxf(m, mx);
-        const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        const float alpha = ex2(m - m_use);
-        float rs = 0.f;
-        uint8_t* prow = sPbase + b * kPBytes + r * 128;
+        // lazy offset: move it (and rescale O in TMEM) only when the max grows by > 2^8
+        float alpha = 1.f;
+        if (j == 0) {
+          m = mx;
+        } else {
+          const bool need = mx > m + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, need)) {
+            const float m_new = need ? mx : m;
+            alpha = ex2(m - m_new);
+            m = m_new;
+#pragma unroll 1
+            for (int c0 = 0; c0 < DH; c0 += 32) {
+              float o[32];
+              tmem_ld32(tmem + lane_base + kColO + c0, o);
+              uint32_t ob[32];
 #pragma unroll
-        for (int c16 = 0; c16 < BN / 8; ++c16) {
-          float p[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            p[e] = ex2(x[c16 * 8 + e] - m_use);
-            rs += p[e];
+              for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(o[c] * alpha);
+              tmem_st32(tmem + lane_base + kColO + c0, ob);
+            }
           }
-          uint4 pk = make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
-                                pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
-          const int blk = c16 >> 3, cc = c16 & 7;
-          *reinterpret_cast<uint4*>(prow + blk * (BM * 128) + ((cc ^ (r & 7)) << 4)) = pk;
+        }
+        const float m_use = m == -INFINITY ? 0.f : m;
+        // pass 2: P = 2^(x - m) in bf16, written over S columns already consumed
+        // (chunk c0 of keys lands in columns [c0/2, c0/2 + 16), read by an earlier chunk)
+        float rs = 0.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          float x[32];
+          tmem_ld32(tmem + lane_base + kColS + c0, x);
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const float4 b4 = *reinterpret_cast<const float4*>(cb + c0 + c);
+            const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+            float p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float v = fmaf(x[c + e], scale_log2, bb[e]);
+              if (masked && kv0 + c0 + c + e > lim) v = -INFINITY;
+              p[e] = ex2(v - m_use);
+              rs += p[e];
+            }
+            pk[c / 2] = pack_bf16(p[0], p[1]);
+            pk[c / 2 + 1] = pack_bf16(p[2], p[3]);
+          }
+          tmem_st16(tmem + lane_base + kColS + c0 / 2, pk);
         }
         l = l * alpha + rs;
-        m = m_new;
-        fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&bars[kPFull + b]);
-        if (j >= 1) {
-          const int pb = (gj - 1) & 1;
-          if (!wait_warp(&bars[kPVFull + pb], parity((gj - 1) >> 1), abort_flag, a.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          float t[DH];
-          tmem_ld64(tmem + lane_base + kColO + pb * DH, t);
-#pragma unroll
-          for (int e = 0; e < DH; ++e) o[e] = fmaf(o[e], alpha_prev, t[e]);
-          tc_fence_before();
-        }
-        alpha_prev = alpha;
+        mbar_arrive(&bars[kPFull]);
       }
       if (!ok) break;
+      float o[DH];
       if (it.nk > 0) {
-        const int gl = g + it.nk - 1, pb = gl & 1;
-        if (!wait_warp(&bars[kPVFull + pb], parity(gl >> 1), abort_flag, a.err)) break;
+        if (!wait_warp(&bars[kPVFull], parity(g - 1), abort_flag, a.err)) break;
         tc_fence_after();
-        float t[DH];
-        tmem_ld64(tmem + lane_base + kColO + pb * DH, t);
-#pragma unroll
-        for (int e = 0; e < DH; ++e) o[e] = fmaf(o[e], alpha_prev, t[e]);
+        tmem_ld64(tmem + lane_base + kColO, o);
         tc_fence_before();
+      } else {
+#pragma unroll
+        for (int c = 0; c < DH; ++c) o[c] = 0.f;
       }
-      g += it.nk;
       if (!row) continue;
-      const long long tok = it.s + i;
-      const float spos = a.slope_pos[it.h], stime = a.slope_time[it.h];
-      const long long t0 = a.ts[it.s];
-      const float rowterm = spos * (float)a.pos[tok] + stime * (float)(a.ts[tok] - t0);
-      if (i >= it.n) {
+      if (cand) {
         // the candidate's own key: literal bias 0, i.e. column term == row term
-        const __nv_bfloat16* qp = (const __nv_bfloat16*)a.q + tok * a.tok_stride + it.h * DH;
-        const __nv_bfloat16* kp = (const __nv_bfloat16*)a.k + tok * a.tok_stride + it.h * DH;
-        const __nv_bfloat16* vp = (const __nv_bfloat16*)a.v + tok * a.tok_stride + it.h * DH;
+        const uint4* qp = reinterpret_cast<const uint4*>(Qg + tok * a.tok_stride + it.h * DH);
+        const uint4* kp = reinterpret_cast<const uint4*>(Kg + tok * a.tok_stride + it.h * DH);
+        const uint4* vp = reinterpret_cast<const uint4*>(Vg + tok * a.tok_stride + it.h * DH);
+        uint4 qa[DH / 8], ka[DH / 8];
+#pragma unroll
+        for (int c = 0; c < DH / 8; ++c) {
+          qa[c] = qp[c];
+          ka[c] = kp[c];
+        }
         float dot = 0.f;
 #pragma unroll
-        for (int c = 0; c < DH; c += 8) {
-          const uint4 qa = *reinterpret_cast<const uint4*>(qp + c);
-          const uint4 ka = *reinterpret_cast<const uint4*>(kp + c);
+        for (int c = 0; c < DH / 8; ++c) {
           float qf[8], kf[8];
-          Elem<__nv_bfloat16>::unpack(qa, qf);
-          Elem<__nv_bfloat16>::unpack(ka, kf);
+          Elem<__nv_bfloat16>::unpack(qa[c], qf);
+          Elem<__nv_bfloat16>::unpack(ka[c], kf);
 #pragma unroll
           for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
         }
-        const float xs = fmaf(dot, scale_log2, rowterm * kLog2e);
+        const float xs = fmaf(dot, scale_log2, rowcb);
         const float m_new = fmaxf(m, xs);
         const float al = ex2(m - m_new), p = ex2(xs - m_new);
         l = l * al + p;
 #pragma unroll
-        for (int c = 0; c < DH; c += 8) {
-          const uint4 va = *reinterpret_cast<const uint4*>(vp + c);
+        for (int c = 0; c < DH / 8; ++c) {
           float vf[8];
-          Elem<__nv_bfloat16>::unpack(va, vf);
+          Elem<__nv_bfloat16>::unpack(vp[c], vf);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) o[c + e] = fmaf(o[c + e], al, p * vf[e]);
+          for (int e = 0; e < 8; ++e) o[c * 8 + e] = fmaf(o[c * 8 + e], al, p * vf[e]);
         }
         m = m_new;
       }
@@ -458,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
         for (int e = 0; e < 8; ++e) f[e] = o[c + e] * inv;
         op[c / 8] = Elem<__nv_bfloat16>::pack(f);
       }
-      if (a.lse) a.lse[(long long)it.h * a.T + tok] = (m + __log2f(l)) * kLn2 - rowterm;
+      if (a.lse) a.lse[(long long)it.h * a.T + tok] = (m + __log2f(l) - rowcb) * kLn2;
     }
   }
 
@@ -501,31 +509,37 @@ static bool make_map(CUtensorMap* m, const void* base, long long T, int H, long 
 
 static int max_tiles_of(int max_seqlen) { return (max_seqlen + BM - 1) / BM; }
 
+static size_t recs_bytes(int B, int max_seqlen) {
+  return ((size_t)B * max_tiles_of(max_seqlen) * kRecInts * 4 + 15) / 16 * 16;
+}
+
 }  // namespace tc
 
 size_t attn_fwd_tc_workspace(int B, long long T, int H, int max_seqlen) {
-  (void)T;
-  (void)H;
-  return 256 + (size_t)B * tc::max_tiles_of(max_seqlen) * sizeof(int32_t);
+  using namespace tc;
+  return kHeaderBytes + recs_bytes(B, max_seqlen) + (size_t)H * scratch_tp(T, B) * sizeof(float);
 }
 
 int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
   using namespace tc;
   if (a.dh != DH || a.dtype != GENRANK_BF16) return GENRANK_ERR_UNSUPPORTED;
   const int max_tiles = max_tiles_of(a.max_seqlen);
-  if (max_tiles >= (1 << kItemTileBits) || a.B >= (1 << (31 - kItemTileBits)))
-    return GENRANK_ERR_UNSUPPORTED;
-  if (a.T > INT32_MAX - 2 * BM) return GENRANK_ERR_UNSUPPORTED;
+  if (a.T + (long long)BM >= INT32_MAX / 2) return GENRANK_ERR_UNSUPPORTED;
   Params p;
   if (!make_map(&p.tq, a.q, a.T, a.H, a.tok_stride) ||
       !make_map(&p.tk, a.k, a.T, a.H, a.tok_stride) ||
       !make_map(&p.tv, a.v, a.T, a.H, a.tok_stride))
     return GENRANK_ERR_CUDA;
   p.a = a;
-  int32_t* ws = (int32_t*)a.ws;
-  p.count = ws;
-  p.items = ws + 64;
-  k_schedule<<<1, 1024, 0, st>>>(a.B, a.T, a.off, a.hist_len, max_tiles, ws + 64, ws, a.err);
+  uint8_t* ws = (uint8_t*)a.ws;
+  int32_t* count = (int32_t*)ws;
+  int4* recs = (int4*)(ws + kHeaderBytes);
+  float* cbias = (float*)(ws + kHeaderBytes + recs_bytes(a.B, a.max_seqlen));
+  p.count = count;
+  p.recs = recs;
+  p.cbias = cbias;
+  p.Tp = scratch_tp(a.T, a.B);
+  k_prologue<<<a.B + 1, 256, 0, st>>>(a, max_tiles, recs, count, cbias, p.Tp);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   static bool attr = false;
   if (!attr) {
@@ -537,7 +551,7 @@ int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  k_attn_fwd_tc<<<sms, kThreads, kSmemBytes, st>>>(p);
+  k_attn_fwd_tc<<<2 * sms, kThreads, kSmemBytes, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
 }
 

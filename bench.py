@@ -287,9 +287,11 @@ def run_native(args, cfg, world, rank, local):
     for k in range(args.steps):
         flush.zero_()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.nvtx.range_push("timed_step")
         s.record()
         gm.forward(dbs[k % 2], attn_events=attn_ev)
         e.record()
+        torch.cuda.nvtx.range_pop()
         ev.append((s, e))
     sync_all()
     clocks = sampler.stop()

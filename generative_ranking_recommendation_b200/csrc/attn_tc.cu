@@ -187,6 +187,112 @@ GR_DEVICE bool wait_warp(uint64_t* bar, uint32_t par, volatile int* abort_flag, 
   return __all_sync(0xffffffffu, ok);
 }
 
+// x = s * scale + c_j for 32 columns starting at key c0 of the tile; columns at or
+// beyond nvalid are masked.  Four independent running maxima shorten the chain.
+template <bool kMasked>
+GR_DEVICE void row_max_chunk(const uint32_t (&s)[32], const float* cb, int c0, int nvalid,
+                             float scale_log2, float (&mx4)[4]) {
+#pragma unroll
+  for (int c = 0; c < 32; c += 4) {
+    const float4 b4 = *reinterpret_cast<const float4*>(cb + c);
+    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float v = fmaf(__uint_as_float(s[c + e]), scale_log2, bb[e]);
+      mx4[e] = fmaxf(mx4[e], (!kMasked || c0 + c + e < nvalid) ? v : -INFINITY);
+    }
+  }
+}
+
+// p = 2^(x - m) for 32 columns, summed into four partial row sums, packed to bf16
+// pairs and stored to 16 TMEM columns at taddr.
+template <bool kMasked>
+GR_DEVICE void exp_pack_store(const uint32_t (&s)[32], const float* cb, int c0, int nvalid,
+                              float scale_log2, float m_use, float (&rs4)[4], uint32_t taddr) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int c = 0; c < 32; c += 4) {
+    const float4 b4 = *reinterpret_cast<const float4*>(cb + c);
+    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float v = fmaf(__uint_as_float(s[c + e]), scale_log2, bb[e] - m_use);
+      p[e] = (!kMasked || c0 + c + e < nvalid) ? ex2(v) : 0.f;
+      rs4[e] += p[e];
+    }
+    pk[c / 2] = pack_bf16(p[0], p[1]);
+    pk[c / 2 + 1] = pack_bf16(p[2], p[3]);
+  }
+  tmem_st16(taddr, pk);
+}
+
+// One key tile of the online softmax for this thread's row (TMEM lane):
+// pass 1 takes the row maximum of x = s * scale + c_j, 32 columns at a time with the
+// next chunk's load in flight; the offset m moves (and O in TMEM is rescaled) only
+// when the maximum grows by more than 2^8; pass 2 writes P = 2^(x - m) as bf16 pairs
+// over S columns already consumed (keys [c0, c0+32) land in columns [c0/2, c0/2+16),
+// which an earlier chunk has read) and adds the row sum into l.
+template <bool kMasked>
+GR_DEVICE void softmax_tile(uint32_t tmem_lane, const float* cb, int nvalid, float scale_log2,
+                            bool first, float& m, float& l) {
+  float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  {
+    uint32_t xa[32], xb[32];
+    tmem_ld32_async(tmem_lane + kColS, xa);
+    tmem_ld_wait(xa);
+#pragma unroll
+    for (int c0 = 0; c0 < BN; c0 += 64) {
+      tmem_ld32_async(tmem_lane + kColS + c0 + 32, xb);
+      row_max_chunk<kMasked>(xa, cb + c0, c0, nvalid, scale_log2, mx4);
+      tmem_ld_wait(xb);
+      if (c0 + 64 < BN) tmem_ld32_async(tmem_lane + kColS + c0 + 64, xa);
+      row_max_chunk<kMasked>(xb, cb + c0 + 32, c0 + 32, nvalid, scale_log2, mx4);
+      if (c0 + 64 < BN) tmem_ld_wait(xa);
+    }
+  }
+  const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+  float alpha = 1.f;
+  if (first) {
+    m = mx;
+  } else {
+    const bool need = mx > m + kRescaleThreshold;
+    if (__any_sync(0xffffffffu, need)) {
+      const float m_new = need ? mx : m;
+      alpha = ex2(m - m_new);
+      m = m_new;
+#pragma unroll 1
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        float o[32];
+        tmem_ld32(tmem_lane + kColO + c0, o);
+        uint32_t ob[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(o[c] * alpha);
+        tmem_st32(tmem_lane + kColO + c0, ob);
+      }
+    }
+  }
+  const float m_use = m == -INFINITY ? 0.f : m;
+  float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+  {
+    uint32_t xa[32], xb[32];
+    tmem_ld32_async(tmem_lane + kColS, xa);
+    tmem_ld_wait(xa);
+#pragma unroll
+    for (int c0 = 0; c0 < BN; c0 += 64) {
+      tmem_ld32_async(tmem_lane + kColS + c0 + 32, xb);
+      exp_pack_store<kMasked>(xa, cb + c0, c0, nvalid, scale_log2, m_use, rs4,
+                              tmem_lane + kColS + c0 / 2);
+      tmem_ld_wait(xb);
+      if (c0 + 64 < BN) tmem_ld32_async(tmem_lane + kColS + c0 + 64, xa);
+      exp_pack_store<kMasked>(xb, cb + c0 + 32, c0 + 32, nvalid, scale_log2, m_use, rs4,
+                              tmem_lane + kColS + (c0 + 32) / 2);
+      if (c0 + 64 < BN) tmem_ld_wait(xa);
+    }
+  }
+  l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+}
+
 __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_constant__ Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -343,72 +449,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
         tc_fence_after();
         const float* cb = sCB + st * BN;
         const bool masked = kv0 + BN - 1 > mask_from;
-        // pass 1: row maximum of the biased scores, 32 columns at a time
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          float x[32];
-          tmem_ld32(tmem + lane_base + kColS + c0, x);
-#pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            const float4 b4 = *reinterpret_cast<const float4*>(cb + c0 + c);
-            const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float v = fmaf(x[c + e], scale_log2, bb[e]);
-              if (masked && kv0 + c0 + c + e > lim) v = -INFINITY;
-              mx = fmaxf(mx, v);
-            }
-          }
-        }
-        // lazy offset: move it (and rescale O in TMEM) only when the max grows by > 2^8
-        float alpha = 1.f;
-        if (j == 0) {
-          m = mx;
-        } else {
-          const bool need = mx > m + kRescaleThreshold;
-          if (__any_sync(0xffffffffu, need)) {
-            const float m_new = need ? mx : m;
-            alpha = ex2(m - m_new);
-            m = m_new;
-#pragma unroll 1
-            for (int c0 = 0; c0 < DH; c0 += 32) {
-              float o[32];
-              tmem_ld32(tmem + lane_base + kColO + c0, o);
-              uint32_t ob[32];
-#pragma unroll
-              for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(o[c] * alpha);
-              tmem_st32(tmem + lane_base + kColO + c0, ob);
-            }
-          }
-        }
-        const float m_use = m == -INFINITY ? 0.f : m;
-        // pass 2: P = 2^(x - m) in bf16, written over S columns already consumed
-        // (chunk c0 of keys lands in columns [c0/2, c0/2 + 16), read by an earlier chunk)
-        float rs = 0.f;
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          float x[32];
-          tmem_ld32(tmem + lane_base + kColS + c0, x);
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            const float4 b4 = *reinterpret_cast<const float4*>(cb + c0 + c);
-            const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
-            float p[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float v = fmaf(x[c + e], scale_log2, bb[e]);
-              if (masked && kv0 + c0 + c + e > lim) v = -INFINITY;
-              p[e] = ex2(v - m_use);
-              rs += p[e];
-            }
-            pk[c / 2] = pack_bf16(p[0], p[1]);
-            pk[c / 2 + 1] = pack_bf16(p[2], p[3]);
-          }
-          tmem_st16(tmem + lane_base + kColS + c0 / 2, pk);
-        }
-        l = l * alpha + rs;
+        const int nvalid = masked ? max(0, min(BN, lim - kv0 + 1)) : BN;
+        if (masked)
+          softmax_tile<true>(tmem + lane_base, cb, nvalid, scale_log2, j == 0, m, l);
+        else
+          softmax_tile<false>(tmem + lane_base, cb, nvalid, scale_log2, j == 0, m, l);
         tc_fence_before();
         mbar_arrive(&bars[kPFull]);
       }

@@ -27,6 +27,7 @@ EXPORTS = (
     "genrank_status_string", "genrank_device_error_string", "genrank_check_error",
     "genrank_alibi_slopes", "genrank_embed_assemble", "genrank_embed_assemble_bwd",
     "genrank_attn_fwd", "genrank_attn_bwd", "genrank_attn_workspace_size",
+    "genrank_attn_fwd_static",
 )
 
 
@@ -71,6 +72,10 @@ def lib():
         L.genrank_attn_bwd.argtypes = [
             _I, _L, _P, _P, _I, _P, _P, _P, _L, _I, _I, _P, _P, _P, _P, _F, _I, _P, _P, _L,
             _P, _P, _P, _P, _P, _Z, _P, _P]
+        L.genrank_attn_fwd_static.restype = _I
+        L.genrank_attn_fwd_static.argtypes = [
+            _I, _L, _P, _P, _I, _P, _P, _P, _L, _I, _I, _P, _P, _P, _P, _F, _I, _P, _L, _P,
+            _P, _P]
         L.genrank_attn_workspace_size.restype = _Z
         L.genrank_attn_workspace_size.argtypes = [_I, _L, _I, _I, _I, _I]
         _lib = L
@@ -191,3 +196,18 @@ def attn_bwd(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos,
         _ptr(dk), _ptr(dv), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
         _ptr(dev_err), _stream(stream))
     _check(rc, "genrank_attn_bwd")
+
+
+def attn_fwd_static(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts,
+                    slope_pos, slope_time, scale, o, o_stride, lse, dev_err, T=None, stream=None):
+    """genrank_attn_fwd_static: the forward without a caller workspace (the library's
+    fixed 16 MiB scratch is used; see include/genrank.h for the rules)."""
+    B = hist_len.numel()
+    T = o.shape[0] if T is None else T
+    sp, st = _host_floats(slope_pos), _host_floats(slope_time)
+    rc = lib().genrank_attn_fwd_static(
+        B, T, _ptr(seq_offsets), _ptr(hist_len), int(max_seqlen), _ptr(q), _ptr(k), _ptr(v),
+        int(tok_stride), H, dh, _ptr(pos), _ptr(ts), ctypes.cast(sp, _P), ctypes.cast(st, _P),
+        float(scale), _dtype_code(q), _ptr(o), int(o_stride), _ptr(lse), _ptr(dev_err),
+        _stream(stream))
+    _check(rc, "genrank_attn_fwd_static")

@@ -185,6 +185,29 @@ int genrank_attn_bwd(int B, int64_t T, const int32_t *seq_offsets, const int32_t
                      void *dv, void *ws, size_t ws_bytes, int32_t *dev_err,
                      genrank_stream_t stream);
 
+/* genrank_attn_fwd for callers that cannot allocate device memory.
+ * The paper has no counterpart of this call; it exists for deployment.  Some
+ * callers cannot call cudaMalloc (or any allocator, torch's included) where they
+ * run attention: serving loops that forbid device allocations after start-up,
+ * or hosts that own all device memory and hand out no scratch.  This call takes
+ * the same arguments as genrank_attn_fwd minus the workspace: its scratch is a
+ * 16 MiB array compiled into the library, which every GPU that loads the library
+ * holds until the process exits.  Inputs and outputs are still the caller's.
+ *   - Sizes whose workspace (genrank_attn_workspace_size(..., 0)) exceeds
+ *     16 MiB are rejected with GENRANK_ERR_WORKSPACE before any launch.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; nothing in it needs to start at zero.  Calls that overlap on the
+ *     GPU (other streams, other host threads) race on it: serialise them.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+int genrank_attn_fwd_static(int B, int64_t T, const int32_t *seq_offsets, const int32_t *hist_len,
+                            int max_seqlen, const void *q, const void *k, const void *v,
+                            int64_t tok_stride, int H, int dh, const int32_t *pos,
+                            const int64_t *ts, const float *slope_pos, const float *slope_time,
+                            float scale, int dtype, void *o, int64_t o_stride, float *lse,
+                            int32_t *dev_err, genrank_stream_t stream);
+
 /* Bytes of workspace genrank_attn_fwd (is_bwd = 0) or genrank_attn_bwd
  * (is_bwd = 1) need for these sizes.  Returns 0 for invalid sizes. */
 size_t genrank_attn_workspace_size(int B, int64_t T, int H, int dh, int max_seqlen, int is_bwd);

@@ -45,7 +45,7 @@ constexpr int DH = 64;   // head dim
 constexpr int kThreads = 192;  // warps 0-3 softmax, warp 4 TMA, warp 5 MMA
 constexpr uint32_t kTileBytes = BM * DH * 2;  // one Q, K or V tile (16 KB)
 constexpr uint32_t kCBBytes = BN * 4;         // column terms of one key tile
-constexpr float kRescaleThreshold = 8.0f;     // log2 units
+constexpr float kOverflowSum = 1.2676506e30f;  // 2^100: a tile's row sum above this is redone
 
 // dynamic shared memory layout (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;                          // 16 KB
@@ -59,8 +59,9 @@ constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
 
 // TMEM columns (per CTA; two CTAs share an SM's 512)
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0;    // S (fp32, 128 columns); P (bf16 pairs) in its first 64
+constexpr uint32_t kColS = 0;    // S (fp32, 128 columns)
 constexpr uint32_t kColO = 128;  // O (fp32, 64 columns)
+constexpr uint32_t kColP = 192;  // P (bf16 pairs, 64 columns)
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);   // Q K-major, K K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, DH, 0, 1);  // P K-major (TMEM), V MN-major
@@ -227,70 +228,88 @@ GR_DEVICE void exp_pack_store(const uint32_t (&s)[32], const float* cb, int c0, 
   tmem_st16(taddr, pk);
 }
 
-// One key tile of the online softmax for this thread's row (TMEM lane):
-// pass 1 takes the row maximum of x = s * scale + c_j, 32 columns at a time with the
-// next chunk's load in flight; the offset m moves (and O in TMEM is rescaled) only
-// when the maximum grows by more than 2^8; pass 2 writes P = 2^(x - m) as bf16 pairs
-// over S columns already consumed (keys [c0, c0+32) land in columns [c0/2, c0/2+16),
-// which an earlier chunk has read) and adds the row sum into l.
+// Row maximum of x = s * scale + c_j over the tile, 32 columns at a time with the
+// next chunk's TMEM load in flight.
 template <bool kMasked>
-GR_DEVICE void softmax_tile(uint32_t tmem_lane, const float* cb, int nvalid, float scale_log2,
-                            bool first, float& m, float& l) {
+GR_DEVICE float tile_max(uint32_t tmem_lane, const float* cb, int nvalid, float scale_log2) {
   float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-  {
-    uint32_t xa[32], xb[32];
-    tmem_ld32_async(tmem_lane + kColS, xa);
-    tmem_ld_wait(xa);
+  uint32_t xa[32], xb[32];
+  tmem_ld32_async(tmem_lane + kColS, xa);
+  tmem_ld_wait(xa);
 #pragma unroll
-    for (int c0 = 0; c0 < BN; c0 += 64) {
-      tmem_ld32_async(tmem_lane + kColS + c0 + 32, xb);
-      row_max_chunk<kMasked>(xa, cb + c0, c0, nvalid, scale_log2, mx4);
-      tmem_ld_wait(xb);
-      if (c0 + 64 < BN) tmem_ld32_async(tmem_lane + kColS + c0 + 64, xa);
-      row_max_chunk<kMasked>(xb, cb + c0 + 32, c0 + 32, nvalid, scale_log2, mx4);
-      if (c0 + 64 < BN) tmem_ld_wait(xa);
-    }
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    tmem_ld32_async(tmem_lane + kColS + c0 + 32, xb);
+    row_max_chunk<kMasked>(xa, cb + c0, c0, nvalid, scale_log2, mx4);
+    tmem_ld_wait(xb);
+    if (c0 + 64 < BN) tmem_ld32_async(tmem_lane + kColS + c0 + 64, xa);
+    row_max_chunk<kMasked>(xb, cb + c0 + 32, c0 + 32, nvalid, scale_log2, mx4);
+    if (c0 + 64 < BN) tmem_ld_wait(xa);
   }
-  const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-  float alpha = 1.f;
-  if (first) {
-    m = mx;
-  } else {
-    const bool need = mx > m + kRescaleThreshold;
-    if (__any_sync(0xffffffffu, need)) {
-      const float m_new = need ? mx : m;
-      alpha = ex2(m - m_new);
-      m = m_new;
-#pragma unroll 1
-      for (int c0 = 0; c0 < DH; c0 += 32) {
-        float o[32];
-        tmem_ld32(tmem_lane + kColO + c0, o);
-        uint32_t ob[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(o[c] * alpha);
-        tmem_st32(tmem_lane + kColO + c0, ob);
-      }
-    }
-  }
-  const float m_use = m == -INFINITY ? 0.f : m;
+  return fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+}
+
+// P = 2^(x - m) for the tile, written as bf16 pairs to the P columns, 32 keys at a
+// time with the next chunk's TMEM load in flight.  Returns the row sum.
+template <bool kMasked>
+GR_DEVICE float tile_exp(uint32_t tmem_lane, const float* cb, int nvalid, float scale_log2,
+                         float m) {
   float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-  {
-    uint32_t xa[32], xb[32];
-    tmem_ld32_async(tmem_lane + kColS, xa);
-    tmem_ld_wait(xa);
+  uint32_t xa[32], xb[32];
+  tmem_ld32_async(tmem_lane + kColS, xa);
+  tmem_ld_wait(xa);
 #pragma unroll
-    for (int c0 = 0; c0 < BN; c0 += 64) {
-      tmem_ld32_async(tmem_lane + kColS + c0 + 32, xb);
-      exp_pack_store<kMasked>(xa, cb + c0, c0, nvalid, scale_log2, m_use, rs4,
-                              tmem_lane + kColS + c0 / 2);
-      tmem_ld_wait(xb);
-      if (c0 + 64 < BN) tmem_ld32_async(tmem_lane + kColS + c0 + 64, xa);
-      exp_pack_store<kMasked>(xb, cb + c0 + 32, c0 + 32, nvalid, scale_log2, m_use, rs4,
-                              tmem_lane + kColS + (c0 + 32) / 2);
-      if (c0 + 64 < BN) tmem_ld_wait(xa);
-    }
+  for (int c0 = 0; c0 < BN; c0 += 64) {
+    tmem_ld32_async(tmem_lane + kColS + c0 + 32, xb);
+    exp_pack_store<kMasked>(xa, cb + c0, c0, nvalid, scale_log2, m, rs4,
+                            tmem_lane + kColP + c0 / 2);
+    tmem_ld_wait(xb);
+    if (c0 + 64 < BN) tmem_ld32_async(tmem_lane + kColS + c0 + 64, xa);
+    exp_pack_store<kMasked>(xb, cb + c0 + 32, c0 + 32, nvalid, scale_log2, m, rs4,
+                            tmem_lane + kColP + (c0 + 32) / 2);
+    if (c0 + 64 < BN) tmem_ld_wait(xa);
   }
-  l = l * alpha + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+  return (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+}
+
+// One key tile of the online softmax for this thread's row (TMEM lane).  Key tiles
+// are visited most recent first; with ALiBi the most recent keys carry the largest
+// bias, so the first tile's maximum is, in practice, the row's maximum.  The first
+// tile fixes the offset m exactly (two passes); later tiles use it in one pass and
+// redo the tile exactly (rescaling O in TMEM) only if the row sum overflows.
+// Before P is written, the previous P V must have finished (it reads P and adds to O).
+template <bool kMasked>
+GR_DEVICE bool softmax_tile(uint32_t tmem_lane, const float* cb, int nvalid, float scale_log2,
+                            bool first, float& m, float& l, uint64_t* pv_bar, int g,
+                            volatile int* abort_flag, int32_t* err) {
+  if (first) m = tile_max<kMasked>(tmem_lane, cb, nvalid, scale_log2);
+  if (g > 0 && !wait_warp(pv_bar, parity(g - 1), abort_flag, err)) return false;
+  tc_fence_after();
+  float rs = tile_exp<kMasked>(tmem_lane, cb, nvalid, scale_log2, m);
+  if (first) {
+    l = rs;
+    return true;
+  }
+  const bool redo = !(rs <= kOverflowSum);
+  if (__any_sync(0xffffffffu, redo)) {
+    // every lane takes part in the .sync.aligned TMEM loads; only redo lanes move m
+    const float mx = tile_max<kMasked>(tmem_lane, cb, nvalid, scale_log2);
+    const float m_new = redo ? fmaxf(m, mx) : m;
+    const float alpha = ex2(m - m_new);
+    m = m_new;
+#pragma unroll 1
+    for (int c0 = 0; c0 < DH; c0 += 32) {
+      float o[32];
+      tmem_ld32(tmem_lane + kColO + c0, o);
+      uint32_t ob[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(o[c] * alpha);
+      tmem_st32(tmem_lane + kColO + c0, ob);
+    }
+    l *= alpha;
+    rs = tile_exp<kMasked>(tmem_lane, cb, nvalid, scale_log2, m);
+  }
+  l += rs;
+  return true;
 }
 
 __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_constant__ Params P) {
@@ -354,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
           break;
         }
         if (lane == 0) {
-          const int kv0 = j * BN;
+          const int kv0 = (it.nk - 1 - j) * BN;  // most recent keys first
           mbar_expect_tx(&bars[kKFull + st], kTileBytes + kCBBytes);
           tma_load_3d(smem + kOffK + st * kTileBytes, &P.tk, &bars[kKFull + st], 0, it.h,
                       it.s + kv0);
@@ -369,46 +388,70 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
     }
   } else if (warp == 5 && lane == 0) {
     // ---------------------------------------------------------------- MMA issuer (one thread)
-    int qi = 0, g = 0;
+    // Per tile g: S_g = Q K_g^T is issued as soon as the softmax has released S_{g-1}
+    // (P lives in its own columns), so it overlaps P_{g-1} V_{g-1}.
     const uint32_t sQ = smem_u32(smem + kOffQ), sK = smem_u32(smem + kOffK),
                    sV = smem_u32(smem + kOffV);
-    bool ok = true;
-    for (int w = blockIdx.x; w < total && ok && !*abort_flag; w += gridDim.x) {
-      const Item it = load_item(P, w);
-      if (it.nk == 0) continue;
-      if (!mbar_wait(&bars[kQFull], parity(qi), abort_flag, a.err)) break;
-      for (int j = 0; j < it.nk; ++j, ++g) {
-        const int st = g & 1;
-        // K landed, and the previous P V finished (S overwrites that P)
-        if (!mbar_wait(&bars[kKFull + st], parity(g >> 1), abort_flag, a.err) ||
-            (g > 0 && !mbar_wait(&bars[kPVFull], parity(g - 1), abort_flag, a.err))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < DH / 16; ++k) {
-          const uint64_t ad = smem_desc_sw128(sQ + k * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sK + st * kTileBytes + k * 32, 16, 1024);
-          mma_bf16_ss(tmem + kColS, ad, bd, kIdescS, k > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars[kSFull]);
-        if (j == it.nk - 1) mma_commit(&bars[kQEmpty]);
-        if (!mbar_wait(&bars[kPFull], parity(g), abort_flag, a.err) ||
-            !mbar_wait(&bars[kVFull + st], parity(g >> 1), abort_flag, a.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < BN / 16; ++k) {
-          const uint64_t bd = smem_desc_sw128(sV + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
-          mma_bf16_ts(tmem + kColO, tmem + kColS + k * 8, bd, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
-        }
-        mma_commit(&bars[kPVFull]);
-        mma_commit(&bars[kKVEmpty + st]);
+    auto next_item = [&](int from, Item& out) -> int {
+      for (int x = from; x < total; x += gridDim.x) {
+        out = load_item(P, x);
+        if (out.nk > 0) return x;
       }
-      ++qi;
+      return -1;
+    };
+    auto issue_s = [&](int gg) {
+      const int st = gg & 1;
+#pragma unroll
+      for (int k = 0; k < DH / 16; ++k) {
+        const uint64_t ad = smem_desc_sw128(sQ + k * 32, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(sK + st * kTileBytes + k * 32, 16, 1024);
+        mma_bf16_ss(tmem + kColS, ad, bd, kIdescS, k > 0 ? 1u : 0u);
+      }
+      mma_commit(&bars[kSFull]);
+    };
+    Item it;
+    int w = next_item(blockIdx.x, it);
+    int qi = 0, g = 0, j = 0;
+    bool ok = w >= 0 && mbar_wait(&bars[kQFull], parity(0), abort_flag, a.err) &&
+              mbar_wait(&bars[kKFull], parity(0), abort_flag, a.err);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0);
+      if (it.nk == 1) mma_commit(&bars[kQEmpty]);
+    }
+    while (ok && !*abort_flag) {
+      if (!mbar_wait(&bars[kPFull], parity(g), abort_flag, a.err)) break;
+      // look ahead: the next tile of this item, or the first tile of the next item
+      Item it2 = it;
+      int w2 = w, j2 = j + 1;
+      if (j2 == it.nk) {
+        w2 = next_item(w + gridDim.x, it2);
+        j2 = 0;
+      }
+      if (w2 >= 0) {
+        if (j2 == 0 && !mbar_wait(&bars[kQFull], parity(qi + 1), abort_flag, a.err)) break;
+        if (!mbar_wait(&bars[kKFull + ((g + 1) & 1)], parity((g + 1) >> 1), abort_flag, a.err))
+          break;
+        tc_fence_after();
+        issue_s(g + 1);
+        if (j2 == it2.nk - 1) mma_commit(&bars[kQEmpty]);
+      }
+      const int st = g & 1;
+      if (!mbar_wait(&bars[kVFull + st], parity(g >> 1), abort_flag, a.err)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < BN / 16; ++k) {
+        const uint64_t bd = smem_desc_sw128(sV + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
+        mma_bf16_ts(tmem + kColO, tmem + kColP + k * 8, bd, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+      }
+      mma_commit(&bars[kPVFull]);
+      mma_commit(&bars[kKVEmpty + st]);
+      ++g;
+      if (w2 < 0) break;
+      if (j2 == 0) ++qi;
+      w = w2;
+      j = j2;
+      it = it2;
     }
   } else if (warp < 4) {
     // ---------------------------------------------------------------- softmax warps 0-3
@@ -440,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
       bool ok = true;
       for (int j = 0; j < it.nk; ++j, ++g) {
         const int st = g & 1;
-        const int kv0 = j * BN;
+        const int kv0 = (it.nk - 1 - j) * BN;  // most recent keys first
         if (!wait_warp(&bars[kSFull], parity(g), abort_flag, a.err) ||
             !wait_warp(&bars[kKFull + st], parity(g >> 1), abort_flag, a.err)) {
           ok = false;
@@ -450,10 +493,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
         const float* cb = sCB + st * BN;
         const bool masked = kv0 + BN - 1 > mask_from;
         const int nvalid = masked ? max(0, min(BN, lim - kv0 + 1)) : BN;
-        if (masked)
-          softmax_tile<true>(tmem + lane_base, cb, nvalid, scale_log2, j == 0, m, l);
-        else
-          softmax_tile<false>(tmem + lane_base, cb, nvalid, scale_log2, j == 0, m, l);
+        ok = masked ? softmax_tile<true>(tmem + lane_base, cb, nvalid, scale_log2, j == 0, m, l,
+                                         &bars[kPVFull], g, abort_flag, a.err)
+                    : softmax_tile<false>(tmem + lane_base, cb, nvalid, scale_log2, j == 0, m, l,
+                                          &bars[kPVFull], g, abort_flag, a.err);
+        if (!ok) break;
         tc_fence_before();
         mbar_arrive(&bars[kPFull]);
       }

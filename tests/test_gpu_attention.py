@@ -256,3 +256,20 @@ def test_bwd_full_size_c3_sampled(G):
     got = run_bwd(G, cfg, batch, pos, qkv, dO)
     want = ref.attn_bwd(qkv[:, 0], qkv[:, 1], qkv[:, 2], dO, batch, pos, users=users)
     _check_grads(cfg, got, want, rows)
+
+
+def test_fwd_older_keys_dominating_take_the_exact_path(G):
+    """Keys are visited most recent first; when much older keys score far higher
+    (beyond 2^100 in a row sum), the tile is recomputed with an exact offset."""
+    cfg = CONFIGS["c1"].with_(B=3)
+    batch = make_batch(cfg, hist_override=[400, 300, 130], m_override=[20, 7, 140])
+    pos, _, _ = ref.meta(batch)
+    qkv = make_qkv(cfg, batch.T, seed=31, std=0.5)
+    for u in range(batch.B):
+        s = batch.seq_offsets[u]
+        qkv[s:s + 100, 1] = 3.0  # oldest keys: large positive scores against ...
+        qkv[s + 100:batch.seq_offsets[u + 1], 0] = 3.0  # ... queries pointing the same way
+    O, L = run_fwd(G, cfg, batch, pos, qkv)
+    Or, Lr = ref.attn(qkv[:, 0], qkv[:, 1], qkv[:, 2], batch, pos)
+    assert np.all(np.isfinite(O)) and np.all(np.isfinite(L))
+    _check(cfg, O, L, Or, Lr, np.arange(batch.T))

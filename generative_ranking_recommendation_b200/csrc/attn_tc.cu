@@ -45,7 +45,8 @@ constexpr int DH = 64;   // head dim
 constexpr int kThreads = 192;  // warps 0-3 softmax, warp 4 TMA, warp 5 MMA
 constexpr uint32_t kTileBytes = BM * DH * 2;  // one Q, K or V tile (16 KB)
 constexpr uint32_t kCBBytes = BN * 4;         // column terms of one key tile
-constexpr float kOverflowSum = 1.2676506e30f;  // 2^100: a tile's row sum above this is redone
+constexpr float kOverflowSum = 1.2676506e30f;   // 2^100: a tile's row sum above this is redone
+constexpr float kUnderflowSum = 7.8886091e-31f;  // 2^-100: a first tile's row sum below this too
 
 // dynamic shared memory layout (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;                          // 16 KB
@@ -271,44 +272,42 @@ GR_DEVICE float tile_exp(uint32_t tmem_lane, const float* cb, int nvalid, float 
   return (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
 }
 
-// One key tile of the online softmax for this thread's row (TMEM lane).  Key tiles
-// are visited most recent first; with ALiBi the most recent keys carry the largest
-// bias, so the first tile's maximum is, in practice, the row's maximum.  The first
-// tile fixes the offset m exactly (two passes); later tiles use it in one pass and
-// redo the tile exactly (rescaling O in TMEM) only if the row sum overflows.
-// Before P is written, the previous P V must have finished (it reads P and adds to O).
+// One key tile of the online softmax for this thread's row (TMEM lane).  The offset
+// m starts at the row's own column term c_i: every visible key has c_j <= c_i, so
+// 2^(x - m) <= 2^(scale q.k log2 e), which overflows only for extreme scores.  Each
+// tile is one pass; a tile whose row sum leaves [2^-100, 2^100] on the first tile
+// (every key far below the offset) or exceeds 2^100 later is redone with the exact
+// offset max(m, tile max), rescaling O in TMEM.  Before P is written, the previous
+// P V must have finished (it reads P and adds to O).
 template <bool kMasked>
 GR_DEVICE bool softmax_tile(uint32_t tmem_lane, const float* cb, int nvalid, float scale_log2,
                             bool first, float& m, float& l, uint64_t* pv_bar, int g,
                             volatile int* abort_flag, int32_t* err) {
-  if (first) m = tile_max<kMasked>(tmem_lane, cb, nvalid, scale_log2);
   if (g > 0 && !wait_warp(pv_bar, parity(g - 1), abort_flag, err)) return false;
   tc_fence_after();
   float rs = tile_exp<kMasked>(tmem_lane, cb, nvalid, scale_log2, m);
-  if (first) {
-    l = rs;
-    return true;
-  }
-  const bool redo = !(rs <= kOverflowSum);
+  const bool redo = !(rs <= kOverflowSum) || (first && rs < kUnderflowSum);
   if (__any_sync(0xffffffffu, redo)) {
     // every lane takes part in the .sync.aligned TMEM loads; only redo lanes move m
     const float mx = tile_max<kMasked>(tmem_lane, cb, nvalid, scale_log2);
-    const float m_new = redo ? fmaxf(m, mx) : m;
-    const float alpha = ex2(m - m_new);
+    const float m_new = redo ? (first ? mx : fmaxf(m, mx)) : m;
+    const float alpha = first ? 1.f : ex2(m - m_new);
     m = m_new;
+    if (!first) {
 #pragma unroll 1
-    for (int c0 = 0; c0 < DH; c0 += 32) {
-      float o[32];
-      tmem_ld32(tmem_lane + kColO + c0, o);
-      uint32_t ob[32];
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        float o[32];
+        tmem_ld32(tmem_lane + kColO + c0, o);
+        uint32_t ob[32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(o[c] * alpha);
-      tmem_st32(tmem_lane + kColO + c0, ob);
+        for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(o[c] * alpha);
+        tmem_st32(tmem_lane + kColO + c0, ob);
+      }
     }
     l *= alpha;
     rs = tile_exp<kMasked>(tmem_lane, cb, nvalid, scale_log2, m);
   }
-  l += rs;
+  l = first ? rs : l + rs;
   return true;
 }
 
@@ -411,6 +410,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
     };
     Item it;
     int w = next_item(blockIdx.x, it);
+    // the record after the current item, loaded one item ahead of its use
+    Item pre = (w >= 0 && w + (int)gridDim.x < total) ? load_item(P, w + gridDim.x) : Item{};
     int qi = 0, g = 0, j = 0;
     bool ok = w >= 0 && mbar_wait(&bars[kQFull], parity(0), abort_flag, a.err) &&
               mbar_wait(&bars[kKFull], parity(0), abort_flag, a.err);
@@ -425,8 +426,16 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
       Item it2 = it;
       int w2 = w, j2 = j + 1;
       if (j2 == it.nk) {
-        w2 = next_item(w + gridDim.x, it2);
         j2 = 0;
+        w2 = w + gridDim.x;
+        if (w2 >= total) {
+          w2 = -1;
+        } else if (pre.nk > 0) {
+          it2 = pre;
+        } else {
+          w2 = next_item(w2 + gridDim.x, it2);  // rare: items without keys to visit
+        }
+        if (w2 >= 0 && w2 + (int)gridDim.x < total) pre = load_item(P, w2 + gridDim.x);
       }
       if (w2 >= 0) {
         if (j2 == 0 && !mbar_wait(&bars[kQFull], parity(qi + 1), abort_flag, a.err)) break;
@@ -462,24 +471,47 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
     const __nv_bfloat16* Kg = (const __nv_bfloat16*)a.k;
     const __nv_bfloat16* Vg = (const __nv_bfloat16*)a.v;
     int g = 0;
+    // the next work item's record is loaded one item ahead, and its candidate rows are
+    // warmed in L2, so that an item starts without a dependent global-load chain
+    Item nx = blockIdx.x < total ? load_item(P, blockIdx.x) : Item{};
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
       __syncwarp();
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      const Item it = load_item(P, w);
+      const Item it = nx;
+      if (w + (int)gridDim.x < total) nx = load_item(P, w + gridDim.x);
       const int i = it.q0 + r;
       const bool row = i < it.L;
       const long long tok = (long long)it.s + i;
       const bool cand = row && i >= it.n;
-      float rowcb = 0.f;
-      if (row) rowcb = P.cbias[(long long)it.h * P.Tp + it.spad + i];
-      if (cand) {  // warm L2 for the epilogue's self-term rows
-        prefetch_l2(Qg + tok * a.tok_stride + it.h * DH);
-        prefetch_l2(Kg + tok * a.tok_stride + it.h * DH);
-        prefetch_l2(Vg + tok * a.tok_stride + it.h * DH);
+      const float rowcb = row ? P.cbias[(long long)it.h * P.Tp + it.spad + i] : 0.f;
+      // candidate self-term: its score now, its value row kept packed until the epilogue
+      float xs = -INFINITY;
+      uint4 va[DH / 8];
+      if (cand) {
+        const uint4* qp = reinterpret_cast<const uint4*>(Qg + tok * a.tok_stride + it.h * DH);
+        const uint4* kp = reinterpret_cast<const uint4*>(Kg + tok * a.tok_stride + it.h * DH);
+        const uint4* vp = reinterpret_cast<const uint4*>(Vg + tok * a.tok_stride + it.h * DH);
+        uint4 qa[DH / 8], ka[DH / 8];
+#pragma unroll
+        for (int c = 0; c < DH / 8; ++c) {
+          qa[c] = qp[c];
+          ka[c] = kp[c];
+          va[c] = vp[c];
+        }
+        float dot = 0.f;
+#pragma unroll
+        for (int c = 0; c < DH / 8; ++c) {
+          float qf[8], kf[8];
+          Elem<__nv_bfloat16>::unpack(qa[c], qf);
+          Elem<__nv_bfloat16>::unpack(ka[c], kf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
+        }
+        xs = fmaf(dot, scale_log2, rowcb);
       }
       const int lim = min(i, it.n - 1);
       const int mask_from = min(it.q0, it.n - 1);  // a tile needs masks if kv0 + 127 > this
-      float m = -INFINITY, l = 0.f;
+      float m = rowcb, l = 0.f;
       bool ok = true;
       for (int j = 0; j < it.nk; ++j, ++g) {
         const int st = g & 1;
@@ -502,6 +534,15 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
         mbar_arrive(&bars[kPFull]);
       }
       if (!ok) break;
+      {  // warm L2 for the next item's candidate rows while this item's P V finishes
+        const int ni = nx.q0 + r;
+        if (w + (int)gridDim.x < total && ni < nx.L && ni >= nx.n) {
+          const long long nt = (long long)nx.s + ni;
+          prefetch_l2(Qg + nt * a.tok_stride + nx.h * DH);
+          prefetch_l2(Kg + nt * a.tok_stride + nx.h * DH);
+          prefetch_l2(Vg + nt * a.tok_stride + nx.h * DH);
+        }
+      }
       float o[DH];
       if (it.nk > 0) {
         if (!wait_warp(&bars[kPVFull], parity(g - 1), abort_flag, a.err)) break;
@@ -511,36 +552,17 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
       } else {
 #pragma unroll
         for (int c = 0; c < DH; ++c) o[c] = 0.f;
+        m = xs;  // nothing visible but the candidate itself
       }
       if (!row) continue;
       if (cand) {
-        // the candidate's own key: literal bias 0, i.e. column term == row term
-        const uint4* qp = reinterpret_cast<const uint4*>(Qg + tok * a.tok_stride + it.h * DH);
-        const uint4* kp = reinterpret_cast<const uint4*>(Kg + tok * a.tok_stride + it.h * DH);
-        const uint4* vp = reinterpret_cast<const uint4*>(Vg + tok * a.tok_stride + it.h * DH);
-        uint4 qa[DH / 8], ka[DH / 8];
-#pragma unroll
-        for (int c = 0; c < DH / 8; ++c) {
-          qa[c] = qp[c];
-          ka[c] = kp[c];
-        }
-        float dot = 0.f;
-#pragma unroll
-        for (int c = 0; c < DH / 8; ++c) {
-          float qf[8], kf[8];
-          Elem<__nv_bfloat16>::unpack(qa[c], qf);
-          Elem<__nv_bfloat16>::unpack(ka[c], kf);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
-        }
-        const float xs = fmaf(dot, scale_log2, rowcb);
         const float m_new = fmaxf(m, xs);
         const float al = ex2(m - m_new), p = ex2(xs - m_new);
         l = l * al + p;
 #pragma unroll
         for (int c = 0; c < DH / 8; ++c) {
           float vf[8];
-          Elem<__nv_bfloat16>::unpack(vp[c], vf);
+          Elem<__nv_bfloat16>::unpack(va[c], vf);
 #pragma unroll
           for (int e = 0; e < 8; ++e) o[c * 8 + e] = fmaf(o[c * 8 + e], al, p * vf[e]);
         }
@@ -645,3 +667,4 @@ int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
 }
 
 }  // namespace gr
+

@@ -165,7 +165,12 @@ int genrank_embed_assemble_bwd(int B, int64_t T, const int32_t* seq_offsets,
 
 size_t genrank_attn_workspace_size(int B, int64_t T, int H, int dh, int max_seqlen, int is_bwd) {
   if (B < 1 || T < 0 || H < 1 || dh < 1 || max_seqlen < 0) return 0;
-  if (is_bwd) return attn_bwd_simt_workspace(B, T, H, dh, max_seqlen);
+  if (is_bwd) {
+    const size_t simt = attn_bwd_simt_workspace(B, T, H, dh, max_seqlen);
+    if (dh != 64) return simt;
+    const size_t tc = attn_bwd_tc_workspace(B, T, H, max_seqlen);
+    return tc > simt ? tc : simt;
+  }
   return attn_fwd_tc_workspace(B, T, H, max_seqlen);
 }
 
@@ -205,7 +210,8 @@ int genrank_attn_bwd(int B, int64_t T, const int32_t* seq_offsets, const int32_t
                              pos, ts, slope_pos, slope_time, scale, dtype, o_stride, dev_err);
   if (rc) return rc;
   if (T > 0 && (!o || !dO || !lse || !dq || !dk || !dv)) return GENRANK_ERR_INVALID_ARG;
-  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return GENRANK_ERR_INVALID_ARG;
+  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(o) || !aligned16(dO))
+    return GENRANK_ERR_INVALID_ARG;
   if (dh != 32 && dh != 64) return GENRANK_ERR_UNSUPPORTED;
   const size_t need = genrank_attn_workspace_size(B, T, H, dh, max_seqlen, 1);
   if (!ws || ws_bytes < need || !aligned16(ws)) return GENRANK_ERR_WORKSPACE;
@@ -221,7 +227,8 @@ int genrank_attn_bwd(int B, int64_t T, const int32_t* seq_offsets, const int32_t
   a.dv = dv;
   a.ws = ws;
   a.ws_bytes = ws_bytes;
-  return launch_attn_bwd_simt(a, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return use_tc(dtype, dh) ? launch_attn_bwd_tc(a, s) : launch_attn_bwd_simt(a, s);
 }
 
 }  // extern "C"

@@ -1,0 +1,669 @@
+// Backward of the jagged masked ALiBi attention on 5th-generation tensor cores.
+//
+// Gradients of O = softmax(S) V with s_ij = scale q_i.k_j - m|p_i - p_j| - m_t|t_i - t_j|
+// ("GenRank [2025]" chapter notes §1.4.2 ALiBi score; §1.4.1 candidate mask): the
+// biases have no parameters, so only dQ, dK, dV exist:
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  D_i = rowsum(dO_i * O_i),
+//   dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Decomposition (bf16 inputs, head dim 64, fp32 accumulation):
+//   * A prologue lists (user, 128-key history tile) work records, longest first,
+//     and writes per token and head the ALiBi column term c_j (log2 units), the
+//     log2-domain LSE in column-term form lse2_i = LSE_i log2 e + c_i, and D_i, so
+//     that p_ij = 2^(scale log2e q_i.k_j + c_j - lse2_i) on every visible pair.
+//   * One CTA per SM walks the records.  For a history key tile [k0, k0+128) the
+//     visible queries are the user's rows i >= j (later history rows and every
+//     candidate); they are visited one 128-row query tile at a time.
+//   * Warp 4 loads K, V once per record and Q, dO, lse2, D per query tile (TMA,
+//     128B swizzle, no multicast; bulk copies for the per-row terms).
+//   * Warp 5 (one thread) issues tcgen05.mma: S^T = K Q^T and dP^T = V dO^T into
+//     TMEM; after the softmax warps have written P^T and dS^T (bf16, shared memory,
+//     UMMA 128B-swizzled K-major layout), dV += P^T dO and dK += dS^T Q accumulate in
+//     TMEM, and dQ_part = dS K is formed from the same dS^T buffer read as an
+//     MN-major operand.  The next tile's S^T, dP^T are issued before this tile's
+//     gradient MMAs.
+//   * Warps 0-3 (one key row per thread) compute P^T and dS^T and, per record, move
+//     dK (times scale) and dV from TMEM to global memory.
+//   * Warps 6-9 (one query row per thread) add each dQ_part into an fp32 dQ
+//     accumulator in global memory with vector reductions.
+//   * Candidate keys are seen only by their own row; a finishing kernel applies that
+//     self term to dq, dk, dv of candidate tokens and writes dq = scale * dQ_acc.
+// Every mbarrier wait is bounded in time; a timeout sets GENRANK_DERR_TIMEOUT,
+// every role drains out of its loop and the CTA frees its tensor memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gr {
+namespace tcb {
+
+constexpr int BM = 128;  // keys per record tile / queries per query tile
+constexpr int DH = 64;
+constexpr int kThreads = 320;  // warps 0-3 softmax, 4 TMA, 5 MMA, 6-9 dQ reduction
+constexpr uint32_t kTileBytes = BM * DH * 2;  // 16 KB
+constexpr uint32_t kRowBytes = BM * 4;        // one per-row fp32 vector of a tile
+constexpr uint32_t kPSBytes = BM * BM * 2;    // 32 KB (P^T or dS^T)
+
+// shared memory (offsets from a 1024-byte aligned base)
+constexpr uint32_t kOffK = 0;
+constexpr uint32_t kOffV = kOffK + kTileBytes;
+constexpr uint32_t kOffQ = kOffV + kTileBytes;         // 2 stages
+constexpr uint32_t kOffDO = kOffQ + 2 * kTileBytes;    // 2 stages
+constexpr uint32_t kOffL2 = kOffDO + 2 * kTileBytes;   // lse2, 2 stages
+constexpr uint32_t kOffD = kOffL2 + 2 * kRowBytes;     // D, 2 stages
+constexpr uint32_t kOffP = kOffD + 2 * kRowBytes;      // P^T
+constexpr uint32_t kOffDS = kOffP + kPSBytes;          // dS^T
+constexpr uint32_t kOffBar = kOffDS + kPSBytes;
+constexpr uint32_t kNumBars = 16;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
+
+// tensor memory
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;     // S^T  (keys x queries, fp32)
+constexpr uint32_t kColDP = 128;  // dP^T
+constexpr uint32_t kColDV = 256;  // dV   (keys x dh)
+constexpr uint32_t kColDK = 320;  // dK
+constexpr uint32_t kColDQ = 384;  // dQ_part, two buffers of 64 (queries x dh)
+
+constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BM, 0, 0);   // K / V K-major, Q / dO K-major
+constexpr uint32_t kIdescKV = idesc_bf16_f32(BM, DH, 0, 1);  // P^T, dS^T K-major; dO, Q MN-major
+constexpr uint32_t kIdescQ = idesc_bf16_f32(BM, DH, 1, 1);   // dS MN-major; K MN-major
+
+constexpr size_t kHeaderBytes = 256;
+
+enum Bar { kKVFull = 0, kKVEmpty = 1, kQDFull = 2, kQDEmpty = 4, kSFull = 6, kPFull = 7,
+           kPSFree = 8, kDQFull = 9, kDQEmpty = 11 };
+
+struct Params {
+  CUtensorMap tq, tk, tv, tdo;
+  AttnArgs a;
+  const int4* recs;
+  const int32_t* count;
+  const float* cbias;  // [H][Tp]
+  const float* lse2;   // [H][Tp]
+  const float* dsum;   // [H][Tp]  (D)
+  float* dqacc;        // [T][H][64]
+  long long Tp;
+};
+
+struct Rec {
+  int s, L, n, k0, nq, spad, h;
+};
+
+GR_DEVICE Rec load_rec(const Params& P, int w) {
+  const int pair = w / P.a.H;
+  const int4 r0 = P.recs[2 * pair];
+  const int4 r1 = P.recs[2 * pair + 1];
+  Rec r;
+  r.h = w - pair * P.a.H;
+  r.s = r0.x;
+  r.L = r0.y;
+  r.n = r0.z;
+  r.k0 = r0.w;
+  r.nq = r1.x;
+  r.spad = r1.y;
+  return r;
+}
+
+__host__ __device__ inline long long seg_start(long long s, int u) {
+  return 4 * ((s + 3) / 4) + 4LL * u;
+}
+__host__ __device__ inline long long scratch_tp(long long T, int B) {
+  return ((T + 4LL * B + 4 + BM) + 3) / 4 * 4;
+}
+
+// ------------------------------------------------------------------------------------------
+// prologue: records (block B) and per-row terms (blocks 0..B-1)
+// ------------------------------------------------------------------------------------------
+constexpr int kMaxBuckets = 257;
+
+__global__ void __launch_bounds__(256) k_bwd_prologue(const __grid_constant__ AttnArgs a,
+                                                      int max_tiles, int4* recs, int32_t* count,
+                                                      float* cbias, float* lse2, float* dsum,
+                                                      long long Tp) {
+  const int b = blockIdx.x;
+  if (b < a.B) {
+    const long long s = a.off[b], e = a.off[b + 1];
+    if (s < 0 || e < s || e > a.T) return;
+    const int L = (int)(e - s);
+    const long long base = seg_start(s, b);
+    const long long t0 = L > 0 ? a.ts[s] : 0;
+    const __nv_bfloat16* O = (const __nv_bfloat16*)a.o;
+    const __nv_bfloat16* G = (const __nv_bfloat16*)a.dO;
+    // one warp per (token, head): D is a 64-long dot, two elements per lane
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int x = wid; x < L * a.H; x += nw) {
+      const int i = x / a.H, h = x - (x / a.H) * a.H;
+      const long long tok = s + i;
+      const uint32_t ow = *reinterpret_cast<const uint32_t*>(O + tok * a.o_stride + h * DH + 2 * lane);
+      const uint32_t gw = *reinterpret_cast<const uint32_t*>(G + tok * a.o_stride + h * DH + 2 * lane);
+      float dd = bf16_lo(ow) * bf16_lo(gw) + bf16_hi(ow) * bf16_hi(gw);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
+      if (lane == 0) {
+        const float c = kLog2e * (a.slope_pos[h] * (float)a.pos[tok] +
+                                  a.slope_time[h] * (float)(a.ts[tok] - t0));
+        const long long idx = (long long)h * Tp + base + i;
+        cbias[idx] = c;
+        lse2[idx] = a.lse_in[(long long)h * a.T + tok] * kLog2e + c;
+        dsum[idx] = dd;
+      }
+    }
+    return;
+  }
+  __shared__ int hist[kMaxBuckets];
+  __shared__ int cursor[kMaxBuckets];
+  for (int i = threadIdx.x; i < kMaxBuckets; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int u = threadIdx.x; u < a.B; u += blockDim.x) {
+      const long long s = a.off[u], e = a.off[u + 1];
+      if (s < 0 || e < s || e > a.T) {
+        if (pass == 0) flag(a.err, GENRANK_DERR_LAYOUT);
+        continue;
+      }
+      const int L = (int)(e - s);
+      const int n = max(0, min(a.hist_len[u], L));
+      const int qtiles = (L + BM - 1) / BM;
+      if (pass == 0 && qtiles > max_tiles) flag(a.err, GENRANK_DERR_LAYOUT);
+      const int ktiles = min((n + BM - 1) / BM, max_tiles);
+      for (int kt = 0; kt < ktiles; ++kt) {
+        const int nq = min(qtiles, max_tiles) - kt;
+        const int bucket = min(nq, kMaxBuckets - 1);
+        if (pass == 0) {
+          atomicAdd(&hist[bucket], 1);
+        } else {
+          const int slot = atomicAdd(&cursor[bucket], 1);
+          recs[2 * slot] = make_int4((int)s, L, n, kt * BM);
+          recs[2 * slot + 1] = make_int4(nq, (int)seg_start(s, u), u, 0);
+        }
+      }
+    }
+    __syncthreads();
+    if (pass == 0 && threadIdx.x == 0) {
+      int acc = 0;
+      for (int q = kMaxBuckets - 1; q >= 0; --q) {
+        cursor[q] = acc;
+        acc += hist[q];
+      }
+      *count = acc;
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// main kernel
+// ------------------------------------------------------------------------------------------
+GR_DEVICE uint32_t parity(int fill) { return (uint32_t)(fill & 1); }
+
+GR_DEVICE bool wait_warp(uint64_t* bar, uint32_t par, volatile int* abort_flag, int32_t* err) {
+  const bool ok = mbar_wait(bar, par, abort_flag, err);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Write 32 bf16 values (16 packed words) of row r, keys/queries [c0, c0+32), into a
+// 128-column operand tile laid out as two 64-column blocks of 128-byte rows with
+// 16-byte chunks XOR-swizzled by row (the UMMA 128B-swizzle canonical layout).
+GR_DEVICE void store_row_chunk(uint8_t* tile, int r, int c0, const uint32_t (&pk)[16]) {
+  const int blk = c0 >> 6;
+  uint8_t* row = tile + blk * (BM * 128) + r * 128;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int cc = ((c0 & 63) >> 3) + q;
+    *reinterpret_cast<uint4*>(row + ((cc ^ (r & 7)) << 4)) =
+        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_constant__ Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const AttnArgs& a = P.a;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[kKVFull], 1);
+    mbar_init(&bars[kKVEmpty], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[kQDFull + i], 1);
+      mbar_init(&bars[kQDEmpty + i], 1);
+      mbar_init(&bars[kDQFull + i], 1);
+      mbar_init(&bars[kDQEmpty + i], 128);
+    }
+    mbar_init(&bars[kSFull], 1);
+    mbar_init(&bars[kPFull], 128);
+    mbar_init(&bars[kPSFree], 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&P.tq);
+    tma_prefetch_desc(&P.tk);
+    tma_prefetch_desc(&P.tv);
+    tma_prefetch_desc(&P.tdo);
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int total = *P.count * a.H;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- TMA producer
+    int it = 0, g = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const Rec rc = load_rec(P, w);
+      if (!wait_warp(&bars[kKVEmpty], parity(it) ^ 1u, abort_flag, a.err)) break;
+      if (lane == 0) {
+        mbar_expect_tx(&bars[kKVFull], 2 * kTileBytes);
+        tma_load_3d(smem + kOffK, &P.tk, &bars[kKVFull], 0, rc.h, rc.s + rc.k0);
+        tma_load_3d(smem + kOffV, &P.tv, &bars[kKVFull], 0, rc.h, rc.s + rc.k0);
+      }
+      const long long roff = (long long)rc.h * P.Tp + rc.spad;
+      bool ok = true;
+      for (int t = 0; t < rc.nq; ++t, ++g) {
+        const int st = g & 1;
+        if (!wait_warp(&bars[kQDEmpty + st], parity(g >> 1) ^ 1u, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          const int q0 = rc.k0 + t * BM;
+          mbar_expect_tx(&bars[kQDFull + st], 2 * kTileBytes + 2 * kRowBytes);
+          tma_load_3d(smem + kOffQ + st * kTileBytes, &P.tq, &bars[kQDFull + st], 0, rc.h,
+                      rc.s + q0);
+          tma_load_3d(smem + kOffDO + st * kTileBytes, &P.tdo, &bars[kQDFull + st], 0, rc.h,
+                      rc.s + q0);
+          bulk_load(smem + kOffL2 + st * kRowBytes, P.lse2 + roff + q0, kRowBytes,
+                    &bars[kQDFull + st]);
+          bulk_load(smem + kOffD + st * kRowBytes, P.dsum + roff + q0, kRowBytes,
+                    &bars[kQDFull + st]);
+        }
+      }
+      if (!ok) break;
+    }
+  } else if (warp == 5 && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    const uint32_t sK = smem_u32(smem + kOffK), sV = smem_u32(smem + kOffV),
+                   sQ = smem_u32(smem + kOffQ), sDO = smem_u32(smem + kOffDO),
+                   sP = smem_u32(smem + kOffP), sDS = smem_u32(smem + kOffDS);
+    auto issue_sdp = [&](int gg) {
+      const int st = gg & 1;
+#pragma unroll
+      for (int k = 0; k < DH / 16; ++k) {
+        mma_bf16_ss(tmem + kColS, smem_desc_sw128(sK + k * 32, 16, 1024),
+                    smem_desc_sw128(sQ + st * kTileBytes + k * 32, 16, 1024), kIdescS,
+                    k > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < DH / 16; ++k) {
+        mma_bf16_ss(tmem + kColDP, smem_desc_sw128(sV + k * 32, 16, 1024),
+                    smem_desc_sw128(sDO + st * kTileBytes + k * 32, 16, 1024), kIdescS,
+                    k > 0 ? 1u : 0u);
+      }
+      mma_commit(&bars[kSFull]);
+    };
+    int it = 0, g = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < total && ok && !*abort_flag; w += gridDim.x, ++it) {
+      const Rec rc = load_rec(P, w);
+      if (!mbar_wait(&bars[kKVFull], parity(it), abort_flag, a.err) ||
+          !mbar_wait(&bars[kQDFull + (g & 1)], parity(g >> 1), abort_flag, a.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      issue_sdp(g);
+      for (int t = 0; t < rc.nq; ++t, ++g) {
+        const int st = g & 1;
+        if (!mbar_wait(&bars[kPFull], parity(g), abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // the next query tile's S^T, dP^T first: the softmax warps need them next
+        if (t + 1 < rc.nq) {
+          if (!mbar_wait(&bars[kQDFull + ((g + 1) & 1)], parity((g + 1) >> 1), abort_flag,
+                         a.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_sdp(g + 1);
+        }
+        // dV += P^T dO ; dK += dS^T Q   (K = 128 queries, 8 steps)
+#pragma unroll
+        for (int k = 0; k < BM / 16; ++k) {
+          const uint32_t aoff = (k >> 2) * (BM * 128) + (k & 3) * 32;
+          const uint64_t bdo =
+              smem_desc_sw128(sDO + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
+          mma_bf16_ss(tmem + kColDV, smem_desc_sw128(sP + aoff, 16, 1024), bdo, kIdescKV,
+                      (t > 0 || k > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < BM / 16; ++k) {
+          const uint32_t aoff = (k >> 2) * (BM * 128) + (k & 3) * 32;
+          const uint64_t bq =
+              smem_desc_sw128(sQ + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
+          mma_bf16_ss(tmem + kColDK, smem_desc_sw128(sDS + aoff, 16, 1024), bq, kIdescKV,
+                      (t > 0 || k > 0) ? 1u : 0u);
+        }
+        // dQ_part = dS K  (M = queries read from dS^T as MN-major, K = 128 keys)
+        const int db = g & 1;
+        if (!mbar_wait(&bars[kDQEmpty + db], parity(g >> 1) ^ 1u, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < BM / 16; ++k) {
+          const uint64_t ads = smem_desc_sw128(sDS + k * 16 * 128, BM * 128, 1024);
+          const uint64_t bk = smem_desc_sw128(sK + k * 16 * 128, kTileBytes, 1024);
+          mma_bf16_ss(tmem + kColDQ + db * DH, ads, bk, kIdescQ, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[kDQFull + db]);
+        mma_commit(&bars[kPSFree]);
+        mma_commit(&bars[kQDEmpty + st]);
+      }
+      if (!ok) break;
+      mma_commit(&bars[kKVEmpty]);
+    }
+  } else if (warp < 4) {
+    // ---------------------------------------------------------------- softmax (key rows)
+    const int r = threadIdx.x;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float scale_log2 = a.scale * kLog2e;
+    const float* sL2 = reinterpret_cast<const float*>(smem + kOffL2);
+    const float* sD = reinterpret_cast<const float*>(smem + kOffD);
+    uint8_t* sP = smem + kOffP;
+    uint8_t* sDS = smem + kOffDS;
+    int g = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      __syncwarp();
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const Rec rc = load_rec(P, w);
+      const int j = rc.k0 + r;  // this thread's key (local index)
+      const bool key = j < rc.n;
+      const float cbj = key ? P.cbias[(long long)rc.h * P.Tp + rc.spad + j] : 0.f;
+      bool ok = true;
+      for (int t = 0; t < rc.nq; ++t, ++g) {
+        const int st = g & 1;
+        const int q0 = rc.k0 + t * BM;
+        if (!wait_warp(&bars[kSFull], parity(g), abort_flag, a.err) ||
+            !wait_warp(&bars[kQDFull + st], parity(g >> 1), abort_flag, a.err) ||
+            (g > 0 && !wait_warp(&bars[kPSFree], parity(g - 1), abort_flag, a.err))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // visible iff key valid, query row inside the user and i >= j
+        const int ilo = max(j, q0);  // first visible query (local index)
+        const int ihi = rc.L;        // one past the last
+        const float* l2 = sL2 + st * BM;
+        const float* dd = sD + st * BM;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BM; c0 += 32) {
+          float sv[32], dp[32];
+          tmem_ld32(tmem + lane_base + kColS + c0, sv);
+          tmem_ld32(tmem + lane_base + kColDP + c0, dp);
+          uint32_t pk[16], dk[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            float p2[2], ds2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int i = q0 + c0 + c + e;
+              const bool vis = key && i >= ilo && i < ihi;
+              const float x = fmaf(sv[c + e], scale_log2, cbj - l2[c0 + c + e]);
+              const float p = vis ? ex2(x) : 0.f;
+              p2[e] = p;
+              ds2[e] = p * (dp[c + e] - dd[c0 + c + e]);
+            }
+            pk[c / 2] = pack_bf16(p2[0], p2[1]);
+            dk[c / 2] = pack_bf16(ds2[0], ds2[1]);
+          }
+          store_row_chunk(sP, r, c0, pk);
+          store_row_chunk(sDS, r, c0, dk);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars[kPFull]);
+      }
+      if (!ok) break;
+      // record epilogue: dK (times scale) and dV of this key tile, once its last
+      // gradient MMAs are done
+      if (!wait_warp(&bars[kPSFree], parity(g - 1), abort_flag, a.err)) break;
+      tc_fence_after();
+      float dvr[DH], dkr[DH];
+      tmem_ld64(tmem + lane_base + kColDV, dvr);
+      tmem_ld64(tmem + lane_base + kColDK, dkr);
+      tc_fence_before();
+      if (key) {
+        const long long tok = (long long)rc.s + j;
+        __nv_bfloat16* dkp = (__nv_bfloat16*)a.dk + tok * a.tok_stride + rc.h * DH;
+        __nv_bfloat16* dvp = (__nv_bfloat16*)a.dv + tok * a.tok_stride + rc.h * DH;
+#pragma unroll
+        for (int c = 0; c < DH; c += 8) {
+          float f[8], v8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            f[e] = dkr[c + e] * a.scale;
+            v8[e] = dvr[c + e];
+          }
+          *reinterpret_cast<uint4*>(dkp + c) = Elem<__nv_bfloat16>::pack(f);
+          *reinterpret_cast<uint4*>(dvp + c) = Elem<__nv_bfloat16>::pack(v8);
+        }
+      }
+    }
+  } else if (warp >= 6) {
+    // ---------------------------------------------------------------- dQ reduction (query rows)
+    const int qlane = 32 * (warp & 3) + lane;  // TMEM lane this thread may read
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    int g = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      __syncwarp();
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const Rec rc = load_rec(P, w);
+      bool ok = true;
+      for (int t = 0; t < rc.nq; ++t, ++g) {
+        const int db = g & 1;
+        if (!wait_warp(&bars[kDQFull + db], parity(g >> 1), abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float dq[DH];
+        tmem_ld64(tmem + lane_base + kColDQ + db * DH, dq);
+        tc_fence_before();
+        mbar_arrive(&bars[kDQEmpty + db]);
+        const int i = rc.k0 + t * BM + qlane;
+        if (i < rc.L) {
+          float* dst = P.dqacc + (((long long)rc.s + i) * a.H + rc.h) * DH;
+#pragma unroll
+          for (int c = 0; c < DH; c += 4)
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + c),
+                         "f"(dq[c]), "f"(dq[c + 1]), "f"(dq[c + 2]), "f"(dq[c + 3])
+                         : "memory");
+        }
+      }
+      if (!ok) break;
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------------------------------
+// finishing kernel: dq from the accumulator, and the candidate self terms
+// ------------------------------------------------------------------------------------------
+// One warp per (token, head), two of the 64 columns per lane.  For a candidate token c
+// (its own key, bias 0): p = exp(scale q.k - LSE), ds = p (dO.v - D),
+// dv = p dO, dk = scale ds q, and dq gains scale ds k.
+__global__ void __launch_bounds__(256) k_bwd_finish(const __grid_constant__ AttnArgs a,
+                                                    const float* __restrict__ dqacc,
+                                                    const float* __restrict__ dsum, long long Tp,
+                                                    int tokens_per_warp) {
+  const int lane = threadIdx.x & 31;
+  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long t0 = warp * tokens_per_warp;
+  const long long tend = min(a.T, (long long)a.off[a.B]);
+  if (t0 >= tend) return;
+  const long long t1 = min(tend, t0 + tokens_per_warp);
+  int u = warp_find_user(a.off, a.B, t0);
+  long long u_beg = a.off[u], u_end = a.off[u + 1];
+  int n = a.hist_len[u];
+  const __nv_bfloat16* Q = (const __nv_bfloat16*)a.q;
+  const __nv_bfloat16* K = (const __nv_bfloat16*)a.k;
+  const __nv_bfloat16* V = (const __nv_bfloat16*)a.v;
+  const __nv_bfloat16* G = (const __nv_bfloat16*)a.dO;
+  for (long long t = t0; t < t1; ++t) {
+    while (t >= u_end && u < a.B - 1) {
+      ++u;
+      u_beg = u_end;
+      u_end = a.off[u + 1];
+      n = a.hist_len[u];
+    }
+    const bool cand = (t - u_beg) >= n;
+    const long long base = seg_start(u_beg, u);
+    for (int h = 0; h < a.H; ++h) {
+      const float2 acc = *reinterpret_cast<const float2*>(dqacc + (t * a.H + h) * DH + 2 * lane);
+      float dq0 = acc.x * a.scale, dq1 = acc.y * a.scale;
+      const long long qo = t * a.tok_stride + h * DH + 2 * lane;
+      if (cand) {
+        const uint32_t qw = *reinterpret_cast<const uint32_t*>(Q + qo);
+        const uint32_t kw = *reinterpret_cast<const uint32_t*>(K + qo);
+        const uint32_t vw = *reinterpret_cast<const uint32_t*>(V + qo);
+        const uint32_t gw =
+            *reinterpret_cast<const uint32_t*>(G + t * a.o_stride + h * DH + 2 * lane);
+        float sdot = bf16_lo(qw) * bf16_lo(kw) + bf16_hi(qw) * bf16_hi(kw);
+        float pdot = bf16_lo(gw) * bf16_lo(vw) + bf16_hi(gw) * bf16_hi(vw);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
+          pdot += __shfl_xor_sync(0xffffffffu, pdot, o);
+        }
+        const long long ridx = (long long)h * Tp + base + (t - u_beg);
+        const float p = expf(sdot * a.scale - a.lse_in[(long long)h * a.T + t]);
+        const float ds = p * (pdot - dsum[ridx]);
+        dq0 += a.scale * ds * bf16_lo(kw);
+        dq1 += a.scale * ds * bf16_hi(kw);
+        *reinterpret_cast<uint32_t*>((__nv_bfloat16*)a.dk + qo) =
+            pack_bf16(a.scale * ds * bf16_lo(qw), a.scale * ds * bf16_hi(qw));
+        *reinterpret_cast<uint32_t*>((__nv_bfloat16*)a.dv + qo) =
+            pack_bf16(p * bf16_lo(gw), p * bf16_hi(gw));
+      }
+      *reinterpret_cast<uint32_t*>((__nv_bfloat16*)a.dq + qo) = pack_bf16(dq0, dq1);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+static bool make_map(CUtensorMap* m, const void* base, long long T, int H, long long stride) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)DH, (cuuint64_t)H, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)DH * 2, (cuuint64_t)stride * 2};
+  cuuint32_t box[3] = {(cuuint32_t)DH, 1, (cuuint32_t)BM};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+static int max_tiles_of(int max_seqlen) { return (max_seqlen + BM - 1) / BM; }
+static size_t recs_bytes(int B, int max_seqlen) {
+  return ((size_t)B * max_tiles_of(max_seqlen) * 32 + 15) / 16 * 16;
+}
+static size_t rows_bytes(long long T, int B, int H) {
+  return ((size_t)H * scratch_tp(T, B) * sizeof(float) + 15) / 16 * 16;
+}
+
+}  // namespace tcb
+
+size_t attn_bwd_tc_workspace(int B, long long T, int H, int max_seqlen) {
+  using namespace tcb;
+  return kHeaderBytes + recs_bytes(B, max_seqlen) + 3 * rows_bytes(T, B, H) +
+         (size_t)T * H * DH * sizeof(float);
+}
+
+int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
+  using namespace tcb;
+  if (a.dh != DH || a.dtype != GENRANK_BF16) return GENRANK_ERR_UNSUPPORTED;
+  if (a.T + (long long)BM >= INT32_MAX / 2) return GENRANK_ERR_UNSUPPORTED;
+  Params p;
+  if (!make_map(&p.tq, a.q, a.T, a.H, a.tok_stride) ||
+      !make_map(&p.tk, a.k, a.T, a.H, a.tok_stride) ||
+      !make_map(&p.tv, a.v, a.T, a.H, a.tok_stride) ||
+      !make_map(&p.tdo, a.dO, a.T, a.H, a.o_stride))
+    return GENRANK_ERR_CUDA;
+  p.a = a;
+  uint8_t* ws = (uint8_t*)a.ws;
+  p.count = (int32_t*)ws;
+  p.recs = (int4*)(ws + kHeaderBytes);
+  const size_t rb = rows_bytes(a.T, a.B, a.H);
+  uint8_t* rows = ws + kHeaderBytes + recs_bytes(a.B, a.max_seqlen);
+  p.cbias = (float*)rows;
+  p.lse2 = (float*)(rows + rb);
+  p.dsum = (float*)(rows + 2 * rb);
+  p.dqacc = (float*)(rows + 3 * rb);
+  p.Tp = scratch_tp(a.T, a.B);
+  if (cudaMemsetAsync(p.dqacc, 0, (size_t)a.T * a.H * DH * sizeof(float), st) != cudaSuccess)
+    return GENRANK_ERR_CUDA;
+  k_bwd_prologue<<<a.B + 1, 256, 0, st>>>(a, max_tiles_of(a.max_seqlen), (int4*)p.recs,
+                                          (int32_t*)p.count, (float*)p.cbias, (float*)p.lse2,
+                                          (float*)p.dsum, p.Tp);
+  if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(k_attn_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes) != cudaSuccess)
+      return GENRANK_ERR_CUDA;
+    attr = true;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  k_attn_bwd_tc<<<sms, kThreads, kSmemBytes, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
+  const long long warps_target = (long long)sms * 64;
+  const long long tpw_ll = (a.T + warps_target - 1) / warps_target;
+  const int tpw = (int)(tpw_ll > 0 ? tpw_ll : 1);
+  const long long warps = (a.T + tpw - 1) / tpw;
+  k_bwd_finish<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(a, p.dqacc, p.dsum, p.Tp, tpw);
+  return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
+}
+
+}  // namespace gr

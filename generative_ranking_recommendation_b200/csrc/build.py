@@ -21,7 +21,7 @@ ROOT = os.path.dirname(PKG)
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgenrank.so")
-SOURCES = ["api.cu", "embed.cu", "attn_simt.cu", "attn_tc.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "embed.cu", "attn_simt.cu", "attn_tc.cu", "attn_bwd_tc.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -103,8 +103,10 @@ int launch_attn_fwd_simt(const AttnArgs& a, cudaStream_t st);
 int launch_attn_bwd_simt(const AttnArgs& a, cudaStream_t st);
 size_t attn_bwd_simt_workspace(int B, long long T, int H, int dh, int max_seqlen);
 
-// tcgen05 / TMEM / TMA attention forward (bf16, dh = 64)
+// tcgen05 / TMEM / TMA attention forward and backward (bf16, dh = 64)
 int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st);
 size_t attn_fwd_tc_workspace(int B, long long T, int H, int max_seqlen);
+int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st);
+size_t attn_bwd_tc_workspace(int B, long long T, int H, int max_seqlen);
 
 }  // namespace gr

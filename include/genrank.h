@@ -176,7 +176,9 @@ int genrank_attn_fwd(int B, int64_t T, const int32_t *seq_offsets, const int32_t
  * of q, k, v (tok_stride).  The biases have no parameters, so there is no bias
  * gradient.  With P = softmax(S): dV = P^T dO, dP = dO V^T,
  * dS = P * (dP - rowsum(dO * O)), dQ = scale dS K, dK = scale dS^T Q.
- * Every token row of dq/dk/dv is written (no accumulation into them). */
+ * Every token row of dq/dk/dv is written (no accumulation into them).
+ * bf16 with dh = 64 runs on tcgen05 tensor cores (fp32 dQ accumulated in the
+ * workspace); fp32, or dh = 32, runs the CUDA-core kernels. */
 int genrank_attn_bwd(int B, int64_t T, const int32_t *seq_offsets, const int32_t *hist_len, int max_seqlen,
                      const void *q, const void *k, const void *v, int64_t tok_stride, int H,
                      int dh, const int32_t *pos, const int64_t *ts, const float *slope_pos,

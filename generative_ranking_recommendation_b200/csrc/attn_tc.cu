@@ -5,31 +5,33 @@
 //   s_ij = scale q_i.k_j - m_h |p_i - p_j| - m_t,h |t_i - t_j|, history rows causal,
 //   candidate rows see all history and themselves.
 //
-// Design (bf16 inputs, head dim 64, fp32 accumulation):
+// Design (bf16 inputs, head dim 64, fp32 accumulation), one CTA per SM:
 //   * A prologue kernel lists (user, 128-row query tile) work records sorted by the
 //     number of 128-key tiles they visit (longest first), and writes the ALiBi
 //     column term c_j = log2(e) (m_h p_j + m_t,h (t_j - t_0)) for every token and
 //     head into a 16-byte aligned scratch layout.  On visible pairs p_i >= p_j and
 //     t_i >= t_j, so the bias is c_j - c_i; c_i cancels in the softmax and only c_j
 //     is added per element; the literal LSE subtracts c_i in the epilogue.
-//   * Persistent grid, two CTAs per SM; each CTA walks the records round-robin
-//     (one head per work item).  Key tiles a query tile never sees are never
-//     visited: history tile t visits key tiles 0..t, candidate rows the history only.
-//   * Warp 4 issues TMA loads (Q; K, V two-stage ring; 128B swizzle, no multicast)
-//     and a bulk copy of the key tile's column terms.
-//   * Warp 5 (one thread) issues tcgen05.mma: S = Q K^T (128 x 128, fp32 in TMEM)
-//     from shared memory, then O += P V (128 x 64, fp32 in TMEM) with P read from
-//     tensor memory, where the softmax left it in place of S (bf16 pairs).
-//   * Warps 0-3 (one query row per thread, one TMEM lane each) load S, add the
-//     column term, mask only tiles that straddle a row's last visible key, and run
-//     the online softmax with a lazily updated offset: O in TMEM is rescaled only
-//     when a row's maximum grows by more than 2^8, so most tiles touch O not at all.
-//   * The other CTA on the SM hides each CTA's per-item latencies (work-record
-//     loads, the epilogue's global loads and stores).
-//   * A candidate's own key lies outside the tiles it visits; its score (bias 0)
-//     is merged into the softmax state in the epilogue on CUDA cores.
-// Every mbarrier wait is bounded in time; a timeout sets GENRANK_DERR_TIMEOUT,
-// every role drains out of its loop and the CTA frees its tensor memory.
+//   * A persistent grid walks the records round-robin (one head per work item).  An
+//     item visits its history key tiles (history tile t: key tiles 0..t; candidate
+//     rows: the history only; most recent keys first) and, when it holds candidate
+//     rows, one diagonal tile: its own rows as keys, of which only each candidate's
+//     own key (bias 0) is kept.  Key tiles a query tile never sees are never visited.
+//   * Warp 12 issues TMA loads (Q with the rows' own column terms, double-buffered;
+//     K, V and their column terms in a five-stage ring; 128B swizzle, no multicast).
+//   * Warp 13 (one thread) issues tcgen05.mma: S = Q K^T (128 x 128, fp32) into one
+//     of two TMEM buffers, the next S before the current P V, and O += P V (128 x 64,
+//     fp32) into the item's TMEM O buffer (two, alternating by item), P (bf16 pairs)
+//     read from one of two TMEM P buffers.
+//   * Warps 0-7 stream the softmax with two threads per query row, each on one half
+//     of the key columns (TMEM access shape 16x32bx2), so two softmax warps share
+//     each SM sub-partition: bias, mask and exponentials in one pass per tile, with
+//     the offset fixed at the row's own column term (every visible key has
+//     c_j <= c_i); a tile whose row sum leaves the safe range is redone exactly and O
+//     rescaled in TMEM.
+//   * Warps 8-11 (one row per thread) finish each item from its O buffer while the
+//     next item runs: O is normalised and written through shared memory as whole
+//     128-byte rows, and the literal LSE is stored.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -42,27 +44,34 @@ namespace tc {
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
 constexpr int DH = 64;   // head dim
-constexpr int kThreads = 192;  // warps 0-3 softmax, warp 4 TMA, warp 5 MMA
+constexpr int kThreads = 448;  // warps 0-7 softmax, 8-11 epilogue, 12 TMA, 13 MMA
+constexpr int kSoftmaxThreads = 256;
+constexpr int kStages = 5;     // K/V ring
 constexpr uint32_t kTileBytes = BM * DH * 2;  // one Q, K or V tile (16 KB)
 constexpr uint32_t kCBBytes = BN * 4;         // column terms of one key tile
 constexpr float kOverflowSum = 1.2676506e30f;   // 2^100: a tile's row sum above this is redone
 constexpr float kUnderflowSum = 7.8886091e-31f;  // 2^-100: a first tile's row sum below this too
 
 // dynamic shared memory layout (offsets from a 1024-byte aligned base)
-constexpr uint32_t kOffQ = 0;                          // 16 KB
-constexpr uint32_t kOffK = kOffQ + kTileBytes;         // 2 x 16 KB
-constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;     // 2 x 16 KB
-constexpr uint32_t kOffCB = kOffV + 2 * kTileBytes;    // 2 x 512 B
-constexpr uint32_t kOffBar = kOffCB + 2 * kCBBytes;    // barriers
-constexpr uint32_t kNumBars = 12;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+constexpr uint32_t kOffQ = 0;                                // 2 x 16 KB
+constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;           // kStages x 16 KB
+constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;     // kStages x 16 KB
+constexpr uint32_t kOffCB = kOffV + kStages * kTileBytes;    // kStages x 512 B
+constexpr uint32_t kOffQCB = kOffCB + kStages * kCBBytes;    // 2 x 512 B: the rows' own terms
+constexpr uint32_t kOffStage = kOffQCB + 2 * kCBBytes;       // O rows staged, 16 KB
+constexpr uint32_t kOffML = kOffStage + BM * DH * 2;         // (m, l) per row, 2 buffers
+constexpr uint32_t kOffRec = kOffML + 2 * BM * 8;            // item record with each Q tile
+constexpr uint32_t kOffBar = kOffRec + 2 * 16;               // barriers
+constexpr uint32_t kNumBars = 17 + 3 * kStages;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;        // tmem base, abort flag
+constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;        // + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
-// TMEM columns (per CTA; two CTAs share an SM's 512)
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0;    // S (fp32, 128 columns)
-constexpr uint32_t kColO = 128;  // O (fp32, 64 columns)
-constexpr uint32_t kColP = 192;  // P (bf16 pairs, 64 columns)
+// TMEM columns (the whole 512 of the SM)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;    // two S buffers (fp32, 128 columns each)
+constexpr uint32_t kColP = 256;  // two P buffers (bf16 pairs, 64 columns each)
+constexpr uint32_t kColO = 384;  // two O buffers (fp32, 64 columns each)
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);   // Q K-major, K K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, DH, 0, 1);  // P K-major (TMEM), V MN-major
@@ -80,11 +89,19 @@ struct Params {
   long long Tp;
 };
 
-enum Bar { kQFull = 0, kQEmpty = 1, kKFull = 2, kVFull = 4, kKVEmpty = 6, kSFull = 8,
-           kPFull = 9, kPVFull = 10 };
+enum Bar {
+  kQFull = 0, kQEmpty = 2, kSFull = 4, kSFree = 6, kPFull = 8, kPFree = 10, kOFull = 12,
+  kOEmpty = 14, kDone = 16, kKFull = 17, kVFull = kKFull + kStages, kKVEmpty = kVFull + kStages
+};
+static_assert(kKVEmpty + kStages <= (int)kNumBars, "barriers");
+
+GR_DEVICE int tiles_of(int q0, int n, int L, int nk) {
+  return nk + (min(q0 + BM, L) > n ? 1 : 0);
+}
 
 struct Item {
   int s, L, n, q0, nk, spad, h;
+  int nt;  // tiles visited: nk key tiles, plus the diagonal tile when candidates are present
 };
 
 GR_DEVICE Item load_item(const Params& P, int w) {
@@ -99,6 +116,7 @@ GR_DEVICE Item load_item(const Params& P, int w) {
   it.q0 = r0.w;
   it.nk = r1.x;
   it.spad = r1.y;
+  it.nt = tiles_of(it.q0, it.n, it.L, it.nk);
   return it;
 }
 
@@ -180,138 +198,201 @@ __global__ void __launch_bounds__(256) k_prologue(const __grid_constant__ AttnAr
 // ------------------------------------------------------------------------------------------
 // the attention kernel
 // ------------------------------------------------------------------------------------------
-GR_DEVICE uint32_t parity(int fill) { return (uint32_t)(fill & 1); }
+GR_DEVICE uint32_t par(int use) { return (uint32_t)(use & 1); }
 
 // Every lane waits (bounded), then the warp agrees, so that the warp stays
 // converged for the .sync.aligned tcgen05 instructions that follow.
-GR_DEVICE bool wait_warp(uint64_t* bar, uint32_t par, volatile int* abort_flag, int32_t* err) {
-  const bool ok = mbar_wait(bar, par, abort_flag, err);
+GR_DEVICE bool wait_warp(uint64_t* bar, uint32_t ph, volatile int* abort_flag, int32_t* err) {
+  const bool ok = mbar_wait(bar, ph, abort_flag, err);
   return __all_sync(0xffffffffu, ok);
 }
 
-// x = s * scale + c_j for 32 columns starting at key c0 of the tile; columns at or
-// beyond nvalid are masked.  Four independent running maxima shorten the chain.
+// Each softmax thread owns one half of a query row: key columns [64 h, 64 h + 64) of
+// every tile (h = lane / 16), reached with the 16x32bx2 TMEM shape: S columns at
+// offset 64, packed P columns at offset 32, O columns at offset 32.
+constexpr int kHalf = BN / 2;
+constexpr int CW = 16;  // key columns per chunk (of the thread's 64)
+GR_DEVICE void s_load(uint32_t taddr, uint32_t (&r)[CW]) { tmem_ld_half16_async<kHalf>(taddr, r); }
+GR_DEVICE void p_store(uint32_t taddr, const uint32_t (&pk)[CW / 2]) {
+  tmem_st_half8_nowait<kHalf / 2>(taddr, pk);
+}
+
+// x = s * scale + c_j for CW columns (key kc0 + c of the tile); keys at or beyond
+// nvalid are masked.  Four independent running maxima shorten the chain.
 template <bool kMasked>
-GR_DEVICE void row_max_chunk(const uint32_t (&s)[32], const float* cb, int c0, int nvalid,
+GR_DEVICE void row_max_chunk(const uint32_t (&s)[CW], const float* cb, int kc0, int nvalid,
                              float scale_log2, float (&mx4)[4]) {
 #pragma unroll
-  for (int c = 0; c < 32; c += 4) {
+  for (int c = 0; c < CW; c += 4) {
     const float4 b4 = *reinterpret_cast<const float4*>(cb + c);
     const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float v = fmaf(__uint_as_float(s[c + e]), scale_log2, bb[e]);
-      mx4[e] = fmaxf(mx4[e], (!kMasked || c0 + c + e < nvalid) ? v : -INFINITY);
+      mx4[e] = fmaxf(mx4[e], (!kMasked || kc0 + c + e < nvalid) ? v : -INFINITY);
     }
   }
 }
 
-// p = 2^(x - m) for 32 columns, summed into four partial row sums, packed to bf16
-// pairs and stored to 16 TMEM columns at taddr.
+// p = 2^(x - m) for CW columns, summed into four partial sums, packed to bf16 pairs
+// and stored (without waiting) to CW / 2 TMEM columns at taddr.
 template <bool kMasked>
-GR_DEVICE void exp_pack_store(const uint32_t (&s)[32], const float* cb, int c0, int nvalid,
+GR_DEVICE void exp_pack_store(const uint32_t (&s)[CW], const float* cb, int kc0, int nvalid,
                               float scale_log2, float m_use, float (&rs4)[4], uint32_t taddr) {
-  uint32_t pk[16];
+  uint32_t pk[CW / 2];
 #pragma unroll
-  for (int c = 0; c < 32; c += 4) {
+  for (int c = 0; c < CW; c += 4) {
     const float4 b4 = *reinterpret_cast<const float4*>(cb + c);
     const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
     float p[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float v = fmaf(__uint_as_float(s[c + e]), scale_log2, bb[e] - m_use);
-      p[e] = (!kMasked || c0 + c + e < nvalid) ? ex2(v) : 0.f;
+      p[e] = (!kMasked || kc0 + c + e < nvalid) ? ex2(v) : 0.f;
       rs4[e] += p[e];
     }
     pk[c / 2] = pack_bf16(p[0], p[1]);
     pk[c / 2 + 1] = pack_bf16(p[2], p[3]);
   }
-  tmem_st16(taddr, pk);
+  p_store(taddr, pk);
 }
 
-// Row maximum of x = s * scale + c_j over the tile, 32 columns at a time with the
-// next chunk's TMEM load in flight.
+// Maximum of x = s * scale + c_j over this thread's half of the tile (S at s_addr,
+// column terms of the half at cb, first key kbase), CW columns at a time with the
+// next chunk's load in flight.
 template <bool kMasked>
-GR_DEVICE float tile_max(uint32_t tmem_lane, const float* cb, int nvalid, float scale_log2) {
+GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, int kbase, int nvalid,
+                         float scale_log2) {
   float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-  uint32_t xa[32], xb[32];
-  tmem_ld32_async(tmem_lane + kColS, xa);
+  uint32_t xa[CW], xb[CW];
+  s_load(s_addr, xa);
   tmem_ld_wait(xa);
 #pragma unroll
-  for (int c0 = 0; c0 < BN; c0 += 64) {
-    tmem_ld32_async(tmem_lane + kColS + c0 + 32, xb);
-    row_max_chunk<kMasked>(xa, cb + c0, c0, nvalid, scale_log2, mx4);
+  for (int c0 = 0; c0 < kHalf; c0 += 2 * CW) {
+    s_load(s_addr + c0 + CW, xb);
+    row_max_chunk<kMasked>(xa, cb + c0, kbase + c0, nvalid, scale_log2, mx4);
     tmem_ld_wait(xb);
-    if (c0 + 64 < BN) tmem_ld32_async(tmem_lane + kColS + c0 + 64, xa);
-    row_max_chunk<kMasked>(xb, cb + c0 + 32, c0 + 32, nvalid, scale_log2, mx4);
-    if (c0 + 64 < BN) tmem_ld_wait(xa);
+    if (c0 + 2 * CW < kHalf) s_load(s_addr + c0 + 2 * CW, xa);
+    row_max_chunk<kMasked>(xb, cb + c0 + CW, kbase + c0 + CW, nvalid, scale_log2, mx4);
+    if (c0 + 2 * CW < kHalf) tmem_ld_wait(xa);
   }
   return fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
 }
 
-// P = 2^(x - m) for the tile, written as bf16 pairs to the P columns, 32 keys at a
-// time with the next chunk's TMEM load in flight.  Returns the row sum.
+// P = 2^(x - m) for this thread's half of the tile, written as bf16 pairs to the P
+// columns at p_addr; the stores have landed when it returns.  Returns the half's sum.
 template <bool kMasked>
-GR_DEVICE float tile_exp(uint32_t tmem_lane, const float* cb, int nvalid, float scale_log2,
-                         float m) {
+GR_DEVICE float tile_exp(uint32_t s_addr, uint32_t p_addr, const float* cb, int kbase,
+                         int nvalid, float scale_log2, float m) {
   float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-  uint32_t xa[32], xb[32];
-  tmem_ld32_async(tmem_lane + kColS, xa);
+  uint32_t xa[CW], xb[CW];
+  s_load(s_addr, xa);
   tmem_ld_wait(xa);
 #pragma unroll
-  for (int c0 = 0; c0 < BN; c0 += 64) {
-    tmem_ld32_async(tmem_lane + kColS + c0 + 32, xb);
-    exp_pack_store<kMasked>(xa, cb + c0, c0, nvalid, scale_log2, m, rs4,
-                            tmem_lane + kColP + c0 / 2);
+  for (int c0 = 0; c0 < kHalf; c0 += 2 * CW) {
+    s_load(s_addr + c0 + CW, xb);
+    exp_pack_store<kMasked>(xa, cb + c0, kbase + c0, nvalid, scale_log2, m, rs4, p_addr + c0 / 2);
     tmem_ld_wait(xb);
-    if (c0 + 64 < BN) tmem_ld32_async(tmem_lane + kColS + c0 + 64, xa);
-    exp_pack_store<kMasked>(xb, cb + c0 + 32, c0 + 32, nvalid, scale_log2, m, rs4,
-                            tmem_lane + kColP + (c0 + 32) / 2);
-    if (c0 + 64 < BN) tmem_ld_wait(xa);
+    if (c0 + 2 * CW < kHalf) s_load(s_addr + c0 + 2 * CW, xa);
+    exp_pack_store<kMasked>(xb, cb + c0 + CW, kbase + c0 + CW, nvalid, scale_log2, m, rs4,
+                            p_addr + (c0 + CW) / 2);
+    if (c0 + 2 * CW < kHalf) tmem_ld_wait(xa);
   }
+  tmem_wait_st();
   return (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
 }
 
-// One key tile of the online softmax for this thread's row (TMEM lane).  The offset
+// O (this thread's 32 columns of its row) *= alpha, once the previous P V has landed.
+GR_DEVICE bool rescale_o(uint32_t o_addr, float alpha, uint64_t* prev_pv, uint32_t prev_ph,
+                         volatile int* abort_flag, int32_t* err) {
+  if (!wait_warp(prev_pv, prev_ph, abort_flag, err)) return false;
+  tc_fence_after();
+  uint32_t o[32];
+  tmem_ld_half32_async<DH / 2>(o_addr, o);
+  tmem_ld_wait(o);
+#pragma unroll
+  for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+  tmem_st_half32_nowait<DH / 2>(o_addr, o);
+  tmem_wait_st();
+  return true;
+}
+
+// One history key tile of the online softmax for this thread's half row.  The offset
 // m starts at the row's own column term c_i: every visible key has c_j <= c_i, so
 // 2^(x - m) <= 2^(scale q.k log2 e), which overflows only for extreme scores.  Each
 // tile is one pass; a tile whose row sum leaves [2^-100, 2^100] on the first tile
 // (every key far below the offset) or exceeds 2^100 later is redone with the exact
-// offset max(m, tile max), rescaling O in TMEM.  Before P is written, the previous
-// P V must have finished (it reads P and adds to O).
+// offset max(m, tile max), rescaling O in TMEM.  Rows past the user's end never
+// redo (their output is not written).
 template <bool kMasked>
-GR_DEVICE bool softmax_tile(uint32_t tmem_lane, const float* cb, int nvalid, float scale_log2,
-                            bool first, float& m, float& l, uint64_t* pv_bar, int g,
+GR_DEVICE bool softmax_tile(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, const float* cb,
+                            int kbase, int nvalid, float scale_log2, bool first, bool row_ok,
+                            float& m, float& l, uint64_t* prev_pv, uint32_t prev_ph,
                             volatile int* abort_flag, int32_t* err) {
-  if (g > 0 && !wait_warp(pv_bar, parity(g - 1), abort_flag, err)) return false;
-  tc_fence_after();
-  float rs = tile_exp<kMasked>(tmem_lane, cb, nvalid, scale_log2, m);
-  const bool redo = !(rs <= kOverflowSum) || (first && rs < kUnderflowSum);
+  float rs = tile_exp<kMasked>(s_addr, p_addr, cb, kbase, nvalid, scale_log2, m);
+  const float rs_row = rs + __shfl_xor_sync(0xffffffffu, rs, 16);
+  const bool redo = row_ok && (!(rs_row <= kOverflowSum) || (first && rs_row < kUnderflowSum));
   if (__any_sync(0xffffffffu, redo)) {
-    // every lane takes part in the .sync.aligned TMEM loads; only redo lanes move m
-    const float mx = tile_max<kMasked>(tmem_lane, cb, nvalid, scale_log2);
+    // every lane takes part in the .sync.aligned TMEM accesses; only redo rows move m
+    float mx = tile_max<kMasked>(s_addr, cb, kbase, nvalid, scale_log2);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
     const float m_new = redo ? (first ? mx : fmaxf(m, mx)) : m;
     const float alpha = first ? 1.f : ex2(m - m_new);
     m = m_new;
-    if (!first) {
-#pragma unroll 1
-      for (int c0 = 0; c0 < DH; c0 += 32) {
-        float o[32];
-        tmem_ld32(tmem_lane + kColO + c0, o);
-        uint32_t ob[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) ob[c] = __float_as_uint(o[c] * alpha);
-        tmem_st32(tmem_lane + kColO + c0, ob);
-      }
-    }
+    if (!first && !rescale_o(o_addr, alpha, prev_pv, prev_ph, abort_flag, err)) return false;
     l *= alpha;
-    rs = tile_exp<kMasked>(tmem_lane, cb, nvalid, scale_log2, m);
+    rs = tile_exp<kMasked>(s_addr, p_addr, cb, kbase, nvalid, scale_log2, m);
   }
   l = first ? rs : l + rs;
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_constant__ Params P) {
+// The diagonal tile: S = Q K^T over the item's own rows, of which a candidate row
+// keeps only its own key (position and time differences 0, so the bias is 0 and the
+// score is relative to c_i).  P is zero but for that key; the offset moves (O
+// rescaled) only if the term would overflow, or is set exactly on a first tile.
+GR_DEVICE bool softmax_diag(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, int rt, int h,
+                            bool cand_row, float rowcb, float scale_log2, bool first, float& m,
+                            float& l, uint64_t* prev_pv, uint32_t prev_ph,
+                            volatile int* abort_flag, int32_t* err) {
+  uint32_t xa[32], xb[32];
+  tmem_ld_half32_async<kHalf>(s_addr, xa);
+  tmem_ld_half32_async<kHalf>(s_addr + 32, xb);
+  tmem_ld_wait(xa);
+  tmem_ld_wait(xb);
+  const int col = rt - kHalf * h;  // the row's own key within this half
+  const bool mine = cand_row && col >= 0 && col < kHalf;
+  float sv = 0.f;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    sv = col == c ? __uint_as_float(xa[c]) : sv;
+    sv = col == c + 32 ? __uint_as_float(xb[c]) : sv;
+  }
+  const float xm = mine ? fmaf(sv, scale_log2, rowcb) : -INFINITY;
+  const float xr = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 16));  // the row's self score
+  const bool move = xr > -INFINITY && (first || xr - m > 100.f);
+  if (!first && __any_sync(0xffffffffu, move)) {
+    const float alpha = move ? ex2(m - xr) : 1.f;
+    if (!rescale_o(o_addr, alpha, prev_pv, prev_ph, abort_flag, err)) return false;
+    l *= alpha;
+  }
+  if (move) m = xr;
+  const float p = mine ? ex2(xm - m) : 0.f;
+  const uint32_t word = (col & 1) ? pack_bf16(0.f, p) : pack_bf16(p, 0.f);
+  uint32_t pk[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) pk[k] = (mine && k == (col >> 1)) ? word : 0u;
+  tmem_st_half32_nowait<kHalf / 2>(p_addr, pk);
+  tmem_wait_st();
+  l = first ? p : l + p;
+  return true;
+}
+
+struct Cursor {  // one key tile in the CTA's sequence: tile j of the qi-th item, g overall
+  int j, g, qi, nt;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_constant__ Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -320,28 +401,35 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   const float* sCB = reinterpret_cast<const float*>(smem + kOffCB);
+  float2* sML = reinterpret_cast<float2*>(smem + kOffML);  // [2][BM]: (m - c_i, l)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[kQFull], 1);
-    mbar_init(&bars[kQEmpty], 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars[kKFull + i], 1);
-      mbar_init(&bars[kVFull + i], 1);
-      mbar_init(&bars[kKVEmpty + i], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars[kQFull + b], 1);
+      mbar_init(&bars[kQEmpty + b], 1 + kSoftmaxThreads);  // last S commit + c_i reads
+      mbar_init(&bars[kSFull + b], 1);
+      mbar_init(&bars[kSFree + b], kSoftmaxThreads);
+      mbar_init(&bars[kPFull + b], kSoftmaxThreads);
+      mbar_init(&bars[kPFree + b], 1);
+      mbar_init(&bars[kOFull + b], 1 + kSoftmaxThreads);  // last P V commit + (m, l)
+      mbar_init(&bars[kOEmpty + b], 128);
     }
-    mbar_init(&bars[kSFull], 1);
-    mbar_init(&bars[kPFull], 128);
-    mbar_init(&bars[kPVFull], 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&bars[kKFull + st], 1);
+      mbar_init(&bars[kVFull + st], 1);
+      mbar_init(&bars[kKVEmpty + st], 1);
+    }
+    mbar_init(&bars[kDone], 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     tma_prefetch_desc(&P.tq);
     tma_prefetch_desc(&P.tk);
     tma_prefetch_desc(&P.tv);
   }
-  if (warp == 5) {
+  if (warp == 13) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -350,29 +438,45 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int total = *P.count * a.H;
+  const float scale_log2 = a.scale * kLog2e;
 
-  if (warp == 4) {
+  if (warp == 12) {
     // ---------------------------------------------------------------- TMA producer
+    // Each Q tile travels with the item's record (q0, n, L, nk); a record with nk < 0
+    // after the last item tells the MMA and softmax warps to stop.
+    int4* sRec = reinterpret_cast<int4*>(smem + kOffRec);
     int qi = 0, g = 0;
-    for (int w = blockIdx.x; w < total; w += gridDim.x) {
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+    bool ok = true;
+    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+        ok = false;
+        break;
+      }
       const Item it = load_item(P, w);
-      if (it.nk == 0) continue;
-      if (!wait_warp(&bars[kQEmpty], parity(qi) ^ 1u, abort_flag, a.err)) break;
-      if (lane == 0) {
-        mbar_expect_tx(&bars[kQFull], kTileBytes);
-        tma_load_3d(smem + kOffQ, &P.tq, &bars[kQFull], 0, it.h, it.s + it.q0);
+      if (it.nt == 0) continue;
+      const int qb = qi & 1;
+      if (!wait_warp(&bars[kQEmpty + qb], par(qi >> 1) ^ 1u, abort_flag, a.err)) {
+        ok = false;
+        break;
       }
       const float* cb_src = P.cbias + (long long)it.h * P.Tp + it.spad;
-      bool ok = true;
-      for (int j = 0; j < it.nk; ++j, ++g) {
-        const int st = g & 1;
-        if (!wait_warp(&bars[kKVEmpty + st], parity(g >> 1) ^ 1u, abort_flag, a.err)) {
+      if (lane == 0) {
+        sRec[qb] = make_int4(it.q0, it.n, it.L, it.nk);
+        mbar_expect_tx(&bars[kQFull + qb], kTileBytes + kCBBytes);
+        tma_load_3d(smem + kOffQ + qb * kTileBytes, &P.tq, &bars[kQFull + qb], 0, it.h,
+                    it.s + it.q0);
+        bulk_load(smem + kOffQCB + qb * kCBBytes, cb_src + it.q0, kCBBytes, &bars[kQFull + qb]);
+      }
+      ++qi;
+      for (int j = 0; j < it.nt; ++j) {
+        const int st = g % kStages;
+        if (!wait_warp(&bars[kKVEmpty + st], par(g / kStages) ^ 1u, abort_flag, a.err)) {
           ok = false;
           break;
         }
         if (lane == 0) {
-          const int kv0 = (it.nk - 1 - j) * BN;  // most recent keys first
+          // history key tiles most recent first, then the item's own rows
+          const int kv0 = j < it.nk ? (it.nk - 1 - j) * BN : it.q0;
           mbar_expect_tx(&bars[kKFull + st], kTileBytes + kCBBytes);
           tma_load_3d(smem + kOffK + st * kTileBytes, &P.tk, &bars[kKFull + st], 0, it.h,
                       it.s + kv0);
@@ -381,203 +485,213 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
           tma_load_3d(smem + kOffV + st * kTileBytes, &P.tv, &bars[kVFull + st], 0, it.h,
                       it.s + kv0);
         }
+        ++g;
       }
-      if (!ok) break;
+    }
+    if (ok && wait_warp(&bars[kQEmpty + (qi & 1)], par(qi >> 1) ^ 1u, abort_flag, a.err)) {
+      if (lane == 0) {
+        sRec[qi & 1] = make_int4(0, 0, 0, -1);
+        mbar_arrive(&bars[kQFull + (qi & 1)]);
+      }
       ++qi;
     }
-  } else if (warp == 5 && lane == 0) {
+    // on the way out, the copies issued last land before the CTA exits
+    if (lane == 0) {
+      for (int x = max(0, g - kStages); x < g; ++x) {
+        mbar_drain(&bars[kKFull + x % kStages], par(x / kStages));
+        mbar_drain(&bars[kVFull + x % kStages], par(x / kStages));
+      }
+      for (int x = max(0, qi - 2); x < qi; ++x) mbar_drain(&bars[kQFull + (x & 1)], par(x >> 1));
+    }
+  } else if (warp == 13) {
     // ---------------------------------------------------------------- MMA issuer (one thread)
-    // Per tile g: S_g = Q K_g^T is issued as soon as the softmax has released S_{g-1}
-    // (P lives in its own columns), so it overlaps P_{g-1} V_{g-1}.
-    const uint32_t sQ = smem_u32(smem + kOffQ), sK = smem_u32(smem + kOffK),
-                   sV = smem_u32(smem + kOffV);
-    auto next_item = [&](int from, Item& out) -> int {
-      for (int x = from; x < total; x += gridDim.x) {
-        out = load_item(P, x);
-        if (out.nk > 0) return x;
-      }
-      return -1;
-    };
-    auto issue_s = [&](int gg) {
-      const int st = gg & 1;
-#pragma unroll
-      for (int k = 0; k < DH / 16; ++k) {
-        const uint64_t ad = smem_desc_sw128(sQ + k * 32, 16, 1024);
-        const uint64_t bd = smem_desc_sw128(sK + st * kTileBytes + k * 32, 16, 1024);
-        mma_bf16_ss(tmem + kColS, ad, bd, kIdescS, k > 0 ? 1u : 0u);
-      }
-      mma_commit(&bars[kSFull]);
-    };
-    Item it;
-    int w = next_item(blockIdx.x, it);
-    // the record after the current item, loaded one item ahead of its use
-    Item pre = (w >= 0 && w + (int)gridDim.x < total) ? load_item(P, w + gridDim.x) : Item{};
-    int qi = 0, g = 0, j = 0;
-    bool ok = w >= 0 && mbar_wait(&bars[kQFull], parity(0), abort_flag, a.err) &&
-              mbar_wait(&bars[kKFull], parity(0), abort_flag, a.err);
-    if (ok) {
-      tc_fence_after();
-      issue_s(0);
-      if (it.nk == 1) mma_commit(&bars[kQEmpty]);
-    }
-    while (ok && !*abort_flag) {
-      if (!mbar_wait(&bars[kPFull], parity(g), abort_flag, a.err)) break;
-      // look ahead: the next tile of this item, or the first tile of the next item
-      Item it2 = it;
-      int w2 = w, j2 = j + 1;
-      if (j2 == it.nk) {
-        j2 = 0;
-        w2 = w + gridDim.x;
-        if (w2 >= total) {
-          w2 = -1;
-        } else if (pre.nk > 0) {
-          it2 = pre;
-        } else {
-          w2 = next_item(w2 + gridDim.x, it2);  // rare: items without keys to visit
-        }
-        if (w2 >= 0 && w2 + (int)gridDim.x < total) pre = load_item(P, w2 + gridDim.x);
-      }
-      if (w2 >= 0) {
-        if (j2 == 0 && !mbar_wait(&bars[kQFull], parity(qi + 1), abort_flag, a.err)) break;
-        if (!mbar_wait(&bars[kKFull + ((g + 1) & 1)], parity((g + 1) >> 1), abort_flag, a.err))
-          break;
+    // Tiles in order g = 0, 1, ...: S_{g+1} = Q K_{g+1}^T goes into the other S buffer
+    // before P_g V_g, so the softmax finds each S ready when it finishes the last one.
+    if (lane == 0) {
+      const uint32_t sQ = smem_u32(smem + kOffQ), sK = smem_u32(smem + kOffK),
+                     sV = smem_u32(smem + kOffV);
+      const int4* sRec = reinterpret_cast<const int4*>(smem + kOffRec);
+      // number of tiles of the qi-th item (its Q tile has landed), or -1 at the end
+      auto tiles = [&](int qi) -> int {
+        if (!mbar_wait(&bars[kQFull + (qi & 1)], par(qi >> 1), abort_flag, a.err)) return -1;
+        const int4 r = sRec[qi & 1];
+        return r.w < 0 ? -1 : tiles_of(r.x, r.y, r.z, r.w);
+      };
+      auto issue_s = [&](const Cursor& t) -> bool {
+        const int sb = t.g & 1, st = t.g % kStages, qb = t.qi & 1;
+        if (!mbar_wait(&bars[kSFree + sb], par(t.g >> 1) ^ 1u, abort_flag, a.err)) return false;
+        if (!mbar_wait(&bars[kKFull + st], par(t.g / kStages), abort_flag, a.err)) return false;
         tc_fence_after();
-        issue_s(g + 1);
-        if (j2 == it2.nk - 1) mma_commit(&bars[kQEmpty]);
-      }
-      const int st = g & 1;
-      if (!mbar_wait(&bars[kVFull + st], parity(g >> 1), abort_flag, a.err)) break;
-      tc_fence_after();
 #pragma unroll
-      for (int k = 0; k < BN / 16; ++k) {
-        const uint64_t bd = smem_desc_sw128(sV + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
-        mma_bf16_ts(tmem + kColO, tmem + kColP + k * 8, bd, kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < DH / 16; ++k) {
+          const uint64_t ad = smem_desc_sw128(sQ + qb * kTileBytes + k * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sK + st * kTileBytes + k * 32, 16, 1024);
+          mma_bf16_ss(tmem + kColS + sb * BN, ad, bd, kIdescS, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars[kSFull + sb]);
+        if (t.j == t.nt - 1) mma_commit(&bars[kQEmpty + qb]);
+        return true;
+      };
+      auto issue_pv = [&](const Cursor& t) -> bool {
+        const int pb = t.g & 1, st = t.g % kStages, ob = t.qi & 1;
+        if (!mbar_wait(&bars[kPFull + pb], par(t.g >> 1), abort_flag, a.err)) return false;
+        if (!mbar_wait(&bars[kVFull + st], par(t.g / kStages), abort_flag, a.err)) return false;
+        if (t.j == 0 && !mbar_wait(&bars[kOEmpty + ob], par(t.qi >> 1) ^ 1u, abort_flag, a.err))
+          return false;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k) {
+          const uint64_t bd =
+              smem_desc_sw128(sV + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
+          mma_bf16_ts(tmem + kColO + ob * DH, tmem + kColP + pb * (BN / 2) + k * 8, bd, kIdescPV,
+                      (t.j > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&bars[kPFree + pb]);
+        mma_commit(&bars[kKVEmpty + st]);
+        if (t.j == t.nt - 1) mma_commit(&bars[kOFull + ob]);
+        return true;
+      };
+      Cursor c{0, 0, 0, tiles(0)};
+      bool ok = c.nt > 0 && issue_s(c);
+      while (ok) {
+        Cursor n = c;
+        ++n.g;
+        if (++n.j == c.nt) {
+          n.j = 0;
+          ++n.qi;
+          n.nt = tiles(n.qi);
+        }
+        const bool more = n.nt > 0;
+        if (more && !issue_s(n)) break;
+        if (!issue_pv(c) || !more) break;
+        c = n;
       }
-      mma_commit(&bars[kPVFull]);
-      mma_commit(&bars[kKVEmpty + st]);
-      ++g;
-      if (w2 < 0) break;
-      if (j2 == 0) ++qi;
-      w = w2;
-      j = j2;
-      it = it2;
+      // every MMA issued has completed before TMEM is freed
+      mma_commit(&bars[kDone]);
+      mbar_drain(&bars[kDone], 0);
     }
-  } else if (warp < 4) {
-    // ---------------------------------------------------------------- softmax warps 0-3
-    const int r = threadIdx.x;  // query row within the tile == TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const float scale_log2 = a.scale * kLog2e;
-    const __nv_bfloat16* Qg = (const __nv_bfloat16*)a.q;
-    const __nv_bfloat16* Kg = (const __nv_bfloat16*)a.k;
-    const __nv_bfloat16* Vg = (const __nv_bfloat16*)a.v;
+    __syncwarp();
+  } else if (warp < 8) {
+    // ---------------------------------------------------------------- softmax warps 0-7
+    const int quad = warp & 3;  // TMEM lane quadrant of the warp
+    const int h = lane >> 4;    // key-column half of each tile
+    const int rt = quad * 32 + (warp >> 2) * 16 + (lane & 15);  // query row within the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32 + (warp >> 2) * 16) << 16);
+    const float* sQCB = reinterpret_cast<const float*>(smem + kOffQCB);
+    const int4* sRec = reinterpret_cast<const int4*>(smem + kOffRec);
     int g = 0;
-    // the next work item's record is loaded one item ahead, and its candidate rows are
-    // warmed in L2, so that an item starts without a dependent global-load chain
-    Item nx = blockIdx.x < total ? load_item(P, blockIdx.x) : Item{};
-    for (int w = blockIdx.x; w < total; w += gridDim.x) {
-      __syncwarp();
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      const Item it = nx;
-      if (w + (int)gridDim.x < total) nx = load_item(P, w + gridDim.x);
-      const int i = it.q0 + r;
-      const bool row = i < it.L;
-      const long long tok = (long long)it.s + i;
-      const bool cand = row && i >= it.n;
-      const float rowcb = row ? P.cbias[(long long)it.h * P.Tp + it.spad + i] : 0.f;
-      // candidate self-term: its score now, its value row kept packed until the epilogue
-      float xs = -INFINITY;
-      uint4 va[DH / 8];
-      if (cand) {
-        const uint4* qp = reinterpret_cast<const uint4*>(Qg + tok * a.tok_stride + it.h * DH);
-        const uint4* kp = reinterpret_cast<const uint4*>(Kg + tok * a.tok_stride + it.h * DH);
-        const uint4* vp = reinterpret_cast<const uint4*>(Vg + tok * a.tok_stride + it.h * DH);
-        uint4 qa[DH / 8], ka[DH / 8];
-#pragma unroll
-        for (int c = 0; c < DH / 8; ++c) {
-          qa[c] = qp[c];
-          ka[c] = kp[c];
-          va[c] = vp[c];
-        }
-        float dot = 0.f;
-#pragma unroll
-        for (int c = 0; c < DH / 8; ++c) {
-          float qf[8], kf[8];
-          Elem<__nv_bfloat16>::unpack(qa[c], qf);
-          Elem<__nv_bfloat16>::unpack(ka[c], kf);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
-        }
-        xs = fmaf(dot, scale_log2, rowcb);
-      }
+    for (int oi = 0;; ++oi) {
+      const int ob = oi & 1;
+      // the item's record and the row's own column term c_i arrive with the Q tile
+      if (!wait_warp(&bars[kQFull + ob], par(oi >> 1), abort_flag, a.err)) break;
+      const int4 rec = sRec[ob];
+      if (rec.w < 0) break;
+      Item it;
+      it.q0 = rec.x;
+      it.n = rec.y;
+      it.L = rec.z;
+      it.nk = rec.w;
+      it.nt = tiles_of(it.q0, it.n, it.L, it.nk);
+      const float rowcb = sQCB[ob * BM + rt];
+      mbar_arrive(&bars[kQEmpty + ob]);
+      const int i = it.q0 + rt;
+      const bool row_ok = i < it.L;
+      const bool cand_row = row_ok && i >= it.n;
       const int lim = min(i, it.n - 1);
       const int mask_from = min(it.q0, it.n - 1);  // a tile needs masks if kv0 + 127 > this
+      const uint32_t o_addr = lane_base + kColO + ob * DH;
       float m = rowcb, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < it.nk; ++j, ++g) {
-        const int st = g & 1;
-        const int kv0 = (it.nk - 1 - j) * BN;  // most recent keys first
-        if (!wait_warp(&bars[kSFull], parity(g), abort_flag, a.err) ||
-            !wait_warp(&bars[kKFull + st], parity(g >> 1), abort_flag, a.err)) {
+      for (int j = 0; j < it.nt; ++j, ++g) {
+        const int sb = g & 1, st = g % kStages;
+        if (!wait_warp(&bars[kSFull + sb], par(g >> 1), abort_flag, a.err) ||
+            !wait_warp(&bars[kKFull + st], par(g / kStages), abort_flag, a.err) ||
+            !wait_warp(&bars[kPFree + sb], par(g >> 1) ^ 1u, abort_flag, a.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const float* cb = sCB + st * BN;
-        const bool masked = kv0 + BN - 1 > mask_from;
-        const int nvalid = masked ? max(0, min(BN, lim - kv0 + 1)) : BN;
-        ok = masked ? softmax_tile<true>(tmem + lane_base, cb, nvalid, scale_log2, j == 0, m, l,
-                                         &bars[kPVFull], g, abort_flag, a.err)
-                    : softmax_tile<false>(tmem + lane_base, cb, nvalid, scale_log2, j == 0, m, l,
-                                          &bars[kPVFull], g, abort_flag, a.err);
+        const uint32_t s_addr = lane_base + kColS + sb * BN;
+        const uint32_t p_addr = lane_base + kColP + sb * (BN / 2);
+        uint64_t* prev_pv = &bars[kPFree + ((g + 1) & 1)];
+        const uint32_t prev_ph = par((g - 1) >> 1);
+        if (j < it.nk) {
+          const int kv0 = (it.nk - 1 - j) * BN;  // most recent keys first
+          const bool masked = kv0 + BN - 1 > mask_from;
+          const int nvalid = masked ? max(0, min(BN, lim - kv0 + 1)) : BN;
+          const float* cb = sCB + st * BN + kHalf * h;
+          ok = masked ? softmax_tile<true>(s_addr, p_addr, o_addr, cb, kHalf * h, nvalid,
+                                           scale_log2, j == 0, row_ok, m, l, prev_pv, prev_ph,
+                                           abort_flag, a.err)
+                      : softmax_tile<false>(s_addr, p_addr, o_addr, cb, kHalf * h, nvalid,
+                                            scale_log2, j == 0, row_ok, m, l, prev_pv, prev_ph,
+                                            abort_flag, a.err);
+        } else {
+          ok = softmax_diag(s_addr, p_addr, o_addr, rt, h, cand_row, rowcb, scale_log2, j == 0,
+                            m, l, prev_pv, prev_ph, abort_flag, a.err);
+        }
         if (!ok) break;
         tc_fence_before();
-        mbar_arrive(&bars[kPFull]);
+        mbar_arrive(&bars[kSFree + sb]);
+        mbar_arrive(&bars[kPFull + sb]);
       }
       if (!ok) break;
-      {  // warm L2 for the next item's candidate rows while this item's P V finishes
-        const int ni = nx.q0 + r;
-        if (w + (int)gridDim.x < total && ni < nx.L && ni >= nx.n) {
-          const long long nt = (long long)nx.s + ni;
-          prefetch_l2(Qg + nt * a.tok_stride + nx.h * DH);
-          prefetch_l2(Kg + nt * a.tok_stride + nx.h * DH);
-          prefetch_l2(Vg + nt * a.tok_stride + nx.h * DH);
-        }
-      }
+      // hand the row's softmax state to the epilogue with the O buffer
+      const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      if (!wait_warp(&bars[kOEmpty + ob], par(oi >> 1) ^ 1u, abort_flag, a.err)) break;
+      if (h == 0) sML[ob * BM + rt] = make_float2(m - rowcb, l_row);
+      mbar_arrive(&bars[kOFull + ob]);
+    }
+  } else if (warp < 12) {
+    // ---------------------------------------------------------------- epilogue warps 8-11
+    const int ew = warp & 3;          // TMEM lane quadrant of the warp
+    const int r = ew * 32 + lane;     // query row within the tile == TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(ew * 32) << 16);
+    __nv_bfloat16* Og = (__nv_bfloat16*)a.o;
+    uint8_t* stage = smem + kOffStage + ew * 32 * (DH * 2);  // this warp's 32 rows
+    int oi = 0;
+    Item nx = blockIdx.x < total ? load_item(P, blockIdx.x) : Item{};
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+      const Item it = nx;
+      if (w + (int)gridDim.x < total) nx = load_item(P, w + gridDim.x);
+      if (it.nt == 0) continue;
+      const int ob = oi & 1;
+      if (!wait_warp(&bars[kOFull + ob], par(oi >> 1), abort_flag, a.err)) break;
+      tc_fence_after();
+      const float2 ml = sML[ob * BM + r];
       float o[DH];
-      if (it.nk > 0) {
-        if (!wait_warp(&bars[kPVFull], parity(g - 1), abort_flag, a.err)) break;
-        tc_fence_after();
-        tmem_ld64(tmem + lane_base + kColO, o);
-        tc_fence_before();
-      } else {
+      tmem_ld64(lane_base + kColO + ob * DH, o);
+      tc_fence_before();
+      mbar_arrive(&bars[kOEmpty + ob]);
+      ++oi;
+      // normalise and stage the row (16-byte chunks XOR-swizzled by row), then write
+      // the warp's 32 rows as whole 128-byte lines
+      const float inv = 1.f / ml.y;
 #pragma unroll
-        for (int c = 0; c < DH; ++c) o[c] = 0.f;
-        m = xs;  // nothing visible but the candidate itself
-      }
-      if (!row) continue;
-      if (cand) {
-        const float m_new = fmaxf(m, xs);
-        const float al = ex2(m - m_new), p = ex2(xs - m_new);
-        l = l * al + p;
-#pragma unroll
-        for (int c = 0; c < DH / 8; ++c) {
-          float vf[8];
-          Elem<__nv_bfloat16>::unpack(va[c], vf);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) o[c * 8 + e] = fmaf(o[c * 8 + e], al, p * vf[e]);
-        }
-        m = m_new;
-      }
-      const float inv = 1.f / l;
-      uint4* op = reinterpret_cast<uint4*>((__nv_bfloat16*)a.o + tok * a.o_stride + it.h * DH);
-#pragma unroll
-      for (int c = 0; c < DH; c += 8) {
+      for (int c = 0; c < DH / 8; ++c) {
         float f[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = o[c + e] * inv;
-        op[c / 8] = Elem<__nv_bfloat16>::pack(f);
+        for (int e = 0; e < 8; ++e) f[e] = o[c * 8 + e] * inv;
+        *reinterpret_cast<uint4*>(stage + lane * (DH * 2) + ((c ^ (lane & 7)) * 16)) =
+            Elem<__nv_bfloat16>::pack(f);
       }
-      if (a.lse) a.lse[(long long)it.h * a.T + tok] = (m + __log2f(l) - rowcb) * kLn2;
+      __syncwarp();
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int rr = k * 4 + (lane >> 3), c = lane & 7;
+        const int ii = it.q0 + ew * 32 + rr;
+        if (ii < it.L) {
+          const uint4 v =
+              *reinterpret_cast<const uint4*>(stage + rr * (DH * 2) + ((c ^ (rr & 7)) * 16));
+          *reinterpret_cast<uint4*>(Og + ((long long)it.s + ii) * a.o_stride + it.h * DH + c * 8) =
+              v;
+        }
+      }
+      __syncwarp();
+      const int i = it.q0 + r;
+      if (i < it.L && a.lse)
+        a.lse[(long long)it.h * a.T + it.s + i] = (ml.x + __log2f(ml.y)) * kLn2;
     }
   }
 
@@ -585,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_fwd_tc(const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 13) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -662,7 +776,7 @@ int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  k_attn_fwd_tc<<<2 * sms, kThreads, kSmemBytes, st>>>(p);
+  k_attn_fwd_tc<<<sms, kThreads, kSmemBytes, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
 }
 

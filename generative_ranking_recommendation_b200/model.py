@@ -144,14 +144,22 @@ class GenRankModel:
     def forward(self, db: DeviceBatch, attn_events=None) -> torch.Tensor:
         """Candidate logits (fp32 [sum m]) for one batch.
 
-        ``attn_events``: optional list; a (start, end) pair of CUDA events recorded
-        on the current stream around each attention launch is appended to it.
+        Every layer's attention runs over all tokens (history rows feed the next
+        layer's keys and values).  After the last attention only candidate rows
+        reach the head, so the last output projection, residual, FFN and final norm
+        run on candidate rows alone.  ``attn_events``: optional list; a (start, end)
+        pair of CUDA events recorded on the current stream around each attention
+        launch is appended to it.
         """
         E, (pos, _, _) = self.embed(db)
         ffn = self.cfg.ffn
-        x = E.float()
-        for W in self.layers:
-            a = (self.rms(x) if ffn else x).to(self.dtype)
+        nl = len(self.layers)
+        x = E.float() if (ffn or nl > 1) else None  # fp32 residual stream where needed
+        for li, W in enumerate(self.layers):
+            if ffn:
+                a = self.rms(x).to(self.dtype)
+            else:
+                a = E if li == 0 else x.to(self.dtype)
             qkv = a @ W["Wqkv"]
             if attn_events is not None:
                 ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -160,13 +168,20 @@ class GenRankModel:
             if attn_events is not None:
                 ev[1].record()
                 attn_events.append(ev)
+            if li == nl - 1:
+                rows = db.cand_rows
+                base = x.index_select(0, rows) if x is not None else E.index_select(0, rows).float()
+                h = base + (o.index_select(0, rows) @ W["Wo"]).float()
+                if ffn:
+                    f = self.rms(h).to(self.dtype)
+                    h = h + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"]).float()
+                    h = self.rms(h)
+                return h @ self.w_head
             x = x + (o @ W["Wo"]).float()
             if ffn:
                 f = self.rms(x).to(self.dtype)
                 x = x + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"]).float()
-        if ffn:
-            x = self.rms(x)
-        return x.index_select(0, db.cand_rows) @ self.w_head
+        raise ValueError("a model needs at least one layer")
 
     # -------------------------------------------------------------------------------------
     def train_step(self, db: DeviceBatch):
@@ -192,18 +207,26 @@ class GenRankModel:
                 return model.attention_bwd(db, qkv, pos, o, lse, do)
 
         ffn = self.cfg.ffn
+        nl = len(self.layers)
         x = Eg.float()
-        for W in self.layers:
+        z = None
+        for li, W in enumerate(self.layers):
             a = (self.rms(x) if ffn else x).to(self.dtype)
             qkv = a @ W["Wqkv"]
             o = _Attn.apply(qkv)
+            if li == nl - 1:  # only candidate rows reach the loss
+                rows = db.cand_rows
+                h = x.index_select(0, rows) + (o.index_select(0, rows) @ W["Wo"]).float()
+                if ffn:
+                    f = self.rms(h).to(self.dtype)
+                    h = h + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"]).float()
+                    h = self.rms(h)
+                z = h @ self.w_head
+                break
             x = x + (o @ W["Wo"]).float()
             if ffn:
                 f = self.rms(x).to(self.dtype)
                 x = x + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"]).float()
-        if ffn:
-            x = self.rms(x)
-        z = x.index_select(0, db.cand_rows) @ self.w_head
         loss = torch.nn.functional.binary_cross_entropy_with_logits(z, db.labels)
         loss.backward()
         dE = Eg.grad.to(self.dtype).contiguous()

@@ -45,7 +45,7 @@ constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
 constexpr int DH = 64;   // head dim
 constexpr int kThreads = 448;  // warps 0-7 softmax, 8-11 epilogue, 12 TMA, 13 MMA
-constexpr int kSoftmaxThreads = 256;
+constexpr int kSoftmaxWarps = 8;  // barrier arrivals are one per warp
 constexpr int kStages = 5;     // K/V ring
 constexpr uint32_t kTileBytes = BM * DH * 2;  // one Q, K or V tile (16 KB)
 constexpr uint32_t kCBBytes = BN * 4;         // column terms of one key tile
@@ -132,11 +132,45 @@ __host__ __device__ inline long long scratch_tp(long long T, int B) {
 // ------------------------------------------------------------------------------------------
 // prologue: work records (block B) and column terms (blocks 0..B-1)
 // ------------------------------------------------------------------------------------------
-constexpr int kMaxNkBuckets = 257;
+constexpr int kMaxTileBuckets = 257;
+constexpr int kSchedThreads = 256;
 
-__global__ void __launch_bounds__(256) k_prologue(const __grid_constant__ AttnArgs a,
-                                                  int max_tiles, int4* recs, int32_t* count,
-                                                  float* cbias, long long Tp) {
+// Exclusive prefix sum over the block's kSchedThreads values; returns the total.
+GR_DEVICE int block_exclusive_scan(int v, int* excl, int* warp_sums) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int w = lane < kSchedThreads / 32 ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kSchedThreads / 32) warp_sums[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  *excl = x - v + (wid > 0 ? warp_sums[wid - 1] : 0);
+  const int total = warp_sums[kSchedThreads / 32 - 1];
+  __syncthreads();
+  return total;
+}
+
+// Work records go out user by user, users with the most query tiles first and each
+// user's query tiles with the most key tiles first: the persistent grid takes
+// consecutive records (times H heads) at the same time, so the items of one user and
+// head run side by side and share their K/V tiles in L2, while the short users fill
+// the tail.
+__global__ void __launch_bounds__(kSchedThreads) k_prologue(const __grid_constant__ AttnArgs a,
+                                                            int max_tiles, int4* recs,
+                                                            int32_t* count, int32_t* uorder,
+                                                            float* cbias, long long Tp) {
   const int b = blockIdx.x;
   if (b < a.B) {
     const long long s = a.off[b], e = a.off[b + 1];
@@ -152,47 +186,58 @@ __global__ void __launch_bounds__(256) k_prologue(const __grid_constant__ AttnAr
     }
     return;
   }
-  // schedule: histogram of visited key tiles, then a scatter longest first
-  __shared__ int hist[kMaxNkBuckets];
-  __shared__ int cursor[kMaxNkBuckets];
-  for (int i = threadIdx.x; i < kMaxNkBuckets; i += blockDim.x) hist[i] = 0;
+  __shared__ int hist[kMaxTileBuckets];
+  __shared__ int warp_sums[kSchedThreads / 32];
+  for (int i = threadIdx.x; i < kMaxTileBuckets; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  for (int pass = 0; pass < 2; ++pass) {
-    for (int u = threadIdx.x; u < a.B; u += blockDim.x) {
-      const long long s = a.off[u], e = a.off[u + 1];
-      if (s < 0 || e < s || e > a.T) {
-        if (pass == 0) flag(a.err, GENRANK_DERR_LAYOUT);
-        continue;
-      }
-      const int L = (int)(e - s);
-      const int n = max(0, min(a.hist_len[u], L));
-      const int tiles_all = (L + BM - 1) / BM;
-      if (pass == 0 && tiles_all > max_tiles) flag(a.err, GENRANK_DERR_LAYOUT);
-      const int tiles = min(tiles_all, max_tiles);
-      for (int t = 0; t < tiles; ++t) {
-        const int kmax = min(t * BM + BM, n);
-        const int nk = kmax > 0 ? (kmax + BN - 1) / BN : 0;
-        const int bucket = min(nk, kMaxNkBuckets - 1);
-        if (pass == 0) {
-          atomicAdd(&hist[bucket], 1);
-        } else {
-          const int slot = atomicAdd(&cursor[bucket], 1);
-          recs[2 * slot] = make_int4((int)s, L, n, t * BM);
-          recs[2 * slot + 1] = make_int4(nk, (int)seg_start(s, u), u, 0);
-        }
-      }
+  auto tiles_of_user = [&](int u, bool check) -> int {
+    const long long s = a.off[u], e = a.off[u + 1];
+    if (s < 0 || e < s || e > a.T) {
+      if (check) flag(a.err, GENRANK_DERR_LAYOUT);
+      return 0;
     }
-    __syncthreads();
-    if (pass == 0 && threadIdx.x == 0) {
-      int acc = 0;
-      for (int q = kMaxNkBuckets - 1; q >= 0; --q) {
-        cursor[q] = acc;
-        acc += hist[q];
-      }
-      *count = acc;
+    const int tiles_all = (int)((e - s + BM - 1) / BM);
+    if (check && tiles_all > max_tiles) flag(a.err, GENRANK_DERR_LAYOUT);
+    return min(tiles_all, max_tiles);
+  };
+  // users bucketed by query tiles, longest first
+  for (int u = threadIdx.x; u < a.B; u += blockDim.x)
+    atomicAdd(&hist[min(tiles_of_user(u, true), kMaxTileBuckets - 1)], 1);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int q = kMaxTileBuckets - 1; q >= 0; --q) {
+      const int c = hist[q];
+      hist[q] = acc;
+      acc += c;
     }
-    __syncthreads();
   }
+  __syncthreads();
+  for (int u = threadIdx.x; u < a.B; u += blockDim.x)
+    uorder[atomicAdd(&hist[min(tiles_of_user(u, false), kMaxTileBuckets - 1)], 1)] = u;
+  __syncthreads();
+  // record slots: prefix sum of the ordered users' tile counts, a chunk per thread
+  const int chunk = (a.B + kSchedThreads - 1) / kSchedThreads;
+  const int k0 = min(a.B, (int)threadIdx.x * chunk), k1 = min(a.B, k0 + chunk);
+  int mine = 0;
+  for (int k = k0; k < k1; ++k) mine += tiles_of_user(uorder[k], false);
+  int slot = 0;
+  const int total = block_exclusive_scan(mine, &slot, warp_sums);
+  for (int k = k0; k < k1; ++k) {
+    const int u = uorder[k];
+    const int tiles = tiles_of_user(u, false);
+    if (tiles == 0) continue;
+    const int s = a.off[u];
+    const int L = a.off[u + 1] - s;
+    const int n = max(0, min(a.hist_len[u], L));
+    for (int t = tiles - 1; t >= 0; --t, ++slot) {
+      const int kmax = min(t * BM + BM, n);
+      const int nk = kmax > 0 ? (kmax + BN - 1) / BN : 0;
+      recs[2 * slot] = make_int4(s, L, n, t * BM);
+      recs[2 * slot + 1] = make_int4(nk, (int)seg_start(s, u), u, 0);
+    }
+  }
+  if (threadIdx.x == 0) *count = total;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -407,13 +452,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
   if (threadIdx.x == 0) {
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars[kQFull + b], 1);
-      mbar_init(&bars[kQEmpty + b], 1 + kSoftmaxThreads);  // last S commit + c_i reads
+      mbar_init(&bars[kQEmpty + b], 1 + kSoftmaxWarps);  // last S commit + c_i reads
       mbar_init(&bars[kSFull + b], 1);
-      mbar_init(&bars[kSFree + b], kSoftmaxThreads);
-      mbar_init(&bars[kPFull + b], kSoftmaxThreads);
+      mbar_init(&bars[kSFree + b], kSoftmaxWarps);
+      mbar_init(&bars[kPFull + b], kSoftmaxWarps);
       mbar_init(&bars[kPFree + b], 1);
-      mbar_init(&bars[kOFull + b], 1 + kSoftmaxThreads);  // last P V commit + (m, l)
-      mbar_init(&bars[kOEmpty + b], 128);
+      mbar_init(&bars[kOFull + b], 1 + kSoftmaxWarps);  // last P V commit + (m, l)
+      mbar_init(&bars[kOEmpty + b], 4);
     }
     for (int st = 0; st < kStages; ++st) {
       mbar_init(&bars[kKFull + st], 1);
@@ -593,7 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       it.nk = rec.w;
       it.nt = tiles_of(it.q0, it.n, it.L, it.nk);
       const float rowcb = sQCB[ob * BM + rt];
-      mbar_arrive(&bars[kQEmpty + ob]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kQEmpty + ob]);
       const int i = it.q0 + rt;
       const bool row_ok = i < it.L;
       const bool cand_row = row_ok && i >= it.n;
@@ -632,15 +678,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
         }
         if (!ok) break;
         tc_fence_before();
-        mbar_arrive(&bars[kSFree + sb]);
-        mbar_arrive(&bars[kPFull + sb]);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars[kSFree + sb]);
+          mbar_arrive(&bars[kPFull + sb]);
+        }
       }
       if (!ok) break;
       // hand the row's softmax state to the epilogue with the O buffer
       const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
       if (!wait_warp(&bars[kOEmpty + ob], par(oi >> 1) ^ 1u, abort_flag, a.err)) break;
       if (h == 0) sML[ob * BM + rt] = make_float2(m - rowcb, l_row);
-      mbar_arrive(&bars[kOFull + ob]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kOFull + ob]);
     }
   } else if (warp < 12) {
     // ---------------------------------------------------------------- epilogue warps 8-11
@@ -663,7 +713,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       float o[DH];
       tmem_ld64(lane_base + kColO + ob * DH, o);
       tc_fence_before();
-      mbar_arrive(&bars[kOEmpty + ob]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kOEmpty + ob]);
       ++oi;
       // normalise and stage the row (16-byte chunks XOR-swizzled by row), then write
       // the warp's 32 rows as whole 128-byte lines
@@ -737,12 +788,14 @@ static int max_tiles_of(int max_seqlen) { return (max_seqlen + BM - 1) / BM; }
 static size_t recs_bytes(int B, int max_seqlen) {
   return ((size_t)B * max_tiles_of(max_seqlen) * kRecInts * 4 + 15) / 16 * 16;
 }
+static size_t users_bytes(int B) { return ((size_t)B * 4 + 15) / 16 * 16; }
 
 }  // namespace tc
 
 size_t attn_fwd_tc_workspace(int B, long long T, int H, int max_seqlen) {
   using namespace tc;
-  return kHeaderBytes + recs_bytes(B, max_seqlen) + (size_t)H * scratch_tp(T, B) * sizeof(float);
+  return kHeaderBytes + recs_bytes(B, max_seqlen) + users_bytes(B) +
+         (size_t)H * scratch_tp(T, B) * sizeof(float);
 }
 
 int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
@@ -759,12 +812,13 @@ int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
   uint8_t* ws = (uint8_t*)a.ws;
   int32_t* count = (int32_t*)ws;
   int4* recs = (int4*)(ws + kHeaderBytes);
-  float* cbias = (float*)(ws + kHeaderBytes + recs_bytes(a.B, a.max_seqlen));
+  int32_t* uorder = (int32_t*)(ws + kHeaderBytes + recs_bytes(a.B, a.max_seqlen));
+  float* cbias = (float*)((uint8_t*)uorder + users_bytes(a.B));
   p.count = count;
   p.recs = recs;
   p.cbias = cbias;
   p.Tp = scratch_tp(a.T, a.B);
-  k_prologue<<<a.B + 1, 256, 0, st>>>(a, max_tiles, recs, count, cbias, p.Tp);
+  k_prologue<<<a.B + 1, kSchedThreads, 0, st>>>(a, max_tiles, recs, count, uorder, cbias, p.Tp);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   static bool attr = false;
   if (!attr) {

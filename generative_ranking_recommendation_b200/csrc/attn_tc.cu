@@ -279,23 +279,31 @@ GR_DEVICE void row_max_chunk(const uint32_t (&s)[CW], const float* cb, int kc0, 
   }
 }
 
-// p = 2^(x - m) for CW columns, summed into four partial sums, packed to bf16 pairs
-// and stored (without waiting) to CW / 2 TMEM columns at taddr.
+// p = 2^(x - m) for CW columns, summed into two pairs of partial sums, packed to
+// bf16 pairs and stored (without waiting) to CW / 2 TMEM columns at taddr.  The
+// bias and scale arithmetic runs on column pairs (two-wide fp32 instructions).
 template <bool kMasked>
 GR_DEVICE void exp_pack_store(const uint32_t (&s)[CW], const float* cb, int kc0, int nvalid,
-                              float scale_log2, float m_use, float (&rs4)[4], uint32_t taddr) {
+                              float scale_log2, float m_use, uint64_t (&rs2)[2], uint32_t taddr) {
+  const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
+  const uint64_t m2 = f2_pack(m_use, m_use);
   uint32_t pk[CW / 2];
 #pragma unroll
   for (int c = 0; c < CW; c += 4) {
     const float4 b4 = *reinterpret_cast<const float4*>(cb + c);
-    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
-    float p[4];
+    const uint64_t t01 = f2_sub(f2_pack(b4.x, b4.y), m2);
+    const uint64_t t23 = f2_sub(f2_pack(b4.z, b4.w), m2);
+    const uint64_t v01 =
+        f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2, t01);
+    const uint64_t v23 =
+        f2_fma(f2_pack(__uint_as_float(s[c + 2]), __uint_as_float(s[c + 3])), sl2, t23);
+    float v[4], p[4];
+    f2_unpack(v01, v[0], v[1]);
+    f2_unpack(v23, v[2], v[3]);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float v = fmaf(__uint_as_float(s[c + e]), scale_log2, bb[e] - m_use);
-      p[e] = (!kMasked || kc0 + c + e < nvalid) ? ex2(v) : 0.f;
-      rs4[e] += p[e];
-    }
+    for (int e = 0; e < 4; ++e) p[e] = (!kMasked || kc0 + c + e < nvalid) ? ex2(v[e]) : 0.f;
+    rs2[0] = f2_add(rs2[0], f2_pack(p[0], p[1]));
+    rs2[1] = f2_add(rs2[1], f2_pack(p[2], p[3]));
     pk[c / 2] = pack_bf16(p[0], p[1]);
     pk[c / 2 + 1] = pack_bf16(p[2], p[3]);
   }
@@ -329,22 +337,25 @@ GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, int kbase, int nvalid
 template <bool kMasked>
 GR_DEVICE float tile_exp(uint32_t s_addr, uint32_t p_addr, const float* cb, int kbase,
                          int nvalid, float scale_log2, float m) {
-  float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+  uint64_t rs2[2] = {0ull, 0ull};  // (+0, +0) pairs
   uint32_t xa[CW], xb[CW];
   s_load(s_addr, xa);
   tmem_ld_wait(xa);
 #pragma unroll
   for (int c0 = 0; c0 < kHalf; c0 += 2 * CW) {
     s_load(s_addr + c0 + CW, xb);
-    exp_pack_store<kMasked>(xa, cb + c0, kbase + c0, nvalid, scale_log2, m, rs4, p_addr + c0 / 2);
+    exp_pack_store<kMasked>(xa, cb + c0, kbase + c0, nvalid, scale_log2, m, rs2, p_addr + c0 / 2);
     tmem_ld_wait(xb);
     if (c0 + 2 * CW < kHalf) s_load(s_addr + c0 + 2 * CW, xa);
-    exp_pack_store<kMasked>(xb, cb + c0 + CW, kbase + c0 + CW, nvalid, scale_log2, m, rs4,
+    exp_pack_store<kMasked>(xb, cb + c0 + CW, kbase + c0 + CW, nvalid, scale_log2, m, rs2,
                             p_addr + (c0 + CW) / 2);
     if (c0 + 2 * CW < kHalf) tmem_ld_wait(xa);
   }
   tmem_wait_st();
-  return (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+  float r0, r1, r2, r3;
+  f2_unpack(rs2[0], r0, r1);
+  f2_unpack(rs2[1], r2, r3);
+  return (r0 + r1) + (r2 + r3);
 }
 
 // O (this thread's 32 columns of its row) *= alpha, once the previous P V has landed.

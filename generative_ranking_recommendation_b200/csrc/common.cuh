@@ -36,6 +36,31 @@ GR_DEVICE uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
+// Packed pairs of fp32 (one 64-bit register pair) and the sm_100 two-wide fp32 ops.
+GR_DEVICE uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+GR_DEVICE void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+GR_DEVICE uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+GR_DEVICE uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+GR_DEVICE uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 GR_DEVICE float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 GR_DEVICE float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 

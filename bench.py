@@ -363,7 +363,10 @@ def run_native(args, cfg, world, rank, local):
                      "avg_launch_ms": attn_avg_ms},
         "e2e": {"value": cands_per_step / (e2e_ms / args.steps / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": 4 * args.steps * cfg.layers,
+        # per step: metadata scan + gather-sum, attention prologue + kernel per layer,
+        # and the fused candidate head of a one-block model without FFN
+        "gpu_launches": args.steps * (2 + 2 * cfg.layers
+                                      + (0 if (cfg.ffn or cfg.layers > 1) else 1)),
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

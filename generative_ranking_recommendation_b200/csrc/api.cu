@@ -163,6 +163,36 @@ int genrank_embed_assemble_bwd(int B, int64_t T, const int32_t* seq_offsets,
   return launch_embed_bwd(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int genrank_candidate_logits(int M, const int64_t* rows, int64_t T, int d, const void* x,
+                             int64_t x_stride, const void* o, int64_t o_stride, int dtype,
+                             const float* w, const float* u, float* z, int32_t* dev_err,
+                             genrank_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (M < 0 || T < 0 || d < 1 || !es || !dev_err) return GENRANK_ERR_INVALID_ARG;
+  if (M == 0) return GENRANK_OK;
+  if (!rows || !x || !o || !w || !u || !z) return GENRANK_ERR_INVALID_ARG;
+  if (x_stride < d || o_stride < d || (d * es) % 16 || (x_stride * es) % 16 ||
+      (o_stride * es) % 16)
+    return GENRANK_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(o) || !aligned16(w) || !aligned16(u))
+    return GENRANK_ERR_INVALID_ARG;
+  CandLogitsArgs a;
+  a.M = M;
+  a.rows = rows;
+  a.T = T;
+  a.d = d;
+  a.x = x;
+  a.x_stride = x_stride;
+  a.o = o;
+  a.o_stride = o_stride;
+  a.dtype = dtype;
+  a.w = w;
+  a.u = u;
+  a.z = z;
+  a.err = dev_err;
+  return launch_cand_logits(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t genrank_attn_workspace_size(int B, int64_t T, int H, int dh, int max_seqlen, int is_bwd) {
   if (B < 1 || T < 0 || H < 1 || dh < 1 || max_seqlen < 0) return 0;
   if (is_bwd) {

@@ -21,7 +21,8 @@ ROOT = os.path.dirname(PKG)
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgenrank.so")
-SOURCES = ["api.cu", "embed.cu", "attn_simt.cu", "attn_tc.cu", "attn_bwd_tc.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "embed.cu", "attn_simt.cu", "attn_tc.cu", "attn_bwd_tc.cu", "noalloc.cu",
+           "head.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

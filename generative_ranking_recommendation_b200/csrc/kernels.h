@@ -95,6 +95,24 @@ struct AttnArgs {
   int32_t* err;
 };
 
+struct CandLogitsArgs {
+  long long M;
+  const int64_t* rows;
+  long long T;
+  int d;
+  const void* x;
+  long long x_stride;  // elements
+  const void* o;
+  long long o_stride;  // elements
+  int dtype;
+  const float* w;
+  const float* u;
+  float* z;
+  int32_t* err;
+};
+
+int launch_cand_logits(const CandLogitsArgs& a, cudaStream_t st);
+
 int launch_embed_fwd(const EmbedFwdArgs& a, cudaStream_t st);
 int launch_embed_bwd(const EmbedBwdArgs& a, cudaStream_t st);
 

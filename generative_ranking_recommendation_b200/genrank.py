@@ -27,7 +27,7 @@ EXPORTS = (
     "genrank_status_string", "genrank_device_error_string", "genrank_check_error",
     "genrank_alibi_slopes", "genrank_embed_assemble", "genrank_embed_assemble_bwd",
     "genrank_attn_fwd", "genrank_attn_bwd", "genrank_attn_workspace_size",
-    "genrank_attn_fwd_static",
+    "genrank_attn_fwd_static", "genrank_candidate_logits",
 )
 
 
@@ -76,6 +76,9 @@ def lib():
         L.genrank_attn_fwd_static.argtypes = [
             _I, _L, _P, _P, _I, _P, _P, _P, _L, _I, _I, _P, _P, _P, _P, _F, _I, _P, _L, _P,
             _P, _P]
+        L.genrank_candidate_logits.restype = _I
+        L.genrank_candidate_logits.argtypes = [
+            _I, _P, _L, _I, _P, _L, _P, _L, _I, _P, _P, _P, _P, _P]
         L.genrank_attn_workspace_size.restype = _Z
         L.genrank_attn_workspace_size.argtypes = [_I, _L, _I, _I, _I, _I]
         _lib = L
@@ -211,3 +214,14 @@ def attn_fwd_static(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, d
         float(scale), _dtype_code(q), _ptr(o), int(o_stride), _ptr(lse), _ptr(dev_err),
         _stream(stream))
     _check(rc, "genrank_attn_fwd_static")
+
+
+def candidate_logits(rows, x, o, w, u, z, dev_err, stream=None):
+    """genrank_candidate_logits: z[c] = x[rows[c]] . w + o[rows[c]] . u (fp32)."""
+    if o.dtype != x.dtype:
+        raise GenRankError("candidate_logits: x and o must share a dtype")
+    rc = lib().genrank_candidate_logits(
+        int(rows.numel()), _ptr(rows), int(x.shape[0]), int(x.shape[1]), _ptr(x),
+        int(x.stride(0)), _ptr(o), int(o.stride(0)), _dtype_code(x), _ptr(w), _ptr(u), _ptr(z),
+        _ptr(dev_err), _stream(stream))
+    _check(rc, "genrank_candidate_logits")

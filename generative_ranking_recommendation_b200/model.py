@@ -6,7 +6,8 @@ around it are torch ops: the fused QKV projection, the output projection and
 residual, pre-RMSNorm (eps 1e-6, unit gain) and the 4d SiLU FFN of the 4-layer
 workloads, the final RMSNorm and the candidate head (a dot with w_head at
 candidate rows only, as the loss lives only at candidate positions:
-"GenRank [2025]" chapter notes §1.3.1).  The residual stream is kept in fp32;
+"GenRank [2025]" chapter notes §1.3.1; for one block without FFN it is the
+library's fused candidate-logits kernel).  The residual stream is kept in fp32;
 projections run in the storage dtype with fp32 accumulation.
 """
 
@@ -95,6 +96,7 @@ class GenRankModel:
         self.scale = 1.0 / math.sqrt(cfg.dh)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self._ws = {}
+        self._head_u = None
 
     # -------------------------------------------------------------------------------------
     def workspace(self, db: DeviceBatch, bwd: bool) -> torch.Tensor:
@@ -135,6 +137,14 @@ class GenRankModel:
                    self.workspace(db, True), self.err, T=db.T)
         return dqkv
 
+    def head_u(self, W) -> torch.Tensor:
+        """u = W_o w_head (fp32 [d]) for the fused candidate head, recomputed when W_o
+        changes in place."""
+        key = (W["Wo"].data_ptr(), W["Wo"]._version)
+        if self._head_u is None or self._head_u[0] != key:
+            self._head_u = (key, (W["Wo"].float() @ self.w_head).contiguous())
+        return self._head_u[1]
+
     @staticmethod
     def rms(x):
         return x * torch.rsqrt((x * x).mean(dim=-1, keepdim=True) + RMS_EPS)
@@ -147,7 +157,9 @@ class GenRankModel:
         Every layer's attention runs over all tokens (history rows feed the next
         layer's keys and values).  After the last attention only candidate rows
         reach the head, so the last output projection, residual, FFN and final norm
-        run on candidate rows alone.  ``attn_events``: optional list; a (start, end)
+        run on candidate rows alone; with one block and no FFN the head is one fused
+        kernel, z = E . w_head + o . (W_o w_head) at candidate rows (the same sum
+        regrouped).  ``attn_events``: optional list; a (start, end)
         pair of CUDA events recorded on the current stream around each attention
         launch is appended to it.
         """
@@ -168,9 +180,15 @@ class GenRankModel:
             if attn_events is not None:
                 ev[1].record()
                 attn_events.append(ev)
+            if li == nl - 1 and x is None:
+                # one block, no FFN: z = E . w_head + o . (W_o w_head) at candidate rows,
+                # one fused gather-dot kernel
+                z = torch.empty(db.cand_rows.numel(), dtype=torch.float32, device=self.device)
+                G.candidate_logits(db.cand_rows, E, o, self.w_head, self.head_u(W), z, self.err)
+                return z
             if li == nl - 1:
                 rows = db.cand_rows
-                base = x.index_select(0, rows) if x is not None else E.index_select(0, rows).float()
+                base = x.index_select(0, rows)
                 h = base + (o.index_select(0, rows) @ W["Wo"]).float()
                 if ffn:
                     f = self.rms(h).to(self.dtype)

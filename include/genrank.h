@@ -210,6 +210,25 @@ int genrank_attn_fwd_static(int B, int64_t T, const int32_t *seq_offsets, const 
                             float scale, int dtype, void *o, int64_t o_stride, float *lse,
                             int32_t *dev_err, genrank_stream_t stream);
 
+/* Candidate logits of a one-block scorer without FFN: the score is read at
+ * candidate positions only (huaxiaozhuan "GenRank [2025]" §1.3.1: the loss and
+ * the ranking output live at candidate positions), and for
+ *   h = x + attn W_o,   z = h . w_head
+ * the logit is z = x . w_head + attn . u with u = W_o w_head (a d-vector the
+ * caller forms once per weights), so the candidate rows are read once and no
+ * [m, d] intermediate is formed:
+ *   z[c] = sum_j x[rows[c], j] w[j] + sum_j o[rows[c], j] u[j]   (fp32 accumulation)
+ * Arguments:
+ *   M            number of candidates (>= 0); rows [M] int64 token rows in [0, T)
+ *   x, o         [T, d] row-major in dtype with row strides x_stride, o_stride
+ *                (elements); 16-byte aligned rows (d, strides: multiples of 16 bytes)
+ *   w, u         [d] fp32, 16-byte aligned; z [M] fp32 output
+ * A row outside [0, T) sets GENRANK_DERR_INDEX and gives z[c] = 0. */
+int genrank_candidate_logits(int M, const int64_t *rows, int64_t T, int d, const void *x,
+                             int64_t x_stride, const void *o, int64_t o_stride, int dtype,
+                             const float *w, const float *u, float *z, int32_t *dev_err,
+                             genrank_stream_t stream);
+
 /* Bytes of workspace genrank_attn_fwd (is_bwd = 0) or genrank_attn_bwd
  * (is_bwd = 1) need for these sizes.  Returns 0 for invalid sizes. */
 size_t genrank_attn_workspace_size(int B, int64_t T, int H, int dh, int max_seqlen, int is_bwd);

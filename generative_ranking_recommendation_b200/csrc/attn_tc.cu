@@ -17,19 +17,19 @@
 //     rows: the history only; most recent keys first) and, when it holds candidate
 //     rows, one diagonal tile: its own rows as keys, of which only each candidate's
 //     own key (bias 0) is kept.  Key tiles a query tile never sees are never visited.
-//   * Warp 12 issues TMA loads (Q with the rows' own column terms, double-buffered;
+//   * Warp 1 issues TMA loads (Q with the rows' own column terms, double-buffered;
 //     K, V and their column terms in a five-stage ring; 128B swizzle, no multicast).
-//   * Warp 13 (one thread) issues tcgen05.mma: S = Q K^T (128 x 128, fp32) into one
+//   * Warp 0 (one thread) issues tcgen05.mma: S = Q K^T (128 x 128, fp32) into one
 //     of two TMEM buffers, the next S before the current P V, and O += P V (128 x 64,
 //     fp32) into the item's TMEM O buffer (two, alternating by item), P (bf16 pairs)
 //     read from one of two TMEM P buffers.
-//   * Warps 0-7 stream the softmax with two threads per query row, each on one half
+//   * Warps 2-9 stream the softmax with two threads per query row, each on one half
 //     of the key columns (TMEM access shape 16x32bx2), so two softmax warps share
 //     each SM sub-partition: bias, mask and exponentials in one pass per tile, with
 //     the offset fixed at the row's own column term (every visible key has
 //     c_j <= c_i); a tile whose row sum leaves the safe range is redone exactly and O
 //     rescaled in TMEM.
-//   * Warps 8-11 (one row per thread) finish each item from its O buffer while the
+//   * Warps 10-13 (one row per thread) finish each item from its O buffer while the
 //     next item runs: O is normalised and written through shared memory as whole
 //     128-byte rows, and the literal LSE is stored.
 #include <cuda.h>
@@ -44,7 +44,7 @@ namespace tc {
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
 constexpr int DH = 64;   // head dim
-constexpr int kThreads = 448;  // warps 0-7 softmax, 8-11 epilogue, 12 TMA, 13 MMA
+constexpr int kThreads = 448;  // warp 0 MMA, 1 TMA, 2-9 softmax, 10-13 epilogue
 constexpr int kSoftmaxWarps = 8;  // barrier arrivals are one per warp
 constexpr int kStages = 5;     // K/V ring
 constexpr uint32_t kTileBytes = BM * DH * 2;  // one Q, K or V tile (16 KB)
@@ -480,12 +480,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 12 && lane == 0) {
+  if (warp == 1 && lane == 0) {
     tma_prefetch_desc(&P.tq);
     tma_prefetch_desc(&P.tk);
     tma_prefetch_desc(&P.tv);
   }
-  if (warp == 13) {
+  if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -496,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
   const int total = *P.count * a.H;
   const float scale_log2 = a.scale * kLog2e;
 
-  if (warp == 12) {
+  if (warp == 1) {
     // ---------------------------------------------------------------- TMA producer
     // Each Q tile travels with the item's record (q0, n, L, nk); a record with nk < 0
     // after the last item tells the MMA and softmax warps to stop.
@@ -559,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       }
       for (int x = max(0, qi - 2); x < qi; ++x) mbar_drain(&bars[kQFull + (x & 1)], par(x >> 1));
     }
-  } else if (warp == 13) {
+  } else if (warp == 0) {
     // ---------------------------------------------------------------- MMA issuer (one thread)
     // Tiles in order g = 0, 1, ...: S_{g+1} = Q K_{g+1}^T goes into the other S buffer
     // before P_g V_g, so the softmax finds each S ready when it finishes the last one.
@@ -627,12 +627,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       mbar_drain(&bars[kDone], 0);
     }
     __syncwarp();
-  } else if (warp < 8) {
-    // ---------------------------------------------------------------- softmax warps 0-7
+  } else if (warp < 10) {
+    // ---------------------------------------------------------------- softmax warps 2-9
     const int quad = warp & 3;  // TMEM lane quadrant of the warp
+    const int rh = (warp - 2) >> 2;  // upper or lower 16 lanes of the quadrant
     const int h = lane >> 4;    // key-column half of each tile
-    const int rt = quad * 32 + (warp >> 2) * 16 + (lane & 15);  // query row within the tile
-    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32 + (warp >> 2) * 16) << 16);
+    const int rt = quad * 32 + rh * 16 + (lane & 15);  // query row within the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32 + rh * 16) << 16);
     const float* sQCB = reinterpret_cast<const float*>(smem + kOffQCB);
     const int4* sRec = reinterpret_cast<const int4*>(smem + kOffRec);
     int g = 0;
@@ -703,8 +704,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kOFull + ob]);
     }
-  } else if (warp < 12) {
-    // ---------------------------------------------------------------- epilogue warps 8-11
+  } else if (warp < 14) {
+    // ---------------------------------------------------------------- epilogue warps 10-13
     const int ew = warp & 3;          // TMEM lane quadrant of the warp
     const int r = ew * 32 + lane;     // query row within the tile == TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(ew * 32) << 16);
@@ -761,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 13) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------------------------------

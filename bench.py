@@ -204,6 +204,23 @@ def dist_setup():
     return world, rank, local
 
 
+def rank_users(B_per_rank: int, rank: int):
+    """The users rank `rank` scores: its own block of B_per_rank (weak scaling; users
+    are independent, so no data crosses ranks)."""
+    return list(range(rank * B_per_rank, (rank + 1) * B_per_rank))
+
+
+def max_over_ranks(values, world: int, device):
+    """Element-wise max over ranks of a list of floats (the slowest rank's times)."""
+    if world == 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def config_block(cfg, world, extra=None):
     c = {"workload": f"inference scoring ({cfg.name}): {cfg.B} users/GPU, history "
                      f"U[{cfg.hist[1]},{cfg.hist[2]}], {cfg.m} candidates, d={cfg.d} "
@@ -260,7 +277,7 @@ def run_native(args, cfg, world, rank, local):
     if world > 1:
         dist.init_process_group("nccl", device_id=dev)
 
-    users = list(range(rank * cfg.B, (rank + 1) * cfg.B))
+    users = rank_users(cfg.B, rank)
     batches = [make_batch(cfg, users=users, seed=cfg.seed + 1000 * k) for k in range(2)]
     mdl = make_model(cfg)
     gm = GenRankModel(cfg, mdl, dev)
@@ -331,10 +348,8 @@ def run_native(args, cfg, world, rank, local):
     e2e_ms = sum(s.elapsed_time(e) for s, e in ev2)
     assert G.check_error(gm.err) == 0, "device error flags raised during the timed region"
 
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, dev)
     if world > 1:
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
         dist.destroy_process_group()
     if rank != 0:
         return

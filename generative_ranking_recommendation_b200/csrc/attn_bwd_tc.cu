@@ -14,18 +14,22 @@
 //   * One CTA per SM walks the records.  For a history key tile [k0, k0+128) the
 //     visible queries are the user's rows i >= j (later history rows and every
 //     candidate); they are visited one 128-row query tile at a time.
-//   * Warp 4 loads K, V once per record and Q, dO, lse2, D per query tile (TMA,
+//   * Warp 1 loads K, V once per record and Q, dO, lse2, D per query tile (TMA,
 //     128B swizzle, no multicast; bulk copies for the per-row terms).
-//   * Warp 5 (one thread) issues tcgen05.mma: S^T = K Q^T and dP^T = V dO^T into
+//   * Warp 0 (one thread) issues tcgen05.mma: S^T = K Q^T and dP^T = V dO^T into
 //     TMEM; after the softmax warps have written P^T and dS^T (bf16, shared memory,
 //     UMMA 128B-swizzled K-major layout), dV += P^T dO and dK += dS^T Q accumulate in
 //     TMEM, and dQ_part = dS K is formed from the same dS^T buffer read as an
 //     MN-major operand.  The next tile's S^T, dP^T are issued before this tile's
 //     gradient MMAs.
-//   * Warps 0-3 (one key row per thread) compute P^T and dS^T and, per record, move
-//     dK (times scale) and dV from TMEM to global memory.
-//   * Warps 6-9 (one query row per thread) add each dQ_part into an fp32 dQ
-//     accumulator in global memory with vector reductions.
+//   * Warps 2-9 (two threads per key row, each on one half of the query columns,
+//     TMEM access shape 16x32bx2, so two of these warps share each SM
+//     sub-partition) compute P^T and dS^T.
+//   * Warps 10-13 (one query row per thread) add each dQ_part into an fp32 dQ
+//     accumulator in global memory with vector reductions and, per record, move dK
+//     (times scale) and dV from TMEM to global memory.
+//   * K and V are double-buffered by record, so the next record's loads and its
+//     first S^T, dP^T overlap the end of the current one.
 //   * Candidate keys are seen only by their own row; a finishing kernel applies that
 //     self term to dq, dk, dv of candidate tokens and writes dq = scale * dQ_acc.
 // Every mbarrier wait is bounded in time; a timeout sets GENRANK_DERR_TIMEOUT,
@@ -41,22 +45,23 @@ namespace tcb {
 
 constexpr int BM = 128;  // keys per record tile / queries per query tile
 constexpr int DH = 64;
-constexpr int kThreads = 320;  // warps 0-3 softmax, 4 TMA, 5 MMA, 6-9 dQ reduction
+constexpr int kThreads = 448;  // warp 0 MMA, 1 TMA, 2-9 softmax, 10-13 dQ reduction
+constexpr int kSoftmaxWarps = 8;
 constexpr uint32_t kTileBytes = BM * DH * 2;  // 16 KB
 constexpr uint32_t kRowBytes = BM * 4;        // one per-row fp32 vector of a tile
 constexpr uint32_t kPSBytes = BM * BM * 2;    // 32 KB (P^T or dS^T)
 
 // shared memory (offsets from a 1024-byte aligned base)
-constexpr uint32_t kOffK = 0;
-constexpr uint32_t kOffV = kOffK + kTileBytes;
-constexpr uint32_t kOffQ = kOffV + kTileBytes;         // 2 stages
+constexpr uint32_t kOffK = 0;                          // 2 stages (one per record)
+constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;     // 2 stages
+constexpr uint32_t kOffQ = kOffV + 2 * kTileBytes;     // 2 stages
 constexpr uint32_t kOffDO = kOffQ + 2 * kTileBytes;    // 2 stages
 constexpr uint32_t kOffL2 = kOffDO + 2 * kTileBytes;   // lse2, 2 stages
 constexpr uint32_t kOffD = kOffL2 + 2 * kRowBytes;     // D, 2 stages
 constexpr uint32_t kOffP = kOffD + 2 * kRowBytes;      // P^T
 constexpr uint32_t kOffDS = kOffP + kPSBytes;          // dS^T
 constexpr uint32_t kOffBar = kOffDS + kPSBytes;
-constexpr uint32_t kNumBars = 16;
+constexpr uint32_t kNumBars = 18;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
 
@@ -74,8 +79,8 @@ constexpr uint32_t kIdescQ = idesc_bf16_f32(BM, DH, 1, 1);   // dS MN-major; K M
 
 constexpr size_t kHeaderBytes = 256;
 
-enum Bar { kKVFull = 0, kKVEmpty = 1, kQDFull = 2, kQDEmpty = 4, kSFull = 6, kPFull = 7,
-           kPSFree = 8, kDQFull = 9, kDQEmpty = 11 };
+enum Bar { kKVFull = 0, kKVEmpty = 2, kQDFull = 4, kQDEmpty = 6, kSFull = 8, kPFull = 9,
+           kPSFree = 10, kDQFull = 11, kDQEmpty = 13, kDKVFull = 15, kDKVEmpty = 16 };
 
 struct Params {
   CUtensorMap tq, tk, tv, tdo;
@@ -122,8 +127,8 @@ constexpr int kMaxBuckets = 257;
 
 __global__ void __launch_bounds__(256) k_bwd_prologue(const __grid_constant__ AttnArgs a,
                                                       int max_tiles, int4* recs, int32_t* count,
-                                                      float* cbias, float* lse2, float* dsum,
-                                                      long long Tp) {
+                                                      int32_t* uorder, float* cbias,
+                                                      float* lse2, float* dsum, long long Tp) {
   const int b = blockIdx.x;
   if (b < a.B) {
     const long long s = a.off[b], e = a.off[b + 1];
@@ -154,45 +159,76 @@ __global__ void __launch_bounds__(256) k_bwd_prologue(const __grid_constant__ At
     }
     return;
   }
+  // Records go out user by user (users with the most history key tiles first, each
+  // user's key tiles in order, so the most query tiles first): the persistent grid
+  // takes consecutive records (times H heads) together, so one user's records run
+  // side by side and share its Q, dO tiles in L2.
   __shared__ int hist[kMaxBuckets];
-  __shared__ int cursor[kMaxBuckets];
+  __shared__ int warp_sums[8];
   for (int i = threadIdx.x; i < kMaxBuckets; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  for (int pass = 0; pass < 2; ++pass) {
-    for (int u = threadIdx.x; u < a.B; u += blockDim.x) {
-      const long long s = a.off[u], e = a.off[u + 1];
-      if (s < 0 || e < s || e > a.T) {
-        if (pass == 0) flag(a.err, GENRANK_DERR_LAYOUT);
-        continue;
-      }
-      const int L = (int)(e - s);
-      const int n = max(0, min(a.hist_len[u], L));
-      const int qtiles = (L + BM - 1) / BM;
-      if (pass == 0 && qtiles > max_tiles) flag(a.err, GENRANK_DERR_LAYOUT);
-      const int ktiles = min((n + BM - 1) / BM, max_tiles);
-      for (int kt = 0; kt < ktiles; ++kt) {
-        const int nq = min(qtiles, max_tiles) - kt;
-        const int bucket = min(nq, kMaxBuckets - 1);
-        if (pass == 0) {
-          atomicAdd(&hist[bucket], 1);
-        } else {
-          const int slot = atomicAdd(&cursor[bucket], 1);
-          recs[2 * slot] = make_int4((int)s, L, n, kt * BM);
-          recs[2 * slot + 1] = make_int4(nq, (int)seg_start(s, u), u, 0);
-        }
-      }
+  auto tiles_of_user = [&](int u, bool check, int* qtiles_out) -> int {
+    const long long s = a.off[u], e = a.off[u + 1];
+    if (s < 0 || e < s || e > a.T) {
+      if (check) flag(a.err, GENRANK_DERR_LAYOUT);
+      *qtiles_out = 0;
+      return 0;
     }
-    __syncthreads();
-    if (pass == 0 && threadIdx.x == 0) {
-      int acc = 0;
-      for (int q = kMaxBuckets - 1; q >= 0; --q) {
-        cursor[q] = acc;
-        acc += hist[q];
-      }
-      *count = acc;
+    const int L = (int)(e - s);
+    const int n = max(0, min(a.hist_len[u], L));
+    const int qtiles = (L + BM - 1) / BM;
+    if (check && qtiles > max_tiles) flag(a.err, GENRANK_DERR_LAYOUT);
+    *qtiles_out = min(qtiles, max_tiles);
+    return min((n + BM - 1) / BM, max_tiles);
+  };
+  int qt = 0;
+  for (int u = threadIdx.x; u < a.B; u += blockDim.x)
+    atomicAdd(&hist[min(tiles_of_user(u, true, &qt), kMaxBuckets - 1)], 1);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int q = kMaxBuckets - 1; q >= 0; --q) {
+      const int c = hist[q];
+      hist[q] = acc;
+      acc += c;
     }
-    __syncthreads();
   }
+  __syncthreads();
+  for (int u = threadIdx.x; u < a.B; u += blockDim.x)
+    uorder[atomicAdd(&hist[min(tiles_of_user(u, false, &qt), kMaxBuckets - 1)], 1)] = u;
+  __syncthreads();
+  // record slots: exclusive prefix sum of the ordered users' key-tile counts
+  const int chunk = (a.B + 255) / 256;
+  const int k0 = min(a.B, (int)threadIdx.x * chunk), k1 = min(a.B, k0 + chunk);
+  int mine = 0;
+  for (int k = k0; k < k1; ++k) mine += tiles_of_user(uorder[k], false, &qt);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int x = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[wid] = x;
+  __syncthreads();
+  int before = 0, total = 0;
+  for (int q = 0; q < 8; ++q) {
+    if (q < wid) before += warp_sums[q];
+    total += warp_sums[q];
+  }
+  int slot = before + x - mine;
+  for (int k = k0; k < k1; ++k) {
+    const int u = uorder[k];
+    const int ktiles = tiles_of_user(u, false, &qt);
+    const int s = a.off[u];
+    const int L = a.off[u + 1] - s;
+    const int n = max(0, min(a.hist_len[u], L));
+    for (int kt = 0; kt < ktiles; ++kt, ++slot) {
+      recs[2 * slot] = make_int4(s, L, n, kt * BM);
+      recs[2 * slot + 1] = make_int4(qt - kt, (int)seg_start(s, u), u, 0);
+    }
+  }
+  if (threadIdx.x == 0) *count = total;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -205,14 +241,15 @@ GR_DEVICE bool wait_warp(uint64_t* bar, uint32_t par, volatile int* abort_flag, 
   return __all_sync(0xffffffffu, ok);
 }
 
-// Write 32 bf16 values (16 packed words) of row r, keys/queries [c0, c0+32), into a
-// 128-column operand tile laid out as two 64-column blocks of 128-byte rows with
-// 16-byte chunks XOR-swizzled by row (the UMMA 128B-swizzle canonical layout).
-GR_DEVICE void store_row_chunk(uint8_t* tile, int r, int c0, const uint32_t (&pk)[16]) {
+// Write 16 bf16 values (8 packed words) of row r, keys/queries [c0, c0+16) with
+// c0 % 16 == 0, into a 128-column operand tile laid out as two 64-column blocks of
+// 128-byte rows with 16-byte chunks XOR-swizzled by row (the UMMA 128B-swizzle
+// canonical layout).
+GR_DEVICE void store_row_chunk16(uint8_t* tile, int r, int c0, const uint32_t (&pk)[8]) {
   const int blk = c0 >> 6;
   uint8_t* row = tile + blk * (BM * 128) + r * 128;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < 2; ++q) {
     const int cc = ((c0 & 63) >> 3) + q;
     *reinterpret_cast<uint4*>(row + ((cc ^ (r & 7)) << 4)) =
         make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
@@ -230,27 +267,31 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[kKVFull], 1);
-    mbar_init(&bars[kKVEmpty], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[kKVFull + i], 1);
+      mbar_init(&bars[kKVEmpty + i], 1);
+    }
+    mbar_init(&bars[kDKVFull], 1);
+    mbar_init(&bars[kDKVEmpty], 4);  // one arrival per dK/dV-storing warp
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[kQDFull + i], 1);
       mbar_init(&bars[kQDEmpty + i], 1);
       mbar_init(&bars[kDQFull + i], 1);
-      mbar_init(&bars[kDQEmpty + i], 128);
+      mbar_init(&bars[kDQEmpty + i], 4);  // one arrival per reducing warp
     }
     mbar_init(&bars[kSFull], 1);
-    mbar_init(&bars[kPFull], 128);
+    mbar_init(&bars[kPFull], kSoftmaxWarps);
     mbar_init(&bars[kPSFree], 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 1 && lane == 0) {
     tma_prefetch_desc(&P.tq);
     tma_prefetch_desc(&P.tk);
     tma_prefetch_desc(&P.tv);
     tma_prefetch_desc(&P.tdo);
   }
-  if (warp == 5) {
+  if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -260,17 +301,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
   const uint32_t tmem = *tmem_slot;
   const int total = *P.count * a.H;
 
-  if (warp == 4) {
+  if (warp == 1) {
     // ---------------------------------------------------------------- TMA producer
     int it = 0, g = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const Rec rc = load_rec(P, w);
-      if (!wait_warp(&bars[kKVEmpty], parity(it) ^ 1u, abort_flag, a.err)) break;
+      const int kvs = it & 1;
+      if (!wait_warp(&bars[kKVEmpty + kvs], parity(it >> 1) ^ 1u, abort_flag, a.err)) break;
       if (lane == 0) {
-        mbar_expect_tx(&bars[kKVFull], 2 * kTileBytes);
-        tma_load_3d(smem + kOffK, &P.tk, &bars[kKVFull], 0, rc.h, rc.s + rc.k0);
-        tma_load_3d(smem + kOffV, &P.tv, &bars[kKVFull], 0, rc.h, rc.s + rc.k0);
+        mbar_expect_tx(&bars[kKVFull + kvs], 2 * kTileBytes);
+        tma_load_3d(smem + kOffK + kvs * kTileBytes, &P.tk, &bars[kKVFull + kvs], 0, rc.h,
+                    rc.s + rc.k0);
+        tma_load_3d(smem + kOffV + kvs * kTileBytes, &P.tv, &bars[kKVFull + kvs], 0, rc.h,
+                    rc.s + rc.k0);
       }
       const long long roff = (long long)rc.h * P.Tp + rc.spad;
       bool ok = true;
@@ -295,22 +339,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
       }
       if (!ok) break;
     }
-  } else if (warp == 5 && lane == 0) {
+  } else if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- MMA issuer
     const uint32_t sK = smem_u32(smem + kOffK), sV = smem_u32(smem + kOffV),
                    sQ = smem_u32(smem + kOffQ), sDO = smem_u32(smem + kOffDO),
                    sP = smem_u32(smem + kOffP), sDS = smem_u32(smem + kOffDS);
-    auto issue_sdp = [&](int gg) {
+    auto issue_sdp = [&](int gg, int kvs) {
       const int st = gg & 1;
 #pragma unroll
       for (int k = 0; k < DH / 16; ++k) {
-        mma_bf16_ss(tmem + kColS, smem_desc_sw128(sK + k * 32, 16, 1024),
+        mma_bf16_ss(tmem + kColS, smem_desc_sw128(sK + kvs * kTileBytes + k * 32, 16, 1024),
                     smem_desc_sw128(sQ + st * kTileBytes + k * 32, 16, 1024), kIdescS,
                     k > 0 ? 1u : 0u);
       }
 #pragma unroll
       for (int k = 0; k < DH / 16; ++k) {
-        mma_bf16_ss(tmem + kColDP, smem_desc_sw128(sV + k * 32, 16, 1024),
+        mma_bf16_ss(tmem + kColDP, smem_desc_sw128(sV + kvs * kTileBytes + k * 32, 16, 1024),
                     smem_desc_sw128(sDO + st * kTileBytes + k * 32, 16, 1024), kIdescS,
                     k > 0 ? 1u : 0u);
       }
@@ -320,13 +364,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
     bool ok = true;
     for (int w = blockIdx.x; w < total && ok && !*abort_flag; w += gridDim.x, ++it) {
       const Rec rc = load_rec(P, w);
-      if (!mbar_wait(&bars[kKVFull], parity(it), abort_flag, a.err) ||
+      const int kvs = it & 1;
+      if (!mbar_wait(&bars[kKVFull + kvs], parity(it >> 1), abort_flag, a.err) ||
           !mbar_wait(&bars[kQDFull + (g & 1)], parity(g >> 1), abort_flag, a.err)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      issue_sdp(g);
+      issue_sdp(g, kvs);
       for (int t = 0; t < rc.nq; ++t, ++g) {
         const int st = g & 1;
         if (!mbar_wait(&bars[kPFull], parity(g), abort_flag, a.err)) {
@@ -342,8 +387,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
             break;
           }
           tc_fence_after();
-          issue_sdp(g + 1);
+          issue_sdp(g + 1, kvs);
         }
+        // the record's first dV, dK overwrite the accumulators: the previous record's
+        // dV, dK must have been read out
+        if (t == 0 && !mbar_wait(&bars[kDKVEmpty], parity(it) ^ 1u, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         // dV += P^T dO ; dK += dS^T Q   (K = 128 queries, 8 steps)
 #pragma unroll
         for (int k = 0; k < BM / 16; ++k) {
@@ -371,7 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
 #pragma unroll
         for (int k = 0; k < BM / 16; ++k) {
           const uint64_t ads = smem_desc_sw128(sDS + k * 16 * 128, BM * 128, 1024);
-          const uint64_t bk = smem_desc_sw128(sK + k * 16 * 128, kTileBytes, 1024);
+          const uint64_t bk =
+              smem_desc_sw128(sK + kvs * kTileBytes + k * 16 * 128, kTileBytes, 1024);
           mma_bf16_ss(tmem + kColDQ + db * DH, ads, bk, kIdescQ, k > 0 ? 1u : 0u);
         }
         mma_commit(&bars[kDQFull + db]);
@@ -379,12 +432,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
         mma_commit(&bars[kQDEmpty + st]);
       }
       if (!ok) break;
-      mma_commit(&bars[kKVEmpty]);
+      mma_commit(&bars[kKVEmpty + kvs]);
+      mma_commit(&bars[kDKVFull]);
     }
-  } else if (warp < 4) {
+  } else if (warp >= 2 && warp < 2 + kSoftmaxWarps) {
     // ---------------------------------------------------------------- softmax (key rows)
-    const int r = threadIdx.x;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int quad = warp & 3;              // TMEM lane quadrant of the warp
+    const int rh = (warp - 2) >> 2;         // upper or lower 16 lanes of the quadrant
+    const int hq = lane >> 4;               // half of the query columns
+    const int r = quad * 32 + rh * 16 + (lane & 15);  // key row within the tile
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32 + rh * 16) << 16);
     const float scale_log2 = a.scale * kLog2e;
     const float* sL2 = reinterpret_cast<const float*>(smem + kOffL2);
     const float* sD = reinterpret_cast<const float*>(smem + kOffD);
@@ -412,68 +469,65 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
         // visible iff key valid, query row inside the user and i >= j
         const int ilo = max(j, q0);  // first visible query (local index)
         const int ihi = rc.L;        // one past the last
-        const float* l2 = sL2 + st * BM;
-        const float* dd = sD + st * BM;
-#pragma unroll 1
-        for (int c0 = 0; c0 < BM; c0 += 32) {
-          float sv[32], dp[32];
-          tmem_ld32(tmem + lane_base + kColS + c0, sv);
-          tmem_ld32(tmem + lane_base + kColDP + c0, dp);
-          uint32_t pk[16], dk[16];
+        const float* l2 = sL2 + st * BM + 64 * hq;
+        const float* dd = sD + st * BM + 64 * hq;
+        const int qbase = q0 + 64 * hq;  // this thread's first query column
+        uint32_t sa[16], da[16], sb[16], db[16];
+        tmem_ld_half16_async<64>(lane_base + kColS, sa);
+        tmem_ld_half16_async<64>(lane_base + kColDP, da);
+        tmem_ld_wait(sa);
+        tmem_ld_wait(da);
+        auto chunk = [&](const uint32_t (&sv)[16], const uint32_t (&dp)[16], int c0) {
+          uint32_t pk[8], dk[8];
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
+          for (int c = 0; c < 16; c += 2) {
             float p2[2], ds2[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int i = q0 + c0 + c + e;
+              const int i = qbase + c0 + c + e;
               const bool vis = key && i >= ilo && i < ihi;
-              const float x = fmaf(sv[c + e], scale_log2, cbj - l2[c0 + c + e]);
+              const float x =
+                  fmaf(__uint_as_float(sv[c + e]), scale_log2, cbj - l2[c0 + c + e]);
               const float p = vis ? ex2(x) : 0.f;
               p2[e] = p;
-              ds2[e] = p * (dp[c + e] - dd[c0 + c + e]);
+              ds2[e] = p * (__uint_as_float(dp[c + e]) - dd[c0 + c + e]);
             }
             pk[c / 2] = pack_bf16(p2[0], p2[1]);
             dk[c / 2] = pack_bf16(ds2[0], ds2[1]);
           }
-          store_row_chunk(sP, r, c0, pk);
-          store_row_chunk(sDS, r, c0, dk);
+          store_row_chunk16(sP, r, 64 * hq + c0, pk);
+          store_row_chunk16(sDS, r, 64 * hq + c0, dk);
+        };
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          tmem_ld_half16_async<64>(lane_base + kColS + c0 + 16, sb);
+          tmem_ld_half16_async<64>(lane_base + kColDP + c0 + 16, db);
+          chunk(sa, da, c0);
+          tmem_ld_wait(sb);
+          tmem_ld_wait(db);
+          if (c0 + 32 < 64) {
+            tmem_ld_half16_async<64>(lane_base + kColS + c0 + 32, sa);
+            tmem_ld_half16_async<64>(lane_base + kColDP + c0 + 32, da);
+          }
+          chunk(sb, db, c0 + 16);
+          if (c0 + 32 < 64) {
+            tmem_ld_wait(sa);
+            tmem_ld_wait(da);
+          }
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&bars[kPFull]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kPFull]);
       }
       if (!ok) break;
-      // record epilogue: dK (times scale) and dV of this key tile, once its last
-      // gradient MMAs are done
-      if (!wait_warp(&bars[kPSFree], parity(g - 1), abort_flag, a.err)) break;
-      tc_fence_after();
-      float dvr[DH], dkr[DH];
-      tmem_ld64(tmem + lane_base + kColDV, dvr);
-      tmem_ld64(tmem + lane_base + kColDK, dkr);
-      tc_fence_before();
-      if (key) {
-        const long long tok = (long long)rc.s + j;
-        __nv_bfloat16* dkp = (__nv_bfloat16*)a.dk + tok * a.tok_stride + rc.h * DH;
-        __nv_bfloat16* dvp = (__nv_bfloat16*)a.dv + tok * a.tok_stride + rc.h * DH;
-#pragma unroll
-        for (int c = 0; c < DH; c += 8) {
-          float f[8], v8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            f[e] = dkr[c + e] * a.scale;
-            v8[e] = dvr[c + e];
-          }
-          *reinterpret_cast<uint4*>(dkp + c) = Elem<__nv_bfloat16>::pack(f);
-          *reinterpret_cast<uint4*>(dvp + c) = Elem<__nv_bfloat16>::pack(v8);
-        }
-      }
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 2 + kSoftmaxWarps) {
     // ---------------------------------------------------------------- dQ reduction (query rows)
     const int qlane = 32 * (warp & 3) + lane;  // TMEM lane this thread may read
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    int g = 0;
-    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+    int g = 0, it = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
       __syncwarp();
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const Rec rc = load_rec(P, w);
@@ -488,7 +542,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
         float dq[DH];
         tmem_ld64(tmem + lane_base + kColDQ + db * DH, dq);
         tc_fence_before();
-        mbar_arrive(&bars[kDQEmpty + db]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kDQEmpty + db]);
         const int i = rc.k0 + t * BM + qlane;
         if (i < rc.L) {
           float* dst = P.dqacc + (((long long)rc.s + i) * a.H + rc.h) * DH;
@@ -500,6 +555,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
         }
       }
       if (!ok) break;
+      // the record's dK (times scale) and dV, key row qlane, once its last gradient MMAs
+      // are done; the accumulators are released before the last stores
+      if (!wait_warp(&bars[kDKVFull], parity(it), abort_flag, a.err)) break;
+      tc_fence_after();
+      const int j = rc.k0 + qlane;
+      const bool key = j < rc.n;
+      const long long tok = (long long)rc.s + j;
+      __nv_bfloat16* dkp = (__nv_bfloat16*)a.dk + tok * a.tok_stride + rc.h * DH;
+      __nv_bfloat16* dvp = (__nv_bfloat16*)a.dv + tok * a.tok_stride + rc.h * DH;
+#pragma unroll 1
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        float dvr[32], dkr[32];
+        tmem_ld32(tmem + lane_base + kColDV + c0, dvr);
+        tmem_ld32(tmem + lane_base + kColDK + c0, dkr);
+        if (c0 + 32 == DH) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[kDKVEmpty]);
+        }
+        if (key) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = dkr[c + e] * a.scale;
+            *reinterpret_cast<uint4*>(dkp + c0 + c) = Elem<__nv_bfloat16>::pack(f);
+            *reinterpret_cast<uint4*>(dvp + c0 + c) = Elem<__nv_bfloat16>::pack(dvr + c);
+          }
+        }
+      }
     }
   }
 
@@ -507,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -607,6 +692,7 @@ static int max_tiles_of(int max_seqlen) { return (max_seqlen + BM - 1) / BM; }
 static size_t recs_bytes(int B, int max_seqlen) {
   return ((size_t)B * max_tiles_of(max_seqlen) * 32 + 15) / 16 * 16;
 }
+static size_t users_bytes(int B) { return ((size_t)B * 4 + 15) / 16 * 16; }
 static size_t rows_bytes(long long T, int B, int H) {
   return ((size_t)H * scratch_tp(T, B) * sizeof(float) + 15) / 16 * 16;
 }
@@ -615,7 +701,7 @@ static size_t rows_bytes(long long T, int B, int H) {
 
 size_t attn_bwd_tc_workspace(int B, long long T, int H, int max_seqlen) {
   using namespace tcb;
-  return kHeaderBytes + recs_bytes(B, max_seqlen) + 3 * rows_bytes(T, B, H) +
+  return kHeaderBytes + recs_bytes(B, max_seqlen) + users_bytes(B) + 3 * rows_bytes(T, B, H) +
          (size_t)T * H * DH * sizeof(float);
 }
 
@@ -634,7 +720,8 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   p.count = (int32_t*)ws;
   p.recs = (int4*)(ws + kHeaderBytes);
   const size_t rb = rows_bytes(a.T, a.B, a.H);
-  uint8_t* rows = ws + kHeaderBytes + recs_bytes(a.B, a.max_seqlen);
+  int32_t* uorder = (int32_t*)(ws + kHeaderBytes + recs_bytes(a.B, a.max_seqlen));
+  uint8_t* rows = (uint8_t*)uorder + users_bytes(a.B);
   p.cbias = (float*)rows;
   p.lse2 = (float*)(rows + rb);
   p.dsum = (float*)(rows + 2 * rb);
@@ -643,8 +730,8 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   if (cudaMemsetAsync(p.dqacc, 0, (size_t)a.T * a.H * DH * sizeof(float), st) != cudaSuccess)
     return GENRANK_ERR_CUDA;
   k_bwd_prologue<<<a.B + 1, 256, 0, st>>>(a, max_tiles_of(a.max_seqlen), (int4*)p.recs,
-                                          (int32_t*)p.count, (float*)p.cbias, (float*)p.lse2,
-                                          (float*)p.dsum, p.Tp);
+                                          (int32_t*)p.count, uorder, (float*)p.cbias,
+                                          (float*)p.lse2, (float*)p.dsum, p.Tp);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   static bool attr = false;
   if (!attr) {

@@ -127,36 +127,12 @@ constexpr int kMaxBuckets = 257;
 
 __global__ void __launch_bounds__(256) k_bwd_prologue(const __grid_constant__ AttnArgs a,
                                                       int max_tiles, int4* recs, int32_t* count,
-                                                      int32_t* uorder, float* cbias,
-                                                      float* lse2, float* dsum, long long Tp) {
+                                                      int32_t* uorder, int32_t* tok_user) {
   const int b = blockIdx.x;
-  if (b < a.B) {
+  if (b < a.B) {  // the owner of every token (read by the per-row kernels)
     const long long s = a.off[b], e = a.off[b + 1];
     if (s < 0 || e < s || e > a.T) return;
-    const int L = (int)(e - s);
-    const long long base = seg_start(s, b);
-    const long long t0 = L > 0 ? a.ts[s] : 0;
-    const __nv_bfloat16* O = (const __nv_bfloat16*)a.o;
-    const __nv_bfloat16* G = (const __nv_bfloat16*)a.dO;
-    // one warp per (token, head): D is a 64-long dot, two elements per lane
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    for (int x = wid; x < L * a.H; x += nw) {
-      const int i = x / a.H, h = x - (x / a.H) * a.H;
-      const long long tok = s + i;
-      const uint32_t ow = *reinterpret_cast<const uint32_t*>(O + tok * a.o_stride + h * DH + 2 * lane);
-      const uint32_t gw = *reinterpret_cast<const uint32_t*>(G + tok * a.o_stride + h * DH + 2 * lane);
-      float dd = bf16_lo(ow) * bf16_lo(gw) + bf16_hi(ow) * bf16_hi(gw);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
-      if (lane == 0) {
-        const float c = kLog2e * (a.slope_pos[h] * (float)a.pos[tok] +
-                                  a.slope_time[h] * (float)(a.ts[tok] - t0));
-        const long long idx = (long long)h * Tp + base + i;
-        cbias[idx] = c;
-        lse2[idx] = a.lse_in[(long long)h * a.T + tok] * kLog2e + c;
-        dsum[idx] = dd;
-      }
-    }
+    for (long long t = s + threadIdx.x; t < e; t += blockDim.x) tok_user[t] = b;
     return;
   }
   // Records go out user by user (users with the most history key tiles first, each
@@ -229,6 +205,46 @@ __global__ void __launch_bounds__(256) k_bwd_prologue(const __grid_constant__ At
     }
   }
   if (threadIdx.x == 0) *count = total;
+}
+
+// Per (token, head) terms, eight lanes per pair (16-byte loads of O and dO rows):
+// c_j = log2 e (m_h p_j + m_t,h (t_j - t_0)), lse2_i = LSE_i log2 e + c_i and
+// D_i = rowsum(dO_i * O_i), at the user's segment of the [H][Tp] scratch.
+__global__ void __launch_bounds__(256) k_bwd_rows(const __grid_constant__ AttnArgs a,
+                                                  const int32_t* __restrict__ tok_user,
+                                                  float* cbias, float* lse2, float* dsum,
+                                                  long long Tp) {
+  const long long x = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 3;  // pair
+  const int sub = threadIdx.x & 7;
+  const long long tend = min(a.T, (long long)a.off[a.B]);
+  const long long tok = x / a.H;
+  const int h = (int)(x - tok * a.H);
+  const bool live = tok < tend;
+  float dd = 0.f;
+  if (live) {
+    const uint4 ov = *reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.o + tok * a.o_stride +
+                                                     h * DH + 8 * sub);
+    const uint4 gv = *reinterpret_cast<const uint4*>(
+        (const __nv_bfloat16*)a.dO + tok * a.o_stride + h * DH + 8 * sub);
+    float of[8], gf[8];
+    Elem<__nv_bfloat16>::unpack(ov, of);
+    Elem<__nv_bfloat16>::unpack(gv, gf);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dd = fmaf(of[e], gf[e], dd);
+  }
+  dd += __shfl_xor_sync(0xffffffffu, dd, 4);
+  dd += __shfl_xor_sync(0xffffffffu, dd, 2);
+  dd += __shfl_xor_sync(0xffffffffu, dd, 1);
+  if (!live || sub != 0) return;
+  const int u = tok_user[tok];
+  if (u < 0 || u >= a.B) return;  // tokens of no valid user (the schedule flags the layout)
+  const long long s = a.off[u];
+  const float c = kLog2e * (a.slope_pos[h] * (float)a.pos[tok] +
+                            a.slope_time[h] * (float)(a.ts[tok] - a.ts[s]));
+  const long long idx = (long long)h * Tp + seg_start(s, u) + (tok - s);
+  cbias[idx] = c;
+  lse2[idx] = a.lse_in[(long long)h * a.T + tok] * kLog2e + c;
+  dsum[idx] = dd;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -598,65 +614,67 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
 // ------------------------------------------------------------------------------------------
 // finishing kernel: dq from the accumulator, and the candidate self terms
 // ------------------------------------------------------------------------------------------
-// One warp per (token, head), two of the 64 columns per lane.  For a candidate token c
-// (its own key, bias 0): p = exp(scale q.k - LSE), ds = p (dO.v - D),
-// dv = p dO, dk = scale ds q, and dq gains scale ds k.
+// Eight lanes per (token, head), eight of the 64 columns per lane (16-byte loads).
+// For a candidate token c (its own key, bias 0): p = exp(scale q.k - LSE),
+// ds = p (dO.v - D), dv = p dO, dk = scale ds q, and dq gains scale ds k.
 __global__ void __launch_bounds__(256) k_bwd_finish(const __grid_constant__ AttnArgs a,
                                                     const float* __restrict__ dqacc,
-                                                    const float* __restrict__ dsum, long long Tp,
-                                                    int tokens_per_warp) {
-  const int lane = threadIdx.x & 31;
-  const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const long long t0 = warp * tokens_per_warp;
+                                                    const float* __restrict__ dsum,
+                                                    const int32_t* __restrict__ tok_user,
+                                                    long long Tp) {
+  const long long x = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 3;  // pair
+  const int sub = threadIdx.x & 7;
   const long long tend = min(a.T, (long long)a.off[a.B]);
-  if (t0 >= tend) return;
-  const long long t1 = min(tend, t0 + tokens_per_warp);
-  int u = warp_find_user(a.off, a.B, t0);
-  long long u_beg = a.off[u], u_end = a.off[u + 1];
-  int n = a.hist_len[u];
-  const __nv_bfloat16* Q = (const __nv_bfloat16*)a.q;
-  const __nv_bfloat16* K = (const __nv_bfloat16*)a.k;
-  const __nv_bfloat16* V = (const __nv_bfloat16*)a.v;
-  const __nv_bfloat16* G = (const __nv_bfloat16*)a.dO;
-  for (long long t = t0; t < t1; ++t) {
-    while (t >= u_end && u < a.B - 1) {
-      ++u;
-      u_beg = u_end;
-      u_end = a.off[u + 1];
-      n = a.hist_len[u];
-    }
-    const bool cand = (t - u_beg) >= n;
-    const long long base = seg_start(u_beg, u);
-    for (int h = 0; h < a.H; ++h) {
-      const float2 acc = *reinterpret_cast<const float2*>(dqacc + (t * a.H + h) * DH + 2 * lane);
-      float dq0 = acc.x * a.scale, dq1 = acc.y * a.scale;
-      const long long qo = t * a.tok_stride + h * DH + 2 * lane;
-      if (cand) {
-        const uint32_t qw = *reinterpret_cast<const uint32_t*>(Q + qo);
-        const uint32_t kw = *reinterpret_cast<const uint32_t*>(K + qo);
-        const uint32_t vw = *reinterpret_cast<const uint32_t*>(V + qo);
-        const uint32_t gw =
-            *reinterpret_cast<const uint32_t*>(G + t * a.o_stride + h * DH + 2 * lane);
-        float sdot = bf16_lo(qw) * bf16_lo(kw) + bf16_hi(qw) * bf16_hi(kw);
-        float pdot = bf16_lo(gw) * bf16_lo(vw) + bf16_hi(gw) * bf16_hi(vw);
+  const long long tok = x / a.H;
+  const int h = (int)(x - tok * a.H);
+  const int u = tok < tend ? tok_user[tok] : -1;
+  const bool owned = u >= 0 && u < a.B;
+  const long long s = owned ? a.off[u] : 0;
+  const bool cand = owned && tok - s >= a.hist_len[u];
+  const long long qo = tok * a.tok_stride + h * DH + 8 * sub;
+  float dq[8], qf[8], kf[8], vf[8], gf[8];
+  float sdot = 0.f, pdot = 0.f;
+  if (owned) {
+    const float4* acc = reinterpret_cast<const float4*>(dqacc + (tok * a.H + h) * DH + 8 * sub);
+    const float4 a0 = acc[0], a1 = acc[1];
+    dq[0] = a0.x; dq[1] = a0.y; dq[2] = a0.z; dq[3] = a0.w;
+    dq[4] = a1.x; dq[5] = a1.y; dq[6] = a1.z; dq[7] = a1.w;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
-          pdot += __shfl_xor_sync(0xffffffffu, pdot, o);
-        }
-        const long long ridx = (long long)h * Tp + base + (t - u_beg);
-        const float p = expf(sdot * a.scale - a.lse_in[(long long)h * a.T + t]);
-        const float ds = p * (pdot - dsum[ridx]);
-        dq0 += a.scale * ds * bf16_lo(kw);
-        dq1 += a.scale * ds * bf16_hi(kw);
-        *reinterpret_cast<uint32_t*>((__nv_bfloat16*)a.dk + qo) =
-            pack_bf16(a.scale * ds * bf16_lo(qw), a.scale * ds * bf16_hi(qw));
-        *reinterpret_cast<uint32_t*>((__nv_bfloat16*)a.dv + qo) =
-            pack_bf16(p * bf16_lo(gw), p * bf16_hi(gw));
-      }
-      *reinterpret_cast<uint32_t*>((__nv_bfloat16*)a.dq + qo) = pack_bf16(dq0, dq1);
+    for (int e = 0; e < 8; ++e) dq[e] *= a.scale;
+  }
+  if (cand) {
+    Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.q + qo), qf);
+    Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.k + qo), kf);
+    Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.v + qo), vf);
+    Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(
+                                    (const __nv_bfloat16*)a.dO + tok * a.o_stride + h * DH + 8 * sub),
+                                gf);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      sdot = fmaf(qf[e], kf[e], sdot);
+      pdot = fmaf(gf[e], vf[e], pdot);
     }
   }
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) {
+    sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
+    pdot += __shfl_xor_sync(0xffffffffu, pdot, o);
+  }
+  if (cand) {
+    const long long ridx = (long long)h * Tp + seg_start(s, u) + (tok - s);
+    const float p = expf(sdot * a.scale - a.lse_in[(long long)h * a.T + tok]);
+    const float ds = p * (pdot - dsum[ridx]);
+    float dk[8], dv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      dq[e] = fmaf(a.scale * ds, kf[e], dq[e]);
+      dk[e] = a.scale * ds * qf[e];
+      dv[e] = p * gf[e];
+    }
+    *reinterpret_cast<uint4*>((__nv_bfloat16*)a.dk + qo) = Elem<__nv_bfloat16>::pack(dk);
+    *reinterpret_cast<uint4*>((__nv_bfloat16*)a.dv + qo) = Elem<__nv_bfloat16>::pack(dv);
+  }
+  if (owned) *reinterpret_cast<uint4*>((__nv_bfloat16*)a.dq + qo) = Elem<__nv_bfloat16>::pack(dq);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -693,6 +711,7 @@ static size_t recs_bytes(int B, int max_seqlen) {
   return ((size_t)B * max_tiles_of(max_seqlen) * 32 + 15) / 16 * 16;
 }
 static size_t users_bytes(int B) { return ((size_t)B * 4 + 15) / 16 * 16; }
+static size_t tokens_bytes(long long T) { return ((size_t)T * 4 + 15) / 16 * 16; }
 static size_t rows_bytes(long long T, int B, int H) {
   return ((size_t)H * scratch_tp(T, B) * sizeof(float) + 15) / 16 * 16;
 }
@@ -701,8 +720,8 @@ static size_t rows_bytes(long long T, int B, int H) {
 
 size_t attn_bwd_tc_workspace(int B, long long T, int H, int max_seqlen) {
   using namespace tcb;
-  return kHeaderBytes + recs_bytes(B, max_seqlen) + users_bytes(B) + 3 * rows_bytes(T, B, H) +
-         (size_t)T * H * DH * sizeof(float);
+  return kHeaderBytes + recs_bytes(B, max_seqlen) + users_bytes(B) + tokens_bytes(T) +
+         3 * rows_bytes(T, B, H) + (size_t)T * H * DH * sizeof(float);
 }
 
 int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
@@ -721,7 +740,8 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   p.recs = (int4*)(ws + kHeaderBytes);
   const size_t rb = rows_bytes(a.T, a.B, a.H);
   int32_t* uorder = (int32_t*)(ws + kHeaderBytes + recs_bytes(a.B, a.max_seqlen));
-  uint8_t* rows = (uint8_t*)uorder + users_bytes(a.B);
+  int32_t* tok_user = (int32_t*)((uint8_t*)uorder + users_bytes(a.B));
+  uint8_t* rows = (uint8_t*)tok_user + tokens_bytes(a.T);
   p.cbias = (float*)rows;
   p.lse2 = (float*)(rows + rb);
   p.dsum = (float*)(rows + 2 * rb);
@@ -729,10 +749,17 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   p.Tp = scratch_tp(a.T, a.B);
   if (cudaMemsetAsync(p.dqacc, 0, (size_t)a.T * a.H * DH * sizeof(float), st) != cudaSuccess)
     return GENRANK_ERR_CUDA;
+  if (a.T > 0 && cudaMemsetAsync(tok_user, 0xff, (size_t)a.T * 4, st) != cudaSuccess)
+    return GENRANK_ERR_CUDA;
   k_bwd_prologue<<<a.B + 1, 256, 0, st>>>(a, max_tiles_of(a.max_seqlen), (int4*)p.recs,
-                                          (int32_t*)p.count, uorder, (float*)p.cbias,
-                                          (float*)p.lse2, (float*)p.dsum, p.Tp);
+                                          (int32_t*)p.count, uorder, tok_user);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
+  const long long pair_blocks = (a.T * a.H + 31) / 32;  // 8 lanes per (token, head)
+  if (pair_blocks > 0) {
+    k_bwd_rows<<<(unsigned)pair_blocks, 256, 0, st>>>(a, tok_user, (float*)p.cbias,
+                                                      (float*)p.lse2, (float*)p.dsum, p.Tp);
+    if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
+  }
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(k_attn_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -745,11 +772,8 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   k_attn_bwd_tc<<<sms, kThreads, kSmemBytes, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
-  const long long warps_target = (long long)sms * 64;
-  const long long tpw_ll = (a.T + warps_target - 1) / warps_target;
-  const int tpw = (int)(tpw_ll > 0 ? tpw_ll : 1);
-  const long long warps = (a.T + tpw - 1) / tpw;
-  k_bwd_finish<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(a, p.dqacc, p.dsum, p.Tp, tpw);
+  if (pair_blocks > 0)
+    k_bwd_finish<<<(unsigned)pair_blocks, 256, 0, st>>>(a, p.dqacc, p.dsum, tok_user, p.Tp);
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
 }
 

@@ -270,7 +270,7 @@ def run_native(args, cfg, world, rank, local):
 
     from gen import make_batch, make_model
     from generative_ranking_recommendation_b200 import genrank as G
-    from generative_ranking_recommendation_b200.model import DeviceBatch, GenRankModel
+    from generative_ranking_recommendation_b200.model import CapturedStep, DeviceBatch, GenRankModel
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -294,59 +294,58 @@ def run_native(args, cfg, world, rank, local):
         gm.forward(dbs[k % 2])
     torch.cuda.synchronize()
     assert G.check_error(gm.err) == 0, "device error flags raised during warm-up"
+    # each batch's step as a CUDA graph (no host launch work inside the step), and the
+    # attention call alone as its own graph for the kernel's roofline timing
+    steps = [CapturedStep(gm, db) for db in dbs]
+    attn = [CapturedStep(gm, db, part="attention") for db in dbs]
+    for k in range(args.warmup):
+        steps[k % 2].run()
+        attn[k % 2].run()
+    torch.cuda.synchronize()
 
-    # ---- device-resident inputs, CUDA events per step, L2 flushed between steps
+    def timed(fn, n):
+        """Device time of n calls of fn, L2 flushed before each (events bracket fn only)."""
+        ev = []
+        for k in range(n):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.nvtx.range_push("timed_step")
+            s.record()
+            fn(k)
+            e.record()
+            torch.cuda.nvtx.range_pop()
+            ev.append((s, e))
+        sync_all()
+        return [s.elapsed_time(e) for s, e in ev]
+
+    # ---- device-resident inputs, one graph replay per step
     sampler = ClockSampler(local)
     sync_all()
     sampler.start()
-    ev = []
-    attn_ev = []
-    for k in range(args.steps):
-        flush.zero_()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.nvtx.range_push("timed_step")
-        s.record()
-        gm.forward(dbs[k % 2], attn_events=attn_ev)
-        e.record()
-        torch.cuda.nvtx.range_pop()
-        ev.append((s, e))
-    sync_all()
+    step_ms = timed(lambda k: steps[k % 2].run(), args.steps)
     clocks = sampler.stop()
-    step_ms = [s.elapsed_time(e) for s, e in ev]
     total_ms = sum(step_ms)
-    attn_ms = [s.elapsed_time(e) for s, e in attn_ev]
+    attn_ms = timed(lambda k: attn[k % 2].run(), args.steps)
 
     # ---- end to end through the public API: pinned host inputs -> device -> logits -> host
     host = [DeviceBatch.host_arrays(b) for b in batches]
     pinned = [[torch.from_numpy(np.ascontiguousarray(a)).pin_memory() for a in h] for h in host]
-    dev_bufs = [[torch.empty(p.shape, dtype=p.dtype, device=dev) for p in ps] for ps in pinned]
-    n_cand = int(sum(b.cand_count.sum() for b in batches[:1]))
-    out_host = torch.empty(n_cand, dtype=torch.float32).pin_memory()
+    n_cand = [int(b.cand_count.sum()) for b in batches]
+    out_host = [torch.empty(n, dtype=torch.float32).pin_memory() for n in n_cand]
     h2d = sum(p.numel() * p.element_size() for p in pinned[0])
-    d2h = out_host.numel() * out_host.element_size()
+    d2h = out_host[0].numel() * out_host[0].element_size()
 
     def e2e_step(k):
         i = k % 2
-        for p, d in zip(pinned[i], dev_bufs[i]):
-            d.copy_(p, non_blocking=True)
-        db = DeviceBatch.from_tensors(batches[i], dev_bufs[i])
-        z = gm.forward(db)
-        out_host.copy_(z, non_blocking=True)
+        steps[i].load(pinned[i])
+        out_host[i].copy_(steps[i].run(), non_blocking=True)
 
     for k in range(2):
         e2e_step(k)
     sync_all()
-    ev2 = []
-    for k in range(args.steps):
-        flush.zero_()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record()
-        e2e_step(k)
-        e.record()
-        ev2.append((s, e))
-    sync_all()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in ev2)
+    e2e_ms = sum(timed(e2e_step, args.steps))
     assert G.check_error(gm.err) == 0, "device error flags raised during the timed region"
+    del steps, attn
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, dev)
     if world > 1:

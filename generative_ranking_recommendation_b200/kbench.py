@@ -3,8 +3,8 @@
     python -m generative_ranking_recommendation_b200.kbench --config c2 \
         [--kernels embed_fwd,attn_fwd,attn_bwd,embed_bwd] [--iters 20] [--warmup 3]
 
-Times each library call with CUDA events (inputs resident in HBM, L2 flushed
-before every timed launch) and prints one JSON line per kernel with its
+Times each library call with CUDA events around a replay of the call captured as
+a CUDA graph (inputs resident in HBM, L2 flushed before every timed replay) and prints one JSON line per kernel with its
 algorithmic throughput: GB/s for the embedding kernels, TFLOP/s for attention
 (4 d flops per visible pair forward, 10 d backward; masked pairs and padding
 not counted).  Attention operands are unit-scale random bf16 values.
@@ -46,15 +46,28 @@ def positions(batch):
 
 
 def timed(fn, iters, warmup, flush):
-    for _ in range(warmup):
+    """Median device time of one call of fn.  The call is captured once as a CUDA
+    graph and replayed, so host work inside it (argument marshalling, tensor-map
+    encoding) cannot idle the GPU inside the timed span; L2 is flushed before each
+    replay."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(max(1, warmup)):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
         fn()
+    graph.replay()
     torch.cuda.synchronize()
     ts = []
     for _ in range(iters):
         flush.zero_()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
-        fn()
+        graph.replay()
         e.record()
         ts.append((s, e))
     torch.cuda.synchronize()

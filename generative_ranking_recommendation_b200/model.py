@@ -258,3 +258,53 @@ class GenRankModel:
                              rtb, dE, grads["item"], grads["action"], grads["pos"], grads["ri"],
                              grads["rt"], self.err)
         return loss.detach(), z.detach(), grads
+
+
+class CapturedStep:
+    """One batch's scoring step captured as a CUDA graph.
+
+    The library calls and the torch ops of ``model.forward(db)`` are recorded once
+    and replayed without host launch work (argument marshalling, tensor-map
+    encoding, dispatch), which otherwise leaves the GPU idle between the short
+    kernels of a step.  The graph reads the batch's device tensors: to score new
+    inputs of the same shapes, copy them into ``db``'s tensors (``load``) and
+    ``run()``.  The logits tensor returned by ``run()`` is overwritten by the next
+    replay.  The captured workspace stays referenced by this object, so later
+    captures of other shapes cannot free it.
+    """
+
+    def __init__(self, model: GenRankModel, db: DeviceBatch, part: str = "forward"):
+        self.model, self.db = model, db
+        stream = torch.cuda.Stream(device=model.device)
+        stream.wait_stream(torch.cuda.current_stream(model.device))
+        with torch.cuda.stream(stream):
+            if part == "attention":  # the first layer's attention alone
+                E, (pos, _, _) = model.embed(db)
+                W = model.layers[0]
+                a = model.rms(E.float()).to(model.dtype) if model.cfg.ffn else E
+                self._qkv, self._pos = a @ W["Wqkv"], pos
+                fn = lambda: model.attention(db, self._qkv, self._pos)[0]  # noqa: E731
+            elif part == "forward":
+                fn = lambda: model.forward(db)  # noqa: E731
+            else:
+                raise ValueError(f"unknown part {part!r}")
+            fn()  # warm-up: function attributes, workspace
+        torch.cuda.current_stream(model.device).wait_stream(stream)
+        torch.cuda.synchronize(model.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.out = fn()
+        self._ws = dict(model._ws)  # keep the captured workspaces alive
+
+    def load(self, tensors):
+        """Copy new per-step inputs (host or device tensors, upload order of
+        ``DeviceBatch.host_arrays``) into the captured batch."""
+        dst = [self.db.seq_offsets, self.db.hist_len, self.db.item_ids, self.db.action_ids,
+               self.db.ts, self.db.cand_rows] + ([self.db.labels] if self.db.labels is not None
+                                                  else [])
+        for d, s in zip(dst, tensors):
+            d.copy_(s, non_blocking=True)
+
+    def run(self) -> torch.Tensor:
+        self.graph.replay()
+        return self.out

@@ -73,3 +73,26 @@ def test_train_step_parity(M):
     assert ref.rel_to_max(got["item"][uniq], gr["item"]) <= 2e-2
     for k in ("action", "pos", "ri", "rt"):
         assert ref.rel_to_max(got[k], gr[k]) <= 2e-2, k
+
+
+@pytest.mark.parametrize("name", ["c0", "c2"])
+def test_captured_step_matches_forward(M, name):
+    """The graph-captured step gives the eager forward's logits bit for bit, and
+    scores new inputs loaded into the captured batch."""
+    cfg = CONFIGS[name]
+    batch = make_batch(cfg, users=list(range(4)))
+    gm = M.GenRankModel(cfg, make_model(cfg), "cuda")
+    db = M.DeviceBatch.from_batch(batch, "cuda")
+    step = M.CapturedStep(gm, db)
+    z0 = step.run().clone()
+    assert torch.equal(z0, gm.forward(M.DeviceBatch.from_batch(batch, "cuda")))
+    # same shapes, other items: load into the captured buffers and replay
+    b2 = make_batch(cfg, users=list(range(4)))
+    b2.item_ids[:] = np.random.default_rng(5).integers(0, cfg.n_item, b2.item_ids.shape)
+    step.load([torch.from_numpy(np.ascontiguousarray(a)) for a in M.DeviceBatch.host_arrays(b2)])
+    z1 = step.run().clone()
+    assert torch.equal(z1, gm.forward(M.DeviceBatch.from_batch(b2, "cuda")))
+    assert not torch.equal(z0, z1)
+    from generative_ranking_recommendation_b200 import genrank as G
+
+    assert G.check_error(gm.err) == 0

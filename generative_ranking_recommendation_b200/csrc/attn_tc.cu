@@ -662,9 +662,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       bool ok = true;
       for (int j = 0; j < it.nt; ++j, ++g) {
         const int sb = g & 1, st = g % kStages;
+        // S_g's commit also covers every MMA issued before it, P_{g-2} V_{g-2} included,
+        // so once S_g is here its P buffer is free as well
         if (!wait_warp(&bars[kSFull + sb], par(g >> 1), abort_flag, a.err) ||
-            !wait_warp(&bars[kKFull + st], par(g / kStages), abort_flag, a.err) ||
-            !wait_warp(&bars[kPFree + sb], par(g >> 1) ^ 1u, abort_flag, a.err)) {
+            !wait_warp(&bars[kKFull + st], par(g / kStages), abort_flag, a.err)) {
           ok = false;
           break;
         }

@@ -227,7 +227,9 @@ def config_block(cfg, world, extra=None):
                      f"({cfg.H}x{cfg.dh}), {cfg.layers} layer, item table {cfg.n_item} rows",
          "global_batch_users": cfg.B * world, "candidates_per_step": cfg.B * cfg.m * world,
          "parallelism": f"users sharded over {world} GPU(s), no collective on the data path",
-         "l2": "flushed (256 MB write) before every timed step"}
+         "l2": "flushed (256 MB write) before every device-timed step and attention launch; "
+               "the pipelined e2e loop is not flushed (a step's working set, with the 512 MB "
+               "item table, is several times the 126 MB L2)"}
     if extra:
         c.update(extra)
     return c
@@ -335,15 +337,39 @@ def run_native(args, cfg, world, rank, local):
     h2d = sum(p.numel() * p.element_size() for p in pinned[0])
     d2h = out_host[0].numel() * out_host[0].element_size()
 
-    def e2e_step(k):
-        i = k % 2
-        steps[i].load(pinned[i])
-        out_host[i].copy_(steps[i].run(), non_blocking=True)
+    # Pipelined as a serving loop runs it: step k+1's inputs cross PCIe on a copy
+    # stream while step k computes (each captured step owns its device buffers, so a
+    # buffer is reloaded only after the step two back has finished with it); every
+    # step still uploads its inputs and reads its logits back inside the timed span.
+    # No L2 flush inside this loop: a step's working set (the 512 MB item table, E,
+    # QKV, O) is several times the 126 MB L2.
+    comp = torch.cuda.current_stream()
+    copy = torch.cuda.Stream(device=dev)
+    loaded = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
 
-    for k in range(2):
-        e2e_step(k)
+    def e2e_loop(n):
+        for k in range(n):
+            i = k % 2
+            with torch.cuda.stream(copy):
+                if k >= 2:
+                    copy.wait_event(done[i])
+                steps[i].load(pinned[i])
+                loaded[i].record(copy)
+            comp.wait_event(loaded[i])
+            out_host[i].copy_(steps[i].run(), non_blocking=True)
+            done[i].record(comp)
+
+    e2e_loop(2)
     sync_all()
-    e2e_ms = sum(timed(e2e_step, args.steps))
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(comp)
+    copy.wait_stream(comp)
+    e2e_loop(args.steps)
+    comp.wait_stream(copy)
+    e.record(comp)
+    sync_all()
+    e2e_ms = s.elapsed_time(e)
     assert G.check_error(gm.err) == 0, "device error flags raised during the timed region"
     del steps, attn
 

@@ -117,8 +117,12 @@ __global__ void __launch_bounds__(256) k_token_meta(
 // the user of its first token with a 32-way search of seq_offsets, then walks
 // forward.  Rows are moved as 16-byte vectors; the five rows are summed in fp32
 // and rounded once.
+// One warp per group of 32 tokens: each lane loads one token's ids (coalesced) and
+// the warp gathers the tokens' five rows with 16-byte vector loads, the row indices
+// broadcast from their lanes by shuffles, two tokens' loads in flight together.
+// At most 64 registers per thread keep four blocks resident per SM.
 template <typename T>
-__global__ void __launch_bounds__(256) k_embed_fwd(
+__global__ void __launch_bounds__(256, 4) k_embed_fwd(
     int B, long long Ttok, const int32_t* __restrict__ off, const int32_t* __restrict__ hist_len,
     const int32_t* __restrict__ item_ids, const int32_t* __restrict__ action_ids,
     const T* __restrict__ item_tab, long long n_item, const T* __restrict__ action_tab,
@@ -127,70 +131,83 @@ __global__ void __launch_bounds__(256) k_embed_fwd(
     const int32_t* __restrict__ pos, const int32_t* __restrict__ req_idx,
     const int32_t* __restrict__ rt_bucket, T* __restrict__ E, int tokens_per_warp, int32_t* err) {
   constexpr int V = Elem<T>::kPerVec;
+  constexpr int U = 2;  // tokens whose row gathers are in flight together
   const int lane = threadIdx.x & 31;
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  long long t0 = warp * tokens_per_warp;
   const long long tend = min(Ttok, (long long)off[B]);
-  if (t0 >= tend) return;
-  const long long t1 = min(tend, t0 + tokens_per_warp);
   const int nv = d / V;
-  int u = warp_find_user(off, B, t0);
-  long long u_end = off[u + 1];
-  long long u_beg = off[u];
-  int n = hist_len[u];
-  for (long long t = t0; t < t1; ++t) {
-    while (t >= u_end && u < B - 1) {
-      ++u;
-      u_beg = u_end;
-      u_end = off[u + 1];
-      n = hist_len[u];
-    }
-    const bool cand = (t - u_beg) >= n;
-    long long it = item_ids[t];
-    if (it < 0 || it >= n_item) {
-      if (lane == 0) flag(err, GENRANK_DERR_ITEM_ID);
-      it = it < 0 ? 0 : n_item - 1;
-    }
-    int a = n_action;  // the mask-action row M
-    if (!cand) {
-      a = action_ids[t];
-      if (a < 0 || a >= n_action) {
-        if (lane == 0) flag(err, GENRANK_DERR_ACTION_ID);
-        a = a < 0 ? 0 : n_action - 1;
+  for (long long t0 = warp * tokens_per_warp; t0 < min(tend, (warp + 1) * tokens_per_warp);
+       t0 += 32) {
+    // one token per lane: its owner, and its five row indices (coalesced id loads)
+    const long long t = t0 + lane;
+    const bool live = t < tend;
+    int u = warp_find_user(off, B, t0);
+    long long it = 0;
+    int a = 0, p = 0, r = 0, b = 0;
+    if (live) {
+      while (u < B - 1 && t >= off[u + 1]) ++u;
+      const bool cand = (t - off[u]) >= hist_len[u];
+      it = item_ids[t];
+      if (it < 0 || it >= n_item) {
+        flag(err, GENRANK_DERR_ITEM_ID);
+        it = it < 0 ? 0 : n_item - 1;
+      }
+      a = n_action;  // the mask-action row M
+      if (!cand) {
+        a = action_ids[t];
+        if (a < 0 || a >= n_action) {
+          flag(err, GENRANK_DERR_ACTION_ID);
+          a = a < 0 ? 0 : n_action - 1;
+        }
+      }
+      p = pos[t];
+      r = req_idx[t];
+      b = rt_bucket[t];
+      if (p < 0 || p >= n_pos || r < 0 || r >= n_ri || b < 0 || b >= n_rt) {
+        // only reachable when the metadata pass rejected this user's layout
+        flag(err, GENRANK_DERR_INDEX);
+        p = min(max(p, 0), n_pos - 1);
+        r = min(max(r, 0), n_ri - 1);
+        b = min(max(b, 0), n_rt - 1);
       }
     }
-    int p = pos[t], r = req_idx[t], b = rt_bucket[t];
-    if (p < 0 || p >= n_pos || r < 0 || r >= n_ri || b < 0 || b >= n_rt) {
-      // only reachable when the metadata pass rejected this user's layout
-      if (lane == 0) flag(err, GENRANK_DERR_INDEX);
-      p = min(max(p, 0), n_pos - 1);
-      r = min(max(r, 0), n_ri - 1);
-      b = min(max(b, 0), n_rt - 1);
-    }
-    const uint4* r0 = reinterpret_cast<const uint4*>(item_tab + it * d);
-    const uint4* r1 = reinterpret_cast<const uint4*>(action_tab + (long long)a * d);
-    const uint4* r2 = reinterpret_cast<const uint4*>(pos_tab + (long long)p * d);
-    const uint4* r3 = reinterpret_cast<const uint4*>(ri_tab + (long long)r * d);
-    const uint4* r4 = reinterpret_cast<const uint4*>(rt_tab + (long long)b * d);
-    uint4* out = reinterpret_cast<uint4*>(E + t * d);
-    for (int v = lane; v < nv; v += 32) {
-      uint4 x0 = __ldg(r0 + v), x1 = __ldg(r1 + v), x2 = __ldg(r2 + v), x3 = __ldg(r3 + v),
-            x4 = __ldg(r4 + v);
-      float f[V], g[V];
-      Elem<T>::unpack(x0, f);
-      Elem<T>::unpack(x1, g);
+    const int nt = (int)min(32LL, tend - t0);
+    // the warp gathers the tokens' rows U at a time, indices broadcast from their lanes
+    for (int k = 0; k < nt; k += U) {
+      const uint4* rows[U][5];
 #pragma unroll
-      for (int k = 0; k < V; ++k) f[k] += g[k];
-      Elem<T>::unpack(x2, g);
+      for (int q = 0; q < U; ++q) {
+        const int src = min(k + q, nt - 1);
+        const long long itq = __shfl_sync(0xffffffffu, it, src);
+        rows[q][0] = reinterpret_cast<const uint4*>(item_tab + itq * d);
+        rows[q][1] = reinterpret_cast<const uint4*>(
+            action_tab + (long long)__shfl_sync(0xffffffffu, a, src) * d);
+        rows[q][2] = reinterpret_cast<const uint4*>(
+            pos_tab + (long long)__shfl_sync(0xffffffffu, p, src) * d);
+        rows[q][3] = reinterpret_cast<const uint4*>(
+            ri_tab + (long long)__shfl_sync(0xffffffffu, r, src) * d);
+        rows[q][4] = reinterpret_cast<const uint4*>(
+            rt_tab + (long long)__shfl_sync(0xffffffffu, b, src) * d);
+      }
+      for (int v = lane; v < nv; v += 32) {
+        uint4 x[U][5];
 #pragma unroll
-      for (int k = 0; k < V; ++k) f[k] += g[k];
-      Elem<T>::unpack(x3, g);
+        for (int q = 0; q < U; ++q)
 #pragma unroll
-      for (int k = 0; k < V; ++k) f[k] += g[k];
-      Elem<T>::unpack(x4, g);
+          for (int c = 0; c < 5; ++c) x[q][c] = __ldg(rows[q][c] + v);
 #pragma unroll
-      for (int k = 0; k < V; ++k) f[k] += g[k];
-      out[v] = Elem<T>::pack(f);
+        for (int q = 0; q < U; ++q) {
+          float f[V], g[V];
+          Elem<T>::unpack(x[q][0], f);
+#pragma unroll
+          for (int c = 1; c < 5; ++c) {
+            Elem<T>::unpack(x[q][c], g);
+#pragma unroll
+            for (int e = 0; e < V; ++e) f[e] += g[e];
+          }
+          if (k + q < nt) reinterpret_cast<uint4*>(E + (t0 + k + q) * d)[v] = Elem<T>::pack(f);
+        }
+      }
     }
   }
 }
@@ -323,9 +340,10 @@ int launch_embed_fwd(const EmbedFwdArgs& a, cudaStream_t st) {
                                     a.pos, a.req_idx, a.rt_bucket, a.err);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   if (a.T == 0) return GENRANK_OK;
-  // enough warps for ~16 resident 256-thread blocks per SM, a few tokens each
+  // one 32-token group per warp (more when the batch is large), so that ~16 blocks of
+  // 256 threads stay resident per SM
   const long long warps_target = (long long)sm_count() * 64 * 4;
-  int tpw = (int)max(1LL, (a.T + warps_target - 1) / warps_target);
+  int tpw = 32 * (int)max(1LL, (a.T + 32 * warps_target - 1) / (32 * warps_target));
   long long warps = (a.T + tpw - 1) / tpw;
   long long blocks = (warps + 7) / 8;
   if (a.dtype == GENRANK_BF16) {

@@ -113,14 +113,12 @@ __global__ void __launch_bounds__(256) k_token_meta(
   }
 }
 
-// Warp-per-token gather-sum.  Each warp owns a contiguous run of tokens, finds
-// the user of its first token with a 32-way search of seq_offsets, then walks
-// forward.  Rows are moved as 16-byte vectors; the five rows are summed in fp32
-// and rounded once.
-// One warp per group of 32 tokens: each lane loads one token's ids (coalesced) and
-// the warp gathers the tokens' five rows with 16-byte vector loads, the row indices
-// broadcast from their lanes by shuffles, two tokens' loads in flight together.
-// At most 64 registers per thread keep four blocks resident per SM.
+// Gather-sum, one warp per group of 32 tokens: the warp finds the user of its first
+// token with a 32-way search of seq_offsets, each lane loads one token's ids
+// (coalesced) and walks to that token's user, then the warp gathers the tokens' five
+// rows with 16-byte vector loads, the row indices broadcast from their lanes by
+// shuffles, two tokens' loads in flight together.  The rows are summed in fp32 and
+// rounded once.  At most 64 registers per thread keep four blocks resident per SM.
 template <typename T>
 __global__ void __launch_bounds__(256, 4) k_embed_fwd(
     int B, long long Ttok, const int32_t* __restrict__ off, const int32_t* __restrict__ hist_len,

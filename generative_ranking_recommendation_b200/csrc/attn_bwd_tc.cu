@@ -17,11 +17,12 @@
 //   * Warp 1 loads K, V once per record and Q, dO, lse2, D per query tile (TMA,
 //     128B swizzle, no multicast; bulk copies for the per-row terms).
 //   * Warp 0 (one thread) issues tcgen05.mma: S^T = K Q^T and dP^T = V dO^T into
-//     TMEM; after the softmax warps have written P^T and dS^T (bf16, shared memory,
-//     UMMA 128B-swizzled K-major layout), dV += P^T dO and dK += dS^T Q accumulate in
-//     TMEM, and dQ_part = dS K is formed from the same dS^T buffer read as an
-//     MN-major operand.  The next tile's S^T, dP^T are issued before this tile's
-//     gradient MMAs.
+//     TMEM.  The softmax warps write P^T (bf16) into TMEM over the S^T columns they
+//     have read and dS^T into shared memory (UMMA 128B-swizzled K-major layout, two
+//     buffers).  Then dV += P^T dO (P^T from TMEM) is issued, the next tile's S^T,
+//     dP^T after it (they overwrite P^T, in order), and dK += dS^T Q and
+//     dQ_part = dS K (dS^T read as an MN-major operand) last, so the softmax of the
+//     next tile waits only for dV and its own S^T, dP^T.
 //   * Warps 2-9 (two threads per key row, each on one half of the query columns,
 //     TMEM access shape 16x32bx2, so two of these warps share each SM
 //     sub-partition) compute P^T and dS^T.
@@ -58,16 +59,15 @@ constexpr uint32_t kOffQ = kOffV + 2 * kTileBytes;     // 2 stages
 constexpr uint32_t kOffDO = kOffQ + 2 * kTileBytes;    // 2 stages
 constexpr uint32_t kOffL2 = kOffDO + 2 * kTileBytes;   // lse2, 2 stages
 constexpr uint32_t kOffD = kOffL2 + 2 * kRowBytes;     // D, 2 stages
-constexpr uint32_t kOffP = kOffD + 2 * kRowBytes;      // P^T
-constexpr uint32_t kOffDS = kOffP + kPSBytes;          // dS^T
-constexpr uint32_t kOffBar = kOffDS + kPSBytes;
+constexpr uint32_t kOffDS = kOffD + 2 * kRowBytes;     // dS^T, 2 buffers
+constexpr uint32_t kOffBar = kOffDS + 2 * kPSBytes;
 constexpr uint32_t kNumBars = 18;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
 
 // tensor memory
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;     // S^T  (keys x queries, fp32)
+constexpr uint32_t kColS = 0;     // S^T  (keys x queries, fp32); then P^T over it (bf16)
 constexpr uint32_t kColDP = 128;  // dP^T
 constexpr uint32_t kColDV = 256;  // dV   (keys x dh)
 constexpr uint32_t kColDK = 320;  // dK
@@ -80,7 +80,7 @@ constexpr uint32_t kIdescQ = idesc_bf16_f32(BM, DH, 1, 1);   // dS MN-major; K M
 constexpr size_t kHeaderBytes = 256;
 
 enum Bar { kKVFull = 0, kKVEmpty = 2, kQDFull = 4, kQDEmpty = 6, kSFull = 8, kPFull = 9,
-           kPSFree = 10, kDQFull = 11, kDQEmpty = 13, kDKVFull = 15, kDKVEmpty = 16 };
+           kDSFree = 10, kDQFull = 12, kDQEmpty = 14, kDKVFull = 16, kDKVEmpty = 17 };
 
 struct Params {
   CUtensorMap tq, tk, tv, tdo;
@@ -297,7 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
     }
     mbar_init(&bars[kSFull], 1);
     mbar_init(&bars[kPFull], kSoftmaxWarps);
-    mbar_init(&bars[kPSFree], 1);
+    mbar_init(&bars[kDSFree], 1);
+    mbar_init(&bars[kDSFree + 1], 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -359,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
     // ---------------------------------------------------------------- MMA issuer
     const uint32_t sK = smem_u32(smem + kOffK), sV = smem_u32(smem + kOffV),
                    sQ = smem_u32(smem + kOffQ), sDO = smem_u32(smem + kOffDO),
-                   sP = smem_u32(smem + kOffP), sDS = smem_u32(smem + kOffDS);
+                   sDS = smem_u32(smem + kOffDS);
     auto issue_sdp = [&](int gg, int kvs) {
       const int st = gg & 1;
 #pragma unroll
@@ -395,7 +396,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
           break;
         }
         tc_fence_after();
-        // the next query tile's S^T, dP^T first: the softmax warps need them next
+        // the record's first dV, dK overwrite the accumulators: the previous record's
+        // dV, dK must have been read out
+        if (t == 0 && !mbar_wait(&bars[kDKVEmpty], parity(it) ^ 1u, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // dV += P^T dO with P^T read from TMEM, where the softmax wrote it over the S^T
+        // columns it had read: queries [16k, 16k+16) at column 64 (k / 4) + 8 (k % 4)
+#pragma unroll
+        for (int k = 0; k < BM / 16; ++k) {
+          const uint64_t bdo =
+              smem_desc_sw128(sDO + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
+          mma_bf16_ts(tmem + kColDV, tmem + kColS + 64 * (k >> 2) + 8 * (k & 3), bdo, kIdescKV,
+                      (t > 0 || k > 0) ? 1u : 0u);
+        }
+        // then the next query tile's S^T, dP^T (after dV has read P^T: in order)
         if (t + 1 < rc.nq) {
           if (!mbar_wait(&bars[kQDFull + ((g + 1) & 1)], parity((g + 1) >> 1), abort_flag,
                          a.err)) {
@@ -405,28 +422,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
           tc_fence_after();
           issue_sdp(g + 1, kvs);
         }
-        // the record's first dV, dK overwrite the accumulators: the previous record's
-        // dV, dK must have been read out
-        if (t == 0 && !mbar_wait(&bars[kDKVEmpty], parity(it) ^ 1u, abort_flag, a.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // dV += P^T dO ; dK += dS^T Q   (K = 128 queries, 8 steps)
-#pragma unroll
-        for (int k = 0; k < BM / 16; ++k) {
-          const uint32_t aoff = (k >> 2) * (BM * 128) + (k & 3) * 32;
-          const uint64_t bdo =
-              smem_desc_sw128(sDO + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
-          mma_bf16_ss(tmem + kColDV, smem_desc_sw128(sP + aoff, 16, 1024), bdo, kIdescKV,
-                      (t > 0 || k > 0) ? 1u : 0u);
-        }
+        // dK += dS^T Q   (K = 128 queries, 8 steps)
+        const uint32_t sDSb = sDS + (g & 1) * kPSBytes;
 #pragma unroll
         for (int k = 0; k < BM / 16; ++k) {
           const uint32_t aoff = (k >> 2) * (BM * 128) + (k & 3) * 32;
           const uint64_t bq =
               smem_desc_sw128(sQ + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
-          mma_bf16_ss(tmem + kColDK, smem_desc_sw128(sDS + aoff, 16, 1024), bq, kIdescKV,
+          mma_bf16_ss(tmem + kColDK, smem_desc_sw128(sDSb + aoff, 16, 1024), bq, kIdescKV,
                       (t > 0 || k > 0) ? 1u : 0u);
         }
         // dQ_part = dS K  (M = queries read from dS^T as MN-major, K = 128 keys)
@@ -438,13 +441,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < BM / 16; ++k) {
-          const uint64_t ads = smem_desc_sw128(sDS + k * 16 * 128, BM * 128, 1024);
+          const uint64_t ads = smem_desc_sw128(sDSb + k * 16 * 128, BM * 128, 1024);
           const uint64_t bk =
               smem_desc_sw128(sK + kvs * kTileBytes + k * 16 * 128, kTileBytes, 1024);
           mma_bf16_ss(tmem + kColDQ + db * DH, ads, bk, kIdescQ, k > 0 ? 1u : 0u);
         }
         mma_commit(&bars[kDQFull + db]);
-        mma_commit(&bars[kPSFree]);
+        mma_commit(&bars[kDSFree + (g & 1)]);
         mma_commit(&bars[kQDEmpty + st]);
       }
       if (!ok) break;
@@ -461,7 +464,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
     const float scale_log2 = a.scale * kLog2e;
     const float* sL2 = reinterpret_cast<const float*>(smem + kOffL2);
     const float* sD = reinterpret_cast<const float*>(smem + kOffD);
-    uint8_t* sP = smem + kOffP;
     uint8_t* sDS = smem + kOffDS;
     int g = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
@@ -475,9 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
       for (int t = 0; t < rc.nq; ++t, ++g) {
         const int st = g & 1;
         const int q0 = rc.k0 + t * BM;
+        // S^T of this tile was issued after the previous dV, so once it is here the
+        // P^T columns are free too
         if (!wait_warp(&bars[kSFull], parity(g), abort_flag, a.err) ||
-            !wait_warp(&bars[kQDFull + st], parity(g >> 1), abort_flag, a.err) ||
-            (g > 0 && !wait_warp(&bars[kPSFree], parity(g - 1), abort_flag, a.err))) {
+            !wait_warp(&bars[kQDFull + st], parity(g >> 1), abort_flag, a.err)) {
           ok = false;
           break;
         }
@@ -493,6 +496,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
         tmem_ld_half16_async<64>(lane_base + kColDP, da);
         tmem_ld_wait(sa);
         tmem_ld_wait(da);
+        // this dS^T buffer was last read by dK, dQ of tile g - 2
+        if (!wait_warp(&bars[kDSFree + st], parity(g >> 1) ^ 1u, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sDSb = sDS + st * kPSBytes;
         auto chunk = [&](const uint32_t (&sv)[16], const uint32_t (&dp)[16], int c0) {
           uint32_t pk[8], dk[8];
 #pragma unroll
@@ -511,8 +520,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
             pk[c / 2] = pack_bf16(p2[0], p2[1]);
             dk[c / 2] = pack_bf16(ds2[0], ds2[1]);
           }
-          store_row_chunk16(sP, r, 64 * hq + c0, pk);
-          store_row_chunk16(sDS, r, 64 * hq + c0, dk);
+          // P^T over the S^T columns already read (16x32bx2: the upper half at +64)
+          tmem_st_half8_nowait<64>(lane_base + kColS + c0 / 2, pk);
+          store_row_chunk16(sDSb, r, 64 * hq + c0, dk);
         };
 #pragma unroll
         for (int c0 = 0; c0 < 64; c0 += 32) {
@@ -531,6 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
             tmem_ld_wait(da);
           }
         }
+        tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();

@@ -502,23 +502,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
           break;
         }
         uint8_t* sDSb = sDS + st * kPSBytes;
+        // 16 query columns: p = 2^(s scale log2e + c_j - lse2_i) on visible pairs and
+        // ds = p (dP - D_i), with the per-query terms read as 16-byte vectors and the
+        // arithmetic on column pairs (two-wide fp32 instructions)
+        const uint64_t sl2 = f2_pack(scale_log2, scale_log2), cb2 = f2_pack(cbj, cbj);
         auto chunk = [&](const uint32_t (&sv)[16], const uint32_t (&dp)[16], int c0) {
           uint32_t pk[8], dk[8];
 #pragma unroll
-          for (int c = 0; c < 16; c += 2) {
-            float p2[2], ds2[2];
+          for (int c = 0; c < 16; c += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(l2 + c0 + c);
+            const float4 d4 = *reinterpret_cast<const float4*>(dd + c0 + c);
+            const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                        sl2, f2_sub(cb2, f2_pack(l4.x, l4.y)));
+            const uint64_t x23 =
+                f2_fma(f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), sl2,
+                       f2_sub(cb2, f2_pack(l4.z, l4.w)));
+            float x[4], p[4];
+            f2_unpack(x01, x[0], x[1]);
+            f2_unpack(x23, x[2], x[3]);
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
+            for (int e = 0; e < 4; ++e) {
               const int i = qbase + c0 + c + e;
-              const bool vis = key && i >= ilo && i < ihi;
-              const float x =
-                  fmaf(__uint_as_float(sv[c + e]), scale_log2, cbj - l2[c0 + c + e]);
-              const float p = vis ? ex2(x) : 0.f;
-              p2[e] = p;
-              ds2[e] = p * (__uint_as_float(dp[c + e]) - dd[c0 + c + e]);
+              p[e] = (key && i >= ilo && i < ihi) ? ex2(x[e]) : 0.f;
             }
-            pk[c / 2] = pack_bf16(p2[0], p2[1]);
-            dk[c / 2] = pack_bf16(ds2[0], ds2[1]);
+            const uint64_t p01 = f2_pack(p[0], p[1]), p23 = f2_pack(p[2], p[3]);
+            const uint64_t ds01 = f2_mul(
+                p01, f2_sub(f2_pack(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
+                            f2_pack(d4.x, d4.y)));
+            const uint64_t ds23 = f2_mul(
+                p23, f2_sub(f2_pack(__uint_as_float(dp[c + 2]), __uint_as_float(dp[c + 3])),
+                            f2_pack(d4.z, d4.w)));
+            float ds[4];
+            f2_unpack(ds01, ds[0], ds[1]);
+            f2_unpack(ds23, ds[2], ds[3]);
+            pk[c / 2] = pack_bf16(p[0], p[1]);
+            pk[c / 2 + 1] = pack_bf16(p[2], p[3]);
+            dk[c / 2] = pack_bf16(ds[0], ds[1]);
+            dk[c / 2 + 1] = pack_bf16(ds[2], ds[3]);
           }
           // P^T over the S^T columns already read (16x32bx2: the upper half at +64)
           tmem_st_half8_nowait<64>(lane_base + kColS + c0 / 2, pk);

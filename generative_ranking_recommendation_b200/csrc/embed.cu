@@ -250,56 +250,76 @@ __global__ void __launch_bounds__(1024) k_embed_bwd(
   const bool col_ok = col < d;
   const long long tend = min(Ttok, (long long)off[B]);
   const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const long long t0 = warp * tokens_per_warp;
-  if (t0 < tend) {
-    const long long t1 = min(tend, t0 + tokens_per_warp);
+  for (long long t0 = warp * tokens_per_warp; t0 < min(tend, (warp + 1) * tokens_per_warp);
+       t0 += 32) {
+    // one token per lane: its owner and its five row indices (coalesced id loads)
+    const long long t = t0 + lane;
     int u = warp_find_user(off, B, t0);
-    long long u_beg = off[u], u_end = off[u + 1];
-    int n = hist_len[u];
-    for (long long t = t0; t < t1; ++t) {
-      while (t >= u_end && u < B - 1) {
-        ++u;
-        u_beg = u_end;
-        u_end = off[u + 1];
-        n = hist_len[u];
-      }
-      const bool cand = (t - u_beg) >= n;
-      long long it = item_ids[t];
-      int a = cand ? n_action : action_ids[t];
-      int p = pos[t], r = req_idx[t], b = rt_bucket[t];
-      bool bad = it < 0 || it >= n_item || a < 0 || a > n_action || p < 0 || p >= n_pos ||
-                 r < 0 || r >= n_ri || b < 0 || b >= n_rt;
+    long long it = -1;
+    int a = 0, p = 0, r = 0, b = 0;
+    if (t < tend) {
+      while (u < B - 1 && t >= off[u + 1]) ++u;
+      const bool cand = (t - off[u]) >= hist_len[u];
+      it = item_ids[t];
+      a = cand ? n_action : action_ids[t];
+      p = pos[t];
+      r = req_idx[t];
+      b = rt_bucket[t];
+      const bool bad = it < 0 || it >= n_item || a < 0 || a > n_action || p < 0 ||
+                       p >= n_pos || r < 0 || r >= n_ri || b < 0 || b >= n_rt;
       if (bad) {
-        if (lane == 0) flag(err, GENRANK_DERR_INDEX);
-        continue;
+        flag(err, GENRANK_DERR_INDEX);
+        it = -1;  // skipped below
       }
-      if (!col_ok) continue;
-      float g0, g1;
-      if (sizeof(T) == 2) {
-        uint32_t w = *reinterpret_cast<const uint32_t*>(dE + t * d + col);
-        g0 = bf16_lo(w);
-        g1 = bf16_hi(w);
-      } else {
-        float2 w = *reinterpret_cast<const float2*>(dE + t * d + col);
-        g0 = w.x;
-        g1 = w.y;
+    }
+    const int nt = (int)min(32LL, tend - t0);
+    // the warp adds the tokens' gradient slices, two tokens' dE loads in flight
+    for (int k = 0; k < nt; k += 2) {
+      long long itq[2];
+      int aq[2], pq[2], rq[2], bq[2];
+      float g0[2], g1[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int src = min(k + q, nt - 1);
+        itq[q] = __shfl_sync(0xffffffffu, it, src);
+        aq[q] = __shfl_sync(0xffffffffu, a, src);
+        pq[q] = __shfl_sync(0xffffffffu, p, src);
+        rq[q] = __shfl_sync(0xffffffffu, r, src);
+        bq[q] = __shfl_sync(0xffffffffu, b, src);
+        g0[q] = g1[q] = 0.f;
+        if (col_ok && itq[q] >= 0 && k + q < nt) {
+          if (sizeof(T) == 2) {
+            const uint32_t w =
+                *reinterpret_cast<const uint32_t*>(dE + (t0 + k + q) * d + col);
+            g0[q] = bf16_lo(w);
+            g1[q] = bf16_hi(w);
+          } else {
+            const float2 w = *reinterpret_cast<const float2*>(dE + (t0 + k + q) * d + col);
+            g0[q] = w.x;
+            g1[q] = w.y;
+          }
+        }
       }
-      red_add_v2(g_item + it * d + col, g0, g1);
-      if (kSmem) {
-        const int cl = 2 * lane;
-        atomicAdd(s_action + a * kBwdCols + cl, g0);
-        atomicAdd(s_action + a * kBwdCols + cl + 1, g1);
-        atomicAdd(s_pos + p * kBwdCols + cl, g0);
-        atomicAdd(s_pos + p * kBwdCols + cl + 1, g1);
-        atomicAdd(s_ri + r * kBwdCols + cl, g0);
-        atomicAdd(s_ri + r * kBwdCols + cl + 1, g1);
-        atomicAdd(s_rt + b * kBwdCols + cl, g0);
-        atomicAdd(s_rt + b * kBwdCols + cl + 1, g1);
-      } else {
-        red_add_v2(g_action + (long long)a * d + col, g0, g1);
-        red_add_v2(g_pos + (long long)p * d + col, g0, g1);
-        red_add_v2(g_ri + (long long)r * d + col, g0, g1);
-        red_add_v2(g_rt + (long long)b * d + col, g0, g1);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (!col_ok || itq[q] < 0 || k + q >= nt) continue;
+        red_add_v2(g_item + itq[q] * d + col, g0[q], g1[q]);
+        if (kSmem) {
+          const int cl = 2 * lane;
+          atomicAdd(s_action + aq[q] * kBwdCols + cl, g0[q]);
+          atomicAdd(s_action + aq[q] * kBwdCols + cl + 1, g1[q]);
+          atomicAdd(s_pos + pq[q] * kBwdCols + cl, g0[q]);
+          atomicAdd(s_pos + pq[q] * kBwdCols + cl + 1, g1[q]);
+          atomicAdd(s_ri + rq[q] * kBwdCols + cl, g0[q]);
+          atomicAdd(s_ri + rq[q] * kBwdCols + cl + 1, g1[q]);
+          atomicAdd(s_rt + bq[q] * kBwdCols + cl, g0[q]);
+          atomicAdd(s_rt + bq[q] * kBwdCols + cl + 1, g1[q]);
+        } else {
+          red_add_v2(g_action + (long long)aq[q] * d + col, g0[q], g1[q]);
+          red_add_v2(g_pos + (long long)pq[q] * d + col, g0[q], g1[q]);
+          red_add_v2(g_ri + (long long)rq[q] * d + col, g0[q], g1[q]);
+          red_add_v2(g_rt + (long long)bq[q] * d + col, g0[q], g1[q]);
+        }
       }
     }
   }
@@ -375,7 +395,8 @@ static int launch_bwd_t(const EmbedBwdArgs& a, cudaStream_t st) {
   // about two waves of one 1024-thread CTA per SM over all slices
   const long long ctas_per_slice = max(1LL, (long long)(2 * sm_count() + slices - 1) / slices);
   const long long warps = ctas_per_slice * 32;
-  const int tpw = (int)max(1LL, (a.T + warps - 1) / warps);
+  // tokens per warp: whole groups of 32 (one token's ids per lane)
+  const int tpw = 32 * (int)max(1LL, (a.T + 32 * warps - 1) / (32 * warps));
   const long long chunks = max(1LL, ((a.T + tpw - 1) / tpw + 31) / 32);
   dim3 grid((unsigned)chunks, (unsigned)slices);
   k_embed_bwd<T, kSmem><<<grid, 1024, smem, st>>>(

@@ -305,13 +305,13 @@ def run_native(args, cfg, world, rank, local):
         attn[k % 2].run()
     torch.cuda.synchronize()
 
-    def timed(fn, n):
+    def timed(fn, n, name="timed_step"):
         """Device time of n calls of fn, L2 flushed before each (events bracket fn only)."""
         ev = []
         for k in range(n):
             flush.zero_()
             s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            torch.cuda.nvtx.range_push("timed_step")
+            torch.cuda.nvtx.range_push(name)
             s.record()
             fn(k)
             e.record()
@@ -327,7 +327,7 @@ def run_native(args, cfg, world, rank, local):
     step_ms = timed(lambda k: steps[k % 2].run(), args.steps)
     clocks = sampler.stop()
     total_ms = sum(step_ms)
-    attn_ms = timed(lambda k: attn[k % 2].run(), args.steps)
+    attn_ms = timed(lambda k: attn[k % 2].run(), args.steps, name="timed_attention")
 
     # ---- end to end through the public API: pinned host inputs -> device -> logits -> host
     host = [DeviceBatch.host_arrays(b) for b in batches]

@@ -16,15 +16,16 @@
 //     candidate); they are visited one 128-row query tile at a time.
 //   * Warp 1 loads K, V once per record and Q, dO, lse2, D per query tile (TMA,
 //     128B swizzle, no multicast; bulk copies for the per-row terms).
-//   * Warp 0 (one thread) issues tcgen05.mma: S^T = K Q^T and dP^T = V dO^T into
-//     TMEM.  The softmax warps write P^T (bf16) into TMEM over the S^T columns they
-//     have read and dS^T into shared memory (UMMA 128B-swizzled K-major layout, two
-//     buffers).  Then dV += P^T dO (P^T from TMEM) is issued, the next tile's S^T,
-//     dP^T after it (they overwrite P^T, in order), and dK += dS^T Q and
-//     dQ_part = dS K (dS^T read as an MN-major operand) last, so the softmax of the
-//     next tile waits only for dV and its own S^T, dP^T.
-//   * Warps 2-9 (two threads per key row, each on one half of the query columns,
-//     TMEM access shape 16x32bx2, so two of these warps share each SM
+//   * Warp 0 (one thread) issues tcgen05.mma.  Each query tile is taken as two halves
+//     of 64 queries: S^T = K Q_x^T and dP^T = V dO_x^T of half x go into TMEM.  The
+//     softmax warps write P^T (bf16) into TMEM over S^T columns they have read and
+//     dS^T into shared memory (UMMA 128B-swizzled K-major layout, two buffers).  When
+//     half x is done, dV += P^T dO_x (P^T from TMEM) and dK += dS^T Q_x are issued,
+//     then half x of the next query tile (of this record or of the next one), which
+//     overwrites P^T in order and runs while the softmax works on the other half.
+//     dQ_part = dS K (dS^T read as an MN-major operand) follows the second half.
+//   * Warps 2-9 (two threads per key row and half, each on 32 of its 64 query
+//     columns, TMEM access shape 16x32bx2, so two of these warps share each SM
 //     sub-partition) compute P^T and dS^T.
 //   * Warps 10-13 (one query row per thread) add each dQ_part into an fp32 dQ
 //     accumulator in global memory with vector reductions and, per record, move dK
@@ -61,7 +62,7 @@ constexpr uint32_t kOffL2 = kOffDO + 2 * kTileBytes;   // lse2, 2 stages
 constexpr uint32_t kOffD = kOffL2 + 2 * kRowBytes;     // D, 2 stages
 constexpr uint32_t kOffDS = kOffD + 2 * kRowBytes;     // dS^T, 2 buffers
 constexpr uint32_t kOffBar = kOffDS + 2 * kPSBytes;
-constexpr uint32_t kNumBars = 18;
+constexpr uint32_t kNumBars = 20;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
 
@@ -73,14 +74,17 @@ constexpr uint32_t kColDV = 256;  // dV   (keys x dh)
 constexpr uint32_t kColDK = 320;  // dK
 constexpr uint32_t kColDQ = 384;  // dQ_part, two buffers of 64 (queries x dh)
 
-constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BM, 0, 0);   // K / V K-major, Q / dO K-major
+constexpr int kQH = BM / 2;  // queries per half tile
+constexpr uint32_t kIdescS = idesc_bf16_f32(BM, kQH, 0, 0);  // K / V K-major, Q / dO K-major
 constexpr uint32_t kIdescKV = idesc_bf16_f32(BM, DH, 0, 1);  // P^T, dS^T K-major; dO, Q MN-major
 constexpr uint32_t kIdescQ = idesc_bf16_f32(BM, DH, 1, 1);   // dS MN-major; K MN-major
 
 constexpr size_t kHeaderBytes = 256;
 
-enum Bar { kKVFull = 0, kKVEmpty = 2, kQDFull = 4, kQDEmpty = 6, kSFull = 8, kPFull = 9,
-           kDSFree = 10, kDQFull = 12, kDQEmpty = 14, kDKVFull = 16, kDKVEmpty = 17 };
+// S^T / dP^T and P^T are handled per query half (64 queries): one S-full and one
+// P-full barrier per half.
+enum Bar { kKVFull = 0, kKVEmpty = 2, kQDFull = 4, kQDEmpty = 6, kSFull = 8, kPFull = 10,
+           kDSFree = 12, kDQFull = 14, kDQEmpty = 16, kDKVFull = 18, kDKVEmpty = 19 };
 
 struct Params {
   CUtensorMap tq, tk, tv, tdo;
@@ -295,8 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
       mbar_init(&bars[kDQFull + i], 1);
       mbar_init(&bars[kDQEmpty + i], 4);  // one arrival per reducing warp
     }
-    mbar_init(&bars[kSFull], 1);
-    mbar_init(&bars[kPFull], kSoftmaxWarps);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars[kSFull + x], 1);
+      mbar_init(&bars[kPFull + x], kSoftmaxWarps);
+    }
     mbar_init(&bars[kDSFree], 1);
     mbar_init(&bars[kDSFree + 1], 1);
     *abort_flag = 0;
@@ -358,39 +364,74 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
     }
   } else if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- MMA issuer
+    // Tiles g = 0, 1, ... run across records; each tile is handled as two query halves
+    // X = 0, 1.  When the softmax has finished half X of tile g, dV and dK take that
+    // half, and half X of the next tile (of this record or of the next one) is issued
+    // at once: it runs while the softmax works on the other half.  dQ of tile g comes
+    // after both halves.
     const uint32_t sK = smem_u32(smem + kOffK), sV = smem_u32(smem + kOffV),
                    sQ = smem_u32(smem + kOffQ), sDO = smem_u32(smem + kOffDO),
                    sDS = smem_u32(smem + kOffDS);
-    auto issue_sdp = [&](int gg, int kvs) {
-      const int st = gg & 1;
+    // S^T = K Q_X^T and dP^T = V dO_X^T for query half X of tile gg (keys of stage kvs)
+    auto issue_sdp = [&](int gg, int kvs, int x) {
+      const uint32_t qoff = (gg & 1) * kTileBytes + x * (kQH * 128);
 #pragma unroll
-      for (int k = 0; k < DH / 16; ++k) {
-        mma_bf16_ss(tmem + kColS, smem_desc_sw128(sK + kvs * kTileBytes + k * 32, 16, 1024),
-                    smem_desc_sw128(sQ + st * kTileBytes + k * 32, 16, 1024), kIdescS,
-                    k > 0 ? 1u : 0u);
+      for (int k = 0; k < DH / 16; ++k)
+        mma_bf16_ss(tmem + kColS + kQH * x,
+                    smem_desc_sw128(sK + kvs * kTileBytes + k * 32, 16, 1024),
+                    smem_desc_sw128(sQ + qoff + k * 32, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
+#pragma unroll
+      for (int k = 0; k < DH / 16; ++k)
+        mma_bf16_ss(tmem + kColDP + kQH * x,
+                    smem_desc_sw128(sV + kvs * kTileBytes + k * 32, 16, 1024),
+                    smem_desc_sw128(sDO + qoff + k * 32, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
+      mma_commit(&bars[kSFull + x]);
+    };
+    // dV += P^T dO_X with P^T read from TMEM, and dK += dS^T Q_X, over query half X
+    // (K = 64 queries).  The softmax wrote P^T over the S^T columns it had read:
+    // queries [16k, 16k + 16) of the half at column 64 x + 32 (k / 2) + 8 (k % 2).
+    auto issue_dvdk = [&](int gg, int x, bool first) {
+      const uint32_t st = gg & 1;
+      const uint32_t sDSb = sDS + st * kPSBytes;
+#pragma unroll
+      for (int k = 0; k < kQH / 16; ++k) {
+        const int kq = (kQH / 16) * x + k;  // 16-query step within the tile
+        const uint64_t bdo =
+            smem_desc_sw128(sDO + st * kTileBytes + kq * 16 * 128, kTileBytes, 1024);
+        mma_bf16_ts(tmem + kColDV, tmem + kColS + kQH * x + 32 * (k >> 1) + 8 * (k & 1), bdo,
+                    kIdescKV, (!first || k > 0) ? 1u : 0u);
       }
 #pragma unroll
-      for (int k = 0; k < DH / 16; ++k) {
-        mma_bf16_ss(tmem + kColDP, smem_desc_sw128(sV + kvs * kTileBytes + k * 32, 16, 1024),
-                    smem_desc_sw128(sDO + st * kTileBytes + k * 32, 16, 1024), kIdescS,
-                    k > 0 ? 1u : 0u);
+      for (int k = 0; k < kQH / 16; ++k) {
+        const int kq = (kQH / 16) * x + k;
+        const uint32_t aoff = x * (BM * 128) + k * 32;
+        const uint64_t bq =
+            smem_desc_sw128(sQ + st * kTileBytes + kq * 16 * 128, kTileBytes, 1024);
+        mma_bf16_ss(tmem + kColDK, smem_desc_sw128(sDSb + aoff, 16, 1024), bq, kIdescKV,
+                    (!first || k > 0) ? 1u : 0u);
       }
-      mma_commit(&bars[kSFull]);
     };
     int it = 0, g = 0;
-    bool ok = true;
-    for (int w = blockIdx.x; w < total && ok && !*abort_flag; w += gridDim.x, ++it) {
+    bool ok = blockIdx.x < total;
+    if (ok) {
+      ok = mbar_wait(&bars[kKVFull], 0u, abort_flag, a.err) &&
+           mbar_wait(&bars[kQDFull], 0u, abort_flag, a.err);
+      if (ok) {
+        tc_fence_after();
+        issue_sdp(0, 0, 0);
+        issue_sdp(0, 0, 1);
+      }
+    }
+    for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
       const Rec rc = load_rec(P, w);
       const int kvs = it & 1;
-      if (!mbar_wait(&bars[kKVFull + kvs], parity(it >> 1), abort_flag, a.err) ||
-          !mbar_wait(&bars[kQDFull + (g & 1)], parity(g >> 1), abort_flag, a.err)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      issue_sdp(g, kvs);
       for (int t = 0; t < rc.nq; ++t, ++g) {
         const int st = g & 1;
+        // the next tile: this record's next query tile, or the next record's first
+        const bool last = t + 1 == rc.nq;
+        const bool has_next = !last || w + (int)gridDim.x < total;
+        const int nkvs = last ? kvs ^ 1 : kvs;
+        // ---- half 0
         if (!mbar_wait(&bars[kPFull], parity(g), abort_flag, a.err)) {
           ok = false;
           break;
@@ -403,62 +444,52 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
           break;
         }
         tc_fence_after();
-        // dV += P^T dO with P^T read from TMEM, where the softmax wrote it over the S^T
-        // columns it had read: queries [16k, 16k+16) at column 64 (k / 4) + 8 (k % 4)
-#pragma unroll
-        for (int k = 0; k < BM / 16; ++k) {
-          const uint64_t bdo =
-              smem_desc_sw128(sDO + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
-          mma_bf16_ts(tmem + kColDV, tmem + kColS + 64 * (k >> 2) + 8 * (k & 3), bdo, kIdescKV,
-                      (t > 0 || k > 0) ? 1u : 0u);
-        }
-        // then the next query tile's S^T, dP^T (after dV has read P^T: in order)
-        if (t + 1 < rc.nq) {
-          if (!mbar_wait(&bars[kQDFull + ((g + 1) & 1)], parity((g + 1) >> 1), abort_flag,
-                         a.err)) {
+        issue_dvdk(g, 0, t == 0);
+        if (has_next) {
+          if ((last && !mbar_wait(&bars[kKVFull + nkvs], parity((it + 1) >> 1), abort_flag,
+                                  a.err)) ||
+              !mbar_wait(&bars[kQDFull + (st ^ 1)], parity((g + 1) >> 1), abort_flag, a.err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_sdp(g + 1, kvs);
+          issue_sdp(g + 1, nkvs, 0);  // after dV has read P^T of half 0 (in order)
         }
-        // dK += dS^T Q   (K = 128 queries, 8 steps)
-        const uint32_t sDSb = sDS + (g & 1) * kPSBytes;
-#pragma unroll
-        for (int k = 0; k < BM / 16; ++k) {
-          const uint32_t aoff = (k >> 2) * (BM * 128) + (k & 3) * 32;
-          const uint64_t bq =
-              smem_desc_sw128(sQ + st * kTileBytes + k * 16 * 128, kTileBytes, 1024);
-          mma_bf16_ss(tmem + kColDK, smem_desc_sw128(sDSb + aoff, 16, 1024), bq, kIdescKV,
-                      (t > 0 || k > 0) ? 1u : 0u);
-        }
-        // dQ_part = dS K  (M = queries read from dS^T as MN-major, K = 128 keys)
-        const int db = g & 1;
-        if (!mbar_wait(&bars[kDQEmpty + db], parity(g >> 1) ^ 1u, abort_flag, a.err)) {
+        // ---- half 1
+        if (!mbar_wait(&bars[kPFull + 1], parity(g), abort_flag, a.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        issue_dvdk(g, 1, false);
+        mma_commit(&bars[kQDEmpty + st]);  // Q, dO of this tile are read for the last time
+        if (last) mma_commit(&bars[kDKVFull]);
+        if (has_next) issue_sdp(g + 1, nkvs, 1);
+        // dQ_part = dS K  (M = queries read from dS^T as MN-major, K = 128 keys)
+        if (!mbar_wait(&bars[kDQEmpty + st], parity(g >> 1) ^ 1u, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sDSb = sDS + st * kPSBytes;
 #pragma unroll
         for (int k = 0; k < BM / 16; ++k) {
           const uint64_t ads = smem_desc_sw128(sDSb + k * 16 * 128, BM * 128, 1024);
           const uint64_t bk =
               smem_desc_sw128(sK + kvs * kTileBytes + k * 16 * 128, kTileBytes, 1024);
-          mma_bf16_ss(tmem + kColDQ + db * DH, ads, bk, kIdescQ, k > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + kColDQ + st * DH, ads, bk, kIdescQ, k > 0 ? 1u : 0u);
         }
-        mma_commit(&bars[kDQFull + db]);
-        mma_commit(&bars[kDSFree + (g & 1)]);
-        mma_commit(&bars[kQDEmpty + st]);
+        mma_commit(&bars[kDQFull + st]);
+        mma_commit(&bars[kDSFree + st]);
+        if (last) mma_commit(&bars[kKVEmpty + kvs]);
       }
-      if (!ok) break;
-      mma_commit(&bars[kKVEmpty + kvs]);
-      mma_commit(&bars[kDKVFull]);
+      if (*abort_flag) ok = false;
     }
   } else if (warp >= 2 && warp < 2 + kSoftmaxWarps) {
     // ---------------------------------------------------------------- softmax (key rows)
     const int quad = warp & 3;              // TMEM lane quadrant of the warp
     const int rh = (warp - 2) >> 2;         // upper or lower 16 lanes of the quadrant
-    const int hq = lane >> 4;               // half of the query columns
+    const int hq = lane >> 4;               // which 32 queries of each half
     const int r = quad * 32 + rh * 16 + (lane & 15);  // key row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32 + rh * 16) << 16);
     const float scale_log2 = a.scale * kLog2e;
@@ -473,99 +504,96 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
       const int j = rc.k0 + r;  // this thread's key (local index)
       const bool key = j < rc.n;
       const float cbj = key ? P.cbias[(long long)rc.h * P.Tp + rc.spad + j] : 0.f;
+      const uint64_t sl2 = f2_pack(scale_log2, scale_log2), cb2 = f2_pack(cbj, cbj);
       bool ok = true;
-      for (int t = 0; t < rc.nq; ++t, ++g) {
+      for (int t = 0; t < rc.nq && ok; ++t, ++g) {
         const int st = g & 1;
         const int q0 = rc.k0 + t * BM;
-        // S^T of this tile was issued after the previous dV, so once it is here the
-        // P^T columns are free too
-        if (!wait_warp(&bars[kSFull], parity(g), abort_flag, a.err) ||
-            !wait_warp(&bars[kQDFull + st], parity(g >> 1), abort_flag, a.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         // visible iff key valid, query row inside the user and i >= j
         const int ilo = max(j, q0);  // first visible query (local index)
         const int ihi = rc.L;        // one past the last
-        const float* l2 = sL2 + st * BM + 64 * hq;
-        const float* dd = sD + st * BM + 64 * hq;
-        const int qbase = q0 + 64 * hq;  // this thread's first query column
-        uint32_t sa[16], da[16], sb[16], db[16];
-        tmem_ld_half16_async<64>(lane_base + kColS, sa);
-        tmem_ld_half16_async<64>(lane_base + kColDP, da);
-        tmem_ld_wait(sa);
-        tmem_ld_wait(da);
-        // this dS^T buffer was last read by dK, dQ of tile g - 2
-        if (!wait_warp(&bars[kDSFree + st], parity(g >> 1) ^ 1u, abort_flag, a.err)) {
-          ok = false;
-          break;
-        }
         uint8_t* sDSb = sDS + st * kPSBytes;
-        // 16 query columns: p = 2^(s scale log2e + c_j - lse2_i) on visible pairs and
-        // ds = p (dP - D_i), with the per-query terms read as 16-byte vectors and the
-        // arithmetic on column pairs (two-wide fp32 instructions)
-        const uint64_t sl2 = f2_pack(scale_log2, scale_log2), cb2 = f2_pack(cbj, cbj);
-        auto chunk = [&](const uint32_t (&sv)[16], const uint32_t (&dp)[16], int c0) {
-          uint32_t pk[8], dk[8];
-#pragma unroll
-          for (int c = 0; c < 16; c += 4) {
-            const float4 l4 = *reinterpret_cast<const float4*>(l2 + c0 + c);
-            const float4 d4 = *reinterpret_cast<const float4*>(dd + c0 + c);
-            const uint64_t x01 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
-                                        sl2, f2_sub(cb2, f2_pack(l4.x, l4.y)));
-            const uint64_t x23 =
-                f2_fma(f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), sl2,
-                       f2_sub(cb2, f2_pack(l4.z, l4.w)));
-            float x[4], p[4];
-            f2_unpack(x01, x[0], x[1]);
-            f2_unpack(x23, x[2], x[3]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int i = qbase + c0 + c + e;
-              p[e] = (key && i >= ilo && i < ihi) ? ex2(x[e]) : 0.f;
-            }
-            const uint64_t p01 = f2_pack(p[0], p[1]), p23 = f2_pack(p[2], p[3]);
-            const uint64_t ds01 = f2_mul(
-                p01, f2_sub(f2_pack(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
-                            f2_pack(d4.x, d4.y)));
-            const uint64_t ds23 = f2_mul(
-                p23, f2_sub(f2_pack(__uint_as_float(dp[c + 2]), __uint_as_float(dp[c + 3])),
-                            f2_pack(d4.z, d4.w)));
-            float ds[4];
-            f2_unpack(ds01, ds[0], ds[1]);
-            f2_unpack(ds23, ds[2], ds[3]);
-            pk[c / 2] = pack_bf16(p[0], p[1]);
-            pk[c / 2 + 1] = pack_bf16(p[2], p[3]);
-            dk[c / 2] = pack_bf16(ds[0], ds[1]);
-            dk[c / 2 + 1] = pack_bf16(ds[2], ds[3]);
+        for (int x = 0; x < 2; ++x) {
+          // half x of S^T was issued after dV had read this half's previous P^T
+          if (!wait_warp(&bars[kSFull + x], parity(g), abort_flag, a.err) ||
+              (x == 0 && !wait_warp(&bars[kQDFull + st], parity(g >> 1), abort_flag, a.err))) {
+            ok = false;
+            break;
           }
-          // P^T over the S^T columns already read (16x32bx2: the upper half at +64)
-          tmem_st_half8_nowait<64>(lane_base + kColS + c0 / 2, pk);
-          store_row_chunk16(sDSb, r, 64 * hq + c0, dk);
-        };
+          tc_fence_after();
+          const int qc = kQH * x + 32 * hq;  // this thread's first query column in the tile
+          const float* l2 = sL2 + st * BM + qc;
+          const float* dd = sD + st * BM + qc;
+          const int qbase = q0 + qc;
+          const uint32_t s_addr = lane_base + kColS + kQH * x;
+          const uint32_t dp_addr = lane_base + kColDP + kQH * x;
+          uint32_t sa[16], da[16], sb[16], db[16];
+          tmem_ld_half16_async<32>(s_addr, sa);
+          tmem_ld_half16_async<32>(dp_addr, da);
+          tmem_ld_wait(sa);
+          tmem_ld_wait(da);
+          tmem_ld_half16_async<32>(s_addr + 16, sb);
+          tmem_ld_half16_async<32>(dp_addr + 16, db);
+          // this dS^T buffer was last read by dK, dQ of tile g - 2
+          if (x == 0 &&
+              !wait_warp(&bars[kDSFree + st], parity(g >> 1) ^ 1u, abort_flag, a.err)) {
+            tmem_ld_wait(sb);
+            ok = false;
+            break;
+          }
+          // 16 query columns: p = 2^(s scale log2e + c_j - lse2_i) on visible pairs and
+          // ds = p (dP - D_i), with the per-query terms read as 16-byte vectors and the
+          // arithmetic on column pairs (two-wide fp32 instructions).  P^T goes over the
+          // first 16 S^T columns this thread has read (16x32bx2: the upper lanes at
+          // +32), dS^T to shared memory.
+          auto chunk = [&](const uint32_t (&sv)[16], const uint32_t (&dp)[16], int c0) {
+            uint32_t pk[8], dk[8];
 #pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          tmem_ld_half16_async<64>(lane_base + kColS + c0 + 16, sb);
-          tmem_ld_half16_async<64>(lane_base + kColDP + c0 + 16, db);
-          chunk(sa, da, c0);
+            for (int c = 0; c < 16; c += 4) {
+              const float4 l4 = *reinterpret_cast<const float4*>(l2 + c0 + c);
+              const float4 d4 = *reinterpret_cast<const float4*>(dd + c0 + c);
+              const uint64_t x01 =
+                  f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2,
+                         f2_sub(cb2, f2_pack(l4.x, l4.y)));
+              const uint64_t x23 =
+                  f2_fma(f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), sl2,
+                         f2_sub(cb2, f2_pack(l4.z, l4.w)));
+              float xv[4], p[4];
+              f2_unpack(x01, xv[0], xv[1]);
+              f2_unpack(x23, xv[2], xv[3]);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int i = qbase + c0 + c + e;
+                p[e] = (key && i >= ilo && i < ihi) ? ex2(xv[e]) : 0.f;
+              }
+              const uint64_t p01 = f2_pack(p[0], p[1]), p23 = f2_pack(p[2], p[3]);
+              const uint64_t ds01 = f2_mul(
+                  p01, f2_sub(f2_pack(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
+                              f2_pack(d4.x, d4.y)));
+              const uint64_t ds23 = f2_mul(
+                  p23, f2_sub(f2_pack(__uint_as_float(dp[c + 2]), __uint_as_float(dp[c + 3])),
+                              f2_pack(d4.z, d4.w)));
+              float ds[4];
+              f2_unpack(ds01, ds[0], ds[1]);
+              f2_unpack(ds23, ds[2], ds[3]);
+              pk[c / 2] = pack_bf16(p[0], p[1]);
+              pk[c / 2 + 1] = pack_bf16(p[2], p[3]);
+              dk[c / 2] = pack_bf16(ds[0], ds[1]);
+              dk[c / 2 + 1] = pack_bf16(ds[2], ds[3]);
+            }
+            tmem_st_half8_nowait<32>(s_addr + c0 / 2, pk);
+            store_row_chunk16(sDSb, r, qc + c0, dk);
+          };
+          chunk(sa, da, 0);  // stores to columns [0, 8): read, not in flight
           tmem_ld_wait(sb);
           tmem_ld_wait(db);
-          if (c0 + 32 < 64) {
-            tmem_ld_half16_async<64>(lane_base + kColS + c0 + 32, sa);
-            tmem_ld_half16_async<64>(lane_base + kColDP + c0 + 32, da);
-          }
-          chunk(sb, db, c0 + 16);
-          if (c0 + 32 < 64) {
-            tmem_ld_wait(sa);
-            tmem_ld_wait(da);
-          }
+          chunk(sb, db, 16);  // stores to columns [8, 16)
+          tmem_wait_st();
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[kPFull + x]);
         }
-        tmem_wait_st();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kPFull]);
       }
       if (!ok) break;
     }
@@ -580,6 +608,42 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
       const Rec rc = load_rec(P, w);
       bool ok = true;
       for (int t = 0; t < rc.nq; ++t, ++g) {
+        if (t + 1 == rc.nq) {
+          // the record's dK (times scale) and dV, key row qlane, once its last dV, dK
+          // MMAs are done (before its last dQ_part); the accumulators are released
+          // before the last stores
+          if (!wait_warp(&bars[kDKVFull], parity(it), abort_flag, a.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int j = rc.k0 + qlane;
+          const bool key = j < rc.n;
+          const long long tok = (long long)rc.s + j;
+          __nv_bfloat16* dkp = (__nv_bfloat16*)a.dk + tok * a.tok_stride + rc.h * DH;
+          __nv_bfloat16* dvp = (__nv_bfloat16*)a.dv + tok * a.tok_stride + rc.h * DH;
+#pragma unroll 1
+          for (int c0 = 0; c0 < DH; c0 += 32) {
+            float dvr[32], dkr[32];
+            tmem_ld32(tmem + lane_base + kColDV + c0, dvr);
+            tmem_ld32(tmem + lane_base + kColDK + c0, dkr);
+            if (c0 + 32 == DH) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars[kDKVEmpty]);
+            }
+            if (key) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 8) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = dkr[c + e] * a.scale;
+                *reinterpret_cast<uint4*>(dkp + c0 + c) = Elem<__nv_bfloat16>::pack(f);
+                *reinterpret_cast<uint4*>(dvp + c0 + c) = Elem<__nv_bfloat16>::pack(dvr + c);
+              }
+            }
+          }
+        }
         const int db = g & 1;
         if (!wait_warp(&bars[kDQFull + db], parity(g >> 1), abort_flag, a.err)) {
           ok = false;
@@ -602,36 +666,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
         }
       }
       if (!ok) break;
-      // the record's dK (times scale) and dV, key row qlane, once its last gradient MMAs
-      // are done; the accumulators are released before the last stores
-      if (!wait_warp(&bars[kDKVFull], parity(it), abort_flag, a.err)) break;
-      tc_fence_after();
-      const int j = rc.k0 + qlane;
-      const bool key = j < rc.n;
-      const long long tok = (long long)rc.s + j;
-      __nv_bfloat16* dkp = (__nv_bfloat16*)a.dk + tok * a.tok_stride + rc.h * DH;
-      __nv_bfloat16* dvp = (__nv_bfloat16*)a.dv + tok * a.tok_stride + rc.h * DH;
-#pragma unroll 1
-      for (int c0 = 0; c0 < DH; c0 += 32) {
-        float dvr[32], dkr[32];
-        tmem_ld32(tmem + lane_base + kColDV + c0, dvr);
-        tmem_ld32(tmem + lane_base + kColDK + c0, dkr);
-        if (c0 + 32 == DH) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars[kDKVEmpty]);
-        }
-        if (key) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            float f[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = dkr[c + e] * a.scale;
-            *reinterpret_cast<uint4*>(dkp + c0 + c) = Elem<__nv_bfloat16>::pack(f);
-            *reinterpret_cast<uint4*>(dvp + c0 + c) = Elem<__nv_bfloat16>::pack(dvr + c);
-          }
-        }
-      }
     }
   }
 
@@ -778,7 +812,11 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   p.dsum = (float*)(rows + 2 * rb);
   p.dqacc = (float*)(rows + 3 * rb);
   p.Tp = scratch_tp(a.T, a.B);
-  if (cudaMemsetAsync(p.dqacc, 0, (size_t)a.T * a.H * DH * sizeof(float), st) != cudaSuccess)
+  // D and the dQ accumulator are adjacent: one memset zeroes both.  A query tile reads D
+  // past its user's last row (the gap before the next user's segment), where a masked
+  // pair's ds = p (dP - D) with p = 0 must stay 0 whatever the workspace held.
+  if (cudaMemsetAsync(rows + 2 * rb, 0, rb + (size_t)a.T * a.H * DH * sizeof(float), st) !=
+      cudaSuccess)
     return GENRANK_ERR_CUDA;
   if (a.T > 0 && cudaMemsetAsync(tok_user, 0xff, (size_t)a.T * 4, st) != cudaSuccess)
     return GENRANK_ERR_CUDA;

@@ -35,8 +35,10 @@ def _dev(x, dtype=None):
     return t.to("cuda", dtype=dtype) if dtype is not None else t.to("cuda")
 
 
-def run_fwd(G, cfg, batch, pos, qkv, need_lse=True):
-    """qkv: [T, 3, H, dh] host array; returns (O [T,H,dh], LSE [H,T]) as float64 numpy."""
+def run_fwd(G, cfg, batch, pos, qkv, need_lse=True, poison=False):
+    """qkv: [T, 3, H, dh] host array; returns (O [T,H,dh], LSE [H,T]) as float64 numpy.
+
+    poison: fill the workspace with 0xff bytes (NaN as fp32) before the call."""
     T, H, dh = batch.T, cfg.H, cfg.dh
     d = H * dh
     tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
@@ -48,6 +50,8 @@ def run_fwd(G, cfg, batch, pos, qkv, need_lse=True):
     msl = int(np.max(np.diff(batch.seq_offsets)))
     ws = torch.empty(G.attn_workspace_size(batch.B, T, H, dh, msl, False), dtype=torch.uint8,
                      device="cuda")
+    if poison:
+        ws.fill_(0xFF)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     sp, st = G.alibi_slopes(H)
     G.attn_fwd(off, hl, msl, q, q[:, d:], q[:, 2 * d:], 3 * d, H, dh, pos_t, ts_t, sp, st,
@@ -97,6 +101,18 @@ def test_fwd_edge_cases(G, dtype, H, dh):
     pos, _, _ = ref.meta(batch)
     qkv = make_qkv(cfg, batch.T, seed=5)
     O, L = run_fwd(G, cfg, batch, pos, qkv)
+    Or, Lr = ref.attn(qkv[:, 0], qkv[:, 1], qkv[:, 2], batch, pos)
+    _check(cfg, O, L, Or, Lr, np.arange(batch.T))
+
+
+def test_fwd_workspace_contents_do_not_matter(G):
+    """The ragged edge cases with the workspace filled with NaN bit patterns."""
+    cfg = CONFIGS["c1"].with_(B=len(EDGE_USERS), H=4, dh=64, dtype="bf16")
+    batch = make_batch(cfg, hist_override=[n for n, _ in EDGE_USERS],
+                       m_override=[m for _, m in EDGE_USERS])
+    pos, _, _ = ref.meta(batch)
+    qkv = make_qkv(cfg, batch.T, seed=6)
+    O, L = run_fwd(G, cfg, batch, pos, qkv, poison=True)
     Or, Lr = ref.attn(qkv[:, 0], qkv[:, 1], qkv[:, 2], batch, pos)
     _check(cfg, O, L, Or, Lr, np.arange(batch.T))
 
@@ -180,7 +196,7 @@ def test_fwd_device_error_flags(G):
 # ------------------------------------------------------------------------------------------
 # backward
 # ------------------------------------------------------------------------------------------
-def run_bwd(G, cfg, batch, pos, qkv, dO):
+def run_bwd(G, cfg, batch, pos, qkv, dO, poison=False):
     T, H, dh = batch.T, cfg.H, cfg.dh
     d = H * dh
     tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
@@ -194,12 +210,16 @@ def run_bwd(G, cfg, batch, pos, qkv, dO):
     sp, st = G.alibi_slopes(H)
     wsf = torch.empty(G.attn_workspace_size(batch.B, T, H, dh, msl, False), dtype=torch.uint8,
                       device="cuda")
+    if poison:
+        wsf.fill_(0xFF)
     G.attn_fwd(off, hl, msl, q, q[:, d:], q[:, 2 * d:], 3 * d, H, dh, pos_t, ts_t, sp, st,
                1.0 / math.sqrt(dh), o, d, lse, wsf, err, T=T)
     g = _dev(dO.reshape(T, d), tdt)
     dq = torch.empty_like(q)
     wsb = torch.empty(G.attn_workspace_size(batch.B, T, H, dh, msl, True), dtype=torch.uint8,
                       device="cuda")
+    if poison:
+        wsb.fill_(0xFF)
     G.attn_bwd(off, hl, msl, q, q[:, d:], q[:, 2 * d:], 3 * d, H, dh, pos_t, ts_t, sp, st,
                1.0 / math.sqrt(dh), o, g, d, lse, dq, dq[:, d:], dq[:, 2 * d:], wsb, err, T=T)
     assert G.check_error(err) == 0
@@ -223,6 +243,20 @@ def test_bwd_parity(G, name, B):
     qkv = make_qkv(cfg, batch.T, seed=21)
     dO = make_qkv(cfg, batch.T, seed=22, n=1)[:, 0]
     got = run_bwd(G, cfg, batch, pos, qkv, dO)
+    want = ref.attn_bwd(qkv[:, 0], qkv[:, 1], qkv[:, 2], dO, batch, pos)
+    _check_grads(cfg, got, want, np.arange(batch.T))
+
+
+@pytest.mark.parametrize("name,B", [("c0", None), ("c3", 6)])
+def test_bwd_workspace_contents_do_not_matter(G, name, B):
+    """Workspaces filled with NaN bit patterns: every scratch value the kernels read must
+    be one they wrote (a query tile's per-row terms past the user's end included)."""
+    cfg = CONFIGS[name] if B is None else CONFIGS[name].with_(B=B)
+    batch = make_batch(cfg)
+    pos, _, _ = ref.meta(batch)
+    qkv = make_qkv(cfg, batch.T, seed=27)
+    dO = make_qkv(cfg, batch.T, seed=28, n=1)[:, 0]
+    got = run_bwd(G, cfg, batch, pos, qkv, dO, poison=True)
     want = ref.attn_bwd(qkv[:, 0], qkv[:, 1], qkv[:, 2], dO, batch, pos)
     _check_grads(cfg, got, want, np.arange(batch.T))
 

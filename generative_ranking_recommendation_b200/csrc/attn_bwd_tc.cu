@@ -128,15 +128,24 @@ __host__ __device__ inline long long scratch_tp(long long T, int B) {
 // prologue: records (block B) and per-row terms (blocks 0..B-1)
 // ------------------------------------------------------------------------------------------
 constexpr int kMaxBuckets = 257;
+// Per-token info: x = (user segment start in the scratch - user start) | kCandBit for a
+// candidate token; y = the float bits of t - t_0 (seconds since the user's first token).
+// Tokens of no valid user keep the memset value, x = -1.
+constexpr int kCandBit = 1 << 30;
 
 __global__ void __launch_bounds__(256) k_bwd_prologue(const __grid_constant__ AttnArgs a,
                                                       int max_tiles, int4* recs, int32_t* count,
-                                                      int32_t* uorder, int32_t* tok_user) {
+                                                      int32_t* uorder, int2* tinfo) {
   const int b = blockIdx.x;
-  if (b < a.B) {  // the owner of every token (read by the per-row kernels)
+  if (b < a.B) {  // per-token facts for the per-row kernels (one independent load there)
     const long long s = a.off[b], e = a.off[b + 1];
     if (s < 0 || e < s || e > a.T) return;
-    for (long long t = s + threadIdx.x; t < e; t += blockDim.x) tok_user[t] = b;
+    const int n = (int)max(0LL, min((long long)a.hist_len[b], e - s));
+    const int segoff = (int)(seg_start(s, b) - s);
+    const long long t0 = e > s ? a.ts[s] : 0;  // (an empty user reads nothing)
+    for (long long t = s + threadIdx.x; t < e; t += blockDim.x)
+      tinfo[t] = make_int2(segoff | (t - s >= n ? kCandBit : 0),
+                           __float_as_int((float)(a.ts[t] - t0)));
     return;
   }
   // Records go out user by user (users with the most history key tiles first, each
@@ -213,9 +222,10 @@ __global__ void __launch_bounds__(256) k_bwd_prologue(const __grid_constant__ At
 
 // Per (token, head) terms, eight lanes per pair (16-byte loads of O and dO rows):
 // c_j = log2 e (m_h p_j + m_t,h (t_j - t_0)), lse2_i = LSE_i log2 e + c_i and
-// D_i = rowsum(dO_i * O_i), at the user's segment of the [H][Tp] scratch.
+// D_i = rowsum(dO_i * O_i), at the user's segment of the [H][Tp] scratch.  Every load
+// is issued up front (the per-token info replaces a chain through the user's offsets).
 __global__ void __launch_bounds__(256) k_bwd_rows(const __grid_constant__ AttnArgs a,
-                                                  const int32_t* __restrict__ tok_user,
+                                                  const int2* __restrict__ tinfo,
                                                   float* cbias, float* lse2, float* dsum,
                                                   long long Tp) {
   const long long x = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 3;  // pair
@@ -224,8 +234,13 @@ __global__ void __launch_bounds__(256) k_bwd_rows(const __grid_constant__ AttnAr
   const long long tok = x / a.H;
   const int h = (int)(x - tok * a.H);
   const bool live = tok < tend;
-  float dd = 0.f;
+  float dd = 0.f, lse = 0.f;
+  int2 ti = make_int2(-1, 0);
+  int pos = 0;
   if (live) {
+    ti = tinfo[tok];
+    pos = a.pos[tok];
+    lse = a.lse_in[(long long)h * a.T + tok];
     const uint4 ov = *reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.o + tok * a.o_stride +
                                                      h * DH + 8 * sub);
     const uint4 gv = *reinterpret_cast<const uint4*>(
@@ -240,14 +255,11 @@ __global__ void __launch_bounds__(256) k_bwd_rows(const __grid_constant__ AttnAr
   dd += __shfl_xor_sync(0xffffffffu, dd, 2);
   dd += __shfl_xor_sync(0xffffffffu, dd, 1);
   if (!live || sub != 0) return;
-  const int u = tok_user[tok];
-  if (u < 0 || u >= a.B) return;  // tokens of no valid user (the schedule flags the layout)
-  const long long s = a.off[u];
-  const float c = kLog2e * (a.slope_pos[h] * (float)a.pos[tok] +
-                            a.slope_time[h] * (float)(a.ts[tok] - a.ts[s]));
-  const long long idx = (long long)h * Tp + seg_start(s, u) + (tok - s);
+  if (ti.x < 0) return;  // tokens of no valid user (the schedule flags the layout)
+  const float c = kLog2e * (a.slope_pos[h] * (float)pos + a.slope_time[h] * __int_as_float(ti.y));
+  const long long idx = (long long)h * Tp + tok + (ti.x & (kCandBit - 1));
   cbias[idx] = c;
-  lse2[idx] = a.lse_in[(long long)h * a.T + tok] * kLog2e + c;
+  lse2[idx] = lse * kLog2e + c;
   dsum[idx] = dd;
 }
 
@@ -369,22 +381,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
     // half, and half X of the next tile (of this record or of the next one) is issued
     // at once: it runs while the softmax works on the other half.  dQ of tile g comes
     // after both halves.
-    const uint32_t sK = smem_u32(smem + kOffK), sV = smem_u32(smem + kOffV),
-                   sQ = smem_u32(smem + kOffQ), sDO = smem_u32(smem + kOffDO),
-                   sDS = smem_u32(smem + kOffDS);
+    // Descriptor bases, built once: an operand's descriptor is its base plus the byte
+    // offset / 16 of the stage, half and k-step (the 14-bit address field never
+    // carries: shared memory is below 256 KB).  Each MMA then costs two adds, which
+    // keeps this thread's instructions between MMAs few: the tensor pipe takes about
+    // one MMA ahead, and this warp shares its sub-partition with the softmax warps.
+    constexpr uint32_t kTileD = kTileBytes >> 4, kPSD = kPSBytes >> 4, kRowD = (16 * 128) >> 4;
+    const uint64_t kmK = smem_desc_sw128(smem_u32(smem + kOffK), 16, 1024);
+    const uint64_t kmV = smem_desc_sw128(smem_u32(smem + kOffV), 16, 1024);
+    const uint64_t kmQ = smem_desc_sw128(smem_u32(smem + kOffQ), 16, 1024);
+    const uint64_t kmDO = smem_desc_sw128(smem_u32(smem + kOffDO), 16, 1024);
+    const uint64_t kmDS = smem_desc_sw128(smem_u32(smem + kOffDS), 16, 1024);
+    const uint64_t mnQ = smem_desc_sw128(smem_u32(smem + kOffQ), kTileBytes, 1024);
+    const uint64_t mnDO = smem_desc_sw128(smem_u32(smem + kOffDO), kTileBytes, 1024);
+    const uint64_t mnK = smem_desc_sw128(smem_u32(smem + kOffK), kTileBytes, 1024);
+    const uint64_t mnDS = smem_desc_sw128(smem_u32(smem + kOffDS), BM * 128, 1024);
     // S^T = K Q_X^T and dP^T = V dO_X^T for query half X of tile gg (keys of stage kvs)
     auto issue_sdp = [&](int gg, int kvs, int x) {
-      const uint32_t qoff = (gg & 1) * kTileBytes + x * (kQH * 128);
+      const uint64_t a_k = kmK + kvs * kTileD, a_v = kmV + kvs * kTileD;
+      const uint32_t qo = (gg & 1) * kTileD + x * ((kQH * 128) >> 4);
+      const uint64_t b_q = kmQ + qo, b_do = kmDO + qo;
 #pragma unroll
       for (int k = 0; k < DH / 16; ++k)
-        mma_bf16_ss(tmem + kColS + kQH * x,
-                    smem_desc_sw128(sK + kvs * kTileBytes + k * 32, 16, 1024),
-                    smem_desc_sw128(sQ + qoff + k * 32, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
+        mma_bf16_ss(tmem + kColS + kQH * x, a_k + 2 * k, b_q + 2 * k, kIdescS, k > 0 ? 1u : 0u);
 #pragma unroll
       for (int k = 0; k < DH / 16; ++k)
-        mma_bf16_ss(tmem + kColDP + kQH * x,
-                    smem_desc_sw128(sV + kvs * kTileBytes + k * 32, 16, 1024),
-                    smem_desc_sw128(sDO + qoff + k * 32, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
+        mma_bf16_ss(tmem + kColDP + kQH * x, a_v + 2 * k, b_do + 2 * k, kIdescS,
+                    k > 0 ? 1u : 0u);
       mma_commit(&bars[kSFull + x]);
     };
     // dV += P^T dO_X with P^T read from TMEM, and dK += dS^T Q_X, over query half X
@@ -392,24 +415,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
     // queries [16k, 16k + 16) of the half at column 64 x + 32 (k / 2) + 8 (k % 2).
     auto issue_dvdk = [&](int gg, int x, bool first) {
       const uint32_t st = gg & 1;
-      const uint32_t sDSb = sDS + st * kPSBytes;
+      const uint32_t ro = st * kTileD + x * (kQH / 16) * kRowD;  // 16-query steps of the half
+      const uint64_t b_do = mnDO + ro, b_q = mnQ + ro;
+      const uint64_t a_ds = kmDS + st * kPSD + x * ((BM * 128) >> 4);
+      const uint32_t a_p = tmem + kColS + kQH * x;
 #pragma unroll
-      for (int k = 0; k < kQH / 16; ++k) {
-        const int kq = (kQH / 16) * x + k;  // 16-query step within the tile
-        const uint64_t bdo =
-            smem_desc_sw128(sDO + st * kTileBytes + kq * 16 * 128, kTileBytes, 1024);
-        mma_bf16_ts(tmem + kColDV, tmem + kColS + kQH * x + 32 * (k >> 1) + 8 * (k & 1), bdo,
+      for (int k = 0; k < kQH / 16; ++k)
+        mma_bf16_ts(tmem + kColDV, a_p + 32 * (k >> 1) + 8 * (k & 1), b_do + k * kRowD,
                     kIdescKV, (!first || k > 0) ? 1u : 0u);
-      }
 #pragma unroll
-      for (int k = 0; k < kQH / 16; ++k) {
-        const int kq = (kQH / 16) * x + k;
-        const uint32_t aoff = x * (BM * 128) + k * 32;
-        const uint64_t bq =
-            smem_desc_sw128(sQ + st * kTileBytes + kq * 16 * 128, kTileBytes, 1024);
-        mma_bf16_ss(tmem + kColDK, smem_desc_sw128(sDSb + aoff, 16, 1024), bq, kIdescKV,
+      for (int k = 0; k < kQH / 16; ++k)
+        mma_bf16_ss(tmem + kColDK, a_ds + 2 * k, b_q + k * kRowD, kIdescKV,
                     (!first || k > 0) ? 1u : 0u);
-      }
     };
     int it = 0, g = 0;
     bool ok = blockIdx.x < total;
@@ -471,13 +488,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
           break;
         }
         tc_fence_after();
-        const uint32_t sDSb = sDS + st * kPSBytes;
+        {
+          const uint64_t a_ds = mnDS + st * kPSD, b_k = mnK + kvs * kTileD;
 #pragma unroll
-        for (int k = 0; k < BM / 16; ++k) {
-          const uint64_t ads = smem_desc_sw128(sDSb + k * 16 * 128, BM * 128, 1024);
-          const uint64_t bk =
-              smem_desc_sw128(sK + kvs * kTileBytes + k * 16 * 128, kTileBytes, 1024);
-          mma_bf16_ss(tmem + kColDQ + st * DH, ads, bk, kIdescQ, k > 0 ? 1u : 0u);
+          for (int k = 0; k < BM / 16; ++k)
+            mma_bf16_ss(tmem + kColDQ + st * DH, a_ds + k * kRowD, b_k + k * kRowD, kIdescQ,
+                        k > 0 ? 1u : 0u);
         }
         mma_commit(&bars[kDQFull + st]);
         mma_commit(&bars[kDSFree + st]);
@@ -677,69 +693,90 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
 }
 
 // ------------------------------------------------------------------------------------------
-// finishing kernel: dq from the accumulator, and the candidate self terms
+// finishing kernels: the candidate self terms, then dq from the accumulator
 // ------------------------------------------------------------------------------------------
-// Eight lanes per (token, head), eight of the 64 columns per lane (16-byte loads).
-// For a candidate token c (its own key, bias 0): p = exp(scale q.k - LSE),
-// ds = p (dO.v - D), dv = p dO, dk = scale ds q, and dq gains scale ds k.
-__global__ void __launch_bounds__(256) k_bwd_finish(const __grid_constant__ AttnArgs a,
-                                                    const float* __restrict__ dqacc,
-                                                    const float* __restrict__ dsum,
-                                                    const int32_t* __restrict__ tok_user,
-                                                    long long Tp) {
-  const long long x = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 3;  // pair
+// One block per user, eight lanes per (candidate, head), eight of the 64 columns per
+// lane (16-byte loads).  A candidate token c is seen only by itself (bias 0):
+// p = exp(scale q.k - LSE), ds = p (dO.v - D), dv = p dO, dk = scale ds q, and the dQ
+// accumulator gains ds k (scaled with the rest by the conversion that follows).  The
+// main kernel has finished with the accumulator, so these rows are read and written
+// plainly; dk, dv of candidate tokens have no other writer.
+__global__ void __launch_bounds__(256) k_bwd_cand(const __grid_constant__ AttnArgs a,
+                                                  float* __restrict__ dqacc,
+                                                  const float* __restrict__ dsum, long long Tp) {
+  const int u = blockIdx.x;
+  const long long s = a.off[u], e = a.off[u + 1];
+  if (s < 0 || e < s || e > a.T) return;  // flagged by the schedule
+  const int L = (int)(e - s);
+  const int n = max(0, min(a.hist_len[u], L));
+  const int pairs = (L - n) * a.H;
+  const long long seg = seg_start(s, u);
   const int sub = threadIdx.x & 7;
-  const long long tend = min(a.T, (long long)a.off[a.B]);
-  const long long tok = x / a.H;
-  const int h = (int)(x - tok * a.H);
-  const int u = tok < tend ? tok_user[tok] : -1;
-  const bool owned = u >= 0 && u < a.B;
-  const long long s = owned ? a.off[u] : 0;
-  const bool cand = owned && tok - s >= a.hist_len[u];
-  const long long qo = tok * a.tok_stride + h * DH + 8 * sub;
-  float dq[8], qf[8], kf[8], vf[8], gf[8];
-  float sdot = 0.f, pdot = 0.f;
-  if (owned) {
-    const float4* acc = reinterpret_cast<const float4*>(dqacc + (tok * a.H + h) * DH + 8 * sub);
-    const float4 a0 = acc[0], a1 = acc[1];
-    dq[0] = a0.x; dq[1] = a0.y; dq[2] = a0.z; dq[3] = a0.w;
-    dq[4] = a1.x; dq[5] = a1.y; dq[6] = a1.z; dq[7] = a1.w;
+  for (int base = 0; base < pairs; base += blockDim.x / 8) {  // uniform trip count
+    const int pr = base + (int)(threadIdx.x >> 3);
+    const bool act = pr < pairs;
+    const int c = act ? n + pr / a.H : n;
+    const int h = act ? pr % a.H : 0;
+    const long long tok = s + c;
+    const long long qo = tok * a.tok_stride + h * DH + 8 * sub;
+    float qf[8], kf[8], vf[8], gf[8];
+    float sdot = 0.f, pdot = 0.f;
+    if (act) {
+      Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.q + qo), qf);
+      Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.k + qo), kf);
+      Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.v + qo), vf);
+      Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(
+                                      (const __nv_bfloat16*)a.dO + tok * a.o_stride + h * DH + 8 * sub),
+                                  gf);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) dq[e] *= a.scale;
-  }
-  if (cand) {
-    Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.q + qo), qf);
-    Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.k + qo), kf);
-    Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>((const __nv_bfloat16*)a.v + qo), vf);
-    Elem<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(
-                                    (const __nv_bfloat16*)a.dO + tok * a.o_stride + h * DH + 8 * sub),
-                                gf);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      sdot = fmaf(qf[e], kf[e], sdot);
-      pdot = fmaf(gf[e], vf[e], pdot);
+      for (int i = 0; i < 8; ++i) {
+        sdot = fmaf(qf[i], kf[i], sdot);
+        pdot = fmaf(gf[i], vf[i], pdot);
+      }
     }
-  }
 #pragma unroll
-  for (int o = 4; o > 0; o >>= 1) {
-    sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
-    pdot += __shfl_xor_sync(0xffffffffu, pdot, o);
-  }
-  if (cand) {
-    const long long ridx = (long long)h * Tp + seg_start(s, u) + (tok - s);
+    for (int o = 4; o > 0; o >>= 1) {
+      sdot += __shfl_xor_sync(0xffffffffu, sdot, o);
+      pdot += __shfl_xor_sync(0xffffffffu, pdot, o);
+    }
+    if (!act) continue;
     const float p = expf(sdot * a.scale - a.lse_in[(long long)h * a.T + tok]);
-    const float ds = p * (pdot - dsum[ridx]);
+    const float ds = p * (pdot - dsum[(long long)h * Tp + seg + c]);
+    float* acc = dqacc + (tok * a.H + h) * DH + 8 * sub;
+    float4 a0 = reinterpret_cast<float4*>(acc)[0], a1 = reinterpret_cast<float4*>(acc)[1];
+    a0.x = fmaf(ds, kf[0], a0.x); a0.y = fmaf(ds, kf[1], a0.y);
+    a0.z = fmaf(ds, kf[2], a0.z); a0.w = fmaf(ds, kf[3], a0.w);
+    a1.x = fmaf(ds, kf[4], a1.x); a1.y = fmaf(ds, kf[5], a1.y);
+    a1.z = fmaf(ds, kf[6], a1.z); a1.w = fmaf(ds, kf[7], a1.w);
+    reinterpret_cast<float4*>(acc)[0] = a0;
+    reinterpret_cast<float4*>(acc)[1] = a1;
     float dk[8], dv[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      dq[e] = fmaf(a.scale * ds, kf[e], dq[e]);
-      dk[e] = a.scale * ds * qf[e];
-      dv[e] = p * gf[e];
+    for (int i = 0; i < 8; ++i) {
+      dk[i] = a.scale * ds * qf[i];
+      dv[i] = p * gf[i];
     }
     *reinterpret_cast<uint4*>((__nv_bfloat16*)a.dk + qo) = Elem<__nv_bfloat16>::pack(dk);
     *reinterpret_cast<uint4*>((__nv_bfloat16*)a.dv + qo) = Elem<__nv_bfloat16>::pack(dv);
   }
-  if (owned) *reinterpret_cast<uint4*>((__nv_bfloat16*)a.dq + qo) = Elem<__nv_bfloat16>::pack(dq);
+}
+
+// dq = scale * dQ_acc for every token of the batch, eight columns per thread: a plain
+// stream (two 16-byte loads, one 16-byte store), at full occupancy.
+__global__ void __launch_bounds__(256) k_bwd_finish(const __grid_constant__ AttnArgs a,
+                                                    const float* __restrict__ dqacc) {
+  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;  // 8-column chunk
+  const long long pair = x >> 3;
+  const long long tend = min(a.T, (long long)a.off[a.B]);
+  const long long tok = pair / a.H;
+  if (tok >= tend) return;
+  const int h = (int)(pair - tok * a.H);
+  const float4* acc = reinterpret_cast<const float4*>(dqacc) + 2 * x;
+  const float4 a0 = acc[0], a1 = acc[1];
+  const float f[8] = {a0.x * a.scale, a0.y * a.scale, a0.z * a.scale, a0.w * a.scale,
+                      a1.x * a.scale, a1.y * a.scale, a1.z * a.scale, a1.w * a.scale};
+  *reinterpret_cast<uint4*>((__nv_bfloat16*)a.dq + tok * a.tok_stride + h * DH +
+                            8 * (int)(x & 7)) = Elem<__nv_bfloat16>::pack(f);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -776,7 +813,7 @@ static size_t recs_bytes(int B, int max_seqlen) {
   return ((size_t)B * max_tiles_of(max_seqlen) * 32 + 15) / 16 * 16;
 }
 static size_t users_bytes(int B) { return ((size_t)B * 4 + 15) / 16 * 16; }
-static size_t tokens_bytes(long long T) { return ((size_t)T * 4 + 15) / 16 * 16; }
+static size_t tokens_bytes(long long T) { return ((size_t)T * 8 + 15) / 16 * 16; }
 static size_t rows_bytes(long long T, int B, int H) {
   return ((size_t)H * scratch_tp(T, B) * sizeof(float) + 15) / 16 * 16;
 }
@@ -805,8 +842,8 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   p.recs = (int4*)(ws + kHeaderBytes);
   const size_t rb = rows_bytes(a.T, a.B, a.H);
   int32_t* uorder = (int32_t*)(ws + kHeaderBytes + recs_bytes(a.B, a.max_seqlen));
-  int32_t* tok_user = (int32_t*)((uint8_t*)uorder + users_bytes(a.B));
-  uint8_t* rows = (uint8_t*)tok_user + tokens_bytes(a.T);
+  int2* tinfo = (int2*)((uint8_t*)uorder + users_bytes(a.B));
+  uint8_t* rows = (uint8_t*)tinfo + tokens_bytes(a.T);
   p.cbias = (float*)rows;
   p.lse2 = (float*)(rows + rb);
   p.dsum = (float*)(rows + 2 * rb);
@@ -818,14 +855,14 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   if (cudaMemsetAsync(rows + 2 * rb, 0, rb + (size_t)a.T * a.H * DH * sizeof(float), st) !=
       cudaSuccess)
     return GENRANK_ERR_CUDA;
-  if (a.T > 0 && cudaMemsetAsync(tok_user, 0xff, (size_t)a.T * 4, st) != cudaSuccess)
+  if (a.T > 0 && cudaMemsetAsync(tinfo, 0xff, (size_t)a.T * 8, st) != cudaSuccess)
     return GENRANK_ERR_CUDA;
   k_bwd_prologue<<<a.B + 1, 256, 0, st>>>(a, max_tiles_of(a.max_seqlen), (int4*)p.recs,
-                                          (int32_t*)p.count, uorder, tok_user);
+                                          (int32_t*)p.count, uorder, tinfo);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   const long long pair_blocks = (a.T * a.H + 31) / 32;  // 8 lanes per (token, head)
   if (pair_blocks > 0) {
-    k_bwd_rows<<<(unsigned)pair_blocks, 256, 0, st>>>(a, tok_user, (float*)p.cbias,
+    k_bwd_rows<<<(unsigned)pair_blocks, 256, 0, st>>>(a, tinfo, (float*)p.cbias,
                                                       (float*)p.lse2, (float*)p.dsum, p.Tp);
     if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   }
@@ -841,8 +878,12 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   k_attn_bwd_tc<<<sms, kThreads, kSmemBytes, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
+  if (a.B > 0) {
+    k_bwd_cand<<<a.B, 256, 0, st>>>(a, p.dqacc, p.dsum, p.Tp);
+    if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
+  }
   if (pair_blocks > 0)
-    k_bwd_finish<<<(unsigned)pair_blocks, 256, 0, st>>>(a, p.dqacc, p.dsum, tok_user, p.Tp);
+    k_bwd_finish<<<(unsigned)pair_blocks, 256, 0, st>>>(a, p.dqacc);
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
 }
 

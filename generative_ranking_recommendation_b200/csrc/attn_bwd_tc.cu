@@ -28,12 +28,15 @@
 //     columns, TMEM access shape 16x32bx2, so two of these warps share each SM
 //     sub-partition) compute P^T and dS^T.
 //   * Warps 10-13 (one query row per thread) add each dQ_part into an fp32 dQ
-//     accumulator in global memory with vector reductions and, per record, move dK
-//     (times scale) and dV from TMEM to global memory.
+//     accumulator in global memory: 32 rows x 32 columns at a time are staged in shared
+//     memory and reduced by the TMA engine (cp.reduce.async.bulk.tensor add), which
+//     keeps the load/store path free for the operand traffic of the tensor cores.  Per
+//     record they move dK (times scale) and dV from TMEM to global memory.
 //   * K and V are double-buffered by record, so the next record's loads and its
 //     first S^T, dP^T overlap the end of the current one.
-//   * Candidate keys are seen only by their own row; a finishing kernel applies that
-//     self term to dq, dk, dv of candidate tokens and writes dq = scale * dQ_acc.
+//   * Candidate keys are seen only by their own row; a small kernel applies that self
+//     term (dk, dv of candidate tokens, and ds k into the dQ accumulator), and a
+//     streaming pass writes dq = scale * dQ_acc.
 // Every mbarrier wait is bounded in time; a timeout sets GENRANK_DERR_TIMEOUT,
 // every role drains out of its loop and the CTA frees its tensor memory.
 #include <cuda.h>
@@ -61,10 +64,14 @@ constexpr uint32_t kOffDO = kOffQ + 2 * kTileBytes;    // 2 stages
 constexpr uint32_t kOffL2 = kOffDO + 2 * kTileBytes;   // lse2, 2 stages
 constexpr uint32_t kOffD = kOffL2 + 2 * kRowBytes;     // D, 2 stages
 constexpr uint32_t kOffDS = kOffD + 2 * kRowBytes;     // dS^T, 2 buffers
-constexpr uint32_t kOffBar = kOffDS + 2 * kPSBytes;
+constexpr uint32_t kOffStage = kOffDS + 2 * kPSBytes;  // dQ_part staging, 4 x 4 KB
+constexpr uint32_t kStageBytes = 32 * 32 * 4;           // 32 rows x 32 fp32 columns
+constexpr uint32_t kOffBar = kOffStage + 4 * kStageBytes;
 constexpr uint32_t kNumBars = 20;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
+static_assert(kOffStage % 1024 == 0, "128B-swizzled staging must be 1024-byte aligned");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 // tensor memory
 constexpr uint32_t kTmemCols = 512;
@@ -88,6 +95,7 @@ enum Bar { kKVFull = 0, kKVEmpty = 2, kQDFull = 4, kQDEmpty = 6, kSFull = 8, kPF
 
 struct Params {
   CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tdq;  // the fp32 dQ accumulator [T][H][64], box 32 columns x 32 rows
   AttnArgs a;
   const int4* recs;
   const int32_t* count;
@@ -325,6 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
     tma_prefetch_desc(&P.tk);
     tma_prefetch_desc(&P.tv);
     tma_prefetch_desc(&P.tdo);
+    tma_prefetch_desc(&P.tdq);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -671,18 +680,37 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kDQEmpty + db]);
-        const int i = rc.k0 + t * BM + qlane;
-        if (i < rc.L) {
-          float* dst = P.dqacc + (((long long)rc.s + i) * a.H + rc.h) * DH;
+        // The warp's 32 query rows go to the accumulator by TMA reduce-add, 32 columns at
+        // a time through a 128B-swizzled staging box (one bulk operation instead of 512
+        // scattered vector reductions; rows past the user's end are staged as zeros).
+        const int r0 = rc.k0 + t * BM + 32 * (warp & 3);  // the warp's first row (local)
+        if (r0 < rc.L) {
+          const bool live = r0 + lane < rc.L;
+          uint8_t* stg = smem + kOffStage + (warp & 3) * kStageBytes;
 #pragma unroll
-          for (int c = 0; c < DH; c += 4)
-            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + c),
-                         "f"(dq[c]), "f"(dq[c + 1]), "f"(dq[c + 2]), "f"(dq[c + 3])
-                         : "memory");
+          for (int c = 0; c < DH; c += 32) {
+            if (lane == 0) bulk_wait_read_all();  // the last reduction has read the box
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float4 v = live ? make_float4(dq[c + 4 * k], dq[c + 4 * k + 1],
+                                                  dq[c + 4 * k + 2], dq[c + 4 * k + 3])
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+              *reinterpret_cast<float4*>(stg + lane * 128 + ((k ^ (lane & 7)) << 4)) = v;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_reduce_add_3d(&P.tdq, stg, c, rc.h, rc.s + r0);
+              bulk_commit();
+            }
+          }
         }
       }
       if (!ok) break;
     }
+    if (lane == 0) bulk_wait_all();  // the accumulator is complete when the kernel ends
+    __syncwarp();
   }
 
   __syncwarp();
@@ -808,6 +836,21 @@ static bool make_map(CUtensorMap* m, const void* base, long long T, int H, long 
          CUDA_SUCCESS;
 }
 
+// The fp32 dQ accumulator [T][H][64]; box = 32 columns x one head x 32 rows, 128-byte
+// swizzle (the staging layout of the reducing warps).
+static bool make_map_f32(CUtensorMap* m, const float* base, long long T, int H) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)DH, (cuuint64_t)H, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)DH * 4, (cuuint64_t)H * DH * 4};
+  cuuint32_t box[3] = {32, 1, 32};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 static int max_tiles_of(int max_seqlen) { return (max_seqlen + BM - 1) / BM; }
 static size_t recs_bytes(int B, int max_seqlen) {
   return ((size_t)B * max_tiles_of(max_seqlen) * 32 + 15) / 16 * 16;
@@ -849,6 +892,7 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   p.dsum = (float*)(rows + 2 * rb);
   p.dqacc = (float*)(rows + 3 * rb);
   p.Tp = scratch_tp(a.T, a.B);
+  if (!make_map_f32(&p.tdq, p.dqacc, a.T, a.H)) return GENRANK_ERR_CUDA;
   // D and the dQ accumulator are adjacent: one memset zeroes both.  A query tile reads D
   // past its user's last row (the gap before the next user's segment), where a masked
   // pair's ds = p (dP - D) with p = 0 must stay 0 whatever the workspace held.

@@ -240,6 +240,20 @@ GR_DEVICE void tma_load_3d(void* smem_dst, const void* tmap, uint64_t* bar, int 
       : "memory");
 }
 
+// Reduce-add of a shared-memory box into a global tensor (tile mode, no multicast), by the
+// TMA engine; completion is tracked per thread in bulk groups.
+GR_DEVICE void tma_reduce_add_3d(const void* tmap, const void* smem_src, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+GR_DEVICE void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The committed bulk groups of this thread have read their shared-memory sources.
+GR_DEVICE void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// The committed bulk groups of this thread have completed.
+GR_DEVICE void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------------------------------------
 // tcgen05 (5th-generation tensor cores, accumulators in tensor memory)
 // ------------------------------------------------------------------------------------------

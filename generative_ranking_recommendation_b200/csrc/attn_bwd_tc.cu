@@ -624,7 +624,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
     }
   } else if (warp >= 2 + kSoftmaxWarps) {
     // ---------------------------------------------------------------- dQ reduction (query rows)
-    const int qlane = 32 * (warp & 3) + lane;  // TMEM lane this thread may read
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     int g = 0, it = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
@@ -634,39 +633,59 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
       bool ok = true;
       for (int t = 0; t < rc.nq; ++t, ++g) {
         if (t + 1 == rc.nq) {
-          // the record's dK (times scale) and dV, key row qlane, once its last dV, dK
-          // MMAs are done (before its last dQ_part); the accumulators are released
-          // before the last stores
+          // the record's dK (times scale), then dV, once its last dV, dK MMAs are
+          // done (before its last dQ_part); the accumulators are released after the dV
+          // load.  Each warp stages its 32 key rows (bf16, 128 bytes each) in its
+          // 128B-swizzled box and writes them as whole rows, four rows per store
+          // instruction; rows of candidate keys and past the user are skipped.
           if (!wait_warp(&bars[kDKVFull], parity(it), abort_flag, a.err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int j = rc.k0 + qlane;
-          const bool key = j < rc.n;
-          const long long tok = (long long)rc.s + j;
-          __nv_bfloat16* dkp = (__nv_bfloat16*)a.dk + tok * a.tok_stride + rc.h * DH;
-          __nv_bfloat16* dvp = (__nv_bfloat16*)a.dv + tok * a.tok_stride + rc.h * DH;
+          uint8_t* stg = smem + kOffStage + (warp & 3) * kStageBytes;
+          const int jr0 = rc.k0 + 32 * (warp & 3);  // the warp's first key row (local)
 #pragma unroll 1
-          for (int c0 = 0; c0 < DH; c0 += 32) {
-            float dvr[32], dkr[32];
-            tmem_ld32(tmem + lane_base + kColDV + c0, dvr);
-            tmem_ld32(tmem + lane_base + kColDK + c0, dkr);
-            if (c0 + 32 == DH) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&bars[kDKVEmpty]);
-            }
-            if (key) {
+          for (int m = 0; m < 2; ++m) {
+            const float mul = m ? 1.f : a.scale;
+            if (lane == 0) bulk_wait_read_all();  // the box's last reduction has read it
+            __syncwarp();
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {  // 32 columns at a time
+              float v[32];
+              tmem_ld32(tmem + lane_base + (m ? kColDV : kColDK) + 32 * hf, v);
+              if (m == 1 && hf == 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[kDKVEmpty]);
+              }
 #pragma unroll
-              for (int c = 0; c < 32; c += 8) {
+              for (int kk = 0; kk < 4; ++kk) {
+                const int k = 4 * hf + kk;
                 float f[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = dkr[c + e] * a.scale;
-                *reinterpret_cast<uint4*>(dkp + c0 + c) = Elem<__nv_bfloat16>::pack(f);
-                *reinterpret_cast<uint4*>(dvp + c0 + c) = Elem<__nv_bfloat16>::pack(dvr + c);
+                for (int e = 0; e < 8; ++e) f[e] = v[8 * kk + e] * mul;
+                *reinterpret_cast<uint4*>(stg + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+                    Elem<__nv_bfloat16>::pack(f);
               }
             }
+            __syncwarp();
+            // lane: row 4q + lane / 8 of the box, 16-byte chunk lane % 8
+            const int c = lane & 7;
+            const int nrows = min(32, rc.n - jr0);  // rows of history keys in the box
+            const uint8_t* src = stg + (lane >> 3) * 128;
+            __nv_bfloat16* dst = (__nv_bfloat16*)(m ? a.dv : a.dk) +
+                                 ((long long)rc.s + jr0 + (lane >> 3)) * a.tok_stride +
+                                 rc.h * DH + 8 * c;
+            const long long dstep = 4LL * a.tok_stride;
+#pragma unroll 2
+            for (int q = 0; q < 8; ++q, src += 4 * 128, dst += dstep) {
+              const int rr = 4 * q + (lane >> 3);
+              if (rr < nrows)
+                *reinterpret_cast<uint4*>(dst) =
+                    *reinterpret_cast<const uint4*>(src + ((c ^ (rr & 7)) << 4));
+            }
+            __syncwarp();  // every lane has read the box before it is written again
           }
         }
         const int db = g & 1;
@@ -723,8 +742,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
 // ------------------------------------------------------------------------------------------
 // finishing kernels: the candidate self terms, then dq from the accumulator
 // ------------------------------------------------------------------------------------------
-// One block per user, eight lanes per (candidate, head), eight of the 64 columns per
-// lane (16-byte loads).  A candidate token c is seen only by itself (bias 0):
+// gridDim.y blocks per user, eight lanes per (candidate, head), eight of the 64
+// columns per lane (16-byte loads).  A candidate token c is seen only by itself (bias 0):
 // p = exp(scale q.k - LSE), ds = p (dO.v - D), dv = p dO, dk = scale ds q, and the dQ
 // accumulator gains ds k (scaled with the rest by the conversion that follows).  The
 // main kernel has finished with the accumulator, so these rows are read and written
@@ -740,7 +759,9 @@ __global__ void __launch_bounds__(256) k_bwd_cand(const __grid_constant__ AttnAr
   const int pairs = (L - n) * a.H;
   const long long seg = seg_start(s, u);
   const int sub = threadIdx.x & 7;
-  for (int base = 0; base < pairs; base += blockDim.x / 8) {  // uniform trip count
+  const int step = (int)gridDim.y * (int)(blockDim.x / 8);
+  for (int base = (int)blockIdx.y * (int)(blockDim.x / 8); base < pairs;
+       base += step) {  // uniform trip count within the block
     const int pr = base + (int)(threadIdx.x >> 3);
     const bool act = pr < pairs;
     const int c = act ? n + pr / a.H : n;
@@ -923,7 +944,7 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   k_attn_bwd_tc<<<sms, kThreads, kSmemBytes, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   if (a.B > 0) {
-    k_bwd_cand<<<a.B, 256, 0, st>>>(a, p.dqacc, p.dsum, p.Tp);
+    k_bwd_cand<<<dim3((unsigned)a.B, 4), 256, 0, st>>>(a, p.dqacc, p.dsum, p.Tp);
     if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   }
   if (pair_blocks > 0)

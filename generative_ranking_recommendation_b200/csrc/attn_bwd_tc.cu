@@ -67,7 +67,7 @@ constexpr uint32_t kOffDS = kOffD + 2 * kRowBytes;     // dS^T, 2 buffers
 constexpr uint32_t kOffStage = kOffDS + 2 * kPSBytes;  // dQ_part staging, 4 x 4 KB
 constexpr uint32_t kStageBytes = 32 * 32 * 4;           // 32 rows x 32 fp32 columns
 constexpr uint32_t kOffBar = kOffStage + 4 * kStageBytes;
-constexpr uint32_t kNumBars = 20;
+constexpr uint32_t kNumBars = 21;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kOffStage % 1024 == 0, "128B-swizzled staging must be 1024-byte aligned");
@@ -91,7 +91,7 @@ constexpr size_t kHeaderBytes = 256;
 // S^T / dP^T and P^T are handled per query half (64 queries): one S-full and one
 // P-full barrier per half.
 enum Bar { kKVFull = 0, kKVEmpty = 2, kQDFull = 4, kQDEmpty = 6, kSFull = 8, kPFull = 10,
-           kDSFree = 12, kDQFull = 14, kDQEmpty = 16, kDKVFull = 18, kDKVEmpty = 19 };
+           kDSFree = 12, kDQFull = 14, kDQEmpty = 16, kDKVFull = 18, kDKVEmpty = 19, kDone = 20 };
 
 struct Params {
   CUtensorMap tq, tk, tv, tdo;
@@ -325,6 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
     }
     mbar_init(&bars[kDSFree], 1);
     mbar_init(&bars[kDSFree + 1], 1);
+    mbar_init(&bars[kDone], 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -348,6 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
   if (warp == 1) {
     // ---------------------------------------------------------------- TMA producer
     int it = 0, g = 0;
+    int kv_n = 0, qd_n = 0;  // K/V and Q/dO loads issued
     for (int w = blockIdx.x; w < total; w += gridDim.x, ++it) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const Rec rc = load_rec(P, w);
@@ -360,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
         tma_load_3d(smem + kOffV + kvs * kTileBytes, &P.tv, &bars[kKVFull + kvs], 0, rc.h,
                     rc.s + rc.k0);
       }
+      kv_n = it + 1;
       const long long roff = (long long)rc.h * P.Tp + rc.spad;
       bool ok = true;
       for (int t = 0; t < rc.nq; ++t, ++g) {
@@ -380,8 +383,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
           bulk_load(smem + kOffD + st * kRowBytes, P.dsum + roff + q0, kRowBytes,
                     &bars[kQDFull + st]);
         }
+        qd_n = g + 1;
       }
       if (!ok) break;
+    }
+    // on the way out (a timeout included), the copies issued last land before the CTA
+    // exits; in a normal run they have long been consumed
+    if (lane == 0) {
+      for (int x = max(0, kv_n - 2); x < kv_n; ++x)
+        mbar_drain(&bars[kKVFull + (x & 1)], parity(x >> 1));
+      for (int x = max(0, qd_n - 2); x < qd_n; ++x)
+        mbar_drain(&bars[kQDFull + (x & 1)], parity(x >> 1));
     }
   } else if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- MMA issuer
@@ -510,6 +522,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
       }
       if (*abort_flag) ok = false;
     }
+    // every MMA issued (on a timeout too) has completed before TMEM is freed
+    mma_commit(&bars[kDone]);
+    mbar_drain(&bars[kDone], 0);
   } else if (warp >= 2 && warp < 2 + kSoftmaxWarps) {
     // ---------------------------------------------------------------- softmax (key rows)
     const int quad = warp & 3;              // TMEM lane quadrant of the warp

@@ -161,7 +161,8 @@ int genrank_embed_assemble_bwd(int B, int64_t T, const int32_t *seq_offsets, con
  *   scale        > 0, normally 1/sqrt(dh)
  *   o            [T, H * dh] output, row stride o_stride elements (dtype)
  *   lse          [H, T] fp32 natural-log LSE output, or NULL to skip
- *   ws, ws_bytes caller scratch of at least genrank_attn_workspace_size(..., 0) bytes
+ *   ws, ws_bytes caller scratch of at least genrank_attn_workspace_size(..., 0) bytes;
+ *                its contents on entry do not matter (nothing needs zeroing)
  * Supported: bf16 with dh = 64 runs the tcgen05/TMEM/TMA kernel; fp32 (any
  * dtype) with dh in {32, 64, 128} runs the CUDA-core kernel.  H <= 64. */
 int genrank_attn_fwd(int B, int64_t T, const int32_t *seq_offsets, const int32_t *hist_len, int max_seqlen,
@@ -178,7 +179,9 @@ int genrank_attn_fwd(int B, int64_t T, const int32_t *seq_offsets, const int32_t
  * dS = P * (dP - rowsum(dO * O)), dQ = scale dS K, dK = scale dS^T Q.
  * Every token row of dq/dk/dv is written (no accumulation into them).
  * bf16 with dh = 64 runs on tcgen05 tensor cores (fp32 dQ accumulated in the
- * workspace); fp32, or dh = 32, runs the CUDA-core kernels. */
+ * workspace); fp32, or dh = 32, runs the CUDA-core kernels.  The workspace
+ * (genrank_attn_workspace_size(..., 1) bytes) needs no initialisation: the call
+ * zeroes what it accumulates into. */
 int genrank_attn_bwd(int B, int64_t T, const int32_t *seq_offsets, const int32_t *hist_len, int max_seqlen,
                      const void *q, const void *k, const void *v, int64_t tok_stride, int H,
                      int dh, const int32_t *pos, const int64_t *ts, const float *slope_pos,

@@ -107,3 +107,46 @@ def test_host_side_argument_checks_return_before_launch(L):
                                  600, fake, 128, fake, 80, 64, 1, fake, fake, fake, fake, fake,
                                  None)
     assert r == 2  # 80 time buckets: beyond what the integer bucket supports
+
+
+def test_backward_workspace_covers_its_regions(L):
+    """The backward scratch holds the fp32 dQ accumulator [T, H, 64], three fp32 per-row
+    arrays [H, T] (column term, log2 LSE, D) and an 8-byte record per token."""
+    from generative_ranking_recommendation_b200 import genrank as G
+
+    B, T, H, dh, msl = 256, 100000, 4, 64, 608
+    nb = G.attn_workspace_size(B, T, H, dh, msl, True)
+    assert nb >= T * H * dh * 4 + 3 * H * T * 4 + T * 8
+    # grows with every token by at least those bytes
+    nb2 = G.attn_workspace_size(B, T + 1000, H, dh, msl, True)
+    assert nb2 - nb >= 1000 * (H * dh * 4 + 3 * H * 4 + 8)
+
+
+def test_backward_host_side_argument_checks(L):
+    """Invalid backward arguments are rejected on the host, without touching a GPU."""
+    P = ctypes.c_void_p
+    fake = P(0x10000)  # never dereferenced: every call below fails its host checks
+    sp = (ctypes.c_float * 4)(0.5, 0.25, 0.125, 0.0625)
+    st = (ctypes.c_float * 4)(*(x / 3600 for x in sp))
+    base = dict(B=1, T=10, off=fake, hl=fake, msl=10, q=fake, k=fake, v=fake, stride=768, H=4,
+                dh=64, pos=fake, ts=fake, scale=0.125, dtype=1, o=fake, dO=fake, ostride=256,
+                lse=fake, dq=fake, dk=fake, dv=fake, ws=fake, wsb=1 << 20, err=fake)
+
+    def call(**kw):
+        a = dict(base)
+        a.update(kw)
+        return L.genrank_attn_bwd(a["B"], a["T"], a["off"], a["hl"], a["msl"], a["q"], a["k"],
+                                  a["v"], a["stride"], a["H"], a["dh"], a["pos"], a["ts"],
+                                  ctypes.cast(sp, P), ctypes.cast(st, P), a["scale"], a["dtype"],
+                                  a["o"], a["dO"], a["ostride"], a["lse"], a["dq"], a["dk"],
+                                  a["dv"], a["ws"], a["wsb"], a["err"], None)
+
+    assert call(B=0) == 1
+    assert call(dO=None) == 1
+    assert call(lse=None) == 1  # the backward needs the forward's LSE
+    assert call(dq=P(0x10008)) == 1  # misaligned output
+    assert call(dtype=7) == 1
+    assert call(dh=48, stride=192, ostride=192) == 2
+    assert call(ws=None) == 3
+    assert call(wsb=16) == 3
+

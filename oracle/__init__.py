@@ -9,12 +9,14 @@ from .genrank_oracle import (  # noqa: F401
     alibi_slopes,
     attention_bwd,
     attention_fwd,
+    attention_fwd_bucketed,
     attention_mask,
     bce_loss,
     block_backward,
     block_forward,
     embed_assemble,
     embed_assemble_bwd,
+    pair_time_bucket,
     time_bucket,
     token_metadata,
 )

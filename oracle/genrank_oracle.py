@@ -22,6 +22,8 @@ position bias on the shared positions p (all candidates at n+1); time bias
 linear, slope_h/3600 per second of |t_i - t_j|; a candidate sees itself;
 positions 1-based; request index clamped to n_ri - 1; bucket(delta) =
 1 + min(n_rt - 2, floor(4 log2(delta + 1))) with 0 for "no earlier request".
+The bucketed time-bias variant uses min(n_rt - 2, floor(4 log2(delta + 1))) per pair
+and the position slopes as its per-bucket slopes.
 
 Every function loops over users (and heads) and writes the definitions out
 with explicit masks; no blocking, fusion or reordering beyond a library
@@ -228,6 +230,67 @@ def attention_bwd(q, k, v, dO, seq_offsets, hist_len, pos, ts, slope_pos, slope_
             dk[s:e, h] = scale * dS.T @ Q
             dv[s:e, h] = P.T @ G
     return dq, dk, dv
+
+
+# ----------------------------------------------------------------------------------------
+# variant: bucketed time bias (a NEXT row of the scope table)
+# ----------------------------------------------------------------------------------------
+
+def pair_time_bucket(delta: int, n_rt: int = 64) -> int:
+    """bucket(t_i - t_j) of the bucketed time bias, for a gap of ``delta`` >= 0 seconds.
+
+    [FUN-EN] §7.2.2 (and its zh twin) writes the time term of the ALiBi bias as
+    -m_t bucket(t_i - t_j) without defining bucket().  Reading: the quarter-octave grid
+    of the pre-request time embedding, floor(4 log2(delta + 1)), saturating at
+    n_rt - 2 (that table's largest gap row) and without its "no earlier request" row,
+    so that two items of one request (delta = 0) are in bucket 0.  As for the
+    embedding, floor(4 log2 x) = bit_length(x^4) - 1 in Python integers.
+    """
+    if delta < 0:
+        raise ValueError("negative gap")
+    k = ((int(delta) + 1) ** 4).bit_length() - 1
+    return min(n_rt - 2, k)
+
+
+def _user_scores_bucketed(Q, K, p, t, slope_pos, slope_tb, scale, n, n_rt):
+    """score_ij = q_i.k_j * scale - m_p (p_i - p_j) - m_t bucket(t_i - t_j) on visible
+    pairs ([FUN-EN] §7.2.2 bias formula; p_i >= p_j and t_i >= t_j there)."""
+    L = len(p)
+    S = (Q @ K.T) * scale
+    mask = attention_mask(n, L)
+    B = np.zeros((L, L))
+    for i in range(L):
+        for j in range(L):
+            if mask[i, j]:
+                B[i, j] = (slope_pos * float(int(p[i]) - int(p[j]))
+                           + slope_tb * float(pair_time_bucket(int(t[i]) - int(t[j]), n_rt)))
+    return np.where(mask, S - B, -np.inf)
+
+
+def attention_fwd_bucketed(q, k, v, seq_offsets, hist_len, pos, ts, slope_pos, slope_tb, scale,
+                           n_rt: int = 64, users=None):
+    """O [T,H,dh] and natural-log LSE [H,T] of the masked attention with the bucketed time
+    bias; the mask and position term are those of ``attention_fwd``."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    T, H, dh = q.shape
+    O = np.zeros((T, H, dh))
+    LSE = np.full((H, T), np.nan)
+    users = range(len(hist_len)) if users is None else users
+    for u in users:
+        s, e, n = int(seq_offsets[u]), int(seq_offsets[u + 1]), int(hist_len[u])
+        p = np.asarray(pos[s:e], np.int64)
+        t = np.asarray(ts[s:e], np.int64)
+        for h in range(H):
+            S = _user_scores_bucketed(q[s:e, h], k[s:e, h], p, t, slope_pos[h], slope_tb[h],
+                                      scale, n, n_rt)
+            mx = S.max(axis=1, keepdims=True)
+            P = np.exp(S - mx)
+            l = P.sum(axis=1, keepdims=True)
+            O[s:e, h] = (P / l) @ v[s:e, h]
+            LSE[h, s:e] = (mx + np.log(l))[:, 0]
+    return O, LSE
 
 
 # ----------------------------------------------------------------------------------------

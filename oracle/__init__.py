@@ -10,6 +10,7 @@ from .genrank_oracle import (  # noqa: F401
     attention_bwd,
     attention_fwd,
     attention_fwd_bucketed,
+    attention_fwd_cached,
     attention_mask,
     bce_loss,
     block_backward,

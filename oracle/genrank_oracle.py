@@ -294,6 +294,57 @@ def attention_fwd_bucketed(q, k, v, seq_offsets, hist_len, pos, ts, slope_pos, s
 
 
 # ----------------------------------------------------------------------------------------
+# variant: scoring candidates against cached history keys and values (a NEXT row)
+# ----------------------------------------------------------------------------------------
+
+def attention_fwd_cached(q_c, k_c, v_c, cand_offsets, k_hist, v_hist, hist_offsets, pos_hist,
+                         ts_hist, ts_cand, slope_pos, slope_time, scale):
+    """O [C,H,dh] and natural-log LSE [H,C] of the candidate rows only, from a cache of the
+    users' history keys and values.
+
+    [HXZ] §1.3.1 credits the KV cache with making generative ranking cheaper as the
+    candidate set grows; [HXZ] §1.4.1 and [FUN-EN] §7.2.1 fix what a candidate sees: the
+    whole history of its user and itself.  User u's history rows are
+    k_hist/v_hist[hist_offsets[u]:hist_offsets[u+1]] with positions pos_hist and times
+    ts_hist; its candidates are rows cand_offsets[u]:cand_offsets[u+1] of q_c, k_c, v_c,
+    all at position n_u + 1 and time ts_cand.  The score of candidate c against history
+    key j is q_c.k_j * scale - m |p_c - p_j| - m_t |t_c - t_j|; against itself it is
+    q_c.k_c * scale (no distance).
+    """
+    q_c = np.asarray(q_c, np.float64)
+    k_c = np.asarray(k_c, np.float64)
+    v_c = np.asarray(v_c, np.float64)
+    k_hist = np.asarray(k_hist, np.float64)
+    v_hist = np.asarray(v_hist, np.float64)
+    C, H, dh = q_c.shape
+    O = np.zeros((C, H, dh))
+    LSE = np.full((H, C), np.nan)
+    for u in range(len(cand_offsets) - 1):
+        hs, he = int(hist_offsets[u]), int(hist_offsets[u + 1])
+        n = he - hs
+        p_c = n + 1
+        for c in range(int(cand_offsets[u]), int(cand_offsets[u + 1])):
+            t_c = int(ts_cand[c])
+            for h in range(H):
+                scores = []
+                values = []
+                for j in range(hs, he):
+                    sj = (float(q_c[c, h] @ k_hist[j, h]) * scale
+                          - slope_pos[h] * abs(p_c - int(pos_hist[j]))
+                          - slope_time[h] * abs(t_c - int(ts_hist[j])))
+                    scores.append(sj)
+                    values.append(v_hist[j, h])
+                scores.append(float(q_c[c, h] @ k_c[c, h]) * scale)
+                values.append(v_c[c, h])
+                sc = np.array(scores)
+                mx = sc.max()
+                w = np.exp(sc - mx)
+                O[c, h] = (w / w.sum()) @ np.array(values)
+                LSE[h, c] = mx + math.log(w.sum())
+    return O, LSE
+
+
+# ----------------------------------------------------------------------------------------
 # the model blocks around the hot path (projections, norms, FFN, head, loss)
 # ----------------------------------------------------------------------------------------
 

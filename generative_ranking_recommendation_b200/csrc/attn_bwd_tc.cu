@@ -7,10 +7,12 @@
 //   dQ = scale dS K,  dK = scale dS^T Q.
 //
 // Decomposition (bf16 inputs, head dim 64, fp32 accumulation):
-//   * A prologue lists (user, 128-key history tile) work records, longest first,
-//     and writes per token and head the ALiBi column term c_j (log2 units), the
-//     log2-domain LSE in column-term form lse2_i = LSE_i log2 e + c_i, and D_i, so
-//     that p_ij = 2^(scale log2e q_i.k_j + c_j - lse2_i) on every visible pair.
+//   * A prologue lists (user, 128-key history tile) work records, longest first, and
+//     a record per token (its user's scratch offset, candidate bit, time since the
+//     user's first token).  A per-row pass then writes per token and head the ALiBi
+//     column term c_j (log2 units), the log2-domain LSE in column-term form
+//     lse2_i = LSE_i log2 e + c_i, and D_i, so that
+//     p_ij = 2^(scale log2e q_i.k_j + c_j - lse2_i) on every visible pair.
 //   * One CTA per SM walks the records.  For a history key tile [k0, k0+128) the
 //     visible queries are the user's rows i >= j (later history rows and every
 //     candidate); they are visited one 128-row query tile at a time.
@@ -31,14 +33,16 @@
 //     accumulator in global memory: 32 rows x 32 columns at a time are staged in shared
 //     memory and reduced by the TMA engine (cp.reduce.async.bulk.tensor add), which
 //     keeps the load/store path free for the operand traffic of the tensor cores.  Per
-//     record they move dK (times scale) and dV from TMEM to global memory.
+//     record they move dK (times scale) and dV from TMEM to global memory through the
+//     same staging box, as whole 128-byte rows.
 //   * K and V are double-buffered by record, so the next record's loads and its
 //     first S^T, dP^T overlap the end of the current one.
 //   * Candidate keys are seen only by their own row; a small kernel applies that self
 //     term (dk, dv of candidate tokens, and ds k into the dQ accumulator), and a
 //     streaming pass writes dq = scale * dQ_acc.
-// Every mbarrier wait is bounded in time; a timeout sets GENRANK_DERR_TIMEOUT,
-// every role drains out of its loop and the CTA frees its tensor memory.
+// Every mbarrier wait is bounded in time; a timeout sets GENRANK_DERR_TIMEOUT, every
+// role drains out of its loop, the copies, MMAs and bulk reductions already issued are
+// waited for (bounded), and the CTA frees its tensor memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

@@ -8,6 +8,7 @@ the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 from .genrank_oracle import (  # noqa: F401
     alibi_slopes,
     attention_bwd,
+    attention_bwd_bucketed,
     attention_fwd,
     attention_fwd_bucketed,
     attention_fwd_cached,

@@ -293,6 +293,34 @@ def attention_fwd_bucketed(q, k, v, seq_offsets, hist_len, pos, ts, slope_pos, s
     return O, LSE
 
 
+def attention_bwd_bucketed(q, k, v, dO, seq_offsets, hist_len, pos, ts, slope_pos, slope_tb,
+                           scale, n_rt: int = 64, users=None):
+    """dQ, dK, dV of ``attention_fwd_bucketed``.  The bucketed bias has no parameters
+    either, so the gradients are those of ``attention_bwd`` with these scores:
+    dV = P^T dO, dS = P * (dP - rowsum(P * dP)), dQ = scale dS K, dK = scale dS^T Q."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    dO = np.asarray(dO, np.float64)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    users = range(len(hist_len)) if users is None else users
+    for u in users:
+        s, e, n = int(seq_offsets[u]), int(seq_offsets[u + 1]), int(hist_len[u])
+        p = np.asarray(pos[s:e], np.int64)
+        t = np.asarray(ts[s:e], np.int64)
+        for h in range(q.shape[1]):
+            Q, K, V, G = q[s:e, h], k[s:e, h], v[s:e, h], dO[s:e, h]
+            S = _user_scores_bucketed(Q, K, p, t, slope_pos[h], slope_tb[h], scale, n, n_rt)
+            P = np.exp(S - S.max(axis=1, keepdims=True))
+            P /= P.sum(axis=1, keepdims=True)
+            dP = G @ V.T
+            dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+            dq[s:e, h] = scale * dS @ K
+            dk[s:e, h] = scale * dS.T @ Q
+            dv[s:e, h] = P.T @ G
+    return dq, dk, dv
+
+
 # ----------------------------------------------------------------------------------------
 # variant: scoring candidates against cached history keys and values (a NEXT row)
 # ----------------------------------------------------------------------------------------

@@ -167,3 +167,27 @@ def test_planted_mistake_bucket_offset_is_caught(monkeypatch):
     except AssertionError:
         return
     raise AssertionError("the planted mistake was not caught")
+
+
+def test_backward_matches_finite_differences():
+    x = _tiny(14, users=((4, 2), (3, 1)), H=2, dh=3)
+    rng = np.random.default_rng(2)
+    G = rng.normal(size=x["q"].shape)
+    dq, dk, dv = oracle.attention_bwd_bucketed(x["q"], x["k"], x["v"], G, x["offs"], x["hl"],
+                                               x["pos"], x["ts"], x["sp"], x["stb"], x["scale"])
+    eps = 1e-6
+
+    def loss(y):
+        return float(np.sum(_call(y)[0] * G))
+
+    for name, grad in (("q", dq), ("k", dk), ("v", dv)):
+        for idx in [(0, 0, 0), (2, 1, 2), (5, 0, 1), (7, 1, 0), (9, 1, 1)]:
+            yp = dict(x)
+            ym = dict(x)
+            yp[name] = x[name].copy()
+            ym[name] = x[name].copy()
+            yp[name][idx] += eps
+            ym[name][idx] -= eps
+            fd = (loss(yp) - loss(ym)) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-7 * max(1.0, abs(fd)), (name, idx, fd, grad[idx])
+

@@ -47,6 +47,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "host_util.h"
 #include "kernels.h"
 
 namespace gr {
@@ -950,16 +951,11 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
                                                       (float*)p.lse2, (float*)p.dsum, p.Tp);
     if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   }
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(k_attn_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes) != cudaSuccess)
-      return GENRANK_ERR_CUDA;
-    attr = true;
-  }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static DeviceOnce smem_attr;
+  if (!set_smem_limit_once(smem_attr, (const void*)k_attn_bwd_tc, (int)kSmemBytes))
+    return GENRANK_ERR_CUDA;
+  const int sms = sm_count_current();
+  if (sms <= 0) return GENRANK_ERR_CUDA;
   k_attn_bwd_tc<<<sms, kThreads, kSmemBytes, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   if (a.B > 0) {

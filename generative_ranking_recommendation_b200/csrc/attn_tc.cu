@@ -36,6 +36,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "host_util.h"
 #include "kernels.h"
 
 namespace gr {
@@ -833,16 +834,11 @@ int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
   p.Tp = scratch_tp(a.T, a.B);
   k_prologue<<<a.B + 1, kSchedThreads, 0, st>>>(a, max_tiles, recs, count, uorder, cbias, p.Tp);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(k_attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes) != cudaSuccess)
-      return GENRANK_ERR_CUDA;
-    attr = true;
-  }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static DeviceOnce smem_attr;
+  if (!set_smem_limit_once(smem_attr, (const void*)k_attn_fwd_tc, (int)kSmemBytes))
+    return GENRANK_ERR_CUDA;
+  const int sms = sm_count_current();
+  if (sms <= 0) return GENRANK_ERR_CUDA;
   k_attn_fwd_tc<<<sms, kThreads, kSmemBytes, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
 }

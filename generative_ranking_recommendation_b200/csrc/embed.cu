@@ -7,6 +7,7 @@
 // request-index embedding |{t_1..t_i}| and the pre-request time embedding
 // bucket(t_i - max_{t_j < t_i} t_j).
 #include "common.cuh"
+#include "host_util.h"
 #include "kernels.h"
 
 namespace gr {
@@ -343,14 +344,8 @@ __global__ void __launch_bounds__(1024) k_embed_bwd(
 // host launchers
 // ------------------------------------------------------------------------------------------
 static int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
+  const int n = sm_count_current();
+  return n > 0 ? n : 148;  // only sizes the grid
 }
 
 int launch_embed_fwd(const EmbedFwdArgs& a, cudaStream_t st) {

@@ -2,6 +2,7 @@
 // candidate rows ("GenRank [2025]" chapter notes §1.3.1: the output lives at
 // candidate positions; u = W_o w_head is formed by the caller).
 #include "common.cuh"
+#include "host_util.h"
 #include "kernels.h"
 
 namespace gr {
@@ -52,9 +53,8 @@ __global__ void __launch_bounds__(256) k_cand_logits(const CandLogitsArgs a) {
 
 int launch_cand_logits(const CandLogitsArgs& a, cudaStream_t st) {
   if (a.M == 0) return GENRANK_OK;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int n = sm_count_current();
+  const int sms = n > 0 ? n : 148;  // only sizes the grid
   const long long blocks = (a.M + 7) / 8;
   const int grid = (int)(blocks < 16LL * sms ? blocks : 16LL * sms);
   if (a.dtype == GENRANK_BF16)

@@ -13,36 +13,31 @@
 // Every GPU on which the library is loaded holds it until the process exits.
 // Host code cannot use the array's name as a device address; its address is
 // looked up once per device with cudaGetSymbolAddress, with that device current.
-#include <mutex>
-
 #include "common.cuh"
+#include "host_util.h"
 #include "kernels.h"
 
 namespace gr {
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_attn_scratch[kStaticScratchBytes];
 
 void* g_scratch_addr[kMaxDevices] = {};
-std::once_flag g_scratch_once[kMaxDevices];
-cudaError_t g_scratch_status[kMaxDevices] = {};
 
-// Address of the scratch array on the current device, looked up on first use.
+// Address of the scratch array on the current device, looked up once per device (with
+// that device current) by cudaGetSymbolAddress.
 void* scratch_for_current_device(int* code) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    *code = GENRANK_ERR_CUDA;
-    return nullptr;
-  }
-  std::call_once(g_scratch_once[dev], [dev] {
+  static DeviceOnce once;
+  const int ok = once.run([](int dev) {
     void* p = nullptr;
-    g_scratch_status[dev] = cudaGetSymbolAddress(&p, g_attn_scratch);
-    g_scratch_addr[dev] = g_scratch_status[dev] == cudaSuccess ? p : nullptr;
+    if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess || !p) return 0;
+    g_scratch_addr[dev] = p;
+    return 1;
   });
-  if (g_scratch_status[dev] != cudaSuccess || !g_scratch_addr[dev]) {
+  int dev = 0;
+  if (ok != 1 || cudaGetDevice(&dev) != cudaSuccess) {
     *code = GENRANK_ERR_CUDA;
     return nullptr;
   }
@@ -64,7 +59,10 @@ int genrank_attn_fwd_static(int B, int64_t T, const int32_t* seq_offsets,
   if (B < 1 || T < 0 || H < 1 || dh < 1 || max_seqlen < 0) return GENRANK_ERR_INVALID_ARG;
   const size_t need = genrank_attn_workspace_size(B, T, H, dh, max_seqlen, 0);
   if (need == 0) return GENRANK_ERR_INVALID_ARG;
-  if (need > gr::kStaticScratchBytes) return GENRANK_ERR_WORKSPACE;
+  // only the tensor-core kernel (bf16, head dim 64) uses scratch; the CUDA-core kernel
+  // runs without any, whatever the sizes
+  const bool uses_scratch = dtype == GENRANK_BF16 && dh == 64;
+  if (uses_scratch && need > gr::kStaticScratchBytes) return GENRANK_ERR_WORKSPACE;
   int code = GENRANK_OK;
   void* ws = gr::scratch_for_current_device(&code);
   if (code != GENRANK_OK) return code;

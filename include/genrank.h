@@ -198,8 +198,10 @@ int genrank_attn_bwd(int B, int64_t T, const int32_t *seq_offsets, const int32_t
  * the same arguments as genrank_attn_fwd minus the workspace: its scratch is a
  * 16 MiB array compiled into the library, which every GPU that loads the library
  * holds until the process exits.  Inputs and outputs are still the caller's.
- *   - Sizes whose workspace (genrank_attn_workspace_size(..., 0)) exceeds
- *     16 MiB are rejected with GENRANK_ERR_WORKSPACE before any launch.
+ *   - Only the tensor-core kernel (bf16, dh = 64) uses the array.  For it, sizes
+ *     whose workspace (genrank_attn_workspace_size(..., 0)) exceeds 16 MiB are
+ *     rejected with GENRANK_ERR_WORKSPACE before any launch; the CUDA-core kernel
+ *     (fp32, or dh = 32) needs no scratch and takes any size.
  *   - The first call on each device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
  *   - Every call on a device shares the one array and leaves its contents

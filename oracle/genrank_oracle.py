@@ -330,9 +330,10 @@ def attention_fwd_cached(q_c, k_c, v_c, cand_offsets, k_hist, v_hist, hist_offse
     """O [C,H,dh] and natural-log LSE [H,C] of the candidate rows only, from a cache of the
     users' history keys and values.
 
-    [HXZ] §1.3.1 credits the KV cache with making generative ranking cheaper as the
-    candidate set grows; [HXZ] §1.4.1 and [FUN-EN] §7.2.1 fix what a candidate sees: the
-    whole history of its user and itself.  User u's history rows are
+    [HXZ] §1.3.2 (its feature-engineering paragraph) credits the KV cache with keeping
+    generative ranking efficient as the candidate set grows, and [FUN-EN] §7.2.1 counts
+    the halved KV cache among the action-oriented layout's gains.  [HXZ] §1.4.1 and
+    [FUN-EN] §7.2.1 fix what a candidate sees: the whole history of its user and itself.  User u's history rows are
     k_hist/v_hist[hist_offsets[u]:hist_offsets[u+1]] with positions pos_hist and times
     ts_hist; its candidates are rows cand_offsets[u]:cand_offsets[u+1] of q_c, k_c, v_c,
     all at position n_u + 1 and time ts_cand.  The score of candidate c against history

@@ -136,11 +136,11 @@ def test_embed_device_error_flags(G):
 # ------------------------------------------------------------------------------------------
 # backward
 # ------------------------------------------------------------------------------------------
-@pytest.mark.parametrize("name,B", [("c0", None), ("c3", None)])
-def test_embed_bwd_parity(G, name, B):
-    cfg = CONFIGS[name] if B is None else CONFIGS[name].with_(B=B)
-    if name == "c3":
-        cfg = cfg.with_(n_item=200_000)
+@pytest.mark.parametrize("name", ["c0", "c3"])
+def test_embed_bwd_parity(G, name):
+    """c3 runs on its full 4M-row item table, so the Zipf(1.05)-hot rows meet the
+    contention they meet in training; rows no token reads must stay exactly zero."""
+    cfg = CONFIGS[name]
     batch = make_batch(cfg)
     mr = ref.meta(batch)
     T, d = batch.T, cfg.d
@@ -162,9 +162,11 @@ def test_embed_bwd_parity(G, name, B):
     want = oracle.embed_assemble_bwd(dE_used, batch.seq_offsets, batch.hist_len, inv,
                                      batch.action_ids, mr, len(uniq), 9, cfg.n_pos, cfg.n_ri,
                                      cfg.n_rt)
-    got_item = g[0].cpu().numpy().astype(np.float64)
-    assert np.all(np.delete(got_item, uniq, axis=0) == 0.0)
-    pairs = [(got_item[uniq], want["item"])] + [
+    touched = torch.zeros(cfg.n_item, dtype=torch.bool, device="cuda")
+    touched[_dev(uniq.astype(np.int64))] = True
+    assert float(g[0][~touched].abs().max()) == 0.0  # on the device: the table is 8 GB at c3
+    got_item = g[0][_dev(uniq.astype(np.int64))].cpu().numpy().astype(np.float64)
+    pairs = [(got_item, want["item"])] + [
         (t.cpu().numpy().astype(np.float64), want[k])
         for t, k in zip(g[1:], ("action", "pos", "ri", "rt"))]
     for got, w in pairs:

@@ -1,8 +1,8 @@
 """Pins for the oracle's candidate scoring from cached history keys and values.
 
 Scoring a request's candidates against a user's cached history must give exactly the
-candidate rows of the full batched attention ("GenRank [2025]" chapter notes §1.3.1 on
-the KV cache; §1.4.1 and fun-rec §7.2.1 on what a candidate sees).
+candidate rows of the full batched attention ("GenRank [2025]" chapter notes §1.3.2 on
+the KV cache, with fun-rec §7.2.1; §1.4.1 and fun-rec §7.2.1 on what a candidate sees).
 """
 
 import math

@@ -85,3 +85,35 @@ def test_static_scratch_rejects_oversized_workloads():
         i = torch.zeros(2, dtype=torch.int32, device="cuda")
         G.attn_fwd_static(i, i[:1], 128, x, x, x, 3 * 1024, 16, 64, i, i.long(), [0.5] * 16,
                           [0.5 / 3600] * 16, 0.125, x, 1024, None, i, T=1_000_000)
+
+
+def test_static_entry_takes_any_size_on_the_cuda_core_path():
+    """fp32 runs the CUDA-core kernel, which needs no scratch: a batch whose tensor-core
+    workspace would exceed the fixed 16 MiB still runs, and matches genrank_attn_fwd."""
+    from generative_ranking_recommendation_b200 import genrank as G
+
+    B, H, dh = 300_000, 1, 32  # users of one history token and one candidate
+    T = 2 * B
+    assert G.attn_workspace_size(B, T, H, 64, 2, False) > (16 << 20)
+    off = torch.arange(0, T + 1, 2, dtype=torch.int32, device="cuda")
+    hl = torch.ones(B, dtype=torch.int32, device="cuda")
+    pos = torch.tensor([1, 2], dtype=torch.int32, device="cuda").repeat(B)
+    ts = (1_700_000_000 + torch.arange(T, dtype=torch.int64, device="cuda") // 2 * 7
+          + torch.tensor([0, 5], dtype=torch.int64, device="cuda").repeat(B))
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    q = torch.randn((T, 3 * H * dh), generator=gen, device="cuda")
+    d = H * dh
+    sp, st = G.alibi_slopes(H)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o_ref = torch.empty((T, d), device="cuda")
+    l_ref = torch.empty((H, T), device="cuda")
+    G.attn_fwd(off, hl, 2, q, q[:, d:], q[:, 2 * d:], 3 * d, H, dh, pos, ts, sp, st,
+               1.0 / math.sqrt(dh), o_ref, d, l_ref, None, err, T=T)
+    for _ in range(2):
+        o = torch.full((T, d), float("nan"), device="cuda")
+        lse = torch.full((H, T), float("nan"), device="cuda")
+        G.attn_fwd_static(off, hl, 2, q, q[:, d:], q[:, 2 * d:], 3 * d, H, dh, pos, ts, sp, st,
+                          1.0 / math.sqrt(dh), o, d, lse, err, T=T)
+        assert G.check_error(err) == 0
+        assert float((o - o_ref).abs().max()) <= 1e-4
+        assert float((lse - l_ref).abs().max()) <= 1e-4

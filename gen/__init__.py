@@ -14,6 +14,8 @@ from .synth import (  # noqa: F401
     Model,
     bf16_round,
     config_by_name,
+    dense_bias_torch,
+    interleave_batch,
     item_rows,
     item_table_torch,
     make_batch,

@@ -364,3 +364,40 @@ def make_qkv(cfg: Config, T: int, seed: int, std: float = 1.0, n: int = 3) -> np
     """Standalone attention operands: ``n`` arrays [T, H, dh] stacked as [T, n, H, dh]."""
     rng = np.random.default_rng([seed, 40])
     return _cast(rng.normal(0.0, std, size=(T, n, cfg.H, cfg.dh)), cfg.dtype)
+
+
+# ----------------------------------------------------------------------------------------
+# comparison inputs: the interleaved layout and a dense per-user bias
+# ----------------------------------------------------------------------------------------
+
+def interleave_batch(batch: Batch) -> Batch:
+    """The same users laid out as the interleaved organisation does: each history
+    interaction becomes two tokens (the item, then its action; both at the interaction's
+    time), followed by the candidates.  Item ids of action tokens are the action index;
+    only the layout matters to the attention that consumes it."""
+    offs, hl, items, acts, ts = [0], [], [], [], []
+    for u in range(batch.B):
+        s, e, n = int(batch.seq_offsets[u]), int(batch.seq_offsets[u + 1]), int(batch.hist_len[u])
+        it2 = np.empty(2 * n, np.int32)
+        it2[0::2] = batch.item_ids[s:s + n]
+        it2[1::2] = batch.action_ids[s:s + n]
+        ac2 = np.empty(2 * n, np.int32)
+        ac2[0::2] = batch.action_ids[s:s + n]
+        ac2[1::2] = batch.action_ids[s:s + n]
+        items += [it2, batch.item_ids[s + n:e]]
+        acts += [ac2, batch.action_ids[s + n:e]]
+        ts += [np.repeat(batch.ts[s:s + n], 2), batch.ts[s + n:e]]
+        hl.append(2 * n)
+        offs.append(offs[-1] + 2 * n + (e - s - n))
+    cat = (lambda xs, dt: np.concatenate(xs).astype(dt) if xs else np.zeros(0, dt))
+    return Batch(batch.cfg, list(batch.users), np.array(offs, np.int32), np.array(hl, np.int32),
+                 cat(items, np.int32), cat(acts, np.int32), cat(ts, np.int64), batch.labels)
+
+
+def dense_bias_torch(seed: int, B: int, Lpad: int, device, std: float = 0.5):
+    """A bf16 [B, Lpad, Lpad] tensor of N(0, std) values (a stand-in for a learned
+    relative bias), drawn on ``device`` by a seeded torch generator."""
+    import torch
+
+    g = torch.Generator(device=device).manual_seed(int(seed))
+    return (torch.randn((B, Lpad, Lpad), generator=g, device=device) * std).to(torch.bfloat16)

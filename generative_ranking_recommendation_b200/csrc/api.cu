@@ -66,6 +66,67 @@ int check_attn_common(int B, int64_t T, const int32_t* off, const int32_t* hl, i
 
 bool use_tc(int dtype, int dh) { return dtype == GENRANK_BF16 && dh == 64; }
 
+// genrank_attn_fwd with the linear or the bucketed time bias
+int attn_fwd_impl(int time_bias, int B, int64_t T, const int32_t* seq_offsets,
+                  const int32_t* hist_len, int max_seqlen, const void* q, const void* k,
+                  const void* v, int64_t tok_stride, int H, int dh, const int32_t* pos,
+                  const int64_t* ts, const float* slope_pos, const float* slope_time, float scale,
+                  int dtype, void* o, int64_t o_stride, float* lse, void* ws, size_t ws_bytes,
+                  int32_t* dev_err, genrank_stream_t stream) {
+  int rc = check_attn_common(B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh,
+                             pos, ts, slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  if (rc) return rc;
+  if (T > 0 && (!o || !aligned16(o))) return GENRANK_ERR_INVALID_ARG;
+  if (!use_tc(dtype, dh) && dh != 32 && dh != 64) return GENRANK_ERR_UNSUPPORTED;
+  const size_t need = genrank_attn_workspace_size(B, T, H, dh, max_seqlen, 0);
+  if (use_tc(dtype, dh) && (!ws || ws_bytes < need || !aligned16(ws))) return GENRANK_ERR_WORKSPACE;
+  if (T == 0) return GENRANK_OK;
+  AttnArgs a;
+  fill_attn(a, B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts,
+            slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  a.time_bias = time_bias;
+  a.o = o;
+  a.lse = lse;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return use_tc(dtype, dh) ? launch_attn_fwd_tc(a, s) : launch_attn_fwd_simt(a, s);
+}
+
+// genrank_attn_bwd with the linear or the bucketed time bias
+int attn_bwd_impl(int time_bias, int B, int64_t T, const int32_t* seq_offsets,
+                  const int32_t* hist_len, int max_seqlen, const void* q, const void* k,
+                  const void* v, int64_t tok_stride, int H, int dh, const int32_t* pos,
+                  const int64_t* ts, const float* slope_pos, const float* slope_time, float scale,
+                  int dtype, const void* o, const void* dO, int64_t o_stride, const float* lse,
+                  void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, int32_t* dev_err,
+                  genrank_stream_t stream) {
+  int rc = check_attn_common(B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh,
+                             pos, ts, slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  if (rc) return rc;
+  if (T > 0 && (!o || !dO || !lse || !dq || !dk || !dv)) return GENRANK_ERR_INVALID_ARG;
+  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(o) || !aligned16(dO))
+    return GENRANK_ERR_INVALID_ARG;
+  if (dh != 32 && dh != 64) return GENRANK_ERR_UNSUPPORTED;
+  const size_t need = genrank_attn_workspace_size(B, T, H, dh, max_seqlen, 1);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return GENRANK_ERR_WORKSPACE;
+  if (T == 0) return GENRANK_OK;
+  AttnArgs a;
+  fill_attn(a, B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts,
+            slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  a.time_bias = time_bias;
+  a.o = const_cast<void*>(o);
+  a.dO = dO;
+  a.lse_in = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return use_tc(dtype, dh) ? launch_attn_bwd_tc(a, s) : launch_attn_bwd_simt(a, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -210,23 +271,127 @@ int genrank_attn_fwd(int B, int64_t T, const int32_t* seq_offsets, const int32_t
                      const float* slope_pos, const float* slope_time, float scale, int dtype,
                      void* o, int64_t o_stride, float* lse, void* ws, size_t ws_bytes,
                      int32_t* dev_err, genrank_stream_t stream) {
-  int rc = check_attn_common(B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh,
-                             pos, ts, slope_pos, slope_time, scale, dtype, o_stride, dev_err);
-  if (rc) return rc;
-  if (T > 0 && (!o || !aligned16(o))) return GENRANK_ERR_INVALID_ARG;
-  if (!use_tc(dtype, dh) && dh != 32 && dh != 64) return GENRANK_ERR_UNSUPPORTED;
+  return attn_fwd_impl(kTimeBiasLinear, B, T, seq_offsets, hist_len, max_seqlen, q, k, v,
+                       tok_stride, H, dh, pos, ts, slope_pos, slope_time, scale, dtype, o,
+                       o_stride, lse, ws, ws_bytes, dev_err, stream);
+}
+
+int genrank_attn_fwd_bucketed(int B, int64_t T, const int32_t* seq_offsets,
+                              const int32_t* hist_len, int max_seqlen, const void* q,
+                              const void* k, const void* v, int64_t tok_stride, int H, int dh,
+                              const int32_t* pos, const int64_t* ts, const float* slope_pos,
+                              const float* slope_tb, float scale, int dtype, void* o,
+                              int64_t o_stride, float* lse, void* ws, size_t ws_bytes,
+                              int32_t* dev_err, genrank_stream_t stream) {
+  if (!use_tc(dtype, dh)) return GENRANK_ERR_UNSUPPORTED;
+  return attn_fwd_impl(kTimeBiasBucketed, B, T, seq_offsets, hist_len, max_seqlen, q, k, v,
+                       tok_stride, H, dh, pos, ts, slope_pos, slope_tb, scale, dtype, o,
+                       o_stride, lse, ws, ws_bytes, dev_err, stream);
+}
+
+int genrank_attn_fwd_dense_bias(int B, int64_t T, const int32_t* seq_offsets,
+                                const int32_t* hist_len, int max_seqlen, const void* q,
+                                const void* k, const void* v, int64_t tok_stride, int H, int dh,
+                                const void* bias, int64_t Lpad, float scale, int dtype, void* o,
+                                int64_t o_stride, float* lse, void* ws, size_t ws_bytes,
+                                int32_t* dev_err, genrank_stream_t stream) {
+  if (B < 1 || T < 0 || max_seqlen < 0 || H < 1 || dh < 1 || !seq_offsets || !hist_len ||
+      !dev_err || !(scale > 0.f) || !isfinite(scale))
+    return GENRANK_ERR_INVALID_ARG;
+  if (H > kMaxHeads) return GENRANK_ERR_UNSUPPORTED;
+  if (!use_tc(dtype, dh)) return GENRANK_ERR_UNSUPPORTED;
+  if (T > 0 && (!q || !k || !v || !o || !bias)) return GENRANK_ERR_INVALID_ARG;
+  if (tok_stride < (int64_t)H * dh || o_stride < (int64_t)H * dh || (tok_stride * 2) % 16 ||
+      (o_stride * 2) % 16)
+    return GENRANK_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(bias))
+    return GENRANK_ERR_INVALID_ARG;
+  // every tile a work item reads lies in the user's Lpad x Lpad block
+  if (Lpad < 128 || Lpad % 128 || Lpad < max_seqlen) return GENRANK_ERR_INVALID_ARG;
   const size_t need = genrank_attn_workspace_size(B, T, H, dh, max_seqlen, 0);
-  if (use_tc(dtype, dh) && (!ws || ws_bytes < need || !aligned16(ws))) return GENRANK_ERR_WORKSPACE;
+  if (!ws || ws_bytes < need || !aligned16(ws)) return GENRANK_ERR_WORKSPACE;
   if (T == 0) return GENRANK_OK;
   AttnArgs a;
-  fill_attn(a, B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts,
-            slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  memset(&a, 0, sizeof(a));
+  a.B = B;
+  a.T = T;
+  a.off = seq_offsets;
+  a.hist_len = hist_len;
+  a.max_seqlen = max_seqlen;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.tok_stride = tok_stride;
+  a.H = H;
+  a.dh = dh;
+  a.scale = scale;
+  a.dtype = dtype;
   a.o = o;
+  a.o_stride = o_stride;
   a.lse = lse;
   a.ws = ws;
   a.ws_bytes = ws_bytes;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return use_tc(dtype, dh) ? launch_attn_fwd_tc(a, s) : launch_attn_fwd_simt(a, s);
+  a.err = dev_err;
+  return launch_attn_fwd_dense(a, bias, Lpad, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t genrank_attn_cached_workspace_size(int B, int64_t C, int64_t Th, int H, int dh,
+                                          int max_cand) {
+  if (B < 1 || C < 0 || Th < 0 || H < 1 || dh < 1 || max_cand < 0) return 0;
+  return attn_fwd_cached_workspace(B, C, Th, H, max_cand);
+}
+
+int genrank_attn_fwd_cached(int B, int64_t C, const int32_t* cand_offsets, int max_cand,
+                            const void* q_c, const void* k_c, const void* v_c,
+                            int64_t cand_stride, int64_t Th, const int32_t* hist_offsets,
+                            const void* k_hist, const void* v_hist, int64_t hist_stride,
+                            const int32_t* pos_hist, const int64_t* ts_hist,
+                            const int64_t* ts_cand, int H, int dh, const float* slope_pos,
+                            const float* slope_time, float scale, int dtype, void* o,
+                            int64_t o_stride, float* lse, void* ws, size_t ws_bytes,
+                            int32_t* dev_err, genrank_stream_t stream) {
+  if (B < 1 || C < 0 || Th < 0 || max_cand < 0 || H < 1 || dh < 1 || !cand_offsets ||
+      !hist_offsets || !ts_cand || !slope_pos || !slope_time || !dev_err || !(scale > 0.f) ||
+      !isfinite(scale))
+    return GENRANK_ERR_INVALID_ARG;
+  if (H > kMaxHeads) return GENRANK_ERR_UNSUPPORTED;
+  const int es = elem_size(dtype);
+  if (!es) return GENRANK_ERR_INVALID_ARG;
+  if (C > 0 && (!q_c || !k_c || !v_c)) return GENRANK_ERR_INVALID_ARG;
+  if (cand_stride < (int64_t)H * dh || o_stride < (int64_t)H * dh ||
+      (cand_stride * es) % 16 || (o_stride * es) % 16 || (dh * es) % 16)
+    return GENRANK_ERR_INVALID_ARG;
+  if (!aligned16(q_c) || !aligned16(k_c) || !aligned16(v_c)) return GENRANK_ERR_INVALID_ARG;
+  for (int h = 0; h < H; ++h)
+    if (!isfinite(slope_pos[h]) || !isfinite(slope_time[h]) || slope_pos[h] < 0.f ||
+        slope_time[h] < 0.f)
+      return GENRANK_ERR_INVALID_ARG;
+  if (Th > 0 && (!k_hist || !v_hist || !pos_hist || !ts_hist)) return GENRANK_ERR_INVALID_ARG;
+  if (Th > 0 && (hist_stride < (int64_t)H * dh || !aligned16(k_hist) || !aligned16(v_hist) ||
+                 (hist_stride * es) % 16))
+    return GENRANK_ERR_INVALID_ARG;
+  if (C > 0 && (!o || !aligned16(o))) return GENRANK_ERR_INVALID_ARG;
+  if (!use_tc(dtype, dh)) return GENRANK_ERR_UNSUPPORTED;
+  const size_t need = genrank_attn_cached_workspace_size(B, C, Th, H, dh, max_cand);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return GENRANK_ERR_WORKSPACE;
+  if (C == 0) return GENRANK_OK;
+  CachedAttnArgs c;
+  memset(&c, 0, sizeof(c));
+  fill_attn(c.a, B, C, cand_offsets, nullptr, max_cand, q_c, k_c, v_c, cand_stride, H, dh,
+            nullptr, ts_cand, slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  c.a.o = o;
+  c.a.lse = lse;
+  c.a.ws = ws;
+  c.a.ws_bytes = ws_bytes;
+  c.hist_off = hist_offsets;
+  c.k_hist = k_hist;
+  c.v_hist = v_hist;
+  c.hist_stride = hist_stride;
+  c.Th = Th;
+  c.pos_hist = pos_hist;
+  c.ts_hist = ts_hist;
+  c.max_cand = max_cand;
+  return launch_attn_fwd_cached(c, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int genrank_attn_bwd(int B, int64_t T, const int32_t* seq_offsets, const int32_t* hist_len,
@@ -236,29 +401,23 @@ int genrank_attn_bwd(int B, int64_t T, const int32_t* seq_offsets, const int32_t
                      const void* o, const void* dO, int64_t o_stride, const float* lse, void* dq,
                      void* dk, void* dv, void* ws, size_t ws_bytes, int32_t* dev_err,
                      genrank_stream_t stream) {
-  int rc = check_attn_common(B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh,
-                             pos, ts, slope_pos, slope_time, scale, dtype, o_stride, dev_err);
-  if (rc) return rc;
-  if (T > 0 && (!o || !dO || !lse || !dq || !dk || !dv)) return GENRANK_ERR_INVALID_ARG;
-  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(o) || !aligned16(dO))
-    return GENRANK_ERR_INVALID_ARG;
-  if (dh != 32 && dh != 64) return GENRANK_ERR_UNSUPPORTED;
-  const size_t need = genrank_attn_workspace_size(B, T, H, dh, max_seqlen, 1);
-  if (!ws || ws_bytes < need || !aligned16(ws)) return GENRANK_ERR_WORKSPACE;
-  if (T == 0) return GENRANK_OK;
-  AttnArgs a;
-  fill_attn(a, B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts,
-            slope_pos, slope_time, scale, dtype, o_stride, dev_err);
-  a.o = const_cast<void*>(o);
-  a.dO = dO;
-  a.lse_in = lse;
-  a.dq = dq;
-  a.dk = dk;
-  a.dv = dv;
-  a.ws = ws;
-  a.ws_bytes = ws_bytes;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return use_tc(dtype, dh) ? launch_attn_bwd_tc(a, s) : launch_attn_bwd_simt(a, s);
+  return attn_bwd_impl(kTimeBiasLinear, B, T, seq_offsets, hist_len, max_seqlen, q, k, v,
+                       tok_stride, H, dh, pos, ts, slope_pos, slope_time, scale, dtype, o, dO,
+                       o_stride, lse, dq, dk, dv, ws, ws_bytes, dev_err, stream);
+}
+
+int genrank_attn_bwd_bucketed(int B, int64_t T, const int32_t* seq_offsets,
+                              const int32_t* hist_len, int max_seqlen, const void* q,
+                              const void* k, const void* v, int64_t tok_stride, int H, int dh,
+                              const int32_t* pos, const int64_t* ts, const float* slope_pos,
+                              const float* slope_tb, float scale, int dtype, const void* o,
+                              const void* dO, int64_t o_stride, const float* lse, void* dq,
+                              void* dk, void* dv, void* ws, size_t ws_bytes, int32_t* dev_err,
+                              genrank_stream_t stream) {
+  if (!use_tc(dtype, dh)) return GENRANK_ERR_UNSUPPORTED;
+  return attn_bwd_impl(kTimeBiasBucketed, B, T, seq_offsets, hist_len, max_seqlen, q, k, v,
+                       tok_stride, H, dh, pos, ts, slope_pos, slope_tb, scale, dtype, o, dO,
+                       o_stride, lse, dq, dk, dv, ws, ws_bytes, dev_err, stream);
 }
 
 }  // extern "C"

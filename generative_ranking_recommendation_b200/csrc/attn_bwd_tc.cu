@@ -68,7 +68,8 @@ constexpr uint32_t kOffQ = kOffV + 2 * kTileBytes;     // 2 stages
 constexpr uint32_t kOffDO = kOffQ + 2 * kTileBytes;    // 2 stages
 constexpr uint32_t kOffL2 = kOffDO + 2 * kTileBytes;   // lse2, 2 stages
 constexpr uint32_t kOffD = kOffL2 + 2 * kRowBytes;     // D, 2 stages
-constexpr uint32_t kOffDS = kOffD + 2 * kRowBytes;     // dS^T, 2 buffers
+constexpr uint32_t kOffTQ = kOffD + 2 * kRowBytes;     // bucketed bias: query times, 2 stages
+constexpr uint32_t kOffDS = kOffTQ + 2 * kRowBytes;    // dS^T, 2 buffers
 constexpr uint32_t kOffStage = kOffDS + 2 * kPSBytes;  // dQ_part staging, 4 x 4 KB
 constexpr uint32_t kStageBytes = 32 * 32 * 4;           // 32 rows x 32 fp32 columns
 constexpr uint32_t kOffBar = kOffStage + 4 * kStageBytes;
@@ -107,6 +108,7 @@ struct Params {
   const float* cbias;  // [H][Tp]
   const float* lse2;   // [H][Tp]
   const float* dsum;   // [H][Tp]  (D)
+  const int32_t* trel; // [Tp] bucketed bias: per-token time since the user's first token
   float* dqacc;        // [T][H][64]
   long long Tp;
 };
@@ -142,9 +144,16 @@ __host__ __device__ inline long long scratch_tp(long long T, int B) {
 // ------------------------------------------------------------------------------------------
 constexpr int kMaxBuckets = 257;
 // Per-token info: x = (user segment start in the scratch - user start) | kCandBit for a
-// candidate token; y = the float bits of t - t_0 (seconds since the user's first token).
+// candidate token; y = the float bits of t - t_0 (seconds since the user's first token),
+// or for the bucketed time bias t - t_0 itself as an int, clamped to [0, kMaxRelTime).
 // Tokens of no valid user keep the memset value, x = -1.
 constexpr int kCandBit = 1 << 30;
+constexpr int kMaxRelTime = 1 << 29;
+// bucketed time bias: see the forward kernel (gap biased so its bits read as the float
+// 2^23 + gap + 1; the bucket is the binary exponent of (gap + 1)^4, capped at 62)
+constexpr int kTimeMagic = 0x4B000001;
+constexpr int kTimeCap = kTimeMagic + 46340;
+constexpr float kTwo23 = 8388608.f;
 
 __global__ void __launch_bounds__(256) k_bwd_prologue(const __grid_constant__ AttnArgs a,
                                                       int max_tiles, int4* recs, int32_t* count,
@@ -156,9 +165,13 @@ __global__ void __launch_bounds__(256) k_bwd_prologue(const __grid_constant__ At
     const int n = (int)max(0LL, min((long long)a.hist_len[b], e - s));
     const int segoff = (int)(seg_start(s, b) - s);
     const long long t0 = e > s ? a.ts[s] : 0;  // (an empty user reads nothing)
-    for (long long t = s + threadIdx.x; t < e; t += blockDim.x)
+    const bool bucket = a.time_bias == kTimeBiasBucketed;
+    for (long long t = s + threadIdx.x; t < e; t += blockDim.x) {
+      const long long dt = a.ts[t] - t0;
       tinfo[t] = make_int2(segoff | (t - s >= n ? kCandBit : 0),
-                           __float_as_int((float)(a.ts[t] - t0)));
+                           bucket ? (int)min(max(dt, 0LL), (long long)kMaxRelTime - 1)
+                                  : __float_as_int((float)dt));
+    }
     return;
   }
   // Records go out user by user (users with the most history key tiles first, each
@@ -237,10 +250,12 @@ __global__ void __launch_bounds__(256) k_bwd_prologue(const __grid_constant__ At
 // c_j = log2 e (m_h p_j + m_t,h (t_j - t_0)), lse2_i = LSE_i log2 e + c_i and
 // D_i = rowsum(dO_i * O_i), at the user's segment of the [H][Tp] scratch.  Every load
 // is issued up front (the per-token info replaces a chain through the user's offsets).
+// With the bucketed time bias, c_j holds the position part only and the token's time
+// goes to trel (written by the head-0 lane).
 __global__ void __launch_bounds__(256) k_bwd_rows(const __grid_constant__ AttnArgs a,
                                                   const int2* __restrict__ tinfo,
                                                   float* cbias, float* lse2, float* dsum,
-                                                  long long Tp) {
+                                                  int32_t* trel, long long Tp) {
   const long long x = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 3;  // pair
   const int sub = threadIdx.x & 7;
   const long long tend = min(a.T, (long long)a.off[a.B]);
@@ -269,8 +284,15 @@ __global__ void __launch_bounds__(256) k_bwd_rows(const __grid_constant__ AttnAr
   dd += __shfl_xor_sync(0xffffffffu, dd, 1);
   if (!live || sub != 0) return;
   if (ti.x < 0) return;  // tokens of no valid user (the schedule flags the layout)
-  const float c = kLog2e * (a.slope_pos[h] * (float)pos + a.slope_time[h] * __int_as_float(ti.y));
-  const long long idx = (long long)h * Tp + tok + (ti.x & (kCandBit - 1));
+  const long long seg_tok = tok + (ti.x & (kCandBit - 1));
+  float c;
+  if (a.time_bias == kTimeBiasBucketed) {
+    c = kLog2e * (a.slope_pos[h] * (float)pos);
+    if (h == 0) trel[seg_tok] = ti.y;
+  } else {
+    c = kLog2e * (a.slope_pos[h] * (float)pos + a.slope_time[h] * __int_as_float(ti.y));
+  }
+  const long long idx = (long long)h * Tp + seg_tok;
   cbias[idx] = c;
   lse2[idx] = lse * kLog2e + c;
   dsum[idx] = dd;
@@ -301,6 +323,7 @@ GR_DEVICE void store_row_chunk16(uint8_t* tile, int r, int c0, const uint32_t (&
   }
 }
 
+template <bool kBucket>
 __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_constant__ Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -378,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
         }
         if (lane == 0) {
           const int q0 = rc.k0 + t * BM;
-          mbar_expect_tx(&bars[kQDFull + st], 2 * kTileBytes + 2 * kRowBytes);
+          mbar_expect_tx(&bars[kQDFull + st], 2 * kTileBytes + (kBucket ? 3 : 2) * kRowBytes);
           tma_load_3d(smem + kOffQ + st * kTileBytes, &P.tq, &bars[kQDFull + st], 0, rc.h,
                       rc.s + q0);
           tma_load_3d(smem + kOffDO + st * kTileBytes, &P.tdo, &bars[kQDFull + st], 0, rc.h,
@@ -387,6 +410,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
                     &bars[kQDFull + st]);
           bulk_load(smem + kOffD + st * kRowBytes, P.dsum + roff + q0, kRowBytes,
                     &bars[kQDFull + st]);
+          if (kBucket)
+            bulk_load(smem + kOffTQ + st * kRowBytes, P.trel + rc.spad + q0, kRowBytes,
+                      &bars[kQDFull + st]);
         }
         qd_n = g + 1;
       }
@@ -540,6 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
     const float scale_log2 = a.scale * kLog2e;
     const float* sL2 = reinterpret_cast<const float*>(smem + kOffL2);
     const float* sD = reinterpret_cast<const float*>(smem + kOffD);
+    const int* sTQ = reinterpret_cast<const int*>(smem + kOffTQ);
     uint8_t* sDS = smem + kOffDS;
     int g = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
@@ -550,6 +577,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
       const bool key = j < rc.n;
       const float cbj = key ? P.cbias[(long long)rc.h * P.Tp + rc.spad + j] : 0.f;
       const uint64_t sl2 = f2_pack(scale_log2, scale_log2), cb2 = f2_pack(cbj, cbj);
+      // bucketed time bias: this key's time, biased (see kTimeMagic), and -m_t log2 e
+      const int tj_m = kBucket && key ? kTimeMagic - P.trel[rc.spad + j] : 0;
+      const float nmt2 = kBucket ? -a.slope_time[rc.h] * kLog2e : 0.f;
       bool ok = true;
       for (int t = 0; t < rc.nq && ok; ++t, ++g) {
         const int st = g & 1;
@@ -569,6 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
           const int qc = kQH * x + 32 * hq;  // this thread's first query column in the tile
           const float* l2 = sL2 + st * BM + qc;
           const float* dd = sD + st * BM + qc;
+          const int* tq = sTQ + st * BM + qc;
           const int qbase = q0 + qc;
           const uint32_t s_addr = lane_base + kColS + kQH * x;
           const uint32_t dp_addr = lane_base + kColDP + kQH * x;
@@ -597,12 +628,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
             for (int c = 0; c < 16; c += 4) {
               const float4 l4 = *reinterpret_cast<const float4*>(l2 + c0 + c);
               const float4 d4 = *reinterpret_cast<const float4*>(dd + c0 + c);
+              uint64_t t01 = f2_sub(cb2, f2_pack(l4.x, l4.y));
+              uint64_t t23 = f2_sub(cb2, f2_pack(l4.z, l4.w));
+              if (kBucket) {  // - m_t bucket(t_i - t_j), four queries at a time
+                const int4 ti = *reinterpret_cast<const int4*>(tq + c0 + c);
+                const uint64_t two23 = f2_pack(kTwo23, kTwo23);
+                const uint64_t g01 = f2_sub(f2_pack(__int_as_float(min(ti.x + tj_m, kTimeCap)),
+                                                    __int_as_float(min(ti.y + tj_m, kTimeCap))),
+                                            two23);
+                const uint64_t g23 = f2_sub(f2_pack(__int_as_float(min(ti.z + tj_m, kTimeCap)),
+                                                    __int_as_float(min(ti.w + tj_m, kTimeCap))),
+                                            two23);
+                const uint64_t s01 = f2_mul(g01, g01), s23 = f2_mul(g23, g23);
+                float q4[4];
+                f2_unpack(f2_mul(s01, s01), q4[0], q4[1]);
+                f2_unpack(f2_mul(s23, s23), q4[2], q4[3]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  q4[e] = __int_as_float((__float_as_int(q4[e]) >> 23) | 0x4B000000);
+                const uint64_t base = f2_pack(kTwo23 + 127.f, kTwo23 + 127.f);
+                const uint64_t nm2 = f2_pack(nmt2, nmt2);
+                t01 = f2_fma(f2_sub(f2_pack(q4[0], q4[1]), base), nm2, t01);
+                t23 = f2_fma(f2_sub(f2_pack(q4[2], q4[3]), base), nm2, t23);
+              }
               const uint64_t x01 =
-                  f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2,
-                         f2_sub(cb2, f2_pack(l4.x, l4.y)));
+                  f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2, t01);
               const uint64_t x23 =
                   f2_fma(f2_pack(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), sl2,
-                         f2_sub(cb2, f2_pack(l4.z, l4.w)));
+                         t23);
               float xv[4], p[4];
               f2_unpack(x01, xv[0], xv[1]);
               f2_unpack(x23, xv[2], xv[3]);
@@ -907,7 +960,7 @@ static size_t rows_bytes(long long T, int B, int H) {
 size_t attn_bwd_tc_workspace(int B, long long T, int H, int max_seqlen) {
   using namespace tcb;
   return kHeaderBytes + recs_bytes(B, max_seqlen) + users_bytes(B) + tokens_bytes(T) +
-         3 * rows_bytes(T, B, H) + (size_t)T * H * DH * sizeof(float);
+         rows_bytes(T, B, 1) + 3 * rows_bytes(T, B, H) + (size_t)T * H * DH * sizeof(float);
 }
 
 int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
@@ -927,7 +980,10 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   const size_t rb = rows_bytes(a.T, a.B, a.H);
   int32_t* uorder = (int32_t*)(ws + kHeaderBytes + recs_bytes(a.B, a.max_seqlen));
   int2* tinfo = (int2*)((uint8_t*)uorder + users_bytes(a.B));
-  uint8_t* rows = (uint8_t*)tinfo + tokens_bytes(a.T);
+  int32_t* trel = (int32_t*)((uint8_t*)tinfo + tokens_bytes(a.T));
+  uint8_t* rows = (uint8_t*)trel + rows_bytes(a.T, a.B, 1);
+  const bool bucket = a.time_bias == kTimeBiasBucketed;
+  p.trel = trel;
   p.cbias = (float*)rows;
   p.lse2 = (float*)(rows + rb);
   p.dsum = (float*)(rows + 2 * rb);
@@ -948,15 +1004,19 @@ int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st) {
   const long long pair_blocks = (a.T * a.H + 31) / 32;  // 8 lanes per (token, head)
   if (pair_blocks > 0) {
     k_bwd_rows<<<(unsigned)pair_blocks, 256, 0, st>>>(a, tinfo, (float*)p.cbias,
-                                                      (float*)p.lse2, (float*)p.dsum, p.Tp);
+                                                      (float*)p.lse2, (float*)p.dsum, trel, p.Tp);
     if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   }
-  static DeviceOnce smem_attr;
-  if (!set_smem_limit_once(smem_attr, (const void*)k_attn_bwd_tc, (int)kSmemBytes))
+  static DeviceOnce smem_attr[2];
+  const void* fn = bucket ? (const void*)k_attn_bwd_tc<true> : (const void*)k_attn_bwd_tc<false>;
+  if (!set_smem_limit_once(smem_attr[bucket ? 1 : 0], fn, (int)kSmemBytes))
     return GENRANK_ERR_CUDA;
   const int sms = sm_count_current();
   if (sms <= 0) return GENRANK_ERR_CUDA;
-  k_attn_bwd_tc<<<sms, kThreads, kSmemBytes, st>>>(p);
+  if (bucket)
+    k_attn_bwd_tc<true><<<sms, kThreads, kSmemBytes, st>>>(p);
+  else
+    k_attn_bwd_tc<false><<<sms, kThreads, kSmemBytes, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   if (a.B > 0) {
     k_bwd_cand<<<dim3((unsigned)a.B, 4), 256, 0, st>>>(a, p.dqacc, p.dsum, p.Tp);

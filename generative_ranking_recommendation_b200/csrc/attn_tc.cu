@@ -35,6 +35,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <climits>
+
 #include "common.cuh"
 #include "host_util.h"
 #include "kernels.h"
@@ -59,14 +61,32 @@ constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;           // kStages x 16 KB
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;     // kStages x 16 KB
 constexpr uint32_t kOffCB = kOffV + kStages * kTileBytes;    // kStages x 512 B
 constexpr uint32_t kOffQCB = kOffCB + kStages * kCBBytes;    // 2 x 512 B: the rows' own terms
-constexpr uint32_t kOffStage = kOffQCB + 2 * kCBBytes;       // O rows staged, 16 KB
+constexpr uint32_t kOffTR = kOffQCB + 2 * kCBBytes;         // bucketed bias: key times, kStages x 512 B
+constexpr uint32_t kOffQTR = kOffTR + kStages * kCBBytes;    // bucketed bias: row times, 2 x 512 B
+constexpr uint32_t kOffStage = kOffQTR + 2 * kCBBytes;       // O rows staged, 16 KB
 constexpr uint32_t kOffML = kOffStage + BM * DH * 2;         // (m, l) per row, 2 buffers
 constexpr uint32_t kOffRec = kOffML + 2 * BM * 8;            // item record with each Q tile
-constexpr uint32_t kOffBar = kOffRec + 2 * 16;               // barriers
+constexpr uint32_t kOffBar = kOffRec + 2 * 32;               // barriers
 constexpr uint32_t kNumBars = 17 + 3 * kStages;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;        // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;        // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kOffStage % 16 == 0 && kOffTR % 16 == 0, "16-byte aligned bulk copies");
+
+// Bucketed time bias (the variant -m_p (p_i - p_j) - m_t bucket(t_i - t_j)):
+//   bucket(D) = min(62, floor(4 log2(D + 1))) for a gap of D >= 0 seconds.
+// floor(4 log2 x) is the binary exponent of x^4; for integer 1 <= x <= 46341 the fp32
+// product fl(fl(x x) fl(x x)) has that exponent exactly (round to nearest even; checked
+// exhaustively over the whole range), and floor(4 log2 46341) = 62, so capping the gap at
+// 46340 saturates the bucket at 62.  The gap arrives as an int32 biased by kTimeMagic, so
+// that its bits read as the float 2^23 + D + 1 (exact for D < 2^23): one subtraction
+// gives x = D + 1 without a conversion instruction, and the exponent field E of x^4 ORed
+// into the same pattern reads as 2^23 + E, from which the bucket E - 127 is one more
+// subtraction.
+constexpr int kTimeMagic = 0x4B000001;           // float bits of 2^23 + 1
+constexpr int kTimeCap = kTimeMagic + 46340;      // gap cap (bucket 62)
+constexpr float kTwo23 = 8388608.f;
+constexpr int kMaxRelTime = 1 << 29;              // per-user times are clamped below this
 
 // TMEM columns (the whole 512 of the SM)
 constexpr uint32_t kTmemCols = 512;
@@ -79,15 +99,25 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, DH, 0, 1);  // P K-major (TMEM)
 
 // scratch layout
 constexpr size_t kHeaderBytes = 256;
-constexpr int kRecInts = 8;  // s, L, n, q0, nk, spad, u, unused
+constexpr int kRecInts = 8;  // s, L, n, q0, nk, spad, u, kb
 
 struct Params {
-  CUtensorMap tq, tk, tv;
+  const int32_t* trel;  // bucketed bias: per-token time since the user's first token, [Tp]
+  const __nv_bfloat16* dbias;  // dense bias: [B][Lpad][Lpad], user-local rows and columns
+  long long Lpad;
+  // tq: query rows; tk, tv: the history keys and values; tkc, tvc: the keys and values
+  // of the query rows themselves (the diagonal tile).  For attention over one jagged
+  // token array all of them cover that array and tkc, tvc equal tk, tv.
+  CUtensorMap tq, tk, tv, tkc, tvc;
   AttnArgs a;
   const int4* recs;      // [count][2] work records
   const int32_t* count;  // number of records
   const float* cbias;    // [H][Tp] column terms (log2 units)
   long long Tp;
+};
+
+struct CachedArgsHolder {
+  CachedAttnArgs c;
 };
 
 enum Bar {
@@ -100,8 +130,11 @@ GR_DEVICE int tiles_of(int q0, int n, int L, int nk) {
   return nk + (min(q0 + BM, L) > n ? 1 : 0);
 }
 
+// One work item: query rows [q0, q0 + 128) of a user whose sequence has L rows, the
+// first n of them history.  Query row i (and the diagonal tile's key i) lives at row
+// s + i of the query-side arrays; history key j at row kb + j of the key-side arrays.
 struct Item {
-  int s, L, n, q0, nk, spad, h;
+  int s, L, n, q0, nk, spad, h, kb, u;
   int nt;  // tiles visited: nk key tiles, plus the diagonal tile when candidates are present
 };
 
@@ -117,6 +150,8 @@ GR_DEVICE Item load_item(const Params& P, int w) {
   it.q0 = r0.w;
   it.nk = r1.x;
   it.spad = r1.y;
+  it.kb = r1.w;
+  it.u = r1.z;
   it.nt = tiles_of(it.q0, it.n, it.L, it.nk);
   return it;
 }
@@ -168,22 +203,32 @@ GR_DEVICE int block_exclusive_scan(int v, int* excl, int* warp_sums) {
 // consecutive records (times H heads) at the same time, so the items of one user and
 // head run side by side and share their K/V tiles in L2, while the short users fill
 // the tail.
+// With trel != null (the bucketed time bias) the column term holds the position part
+// only, and trel[i] = t_i - t_0 (clamped to [0, kMaxRelTime)) carries the time.  With
+// cbias == null (a dense bias) only the records are written.
 __global__ void __launch_bounds__(kSchedThreads) k_prologue(const __grid_constant__ AttnArgs a,
                                                             int max_tiles, int4* recs,
                                                             int32_t* count, int32_t* uorder,
-                                                            float* cbias, long long Tp) {
+                                                            float* cbias, int32_t* trel,
+                                                            long long Tp) {
   const int b = blockIdx.x;
   if (b < a.B) {
     const long long s = a.off[b], e = a.off[b + 1];
-    if (s < 0 || e < s || e > a.T) return;  // flagged by the schedule block
+    if (s < 0 || e < s || e > a.T || !cbias) return;  // layout flagged by the schedule block
     const int L = (int)(e - s);
     const long long base = seg_start(s, b);
     const long long t0 = L > 0 ? a.ts[s] : 0;
     for (int i = threadIdx.x; i < L; i += blockDim.x) {
       const float p = (float)a.pos[s + i];
-      const float dt = (float)(a.ts[s + i] - t0);
-      for (int h = 0; h < a.H; ++h)
-        cbias[(long long)h * Tp + base + i] = kLog2e * (a.slope_pos[h] * p + a.slope_time[h] * dt);
+      const long long dtl = a.ts[s + i] - t0;
+      if (trel) {
+        trel[base + i] = (int)min(max(dtl, 0LL), (long long)kMaxRelTime - 1);
+        for (int h = 0; h < a.H; ++h) cbias[(long long)h * Tp + base + i] = kLog2e * (a.slope_pos[h] * p);
+      } else {
+        const float dt = (float)dtl;
+        for (int h = 0; h < a.H; ++h)
+          cbias[(long long)h * Tp + base + i] = kLog2e * (a.slope_pos[h] * p + a.slope_time[h] * dt);
+      }
     }
     return;
   }
@@ -235,7 +280,111 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue(const __grid_constan
       const int kmax = min(t * BM + BM, n);
       const int nk = kmax > 0 ? (kmax + BN - 1) / BN : 0;
       recs[2 * slot] = make_int4(s, L, n, t * BM);
-      recs[2 * slot + 1] = make_int4(nk, (int)seg_start(s, u), u, 0);
+      recs[2 * slot + 1] = make_int4(nk, (int)seg_start(s, u), u, s);
+    }
+  }
+  if (threadIdx.x == 0) *count = total;
+}
+
+// ------------------------------------------------------------------------------------------
+// prologue of candidate scoring from a history key/value cache
+// ------------------------------------------------------------------------------------------
+// User u has n = hist_off[u+1] - hist_off[u] cached history rows and m candidate rows
+// [off[u], off[u+1]).  Its local sequence is the history followed by the candidates, so
+// the column terms and the work items are those of the full attention: candidate query
+// tiles start at q0 = n + 128 t, query row i (>= n) is candidate row off[u] + i - n, and
+// history key j is cache row hist_off[u] + j.  Blocks 0..B-1 write the column terms
+// (history: the cached positions and times; candidates: position n + 1 and their request
+// time) and check the orders the separable bias relies on; block B writes the records.
+GR_DEVICE bool cached_user(const CachedAttnArgs& c, int u, int& cs, int& n, int& m, int& hs) {
+  const long long cs_ = c.a.off[u], ce = c.a.off[u + 1];
+  const long long hs_ = c.hist_off[u], he = c.hist_off[u + 1];
+  if (cs_ < 0 || ce < cs_ || ce > c.a.T || hs_ < 0 || he < hs_ || he > c.Th) return false;
+  cs = (int)cs_;
+  hs = (int)hs_;
+  n = (int)(he - hs_);
+  m = (int)(ce - cs_);
+  return true;
+}
+
+__global__ void __launch_bounds__(kSchedThreads) k_prologue_cached(
+    const __grid_constant__ CachedArgsHolder ch, int max_tiles, int4* recs, int32_t* count,
+    int32_t* uorder, float* cbias, long long Tp) {
+  const CachedAttnArgs& c = ch.c;
+  const AttnArgs& a = c.a;
+  const int b = blockIdx.x;
+  if (b < a.B) {
+    int cs, n, m, hs;
+    if (!cached_user(c, b, cs, n, m, hs)) return;  // flagged by the schedule block
+    const int L = n + m;
+    const long long base = seg_start((long long)hs + cs, b);
+    const long long t0 = n > 0 ? c.ts_hist[hs] : (m > 0 ? a.ts[cs] : 0);
+    const long long t_last = n > 0 ? c.ts_hist[hs + n - 1] : LLONG_MIN;
+    for (int i = threadIdx.x; i < L; i += blockDim.x) {
+      int p;
+      long long t;
+      if (i < n) {
+        p = c.pos_hist[hs + i];
+        t = c.ts_hist[hs + i];
+        if (p < 0 || p > n + 1) flag(a.err, GENRANK_DERR_POS_RANGE);
+        if (i > 0 && t < c.ts_hist[hs + i - 1]) flag(a.err, GENRANK_DERR_TS_ORDER);
+      } else {
+        p = n + 1;
+        t = a.ts[cs + i - n];
+        if (t < t_last) flag(a.err, GENRANK_DERR_TS_ORDER);
+      }
+      const float pf = (float)p, dt = (float)(t - t0);
+      for (int h = 0; h < a.H; ++h)
+        cbias[(long long)h * Tp + base + i] = kLog2e * (a.slope_pos[h] * pf + a.slope_time[h] * dt);
+    }
+    return;
+  }
+  __shared__ int hist[kMaxTileBuckets];
+  __shared__ int warp_sums[kSchedThreads / 32];
+  for (int i = threadIdx.x; i < kMaxTileBuckets; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  auto tiles_of_user = [&](int u, bool check) -> int {
+    int cs, n, m, hs;
+    if (!cached_user(c, u, cs, n, m, hs)) {
+      if (check) flag(a.err, GENRANK_DERR_LAYOUT);
+      return 0;
+    }
+    const int tiles_all = (m + BM - 1) / BM;
+    if (check && tiles_all > max_tiles) flag(a.err, GENRANK_DERR_LAYOUT);
+    return min(tiles_all, max_tiles);
+  };
+  for (int u = threadIdx.x; u < a.B; u += blockDim.x)
+    atomicAdd(&hist[min(tiles_of_user(u, true), kMaxTileBuckets - 1)], 1);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int q = kMaxTileBuckets - 1; q >= 0; --q) {
+      const int cnt = hist[q];
+      hist[q] = acc;
+      acc += cnt;
+    }
+  }
+  __syncthreads();
+  for (int u = threadIdx.x; u < a.B; u += blockDim.x)
+    uorder[atomicAdd(&hist[min(tiles_of_user(u, false), kMaxTileBuckets - 1)], 1)] = u;
+  __syncthreads();
+  const int chunk = (a.B + kSchedThreads - 1) / kSchedThreads;
+  const int k0 = min(a.B, (int)threadIdx.x * chunk), k1 = min(a.B, k0 + chunk);
+  int mine = 0;
+  for (int k = k0; k < k1; ++k) mine += tiles_of_user(uorder[k], false);
+  int slot = 0;
+  const int total = block_exclusive_scan(mine, &slot, warp_sums);
+  for (int k = k0; k < k1; ++k) {
+    const int u = uorder[k];
+    const int tiles = tiles_of_user(u, false);
+    if (tiles == 0) continue;
+    int cs, n, m, hs;
+    cached_user(c, u, cs, n, m, hs);
+    const int nk = (n + BN - 1) / BN;
+    const int seg = (int)seg_start((long long)hs + cs, u);
+    for (int t = tiles - 1; t >= 0; --t, ++slot) {
+      recs[2 * slot] = make_int4(cs - n, n + m, n, n + t * BM);
+      recs[2 * slot + 1] = make_int4(nk, seg, u, hs);
     }
   }
   if (threadIdx.x == 0) *count = total;
@@ -263,15 +412,67 @@ GR_DEVICE void p_store(uint32_t taddr, const uint32_t (&pk)[CW / 2]) {
   tmem_st_half8_nowait<kHalf / 2>(taddr, pk);
 }
 
-// x = s * scale + c_j for CW columns (key kc0 + c of the tile); keys at or beyond
-// nvalid are masked.  Four independent running maxima shorten the chain.
-template <bool kMasked>
-GR_DEVICE void row_max_chunk(const uint32_t (&s)[CW], const float* cb, int kc0, int nvalid,
-                             float scale_log2, float (&mx4)[4]) {
+// The bucketed time bias of one softmax thread: the key times of its columns (shared
+// memory, indexed like the column terms), its row's time + kTimeMagic, and -m_t log2 e
+// of the item's head.  Unused (and compiled out) for the linear time bias.
+struct TB {
+  const int* tr;
+  int ti_m;
+  float nmt2;
+  GR_DEVICE TB at(int off) const { return TB{tr + off, ti_m, nmt2}; }
+};
+
+// bucket(t_i - t_j) of four consecutive keys, as two pairs of floats (see kTimeMagic).
+GR_DEVICE void buckets4(const TB& tb, int c, uint64_t& b01, uint64_t& b23) {
+  const int4 t = *reinterpret_cast<const int4*>(tb.tr + c);
+  const uint64_t two23 = f2_pack(kTwo23, kTwo23);
+  const uint64_t x01 = f2_sub(f2_pack(__int_as_float(min(tb.ti_m - t.x, kTimeCap)),
+                                      __int_as_float(min(tb.ti_m - t.y, kTimeCap))), two23);
+  const uint64_t x23 = f2_sub(f2_pack(__int_as_float(min(tb.ti_m - t.z, kTimeCap)),
+                                      __int_as_float(min(tb.ti_m - t.w, kTimeCap))), two23);
+  const uint64_t sq01 = f2_mul(x01, x01), sq23 = f2_mul(x23, x23);
+  float q[4];
+  f2_unpack(f2_mul(sq01, sq01), q[0], q[1]);
+  f2_unpack(f2_mul(sq23, sq23), q[2], q[3]);
+  float e[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) e[k] = __int_as_float((__float_as_int(q[k]) >> 23) | 0x4B000000);
+  const uint64_t base = f2_pack(kTwo23 + 127.f, kTwo23 + 127.f);
+  b01 = f2_sub(f2_pack(e[0], e[1]), base);
+  b23 = f2_sub(f2_pack(e[2], e[3]), base);
+}
+
+// x = s * scale + c_j (- m_t bucket for the bucketed bias) for CW columns (key kc0 + c of
+// the tile); keys at or beyond nvalid are masked.  Four independent running maxima
+// shorten the chain.
+template <bool kMasked, bool kBucket, bool kDense>
+GR_DEVICE void row_max_chunk(const uint32_t (&s)[CW], const float* cb, const TB& tb,
+                             const uint32_t* bw, int kc0, int nvalid, float scale_log2,
+                             float (&mx4)[4]) {
 #pragma unroll
   for (int c = 0; c < CW; c += 4) {
-    const float4 b4 = *reinterpret_cast<const float4*>(cb + c);
-    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+    float bb[4];
+    if (kDense) {  // the dense bias of these keys, bf16 pairs
+      bb[0] = kLog2e * bf16_lo(bw[c / 2]);
+      bb[1] = kLog2e * bf16_hi(bw[c / 2]);
+      bb[2] = kLog2e * bf16_lo(bw[c / 2 + 1]);
+      bb[3] = kLog2e * bf16_hi(bw[c / 2 + 1]);
+    } else {
+      const float4 b4 = *reinterpret_cast<const float4*>(cb + c);
+      bb[0] = b4.x;
+      bb[1] = b4.y;
+      bb[2] = b4.z;
+      bb[3] = b4.w;
+    }
+    if (kBucket) {
+      uint64_t b01, b23;
+      buckets4(tb, c, b01, b23);
+      float k[4];
+      f2_unpack(b01, k[0], k[1]);
+      f2_unpack(b23, k[2], k[3]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) bb[e] = fmaf(k[e], tb.nmt2, bb[e]);
+    }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float v = fmaf(__uint_as_float(s[c + e]), scale_log2, bb[e]);
@@ -283,17 +484,32 @@ GR_DEVICE void row_max_chunk(const uint32_t (&s)[CW], const float* cb, int kc0, 
 // p = 2^(x - m) for CW columns, summed into two pairs of partial sums, packed to
 // bf16 pairs and stored (without waiting) to CW / 2 TMEM columns at taddr.  The
 // bias and scale arithmetic runs on column pairs (two-wide fp32 instructions).
-template <bool kMasked>
-GR_DEVICE void exp_pack_store(const uint32_t (&s)[CW], const float* cb, int kc0, int nvalid,
-                              float scale_log2, float m_use, uint64_t (&rs2)[2], uint32_t taddr) {
+template <bool kMasked, bool kBucket, bool kDense>
+GR_DEVICE void exp_pack_store(const uint32_t (&s)[CW], const float* cb, const TB& tb,
+                              const uint32_t* bw, int kc0, int nvalid, float scale_log2,
+                              float m_use, uint64_t (&rs2)[2], uint32_t taddr) {
   const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
   const uint64_t m2 = f2_pack(m_use, m_use);
   uint32_t pk[CW / 2];
 #pragma unroll
   for (int c = 0; c < CW; c += 4) {
-    const float4 b4 = *reinterpret_cast<const float4*>(cb + c);
-    const uint64_t t01 = f2_sub(f2_pack(b4.x, b4.y), m2);
-    const uint64_t t23 = f2_sub(f2_pack(b4.z, b4.w), m2);
+    uint64_t t01, t23;
+    if (kDense) {  // bias log2 e - m, from the bf16 pairs of the dense bias
+      const uint64_t l2e = f2_pack(kLog2e, kLog2e), nm2 = f2_pack(-m_use, -m_use);
+      t01 = f2_fma(f2_pack(bf16_lo(bw[c / 2]), bf16_hi(bw[c / 2])), l2e, nm2);
+      t23 = f2_fma(f2_pack(bf16_lo(bw[c / 2 + 1]), bf16_hi(bw[c / 2 + 1])), l2e, nm2);
+    } else {
+      const float4 b4 = *reinterpret_cast<const float4*>(cb + c);
+      t01 = f2_sub(f2_pack(b4.x, b4.y), m2);
+      t23 = f2_sub(f2_pack(b4.z, b4.w), m2);
+    }
+    if (kBucket) {
+      uint64_t b01, b23;
+      buckets4(tb, c, b01, b23);
+      const uint64_t nm2 = f2_pack(tb.nmt2, tb.nmt2);
+      t01 = f2_fma(b01, nm2, t01);
+      t23 = f2_fma(b23, nm2, t23);
+    }
     const uint64_t v01 =
         f2_fma(f2_pack(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sl2, t01);
     const uint64_t v23 =
@@ -311,12 +527,11 @@ GR_DEVICE void exp_pack_store(const uint32_t (&s)[CW], const float* cb, int kc0,
   p_store(taddr, pk);
 }
 
-// Maximum of x = s * scale + c_j over this thread's half of the tile (S at s_addr,
-// column terms of the half at cb, first key kbase), CW columns at a time with the
-// next chunk's load in flight.
-template <bool kMasked>
-GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, int kbase, int nvalid,
-                         float scale_log2) {
+// Maximum of x over this thread's half of the tile (S at s_addr, column terms of the
+// half at cb, first key kbase), CW columns at a time with the next chunk's load in flight.
+template <bool kMasked, bool kBucket, bool kDense>
+GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, const TB& tb, const uint32_t* bw,
+                         int kbase, int nvalid, float scale_log2) {
   float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   uint32_t xa[CW], xb[CW];
   s_load(s_addr, xa);
@@ -324,10 +539,12 @@ GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, int kbase, int nvalid
 #pragma unroll
   for (int c0 = 0; c0 < kHalf; c0 += 2 * CW) {
     s_load(s_addr + c0 + CW, xb);
-    row_max_chunk<kMasked>(xa, cb + c0, kbase + c0, nvalid, scale_log2, mx4);
+    row_max_chunk<kMasked, kBucket, kDense>(xa, cb + c0, tb.at(c0), bw + c0 / 2, kbase + c0,
+                                            nvalid, scale_log2, mx4);
     tmem_ld_wait(xb);
     if (c0 + 2 * CW < kHalf) s_load(s_addr + c0 + 2 * CW, xa);
-    row_max_chunk<kMasked>(xb, cb + c0 + CW, kbase + c0 + CW, nvalid, scale_log2, mx4);
+    row_max_chunk<kMasked, kBucket, kDense>(xb, cb + c0 + CW, tb.at(c0 + CW), bw + (c0 + CW) / 2,
+                                            kbase + c0 + CW, nvalid, scale_log2, mx4);
     if (c0 + 2 * CW < kHalf) tmem_ld_wait(xa);
   }
   return fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
@@ -335,9 +552,9 @@ GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, int kbase, int nvalid
 
 // P = 2^(x - m) for this thread's half of the tile, written as bf16 pairs to the P
 // columns at p_addr; the stores have landed when it returns.  Returns the half's sum.
-template <bool kMasked>
-GR_DEVICE float tile_exp(uint32_t s_addr, uint32_t p_addr, const float* cb, int kbase,
-                         int nvalid, float scale_log2, float m) {
+template <bool kMasked, bool kBucket, bool kDense>
+GR_DEVICE float tile_exp(uint32_t s_addr, uint32_t p_addr, const float* cb, const TB& tb,
+                         const uint32_t* bw, int kbase, int nvalid, float scale_log2, float m) {
   uint64_t rs2[2] = {0ull, 0ull};  // (+0, +0) pairs
   uint32_t xa[CW], xb[CW];
   s_load(s_addr, xa);
@@ -345,11 +562,13 @@ GR_DEVICE float tile_exp(uint32_t s_addr, uint32_t p_addr, const float* cb, int 
 #pragma unroll
   for (int c0 = 0; c0 < kHalf; c0 += 2 * CW) {
     s_load(s_addr + c0 + CW, xb);
-    exp_pack_store<kMasked>(xa, cb + c0, kbase + c0, nvalid, scale_log2, m, rs2, p_addr + c0 / 2);
+    exp_pack_store<kMasked, kBucket, kDense>(xa, cb + c0, tb.at(c0), bw + c0 / 2, kbase + c0,
+                                             nvalid, scale_log2, m, rs2, p_addr + c0 / 2);
     tmem_ld_wait(xb);
     if (c0 + 2 * CW < kHalf) s_load(s_addr + c0 + 2 * CW, xa);
-    exp_pack_store<kMasked>(xb, cb + c0 + CW, kbase + c0 + CW, nvalid, scale_log2, m, rs2,
-                            p_addr + (c0 + CW) / 2);
+    exp_pack_store<kMasked, kBucket, kDense>(xb, cb + c0 + CW, tb.at(c0 + CW), bw + (c0 + CW) / 2,
+                                             kbase + c0 + CW, nvalid, scale_log2, m, rs2,
+                                             p_addr + (c0 + CW) / 2);
     if (c0 + 2 * CW < kHalf) tmem_ld_wait(xa);
   }
   tmem_wait_st();
@@ -381,24 +600,27 @@ GR_DEVICE bool rescale_o(uint32_t o_addr, float alpha, uint64_t* prev_pv, uint32
 // (every key far below the offset) or exceeds 2^100 later is redone with the exact
 // offset max(m, tile max), rescaling O in TMEM.  Rows past the user's end never
 // redo (their output is not written).
-template <bool kMasked>
+template <bool kMasked, bool kBucket, bool kDense>
 GR_DEVICE bool softmax_tile(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, const float* cb,
-                            int kbase, int nvalid, float scale_log2, bool first, bool row_ok,
-                            float& m, float& l, uint64_t* prev_pv, uint32_t prev_ph,
-                            volatile int* abort_flag, int32_t* err) {
-  float rs = tile_exp<kMasked>(s_addr, p_addr, cb, kbase, nvalid, scale_log2, m);
+                            const TB& tb, const uint32_t* bw, int kbase, int nvalid,
+                            float scale_log2, bool first, bool row_ok, float& m, float& l,
+                            uint64_t* prev_pv, uint32_t prev_ph, volatile int* abort_flag,
+                            int32_t* err) {
+  float rs = tile_exp<kMasked, kBucket, kDense>(s_addr, p_addr, cb, tb, bw, kbase, nvalid,
+                                                scale_log2, m);
   const float rs_row = rs + __shfl_xor_sync(0xffffffffu, rs, 16);
   const bool redo = row_ok && (!(rs_row <= kOverflowSum) || (first && rs_row < kUnderflowSum));
   if (__any_sync(0xffffffffu, redo)) {
     // every lane takes part in the .sync.aligned TMEM accesses; only redo rows move m
-    float mx = tile_max<kMasked>(s_addr, cb, kbase, nvalid, scale_log2);
+    float mx = tile_max<kMasked, kBucket, kDense>(s_addr, cb, tb, bw, kbase, nvalid, scale_log2);
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
     const float m_new = redo ? (first ? mx : fmaxf(m, mx)) : m;
     const float alpha = first ? 1.f : ex2(m - m_new);
     m = m_new;
     if (!first && !rescale_o(o_addr, alpha, prev_pv, prev_ph, abort_flag, err)) return false;
     l *= alpha;
-    rs = tile_exp<kMasked>(s_addr, p_addr, cb, kbase, nvalid, scale_log2, m);
+    rs = tile_exp<kMasked, kBucket, kDense>(s_addr, p_addr, cb, tb, bw, kbase, nvalid,
+                                            scale_log2, m);
   }
   l = first ? rs : l + rs;
   return true;
@@ -411,7 +633,7 @@ GR_DEVICE bool softmax_tile(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, c
 GR_DEVICE bool softmax_diag(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, int rt, int h,
                             bool cand_row, float rowcb, float scale_log2, bool first, float& m,
                             float& l, uint64_t* prev_pv, uint32_t prev_ph,
-                            volatile int* abort_flag, int32_t* err) {
+                            volatile int* abort_flag, int32_t* err, float diagb = 0.f) {
   uint32_t xa[32], xb[32];
   tmem_ld_half32_async<kHalf>(s_addr, xa);
   tmem_ld_half32_async<kHalf>(s_addr + 32, xb);
@@ -425,7 +647,7 @@ GR_DEVICE bool softmax_diag(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, i
     sv = col == c ? __uint_as_float(xa[c]) : sv;
     sv = col == c + 32 ? __uint_as_float(xb[c]) : sv;
   }
-  const float xm = mine ? fmaf(sv, scale_log2, rowcb) : -INFINITY;
+  const float xm = mine ? fmaf(sv, scale_log2, rowcb + diagb) : -INFINITY;
   const float xr = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 16));  // the row's self score
   const bool move = xr > -INFINITY && (first || xr - m > 100.f);
   if (!first && __any_sync(0xffffffffu, move)) {
@@ -449,6 +671,7 @@ struct Cursor {  // one key tile in the CTA's sequence: tile j of the qi-th item
   int j, g, qi, nt;
 };
 
+template <bool kBucket, bool kDense>
 __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_constant__ Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -485,6 +708,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
     tma_prefetch_desc(&P.tq);
     tma_prefetch_desc(&P.tk);
     tma_prefetch_desc(&P.tv);
+    tma_prefetch_desc(&P.tkc);
+    tma_prefetch_desc(&P.tvc);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -517,12 +742,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
         break;
       }
       const float* cb_src = P.cbias + (long long)it.h * P.Tp + it.spad;
+      const int32_t* tr_src = kBucket ? P.trel + it.spad : nullptr;
       if (lane == 0) {
-        sRec[qb] = make_int4(it.q0, it.n, it.L, it.nk);
-        mbar_expect_tx(&bars[kQFull + qb], kTileBytes + kCBBytes);
+        sRec[2 * qb] = make_int4(it.q0, it.n, it.L, it.nk);
+        sRec[2 * qb + 1] = make_int4(it.h, it.u, 0, 0);
+        mbar_expect_tx(&bars[kQFull + qb],
+                       kTileBytes + (kDense ? 0 : (kBucket ? 2 : 1) * kCBBytes));
         tma_load_3d(smem + kOffQ + qb * kTileBytes, &P.tq, &bars[kQFull + qb], 0, it.h,
                     it.s + it.q0);
-        bulk_load(smem + kOffQCB + qb * kCBBytes, cb_src + it.q0, kCBBytes, &bars[kQFull + qb]);
+        if (!kDense)
+          bulk_load(smem + kOffQCB + qb * kCBBytes, cb_src + it.q0, kCBBytes, &bars[kQFull + qb]);
+        if (kBucket)
+          bulk_load(smem + kOffQTR + qb * kCBBytes, tr_src + it.q0, kCBBytes, &bars[kQFull + qb]);
       }
       ++qi;
       for (int j = 0; j < it.nt; ++j) {
@@ -533,21 +764,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
         }
         if (lane == 0) {
           // history key tiles most recent first, then the item's own rows
-          const int kv0 = j < it.nk ? (it.nk - 1 - j) * BN : it.q0;
-          mbar_expect_tx(&bars[kKFull + st], kTileBytes + kCBBytes);
-          tma_load_3d(smem + kOffK + st * kTileBytes, &P.tk, &bars[kKFull + st], 0, it.h,
-                      it.s + kv0);
-          bulk_load(smem + kOffCB + st * kCBBytes, cb_src + kv0, kCBBytes, &bars[kKFull + st]);
+          const bool hist = j < it.nk;
+          const int kv0 = hist ? (it.nk - 1 - j) * BN : it.q0;
+          const int row = hist ? it.kb + kv0 : it.s + kv0;
+          mbar_expect_tx(&bars[kKFull + st],
+                         kTileBytes + (kDense ? 0 : (kBucket ? 2 : 1) * kCBBytes));
+          tma_load_3d(smem + kOffK + st * kTileBytes, hist ? &P.tk : &P.tkc, &bars[kKFull + st],
+                      0, it.h, row);
+          if (!kDense)
+            bulk_load(smem + kOffCB + st * kCBBytes, cb_src + kv0, kCBBytes, &bars[kKFull + st]);
+          if (kBucket)
+            bulk_load(smem + kOffTR + st * kCBBytes, tr_src + kv0, kCBBytes, &bars[kKFull + st]);
           mbar_expect_tx(&bars[kVFull + st], kTileBytes);
-          tma_load_3d(smem + kOffV + st * kTileBytes, &P.tv, &bars[kVFull + st], 0, it.h,
-                      it.s + kv0);
+          tma_load_3d(smem + kOffV + st * kTileBytes, hist ? &P.tv : &P.tvc, &bars[kVFull + st],
+                      0, it.h, row);
         }
         ++g;
       }
     }
     if (ok && wait_warp(&bars[kQEmpty + (qi & 1)], par(qi >> 1) ^ 1u, abort_flag, a.err)) {
       if (lane == 0) {
-        sRec[qi & 1] = make_int4(0, 0, 0, -1);
+        sRec[2 * (qi & 1)] = make_int4(0, 0, 0, -1);
         mbar_arrive(&bars[kQFull + (qi & 1)]);
       }
       ++qi;
@@ -571,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       // number of tiles of the qi-th item (its Q tile has landed), or -1 at the end
       auto tiles = [&](int qi) -> int {
         if (!mbar_wait(&bars[kQFull + (qi & 1)], par(qi >> 1), abort_flag, a.err)) return -1;
-        const int4 r = sRec[qi & 1];
+        const int4 r = sRec[2 * (qi & 1)];
         return r.w < 0 ? -1 : tiles_of(r.x, r.y, r.z, r.w);
       };
       auto issue_s = [&](const Cursor& t) -> bool {
@@ -636,13 +873,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
     const int rt = quad * 32 + rh * 16 + (lane & 15);  // query row within the tile
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32 + rh * 16) << 16);
     const float* sQCB = reinterpret_cast<const float*>(smem + kOffQCB);
+    const int* sQTR = reinterpret_cast<const int*>(smem + kOffQTR);
+    const int* sTR = reinterpret_cast<const int*>(smem + kOffTR);
     const int4* sRec = reinterpret_cast<const int4*>(smem + kOffRec);
     int g = 0;
     for (int oi = 0;; ++oi) {
       const int ob = oi & 1;
       // the item's record and the row's own column term c_i arrive with the Q tile
       if (!wait_warp(&bars[kQFull + ob], par(oi >> 1), abort_flag, a.err)) break;
-      const int4 rec = sRec[ob];
+      const int4 rec = sRec[2 * ob];
       if (rec.w < 0) break;
       Item it;
       it.q0 = rec.x;
@@ -650,7 +889,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       it.L = rec.z;
       it.nk = rec.w;
       it.nt = tiles_of(it.q0, it.n, it.L, it.nk);
-      const float rowcb = sQCB[ob * BM + rt];
+      // the fixed offset starts at the row's own column term; a dense bias has no such
+      // bound, so its offset starts at 0 and the redo path moves it when needed
+      const float rowcb = kDense ? 0.f : sQCB[ob * BM + rt];
+      const __nv_bfloat16* brow = nullptr;  // dense bias: this thread's row of the user's block
+      if (kDense)
+        brow = P.dbias + ((long long)sRec[2 * ob + 1].y * P.Lpad + it.q0 + rt) * P.Lpad + kHalf * h;
+      TB tb{nullptr, 0, 0.f};
+      if (kBucket) {
+        const int hh = sRec[2 * ob + 1].x;
+        tb.ti_m = sQTR[ob * BM + rt] + kTimeMagic;
+        tb.nmt2 = -a.slope_time[hh] * kLog2e;
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kQEmpty + ob]);
       const int i = it.q0 + rt;
@@ -663,6 +913,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       bool ok = true;
       for (int j = 0; j < it.nt; ++j, ++g) {
         const int sb = g & 1, st = g % kStages;
+        // dense bias: this thread's 64 values of the tile (one 128-byte line), requested
+        // before the wait for S so that the load overlaps it
+        uint32_t bw[kDense ? kHalf / 2 : 1];
+        float diagb = 0.f;
+        if (kDense) {
+          if (j < it.nk) {
+            const uint4* src = reinterpret_cast<const uint4*>(brow + (it.nk - 1 - j) * BN);
+#pragma unroll
+            for (int c = 0; c < kHalf / 8; ++c) {
+              const uint4 w4 = __ldg(src + c);
+              bw[4 * c] = w4.x;
+              bw[4 * c + 1] = w4.y;
+              bw[4 * c + 2] = w4.z;
+              bw[4 * c + 3] = w4.w;
+            }
+          } else {  // the diagonal tile: the row's own entry
+            diagb = kLog2e * __bfloat162float(brow[it.q0 + rt - kHalf * h]);
+          }
+        }
         // S_g's commit also covers every MMA issued before it, P_{g-2} V_{g-2} included,
         // so once S_g is here its P buffer is free as well
         if (!wait_warp(&bars[kSFull + sb], par(g >> 1), abort_flag, a.err) ||
@@ -680,15 +949,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
           const bool masked = kv0 + BN - 1 > mask_from;
           const int nvalid = masked ? max(0, min(BN, lim - kv0 + 1)) : BN;
           const float* cb = sCB + st * BN + kHalf * h;
-          ok = masked ? softmax_tile<true>(s_addr, p_addr, o_addr, cb, kHalf * h, nvalid,
-                                           scale_log2, j == 0, row_ok, m, l, prev_pv, prev_ph,
-                                           abort_flag, a.err)
-                      : softmax_tile<false>(s_addr, p_addr, o_addr, cb, kHalf * h, nvalid,
-                                            scale_log2, j == 0, row_ok, m, l, prev_pv, prev_ph,
-                                            abort_flag, a.err);
+          if (kBucket) tb.tr = sTR + st * BN + kHalf * h;
+          ok = masked ? softmax_tile<true, kBucket, kDense>(
+                            s_addr, p_addr, o_addr, cb, tb, bw, kHalf * h, nvalid, scale_log2,
+                            j == 0, row_ok, m, l, prev_pv, prev_ph, abort_flag, a.err)
+                      : softmax_tile<false, kBucket, kDense>(
+                            s_addr, p_addr, o_addr, cb, tb, bw, kHalf * h, nvalid, scale_log2,
+                            j == 0, row_ok, m, l, prev_pv, prev_ph, abort_flag, a.err);
         } else {
           ok = softmax_diag(s_addr, p_addr, o_addr, rt, h, cand_row, rowcb, scale_log2, j == 0,
-                            m, l, prev_pv, prev_ph, abort_flag, a.err);
+                            m, l, prev_pv, prev_ph, abort_flag, a.err, diagb);
         }
         if (!ok) break;
         tc_fence_before();
@@ -799,6 +1069,27 @@ static bool make_map(CUtensorMap* m, const void* base, long long T, int H, long 
 
 static int max_tiles_of(int max_seqlen) { return (max_seqlen + BM - 1) / BM; }
 
+// the kernels' dynamic shared-memory limit, raised once per device and variant
+static DeviceOnce fwd_smem_attr[3];
+
+// mode: the time bias (kTimeBiasLinear, kTimeBiasBucketed) or kDenseBiasMode
+constexpr int kDenseBiasMode = 2;
+static int launch_kernel(const Params& p, int mode, cudaStream_t st) {
+  const void* fn = mode == kTimeBiasBucketed ? (const void*)k_attn_fwd_tc<true, false>
+                   : mode == kDenseBiasMode  ? (const void*)k_attn_fwd_tc<false, true>
+                                             : (const void*)k_attn_fwd_tc<false, false>;
+  if (!set_smem_limit_once(fwd_smem_attr[mode], fn, (int)kSmemBytes)) return GENRANK_ERR_CUDA;
+  const int sms = sm_count_current();
+  if (sms <= 0) return GENRANK_ERR_CUDA;
+  if (mode == kTimeBiasBucketed)
+    k_attn_fwd_tc<true, false><<<sms, kThreads, kSmemBytes, st>>>(p);
+  else if (mode == kDenseBiasMode)
+    k_attn_fwd_tc<false, true><<<sms, kThreads, kSmemBytes, st>>>(p);
+  else
+    k_attn_fwd_tc<false, false><<<sms, kThreads, kSmemBytes, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
+}
+
 static size_t recs_bytes(int B, int max_seqlen) {
   return ((size_t)B * max_tiles_of(max_seqlen) * kRecInts * 4 + 15) / 16 * 16;
 }
@@ -808,8 +1099,9 @@ static size_t users_bytes(int B) { return ((size_t)B * 4 + 15) / 16 * 16; }
 
 size_t attn_fwd_tc_workspace(int B, long long T, int H, int max_seqlen) {
   using namespace tc;
+  // records, user order, column terms [H][Tp] and (bucketed bias) token times [Tp]
   return kHeaderBytes + recs_bytes(B, max_seqlen) + users_bytes(B) +
-         (size_t)H * scratch_tp(T, B) * sizeof(float);
+         (size_t)(H + 1) * scratch_tp(T, B) * sizeof(float);
 }
 
 int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
@@ -822,6 +1114,8 @@ int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
       !make_map(&p.tk, a.k, a.T, a.H, a.tok_stride) ||
       !make_map(&p.tv, a.v, a.T, a.H, a.tok_stride))
     return GENRANK_ERR_CUDA;
+  p.tkc = p.tk;
+  p.tvc = p.tv;
   p.a = a;
   uint8_t* ws = (uint8_t*)a.ws;
   int32_t* count = (int32_t*)ws;
@@ -832,15 +1126,90 @@ int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
   p.recs = recs;
   p.cbias = cbias;
   p.Tp = scratch_tp(a.T, a.B);
-  k_prologue<<<a.B + 1, kSchedThreads, 0, st>>>(a, max_tiles, recs, count, uorder, cbias, p.Tp);
+  const bool bucket = a.time_bias == kTimeBiasBucketed;
+  int32_t* trel = bucket ? (int32_t*)(cbias + (size_t)a.H * p.Tp) : nullptr;
+  p.trel = trel;
+  k_prologue<<<a.B + 1, kSchedThreads, 0, st>>>(a, max_tiles, recs, count, uorder, cbias, trel,
+                                                p.Tp);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
-  static DeviceOnce smem_attr;
-  if (!set_smem_limit_once(smem_attr, (const void*)k_attn_fwd_tc, (int)kSmemBytes))
+  p.dbias = nullptr;
+  p.Lpad = 0;
+  return launch_kernel(p, a.time_bias == kTimeBiasBucketed ? kTimeBiasBucketed : kTimeBiasLinear,
+                       st);
+}
+
+int launch_attn_fwd_dense(const AttnArgs& a, const void* bias, long long Lpad, cudaStream_t st) {
+  using namespace tc;
+  if (a.dh != DH || a.dtype != GENRANK_BF16) return GENRANK_ERR_UNSUPPORTED;
+  if (a.T + (long long)BM >= INT32_MAX / 2) return GENRANK_ERR_UNSUPPORTED;
+  Params p;
+  if (!make_map(&p.tq, a.q, a.T, a.H, a.tok_stride) ||
+      !make_map(&p.tk, a.k, a.T, a.H, a.tok_stride) ||
+      !make_map(&p.tv, a.v, a.T, a.H, a.tok_stride))
     return GENRANK_ERR_CUDA;
-  const int sms = sm_count_current();
-  if (sms <= 0) return GENRANK_ERR_CUDA;
-  k_attn_fwd_tc<<<sms, kThreads, kSmemBytes, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
+  p.tkc = p.tk;
+  p.tvc = p.tv;
+  p.a = a;
+  uint8_t* ws = (uint8_t*)a.ws;
+  int32_t* count = (int32_t*)ws;
+  int4* recs = (int4*)(ws + kHeaderBytes);
+  int32_t* uorder = (int32_t*)(ws + kHeaderBytes + recs_bytes(a.B, a.max_seqlen));
+  float* cbias = (float*)((uint8_t*)uorder + users_bytes(a.B));
+  p.count = count;
+  p.recs = recs;
+  p.cbias = cbias;  // not read by the dense-bias kernel
+  p.Tp = scratch_tp(a.T, a.B);
+  p.trel = nullptr;
+  p.dbias = (const __nv_bfloat16*)bias;
+  p.Lpad = Lpad;
+  k_prologue<<<a.B + 1, kSchedThreads, 0, st>>>(a, max_tiles_of(a.max_seqlen), recs, count,
+                                                uorder, nullptr, nullptr, p.Tp);
+  if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
+  return launch_kernel(p, kDenseBiasMode, st);
+}
+
+size_t attn_fwd_cached_workspace(int B, long long C, long long Th, int H, int max_cand) {
+  using namespace tc;
+  return kHeaderBytes + recs_bytes(B, max_cand) + users_bytes(B) +
+         (size_t)H * scratch_tp(C + Th, B) * sizeof(float);
+}
+
+int launch_attn_fwd_cached(const CachedAttnArgs& c, cudaStream_t st) {
+  using namespace tc;
+  const AttnArgs& a = c.a;
+  if (a.dh != DH || a.dtype != GENRANK_BF16) return GENRANK_ERR_UNSUPPORTED;
+  if (a.T + c.Th + (long long)BM >= INT32_MAX / 2) return GENRANK_ERR_UNSUPPORTED;
+  Params p;
+  if (!make_map(&p.tq, a.q, a.T, a.H, a.tok_stride) ||
+      !make_map(&p.tkc, a.k, a.T, a.H, a.tok_stride) ||
+      !make_map(&p.tvc, a.v, a.T, a.H, a.tok_stride))
+    return GENRANK_ERR_CUDA;
+  if (c.Th > 0) {
+    if (!make_map(&p.tk, c.k_hist, c.Th, a.H, c.hist_stride) ||
+        !make_map(&p.tv, c.v_hist, c.Th, a.H, c.hist_stride))
+      return GENRANK_ERR_CUDA;
+  } else {  // no history anywhere: no history tile is ever loaded
+    p.tk = p.tkc;
+    p.tv = p.tvc;
+  }
+  p.a = a;
+  uint8_t* ws = (uint8_t*)a.ws;
+  int32_t* count = (int32_t*)ws;
+  int4* recs = (int4*)(ws + kHeaderBytes);
+  int32_t* uorder = (int32_t*)(ws + kHeaderBytes + recs_bytes(a.B, c.max_cand));
+  float* cbias = (float*)((uint8_t*)uorder + users_bytes(a.B));
+  p.count = count;
+  p.recs = recs;
+  p.cbias = cbias;
+  p.Tp = scratch_tp(a.T + c.Th, a.B);
+  CachedArgsHolder holder{c};
+  k_prologue_cached<<<a.B + 1, kSchedThreads, 0, st>>>(holder, max_tiles_of(c.max_cand), recs,
+                                                       count, uorder, cbias, p.Tp);
+  if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
+  p.trel = nullptr;
+  p.dbias = nullptr;
+  p.Lpad = 0;
+  return launch_kernel(p, kTimeBiasLinear, st);
 }
 
 }  // namespace gr

@@ -62,6 +62,11 @@ struct EmbedBwdArgs {
 
 constexpr int kMaxHeads = 64;
 
+// time term of the ALiBi bias: linear in seconds, slope_time[h] per second, or bucketed,
+// slope_time[h] per bucket of min(62, floor(4 log2(|t_i - t_j| + 1)))
+constexpr int kTimeBiasLinear = 0;
+constexpr int kTimeBiasBucketed = 1;
+
 // Everything an attention launch needs; slopes are copied by value.
 struct AttnArgs {
   int B;
@@ -81,6 +86,7 @@ struct AttnArgs {
   float slope_time[kMaxHeads];
   float scale;
   int dtype;
+  int time_bias;  // kTimeBiasLinear or kTimeBiasBucketed
   void* o;
   long long o_stride;  // elements
   float* lse;          // [H, T] or null
@@ -93,6 +99,22 @@ struct AttnArgs {
   void* ws;
   size_t ws_bytes;
   int32_t* err;
+};
+
+// Candidates scored against a cache of their users' history keys and values: `a`
+// describes the candidate rows (a.off = candidate offsets [B+1], a.q/k/v = candidate
+// projections with a.tok_stride, a.T = C candidate rows, a.ts = the candidates' request
+// times [C], a.o / a.lse = outputs [C, H*dh] / [H, C]); the cache has Th rows.
+struct CachedAttnArgs {
+  AttnArgs a;
+  const int32_t* hist_off;  // [B+1] rows of user u's history in the cache
+  const void* k_hist;
+  const void* v_hist;
+  long long hist_stride;  // elements
+  long long Th;
+  const int32_t* pos_hist;  // [Th]
+  const int64_t* ts_hist;   // [Th]
+  int max_cand;             // bound of the candidates per user
 };
 
 struct CandLogitsArgs {
@@ -124,6 +146,10 @@ size_t attn_bwd_simt_workspace(int B, long long T, int H, int dh, int max_seqlen
 // tcgen05 / TMEM / TMA attention forward and backward (bf16, dh = 64)
 int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st);
 size_t attn_fwd_tc_workspace(int B, long long T, int H, int max_seqlen);
+int launch_attn_fwd_cached(const CachedAttnArgs& c, cudaStream_t st);
+// forward with a dense per-user bias [B][Lpad][Lpad] (bf16) in place of the ALiBi terms
+int launch_attn_fwd_dense(const AttnArgs& a, const void* bias, long long Lpad, cudaStream_t st);
+size_t attn_fwd_cached_workspace(int B, long long C, long long Th, int H, int max_cand);
 int launch_attn_bwd_tc(const AttnArgs& a, cudaStream_t st);
 size_t attn_bwd_tc_workspace(int B, long long T, int H, int max_seqlen);
 

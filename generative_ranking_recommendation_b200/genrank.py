@@ -27,7 +27,9 @@ EXPORTS = (
     "genrank_status_string", "genrank_device_error_string", "genrank_check_error",
     "genrank_alibi_slopes", "genrank_embed_assemble", "genrank_embed_assemble_bwd",
     "genrank_attn_fwd", "genrank_attn_bwd", "genrank_attn_workspace_size",
-    "genrank_attn_fwd_static", "genrank_candidate_logits",
+    "genrank_attn_fwd_static", "genrank_candidate_logits", "genrank_attn_fwd_cached",
+    "genrank_attn_cached_workspace_size", "genrank_attn_fwd_bucketed",
+    "genrank_attn_bwd_bucketed", "genrank_attn_fwd_dense_bias",
 )
 
 
@@ -68,10 +70,18 @@ def lib():
         L.genrank_attn_fwd.argtypes = [
             _I, _L, _P, _P, _I, _P, _P, _P, _L, _I, _I, _P, _P, _P, _P, _F, _I, _P, _L, _P,
             _P, _Z, _P, _P]
+        L.genrank_attn_fwd_bucketed.restype = _I
+        L.genrank_attn_fwd_bucketed.argtypes = L.genrank_attn_fwd.argtypes
         L.genrank_attn_bwd.restype = _I
         L.genrank_attn_bwd.argtypes = [
             _I, _L, _P, _P, _I, _P, _P, _P, _L, _I, _I, _P, _P, _P, _P, _F, _I, _P, _P, _L,
             _P, _P, _P, _P, _P, _Z, _P, _P]
+        L.genrank_attn_fwd_dense_bias.restype = _I
+        L.genrank_attn_fwd_dense_bias.argtypes = [
+            _I, _L, _P, _P, _I, _P, _P, _P, _L, _I, _I, _P, _L, _F, _I, _P, _L, _P, _P, _Z, _P,
+            _P]
+        L.genrank_attn_bwd_bucketed.restype = _I
+        L.genrank_attn_bwd_bucketed.argtypes = L.genrank_attn_bwd.argtypes
         L.genrank_attn_fwd_static.restype = _I
         L.genrank_attn_fwd_static.argtypes = [
             _I, _L, _P, _P, _I, _P, _P, _P, _L, _I, _I, _P, _P, _P, _P, _F, _I, _P, _L, _P,
@@ -79,6 +89,12 @@ def lib():
         L.genrank_candidate_logits.restype = _I
         L.genrank_candidate_logits.argtypes = [
             _I, _P, _L, _I, _P, _L, _P, _L, _I, _P, _P, _P, _P, _P]
+        L.genrank_attn_fwd_cached.restype = _I
+        L.genrank_attn_fwd_cached.argtypes = [
+            _I, _L, _P, _I, _P, _P, _P, _L, _L, _P, _P, _P, _L, _P, _P, _P, _I, _I, _P, _P, _F,
+            _I, _P, _L, _P, _P, _Z, _P, _P]
+        L.genrank_attn_cached_workspace_size.restype = _Z
+        L.genrank_attn_cached_workspace_size.argtypes = [_I, _L, _L, _I, _I, _I]
         L.genrank_attn_workspace_size.restype = _Z
         L.genrank_attn_workspace_size.argtypes = [_I, _L, _I, _I, _I, _I]
         _lib = L
@@ -171,34 +187,40 @@ def _host_floats(xs):
 
 
 def attn_fwd(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts, slope_pos,
-             slope_time, scale, o, o_stride, lse, ws, dev_err, T=None, stream=None):
-    """genrank_attn_fwd.  q/k/v are tensors whose data_ptr is the first element of
-    head 0 of token 0 (views into a fused QKV buffer are fine); slopes are host lists."""
+             slope_time, scale, o, o_stride, lse, ws, dev_err, T=None, stream=None,
+             bucketed=False):
+    """genrank_attn_fwd (genrank_attn_fwd_bucketed with ``bucketed``, slope_time then
+    being the slope per time bucket).  q/k/v are tensors whose data_ptr is the first
+    element of head 0 of token 0 (views into a fused QKV buffer are fine); slopes are
+    host lists."""
     B = hist_len.numel()
     T = o.shape[0] if T is None else T
     sp, st = _host_floats(slope_pos), _host_floats(slope_time)
-    rc = lib().genrank_attn_fwd(
+    fn = lib().genrank_attn_fwd_bucketed if bucketed else lib().genrank_attn_fwd
+    rc = fn(
         B, T, _ptr(seq_offsets), _ptr(hist_len), int(max_seqlen), _ptr(q), _ptr(k), _ptr(v),
         int(tok_stride), H, dh, _ptr(pos), _ptr(ts), ctypes.cast(sp, _P), ctypes.cast(st, _P),
         float(scale), _dtype_code(q), _ptr(o), int(o_stride), _ptr(lse), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream))
-    _check(rc, "genrank_attn_fwd")
+    _check(rc, "genrank_attn_fwd_bucketed" if bucketed else "genrank_attn_fwd")
 
 
 def attn_bwd(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts, slope_pos,
              slope_time, scale, o, dO, o_stride, lse, dq, dk, dv, ws, dev_err, T=None,
-             stream=None):
-    """genrank_attn_bwd; dq/dk/dv share the layout (tok_stride) of q/k/v."""
+             stream=None, bucketed=False):
+    """genrank_attn_bwd (genrank_attn_bwd_bucketed with ``bucketed``); dq/dk/dv share
+    the layout (tok_stride) of q/k/v."""
     B = hist_len.numel()
     T = o.shape[0] if T is None else T
     sp, st = _host_floats(slope_pos), _host_floats(slope_time)
-    rc = lib().genrank_attn_bwd(
+    fn = lib().genrank_attn_bwd_bucketed if bucketed else lib().genrank_attn_bwd
+    rc = fn(
         B, T, _ptr(seq_offsets), _ptr(hist_len), int(max_seqlen), _ptr(q), _ptr(k), _ptr(v),
         int(tok_stride), H, dh, _ptr(pos), _ptr(ts), ctypes.cast(sp, _P), ctypes.cast(st, _P),
         float(scale), _dtype_code(q), _ptr(o), _ptr(dO), int(o_stride), _ptr(lse), _ptr(dq),
         _ptr(dk), _ptr(dv), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
         _ptr(dev_err), _stream(stream))
-    _check(rc, "genrank_attn_bwd")
+    _check(rc, "genrank_attn_bwd_bucketed" if bucketed else "genrank_attn_bwd")
 
 
 def attn_fwd_static(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts,
@@ -225,3 +247,41 @@ def candidate_logits(rows, x, o, w, u, z, dev_err, stream=None):
         int(x.stride(0)), _ptr(o), int(o.stride(0)), _dtype_code(x), _ptr(w), _ptr(u), _ptr(z),
         _ptr(dev_err), _stream(stream))
     _check(rc, "genrank_candidate_logits")
+
+
+def attn_cached_workspace_size(B, C, Th, H, dh, max_cand) -> int:
+    return int(lib().genrank_attn_cached_workspace_size(B, C, Th, H, dh, max_cand))
+
+
+def attn_fwd_cached(cand_offsets, max_cand, q_c, k_c, v_c, cand_stride, hist_offsets, k_hist,
+                    v_hist, hist_stride, pos_hist, ts_hist, ts_cand, H, dh, slope_pos,
+                    slope_time, scale, o, o_stride, lse, ws, dev_err, C=None, Th=None,
+                    stream=None):
+    """genrank_attn_fwd_cached: candidate rows scored against a history K/V cache.  The
+    candidate and cache tensors are views whose data_ptr is head 0 of row 0; C and Th
+    default to the row counts of o and pos_hist."""
+    B = cand_offsets.numel() - 1
+    C = o.shape[0] if C is None else C
+    Th = (pos_hist.numel() if pos_hist is not None else 0) if Th is None else Th
+    sp, st = _host_floats(slope_pos), _host_floats(slope_time)
+    rc = lib().genrank_attn_fwd_cached(
+        B, int(C), _ptr(cand_offsets), int(max_cand), _ptr(q_c), _ptr(k_c), _ptr(v_c),
+        int(cand_stride), int(Th), _ptr(hist_offsets), _ptr(k_hist), _ptr(v_hist),
+        int(hist_stride), _ptr(pos_hist), _ptr(ts_hist), _ptr(ts_cand), H, dh,
+        ctypes.cast(sp, _P), ctypes.cast(st, _P), float(scale), _dtype_code(q_c), _ptr(o),
+        int(o_stride), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _ptr(dev_err), _stream(stream))
+    _check(rc, "genrank_attn_fwd_cached")
+
+
+def attn_fwd_dense_bias(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, bias,
+                        scale, o, o_stride, lse, ws, dev_err, T=None, stream=None):
+    """genrank_attn_fwd_dense_bias: bias is a bf16 [B, Lpad, Lpad] tensor."""
+    B = hist_len.numel()
+    T = o.shape[0] if T is None else T
+    rc = lib().genrank_attn_fwd_dense_bias(
+        B, int(T), _ptr(seq_offsets), _ptr(hist_len), int(max_seqlen), _ptr(q), _ptr(k),
+        _ptr(v), int(tok_stride), H, dh, _ptr(bias), int(bias.shape[-1]), float(scale),
+        _dtype_code(q), _ptr(o), int(o_stride), _ptr(lse), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream))
+    _check(rc, "genrank_attn_fwd_dense_bias")

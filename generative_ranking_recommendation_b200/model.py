@@ -284,6 +284,8 @@ class CapturedStep:
                 a = model.rms(E.float()).to(model.dtype) if model.cfg.ffn else E
                 self._qkv, self._pos = a @ W["Wqkv"], pos
                 fn = lambda: model.attention(db, self._qkv, self._pos)[0]  # noqa: E731
+            elif part == "embed":  # metadata + gather-sum alone
+                fn = lambda: model.embed(db)[0]  # noqa: E731
             elif part == "forward":
                 fn = lambda: model.forward(db)  # noqa: E731
             else:

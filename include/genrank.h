@@ -190,6 +190,109 @@ int genrank_attn_bwd(int B, int64_t T, const int32_t *seq_offsets, const int32_t
                      void *dv, void *ws, size_t ws_bytes, int32_t *dev_err,
                      genrank_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Bucketed time bias.  fun-rec "The Overall Generative Ranking Paradigm" §7.2.2 (and
+ * its zh twin) writes the ALiBi bias as
+ *   -m_p (p_i - p_j) - m_t bucket(t_i - t_j)
+ * without defining bucket().  This library's reading: the quarter-octave grid of the
+ * pre-request time embedding, bucket(D) = min(62, floor(4 log2(D + 1))) for a gap of D
+ * seconds (two items of one request share bucket 0; gaps from about 12.9 h on share
+ * bucket 62).  Same arguments, layouts, workspace sizes and error behaviour as
+ * genrank_attn_fwd / genrank_attn_bwd, except that slope_tb[h] is the slope per
+ * bucket (the plainest reading takes slope_tb = slope_pos).  Unlike the linear time
+ * bias this term does not split into a row part and a column part, so the kernels
+ * evaluate the bucket for every visible pair (exactly, in fp32: the binary exponent
+ * of (D + 1)^4 for D + 1 <= 46341).  Per-user time spans are clamped to 2^29 s.
+ * bf16 with dh = 64 only; anything else returns GENRANK_ERR_UNSUPPORTED. */
+int genrank_attn_fwd_bucketed(int B, int64_t T, const int32_t *seq_offsets,
+                              const int32_t *hist_len, int max_seqlen, const void *q,
+                              const void *k, const void *v, int64_t tok_stride, int H, int dh,
+                              const int32_t *pos, const int64_t *ts, const float *slope_pos,
+                              const float *slope_tb, float scale, int dtype, void *o,
+                              int64_t o_stride, float *lse, void *ws, size_t ws_bytes,
+                              int32_t *dev_err, genrank_stream_t stream);
+
+/* Gradients of genrank_attn_fwd_bucketed (the bucketed bias has no parameters either):
+ * dV = P^T dO, dS = P * (dP - rowsum(dO * O)), dQ = scale dS K, dK = scale dS^T Q. */
+int genrank_attn_bwd_bucketed(int B, int64_t T, const int32_t *seq_offsets,
+                              const int32_t *hist_len, int max_seqlen, const void *q,
+                              const void *k, const void *v, int64_t tok_stride, int H, int dh,
+                              const int32_t *pos, const int64_t *ts, const float *slope_pos,
+                              const float *slope_tb, float scale, int dtype, const void *o,
+                              const void *dO, int64_t o_stride, const float *lse, void *dq,
+                              void *dk, void *dv, void *ws, size_t ws_bytes, int32_t *dev_err,
+                              genrank_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Comparison path: attention with a dense per-user N x N bias read from memory, the
+ * relative attention bias of the interleaved organisation that GenRank replaces
+ * (fun-rec "The Overall Generative Ranking Paradigm" §7.2.2: score_ij = q_i.k_j/sqrt(d)
+ * + rab(i, j), an N x N matrix whose I/O grows with the square of the length; §7.2.0:
+ * the interleaved sequence spends two tokens per interaction, 2 n_c + m in all;
+ * huaxiaozhuan "GenRank [2025]" §1.4.2).  It runs the forward kernel with the ALiBi
+ * terms replaced by one bf16 bias value per visible pair:
+ *   s_ij = scale q_i.k_j + bias[u][i][j]      (i, j local to user u)
+ * with the mask of genrank_attn_fwd (history causal; a candidate sees the history and
+ * itself), so the two layouts and the two biases can be timed on the same kernels.
+ * Arguments as genrank_attn_fwd (same workspace size), minus pos/ts/slopes, plus:
+ *   bias   [B][Lpad][Lpad] bf16, shared by the heads, row-major, 16-byte aligned
+ *   Lpad   a multiple of 128 and >= max_seqlen (every tile read stays in the block)
+ * bf16 with dh = 64 only; anything else returns GENRANK_ERR_UNSUPPORTED.  The row
+ * offset starts at 0 (no sign bound holds for a learned bias); a tile whose row sum
+ * leaves [2^-100, 2^100] is redone with its exact maximum. */
+int genrank_attn_fwd_dense_bias(int B, int64_t T, const int32_t *seq_offsets,
+                                const int32_t *hist_len, int max_seqlen, const void *q,
+                                const void *k, const void *v, int64_t tok_stride, int H, int dh,
+                                const void *bias, int64_t Lpad, float scale, int dtype, void *o,
+                                int64_t o_stride, float *lse, void *ws, size_t ws_bytes,
+                                int32_t *dev_err, genrank_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Candidate scoring from cached history keys and values (KV-cached serving).
+ * huaxiaozhuan "GenRank [2025]" §1.3.2 (feature-engineering paragraph) credits the
+ * KV cache with keeping generative ranking efficient as the candidate set grows,
+ * and fun-rec "The Overall Generative Ranking Paradigm" §7.2.1 counts the halved KV
+ * cache among the action-oriented layout's gains.  A user's history keys and values
+ * do not depend on the candidates (history rows are causal, §1.3.1), so a server
+ * keeps them and scores each request's candidates against them.  For user u with
+ * n_u = hist_offsets[u+1] - hist_offsets[u] cached rows and candidate rows
+ * [cand_offsets[u], cand_offsets[u+1]), every candidate c (position n_u + 1, time
+ * ts_cand[c]) sees the whole history and itself (§1.4.1):
+ *   s_cj = scale q_c.k_j - slope_pos[h] |p_c - p_j| - slope_time[h] |t_c - t_j|
+ *   s_cc = scale q_c.k_c
+ *   O_c = sum softmax(s) v over {history of u} + {c};  LSE_c = log sum exp(s)
+ * which equals the candidate rows of genrank_attn_fwd over history + candidates.
+ * Arguments:
+ *   B, cand_offsets [B+1]   users and their candidate rows (C = cand_offsets[B] rows)
+ *   max_cand                an upper bound of cand_offsets[u+1] - cand_offsets[u]
+ *   q_c, k_c, v_c           candidate projections, [C] rows of H * dh with row
+ *                           stride cand_stride (as genrank_attn_fwd's q, k, v)
+ *   Th, hist_offsets [B+1]  the cache: user u owns rows [hist_offsets[u],
+ *                           hist_offsets[u+1]) of k_hist, v_hist ([Th] rows of H*dh,
+ *                           stride hist_stride), pos_hist [Th] int32 (the 1-based
+ *                           positions, <= n_u + 1) and ts_hist [Th] int64 seconds,
+ *                           non-decreasing per user
+ *   ts_cand [C] int64       each candidate's request time, >= its user's last history time
+ *   o [C, H*dh] (o_stride), lse [H, C] fp32 (or NULL): outputs for the candidate rows
+ *   ws, ws_bytes            at least genrank_attn_cached_workspace_size(...) bytes;
+ *                           contents on entry do not matter
+ * bf16 with dh = 64 only (tcgen05/TMEM/TMA kernel); anything else returns
+ * GENRANK_ERR_UNSUPPORTED.  Device-detected: GENRANK_DERR_LAYOUT (offsets beyond C
+ * or Th, more than max_cand candidates), GENRANK_DERR_TS_ORDER, GENRANK_DERR_POS_RANGE. */
+int genrank_attn_fwd_cached(int B, int64_t C, const int32_t *cand_offsets, int max_cand,
+                            const void *q_c, const void *k_c, const void *v_c,
+                            int64_t cand_stride, int64_t Th, const int32_t *hist_offsets,
+                            const void *k_hist, const void *v_hist, int64_t hist_stride,
+                            const int32_t *pos_hist, const int64_t *ts_hist,
+                            const int64_t *ts_cand, int H, int dh, const float *slope_pos,
+                            const float *slope_time, float scale, int dtype, void *o,
+                            int64_t o_stride, float *lse, void *ws, size_t ws_bytes,
+                            int32_t *dev_err, genrank_stream_t stream);
+
+/* Bytes of workspace genrank_attn_fwd_cached needs for these sizes (0 if invalid). */
+size_t genrank_attn_cached_workspace_size(int B, int64_t C, int64_t Th, int H, int dh,
+                                          int max_cand);
+
 /* genrank_attn_fwd for callers that cannot allocate device memory.
  * The paper has no counterpart of this call; it exists for deployment.  Some
  * callers cannot call cudaMalloc (or any allocator, torch's included) where they

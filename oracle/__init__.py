@@ -12,12 +12,14 @@ from .genrank_oracle import (  # noqa: F401
     attention_fwd,
     attention_fwd_bucketed,
     attention_fwd_cached,
+    attention_fwd_dense_bias,
     attention_mask,
     bce_loss,
     block_backward,
     block_forward,
     embed_assemble,
     embed_assemble_bwd,
+    interleaved_layout,
     pair_time_bucket,
     time_bucket,
     token_metadata,

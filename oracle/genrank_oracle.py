@@ -374,6 +374,55 @@ def attention_fwd_cached(q_c, k_c, v_c, cand_offsets, k_hist, v_hist, hist_offse
 
 
 # ----------------------------------------------------------------------------------------
+# comparison: the interleaved layout with a dense N x N relative bias (a NEXT row)
+# ----------------------------------------------------------------------------------------
+
+def interleaved_layout(seq_offsets, hist_len):
+    """Token layout of the interleaved organisation for the same users: each history
+    interaction spends two tokens (its item, then its action), so a user with n history
+    interactions and m candidates has 2n + m tokens ([FUN-EN] §7.2.0, the interleaving
+    [Phi_0, a_0, Phi_1, a_1, ...] and its length 2 n_c + m; [HXZ] §1.4.1).  Returns the
+    new offsets [B+1] and history lengths [B] (= 2n)."""
+    n = np.asarray(hist_len, np.int64)
+    m = np.diff(np.asarray(seq_offsets, np.int64)) - n
+    off = np.zeros(len(n) + 1, np.int64)
+    off[1:] = np.cumsum(2 * n + m)
+    return off, 2 * n
+
+
+def attention_fwd_dense_bias(q, k, v, seq_offsets, hist_len, bias, scale, users=None):
+    """O [T,H,dh] and natural-log LSE [H,T] with a dense per-user bias read for every pair.
+
+    [FUN-EN] §7.2.2 writes the relative attention bias of the interleaved model as
+    score_ij = q_i.k_j / sqrt(d) + rab(i, j), an N x N matrix per sequence that the
+    forward reads in full; [HXZ] §1.4.2 notes that its I/O grows with the square of the
+    length.  Here bias[u] is user u's [Lpad, Lpad] matrix (shared by the heads), local
+    indices; the mask is the one of ``attention_fwd`` (history causal, a candidate sees
+    the history and itself).
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    T, H, dh = q.shape
+    O = np.zeros((T, H, dh))
+    LSE = np.full((H, T), np.nan)
+    users = range(len(hist_len)) if users is None else users
+    for u in users:
+        s, e, n = int(seq_offsets[u]), int(seq_offsets[u + 1]), int(hist_len[u])
+        L = e - s
+        Bu = np.asarray(bias[u][:L, :L], np.float64)
+        mask = attention_mask(n, L)
+        for h in range(H):
+            S = np.where(mask, (q[s:e, h] @ k[s:e, h].T) * scale + Bu, -np.inf)
+            mx = S.max(axis=1, keepdims=True)
+            P = np.exp(S - mx)
+            l = P.sum(axis=1, keepdims=True)
+            O[s:e, h] = (P / l) @ v[s:e, h]
+            LSE[h, s:e] = (mx + np.log(l))[:, 0]
+    return O, LSE
+
+
+# ----------------------------------------------------------------------------------------
 # the model blocks around the hot path (projections, norms, FFN, head, loss)
 # ----------------------------------------------------------------------------------------
 

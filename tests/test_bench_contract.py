@@ -35,3 +35,23 @@ def test_warmup_below_three_is_refused():
                         "--steps", "1", "--warmup", "2"], cwd=ROOT, capture_output=True,
                        text=True, timeout=120)
     assert r.returncode != 0
+
+
+def test_config_block_describes_every_workload():
+    """Every configuration's history kind (uniform, fixed, lognormal) and mode (scoring or
+    training) is named in the bench line's workload description."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from gen import CONFIGS
+
+    for name, cfg in CONFIGS.items():
+        c = bench.config_block(cfg, 2)
+        w = c["workload"]
+        assert name in w and c["config"] == name
+        assert ("training step" in w) == cfg.training
+        assert ("inference scoring" in w) == (not cfg.training)
+        kind = cfg.hist[0]
+        assert {"uniform": "U[", "fixed": "every history at", "lognormal": "lognormal("}[kind] in w
+        assert c["global_batch_users"] == 2 * cfg.B
+        assert c["candidates_per_step"] == 2 * cfg.B * cfg.m
+    assert bench.DEFAULT_CONFIG == "c2"

@@ -335,6 +335,87 @@ int genrank_attn_fwd_dense_bias(int B, int64_t T, const int32_t* seq_offsets,
   return launch_attn_fwd_dense(a, bias, Lpad, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int genrank_linear(int M, int N, int K, const void* A, int64_t lda, const void* Wt, int64_t ldw,
+                   int epilogue, void* C, int64_t ldc, int32_t* dev_err,
+                   genrank_stream_t stream) {
+  if (M < 0 || N < 1 || K < 1 || !dev_err) return GENRANK_ERR_INVALID_ARG;
+  if (epilogue != GENRANK_EPI_STORE && epilogue != GENRANK_EPI_SILU) return GENRANK_ERR_INVALID_ARG;
+  if (N % 256 || K % 64) return GENRANK_ERR_UNSUPPORTED;
+  if (M == 0) return GENRANK_OK;
+  if (!A || !Wt || !C || !aligned16(A) || !aligned16(Wt) || !aligned16(C))
+    return GENRANK_ERR_INVALID_ARG;
+  if (lda < K || ldw < K || ldc < N || (lda * 2) % 16 || (ldw * 2) % 16 || (ldc * 2) % 16)
+    return GENRANK_ERR_INVALID_ARG;
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.a = A;
+  g.lda = lda;
+  g.w = Wt;
+  g.ldw = ldw;
+  g.epilogue = epilogue == GENRANK_EPI_SILU ? kEpiSilu : kEpiStore;
+  g.c = C;
+  g.ldc = ldc;
+  g.err = dev_err;
+  return launch_gemm_tc(g, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int genrank_linear_residual_rmsnorm(int M, int d, int K, const void* A, int64_t lda,
+                                    const void* Wt, int64_t ldw, const float* x_in,
+                                    float* x_out, int64_t ldx, void* a_out, int64_t lda_out,
+                                    const float* w_head, float* z, float eps, int32_t* dev_err,
+                                    genrank_stream_t stream) {
+  if (M < 0 || d < 1 || K < 1 || !dev_err || !(eps >= 0.f)) return GENRANK_ERR_INVALID_ARG;
+  if (d != 512 || K % 64) return GENRANK_ERR_UNSUPPORTED;
+  if (M == 0) return GENRANK_OK;
+  if (!A || !Wt || !x_in || !x_out || (!a_out && !w_head) || (w_head && !z))
+    return GENRANK_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(Wt) || !aligned16(x_in) || !aligned16(x_out) ||
+      (a_out && !aligned16(a_out)) || (w_head && !aligned16(w_head)))
+    return GENRANK_ERR_INVALID_ARG;
+  if (lda < K || ldw < K || ldx < d || (a_out && lda_out < d) || (lda * 2) % 16 ||
+      (ldw * 2) % 16 || (ldx * 4) % 16 || (a_out && (lda_out * 2) % 16))
+    return GENRANK_ERR_INVALID_ARG;
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.M = M;
+  g.N = d;
+  g.K = K;
+  g.a = A;
+  g.lda = lda;
+  g.w = Wt;
+  g.ldw = ldw;
+  g.epilogue = kEpiResRms;
+  g.x_in = x_in;
+  g.x_out = x_out;
+  g.ldx = ldx;
+  g.a_out = a_out;
+  g.lda_out = lda_out;
+  g.w_head = w_head;
+  g.z = z;
+  g.eps = eps;
+  g.err = dev_err;
+  return launch_gemm_tc(g, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int genrank_rmsnorm(int64_t M, int d, const void* x, int64_t ldx, int dtype, float* x_out,
+                    int64_t ldxo, void* a_out, int64_t lda_out, float eps, int32_t* dev_err,
+                    genrank_stream_t stream) {
+  const int es = elem_size(dtype);
+  if (M < 0 || d < 1 || !es || !dev_err || !(eps >= 0.f)) return GENRANK_ERR_INVALID_ARG;
+  if ((d * es) % 16 || d % 8) return GENRANK_ERR_UNSUPPORTED;
+  if (M == 0) return GENRANK_OK;
+  if (!x || !a_out || !aligned16(x) || !aligned16(a_out) || (x_out && !aligned16(x_out)))
+    return GENRANK_ERR_INVALID_ARG;
+  if (ldx < d || lda_out < d || (x_out && ldxo < d) || (ldx * es) % 16 || (lda_out * 2) % 16 ||
+      (x_out && (ldxo * 4) % 16))
+    return GENRANK_ERR_INVALID_ARG;
+  return launch_rmsnorm(M, d, x, ldx, dtype, x_out, ldxo, a_out, lda_out, eps,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t genrank_attn_cached_workspace_size(int B, int64_t C, int64_t Th, int H, int dh,
                                           int max_cand) {
   if (B < 1 || C < 0 || Th < 0 || H < 1 || dh < 1 || max_cand < 0) return 0;

@@ -99,7 +99,7 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, DH, 0, 1);  // P K-major (TMEM)
 
 // scratch layout
 constexpr size_t kHeaderBytes = 256;
-constexpr int kRecInts = 8;  // s, L, n, q0, nk, spad, u, kb
+constexpr int kRecInts = 12;  // s, L, n, q0, nk, spad, u, kb, rb, 3 unused
 
 struct Params {
   const int32_t* trel;  // bucketed bias: per-token time since the user's first token, [Tp]
@@ -133,15 +133,18 @@ GR_DEVICE int tiles_of(int q0, int n, int L, int nk) {
 // One work item: query rows [q0, q0 + 128) of a user whose sequence has L rows, the
 // first n of them history.  Query row i (and the diagonal tile's key i) lives at row
 // s + i of the query-side arrays; history key j at row kb + j of the key-side arrays.
+// Column terms: history key j at spad + j, query row i (and diagonal key i) at rb + i;
+// both spad and rb + q0 are multiples of 4 (16-byte aligned bulk copies).
 struct Item {
-  int s, L, n, q0, nk, spad, h, kb, u;
+  int s, L, n, q0, nk, spad, h, kb, u, rb;
   int nt;  // tiles visited: nk key tiles, plus the diagonal tile when candidates are present
 };
 
 GR_DEVICE Item load_item(const Params& P, int w) {
   const int pair = w / P.a.H;
-  const int4 r0 = P.recs[2 * pair];
-  const int4 r1 = P.recs[2 * pair + 1];
+  const int4 r0 = P.recs[3 * pair];
+  const int4 r1 = P.recs[3 * pair + 1];
+  const int4 r2 = P.recs[3 * pair + 2];
   Item it;
   it.h = w - pair * P.a.H;
   it.s = r0.x;
@@ -152,6 +155,7 @@ GR_DEVICE Item load_item(const Params& P, int w) {
   it.spad = r1.y;
   it.kb = r1.w;
   it.u = r1.z;
+  it.rb = r2.x;
   it.nt = tiles_of(it.q0, it.n, it.L, it.nk);
   return it;
 }
@@ -163,6 +167,15 @@ __host__ __device__ inline long long seg_start(long long s, int u) {
 }
 __host__ __device__ inline long long scratch_tp(long long T, int B) {
   return ((T + 4LL * B + 4 + BN) + 3) / 4 * 4;
+}
+// Candidate scoring from a cache: a user's segment holds its n history terms, padding to a
+// multiple of 4, then its m candidates' terms (at most L + 3 entries), so segments start
+// 8 entries apart beyond their lengths.
+__host__ __device__ inline long long seg_start_cached(long long s, int u) {
+  return 4 * ((s + 3) / 4) + 8LL * u;
+}
+__host__ __device__ inline long long scratch_tp_cached(long long T, int B) {
+  return ((T + 8LL * B + 8 + BN) + 3) / 4 * 4;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -279,8 +292,10 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue(const __grid_constan
     for (int t = tiles - 1; t >= 0; --t, ++slot) {
       const int kmax = min(t * BM + BM, n);
       const int nk = kmax > 0 ? (kmax + BN - 1) / BN : 0;
-      recs[2 * slot] = make_int4(s, L, n, t * BM);
-      recs[2 * slot + 1] = make_int4(nk, (int)seg_start(s, u), u, s);
+      const int seg = (int)seg_start(s, u);
+      recs[3 * slot] = make_int4(s, L, n, t * BM);
+      recs[3 * slot + 1] = make_int4(nk, seg, u, s);
+      recs[3 * slot + 2] = make_int4(seg, 0, 0, 0);
     }
   }
   if (threadIdx.x == 0) *count = total;
@@ -317,7 +332,8 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue_cached(
     int cs, n, m, hs;
     if (!cached_user(c, b, cs, n, m, hs)) return;  // flagged by the schedule block
     const int L = n + m;
-    const long long base = seg_start((long long)hs + cs, b);
+    const long long base = seg_start_cached((long long)hs + cs, b);
+    const int n4 = (n + 3) & ~3;  // candidates' terms start 16-byte aligned
     const long long t0 = n > 0 ? c.ts_hist[hs] : (m > 0 ? a.ts[cs] : 0);
     const long long t_last = n > 0 ? c.ts_hist[hs + n - 1] : LLONG_MIN;
     for (int i = threadIdx.x; i < L; i += blockDim.x) {
@@ -334,8 +350,9 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue_cached(
         if (t < t_last) flag(a.err, GENRANK_DERR_TS_ORDER);
       }
       const float pf = (float)p, dt = (float)(t - t0);
+      const long long at = base + (i < n ? i : n4 + (i - n));
       for (int h = 0; h < a.H; ++h)
-        cbias[(long long)h * Tp + base + i] = kLog2e * (a.slope_pos[h] * pf + a.slope_time[h] * dt);
+        cbias[(long long)h * Tp + at] = kLog2e * (a.slope_pos[h] * pf + a.slope_time[h] * dt);
     }
     return;
   }
@@ -381,10 +398,12 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue_cached(
     int cs, n, m, hs;
     cached_user(c, u, cs, n, m, hs);
     const int nk = (n + BN - 1) / BN;
-    const int seg = (int)seg_start((long long)hs + cs, u);
+    const int seg = (int)seg_start_cached((long long)hs + cs, u);
+    const int n4 = (n + 3) & ~3;
     for (int t = tiles - 1; t >= 0; --t, ++slot) {
-      recs[2 * slot] = make_int4(cs - n, n + m, n, n + t * BM);
-      recs[2 * slot + 1] = make_int4(nk, seg, u, hs);
+      recs[3 * slot] = make_int4(cs - n, n + m, n, n + t * BM);
+      recs[3 * slot + 1] = make_int4(nk, seg, u, hs);
+      recs[3 * slot + 2] = make_int4(seg + n4 - n, 0, 0, 0);  // rb: rb + q0 = seg + n4 + 128 t
     }
   }
   if (threadIdx.x == 0) *count = total;
@@ -741,7 +760,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
         ok = false;
         break;
       }
-      const float* cb_src = P.cbias + (long long)it.h * P.Tp + it.spad;
+      const float* cb_src = P.cbias + (long long)it.h * P.Tp + it.spad;  // history keys
+      const float* cbr_src = P.cbias + (long long)it.h * P.Tp + it.rb;   // query rows
       const int32_t* tr_src = kBucket ? P.trel + it.spad : nullptr;
       if (lane == 0) {
         sRec[2 * qb] = make_int4(it.q0, it.n, it.L, it.nk);
@@ -751,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
         tma_load_3d(smem + kOffQ + qb * kTileBytes, &P.tq, &bars[kQFull + qb], 0, it.h,
                     it.s + it.q0);
         if (!kDense)
-          bulk_load(smem + kOffQCB + qb * kCBBytes, cb_src + it.q0, kCBBytes, &bars[kQFull + qb]);
+          bulk_load(smem + kOffQCB + qb * kCBBytes, cbr_src + it.q0, kCBBytes, &bars[kQFull + qb]);
         if (kBucket)
           bulk_load(smem + kOffQTR + qb * kCBBytes, tr_src + it.q0, kCBBytes, &bars[kQFull + qb]);
       }
@@ -772,7 +792,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
           tma_load_3d(smem + kOffK + st * kTileBytes, hist ? &P.tk : &P.tkc, &bars[kKFull + st],
                       0, it.h, row);
           if (!kDense)
-            bulk_load(smem + kOffCB + st * kCBBytes, cb_src + kv0, kCBBytes, &bars[kKFull + st]);
+            bulk_load(smem + kOffCB + st * kCBBytes, hist ? cb_src + kv0 : cbr_src + kv0, kCBBytes,
+                      &bars[kKFull + st]);
           if (kBucket)
             bulk_load(smem + kOffTR + st * kCBBytes, tr_src + kv0, kCBBytes, &bars[kKFull + st]);
           mbar_expect_tx(&bars[kVFull + st], kTileBytes);
@@ -1171,7 +1192,7 @@ int launch_attn_fwd_dense(const AttnArgs& a, const void* bias, long long Lpad, c
 size_t attn_fwd_cached_workspace(int B, long long C, long long Th, int H, int max_cand) {
   using namespace tc;
   return kHeaderBytes + recs_bytes(B, max_cand) + users_bytes(B) +
-         (size_t)H * scratch_tp(C + Th, B) * sizeof(float);
+         (size_t)H * scratch_tp_cached(C + Th, B) * sizeof(float);
 }
 
 int launch_attn_fwd_cached(const CachedAttnArgs& c, cudaStream_t st) {
@@ -1201,7 +1222,7 @@ int launch_attn_fwd_cached(const CachedAttnArgs& c, cudaStream_t st) {
   p.count = count;
   p.recs = recs;
   p.cbias = cbias;
-  p.Tp = scratch_tp(a.T + c.Th, a.B);
+  p.Tp = scratch_tp_cached(a.T + c.Th, a.B);
   CachedArgsHolder holder{c};
   k_prologue_cached<<<a.B + 1, kSchedThreads, 0, st>>>(holder, max_tiles_of(c.max_cand), recs,
                                                        count, uorder, cbias, p.Tp);

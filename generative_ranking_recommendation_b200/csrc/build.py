@@ -22,7 +22,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgenrank.so")
 SOURCES = ["api.cu", "embed.cu", "attn_simt.cu", "attn_tc.cu", "attn_bwd_tc.cu", "noalloc.cu",
-           "head.cu"]
+           "head.cu", "gemm_tc.cu"]
 HEADERS = ["common.cuh", "kernels.h", "host_util.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

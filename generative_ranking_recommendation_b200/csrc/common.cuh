@@ -240,6 +240,14 @@ GR_DEVICE void tma_load_3d(void* smem_dst, const void* tmap, uint64_t* bar, int 
       : "memory");
 }
 
+GR_DEVICE void tma_load_2d(void* smem_dst, const void* tmap, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
 // Reduce-add of a shared-memory box into a global tensor (tile mode, no multicast), by the
 // TMA engine; completion is tracked per thread in bulk groups.
 GR_DEVICE void tma_reduce_add_3d(const void* tmap, const void* smem_src, int c0, int c1, int c2) {

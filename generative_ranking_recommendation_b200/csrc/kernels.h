@@ -117,6 +117,33 @@ struct CachedAttnArgs {
   int max_cand;             // bound of the candidates per user
 };
 
+// C = A Wt^T on tensor cores with a fused epilogue (bf16 A [M][K], Wt [N][K], K-major)
+constexpr int kEpiStore = 0;   // C = bf16(A W)
+constexpr int kEpiSilu = 1;    // C = bf16(SiLU(A W))
+constexpr int kEpiResRms = 2;  // x_out = x_in + A W; a_out = bf16(rms(x_out)); z = rms . w
+struct GemmArgs {
+  int M, N, K;
+  const void* a;
+  long long lda;
+  const void* w;  // Wt [N][K]
+  long long ldw;
+  int epilogue;
+  void* c;  // store / silu: [M][N] bf16
+  long long ldc;
+  const float* x_in;  // res+rms: [M][N] fp32 residual stream in and out (may alias)
+  float* x_out;
+  long long ldx;
+  void* a_out;  // res+rms: [M][N] bf16 normalised rows, or null
+  long long lda_out;
+  const float* w_head;  // res+rms: [N] fp32 head vector, or null
+  float* z;             // res+rms: [M] fp32 head output
+  float eps;
+  int32_t* err;
+};
+int launch_gemm_tc(const GemmArgs& g, cudaStream_t st);
+int launch_rmsnorm(long long M, int d, const void* x, long long ldx, int x_dtype, float* x_out,
+                   long long ldxo, void* a_out, long long lda, float eps, cudaStream_t st);
+
 struct CandLogitsArgs {
   long long M;
   const int64_t* rows;

@@ -29,8 +29,10 @@ EXPORTS = (
     "genrank_attn_fwd", "genrank_attn_bwd", "genrank_attn_workspace_size",
     "genrank_attn_fwd_static", "genrank_candidate_logits", "genrank_attn_fwd_cached",
     "genrank_attn_cached_workspace_size", "genrank_attn_fwd_bucketed",
-    "genrank_attn_bwd_bucketed", "genrank_attn_fwd_dense_bias",
+    "genrank_attn_bwd_bucketed", "genrank_attn_fwd_dense_bias", "genrank_linear",
+    "genrank_linear_residual_rmsnorm", "genrank_rmsnorm",
 )
+EPI_STORE, EPI_SILU = 0, 1
 
 
 class GenRankError(RuntimeError):
@@ -80,6 +82,13 @@ def lib():
         L.genrank_attn_fwd_dense_bias.argtypes = [
             _I, _L, _P, _P, _I, _P, _P, _P, _L, _I, _I, _P, _L, _F, _I, _P, _L, _P, _P, _Z, _P,
             _P]
+        L.genrank_linear.restype = _I
+        L.genrank_linear.argtypes = [_I, _I, _I, _P, _L, _P, _L, _I, _P, _L, _P, _P]
+        L.genrank_linear_residual_rmsnorm.restype = _I
+        L.genrank_linear_residual_rmsnorm.argtypes = [
+            _I, _I, _I, _P, _L, _P, _L, _P, _P, _L, _P, _L, _P, _P, _F, _P, _P]
+        L.genrank_rmsnorm.restype = _I
+        L.genrank_rmsnorm.argtypes = [_L, _I, _P, _L, _I, _P, _L, _P, _L, _F, _P, _P]
         L.genrank_attn_bwd_bucketed.restype = _I
         L.genrank_attn_bwd_bucketed.argtypes = L.genrank_attn_bwd.argtypes
         L.genrank_attn_fwd_static.restype = _I
@@ -285,3 +294,38 @@ def attn_fwd_dense_bias(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, 
         _dtype_code(q), _ptr(o), int(o_stride), _ptr(lse), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream))
     _check(rc, "genrank_attn_fwd_dense_bias")
+
+
+def linear(A, Wt, C, dev_err, epilogue=EPI_STORE, stream=None):
+    """genrank_linear: C = bf16(A Wt^T), or bf16(SiLU(A Wt^T)) with EPI_SILU.  A [M, K],
+    Wt [N, K] (the transposed weight), C [M, N]; bf16, row strides from the tensors."""
+    M, K = A.shape
+    N = Wt.shape[0]
+    rc = lib().genrank_linear(int(M), int(N), int(K), _ptr(A), int(A.stride(0)), _ptr(Wt),
+                              int(Wt.stride(0)), int(epilogue), _ptr(C), int(C.stride(0)),
+                              _ptr(dev_err), _stream(stream))
+    _check(rc, "genrank_linear")
+
+
+def linear_residual_rmsnorm(A, Wt, x_in, x_out, a_out, dev_err, w_head=None, z=None,
+                            eps=1e-6, stream=None):
+    """genrank_linear_residual_rmsnorm: x_out = x_in + A Wt^T (fp32), a_out = bf16 rms of
+    it (or None), z = rms(x_out) . w_head when w_head is given."""
+    M, K = A.shape
+    d = Wt.shape[0]
+    rc = lib().genrank_linear_residual_rmsnorm(
+        int(M), int(d), int(K), _ptr(A), int(A.stride(0)), _ptr(Wt), int(Wt.stride(0)),
+        _ptr(x_in), _ptr(x_out), int(x_out.stride(0)), _ptr(a_out),
+        int(a_out.stride(0)) if a_out is not None else 0, _ptr(w_head), _ptr(z), float(eps),
+        _ptr(dev_err), _stream(stream))
+    _check(rc, "genrank_linear_residual_rmsnorm")
+
+
+def rmsnorm(x, a_out, dev_err, x_out=None, eps=1e-6, stream=None):
+    """genrank_rmsnorm: a_out = bf16 rms(x); x_out = fp32 copy of x when given."""
+    M, d = x.shape
+    rc = lib().genrank_rmsnorm(int(M), int(d), _ptr(x), int(x.stride(0)), _dtype_code(x),
+                               _ptr(x_out), int(x_out.stride(0)) if x_out is not None else 0,
+                               _ptr(a_out), int(a_out.stride(0)), float(eps), _ptr(dev_err),
+                               _stream(stream))
+    _check(rc, "genrank_rmsnorm")

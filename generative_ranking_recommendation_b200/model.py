@@ -89,6 +89,9 @@ class GenRankModel:
             if cfg.ffn:
                 W["W1"] = _tt(L["W1"], dt, dev)
                 W["W2"] = _tt(L["W2"], dt, dev)
+            # the library's linear layers take each weight transposed ([N][K], K-major)
+            for k in list(W):
+                W[k + "T"] = W[k].t().contiguous()
             self.layers.append(W)
         self.w_head = _tt(model.w_head, torch.float32, dev)
         self.H, self.dh, self.d = cfg.H, cfg.dh, cfg.d
@@ -97,6 +100,12 @@ class GenRankModel:
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self._ws = {}
         self._head_u = None
+        # the scoring step runs its projections on the library's tensor-core linear
+        # layers (bf16; widths the tiles divide), the four-layer block with the fused
+        # residual + RMSNorm epilogues (d = 512); otherwise the blocks are torch ops
+        d = cfg.d
+        self.fused_qkv = cfg.dtype == "bf16" and (3 * d) % 256 == 0 and d % 64 == 0
+        self.fused_blocks = self.fused_qkv and cfg.ffn and d == 512
 
     # -------------------------------------------------------------------------------------
     def workspace(self, db: DeviceBatch, bwd: bool) -> torch.Tensor:
@@ -150,9 +159,67 @@ class GenRankModel:
         return x * torch.rsqrt((x * x).mean(dim=-1, keepdim=True) + RMS_EPS)
 
     # -------------------------------------------------------------------------------------
+    def _event(self, attn_events):
+        if attn_events is None:
+            return None
+        ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        ev[0].record()
+        attn_events.append(ev)
+        return ev
+
+    def _linear(self, a, Wt, epilogue=G.EPI_STORE):
+        out = torch.empty((a.shape[0], Wt.shape[0]), dtype=self.dtype, device=self.device)
+        G.linear(a, Wt, out, self.err, epilogue=epilogue)
+        return out
+
     @torch.no_grad()
-    def forward(self, db: DeviceBatch, attn_events=None) -> torch.Tensor:
+    def forward(self, db: DeviceBatch, attn_events=None, blocks: str = "auto") -> torch.Tensor:
         """Candidate logits (fp32 [sum m]) for one batch.
+
+        ``blocks``: "auto" runs the projections, norms and FFN on the library's fused
+        tensor-core linear layers where the shapes allow (``fused_blocks`` /
+        ``fused_qkv``), "torch" runs them as torch ops (cuBLAS + elementwise kernels).
+        """
+        if blocks == "auto" and self.fused_blocks:
+            return self._forward_fused(db, attn_events)
+        return self._forward_torch(db, attn_events, fused_qkv=blocks == "auto" and self.fused_qkv)
+
+    def _forward_fused(self, db: DeviceBatch, attn_events=None) -> torch.Tensor:
+        """The four-layer scoring step on the library's kernels end to end: embedding
+        assembly, RMSNorm, per layer the QKV projection, the attention, W_o with the
+        residual update and the next RMSNorm in its epilogue, W1 with SiLU in its
+        epilogue and W2 with the residual update and the next RMSNorm; the last layer's
+        W_o and FFN run on candidate rows only and its W2 epilogue applies the final
+        RMSNorm and the head."""
+        E, (pos, _, _) = self.embed(db)
+        T, d, dev = db.T, self.d, self.device
+        x = torch.empty((T, d), dtype=torch.float32, device=dev)
+        a = torch.empty((T, d), dtype=self.dtype, device=dev)
+        G.rmsnorm(E, a, self.err, x_out=x, eps=RMS_EPS)
+        nl = len(self.layers)
+        for li, W in enumerate(self.layers):
+            qkv = self._linear(a, W["WqkvT"])
+            ev = self._event(attn_events)
+            o, _ = self.attention(db, qkv, pos)
+            if ev is not None:
+                ev[1].record()
+            if li == nl - 1:  # only candidate rows reach the head
+                rows = db.cand_rows
+                o, x = o.index_select(0, rows), x.index_select(0, rows)
+            a2 = torch.empty_like(o)
+            G.linear_residual_rmsnorm(o, W["WoT"], x, x, a2, self.err, eps=RMS_EPS)
+            u = self._linear(a2, W["W1T"], G.EPI_SILU)
+            if li == nl - 1:
+                z = torch.empty(x.shape[0], dtype=torch.float32, device=dev)
+                G.linear_residual_rmsnorm(u, W["W2T"], x, x, None, self.err, w_head=self.w_head,
+                                          z=z, eps=RMS_EPS)
+                return z
+            G.linear_residual_rmsnorm(u, W["W2T"], x, x, a, self.err, eps=RMS_EPS)
+        raise ValueError("a model needs at least one layer")
+
+    def _forward_torch(self, db: DeviceBatch, attn_events=None, fused_qkv=False) -> torch.Tensor:
+        """Candidate logits with the blocks as torch ops (the QKV projection optionally on
+        the library's linear layer).
 
         Every layer's attention runs over all tokens (history rows feed the next
         layer's keys and values).  After the last attention only candidate rows
@@ -172,14 +239,11 @@ class GenRankModel:
                 a = self.rms(x).to(self.dtype)
             else:
                 a = E if li == 0 else x.to(self.dtype)
-            qkv = a @ W["Wqkv"]
-            if attn_events is not None:
-                ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                ev[0].record()
+            qkv = self._linear(a, W["WqkvT"]) if fused_qkv else a @ W["Wqkv"]
+            ev = self._event(attn_events)
             o, _ = self.attention(db, qkv, pos)
-            if attn_events is not None:
+            if ev is not None:
                 ev[1].record()
-                attn_events.append(ev)
             if li == nl - 1 and x is None:
                 # one block, no FFN: z = E . w_head + o . (W_o w_head) at candidate rows,
                 # one fused gather-dot kernel

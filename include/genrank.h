@@ -337,6 +337,45 @@ int genrank_candidate_logits(int M, const int64_t *rows, int64_t T, int d, const
                              const float *w, const float *u, float *z, int32_t *dev_err,
                              genrank_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * The blocks around the attention, on tensor cores with fused epilogues.
+ * huaxiaozhuan "GenRank [2025]" §1.4.1 and fun-rec §7.2.1: the action-oriented layout
+ * halves the tokens and so the linear-projection cost; the four-layer workloads'
+ * block is pre-RMSNorm (unit gain) attention and a 4d SiLU FFN, each added to an fp32
+ * residual stream, with a final RMSNorm and the candidate head.  Matrices are
+ * row-major; A and the weights are bf16, and a weight W [K][N] is passed TRANSPOSED,
+ * Wt [N][K] (each output column's weights contiguous), so both tensor-core operands
+ * are K-major.  Accumulation is fp32 in tensor memory.  Pointers 16-byte aligned,
+ * row strides (elements) multiples of 16 bytes. */
+enum { GENRANK_EPI_STORE = 0, GENRANK_EPI_SILU = 1 };
+
+/* C [M][N] = bf16(A W) (GENRANK_EPI_STORE) or bf16(SiLU(A W)) (GENRANK_EPI_SILU),
+ * A [M][K], Wt [N][K].  N a multiple of 256, K a multiple of 64, else
+ * GENRANK_ERR_UNSUPPORTED. */
+int genrank_linear(int M, int N, int K, const void *A, int64_t lda, const void *Wt, int64_t ldw,
+                   int epilogue, void *C, int64_t ldc, int32_t *dev_err,
+                   genrank_stream_t stream);
+
+/* The residual update and the next RMSNorm in one pass over each row:
+ *   x_out = x_in + A W                      (fp32 [M][d]; x_out may equal x_in)
+ *   a_out = bf16(x_out / sqrt(mean_j x_out_j^2 + eps))     (or NULL)
+ *   z     = (x_out / sqrt(mean_j x_out_j^2 + eps)) . w_head (when w_head != NULL; z [M])
+ * A [M][K] bf16, Wt [d][K] bf16.  d must be 512 (one 128 x 512 fp32 tile fills tensor
+ * memory), K a multiple of 64; else GENRANK_ERR_UNSUPPORTED.  At least one of a_out
+ * and w_head must be given. */
+int genrank_linear_residual_rmsnorm(int M, int d, int K, const void *A, int64_t lda,
+                                    const void *Wt, int64_t ldw, const float *x_in,
+                                    float *x_out, int64_t ldx, void *a_out, int64_t lda_out,
+                                    const float *w_head, float *z, float eps, int32_t *dev_err,
+                                    genrank_stream_t stream);
+
+/* a_out [M][d] = bf16(x / sqrt(mean_j x_j^2 + eps)) for x [M][d] in dtype, and x_out =
+ * fp32 copy of x when x_out != NULL (the residual stream of the first block).  d a
+ * multiple of 8 with d * sizeof(dtype) a multiple of 16. */
+int genrank_rmsnorm(int64_t M, int d, const void *x, int64_t ldx, int dtype, float *x_out,
+                    int64_t ldxo, void *a_out, int64_t lda_out, float eps, int32_t *dev_err,
+                    genrank_stream_t stream);
+
 /* Bytes of workspace genrank_attn_fwd (is_bwd = 0) or genrank_attn_bwd
  * (is_bwd = 1) need for these sizes.  Returns 0 for invalid sizes. */
 size_t genrank_attn_workspace_size(int B, int64_t T, int H, int dh, int max_seqlen, int is_bwd);

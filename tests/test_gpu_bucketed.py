@@ -72,11 +72,10 @@ def run(G, cfg, batch, pos, qkv, dO=None, bucketed=True, slope_scale=1.0):
     return out
 
 
-def _rel_rows(a, b, name):
-    assert ref.rel_to_max(a, b) <= BF16_TOL, name
-    err = np.abs(a - b).max(axis=(1, 2))
-    den = np.maximum(np.abs(b).max(axis=(1, 2)), np.abs(b).max() / 16.0)
-    assert np.max(err / den) <= BF16_TOL, (name, int(np.argmax(err / den)))
+def _rel_rows(a, b, name, noise=None):
+    """Relative to the max plus the per-token bound; for dq the noise floor the bf16 O
+    carries into D_i (see ref.dq_noise_floor)."""
+    ref.check_rows(a, b, BF16_TOL, name, noise=noise)
 
 
 def _boundary_batch(cfg):
@@ -115,8 +114,9 @@ def test_bucketed_fwd_bwd_parity(G, slope_scale):
     want = _oracle(batch, pos, qkv, cfg.H, cfg.dh, dO, slope_scale=slope_scale)
     _rel_rows(got[0], want[0], "O")
     assert np.max(np.abs(got[1] - want[1])) <= 2e-2
+    noise = ref.dq_noise_floor(qkv[:, 1], dO, want[0], batch.seq_offsets, 1.0 / math.sqrt(cfg.dh))
     for k, name in zip(range(2, 5), ("dq", "dk", "dv")):
-        _rel_rows(got[k], want[k], name)
+        _rel_rows(got[k], want[k], name, noise if name == "dq" else None)
 
 
 def test_bucketed_parity_random_users(G):
@@ -130,8 +130,9 @@ def test_bucketed_parity_random_users(G):
     want = _oracle(batch, pos, qkv, cfg.H, cfg.dh, dO)
     _rel_rows(got[0], want[0], "O")
     assert np.max(np.abs(got[1] - want[1])) <= 2e-2
+    noise = ref.dq_noise_floor(qkv[:, 1], dO, want[0], batch.seq_offsets, 1.0 / math.sqrt(cfg.dh))
     for k, name in zip(range(2, 5), ("dq", "dk", "dv")):
-        _rel_rows(got[k], want[k], name)
+        _rel_rows(got[k], want[k], name, noise if name == "dq" else None)
 
 
 def test_one_request_per_user_equals_linear_bias_bitwise(G):
@@ -175,5 +176,6 @@ def test_bucketed_full_size_c3_sampled(G):
     rows = ref.user_rows(batch, users)
     _rel_rows(got[0][rows], O[rows], "O")
     assert np.max(np.abs(got[1][:, rows] - L[:, rows])) <= 2e-2
+    noise = ref.dq_noise_floor(qkv[:, 1], dO, O, batch.seq_offsets, 1.0 / math.sqrt(cfg.dh))
     for k, (name, w) in enumerate((("dq", dq), ("dk", dk), ("dv", dv))):
-        _rel_rows(got[2 + k][rows], w[rows], name)
+        _rel_rows(got[2 + k][rows], w[rows], name, noise[rows] if name == "dq" else None)

@@ -96,3 +96,20 @@ def test_captured_step_matches_forward(M, name):
     from generative_ranking_recommendation_b200 import genrank as G
 
     assert G.check_error(gm.err) == 0
+
+
+@pytest.mark.parametrize("name", ["c2", "c1"])
+def test_fused_blocks_match_torch_blocks(M, name):
+    """The scoring step on the library's fused linear layers and the same step with the
+    blocks as torch ops give the same logits within the bf16 tolerance."""
+    cfg = CONFIGS[name]
+    batch = make_batch(cfg, users=list(range(16)))
+    gm = M.GenRankModel(cfg, make_model(cfg), "cuda")
+    assert gm.fused_qkv and gm.fused_blocks == (name == "c2")
+    db = M.DeviceBatch.from_batch(batch, "cuda")
+    z_fused = gm.forward(db).double().cpu().numpy()
+    z_torch = gm.forward(db, blocks="torch").double().cpu().numpy()
+    assert ref.rel_to_max(z_fused, z_torch) <= 2e-2
+    from generative_ranking_recommendation_b200 import genrank as G
+
+    assert G.check_error(gm.err) == 0

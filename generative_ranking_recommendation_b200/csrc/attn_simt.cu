@@ -60,13 +60,13 @@ __global__ void __launch_bounds__(128) k_attn_fwd_simt(const __grid_constant__ A
   __shared__ float sK[kChunk][DH + 1], sV[kChunk][DH + 1];
   __shared__ int sP[kChunk];
   __shared__ long long sT[kChunk];
-  const int u = blockIdx.z, h = blockIdx.y;
+  const int u = blockIdx.x, h = blockIdx.y;
   const UserSpan us = user_span(a, u);
   if (!us.ok) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && h == 0) flag(a.err, GENRANK_DERR_LAYOUT);
+    if (threadIdx.x == 0 && blockIdx.z == 0 && h == 0) flag(a.err, GENRANK_DERR_LAYOUT);
     return;
   }
-  const int q0 = blockIdx.x * R;
+  const int q0 = blockIdx.z * R;
   if (q0 >= us.L) return;
   const int r = threadIdx.x / G, g = threadIdx.x % G;
   const int i = q0 + r;
@@ -189,13 +189,13 @@ __global__ void __launch_bounds__(128) k_attn_bwd_dq_simt(const __grid_constant_
   __shared__ float sK[kChunk][DH + 1], sV[kChunk][DH + 1];
   __shared__ int sP[kChunk];
   __shared__ long long sT[kChunk];
-  const int u = blockIdx.z, h = blockIdx.y;
+  const int u = blockIdx.x, h = blockIdx.y;
   const UserSpan us = user_span(a, u);
   if (!us.ok) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && h == 0) flag(a.err, GENRANK_DERR_LAYOUT);
+    if (threadIdx.x == 0 && blockIdx.z == 0 && h == 0) flag(a.err, GENRANK_DERR_LAYOUT);
     return;
   }
-  const int q0 = blockIdx.x * R;
+  const int q0 = blockIdx.z * R;
   if (q0 >= us.L) return;
   const int r = threadIdx.x / G, g = threadIdx.x % G;
   const int i = q0 + r;
@@ -291,13 +291,13 @@ __global__ void __launch_bounds__(128) k_attn_bwd_dkv_simt(const __grid_constant
   __shared__ float sL[kChunk], sD[kChunk];
   __shared__ int sP[kChunk];
   __shared__ long long sT[kChunk];
-  const int u = blockIdx.z, h = blockIdx.y;
+  const int u = blockIdx.x, h = blockIdx.y;
   const UserSpan us = user_span(a, u);
   if (!us.ok) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && h == 0) flag(a.err, GENRANK_DERR_LAYOUT);
+    if (threadIdx.x == 0 && blockIdx.z == 0 && h == 0) flag(a.err, GENRANK_DERR_LAYOUT);
     return;
   }
-  const int k0 = blockIdx.x * R;
+  const int k0 = blockIdx.z * R;
   if (k0 >= us.L) return;
   const int r = threadIdx.x / G, g = threadIdx.x % G;
   const int j = k0 + r;
@@ -401,8 +401,11 @@ __global__ void __launch_bounds__(128) k_attn_bwd_dkv_simt(const __grid_constant
 template <typename T, int DH>
 static int fwd_t(const AttnArgs& a, cudaStream_t st) {
   constexpr int R = 128 / (DH / 32);
-  dim3 grid((a.max_seqlen + R - 1) / R, a.H, a.B);
-  if (grid.x == 0) return GENRANK_OK;
+  // users on x (up to 2^31 - 1 of them), heads on y, row blocks on z
+  const int rblocks = (a.max_seqlen + R - 1) / R;
+  if (rblocks == 0) return GENRANK_OK;
+  if (rblocks > 65535) return GENRANK_ERR_UNSUPPORTED;
+  dim3 grid(a.B, a.H, rblocks);
   k_attn_fwd_simt<T, DH><<<grid, 128, 0, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
 }
@@ -428,7 +431,10 @@ static int bwd_t(const AttnArgs& a, cudaStream_t st) {
   const long long nth = a.T * a.H;
   if (nth == 0) return GENRANK_OK;
   k_attn_bwd_dot<T><<<(unsigned)((nth + 255) / 256), 256, 0, st>>>(a, Dw);
-  dim3 grid((a.max_seqlen + R - 1) / R, a.H, a.B);
+  const int rblocks = (a.max_seqlen + R - 1) / R;
+  if (rblocks == 0) return GENRANK_OK;
+  if (rblocks > 65535) return GENRANK_ERR_UNSUPPORTED;
+  dim3 grid(a.B, a.H, rblocks);
   k_attn_bwd_dq_simt<T, DH><<<grid, 128, 0, st>>>(a, Dw);
   k_attn_bwd_dkv_simt<T, DH><<<grid, 128, 0, st>>>(a, Dw);
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;

@@ -16,14 +16,18 @@
 // so the residual stream is read and written once per update and the normalised
 // activations never take a separate pass.
 //
-// Design, one CTA per SM (persistent), 192 threads:
-//   * warp 1 issues TMA loads of 128 x 64 A tiles and BN x 64 Wt tiles (128B swizzle,
-//     no multicast) into a ring of stages;
+// Design, one CTA per SM (persistent), 320 threads:
+//   * warp 1 issues TMA loads of 128 x 64 A tiles and 256 x 64 Wt tiles (128B swizzle,
+//     no multicast) into a four-stage ring (48 KB a stage);
 //   * warp 0 (one thread) issues tcgen05.mma M = 128, N = 256, K = 16 (four per 64-wide
-//     k-step, two side by side for BN = 512) into a TMEM accumulator; the store and SiLU
-//     epilogues double-buffer the accumulator (2 x 256 columns) so a tile's epilogue
-//     overlaps the next tile's MMAs; res+rms uses all 512 columns for one tile;
-//   * warps 2-5 (one accumulator row per thread) run the epilogue from TMEM.
+//     k-step) into a TMEM accumulator.  The store and SiLU epilogues double-buffer the
+//     accumulator (2 x 256 columns) so a tile's epilogue overlaps the next tile's MMAs.
+//     res+rms computes its row (d = 512) as two 256-column halves one after the other,
+//     into columns [0, 256) and [256, 512): the first half's residual pass overlaps the
+//     second half's MMAs;
+//   * warps 2-9 run the epilogue from TMEM, two warps per TMEM lane quadrant (one row
+//     per thread), each on half of a 256-column block; res+rms combines the two warps'
+//     row sums of squares (and head partial sums) through shared memory.
 // Tiles are ordered with the N tiles of one M tile adjacent, so CTAs running them at the
 // same time share the A tile in L2.  Every mbarrier wait is bounded.
 #include <cuda.h>
@@ -37,27 +41,24 @@ namespace gr {
 namespace tg {
 
 constexpr int BM = 128;
+constexpr int BN = 256;  // columns per MMA block (one accumulator buffer)
 constexpr int BK = 64;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kStages = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kIdesc = idesc_bf16_f32(BM, 256, 0, 0);  // A K-major, Wt K-major
-
-template <int kEpi>
-struct Cfg {
-  static constexpr int BN = kEpi == kEpiResRms ? 512 : 256;
-  static constexpr int kStages = kEpi == kEpiResRms ? 2 : 4;
-  static constexpr int kAccBufs = kEpi == kEpiResRms ? 1 : 2;
-  static constexpr uint32_t kABytes = BM * BK * 2;  // 16 KB
-  static constexpr uint32_t kBBytes = BN * BK * 2;  // 32 or 64 KB
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kOffBar = kStages * kStageBytes;
-  // barriers: full[S], empty[S], acc_full[2], acc_empty[2], done
-  static constexpr uint32_t kNumBars = 2 * kStages + 5;
-  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr uint32_t kSmem = kOffMisc + 16 + 1024;
-  static_assert(kSmem <= 227 * 1024, "shared memory");
-  static_assert(kStageBytes % 1024 == 0, "1024-byte aligned stages");
-};
+constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, 0, 0);  // A K-major, Wt K-major
+constexpr uint32_t kABytes = BM * BK * 2;                    // 16 KB
+constexpr uint32_t kBBytes = BN * BK * 2;                    // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kOffRed = kStages * kStageBytes;          // res+rms: [2][BM] partial sums
+constexpr uint32_t kOffBar = kOffRed + 2 * 2 * BM * 4;
+// barriers: full[S], empty[S], acc_full[2], acc_empty[2], done
+constexpr uint32_t kNumBars = 2 * kStages + 5;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmem = kOffMisc + 16 + 1024;
+static_assert(kSmem <= 227 * 1024, "shared memory");
+static_assert(kStageBytes % 1024 == 0, "1024-byte aligned stages");
 
 struct Params {
   CUtensorMap ta, tb;
@@ -71,7 +72,17 @@ GR_DEVICE bool wait_warp(uint64_t* bar, uint32_t ph, volatile int* abort_flag, i
   return __all_sync(0xffffffffu, ok);
 }
 
-GR_DEVICE float silu(float v) { return v / (1.f + __expf(-v)); }
+GR_DEVICE float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// SiLU(v) = v sigmoid(v) = v/2 + (v/2) tanh(v/2): one MUFU operation per element (the
+// result is rounded to bf16, well above the approximation's error)
+GR_DEVICE float silu(float v) {
+  const float h = 0.5f * v;
+  return fmaf(h, tanh_approx(h), h);
+}
 
 // 32 fp32 values to 16 bf16 pairs, stored as four 16-byte vectors at dst.
 GR_DEVICE void store_bf16x32(__nv_bfloat16* dst, const float* v) {
@@ -83,31 +94,40 @@ GR_DEVICE void store_bf16x32(__nv_bfloat16* dst, const float* v) {
                        pack_bf16(v[8 * q + 6], v[8 * q + 7]));
 }
 
+GR_DEVICE void load_f32x32(const float* src, float4 (&x)[8]) {
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) x[e] = s4[e];
+}
+
 template <int kEpi>
 __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__ Params P) {
-  using C = Cfg<kEpi>;
+  constexpr bool kRes = kEpi == kEpiResRms;
+  constexpr int kHalves = kRes ? 2 : 1;  // 256-column blocks per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const GemmArgs& g = P.g;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* full = bars;
-  uint64_t* empty = bars + C::kStages;
-  uint64_t* acc_full = bars + 2 * C::kStages;
+  uint64_t* empty = bars + kStages;
+  uint64_t* acc_full = bars + 2 * kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* done = acc_full + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  // res+rms partial sums: [ss of warp ch 0][ss of ch 1][head of ch 0][head of ch 1], BM each
+  float* red = reinterpret_cast<float*>(smem + kOffRed);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+      mbar_init(&acc_empty[b], kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -126,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int m_tiles = (g.M + BM - 1) / BM;
-  const int n_tiles = g.N / C::BN;
+  const int n_tiles = kRes ? 1 : g.N / BN;
   const int tiles = m_tiles * n_tiles;
   const int ksteps = g.K / BK;
 
@@ -136,59 +156,55 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     bool ok = true;
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
       const int mt = t / n_tiles, nt = t - mt * n_tiles;
-      for (int ks = 0; ks < ksteps; ++ks, ++it) {
-        const int st = it % C::kStages;
-        if (!wait_warp(&empty[st], par(it / C::kStages) ^ 1u, abort_flag, g.err)) {
-          ok = false;
-          break;
-        }
-        if (lane == 0) {
-          uint8_t* sa = smem + st * C::kStageBytes;
-          uint8_t* sb = sa + C::kABytes;
-          mbar_expect_tx(&full[st], C::kStageBytes);
-          tma_load_2d(sa, &P.ta, &full[st], ks * BK, mt * BM);
-#pragma unroll
-          for (int h = 0; h < C::BN / 256; ++h)
-            tma_load_2d(sb + h * (256 * BK * 2), &P.tb, &full[st], ks * BK, nt * C::BN + 256 * h);
+      for (int h = 0; h < kHalves && ok; ++h) {
+        for (int ks = 0; ks < ksteps; ++ks, ++it) {
+          const int st = it % kStages;
+          if (!wait_warp(&empty[st], par(it / kStages) ^ 1u, abort_flag, g.err)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            uint8_t* sa = smem + st * kStageBytes;
+            mbar_expect_tx(&full[st], kStageBytes);
+            tma_load_2d(sa, &P.ta, &full[st], ks * BK, mt * BM);
+            tma_load_2d(sa + kABytes, &P.tb, &full[st], ks * BK, (nt + h) * BN);
+          }
         }
       }
     }
     // the copies issued last land before the CTA exits
     if (lane == 0)
-      for (int x = max(0, it - C::kStages); x < it; ++x)
-        mbar_drain(&full[x % C::kStages], par(x / C::kStages));
+      for (int x = max(0, it - kStages); x < it; ++x) mbar_drain(&full[x % kStages], par(x / kStages));
   } else if (warp == 0) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int it = 0, tc = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
-        const int buf = tc % C::kAccBufs;
-        if (!mbar_wait(&acc_empty[buf], par(tc / C::kAccBufs) ^ 1u, abort_flag, g.err)) break;
+        const int buf = kRes ? 0 : (tc & 1);
+        const uint32_t ph_empty = kRes ? par(tc) ^ 1u : par(tc >> 1) ^ 1u;
+        if (!mbar_wait(&acc_empty[buf], ph_empty, abort_flag, g.err)) break;
         tc_fence_after();
-        const uint32_t acc = tmem + (uint32_t)(buf * 256);
-        for (int ks = 0; ks < ksteps; ++ks, ++it) {
-          const int st = it % C::kStages;
-          if (!mbar_wait(&full[st], par(it / C::kStages), abort_flag, g.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + st * C::kStageBytes);
-          const uint32_t sb = sa + C::kABytes;
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
-#pragma unroll
-            for (int h = 0; h < C::BN / 256; ++h) {
-              const uint64_t bd = smem_desc_sw128(sb + h * (256 * BK * 2) + kk * 32, 16, 1024);
-              mma_bf16_ss(acc + h * 256, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+        for (int h = 0; h < kHalves && ok; ++h) {
+          const uint32_t acc = tmem + (uint32_t)((kRes ? h : buf) * BN);
+          for (int ks = 0; ks < ksteps; ++ks, ++it) {
+            const int st = it % kStages;
+            if (!mbar_wait(&full[st], par(it / kStages), abort_flag, g.err)) {
+              ok = false;
+              break;
             }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + st * kStageBytes);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(sa + kABytes + kk * 32, 16, 1024);
+              mma_bf16_ss(acc, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&empty[st]);  // the stage is free once these MMAs have read it
           }
-          mma_commit(&empty[st]);  // the stage is free once these MMAs have read it
+          if (ok) mma_commit(&acc_full[kRes ? h : buf]);
         }
-        if (!ok) break;
-        mma_commit(&acc_full[buf]);
       }
       // every MMA issued has completed before TMEM is freed
       mma_commit(done);
@@ -196,22 +212,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------------ epilogue warps 2-5
-    const int q = warp & 3;  // TMEM lane quadrant
+    // ------------------------------------------------------------------ epilogue warps 2-9
+    const int q = warp & 3;          // TMEM lane quadrant
+    const int ch = (warp - 2) >> 2;  // which 128 columns of each 256-column block
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
+    const int rloc = q * 32 + lane;  // row within the tile
     int tc = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
       const int mt = t / n_tiles, nt = t - mt * n_tiles;
-      const int buf = tc % C::kAccBufs;
-      if (!wait_warp(&acc_full[buf], par(tc / C::kAccBufs), abort_flag, g.err)) break;
-      tc_fence_after();
-      const long long row = (long long)mt * BM + q * 32 + lane;
+      const long long row = (long long)mt * BM + rloc;
       const bool valid = row < g.M;
-      const uint32_t acc = lane_base + (uint32_t)(buf * 256);
-      if (kEpi != kEpiResRms) {
-        __nv_bfloat16* crow = (__nv_bfloat16*)g.c + row * g.ldc + (long long)nt * C::BN;
+      if (!kRes) {
+        const int buf = tc & 1;
+        if (!wait_warp(&acc_full[buf], par(tc >> 1), abort_flag, g.err)) break;
+        tc_fence_after();
+        const uint32_t acc = lane_base + (uint32_t)(buf * BN + ch * 128);
+        __nv_bfloat16* crow = (__nv_bfloat16*)g.c + row * g.ldc + (long long)nt * BN + ch * 128;
 #pragma unroll 1
-        for (int c = 0; c < C::BN; c += 32) {
+        for (int c = 0; c < 128; c += 32) {
           float v[32];
           tmem_ld32(acc + c, v);
           if (kEpi == kEpiSilu) {
@@ -220,51 +238,78 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
           }
           if (valid) store_bf16x32(crow + c, v);
         }
-      } else {
-        // x_out = x_in + acc over the whole row (d columns), kept in TMEM for the
-        // second pass; then the normalised row and the optional head dot product
-        const float* xin = g.x_in + row * g.ldx;
-        float* xout = g.x_out + row * g.ldx;
-        float ss = 0.f;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        continue;
+      }
+      // res+rms: pass 1 per half as soon as its MMAs are done: y = x_in + acc, kept in
+      // TMEM, written to x_out, its squares summed; then the row's scale and pass 2
+      const float* xin = g.x_in + row * g.ldx;
+      float* xout = g.x_out + row * g.ldx;
+      // A failed (timed-out) wait skips the work but not the named barriers below, so
+      // the other warp of the quadrant never waits for a partner that has left.
+      float ss = 0.f;
+      bool ok = true;
+      for (int h = 0; h < 2 && ok; ++h) {
+        if (!wait_warp(&acc_full[h], par(tc), abort_flag, g.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int c0 = h * BN + ch * 128;
+        float4 xn[8];
+        if (valid) load_f32x32(xin + c0, xn);
 #pragma unroll 1
-        for (int c = 0; c < g.N; c += 32) {
+        for (int c = 0; c < 128; c += 32) {
+          float4 xv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xv[e] = xn[e];
+          if (valid && c + 32 < 128) load_f32x32(xin + c0 + c + 32, xn);  // next chunk in flight
           float v[32];
-          tmem_ld32(acc + c, v);
-          if (valid) {
-            const float4* x4 = reinterpret_cast<const float4*>(xin + c);
-            float4* o4 = reinterpret_cast<float4*>(xout + c);
+          tmem_ld32(lane_base + c0 + c, v);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float4 xv = x4[e];
-              xv.x += v[4 * e];
-              xv.y += v[4 * e + 1];
-              xv.z += v[4 * e + 2];
-              xv.w += v[4 * e + 3];
-              v[4 * e] = xv.x;
-              v[4 * e + 1] = xv.y;
-              v[4 * e + 2] = xv.z;
-              v[4 * e + 3] = xv.w;
-              o4[e] = xv;
-            }
+          for (int e = 0; e < 8; ++e) {
+            xv[e].x += v[4 * e];
+            xv[e].y += v[4 * e + 1];
+            xv[e].z += v[4 * e + 2];
+            xv[e].w += v[4 * e + 3];
+            v[4 * e] = xv[e].x;
+            v[4 * e + 1] = xv[e].y;
+            v[4 * e + 2] = xv[e].z;
+            v[4 * e + 3] = xv[e].w;
           }
+          if (valid) {
+            float4* o4 = reinterpret_cast<float4*>(xout + c0 + c);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ss = fmaf(v[e], v[e], ss);
+            for (int e = 0; e < 8; ++e) o4[e] = xv[e];
+          }
           uint32_t w[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(v[e]);
-          tmem_st32(acc + c, w);
+          for (int e = 0; e < 32; ++e) {
+            ss = fmaf(v[e], v[e], ss);
+            w[e] = __float_as_uint(v[e]);
+          }
+          tmem_st32(lane_base + c0 + c, w);
         }
-        const float r = rsqrtf(ss / (float)g.N + g.eps);
-        float z = 0.f;
+      }
+      // the row's sum of squares over both warps of this quadrant
+      red[ch * BM + rloc] = ss;
+      named_bar_sync(1 + q, 64);
+      const float r = rsqrtf((red[rloc] + red[BM + rloc]) / (float)g.N + g.eps);
+      float z = 0.f;
+      for (int h = 0; h < 2 && ok; ++h) {
+        const int c0 = h * BN + ch * 128;
 #pragma unroll 1
-        for (int c = 0; c < g.N; c += 32) {
+        for (int c = 0; c < 128; c += 32) {
           float v[32];
-          tmem_ld32(acc + c, v);
+          tmem_ld32(lane_base + c0 + c, v);
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] *= r;
-          if (valid && g.a_out) store_bf16x32((__nv_bfloat16*)g.a_out + row * g.lda_out + c, v);
+          if (valid && g.a_out)
+            store_bf16x32((__nv_bfloat16*)g.a_out + row * g.lda_out + c0 + c, v);
           if (g.w_head) {
-            const float4* w4 = reinterpret_cast<const float4*>(g.w_head + c);
+            const float4* w4 = reinterpret_cast<const float4*>(g.w_head + c0 + c);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const float4 wv = w4[e];
@@ -275,11 +320,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
             }
           }
         }
-        if (valid && g.w_head) g.z[row] = z;
       }
+      if (g.w_head) {
+        red[2 * BM + ch * BM + rloc] = z;
+        named_bar_sync(1 + q, 64);
+        if (ch == 0 && valid) g.z[row] = red[2 * BM + rloc] + red[3 * BM + rloc];
+      }
+      // the partial-sum slots are reused by the next tile only after both warps of the
+      // quadrant have read them
+      named_bar_sync(1 + q, 64);
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (lane == 0) mbar_arrive(&acc_empty[0]);
     }
   }
 
@@ -364,18 +417,18 @@ static DeviceOnce gemm_smem_attr[3];
 
 template <int kEpi>
 static int launch_t(const GemmArgs& g, cudaStream_t st) {
-  using C = Cfg<kEpi>;
   Params p;
-  if (!make_map(&p.ta, g.a, g.M, g.K, g.lda, BM) || !make_map(&p.tb, g.w, g.N, g.K, g.ldw, 256))
+  if (!make_map(&p.ta, g.a, g.M, g.K, g.lda, BM) || !make_map(&p.tb, g.w, g.N, g.K, g.ldw, BN))
     return GENRANK_ERR_CUDA;
   p.g = g;
-  if (!set_smem_limit_once(gemm_smem_attr[kEpi], (const void*)k_gemm_tc<kEpi>, (int)C::kSmem))
+  if (!set_smem_limit_once(gemm_smem_attr[kEpi], (const void*)k_gemm_tc<kEpi>, (int)kSmem))
     return GENRANK_ERR_CUDA;
   const int sms = sm_count_current();
   if (sms <= 0) return GENRANK_ERR_CUDA;
-  const long long tiles = (long long)((g.M + BM - 1) / BM) * (g.N / C::BN);
+  const long long tiles =
+      (long long)((g.M + BM - 1) / BM) * (kEpi == kEpiResRms ? 1 : g.N / BN);
   const int grid = (int)(tiles < sms ? tiles : sms);
-  k_gemm_tc<kEpi><<<grid, kThreads, C::kSmem, st>>>(p);
+  k_gemm_tc<kEpi><<<grid, kThreads, kSmem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
 }
 

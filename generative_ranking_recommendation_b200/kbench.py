@@ -1,7 +1,7 @@
 """Per-kernel benchmark of the hot path on one workload configuration.
 
     python -m generative_ranking_recommendation_b200.kbench --config c2 \
-        [--kernels embed_fwd,attn_fwd,attn_bwd,embed_bwd] [--iters 20] [--warmup 3]
+        [--kernels embed_fwd,attn_fwd,attn_bwd,embed_bwd,linear] [--iters 20] [--warmup 3]
 
 Times each library call with CUDA events around a replay of the call captured as
 a CUDA graph (inputs resident in HBM, L2 flushed before every timed replay) and prints one JSON line per kernel with its
@@ -168,6 +168,47 @@ def main(argv=None):
             fl = 10.0 * d * pairs
             print(json.dumps({**base, "kernel": "attn_bwd", "ms": ms, "TFLOP_per_s": fl / ms / 1e9,
                               "algorithmic_flops": fl, "visible_pairs": pairs}), flush=True)
+    if "linear" in kernels:
+        # the four-layer block's linear layers at this workload's token count, on the
+        # library's fused tensor-core kernels and, for comparison, as torch ops (cuBLAS
+        # GEMM + elementwise kernels); 2 M N K flops per GEMM
+        gg = torch.Generator(device=dev)
+        gg.manual_seed(7)
+        bf = torch.bfloat16
+        a = torch.randn((T, d), device=dev, generator=gg).to(bf)
+        wqkv = (torch.randn((3 * d, d), device=dev, generator=gg) / math.sqrt(d)).to(bf)
+        wo = (torch.randn((d, d), device=dev, generator=gg) / math.sqrt(d)).to(bf)
+        w1 = (torch.randn((4 * d, d), device=dev, generator=gg) / math.sqrt(d)).to(bf)
+        w2 = (torch.randn((d, 4 * d), device=dev, generator=gg) / math.sqrt(4 * d)).to(bf)
+        x = torch.randn((T, d), device=dev, generator=gg)
+        u = torch.randn((T, 4 * d), device=dev, generator=gg).to(bf)
+        out3 = torch.empty((T, 3 * d), dtype=bf, device=dev)
+        out4 = torch.empty((T, 4 * d), dtype=bf, device=dev)
+        a2 = torch.empty((T, d), dtype=bf, device=dev)
+
+        def rms(v):
+            return v * torch.rsqrt((v * v).mean(dim=-1, keepdim=True) + 1e-6)
+
+        cases = [
+            ("qkv", 3 * d, d, lambda: G.linear(a, wqkv, out3, err),
+             lambda: a @ wqkv.t()),
+            ("w1_silu", 4 * d, d, lambda: G.linear(a, w1, out4, err, epilogue=G.EPI_SILU),
+             lambda: torch.nn.functional.silu(a @ w1.t())),
+            ("wo_res_rms", d, d, lambda: G.linear_residual_rmsnorm(a, wo, x, x, a2, err),
+             lambda: rms(x + (a @ wo.t()).float()).to(bf)),
+            ("w2_res_rms", d, 4 * d, lambda: G.linear_residual_rmsnorm(u, w2, x, x, a2, err),
+             lambda: rms(x + (u @ w2.t()).float()).to(bf)),
+        ]
+        for name, N, K, ours, theirs in cases:
+            if d != 512 and name.endswith("res_rms"):
+                continue
+            fl = 2.0 * T * N * K
+            ms = timed(ours, args.iters, args.warmup, flush)
+            ms_t = timed(theirs, args.iters, args.warmup, flush)
+            print(json.dumps({**base, "kernel": f"linear_{name}", "ms": ms,
+                              "TFLOP_per_s": fl / ms / 1e9, "torch_ms": ms_t,
+                              "torch_TFLOP_per_s": fl / ms_t / 1e9, "M": T, "N": N, "K": K}),
+                  flush=True)
     code = G.check_error(err)
     if code:
         raise SystemExit(f"device error flags: {code}")

@@ -1,7 +1,8 @@
 """Per-kernel benchmark of the hot path on one workload configuration.
 
     python -m generative_ranking_recommendation_b200.kbench --config c2 \
-        [--kernels embed_fwd,attn_fwd,attn_bwd,embed_bwd,linear] [--iters 20] [--warmup 3]
+        [--kernels embed_fwd,attn_fwd,attn_bwd,embed_bwd,linear,bucketed,cached,hstu]
+        [--iters 20] [--warmup 3] [--users B]
 
 Times each library call with CUDA events around a replay of the call captured as
 a CUDA graph (inputs resident in HBM, L2 flushed before every timed replay) and prints one JSON line per kernel with its
@@ -80,8 +81,11 @@ def main(argv=None):
     ap.add_argument("--kernels", default="embed_fwd,attn_fwd,attn_bwd,embed_bwd")
     ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--users", type=int, default=None, help="batch size (default: the config's)")
     args = ap.parse_args(argv)
     cfg = CONFIGS[args.config]
+    if args.users:
+        cfg = cfg.with_(B=args.users)
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     batch = make_batch(cfg)
@@ -168,6 +172,126 @@ def main(argv=None):
             fl = 10.0 * d * pairs
             print(json.dumps({**base, "kernel": "attn_bwd", "ms": ms, "TFLOP_per_s": fl / ms / 1e9,
                               "algorithmic_flops": fl, "visible_pairs": pairs}), flush=True)
+    if "bucketed" in kernels:
+        # the bucketed time bias against the linear one on the same operands
+        g = torch.Generator(device=dev)
+        g.manual_seed(cfg.seed)
+        qkv = torch.randn((T, 3 * d), device=dev, generator=g).to(tdt)
+        do = torch.randn((T, d), device=dev, generator=g).to(tdt)
+        o = torch.empty((T, d), dtype=tdt, device=dev)
+        lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+        dqkv = torch.empty_like(qkv)
+        wsf = torch.empty(G.attn_workspace_size(batch.B, T, H, dh, msl, False), dtype=torch.uint8,
+                          device=dev)
+        wsb = torch.empty(G.attn_workspace_size(batch.B, T, H, dh, msl, True), dtype=torch.uint8,
+                          device=dev)
+        for bucketed in (False, True):
+            slope_t = sp if bucketed else st
+
+            def ff():
+                G.attn_fwd(off, hl, msl, qkv, qkv[:, d:], qkv[:, 2 * d:], 3 * d, H, dh, pos, ts,
+                           sp, slope_t, scale, o, d, lse, wsf, err, T=T, bucketed=bucketed)
+
+            def fb():
+                G.attn_bwd(off, hl, msl, qkv, qkv[:, d:], qkv[:, 2 * d:], 3 * d, H, dh, pos, ts,
+                           sp, slope_t, scale, o, do, d, lse, dqkv, dqkv[:, d:], dqkv[:, 2 * d:],
+                           wsb, err, T=T, bucketed=bucketed)
+
+            ms_f = timed(ff, args.iters, args.warmup, flush)
+            ff()
+            ms_b = timed(fb, args.iters, args.warmup, flush)
+            tag = "bucketed" if bucketed else "linear"
+            print(json.dumps({**base, "kernel": f"attn_{tag}", "fwd_ms": ms_f,
+                              "fwd_TFLOP_per_s": 4.0 * d * pairs / ms_f / 1e9, "bwd_ms": ms_b,
+                              "bwd_TFLOP_per_s": 10.0 * d * pairs / ms_b / 1e9}), flush=True)
+
+    if "cached" in kernels:
+        # candidates scored against a history K/V cache, against the full attention over
+        # history + candidates (whose candidate rows it equals)
+        g = torch.Generator(device=dev)
+        g.manual_seed(cfg.seed)
+        qkv = torch.randn((T, 3 * d), device=dev, generator=g).to(tdt)
+        n_u = batch.hist_len.astype(np.int64)
+        hist_rows = np.concatenate([np.arange(batch.seq_offsets[u], batch.seq_offsets[u] + n_u[u])
+                                    for u in range(batch.B)])
+        cand_rows = np.concatenate([np.arange(batch.seq_offsets[u] + n_u[u], batch.seq_offsets[u + 1])
+                                    for u in range(batch.B)])
+        hr = torch.from_numpy(hist_rows).to(dev)
+        cr = torch.from_numpy(cand_rows).to(dev)
+        kv = qkv[:, d:].index_select(0, hr).contiguous()  # [Th, 2d]
+        qc = qkv.index_select(0, cr).contiguous()          # [C, 3d]
+        C, Th = int(cr.numel()), int(hr.numel())
+        hoff = torch.from_numpy(np.concatenate([[0], np.cumsum(n_u)]).astype(np.int32)).to(dev)
+        m_u = np.diff(batch.seq_offsets).astype(np.int64) - n_u
+        coff = torch.from_numpy(np.concatenate([[0], np.cumsum(m_u)]).astype(np.int32)).to(dev)
+        pos_h = pos.index_select(0, hr).contiguous()
+        ts_h, ts_c = ts.index_select(0, hr).contiguous(), ts.index_select(0, cr).contiguous()
+        oc = torch.empty((C, d), dtype=tdt, device=dev)
+        of = torch.empty((T, d), dtype=tdt, device=dev)
+        m_max = int(m_u.max())
+        wsc = torch.empty(G.attn_cached_workspace_size(batch.B, C, Th, H, dh, m_max),
+                          dtype=torch.uint8, device=dev)
+        wsf = torch.empty(G.attn_workspace_size(batch.B, T, H, dh, msl, False), dtype=torch.uint8,
+                          device=dev)
+
+        def fc():
+            G.attn_fwd_cached(coff, m_max, qc, qc[:, d:], qc[:, 2 * d:], 3 * d, hoff, kv,
+                              kv[:, d:], 2 * d, pos_h, ts_h, ts_c, H, dh, sp, st, scale, oc, d,
+                              None, wsc, err, C=C, Th=Th)
+
+        def ffull():
+            G.attn_fwd(off, hl, msl, qkv, qkv[:, d:], qkv[:, 2 * d:], 3 * d, H, dh, pos, ts, sp,
+                       st, scale, of, d, None, wsf, err, T=T)
+
+        cand_pairs = int(np.sum(m_u * n_u + m_u))
+        ms_c = timed(fc, args.iters, args.warmup, flush)
+        ms_f = timed(ffull, args.iters, args.warmup, flush)
+        print(json.dumps({**base, "kernel": "attn_cached", "ms": ms_c, "full_ms": ms_f,
+                          "candidates": C, "candidates_per_s": C / ms_c * 1e3,
+                          "TFLOP_per_s": 4.0 * d * cand_pairs / ms_c / 1e9,
+                          "speedup_vs_full": ms_f / ms_c}), flush=True)
+
+    if "hstu" in kernels:
+        # the interleaved layout (2n + m tokens) with a dense N x N bias read from HBM,
+        # against the action-oriented layout (n + m tokens) with the ALiBi terms computed
+        # on the fly, both on the same tensor-core attention kernel
+        from gen import dense_bias_torch, interleave_batch
+
+        ib = interleave_batch(batch)
+        Ti = ib.T
+        msl_i = int(np.max(np.diff(ib.seq_offsets)))
+        Lpad = (msl_i + 127) // 128 * 128
+        bias = dense_bias_torch(cfg.seed, ib.B, Lpad, dev)
+        g = torch.Generator(device=dev)
+        g.manual_seed(cfg.seed)
+        qkv_i = torch.randn((Ti, 3 * d), device=dev, generator=g).to(tdt)
+        qkv = torch.randn((T, 3 * d), device=dev, generator=g).to(tdt)
+        o_i = torch.empty((Ti, d), dtype=tdt, device=dev)
+        o = torch.empty((T, d), dtype=tdt, device=dev)
+        off_i = torch.from_numpy(ib.seq_offsets).to(dev)
+        hl_i = torch.from_numpy(ib.hist_len).to(dev)
+        ws_i = torch.empty(G.attn_workspace_size(ib.B, Ti, H, dh, msl_i, False),
+                           dtype=torch.uint8, device=dev)
+        ws = torch.empty(G.attn_workspace_size(batch.B, T, H, dh, msl, False), dtype=torch.uint8,
+                         device=dev)
+
+        def fh():
+            G.attn_fwd_dense_bias(off_i, hl_i, msl_i, qkv_i, qkv_i[:, d:], qkv_i[:, 2 * d:],
+                                  3 * d, H, dh, bias, scale, o_i, d, None, ws_i, err, T=Ti)
+
+        def fg():
+            G.attn_fwd(off, hl, msl, qkv, qkv[:, d:], qkv[:, 2 * d:], 3 * d, H, dh, pos, ts, sp,
+                       st, scale, o, d, None, ws, err, T=T)
+
+        ms_h = timed(fh, args.iters, args.warmup, flush)
+        ms_g = timed(fg, args.iters, args.warmup, flush)
+        pairs_i = visible_pairs(ib.seq_offsets, ib.hist_len)
+        print(json.dumps({**base, "kernel": "attn_hstu_shaped", "interleaved_ms": ms_h,
+                          "interleaved_tokens": Ti, "interleaved_pairs": pairs_i,
+                          "bias_bytes": int(bias.numel() * 2), "action_oriented_ms": ms_g,
+                          "action_oriented_tokens": T, "action_oriented_pairs": pairs,
+                          "time_ratio": ms_g / ms_h, "pair_ratio": pairs / pairs_i}), flush=True)
+
     if "linear" in kernels:
         # the four-layer block's linear layers at this workload's token count, on the
         # library's fused tensor-core kernels and, for comparison, as torch ops (cuBLAS

@@ -105,41 +105,73 @@ def attn_bwd(q, k, v, dO, batch, pos, users=None):
                                 sp, st, 1.0 / math.sqrt(dh), users=users)
 
 
-def dq_noise_floor(k, dO, O, seq_offsets, scale):
-    """Per (token, head) absolute error of dq that the bf16 path carries by construction.
-
-    dq_i = scale sum_j P_ij (dP_ij - D_i) k_j with D_i = rowsum(dO_i * O_i) taken from O
-    as stored in bf16: O's rounding (relative 2^-9 per element) moves D_i by up to
-    2^-9 sum_e |dO_ie O_ie|, and that shift reaches dq_i as scale * dD_i * sum_j P_ij k_j,
-    at most scale * |dD_i| * max_j |k_j| (the P_ij sum to 1).  Rows whose dP_ij - D_i
-    nearly cancel (one dominant key, e.g. a user's first tokens) have dq far below that
-    size, so a per-row relative bound alone cannot hold there.  Returned with a factor 4
-    of slack (2^-7) for the other bf16 roundings on the path."""
-    k = np.asarray(k, np.float64)
-    T, H, _ = k.shape
-    out = np.zeros((T, H))
-    dd = (np.abs(np.asarray(dO, np.float64)) * np.abs(np.asarray(O, np.float64))).sum(-1)
-    for u in range(len(seq_offsets) - 1):
-        s, e = int(seq_offsets[u]), int(seq_offsets[u + 1])
-        if e > s:
-            kmax = np.abs(k[s:e]).max(axis=(0, 2))  # per head
-            out[s:e] = scale * 2.0 ** -7 * dd[s:e] * kmax[None, :]
-    return out
+def attention_probs(fwd, q, k, batch, pos, u):
+    """The oracle's attention probabilities P[i, h, j] of user u, read off its forward
+    with one-hot values (v_j = e_j gives O_i = sum_j P_ij e_j = P_i).  ``fwd(q, k, v,
+    seq_offsets, hist_len, pos, ts)`` is an oracle forward (linear or bucketed bias)."""
+    sub = sub_batch(batch, [u])
+    rows = user_rows(batch, [u])
+    L, H, dh = len(rows), q.shape[1], q.shape[2]
+    P = np.zeros((L, H, L))
+    for c0 in range(0, L, dh):  # dh one-hot value columns per call
+        c1 = min(L, c0 + dh)
+        v = np.zeros((L, H, dh))
+        for h in range(H):
+            v[c0:c1, h, :c1 - c0] = np.eye(c1 - c0)
+        O, _ = fwd(q[rows], k[rows], v, sub.seq_offsets, sub.hist_len, np.asarray(pos)[rows],
+                   sub.ts)
+        P[:, :, c0:c1] = O[:, :, :c1 - c0]
+    return P
 
 
-def check_rows(got, want, tol, name, floor=None, noise=None):
+def grad_noise_floors(fwd, q, k, v, dO, O, batch, pos, users, scale):
+    """Per (token, head) absolute errors that the bf16 backward carries by construction,
+    for dq, dk and dv.
+
+    With P from the oracle, dP = dO V^T and D_i = rowsum(dO_i * O_i):
+      * D_i is formed from O as the forward wrote it: P rounded to bf16 before P V and O
+        rounded to bf16, each element off by up to 2^-9 (|O_ie| + sum_j P_ij |v_je|), which
+        moves D_i by up to 2^-9 sum_e |dO_ie| (|O_ie| + (P |V|)_ie);
+      * dS_ij = P_ij (dP_ij - D_i) is rounded to bf16 once (2^-9 of |dS_ij|);
+      * P is rounded to bf16 for dV = P^T dO.
+    So |ddq_i| <= scale max|k| sum_j E_ij, |ddk_j| <= scale max|q| sum_i E_ij with
+    E_ij = P_ij 2^-9 (sum_e |dO_ie| (|O_ie| + (P |V|)_ie) + |dP_ij - D_i|), and |ddv_j| <= 2^-9
+    max|dO| sum_i P_ij.  Rows whose terms nearly cancel (a user's first tokens; keys
+    seen by few queries) have gradients far below these sums, where a per-row relative
+    bound alone cannot hold.  Returned with a factor 4 of slack (2^-7 for 2^-9)."""
+    q, k, v, dO, O = (np.asarray(x, np.float64) for x in (q, k, v, dO, O))
+    T, H, _ = q.shape
+    nq, nk, nv = np.zeros((T, H)), np.zeros((T, H)), np.zeros((T, H))
+    for u in users:
+        rows = user_rows(batch, [u])
+        if len(rows) == 0:
+            continue
+        P = attention_probs(fwd, q, k, batch, pos, u)
+        for h in range(H):
+            Ph = P[:, h, :]
+            g, vv, oo = dO[rows, h], v[rows, h], O[rows, h]
+            dP = g @ vv.T
+            D = (g * oo).sum(-1)
+            A = (np.abs(g) * (np.abs(oo) + Ph @ np.abs(vv))).sum(-1)
+            E = Ph * (A[:, None] + np.abs(dP - D[:, None])) * 2.0 ** -7
+            nq[rows, h] = scale * np.abs(k[rows, h]).max() * E.sum(axis=1)
+            nk[rows, h] = scale * np.abs(q[rows, h]).max() * E.sum(axis=0)
+            nv[rows, h] = 2.0 ** -7 * np.abs(g).max() * Ph.sum(axis=0)
+    return nq, nk, nv
+
+
+def check_rows(got, want, tol, name, floor_frac=1.0 / 16.0, noise=None):
     """Relative-to-max bound, and a per-token bound over all heads: each row's error
-    within tol of max(its own magnitude, the tensor's max / 16), plus an optional
-    absolute per (token, head) noise allowance ``noise``."""
+    within tol of max(its own magnitude, floor_frac * the tensor's max), plus an
+    optional absolute per (token, head) noise allowance ``noise``."""
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)
     assert rel_to_max(got, want) <= tol, name
     err = np.abs(got - want).max(axis=-1)  # [rows, H]
     mag = np.abs(want).max(axis=-1)
     gmax = np.abs(want).max()
-    allow = tol * np.maximum(mag.max(axis=1, keepdims=True), gmax / 16.0 if floor is None else floor)
-    if noise is not None:
-        allow = allow + noise
+    allow = tol * np.maximum(mag.max(axis=1, keepdims=True), floor_frac * gmax)
+    allow = np.broadcast_to(allow + (0.0 if noise is None else noise), err.shape)
     bad = err > allow
     if bad.any():
         r, h = np.argwhere(bad)[0]

@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import ref
 from gen import CONFIGS, make_batch, make_qkv
 
@@ -230,20 +231,26 @@ def run_bwd(G, cfg, batch, pos, qkv, dO, poison=False):
 def _check_grads(cfg, got, want, rows, qkv=None, dO=None, batch=None, pos=None, users=None):
     """fp32: max-abs bound.  bf16: relative to the max, plus a per-token bound over all
     heads (so that one wrong row, a candidate's dk/dv or a short user's dq, cannot hide
-    behind the tensor's max): 2e-2 of max(the row's magnitude, 1/8 of the tensor's max),
-    and for dq the noise floor that the bf16 O carries into D_i (``ref.dq_noise_floor``,
-    from the oracle's O)."""
-    noise = None
+    behind the tensor's max): each row within 2e-2 of max(its magnitude, 1/16 of the
+    tensor's max) plus the absolute error the bf16 path carries by construction
+    (``ref.grad_noise_floors``, from the oracle's probabilities and O)."""
+    noise = (None, None, None)
     if cfg.dtype != "f32" and qkv is not None:
+        sp, st = ref.slopes(cfg.H)
+        scale = 1.0 / math.sqrt(cfg.dh)
+
+        def fwd(q, k, v, offs, hl, p, ts):
+            return oracle.attention_fwd(q, k, v, offs, hl, p, ts, sp, st, scale)
+
+        us = range(batch.B) if users is None else users
         O, _ = ref.attn(qkv[:, 0], qkv[:, 1], qkv[:, 2], batch, pos, users=users)
-        noise = ref.dq_noise_floor(qkv[:, 1], dO, O, batch.seq_offsets,
-                                   1.0 / math.sqrt(cfg.dh))[rows]
-    for name, a, b in zip(("dq", "dk", "dv"), got, want):
+        noise = tuple(x[rows] for x in ref.grad_noise_floors(
+            fwd, qkv[:, 0], qkv[:, 1], qkv[:, 2], dO, O, batch, pos, us, scale))
+    for name, a, b, nz in zip(("dq", "dk", "dv"), got, want, noise):
         if cfg.dtype == "f32":
             assert np.max(np.abs(a[rows] - b[rows])) <= F32_TOL, name
         else:
-            ref.check_rows(a[rows], b[rows], BF16_TOL, name, floor_frac=1.0 / 8.0,
-                           noise=noise if name == "dq" else None)
+            ref.check_rows(a[rows], b[rows], BF16_TOL, name, noise=nz)
 
 
 @pytest.mark.parametrize("name,B", [("c0", None), ("c3", 6)])

@@ -73,10 +73,21 @@ def run(G, cfg, batch, pos, qkv, dO=None, bucketed=True, slope_scale=1.0):
 
 
 def _rel_rows(a, b, name, noise=None):
-    """Relative to the max plus the per-token bound; for dq the noise floor the bf16 O
-    carries into D_i (see ref.dq_noise_floor)."""
-    ref.check_rows(a, b, BF16_TOL, name, floor_frac=1.0 / 8.0 if name != "O" else 1.0 / 16.0,
-                   noise=noise)
+    """Relative to the max plus the per-token bound, with the gradients' noise floors
+    (see ref.grad_noise_floors)."""
+    ref.check_rows(a, b, BF16_TOL, name, noise=noise)
+
+
+def _noise(batch, pos, qkv, dO, O, H, dh, users=None, slope_scale=1.0):
+    sp = oracle.alibi_slopes(H) * slope_scale
+    scale = 1.0 / math.sqrt(dh)
+
+    def fwd(q, k, v, offs, hl, p, ts):
+        return oracle.attention_fwd_bucketed(q, k, v, offs, hl, p, ts, sp, sp, scale)
+
+    us = range(batch.B) if users is None else users
+    return ref.grad_noise_floors(fwd, qkv[:, 0], qkv[:, 1], qkv[:, 2], dO, O, batch, pos, us,
+                                 scale)
 
 
 def _boundary_batch(cfg):
@@ -115,9 +126,9 @@ def test_bucketed_fwd_bwd_parity(G, slope_scale):
     want = _oracle(batch, pos, qkv, cfg.H, cfg.dh, dO, slope_scale=slope_scale)
     _rel_rows(got[0], want[0], "O")
     assert np.max(np.abs(got[1] - want[1])) <= 2e-2
-    noise = ref.dq_noise_floor(qkv[:, 1], dO, want[0], batch.seq_offsets, 1.0 / math.sqrt(cfg.dh))
+    noise = _noise(batch, pos, qkv, dO, want[0], cfg.H, cfg.dh, slope_scale=slope_scale)
     for k, name in zip(range(2, 5), ("dq", "dk", "dv")):
-        _rel_rows(got[k], want[k], name, noise if name == "dq" else None)
+        _rel_rows(got[k], want[k], name, noise[k - 2])
 
 
 def test_bucketed_parity_random_users(G):
@@ -131,9 +142,9 @@ def test_bucketed_parity_random_users(G):
     want = _oracle(batch, pos, qkv, cfg.H, cfg.dh, dO)
     _rel_rows(got[0], want[0], "O")
     assert np.max(np.abs(got[1] - want[1])) <= 2e-2
-    noise = ref.dq_noise_floor(qkv[:, 1], dO, want[0], batch.seq_offsets, 1.0 / math.sqrt(cfg.dh))
+    noise = _noise(batch, pos, qkv, dO, want[0], cfg.H, cfg.dh, slope_scale=1.0)
     for k, name in zip(range(2, 5), ("dq", "dk", "dv")):
-        _rel_rows(got[k], want[k], name, noise if name == "dq" else None)
+        _rel_rows(got[k], want[k], name, noise[k - 2])
 
 
 def test_one_request_per_user_equals_linear_bias_bitwise(G):
@@ -177,6 +188,6 @@ def test_bucketed_full_size_c3_sampled(G):
     rows = ref.user_rows(batch, users)
     _rel_rows(got[0][rows], O[rows], "O")
     assert np.max(np.abs(got[1][:, rows] - L[:, rows])) <= 2e-2
-    noise = ref.dq_noise_floor(qkv[:, 1], dO, O, batch.seq_offsets, 1.0 / math.sqrt(cfg.dh))
+    noise = _noise(batch, pos, qkv, dO, O, cfg.H, cfg.dh, users=users)
     for k, (name, w) in enumerate((("dq", dq), ("dk", dk), ("dv", dv))):
-        _rel_rows(got[2 + k][rows], w[rows], name, noise[rows] if name == "dq" else None)
+        _rel_rows(got[2 + k][rows], w[rows], name, noise[k][rows])

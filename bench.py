@@ -588,10 +588,11 @@ def run_native(args, cfg, world, rank, local):
     hbm = float(peaks["hbm_gbs"])
     burst_src = f"{src} bf16 (burst, cuBLAS GEMM)"
     kernels = []
+    if rank == 0 and training:  # the training step's roofline is the attention backward
+        kernels.append(_attention_kernel_line(torch, G, timer, cfg, args.steps, True,
+                                              peak_burst, burst_src, dev))
     if rank == 0 and not args.no_extra_kernels:
         if training:
-            kernels.append(_attention_kernel_line(torch, G, timer, cfg, args.steps, True,
-                                                  peak_burst, burst_src, dev))
             kernels.append(_attention_kernel_line(torch, G, timer, cfg, args.steps, False,
                                                   peak_burst, burst_src, dev))
         else:

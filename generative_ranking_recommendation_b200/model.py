@@ -104,8 +104,11 @@ class GenRankModel:
         # layers (bf16; widths the tiles divide), the four-layer block with the fused
         # residual + RMSNorm epilogues (d = 512); otherwise the blocks are torch ops
         d = cfg.d
-        self.fused_qkv = cfg.dtype == "bf16" and (3 * d) % 256 == 0 and d % 64 == 0
-        self.fused_blocks = self.fused_qkv and cfg.ffn and d == 512
+        self.fused_blocks = (cfg.dtype == "bf16" and cfg.ffn and d == 512)
+        # a lone QKV projection (the one-block workloads) stays on cuBLAS, which is
+        # faster than the library's plain-store GEMM at these shapes; set True to use
+        # the library's linear layer for it too
+        self.fused_qkv = False
 
     # -------------------------------------------------------------------------------------
     def workspace(self, db: DeviceBatch, bwd: bool) -> torch.Tensor:

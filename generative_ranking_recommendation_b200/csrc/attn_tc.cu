@@ -441,6 +441,26 @@ struct TB {
   GR_DEVICE TB at(int off) const { return TB{tr + off, ti_m, nmt2}; }
 };
 
+// The dense bias of one softmax thread's 64 key columns: the first 32 columns' bf16
+// pairs, loaded before the wait for S (which also brings the row's 128-byte line into
+// L1), and the row in global memory, from which the other 32 columns are loaded when
+// that half of the tile starts.  Keeping 16 words live instead of 32 avoids spilling.
+struct DB {
+  const uint32_t* w0;
+  const uint4* src;
+};
+
+GR_DEVICE void load_bias16(const uint4* src, uint32_t (&w)[16]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 v = __ldg(src + c);
+    w[4 * c] = v.x;
+    w[4 * c + 1] = v.y;
+    w[4 * c + 2] = v.z;
+    w[4 * c + 3] = v.w;
+  }
+}
+
 // bucket(t_i - t_j) of four consecutive keys, as two pairs of floats (see kTimeMagic).
 GR_DEVICE void buckets4(const TB& tb, int c, uint64_t& b01, uint64_t& b23) {
   const int4 t = *reinterpret_cast<const int4*>(tb.tr + c);
@@ -549,21 +569,32 @@ GR_DEVICE void exp_pack_store(const uint32_t (&s)[CW], const float* cb, const TB
 // Maximum of x over this thread's half of the tile (S at s_addr, column terms of the
 // half at cb, first key kbase), CW columns at a time with the next chunk's load in flight.
 template <bool kMasked, bool kBucket, bool kDense>
-GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, const TB& tb, const uint32_t* bw,
+GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, const TB& tb, const DB& db,
                          int kbase, int nvalid, float scale_log2) {
   float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   uint32_t xa[CW], xb[CW];
+  uint32_t w1[kDense ? 16 : 1];
   s_load(s_addr, xa);
   tmem_ld_wait(xa);
 #pragma unroll
   for (int c0 = 0; c0 < kHalf; c0 += 2 * CW) {
+    const uint32_t* bw = nullptr;
+    if constexpr (kDense) {
+      if (c0 == 0) {
+        bw = db.w0;
+      } else {
+        load_bias16(db.src + 4, w1);
+        bw = w1;
+      }
+    }
     s_load(s_addr + c0 + CW, xb);
-    row_max_chunk<kMasked, kBucket, kDense>(xa, cb + c0, tb.at(c0), bw + c0 / 2, kbase + c0,
-                                            nvalid, scale_log2, mx4);
+    row_max_chunk<kMasked, kBucket, kDense>(xa, cb + c0, tb.at(c0), bw, kbase + c0, nvalid,
+                                            scale_log2, mx4);
     tmem_ld_wait(xb);
     if (c0 + 2 * CW < kHalf) s_load(s_addr + c0 + 2 * CW, xa);
-    row_max_chunk<kMasked, kBucket, kDense>(xb, cb + c0 + CW, tb.at(c0 + CW), bw + (c0 + CW) / 2,
-                                            kbase + c0 + CW, nvalid, scale_log2, mx4);
+    row_max_chunk<kMasked, kBucket, kDense>(xb, cb + c0 + CW, tb.at(c0 + CW),
+                                            kDense ? bw + CW / 2 : bw, kbase + c0 + CW, nvalid,
+                                            scale_log2, mx4);
     if (c0 + 2 * CW < kHalf) tmem_ld_wait(xa);
   }
   return fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
@@ -573,21 +604,31 @@ GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, const TB& tb, const u
 // columns at p_addr; the stores have landed when it returns.  Returns the half's sum.
 template <bool kMasked, bool kBucket, bool kDense>
 GR_DEVICE float tile_exp(uint32_t s_addr, uint32_t p_addr, const float* cb, const TB& tb,
-                         const uint32_t* bw, int kbase, int nvalid, float scale_log2, float m) {
+                         const DB& db, int kbase, int nvalid, float scale_log2, float m) {
   uint64_t rs2[2] = {0ull, 0ull};  // (+0, +0) pairs
   uint32_t xa[CW], xb[CW];
+  uint32_t w1[kDense ? 16 : 1];
   s_load(s_addr, xa);
   tmem_ld_wait(xa);
 #pragma unroll
   for (int c0 = 0; c0 < kHalf; c0 += 2 * CW) {
+    const uint32_t* bw = nullptr;
+    if constexpr (kDense) {
+      if (c0 == 0) {
+        bw = db.w0;
+      } else {
+        load_bias16(db.src + 4, w1);
+        bw = w1;
+      }
+    }
     s_load(s_addr + c0 + CW, xb);
-    exp_pack_store<kMasked, kBucket, kDense>(xa, cb + c0, tb.at(c0), bw + c0 / 2, kbase + c0,
-                                             nvalid, scale_log2, m, rs2, p_addr + c0 / 2);
+    exp_pack_store<kMasked, kBucket, kDense>(xa, cb + c0, tb.at(c0), bw, kbase + c0, nvalid,
+                                             scale_log2, m, rs2, p_addr + c0 / 2);
     tmem_ld_wait(xb);
     if (c0 + 2 * CW < kHalf) s_load(s_addr + c0 + 2 * CW, xa);
-    exp_pack_store<kMasked, kBucket, kDense>(xb, cb + c0 + CW, tb.at(c0 + CW), bw + (c0 + CW) / 2,
-                                             kbase + c0 + CW, nvalid, scale_log2, m, rs2,
-                                             p_addr + (c0 + CW) / 2);
+    exp_pack_store<kMasked, kBucket, kDense>(xb, cb + c0 + CW, tb.at(c0 + CW),
+                                             kDense ? bw + CW / 2 : bw, kbase + c0 + CW, nvalid,
+                                             scale_log2, m, rs2, p_addr + (c0 + CW) / 2);
     if (c0 + 2 * CW < kHalf) tmem_ld_wait(xa);
   }
   tmem_wait_st();
@@ -621,7 +662,7 @@ GR_DEVICE bool rescale_o(uint32_t o_addr, float alpha, uint64_t* prev_pv, uint32
 // redo (their output is not written).
 template <bool kMasked, bool kBucket, bool kDense>
 GR_DEVICE bool softmax_tile(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, const float* cb,
-                            const TB& tb, const uint32_t* bw, int kbase, int nvalid,
+                            const TB& tb, const DB& bw, int kbase, int nvalid,
                             float scale_log2, bool first, bool row_ok, float& m, float& l,
                             uint64_t* prev_pv, uint32_t prev_ph, volatile int* abort_flag,
                             int32_t* err) {
@@ -936,19 +977,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
         const int sb = g & 1, st = g % kStages;
         // dense bias: this thread's 64 values of the tile (one 128-byte line), requested
         // before the wait for S so that the load overlaps it
-        uint32_t bw[kDense ? kHalf / 2 : 1];
+        uint32_t bw0[kDense ? 16 : 1];
+        DB bw{bw0, nullptr};
         float diagb = 0.f;
-        if (kDense) {
+        if constexpr (kDense) {
           if (j < it.nk) {
-            const uint4* src = reinterpret_cast<const uint4*>(brow + (it.nk - 1 - j) * BN);
-#pragma unroll
-            for (int c = 0; c < kHalf / 8; ++c) {
-              const uint4 w4 = __ldg(src + c);
-              bw[4 * c] = w4.x;
-              bw[4 * c + 1] = w4.y;
-              bw[4 * c + 2] = w4.z;
-              bw[4 * c + 3] = w4.w;
-            }
+            bw.src = reinterpret_cast<const uint4*>(brow + (it.nk - 1 - j) * BN);
+            load_bias16(bw.src, bw0);
           } else {  // the diagonal tile: the row's own entry
             diagb = kLog2e * __bfloat162float(brow[it.q0 + rt - kHalf * h]);
           }

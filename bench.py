@@ -453,6 +453,55 @@ def _attention_kernel_line(torch, G, timer, cfg, steps, backward, peak, peak_src
             "algorithmic_flops_per_launch": flops}
 
 
+def _linear_kernel_lines(torch, G, timer, cfg, steps, peak, peak_src, hbm, hbm_src, dev):
+    """Roofline lines of the four-layer block's linear layers (library tensor-core GEMMs
+    with fused epilogues) at the workload's token count, on random bf16 operands: 2 M N K
+    algorithmic flops each, and for the residual + RMSNorm layers also their algorithmic
+    HBM bytes (A in, the fp32 residual in and out, the bf16 normalised row out)."""
+    from gen import make_batch
+
+    T = make_batch(cfg).T
+    d = cfg.d
+    gen = torch.Generator(device=dev).manual_seed(7)
+    bf = torch.bfloat16
+    a = torch.randn((T, d), device=dev, generator=gen).to(bf)
+    u = torch.randn((T, 4 * d), device=dev, generator=gen).to(bf)
+    x = torch.randn((T, d), device=dev, generator=gen)
+    ws = {"qkv": (torch.randn((3 * d, d), device=dev, generator=gen) / d ** 0.5).to(bf),
+          "w1": (torch.randn((4 * d, d), device=dev, generator=gen) / d ** 0.5).to(bf),
+          "wo": (torch.randn((d, d), device=dev, generator=gen) / d ** 0.5).to(bf),
+          "w2": (torch.randn((d, 4 * d), device=dev, generator=gen) / (4 * d) ** 0.5).to(bf)}
+    out3 = torch.empty((T, 3 * d), dtype=bf, device=dev)
+    out4 = torch.empty((T, 4 * d), dtype=bf, device=dev)
+    a2 = torch.empty((T, d), dtype=bf, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    cases = [("QKV projection (store)", 3 * d, d, None,
+              lambda: G.linear(a, ws["qkv"], out3, err)),
+             ("W1 (SiLU epilogue)", 4 * d, d, None,
+              lambda: G.linear(a, ws["w1"], out4, err, epilogue=G.EPI_SILU)),
+             ("W_o (residual + RMSNorm epilogue)", d, d, T * (2 * d + 8 * d + 2 * d),
+              lambda: G.linear_residual_rmsnorm(a, ws["wo"], x, x, a2, err)),
+             ("W2 (residual + RMSNorm epilogue)", d, 4 * d, T * (8 * d + 8 * d + 2 * d),
+              lambda: G.linear_residual_rmsnorm(u, ws["w2"], x, x, a2, err))]
+    lines = []
+    for name, N, K, nbytes, fn in cases:
+        g = timer.graph(fn)
+        ms = float(np.mean(timer.time(lambda k: g.replay(), steps, name="timed_kernel")))
+        fl = 2.0 * T * N * K
+        line = {"kernel": f"k_gemm_tc: {name}", "workload": f"{cfg.name} token count "
+                f"(M={T}, N={N}, K={K}), random bf16 operands", "bound": "tensor",
+                "achieved": fl / (ms / 1e3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                "frac": fl / (ms / 1e3) / 1e12 / peak, "peak_source": peak_src,
+                "avg_launch_ms": ms, "algorithmic_flops_per_launch": fl}
+        if nbytes:
+            gbs = nbytes / (ms / 1e3) / 1e9
+            line["hbm"] = {"achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                           "peak_source": hbm_src, "algorithmic_bytes_per_launch": nbytes}
+        lines.append(line)
+    assert G.check_error(err) == 0, "device error flags raised in a kernel timing"
+    return lines
+
+
 def run_native(args, cfg, world, rank, local):
     import torch
     import torch.distributed as dist
@@ -601,6 +650,10 @@ def run_native(args, cfg, world, rank, local):
                     kernels.append(_attention_kernel_line(torch, G, timer, extra_cfg,
                                                           args.steps, bwd, peak_burst,
                                                           burst_src, dev))
+            if gm.fused_blocks:
+                kernels += _linear_kernel_lines(torch, G, timer, cfg, args.steps, peak_burst,
+                                                burst_src, hbm, f"{src} HBM copy bandwidth",
+                                                dev)
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:

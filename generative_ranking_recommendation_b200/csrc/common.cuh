@@ -256,6 +256,14 @@ GR_DEVICE void tma_reduce_add_3d(const void* tmap, const void* smem_src, int c0,
       ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// Store of a shared-memory box to a global tensor (tile mode, no multicast), by the TMA
+// engine; completion is tracked per thread in bulk groups.
+GR_DEVICE void tma_store_2d(const void* tmap, const void* smem_src, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+      : "memory");
+}
 GR_DEVICE void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // The committed bulk groups of this thread have read their shared-memory sources.
 GR_DEVICE void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

@@ -51,8 +51,12 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, 0, 0);  // A K-major, Wt K-ma
 constexpr uint32_t kABytes = BM * BK * 2;                    // 16 KB
 constexpr uint32_t kBBytes = BN * BK * 2;                    // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr uint32_t kOffRed = kStages * kStageBytes;          // res+rms: [2][BM] partial sums
-constexpr uint32_t kOffBar = kOffRed + 2 * 2 * BM * 4;
+// after the stages: store / SiLU stage their 32 x 32 bf16 output chunks here for the TMA
+// store (two 2 KB buffers per epilogue warp); res+rms keeps its row partial sums here
+constexpr uint32_t kOffRed = kStages * kStageBytes;
+constexpr uint32_t kChunkBytes = 32 * 32 * 2;
+constexpr uint32_t kOffBar = kOffRed + kEpiWarps * 2 * kChunkBytes;
+static_assert(kEpiWarps * 2 * kChunkBytes >= 2 * 2 * BM * 4, "partial sums fit");
 // barriers: full[S], empty[S], acc_full[2], acc_empty[2], done
 constexpr uint32_t kNumBars = 2 * kStages + 5;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
@@ -62,6 +66,7 @@ static_assert(kStageBytes % 1024 == 0, "1024-byte aligned stages");
 
 struct Params {
   CUtensorMap ta, tb;
+  CUtensorMap tc;  // store / SiLU: C [M][N] bf16, box 32 x 32, no swizzle
   GemmArgs g;
 };
 
@@ -71,6 +76,9 @@ GR_DEVICE bool wait_warp(uint64_t* bar, uint32_t ph, volatile int* abort_flag, i
   const bool ok = mbar_wait(bar, ph, abort_flag, err);
   return __all_sync(0xffffffffu, ok);
 }
+
+// At most one committed bulk group of this thread has yet to finish reading its source.
+GR_DEVICE void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 
 GR_DEVICE float tanh_approx(float x) {
   float y;
@@ -136,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   if (warp == 1 && lane == 0) {
     tma_prefetch_desc(&P.ta);
     tma_prefetch_desc(&P.tb);
+    if (!kRes) tma_prefetch_desc(&P.tc);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -217,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     const int ch = (warp - 2) >> 2;  // which 128 columns of each 256-column block
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const int rloc = q * 32 + lane;  // row within the tile
+    uint8_t* stage = smem + kOffRed + (warp - 2) * 2 * kChunkBytes;  // this warp's buffers
     int tc = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
       const int mt = t / n_tiles, nt = t - mt * n_tiles;
@@ -227,7 +237,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         if (!wait_warp(&acc_full[buf], par(tc >> 1), abort_flag, g.err)) break;
         tc_fence_after();
         const uint32_t acc = lane_base + (uint32_t)(buf * BN + ch * 128);
-        __nv_bfloat16* crow = (__nv_bfloat16*)g.c + row * g.ldc + (long long)nt * BN + ch * 128;
+        // each 32 x 32 chunk (the warp's rows, 32 columns) is written to one of the warp's
+        // two shared-memory buffers and stored by the TMA engine as whole lines; rows past
+        // M are clipped by the tensor map
+        const int gcol = nt * BN + ch * 128;
 #pragma unroll 1
         for (int c = 0; c < 128; c += 32) {
           float v[32];
@@ -236,7 +249,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = silu(v[e]);
           }
-          if (valid) store_bf16x32(crow + c, v);
+          uint8_t* box = stage + ((c >> 5) & 1) * kChunkBytes;
+          if (lane == 0) bulk_wait_read_1();  // the store that last read this buffer is done
+          __syncwarp();
+          store_bf16x32(reinterpret_cast<__nv_bfloat16*>(box + lane * 64), v);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && mt * BM + q * 32 < g.M) {  // boxes wholly past M are skipped
+            tma_store_2d(&P.tc, box, gcol + c, mt * BM + q * 32);
+            bulk_commit();
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -336,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     }
   }
 
+  if (!kRes && warp >= 2 && lane == 0) bulk_wait_all();  // the output stores have landed
   __syncwarp();
   tc_fence_before();
   __syncthreads();
@@ -415,11 +438,26 @@ static bool make_map(CUtensorMap* m, const void* base, long long rows, int K, lo
 
 static DeviceOnce gemm_smem_attr[3];
 
+// C [rows][N] bf16 with row stride ld elements; box 32 x 32, no swizzle (TMA store).
+static bool make_store_map(CUtensorMap* m, void* base, long long rows, int N, long long ld) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 template <int kEpi>
 static int launch_t(const GemmArgs& g, cudaStream_t st) {
   Params p;
   if (!make_map(&p.ta, g.a, g.M, g.K, g.lda, BM) || !make_map(&p.tb, g.w, g.N, g.K, g.ldw, BN))
     return GENRANK_ERR_CUDA;
+  if (kEpi != kEpiResRms && !make_store_map(&p.tc, g.c, g.M, g.N, g.ldc)) return GENRANK_ERR_CUDA;
   p.g = g;
   if (!set_smem_limit_once(gemm_smem_attr[kEpi], (const void*)k_gemm_tc<kEpi>, (int)kSmem))
     return GENRANK_ERR_CUDA;

@@ -27,7 +27,10 @@
 //     second half's MMAs;
 //   * warps 2-9 run the epilogue from TMEM, two warps per TMEM lane quadrant (one row
 //     per thread), each on half of a 256-column block; res+rms combines the two warps'
-//     row sums of squares (and head partial sums) through shared memory.
+//     row sums of squares (and head partial sums) through shared memory.  Outputs leave
+//     through two 2 KB shared-memory boxes per warp (64-byte swizzle, so one-row-per-
+//     thread writes hit every bank) as TMA stores of whole lines; the residual rows are
+//     bulk-prefetched into L2 when the tile's first loads are issued.
 // Tiles are ordered with the N tiles of one M tile adjacent, so CTAs running them at the
 // same time share the A tile in L2.  Every mbarrier wait is bounded.
 #include <cuda.h>
@@ -51,12 +54,13 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, 0, 0);  // A K-major, Wt K-ma
 constexpr uint32_t kABytes = BM * BK * 2;                    // 16 KB
 constexpr uint32_t kBBytes = BN * BK * 2;                    // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-// after the stages: store / SiLU stage their 32 x 32 bf16 output chunks here for the TMA
-// store (two 2 KB buffers per epilogue warp); res+rms keeps its row partial sums here
-constexpr uint32_t kOffRed = kStages * kStageBytes;
-constexpr uint32_t kChunkBytes = 32 * 32 * 2;
-constexpr uint32_t kOffBar = kOffRed + kEpiWarps * 2 * kChunkBytes;
-static_assert(kEpiWarps * 2 * kChunkBytes >= 2 * 2 * BM * 4, "partial sums fit");
+// after the stages: each epilogue warp's two 2 KB output boxes (32 rows x 32 bf16 columns,
+// or 32 rows x 16 fp32 columns), written by its threads and stored by the TMA engine;
+// then the residual + RMSNorm row partial sums (one float per row and column half)
+constexpr uint32_t kOffBox = kStages * kStageBytes;
+constexpr uint32_t kChunkBytes = 2048;
+constexpr uint32_t kOffRed = kOffBox + kEpiWarps * 2 * kChunkBytes;
+constexpr uint32_t kOffBar = kOffRed + 2 * BM * 4;
 // barriers: full[S], empty[S], acc_full[2], acc_empty[2], done
 constexpr uint32_t kNumBars = 2 * kStages + 5;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
@@ -66,7 +70,8 @@ static_assert(kStageBytes % 1024 == 0, "1024-byte aligned stages");
 
 struct Params {
   CUtensorMap ta, tb;
-  CUtensorMap tc;  // store / SiLU: C [M][N] bf16, box 32 x 32, no swizzle
+  CUtensorMap tc;  // C (store / SiLU) or a_out (res+rms): bf16, box 32 x 32, 64-byte swizzle
+  CUtensorMap tx;  // res+rms: x_out, fp32, box 16 x 32, 64-byte swizzle
   GemmArgs g;
 };
 
@@ -92,14 +97,18 @@ GR_DEVICE float silu(float v) {
   return fmaf(h, tanh_approx(h), h);
 }
 
-// 32 fp32 values to 16 bf16 pairs, stored as four 16-byte vectors at dst.
-GR_DEVICE void store_bf16x32(__nv_bfloat16* dst, const float* v) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+// Byte offset of 16-byte unit j of row r in a box of 64-byte rows written with the TMA
+// engine's 64-byte swizzle (unit index XOR address bits 7-8; the box is 512-byte aligned),
+// so a warp writing one row per thread spreads its stores over all banks.
+GR_DEVICE uint32_t sw64(int r, int j) { return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4)); }
+
+// 32 fp32 values to bf16, as row r of a 32 x 32 bf16 box (64-byte swizzle).
+GR_DEVICE void box_bf16x32(uint8_t* box, int r, const float* v) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
-    d4[q] = make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                       pack_bf16(v[8 * q + 4], v[8 * q + 5]),
-                       pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(box + sw64(r, j)) =
+        make_uint4(pack_bf16(v[8 * j], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
+                   pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
 }
 
 GR_DEVICE void load_f32x32(const float* src, float4 (&x)[8]) {
@@ -122,7 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   uint64_t* acc_full = bars + 2 * kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* done = acc_full + 4;
-  // res+rms partial sums: [ss of warp ch 0][ss of ch 1][head of ch 0][head of ch 1], BM each
+  // res+rms partial sums, [warp ch 0][warp ch 1] x BM rows: the sums of squares, then
+  // the head's dot products
   float* red = reinterpret_cast<float*>(smem + kOffRed);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
@@ -144,7 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   if (warp == 1 && lane == 0) {
     tma_prefetch_desc(&P.ta);
     tma_prefetch_desc(&P.tb);
-    if (!kRes) tma_prefetch_desc(&P.tc);
+    if (!kRes || g.a_out) tma_prefetch_desc(&P.tc);
+    if (kRes) tma_prefetch_desc(&P.tx);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -165,6 +176,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     bool ok = true;
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
       const int mt = t / n_tiles, nt = t - mt * n_tiles;
+      if (kRes) {
+        // the tile's residual rows head for L2 while its MMAs run, so the epilogue's
+        // reads of them wait on L2 rather than DRAM
+        for (int r = lane; r < BM && mt * BM + r < g.M; r += 32)
+          bulk_prefetch_l2(g.x_in + (long long)(mt * BM + r) * g.ldx, (uint32_t)g.N * 4u);
+      }
       for (int h = 0; h < kHalves && ok; ++h) {
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
           const int st = it % kStages;
@@ -226,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     const int ch = (warp - 2) >> 2;  // which 128 columns of each 256-column block
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const int rloc = q * 32 + lane;  // row within the tile
-    uint8_t* stage = smem + kOffRed + (warp - 2) * 2 * kChunkBytes;  // this warp's buffers
+    uint8_t* stage = smem + kOffBox + (warp - 2) * 2 * kChunkBytes;  // this warp's boxes
+    const int box_row = q * 32;  // + mt * BM: the warp's first row in C
     int tc = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
       const int mt = t / n_tiles, nt = t - mt * n_tiles;
@@ -252,11 +270,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
           uint8_t* box = stage + ((c >> 5) & 1) * kChunkBytes;
           if (lane == 0) bulk_wait_read_1();  // the store that last read this buffer is done
           __syncwarp();
-          store_bf16x32(reinterpret_cast<__nv_bfloat16*>(box + lane * 64), v);
+          box_bf16x32(box, lane, v);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0 && mt * BM + q * 32 < g.M) {  // boxes wholly past M are skipped
-            tma_store_2d(&P.tc, box, gcol + c, mt * BM + q * 32);
+          if (lane == 0 && mt * BM + box_row < g.M) {  // boxes wholly past M are skipped
+            tma_store_2d(&P.tc, box, gcol + c, mt * BM + box_row);
             bulk_commit();
           }
         }
@@ -266,9 +284,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         continue;
       }
       // res+rms: pass 1 per half as soon as its MMAs are done: y = x_in + acc, kept in
-      // TMEM, written to x_out, its squares summed; then the row's scale and pass 2
+      // TMEM, staged in the warp's two boxes (32 rows x 16 fp32 columns each) and stored
+      // to x_out by the TMA engine, its squares summed; then the row's scale and pass 2,
+      // whose bf16 rows go out through the same boxes
       const float* xin = g.x_in + row * g.ldx;
-      float* xout = g.x_out + row * g.ldx;
+      const bool rows_in = mt * BM + box_row < g.M;  // boxes wholly past M are skipped
       // A failed (timed-out) wait skips the work but not the named barriers below, so
       // the other warp of the quadrant never waits for a partner that has left.
       float ss = 0.f;
@@ -286,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         for (int c = 0; c < 128; c += 32) {
           float4 xv[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) xv[e] = xn[e];
+          for (int e = 0; e < 8; ++e) xv[e] = valid ? xn[e] : make_float4(0.f, 0.f, 0.f, 0.f);
           if (valid && c + 32 < 128) load_f32x32(xin + c0 + c + 32, xn);  // next chunk in flight
           float v[32];
           tmem_ld32(lane_base + c0 + c, v);
@@ -301,10 +321,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
             v[4 * e + 2] = xv[e].z;
             v[4 * e + 3] = xv[e].w;
           }
-          if (valid) {
-            float4* o4 = reinterpret_cast<float4*>(xout + c0 + c);
+          if (lane == 0) bulk_wait_read_all();  // the previous chunk's stores have read the boxes
+          __syncwarp();
 #pragma unroll
-            for (int e = 0; e < 8; ++e) o4[e] = xv[e];
+          for (int e = 0; e < 8; ++e)
+            *reinterpret_cast<float4*>(stage + (e >> 2) * kChunkBytes + sw64(lane, e & 3)) = xv[e];
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && rows_in) {
+            tma_store_2d(&P.tx, stage, c0 + c, mt * BM + box_row);
+            tma_store_2d(&P.tx, stage + kChunkBytes, c0 + c + 16, mt * BM + box_row);
+            bulk_commit();
           }
           uint32_t w[32];
 #pragma unroll
@@ -319,6 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       red[ch * BM + rloc] = ss;
       named_bar_sync(1 + q, 64);
       const float r = rsqrtf((red[rloc] + red[BM + rloc]) / (float)g.N + g.eps);
+      if (lane == 0) bulk_wait_read_all();  // pass 1's last stores have read the boxes
+      __syncwarp();
       float z = 0.f;
       for (int h = 0; h < 2 && ok; ++h) {
         const int c0 = h * BN + ch * 128;
@@ -328,8 +357,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
           tmem_ld32(lane_base + c0 + c, v);
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] *= r;
-          if (valid && g.a_out)
-            store_bf16x32((__nv_bfloat16*)g.a_out + row * g.lda_out + c0 + c, v);
+          if (g.a_out) {
+            uint8_t* box = stage + ((c >> 5) & 1) * kChunkBytes;
+            if (lane == 0) bulk_wait_read_1();  // the store that last read this box is done
+            __syncwarp();
+            box_bf16x32(box, lane, v);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && rows_in) {
+              tma_store_2d(&P.tc, box, c0 + c, mt * BM + box_row);
+              bulk_commit();
+            }
+          }
           if (g.w_head) {
             const float4* w4 = reinterpret_cast<const float4*>(g.w_head + c0 + c);
 #pragma unroll
@@ -344,9 +383,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         }
       }
       if (g.w_head) {
-        red[2 * BM + ch * BM + rloc] = z;
+        named_bar_sync(1 + q, 64);  // both warps have read the sums of squares
+        red[ch * BM + rloc] = z;
         named_bar_sync(1 + q, 64);
-        if (ch == 0 && valid) g.z[row] = red[2 * BM + rloc] + red[3 * BM + rloc];
+        if (ch == 0 && valid) g.z[row] = red[rloc] + red[BM + rloc];
       }
       // the partial-sum slots are reused by the next tile only after both warps of the
       // quadrant have read them
@@ -358,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     }
   }
 
-  if (!kRes && warp >= 2 && lane == 0) bulk_wait_all();  // the output stores have landed
+  if (warp >= 2 && lane == 0) bulk_wait_all();  // the output stores have landed
   __syncwarp();
   tc_fence_before();
   __syncthreads();
@@ -438,18 +478,21 @@ static bool make_map(CUtensorMap* m, const void* base, long long rows, int K, lo
 
 static DeviceOnce gemm_smem_attr[3];
 
-// C [rows][N] bf16 with row stride ld elements; box 32 x 32, no swizzle (TMA store).
-static bool make_store_map(CUtensorMap* m, void* base, long long rows, int N, long long ld) {
+// [rows][N] output (bf16 or fp32) with row stride ld elements, for TMA stores of 32-row
+// boxes of 64 bytes (32 bf16 or 16 fp32 columns) with the 64-byte swizzle.
+static bool make_store_map(CUtensorMap* m, void* base, long long rows, int N, long long ld,
+                           bool f32) {
   auto fn = encode_fn();
   if (!fn) return false;
+  const int es = f32 ? 4 : 2;
   cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-  cuuint32_t box[2] = {32, 32};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+  cuuint64_t strides[1] = {(cuuint64_t)ld * es};
+  cuuint32_t box[2] = {(cuuint32_t)(64 / es), 32};
+  cuuint32_t elem_strides[2] = {1, 1};
+  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base,
+            dims, strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int kEpi>
@@ -457,7 +500,13 @@ static int launch_t(const GemmArgs& g, cudaStream_t st) {
   Params p;
   if (!make_map(&p.ta, g.a, g.M, g.K, g.lda, BM) || !make_map(&p.tb, g.w, g.N, g.K, g.ldw, BN))
     return GENRANK_ERR_CUDA;
-  if (kEpi != kEpiResRms && !make_store_map(&p.tc, g.c, g.M, g.N, g.ldc)) return GENRANK_ERR_CUDA;
+  if (kEpi == kEpiResRms) {
+    if (!make_store_map(&p.tx, g.x_out, g.M, g.N, g.ldx, true) ||
+        (g.a_out && !make_store_map(&p.tc, g.a_out, g.M, g.N, g.lda_out, false)))
+      return GENRANK_ERR_CUDA;
+  } else if (!make_store_map(&p.tc, g.c, g.M, g.N, g.ldc, false)) {
+    return GENRANK_ERR_CUDA;
+  }
   p.g = g;
   if (!set_smem_limit_once(gemm_smem_attr[kEpi], (const void*)k_gemm_tc<kEpi>, (int)kSmem))
     return GENRANK_ERR_CUDA;

@@ -48,30 +48,42 @@ constexpr int BN = 256;  // columns per MMA block (one accumulator buffer)
 constexpr int BK = 64;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int kStages = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, 0, 0);  // A K-major, Wt K-major
 constexpr uint32_t kABytes = BM * BK * 2;                    // 16 KB
 constexpr uint32_t kBBytes = BN * BK * 2;                    // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
-// after the stages: each epilogue warp's two 2 KB output boxes (32 rows x 32 bf16 columns,
-// or 32 rows x 16 fp32 columns), written by its threads and stored by the TMA engine;
-// then the residual + RMSNorm row partial sums (one float per row and column half)
-constexpr uint32_t kOffBox = kStages * kStageBytes;
-constexpr uint32_t kChunkBytes = 2048;
-constexpr uint32_t kOffRed = kOffBox + kEpiWarps * 2 * kChunkBytes;
-constexpr uint32_t kOffBar = kOffRed + 2 * BM * 4;
-// barriers: full[S], empty[S], acc_full[2], acc_empty[2], done
-constexpr uint32_t kNumBars = 2 * kStages + 5;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kSmem = kOffMisc + 16 + 1024;
-static_assert(kSmem <= 227 * 1024, "shared memory");
+constexpr uint32_t kBoxBytes = 2048;  // 32 rows x 64 bytes (32 bf16 or 16 fp32 columns)
+constexpr int kXBufs = 4;             // res+rms: residual boxes in flight per epilogue warp
+
+// Shared memory of each epilogue, after the operand stages:
+//   store / SiLU: four stages; two output boxes per epilogue warp (ping-pong).
+//   res+rms: three stages (room for the residual boxes); per epilogue warp kXBufs boxes
+//     the residual rows are loaded into and one output box; then the row partial sums
+//     (one float per row and column half).
+// Then the barriers: full[S], empty[S], acc_full[2], acc_empty[2], done and, for res+rms,
+// one per residual box.
+template <bool kRes>
+struct Layout {
+  static constexpr int kStages = kRes ? 3 : 4;
+  static constexpr uint32_t kOffBox = kStages * kStageBytes;
+  static constexpr uint32_t kXBytes = kRes ? kEpiWarps * kXBufs * kBoxBytes : 0;
+  static constexpr uint32_t kOutBoxes = kRes ? 1 : 2;
+  static constexpr uint32_t kOffOut = kOffBox + kXBytes;
+  static constexpr uint32_t kOffRed = kOffOut + kEpiWarps * kOutBoxes * kBoxBytes;
+  static constexpr uint32_t kOffBar = kOffRed + (kRes ? 2 * BM * 4 : 0);
+  static constexpr uint32_t kNumBars = 2 * kStages + 5 + (kRes ? kEpiWarps * kXBufs : 0);
+  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kSmem = kOffMisc + 16 + 1024;
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+};
 static_assert(kStageBytes % 1024 == 0, "1024-byte aligned stages");
 
 struct Params {
   CUtensorMap ta, tb;
   CUtensorMap tc;  // C (store / SiLU) or a_out (res+rms): bf16, box 32 x 32, 64-byte swizzle
-  CUtensorMap tx;  // res+rms: x_out, fp32, box 16 x 32, 64-byte swizzle
+  CUtensorMap tx;   // res+rms: x_out, fp32, box 16 x 32, 64-byte swizzle (TMA store)
+  CUtensorMap txi;  // res+rms: x_in, the same geometry (TMA load)
   GemmArgs g;
 };
 
@@ -120,22 +132,25 @@ GR_DEVICE void load_f32x32(const float* src, float4 (&x)[8]) {
 template <int kEpi>
 __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__ Params P) {
   constexpr bool kRes = kEpi == kEpiResRms;
+  using L = Layout<kRes>;
+  constexpr int kStages = L::kStages;
   constexpr int kHalves = kRes ? 2 : 1;  // 256-column blocks per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const GemmArgs& g = P.g;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
   uint64_t* acc_full = bars + 2 * kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* done = acc_full + 4;
+  uint64_t* xbar = acc_full + 5;  // res+rms: [epilogue warp][kXBufs] residual box loads
   // res+rms partial sums, [warp ch 0][warp ch 1] x BM rows: the sums of squares, then
   // the head's dot products
-  float* red = reinterpret_cast<float*>(smem + kOffRed);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  float* red = reinterpret_cast<float*>(smem + L::kOffRed);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -148,6 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       mbar_init(&acc_empty[b], kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(done, 1);
+    if (kRes)
+      for (int b = 0; b < kEpiWarps * kXBufs; ++b) mbar_init(&xbar[b], 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -155,7 +172,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     tma_prefetch_desc(&P.ta);
     tma_prefetch_desc(&P.tb);
     if (!kRes || g.a_out) tma_prefetch_desc(&P.tc);
-    if (kRes) tma_prefetch_desc(&P.tx);
+    if (kRes) {
+      tma_prefetch_desc(&P.tx);
+      tma_prefetch_desc(&P.txi);
+    }
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -177,8 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
       const int mt = t / n_tiles, nt = t - mt * n_tiles;
       if (kRes) {
-        // the tile's residual rows head for L2 while its MMAs run, so the epilogue's
-        // reads of them wait on L2 rather than DRAM
+        // the tile's residual rows head for L2 while its MMAs run
         for (int r = lane; r < BM && mt * BM + r < g.M; r += 32)
           bulk_prefetch_l2(g.x_in + (long long)(mt * BM + r) * g.ldx, (uint32_t)g.N * 4u);
       }
@@ -239,25 +258,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue warps 2-9
-    const int q = warp & 3;          // TMEM lane quadrant
-    const int ch = (warp - 2) >> 2;  // which 128 columns of each 256-column block
+    const int ew = warp - 2;
+    const int q = warp & 3;  // TMEM lane quadrant
+    const int ch = ew >> 2;  // which 128 columns of each 256-column block
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const int rloc = q * 32 + lane;  // row within the tile
-    uint8_t* stage = smem + kOffBox + (warp - 2) * 2 * kChunkBytes;  // this warp's boxes
-    const int box_row = q * 32;  // + mt * BM: the warp's first row in C
-    int tc = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
-      const int mt = t / n_tiles, nt = t - mt * n_tiles;
-      const long long row = (long long)mt * BM + rloc;
-      const bool valid = row < g.M;
-      if (!kRes) {
+    const int box_row = q * 32;      // + mt * BM: the warp's first row in C
+    uint8_t* out = smem + L::kOffOut + ew * L::kOutBoxes * kBoxBytes;  // output boxes
+    if (!kRes) {
+      int tc = 0;
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
+        const int mt = t / n_tiles, nt = t - mt * n_tiles;
         const int buf = tc & 1;
         if (!wait_warp(&acc_full[buf], par(tc >> 1), abort_flag, g.err)) break;
         tc_fence_after();
         const uint32_t acc = lane_base + (uint32_t)(buf * BN + ch * 128);
         // each 32 x 32 chunk (the warp's rows, 32 columns) is written to one of the warp's
-        // two shared-memory buffers and stored by the TMA engine as whole lines; rows past
-        // M are clipped by the tensor map
+        // two boxes and stored by the TMA engine as whole lines; rows past M are clipped
+        // by the tensor map
         const int gcol = nt * BN + ch * 128;
 #pragma unroll 1
         for (int c = 0; c < 128; c += 32) {
@@ -267,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = silu(v[e]);
           }
-          uint8_t* box = stage + ((c >> 5) & 1) * kChunkBytes;
-          if (lane == 0) bulk_wait_read_1();  // the store that last read this buffer is done
+          uint8_t* box = out + ((c >> 5) & 1) * kBoxBytes;
+          if (lane == 0) bulk_wait_read_1();  // the store that last read this box is done
           __syncwarp();
           box_bf16x32(box, lane, v);
           fence_proxy_async_smem();
@@ -281,120 +299,150 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        continue;
       }
-      // res+rms: pass 1 per half as soon as its MMAs are done: y = x_in + acc, kept in
-      // TMEM, staged in the warp's two boxes (32 rows x 16 fp32 columns each) and stored
-      // to x_out by the TMA engine, its squares summed; then the row's scale and pass 2,
-      // whose bf16 rows go out through the same boxes
-      const float* xin = g.x_in + row * g.ldx;
-      const bool rows_in = mt * BM + box_row < g.M;  // boxes wholly past M are skipped
-      // A failed (timed-out) wait skips the work but not the named barriers below, so
-      // the other warp of the quadrant never waits for a partner that has left.
-      float ss = 0.f;
+    } else {
+      // res+rms.  The warp's residual boxes (32 rows x 16 fp32 columns, 16 a tile: 8 per
+      // 256-column half) are numbered across its tiles; box n goes to buffer n % kXBufs,
+      // and the load of box n + kXBufs is issued as soon as box n has been read, so the
+      // next tile's first boxes load while this tile's normalisation runs.
+      uint8_t* xb = smem + L::kOffBox + ew * kXBufs * kBoxBytes;
+      uint64_t* xw = xbar + ew * kXBufs;
+      const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+      const int nbox = 16 * my_tiles;
+      int ld = 0;  // residual boxes whose loads were issued
+      auto issue = [&](int n) {  // lane 0: load residual box n
+        const int t = blockIdx.x + (n >> 4) * gridDim.x;
+        const int col = ((n >> 3) & 1) * BN + ch * 128 + (n & 7) * 16;
+        const int b = n % kXBufs;
+        mbar_expect_tx(&xw[b], kBoxBytes);
+        tma_load_2d(xb + b * kBoxBytes, &P.txi, &xw[b], col, t * BM + box_row);
+      };
+      if (lane == 0)
+        for (; ld < kXBufs && ld < nbox; ++ld) issue(ld);
+      ld = min(kXBufs, nbox);
+      int n = 0;  // residual boxes consumed
+      int tc = 0;
+      // A failed (timed-out) wait skips the work but not the named barriers below, so the
+      // other warp of the quadrant never waits for a partner that has left.
       bool ok = true;
-      for (int h = 0; h < 2 && ok; ++h) {
-        if (!wait_warp(&acc_full[h], par(tc), abort_flag, g.err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int c0 = h * BN + ch * 128;
-        float4 xn[8];
-        if (valid) load_f32x32(xin + c0, xn);
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
+        const int mt = t;
+        const long long row = (long long)mt * BM + rloc;
+        const bool valid = row < g.M;
+        const bool rows_in = mt * BM + box_row < g.M;  // boxes wholly past M are skipped
+        // pass 1 per half as soon as its MMAs are done: y = x_in + acc, kept in TMEM,
+        // written to x_out through the output box, its squares summed
+        float ss = 0.f;
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!wait_warp(&acc_full[h], par(tc), abort_flag, g.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int c0 = h * BN + ch * 128;
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          float4 xv[8];
+          for (int c = 0; c < 128; c += 16, ++n) {
+            uint32_t a[16];
+            tmem_ld16_async(lane_base + c0 + c, a);
+            const int b = n % kXBufs;
+            if (!wait_warp(&xw[b], par(n / kXBufs), abort_flag, g.err)) {
+              tmem_ld_wait(a);
+              ok = false;
+              break;
+            }
+            const uint8_t* xs = xb + b * kBoxBytes;
+            float4 y[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) xv[e] = valid ? xn[e] : make_float4(0.f, 0.f, 0.f, 0.f);
-          if (valid && c + 32 < 128) load_f32x32(xin + c0 + c + 32, xn);  // next chunk in flight
-          float v[32];
-          tmem_ld32(lane_base + c0 + c, v);
+            for (int e = 0; e < 4; ++e) y[e] = *reinterpret_cast<const float4*>(xs + sw64(lane, e));
+            tmem_ld_wait(a);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            xv[e].x += v[4 * e];
-            xv[e].y += v[4 * e + 1];
-            xv[e].z += v[4 * e + 2];
-            xv[e].w += v[4 * e + 3];
-            v[4 * e] = xv[e].x;
-            v[4 * e + 1] = xv[e].y;
-            v[4 * e + 2] = xv[e].z;
-            v[4 * e + 3] = xv[e].w;
-          }
-          if (lane == 0) bulk_wait_read_all();  // the previous chunk's stores have read the boxes
-          __syncwarp();
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            *reinterpret_cast<float4*>(stage + (e >> 2) * kChunkBytes + sw64(lane, e & 3)) = xv[e];
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && rows_in) {
-            tma_store_2d(&P.tx, stage, c0 + c, mt * BM + box_row);
-            tma_store_2d(&P.tx, stage + kChunkBytes, c0 + c + 16, mt * BM + box_row);
-            bulk_commit();
-          }
-          uint32_t w[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            ss = fmaf(v[e], v[e], ss);
-            w[e] = __float_as_uint(v[e]);
-          }
-          tmem_st32(lane_base + c0 + c, w);
-        }
-      }
-      // the row's sum of squares over both warps of this quadrant
-      red[ch * BM + rloc] = ss;
-      named_bar_sync(1 + q, 64);
-      const float r = rsqrtf((red[rloc] + red[BM + rloc]) / (float)g.N + g.eps);
-      if (lane == 0) bulk_wait_read_all();  // pass 1's last stores have read the boxes
-      __syncwarp();
-      float z = 0.f;
-      for (int h = 0; h < 2 && ok; ++h) {
-        const int c0 = h * BN + ch * 128;
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          float v[32];
-          tmem_ld32(lane_base + c0 + c, v);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] *= r;
-          if (g.a_out) {
-            uint8_t* box = stage + ((c >> 5) & 1) * kChunkBytes;
-            if (lane == 0) bulk_wait_read_1();  // the store that last read this box is done
+            for (int e = 0; e < 4; ++e) {
+              y[e].x += __uint_as_float(a[4 * e]);
+              y[e].y += __uint_as_float(a[4 * e + 1]);
+              y[e].z += __uint_as_float(a[4 * e + 2]);
+              y[e].w += __uint_as_float(a[4 * e + 3]);
+              ss = fmaf(y[e].x, y[e].x, ss);
+              ss = fmaf(y[e].y, y[e].y, ss);
+              ss = fmaf(y[e].z, y[e].z, ss);
+              ss = fmaf(y[e].w, y[e].w, ss);
+              a[4 * e] = __float_as_uint(y[e].x);
+              a[4 * e + 1] = __float_as_uint(y[e].y);
+              a[4 * e + 2] = __float_as_uint(y[e].z);
+              a[4 * e + 3] = __float_as_uint(y[e].w);
+            }
+            tmem_st16(lane_base + c0 + c, a);
+            __syncwarp();  // every lane has read the residual box: reload it
+            if (lane == 0) {
+              if (ld < nbox) issue(ld);
+              bulk_wait_read_all();  // the output box's previous store has read it
+            }
+            ++ld;
             __syncwarp();
-            box_bf16x32(box, lane, v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) *reinterpret_cast<float4*>(out + sw64(lane, e)) = y[e];
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0 && rows_in) {
-              tma_store_2d(&P.tc, box, c0 + c, mt * BM + box_row);
+              tma_store_2d(&P.tx, out, c0 + c, mt * BM + box_row);
               bulk_commit();
             }
           }
-          if (g.w_head) {
-            const float4* w4 = reinterpret_cast<const float4*>(g.w_head + c0 + c);
+        }
+        // the row's sum of squares over both warps of this quadrant
+        red[ch * BM + rloc] = ss;
+        named_bar_sync(1 + q, 64);
+        const float r = rsqrtf((red[rloc] + red[BM + rloc]) / (float)g.N + g.eps);
+        // pass 2: the normalised row, to a_out in bf16 and into the head's dot product
+        float z = 0.f;
+        for (int h = 0; h < 2 && ok; ++h) {
+          const int c0 = h * BN + ch * 128;
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 32) {
+            float v[32];
+            tmem_ld32(lane_base + c0 + c, v);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float4 wv = w4[e];
-              z = fmaf(v[4 * e], wv.x, z);
-              z = fmaf(v[4 * e + 1], wv.y, z);
-              z = fmaf(v[4 * e + 2], wv.z, z);
-              z = fmaf(v[4 * e + 3], wv.w, z);
+            for (int e = 0; e < 32; ++e) v[e] *= r;
+            if (g.a_out) {
+              if (lane == 0) bulk_wait_read_all();  // the output box's previous store is done
+              __syncwarp();
+              box_bf16x32(out, lane, v);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0 && rows_in) {
+                tma_store_2d(&P.tc, out, c0 + c, mt * BM + box_row);
+                bulk_commit();
+              }
+            }
+            if (g.w_head) {
+              const float4* w4 = reinterpret_cast<const float4*>(g.w_head + c0 + c);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float4 wv = w4[e];
+                z = fmaf(v[4 * e], wv.x, z);
+                z = fmaf(v[4 * e + 1], wv.y, z);
+                z = fmaf(v[4 * e + 2], wv.z, z);
+                z = fmaf(v[4 * e + 3], wv.w, z);
+              }
             }
           }
         }
-      }
-      if (g.w_head) {
-        named_bar_sync(1 + q, 64);  // both warps have read the sums of squares
-        red[ch * BM + rloc] = z;
+        if (g.w_head) {
+          named_bar_sync(1 + q, 64);  // both warps have read the sums of squares
+          red[ch * BM + rloc] = z;
+          named_bar_sync(1 + q, 64);
+          if (ch == 0 && valid) g.z[row] = red[rloc] + red[BM + rloc];
+        }
+        // the partial-sum slots are reused by the next tile only after both warps of the
+        // quadrant have read them
         named_bar_sync(1 + q, 64);
-        if (ch == 0 && valid) g.z[row] = red[rloc] + red[BM + rloc];
+        if (!ok) break;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[0]);
       }
-      // the partial-sum slots are reused by the next tile only after both warps of the
-      // quadrant have read them
-      named_bar_sync(1 + q, 64);
-      if (!ok) break;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[0]);
+      // residual boxes still in flight (a failed wait) land before the CTA exits
+      if (lane == 0)
+        for (int x = n; x < min(ld, nbox); ++x) mbar_drain(&xw[x % kXBufs], par(x / kXBufs));
     }
   }
 
@@ -502,13 +550,15 @@ static int launch_t(const GemmArgs& g, cudaStream_t st) {
     return GENRANK_ERR_CUDA;
   if (kEpi == kEpiResRms) {
     if (!make_store_map(&p.tx, g.x_out, g.M, g.N, g.ldx, true) ||
+        !make_store_map(&p.txi, const_cast<float*>(g.x_in), g.M, g.N, g.ldx, true) ||
         (g.a_out && !make_store_map(&p.tc, g.a_out, g.M, g.N, g.lda_out, false)))
       return GENRANK_ERR_CUDA;
   } else if (!make_store_map(&p.tc, g.c, g.M, g.N, g.ldc, false)) {
     return GENRANK_ERR_CUDA;
   }
   p.g = g;
-  if (!set_smem_limit_once(gemm_smem_attr[kEpi], (const void*)k_gemm_tc<kEpi>, (int)kSmem))
+  constexpr int kSmem = (int)Layout<kEpi == kEpiResRms>::kSmem;
+  if (!set_smem_limit_once(gemm_smem_attr[kEpi], (const void*)k_gemm_tc<kEpi>, kSmem))
     return GENRANK_ERR_CUDA;
   const int sms = sm_count_current();
   if (sms <= 0) return GENRANK_ERR_CUDA;

@@ -493,14 +493,6 @@ GR_DEVICE void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
 }
 
-// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned address, size a multiple of 16);
-// nothing waits for it.
-GR_DEVICE void bulk_prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
-               "r"(bytes)
-               : "memory");
-}
-
 // Shared-memory matrix descriptor for tcgen05 (Blackwell layout, version 1):
 // start address, leading/stride byte offsets (>> 4), 128-byte swizzle.
 GR_DEVICE uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {

@@ -18,19 +18,21 @@
 //
 // Design, one CTA per SM (persistent), 320 threads:
 //   * warp 1 issues TMA loads of 128 x 64 A tiles and 256 x 64 Wt tiles (128B swizzle,
-//     no multicast) into a four-stage ring (48 KB a stage);
+//     no multicast) into a ring of 48 KB stages (four; three for res+rms);
 //   * warp 0 (one thread) issues tcgen05.mma M = 128, N = 256, K = 16 (four per 64-wide
 //     k-step) into a TMEM accumulator.  The store and SiLU epilogues double-buffer the
 //     accumulator (2 x 256 columns) so a tile's epilogue overlaps the next tile's MMAs.
-//     res+rms computes its row (d = 512) as two 256-column halves one after the other,
-//     into columns [0, 256) and [256, 512): the first half's residual pass overlaps the
-//     second half's MMAs;
+//     res+rms computes its row (d = 512) as two 256-column halves, into columns [0, 256)
+//     and [256, 512), taking turns every 16 k-steps (the A rows of a chunk are re-read
+//     from L2, not DRAM): the first half completes a chunk early and its residual pass
+//     overlaps the second half's last MMAs, and each half's columns are released as soon
+//     as the normalisation has read them;
 //   * warps 2-9 run the epilogue from TMEM, two warps per TMEM lane quadrant (one row
 //     per thread), each on half of a 256-column block; res+rms combines the two warps'
 //     row sums of squares (and head partial sums) through shared memory.  Outputs leave
-//     through two 2 KB shared-memory boxes per warp (64-byte swizzle, so one-row-per-
-//     thread writes hit every bank) as TMA stores of whole lines; the residual rows are
-//     bulk-prefetched into L2 when the tile's first loads are issued.
+//     through 2 KB shared-memory boxes (64-byte swizzle, so one-row-per-thread writes
+//     hit every bank) as TMA stores of whole lines; res+rms loads its residual rows the
+//     same way, four boxes ahead of use per warp.
 // Tiles are ordered with the N tiles of one M tile adjacent, so CTAs running them at the
 // same time share the A tile in L2.  Every mbarrier wait is bounded.
 #include <cuda.h>
@@ -53,6 +55,10 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, 0, 0);  // A K-major, Wt K-ma
 constexpr uint32_t kABytes = BM * BK * 2;                    // 16 KB
 constexpr uint32_t kBBytes = BN * BK * 2;                    // 32 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
+// res+rms: the two 256-column halves take turns in chunks of this many k-steps, so a
+// tile's A rows are read from DRAM once (the other half's read of the chunk hits L2) and
+// the first half still completes one chunk ahead of the second
+constexpr int kChunkSteps = 16;
 constexpr uint32_t kBoxBytes = 2048;  // 32 rows x 64 bytes (32 bf16 or 16 fp32 columns)
 constexpr int kXBufs = 4;             // res+rms: residual boxes in flight per epilogue warp
 
@@ -119,6 +125,16 @@ GR_DEVICE void box_bf16x32(uint8_t* box, int r, const float* v) {
 #pragma unroll
   for (int j = 0; j < 4; ++j)
     *reinterpret_cast<uint4*>(box + sw64(r, j)) =
+        make_uint4(pack_bf16(v[8 * j], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
+                   pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
+}
+
+// 16 fp32 values to bf16, as columns [16 half, 16 half + 16) of row r of a 32 x 32 bf16
+// box (64-byte swizzle).
+GR_DEVICE void box_bf16x16(uint8_t* box, int r, int half, const float* v) {
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    *reinterpret_cast<uint4*>(box + sw64(r, 2 * half + j)) =
         make_uint4(pack_bf16(v[8 * j], v[8 * j + 1]), pack_bf16(v[8 * j + 2], v[8 * j + 3]),
                    pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
 }
@@ -196,23 +212,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     bool ok = true;
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
       const int mt = t / n_tiles, nt = t - mt * n_tiles;
-      if (kRes) {
-        // the tile's residual rows head for L2 while its MMAs run
-        for (int r = lane; r < BM && mt * BM + r < g.M; r += 32)
-          bulk_prefetch_l2(g.x_in + (long long)(mt * BM + r) * g.ldx, (uint32_t)g.N * 4u);
-      }
-      for (int h = 0; h < kHalves && ok; ++h) {
-        for (int ks = 0; ks < ksteps; ++ks, ++it) {
-          const int st = it % kStages;
-          if (!wait_warp(&empty[st], par(it / kStages) ^ 1u, abort_flag, g.err)) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) {
-            uint8_t* sa = smem + st * kStageBytes;
-            mbar_expect_tx(&full[st], kStageBytes);
-            tma_load_2d(sa, &P.ta, &full[st], ks * BK, mt * BM);
-            tma_load_2d(sa + kABytes, &P.tb, &full[st], ks * BK, (nt + h) * BN);
+      for (int k0 = 0; k0 < ksteps && ok; k0 += kChunkSteps) {
+        const int k1 = min(ksteps, k0 + kChunkSteps);
+        for (int h = 0; h < kHalves && ok; ++h) {
+          for (int ks = k0; ks < k1; ++ks, ++it) {
+            const int st = it % kStages;
+            if (!wait_warp(&empty[st], par(it / kStages) ^ 1u, abort_flag, g.err)) {
+              ok = false;
+              break;
+            }
+            if (lane == 0) {
+              uint8_t* sa = smem + st * kStageBytes;
+              mbar_expect_tx(&full[st], kStageBytes);
+              tma_load_2d(sa, &P.ta, &full[st], ks * BK, mt * BM);
+              tma_load_2d(sa + kABytes, &P.tb, &full[st], ks * BK, (nt + h) * BN);
+            }
           }
         }
       }
@@ -228,27 +242,39 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
         const int buf = kRes ? 0 : (tc & 1);
         const uint32_t ph_empty = kRes ? par(tc) ^ 1u : par(tc >> 1) ^ 1u;
-        if (!mbar_wait(&acc_empty[buf], ph_empty, abort_flag, g.err)) break;
-        tc_fence_after();
-        for (int h = 0; h < kHalves && ok; ++h) {
-          const uint32_t acc = tmem + (uint32_t)((kRes ? h : buf) * BN);
-          for (int ks = 0; ks < ksteps; ++ks, ++it) {
-            const int st = it % kStages;
-            if (!mbar_wait(&full[st], par(it / kStages), abort_flag, g.err)) {
-              ok = false;
-              break;
+        if (!kRes) {
+          if (!mbar_wait(&acc_empty[buf], ph_empty, abort_flag, g.err)) break;
+          tc_fence_after();
+        }
+        for (int k0 = 0; k0 < ksteps && ok; k0 += kChunkSteps) {
+          const int k1 = min(ksteps, k0 + kChunkSteps);
+          for (int h = 0; h < kHalves && ok; ++h) {
+            if (kRes && k0 == 0) {  // each half's columns are released on their own
+              if (!mbar_wait(&acc_empty[h], ph_empty, abort_flag, g.err)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
             }
-            tc_fence_after();
-            const uint32_t sa = smem_u32(smem + st * kStageBytes);
+            const uint32_t acc = tmem + (uint32_t)((kRes ? h : buf) * BN);
+            for (int ks = k0; ks < k1; ++ks, ++it) {
+              const int st = it % kStages;
+              if (!mbar_wait(&full[st], par(it / kStages), abort_flag, g.err)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t sa = smem_u32(smem + st * kStageBytes);
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(sa + kABytes + kk * 32, 16, 1024);
-              mma_bf16_ss(acc, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < BK / 16; ++kk) {
+                const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
+                const uint64_t bd = smem_desc_sw128(sa + kABytes + kk * 32, 16, 1024);
+                mma_bf16_ss(acc, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+              }
+              mma_commit(&empty[st]);  // the stage is free once these MMAs have read it
             }
-            mma_commit(&empty[st]);  // the stage is free once these MMAs have read it
+            if (ok && k1 == ksteps) mma_commit(&acc_full[kRes ? h : buf]);
           }
-          if (ok) mma_commit(&acc_full[kRes ? h : buf]);
         }
       }
       // every MMA issued has completed before TMEM is freed
@@ -305,22 +331,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       // 256-column half) are numbered across its tiles; box n goes to buffer n % kXBufs,
       // and the load of box n + kXBufs is issued as soon as box n has been read, so the
       // next tile's first boxes load while this tile's normalisation runs.
+      constexpr int kPerTile = 16;
       uint8_t* xb = smem + L::kOffBox + ew * kXBufs * kBoxBytes;
       uint64_t* xw = xbar + ew * kXBufs;
       const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-      const int nbox = 16 * my_tiles;
-      int ld = 0;  // residual boxes whose loads were issued
-      auto issue = [&](int n) {  // lane 0: load residual box n
-        const int t = blockIdx.x + (n >> 4) * gridDim.x;
-        const int col = ((n >> 3) & 1) * BN + ch * 128 + (n & 7) * 16;
+      const int nbox = kPerTile * my_tiles;
+      auto issue = [&](int n) {  // lane 0: load box n
+        const int t = blockIdx.x + (n / kPerTile) * gridDim.x;
+        const int w = n % kPerTile;
+        const int col = ((w >> 3) & 1) * BN + ch * 128 + (w & 7) * 16;
         const int b = n % kXBufs;
         mbar_expect_tx(&xw[b], kBoxBytes);
         tma_load_2d(xb + b * kBoxBytes, &P.txi, &xw[b], col, t * BM + box_row);
       };
+      int ld = 0;  // boxes whose loads were issued
       if (lane == 0)
-        for (; ld < kXBufs && ld < nbox; ++ld) issue(ld);
+        for (int x = 0; x < kXBufs && x < nbox; ++x) issue(x);
       ld = min(kXBufs, nbox);
-      int n = 0;  // residual boxes consumed
+      int n = 0;  // boxes consumed
+      // waits for box n; false (the error recorded) when it timed out
+      auto wait_box = [&](int x) { return wait_warp(&xw[x % kXBufs], par(x / kXBufs), abort_flag, g.err); };
+      // after box n has been read by every lane: the next load
+      auto next_load = [&]() {
+        __syncwarp();
+        if (ld < nbox && lane == 0) issue(ld);
+        ++ld;
+      };
       int tc = 0;
       // A failed (timed-out) wait skips the work but not the named barriers below, so the
       // other warp of the quadrant never waits for a partner that has left.
@@ -344,13 +380,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
           for (int c = 0; c < 128; c += 16, ++n) {
             uint32_t a[16];
             tmem_ld16_async(lane_base + c0 + c, a);
-            const int b = n % kXBufs;
-            if (!wait_warp(&xw[b], par(n / kXBufs), abort_flag, g.err)) {
+            if (!wait_box(n)) {
               tmem_ld_wait(a);
               ok = false;
               break;
             }
-            const uint8_t* xs = xb + b * kBoxBytes;
+            const uint8_t* xs = xb + (n % kXBufs) * kBoxBytes;
             float4 y[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) y[e] = *reinterpret_cast<const float4*>(xs + sw64(lane, e));
@@ -371,12 +406,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
               a[4 * e + 3] = __float_as_uint(y[e].w);
             }
             tmem_st16(lane_base + c0 + c, a);
-            __syncwarp();  // every lane has read the residual box: reload it
-            if (lane == 0) {
-              if (ld < nbox) issue(ld);
-              bulk_wait_read_all();  // the output box's previous store has read it
-            }
-            ++ld;
+            next_load();
+            if (lane == 0) bulk_wait_read_all();  // the output box's previous store has read it
             __syncwarp();
 #pragma unroll
             for (int e = 0; e < 4; ++e) *reinterpret_cast<float4*>(out + sw64(lane, e)) = y[e];
@@ -392,31 +423,45 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         red[ch * BM + rloc] = ss;
         named_bar_sync(1 + q, 64);
         const float r = rsqrtf((red[rloc] + red[BM + rloc]) / (float)g.N + g.eps);
-        // pass 2: the normalised row, to a_out in bf16 and into the head's dot product
+        // pass 2: the normalised row, to a_out in bf16 and into the head's dot product, 16
+        // columns a step (an a_out box takes two); each half's accumulator columns go back
+        // to the MMAs as soon as they have been read, so the next tile's first half overlaps
+        // this tile's second
         float z = 0.f;
         for (int h = 0; h < 2 && ok; ++h) {
           const int c0 = h * BN + ch * 128;
 #pragma unroll 1
-          for (int c = 0; c < 128; c += 32) {
-            float v[32];
-            tmem_ld32(lane_base + c0 + c, v);
+          for (int c = 0; c < 128; c += 16) {
+            float v[16];
+            {
+              uint32_t a[16];
+              tmem_ld16_async(lane_base + c0 + c, a);
+              tmem_ld_wait(a);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] *= r;
+              for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(a[e]);
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] *= r;
             if (g.a_out) {
-              if (lane == 0) bulk_wait_read_all();  // the output box's previous store is done
-              __syncwarp();
-              box_bf16x32(out, lane, v);
-              fence_proxy_async_smem();
-              __syncwarp();
-              if (lane == 0 && rows_in) {
-                tma_store_2d(&P.tc, out, c0 + c, mt * BM + box_row);
-                bulk_commit();
+              const int half = (c >> 4) & 1;
+              if (half == 0) {
+                if (lane == 0) bulk_wait_read_all();  // the output box's previous store is done
+                __syncwarp();
+              }
+              box_bf16x16(out, lane, half, v);
+              if (half == 1) {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && rows_in) {
+                  tma_store_2d(&P.tc, out, c0 + c - 16, mt * BM + box_row);
+                  bulk_commit();
+                }
               }
             }
             if (g.w_head) {
               const float4* w4 = reinterpret_cast<const float4*>(g.w_head + c0 + c);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
+              for (int e = 0; e < 4; ++e) {
                 const float4 wv = w4[e];
                 z = fmaf(v[4 * e], wv.x, z);
                 z = fmaf(v[4 * e + 1], wv.y, z);
@@ -425,6 +470,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
               }
             }
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[h]);
         }
         if (g.w_head) {
           named_bar_sync(1 + q, 64);  // both warps have read the sums of squares
@@ -436,11 +484,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         // quadrant have read them
         named_bar_sync(1 + q, 64);
         if (!ok) break;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[0]);
       }
-      // residual boxes still in flight (a failed wait) land before the CTA exits
+      // boxes still in flight (a failed wait) land before the CTA exits
       if (lane == 0)
         for (int x = n; x < min(ld, nbox); ++x) mbar_drain(&xw[x % kXBufs], par(x / kXBufs));
     }

@@ -86,6 +86,57 @@ def test_linear_residual_rmsnorm_parity(G, M, K, head):
         assert ref.rel_to_max(z.double().cpu().numpy(), _rms(xo) @ w.double().cpu().numpy()) <= 2e-2
 
 
+@pytest.mark.parametrize("M,K", [(50_000, 512), (40_001, 2048)])
+def test_linear_residual_rmsnorm_many_tiles(G, M, K):
+    """Several row tiles per CTA (each CTA of the persistent grid loads its next tile's
+    residual rows while finishing the current one), out of place, with the head; the
+    float64 reference runs on the device."""
+    d = 512
+    A = _bf((M, K), 7, 1.0)
+    Wt = _bf((d, K), 8, 1.0 / np.sqrt(K))
+    x = torch.randn((M, d), generator=torch.Generator(device="cuda").manual_seed(9),
+                    device="cuda")
+    x0 = x.clone()
+    xo = torch.full_like(x, float("nan"))
+    a_out = torch.full((M, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    w = torch.randn(d, generator=torch.Generator(device="cuda").manual_seed(10), device="cuda")
+    z = torch.full((M,), float("nan"), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    G.linear_residual_rmsnorm(A, Wt, x, xo, a_out, err, w_head=w, z=z)
+    assert G.check_error(err) == 0
+    assert torch.equal(x, x0)
+    want = x.double() + A.double() @ Wt.double().T
+    got = xo.double()
+    assert float((got - want).abs().max() / want.abs().max()) <= 1e-3
+    nrm = want / torch.sqrt((want * want).mean(dim=1, keepdim=True) + EPS)
+    an = a_out.double()
+    err_r = (an - nrm).abs().max(dim=1).values
+    den = torch.clamp(nrm.abs().max(dim=1).values, min=float(nrm.abs().max()) / 16.0)
+    assert float((err_r / den).max()) <= 2e-2
+    zw = nrm @ w.double()
+    assert float((z.double() - zw).abs().max() / zw.abs().max()) <= 2e-2
+
+
+def test_linear_residual_rmsnorm_head_only(G):
+    """The last block's form: no normalised rows written, only the head's logits."""
+    M, K, d = 333, 2048, 512
+    A = _bf((M, K), 11, 1.0)
+    Wt = _bf((d, K), 12, 1.0 / np.sqrt(K))
+    x = torch.randn((M, d), generator=torch.Generator(device="cuda").manual_seed(13),
+                    device="cuda")
+    x_np = x.double().cpu().numpy()
+    xo = torch.empty_like(x)
+    w = torch.randn(d, generator=torch.Generator(device="cuda").manual_seed(14), device="cuda")
+    z = torch.full((M,), float("nan"), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    G.linear_residual_rmsnorm(A, Wt, x, xo, None, err, w_head=w, z=z)
+    assert G.check_error(err) == 0
+    want = x_np + _np(A) @ _np(Wt).T
+    assert ref.rel_to_max(xo.double().cpu().numpy(), want) <= 1e-3
+    zw = _rms(want) @ w.double().cpu().numpy()
+    assert ref.rel_to_max(z.double().cpu().numpy(), zw) <= 2e-2
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_rmsnorm_parity(G, dtype):
     M, d = 777, 512

@@ -26,7 +26,8 @@
 //     and [256, 512), taking turns every 16 k-steps (the A rows of a chunk are re-read
 //     from L2, not DRAM): the first half completes a chunk early and its residual pass
 //     overlaps the second half's last MMAs, and each half's columns are released as soon
-//     as the normalisation has read them;
+//     as the normalisation has read them (for K >= 1024, as soon as the residual pass has
+//     read them, the normalisation then re-reading the stored fp32 rows by TMA);
 //   * warps 2-9 run the epilogue from TMEM, two warps per TMEM lane quadrant (one row
 //     per thread), each on half of a 256-column block; res+rms combines the two warps'
 //     row sums of squares (and head partial sums) through shared memory.  Outputs leave
@@ -59,6 +60,11 @@ constexpr uint32_t kStageBytes = kABytes + kBBytes;
 // tile's A rows are read from DRAM once (the other half's read of the chunk hits L2) and
 // the first half still completes one chunk ahead of the second
 constexpr int kChunkSteps = 16;
+// res+rms for long K (K >= kReleaseMinK): each TMEM half goes back to the MMAs as soon as
+// its residual pass has read it, and the normalisation re-reads the stored fp32 rows
+// (still in L2) by TMA, so the next tile's MMAs overlap the rest of the epilogue
+constexpr int kEpiResRmsRel = 3;
+constexpr int kReleaseMinK = 1024;
 constexpr uint32_t kBoxBytes = 2048;  // 32 rows x 64 bytes (32 bf16 or 16 fp32 columns)
 constexpr int kXBufs = 4;             // res+rms: residual boxes in flight per epilogue warp
 
@@ -147,7 +153,8 @@ GR_DEVICE void load_f32x32(const float* src, float4 (&x)[8]) {
 
 template <int kEpi>
 __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__ Params P) {
-  constexpr bool kRes = kEpi == kEpiResRms;
+  constexpr bool kRes = kEpi == kEpiResRms || kEpi == kEpiResRmsRel;
+  constexpr bool kRel = kEpi == kEpiResRmsRel;
   using L = Layout<kRes>;
   constexpr int kStages = L::kStages;
   constexpr int kHalves = kRes ? 2 : 1;  // 256-column blocks per tile
@@ -328,10 +335,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       }
     } else {
       // res+rms.  The warp's residual boxes (32 rows x 16 fp32 columns, 16 a tile: 8 per
-      // 256-column half) are numbered across its tiles; box n goes to buffer n % kXBufs,
+      // 256-column half; with the early release another 16 of the stored rows for the
+      // normalisation) are numbered across its tiles; box n goes to buffer n % kXBufs,
       // and the load of box n + kXBufs is issued as soon as box n has been read, so the
-      // next tile's first boxes load while this tile's normalisation runs.
-      constexpr int kPerTile = 16;
+      // next tile's first boxes load while this tile's normalisation runs.  A re-read of
+      // the stored rows is issued only once the tile's stores have completed.
+      constexpr int kPerTile = kRel ? 32 : 16;
       uint8_t* xb = smem + L::kOffBox + ew * kXBufs * kBoxBytes;
       uint64_t* xw = xbar + ew * kXBufs;
       const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
@@ -342,7 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         const int col = ((w >> 3) & 1) * BN + ch * 128 + (w & 7) * 16;
         const int b = n % kXBufs;
         mbar_expect_tx(&xw[b], kBoxBytes);
-        tma_load_2d(xb + b * kBoxBytes, &P.txi, &xw[b], col, t * BM + box_row);
+        tma_load_2d(xb + b * kBoxBytes, w < 16 ? (const void*)&P.txi : (const void*)&P.tx, &xw[b],
+                    col, t * BM + box_row);
       };
       int ld = 0;  // boxes whose loads were issued
       if (lane == 0)
@@ -351,11 +361,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       int n = 0;  // boxes consumed
       // waits for box n; false (the error recorded) when it timed out
       auto wait_box = [&](int x) { return wait_warp(&xw[x % kXBufs], par(x / kXBufs), abort_flag, g.err); };
-      // after box n has been read by every lane: the next load
-      auto next_load = [&]() {
+      // after box n has been read by every lane: the next load, unless it is a re-read
+      // of this tile's stored rows and the residual pass is still running
+      auto next_load = [&](bool pass1) {
         __syncwarp();
-        if (ld < nbox && lane == 0) issue(ld);
-        ++ld;
+        const bool go = ld < nbox && !(kRel && pass1 && (ld % kPerTile) >= 16);
+        if (go && lane == 0) issue(ld);
+        if (go) ++ld;
       };
       int tc = 0;
       // A failed (timed-out) wait skips the work but not the named barriers below, so the
@@ -405,8 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
               a[4 * e + 2] = __float_as_uint(y[e].z);
               a[4 * e + 3] = __float_as_uint(y[e].w);
             }
-            tmem_st16(lane_base + c0 + c, a);
-            next_load();
+            if (!kRel) tmem_st16(lane_base + c0 + c, a);
+            next_load(true);
             if (lane == 0) bulk_wait_read_all();  // the output box's previous store has read it
             __syncwarp();
 #pragma unroll
@@ -418,22 +430,48 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
               bulk_commit();
             }
           }
+          if (kRel && ok) {  // this half's accumulator columns go back to the MMAs
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[h]);
+          }
         }
         // the row's sum of squares over both warps of this quadrant
         red[ch * BM + rloc] = ss;
         named_bar_sync(1 + q, 64);
         const float r = rsqrtf((red[rloc] + red[BM + rloc]) / (float)g.N + g.eps);
+        if (kRel && ok) {
+          // the stored rows are re-read once the tile's stores have completed
+          if (lane == 0) bulk_wait_all();
+          for (int x = 0; x < kXBufs; ++x) next_load(false);
+        }
         // pass 2: the normalised row, to a_out in bf16 and into the head's dot product, 16
-        // columns a step (an a_out box takes two); each half's accumulator columns go back
-        // to the MMAs as soon as they have been read, so the next tile's first half overlaps
-        // this tile's second
+        // columns a step (an a_out box takes two); unless released already, each half's
+        // accumulator columns go back to the MMAs as soon as they have been read, so the
+        // next tile's first half overlaps this tile's second
         float z = 0.f;
         for (int h = 0; h < 2 && ok; ++h) {
           const int c0 = h * BN + ch * 128;
 #pragma unroll 1
           for (int c = 0; c < 128; c += 16) {
             float v[16];
-            {
+            if (kRel) {
+              if (!wait_box(n)) {
+                ok = false;
+                break;
+              }
+              const uint8_t* xs = xb + (n % kXBufs) * kBoxBytes;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float4 y = *reinterpret_cast<const float4*>(xs + sw64(lane, e));
+                v[4 * e] = y.x;
+                v[4 * e + 1] = y.y;
+                v[4 * e + 2] = y.z;
+                v[4 * e + 3] = y.w;
+              }
+              ++n;
+              next_load(false);
+            } else {
               uint32_t a[16];
               tmem_ld16_async(lane_base + c0 + c, a);
               tmem_ld_wait(a);
@@ -470,9 +508,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
               }
             }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[h]);
+          if (!kRel) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[h]);
+          }
         }
         if (g.w_head) {
           named_bar_sync(1 + q, 64);  // both warps have read the sums of squares
@@ -569,7 +609,7 @@ static bool make_map(CUtensorMap* m, const void* base, long long rows, int K, lo
          CUDA_SUCCESS;
 }
 
-static DeviceOnce gemm_smem_attr[3];
+static DeviceOnce gemm_smem_attr[4];
 
 // [rows][N] output (bf16 or fp32) with row stride ld elements, for TMA stores of 32-row
 // boxes of 64 bytes (32 bf16 or 16 fp32 columns) with the 64-byte swizzle.
@@ -593,7 +633,7 @@ static int launch_t(const GemmArgs& g, cudaStream_t st) {
   Params p;
   if (!make_map(&p.ta, g.a, g.M, g.K, g.lda, BM) || !make_map(&p.tb, g.w, g.N, g.K, g.ldw, BN))
     return GENRANK_ERR_CUDA;
-  if (kEpi == kEpiResRms) {
+  if (kEpi >= kEpiResRms) {
     if (!make_store_map(&p.tx, g.x_out, g.M, g.N, g.ldx, true) ||
         !make_store_map(&p.txi, const_cast<float*>(g.x_in), g.M, g.N, g.ldx, true) ||
         (g.a_out && !make_store_map(&p.tc, g.a_out, g.M, g.N, g.lda_out, false)))
@@ -602,13 +642,13 @@ static int launch_t(const GemmArgs& g, cudaStream_t st) {
     return GENRANK_ERR_CUDA;
   }
   p.g = g;
-  constexpr int kSmem = (int)Layout<kEpi == kEpiResRms>::kSmem;
+  constexpr int kSmem = (int)Layout<kEpi >= kEpiResRms>::kSmem;
   if (!set_smem_limit_once(gemm_smem_attr[kEpi], (const void*)k_gemm_tc<kEpi>, kSmem))
     return GENRANK_ERR_CUDA;
   const int sms = sm_count_current();
   if (sms <= 0) return GENRANK_ERR_CUDA;
   const long long tiles =
-      (long long)((g.M + BM - 1) / BM) * (kEpi == kEpiResRms ? 1 : g.N / BN);
+      (long long)((g.M + BM - 1) / BM) * (kEpi >= kEpiResRms ? 1 : g.N / BN);
   const int grid = (int)(tiles < sms ? tiles : sms);
   k_gemm_tc<kEpi><<<grid, kThreads, kSmem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
@@ -622,7 +662,8 @@ int launch_gemm_tc(const GemmArgs& g, cudaStream_t st) {
   switch (g.epilogue) {
     case kEpiStore: return launch_t<kEpiStore>(g, st);
     case kEpiSilu: return launch_t<kEpiSilu>(g, st);
-    case kEpiResRms: return launch_t<kEpiResRms>(g, st);
+    case kEpiResRms:
+      return g.K >= kReleaseMinK ? launch_t<kEpiResRmsRel>(g, st) : launch_t<kEpiResRms>(g, st);
     default: return GENRANK_ERR_INVALID_ARG;
   }
 }

@@ -36,6 +36,7 @@
 #include <cudaTypedefs.h>
 
 #include <climits>
+#include <type_traits>
 
 #include "common.cuh"
 #include "host_util.h"
@@ -973,7 +974,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       const uint32_t o_addr = lane_base + kColO + ob * DH;
       float m = rowcb, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < it.nt; ++j, ++g) {
+      // One key tile: the per-row mask can only reach the first tile an item visits
+      // (its diagonal history tile, or the last, partial history tile of a candidate
+      // tile), so that tile runs the masked form and every later one the plain form;
+      // the plain loop then holds a single copy of the tile code.
+      auto step = [&](int j, auto masked_form) -> bool {
+        constexpr bool kM = decltype(masked_form)::value;
         const int sb = g & 1, st = g % kStages;
         // dense bias: this thread's 64 values of the tile (one 128-byte line), requested
         // before the wait for S so that the load overlaps it
@@ -991,38 +997,54 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
         // S_g's commit also covers every MMA issued before it, P_{g-2} V_{g-2} included,
         // so once S_g is here its P buffer is free as well
         if (!wait_warp(&bars[kSFull + sb], par(g >> 1), abort_flag, a.err) ||
-            !wait_warp(&bars[kKFull + st], par(g / kStages), abort_flag, a.err)) {
-          ok = false;
-          break;
-        }
+            !wait_warp(&bars[kKFull + st], par(g / kStages), abort_flag, a.err))
+          return false;
         tc_fence_after();
         const uint32_t s_addr = lane_base + kColS + sb * BN;
         const uint32_t p_addr = lane_base + kColP + sb * (BN / 2);
         uint64_t* prev_pv = &bars[kPFree + ((g + 1) & 1)];
         const uint32_t prev_ph = par((g - 1) >> 1);
+        bool done;
         if (j < it.nk) {
           const int kv0 = (it.nk - 1 - j) * BN;  // most recent keys first
-          const bool masked = kv0 + BN - 1 > mask_from;
-          const int nvalid = masked ? max(0, min(BN, lim - kv0 + 1)) : BN;
           const float* cb = sCB + st * BN + kHalf * h;
           if (kBucket) tb.tr = sTR + st * BN + kHalf * h;
-          ok = masked ? softmax_tile<true, kBucket, kDense>(
-                            s_addr, p_addr, o_addr, cb, tb, bw, kHalf * h, nvalid, scale_log2,
-                            j == 0, row_ok, m, l, prev_pv, prev_ph, abort_flag, a.err)
-                      : softmax_tile<false, kBucket, kDense>(
-                            s_addr, p_addr, o_addr, cb, tb, bw, kHalf * h, nvalid, scale_log2,
-                            j == 0, row_ok, m, l, prev_pv, prev_ph, abort_flag, a.err);
+          if constexpr (kM) {
+            // keys past the row's last visible key are masked (none on an unmasked tile)
+            const int nvalid = max(0, min(BN, lim - kv0 + 1));
+            done = softmax_tile<true, kBucket, kDense>(
+                s_addr, p_addr, o_addr, cb, tb, bw, kHalf * h, nvalid, scale_log2, j == 0,
+                row_ok, m, l, prev_pv, prev_ph, abort_flag, a.err);
+          } else {
+            if (kv0 + BN - 1 > mask_from) flag(a.err, GENRANK_DERR_LAYOUT);  // not reachable
+            done = softmax_tile<false, kBucket, kDense>(
+                s_addr, p_addr, o_addr, cb, tb, bw, kHalf * h, BN, scale_log2, j == 0,
+                row_ok, m, l, prev_pv, prev_ph, abort_flag, a.err);
+          }
         } else {
-          ok = softmax_diag(s_addr, p_addr, o_addr, rt, h, cand_row, rowcb, scale_log2, j == 0,
-                            m, l, prev_pv, prev_ph, abort_flag, a.err, diagb);
+          done = softmax_diag(s_addr, p_addr, o_addr, rt, h, cand_row, rowcb, scale_log2,
+                              j == 0, m, l, prev_pv, prev_ph, abort_flag, a.err, diagb);
         }
-        if (!ok) break;
+        if (!done) return false;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&bars[kSFree + sb]);
           mbar_arrive(&bars[kPFull + sb]);
         }
+        return true;
+      };
+      if constexpr (kDense) {  // one loop: peeling adds spills to this form's larger state
+        for (int j = 0; ok && j < it.nt; ++j, ++g)
+          ok = (j < it.nk && (it.nk - 1 - j) * BN + BN - 1 > mask_from)
+                   ? step(j, std::true_type{})
+                   : step(j, std::false_type{});
+      } else {
+        if (it.nt > 0) {
+          ok = step(0, std::true_type{});
+          ++g;
+        }
+        for (int j = 1; ok && j < it.nt; ++j, ++g) ok = step(j, std::false_type{});
       }
       if (!ok) break;
       // hand the row's softmax state to the epilogue with the O buffer

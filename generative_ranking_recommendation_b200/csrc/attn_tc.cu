@@ -244,6 +244,14 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue(const __grid_constan
           cbias[(long long)h * Tp + base + i] = kLog2e * (a.slope_pos[h] * p + a.slope_time[h] * dt);
       }
     }
+    // the entries up to the next user's segment (up to the end for the last user) are
+    // zeroed: a key tile reads up to 127 entries past a user's last token, and the
+    // attention kernel relies on every entry it reads being finite
+    const long long next = b + 1 < a.B ? seg_start(e, b + 1) : Tp;
+    for (long long i = base + L + threadIdx.x; i < next; i += blockDim.x) {
+      if (trel) trel[i] = 0;
+      for (int h = 0; h < a.H; ++h) cbias[(long long)h * Tp + i] = 0.f;
+    }
     return;
   }
   __shared__ int hist[kMaxTileBuckets];
@@ -354,6 +362,18 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue_cached(
       const long long at = base + (i < n ? i : n4 + (i - n));
       for (int h = 0; h < a.H; ++h)
         cbias[(long long)h * Tp + at] = kLog2e * (a.slope_pos[h] * pf + a.slope_time[h] * dt);
+    }
+    // the padding after the history and the entries up to the next user's segment (up
+    // to the end for the last user) are zeroed: the attention kernel relies on every
+    // column term a key tile reads being finite
+    long long next = Tp;
+    if (b + 1 < a.B) {
+      int cs1, n1, m1, hs1;
+      if (cached_user(c, b + 1, cs1, n1, m1, hs1)) next = seg_start_cached((long long)hs1 + cs1, b + 1);
+    }
+    for (long long i = base + n + threadIdx.x; i < next; i += blockDim.x) {
+      if (i >= base + n4 && i < base + n4 + m) continue;
+      for (int h = 0; h < a.H; ++h) cbias[(long long)h * Tp + i] = 0.f;
     }
     return;
   }
@@ -521,16 +541,15 @@ GR_DEVICE void row_max_chunk(const uint32_t (&s)[CW], const float* cb, const TB&
   }
 }
 
-// p = 2^(x - m) for CW columns, summed into two pairs of partial sums, packed to
-// bf16 pairs and stored (without waiting) to CW / 2 TMEM columns at taddr.  The
-// bias and scale arithmetic runs on column pairs (two-wide fp32 instructions).
+// p = 2^(x - m) for CW columns, summed into two pairs of partial sums and packed to
+// bf16 pairs in pk.  The bias and scale arithmetic runs on column pairs (two-wide fp32
+// instructions).
 template <bool kMasked, bool kBucket, bool kDense>
-GR_DEVICE void exp_pack_store(const uint32_t (&s)[CW], const float* cb, const TB& tb,
-                              const uint32_t* bw, int kc0, int nvalid, float scale_log2,
-                              float m_use, uint64_t (&rs2)[2], uint32_t taddr) {
+GR_DEVICE void exp_pack(const uint32_t (&s)[CW], const float* cb, const TB& tb,
+                        const uint32_t* bw, int kc0, int nvalid, float scale_log2, float m_use,
+                        uint64_t (&rs2)[2], uint32_t (&pk)[CW / 2]) {
   const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
   const uint64_t m2 = f2_pack(m_use, m_use);
-  uint32_t pk[CW / 2];
 #pragma unroll
   for (int c = 0; c < CW; c += 4) {
     uint64_t t01, t23;
@@ -563,6 +582,33 @@ GR_DEVICE void exp_pack_store(const uint32_t (&s)[CW], const float* cb, const TB
     rs2[1] = f2_add(rs2[1], f2_pack(p[2], p[3]));
     pk[c / 2] = pack_bf16(p[0], p[1]);
     pk[c / 2 + 1] = pack_bf16(p[2], p[3]);
+  }
+}
+
+// One chunk of P: computed, then stored (without waiting) to CW / 2 TMEM columns at
+// taddr.  A masked tile's chunk is, for each thread, wholly visible (the plain code),
+// wholly masked (zeros, no exponentials) or the one chunk the row's mask cuts: there
+// the masked keys' scores become -inf, so that 2^(x - m) = +0 for them (their column
+// terms are finite: the prologue writes every entry a key tile can read).  The dense
+// form keeps a select per key (its bias rows past a user's end are the caller's).  The
+// branches only compute, so the warp is converged again for the store.
+template <bool kMasked, bool kBucket, bool kDense>
+GR_DEVICE void exp_pack_store(uint32_t (&s)[CW], const float* cb, const TB& tb,
+                              const uint32_t* bw, int kc0, int nvalid, float scale_log2,
+                              float m_use, uint64_t (&rs2)[2], uint32_t taddr) {
+  uint32_t pk[CW / 2];
+  if (kDense || !kMasked) {
+    exp_pack<kMasked, kBucket, kDense>(s, cb, tb, bw, kc0, nvalid, scale_log2, m_use, rs2, pk);
+  } else if (kc0 >= nvalid) {
+#pragma unroll
+    for (int k = 0; k < CW / 2; ++k) pk[k] = 0u;
+  } else {
+    if (kc0 + CW > nvalid) {
+#pragma unroll
+      for (int e = 0; e < CW; ++e)
+        if (kc0 + e >= nvalid) s[e] = 0xff800000u;  // -inf
+    }
+    exp_pack<false, kBucket, kDense>(s, cb, tb, bw, kc0, nvalid, scale_log2, m_use, rs2, pk);
   }
   p_store(taddr, pk);
 }

@@ -735,25 +735,24 @@ GR_DEVICE bool softmax_tile(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, c
 
 // The diagonal tile: S = Q K^T over the item's own rows, of which a candidate row
 // keeps only its own key (position and time differences 0, so the bias is 0 and the
-// score is relative to c_i).  P is zero but for that key; the offset moves (O
-// rescaled) only if the term would overflow, or is set exactly on a first tile.
+// score is relative to c_i).  A warp's 16 rows have their own keys in one 16-key chunk
+// of one half of the tile, so only that chunk is read (by the threads of that half) and
+// P is zero elsewhere.  The offset moves (O rescaled) only if the term would overflow,
+// or is set exactly on a first tile.
 GR_DEVICE bool softmax_diag(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, int rt, int h,
                             bool cand_row, float rowcb, float scale_log2, bool first, float& m,
                             float& l, uint64_t* prev_pv, uint32_t prev_ph,
                             volatile int* abort_flag, int32_t* err, float diagb = 0.f) {
-  uint32_t xa[32], xb[32];
-  tmem_ld_half32_async<kHalf>(s_addr, xa);
-  tmem_ld_half32_async<kHalf>(s_addr + 32, xb);
-  tmem_ld_wait(xa);
-  tmem_ld_wait(xb);
-  const int col = rt - kHalf * h;  // the row's own key within this half
-  const bool mine = cand_row && col >= 0 && col < kHalf;
+  const int r0 = rt & ~15;  // the warp's first row
+  const int c0 = r0 & (kHalf - 1);  // their own keys: columns [r0, r0 + 16), in half r0 / 64
+  uint32_t x[16];
+  tmem_ld_half16_async<kHalf>(s_addr + c0, x);
+  tmem_ld_wait(x);
+  const bool mine = cand_row && h == r0 / kHalf;
+  const int e = rt & 15;
   float sv = 0.f;
 #pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    sv = col == c ? __uint_as_float(xa[c]) : sv;
-    sv = col == c + 32 ? __uint_as_float(xb[c]) : sv;
-  }
+  for (int c = 0; c < 16; ++c) sv = e == c ? __uint_as_float(x[c]) : sv;
   const float xm = mine ? fmaf(sv, scale_log2, rowcb + diagb) : -INFINITY;
   const float xr = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 16));  // the row's self score
   const bool move = xr > -INFINITY && (first || xr - m > 100.f);
@@ -764,11 +763,22 @@ GR_DEVICE bool softmax_diag(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, i
   }
   if (move) m = xr;
   const float p = mine ? ex2(xm - m) : 0.f;
-  const uint32_t word = (col & 1) ? pack_bf16(0.f, p) : pack_bf16(p, 0.f);
-  uint32_t pk[32];
+  const uint32_t word = (e & 1) ? pack_bf16(0.f, p) : pack_bf16(p, 0.f);
+  uint32_t pk[8], zero[8];
 #pragma unroll
-  for (int k = 0; k < 32; ++k) pk[k] = (mine && k == (col >> 1)) ? word : 0u;
-  tmem_st_half32_nowait<kHalf / 2>(p_addr, pk);
+  for (int k = 0; k < 8; ++k) {
+    pk[k] = (mine && k == (e >> 1)) ? word : 0u;
+    zero[k] = 0u;
+  }
+  // the half's 32 P columns in four stores of 8: the own-key chunk, zeros elsewhere
+  // (c0 is the same for the whole warp, so the branch does not diverge)
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (k * 16 == c0)
+      tmem_st_half8_nowait<kHalf / 2>(p_addr + 8 * k, pk);
+    else
+      tmem_st_half8_nowait<kHalf / 2>(p_addr + 8 * k, zero);
+  }
   tmem_wait_st();
   l = first ? p : l + p;
   return true;

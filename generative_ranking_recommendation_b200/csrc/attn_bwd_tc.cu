@@ -46,6 +46,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "host_util.h"
 #include "kernels.h"
@@ -577,6 +579,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
       const bool key = j < rc.n;
       const float cbj = key ? P.cbias[(long long)rc.h * P.Tp + rc.spad + j] : 0.f;
       const uint64_t sl2 = f2_pack(scale_log2, scale_log2), cb2 = f2_pack(cbj, cbj);
+      // on a query tile wholly inside the user and past the diagonal every query sees
+      // every key row, so only the key row's own validity is left: a row past the
+      // user's history gets c_j = -inf there, and 2^-inf = 0 needs no select
+      const float cbf = key ? cbj : -INFINITY;
+      const uint64_t cb2f = f2_pack(cbf, cbf);
       // bucketed time bias: this key's time, biased (see kTimeMagic), and -m_t log2 e
       const int tj_m = kBucket && key ? kTimeMagic - P.trel[rc.spad + j] : 0;
       const float nmt2 = kBucket ? -a.slope_time[rc.h] * kLog2e : 0.f;
@@ -622,14 +629,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
           // arithmetic on column pairs (two-wide fp32 instructions).  P^T goes over the
           // first 16 S^T columns this thread has read (16x32bx2: the upper lanes at
           // +32), dS^T to shared memory.
-          auto chunk = [&](const uint32_t (&sv)[16], const uint32_t (&dp)[16], int c0) {
+          auto chunk = [&](const uint32_t (&sv)[16], const uint32_t (&dp)[16], int c0,
+                           auto full_tile) {
+            constexpr bool kFull = decltype(full_tile)::value;
             uint32_t pk[8], dk[8];
 #pragma unroll
             for (int c = 0; c < 16; c += 4) {
               const float4 l4 = *reinterpret_cast<const float4*>(l2 + c0 + c);
               const float4 d4 = *reinterpret_cast<const float4*>(dd + c0 + c);
-              uint64_t t01 = f2_sub(cb2, f2_pack(l4.x, l4.y));
-              uint64_t t23 = f2_sub(cb2, f2_pack(l4.z, l4.w));
+              uint64_t t01 = f2_sub(kFull ? cb2f : cb2, f2_pack(l4.x, l4.y));
+              uint64_t t23 = f2_sub(kFull ? cb2f : cb2, f2_pack(l4.z, l4.w));
               if (kBucket) {  // - m_t bucket(t_i - t_j), four queries at a time
                 const int4 ti = *reinterpret_cast<const int4*>(tq + c0 + c);
                 const uint64_t two23 = f2_pack(kTwo23, kTwo23);
@@ -662,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int i = qbase + c0 + c + e;
-                p[e] = (key && i >= ilo && i < ihi) ? ex2(xv[e]) : 0.f;
+                p[e] = (kFull || (key && i >= ilo && i < ihi)) ? ex2(xv[e]) : 0.f;
               }
               const uint64_t p01 = f2_pack(p[0], p[1]), p23 = f2_pack(p[2], p[3]);
               const uint64_t ds01 = f2_mul(
@@ -682,10 +691,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_bwd_tc(const __grid_consta
             tmem_st_half8_nowait<32>(s_addr + c0 / 2, pk);
             store_row_chunk16(sDSb, r, qc + c0, dk);
           };
-          chunk(sa, da, 0);  // stores to columns [0, 8): read, not in flight
-          tmem_ld_wait(sb);
-          tmem_ld_wait(db);
-          chunk(sb, db, 16);  // stores to columns [8, 16)
+          auto both = [&](auto full_tile) {
+            chunk(sa, da, 0, full_tile);  // stores to columns [0, 8): read, not in flight
+            tmem_ld_wait(sb);
+            tmem_ld_wait(db);
+            chunk(sb, db, 16, full_tile);  // stores to columns [8, 16)
+          };
+          // the same for the whole warp: the record's tile t and the user's length (the
+          // bucketed form keeps one copy of the chunk code: a second one spills there)
+          if (!kBucket && t > 0 && q0 + BM <= ihi)
+            both(std::true_type{});
+          else
+            both(std::false_type{});
           tmem_wait_st();
           fence_proxy_async_smem();
           tc_fence_before();

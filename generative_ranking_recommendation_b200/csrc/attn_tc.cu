@@ -1095,6 +1095,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
           ok = (j < it.nk && (it.nk - 1 - j) * BN + BN - 1 > mask_from)
                    ? step(j, std::true_type{})
                    : step(j, std::false_type{});
+      } else if constexpr (kBucket) {
+        // one copy of the tile code for every tile (faster for this form than a peeled
+        // first tile): an unmasked tile has nvalid = 128 and takes the visible-chunk
+        // branch throughout
+        for (int j = 0; ok && j < it.nt; ++j, ++g) ok = step(j, std::true_type{});
       } else {
         if (it.nt > 0) {
           ok = step(0, std::true_type{});

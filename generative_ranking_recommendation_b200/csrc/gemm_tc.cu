@@ -145,12 +145,6 @@ GR_DEVICE void box_bf16x16(uint8_t* box, int r, int half, const float* v) {
                    pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
 }
 
-GR_DEVICE void load_f32x32(const float* src, float4 (&x)[8]) {
-  const float4* s4 = reinterpret_cast<const float4*>(src);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) x[e] = s4[e];
-}
-
 template <int kEpi>
 __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__ Params P) {
   constexpr bool kRes = kEpi == kEpiResRms || kEpi == kEpiResRmsRel;

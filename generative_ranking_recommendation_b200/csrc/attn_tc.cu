@@ -448,9 +448,14 @@ GR_DEVICE bool wait_warp(uint64_t* bar, uint32_t ph, volatile int* abort_flag, i
 constexpr int kHalf = BN / 2;
 constexpr int CW = 16;  // key columns per chunk (of the thread's 64)
 GR_DEVICE void s_load(uint32_t taddr, uint32_t (&r)[CW]) { tmem_ld_half16_async<kHalf>(taddr, r); }
+template <int kOff = kHalf / 2>
 GR_DEVICE void p_store(uint32_t taddr, const uint32_t (&pk)[CW / 2]) {
-  tmem_st_half8_nowait<kHalf / 2>(taddr, pk);
+  tmem_st_half8_nowait<kOff>(taddr, pk);
 }
+// A masked tile can instead interleave the halves by 16-key chunks: threads 0-15 take
+// the even chunks, threads 16-31 the odd ones, so that the two halves of a warp agree
+// on which chunks a row's mask leaves visible or hides (but for the chunk it cuts).
+GR_DEVICE void s_load_il(uint32_t taddr, uint32_t (&r)[CW]) { tmem_ld_half16_async<CW>(taddr, r); }
 
 // The bucketed time bias of one softmax thread: the key times of its columns (shared
 // memory, indexed like the column terms), its row's time + kTimeMagic, and -m_t log2 e
@@ -592,7 +597,7 @@ GR_DEVICE void exp_pack(const uint32_t (&s)[CW], const float* cb, const TB& tb,
 // terms are finite: the prologue writes every entry a key tile can read).  The dense
 // form keeps a select per key (its bias rows past a user's end are the caller's).  The
 // branches only compute, so the warp is converged again for the store.
-template <bool kMasked, bool kBucket, bool kDense>
+template <bool kMasked, bool kBucket, bool kDense, int kPOff = kHalf / 2>
 GR_DEVICE void exp_pack_store(uint32_t (&s)[CW], const float* cb, const TB& tb,
                               const uint32_t* bw, int kc0, int nvalid, float scale_log2,
                               float m_use, uint64_t (&rs2)[2], uint32_t taddr) {
@@ -610,7 +615,7 @@ GR_DEVICE void exp_pack_store(uint32_t (&s)[CW], const float* cb, const TB& tb,
     }
     exp_pack<false, kBucket, kDense>(s, cb, tb, bw, kc0, nvalid, scale_log2, m_use, rs2, pk);
   }
-  p_store(taddr, pk);
+  p_store<kPOff>(taddr, pk);
 }
 
 // Maximum of x over this thread's half of the tile (S at s_addr, column terms of the
@@ -654,6 +659,32 @@ GR_DEVICE float tile_exp(uint32_t s_addr, uint32_t p_addr, const float* cb, cons
                          const DB& db, int kbase, int nvalid, float scale_log2, float m) {
   uint64_t rs2[2] = {0ull, 0ull};  // (+0, +0) pairs
   uint32_t xa[CW], xb[CW];
+  if constexpr (kMasked && !kDense) {
+    // the halves interleaved by chunks (see s_load_il); P lands in the same columns
+    const int hh = kbase / kHalf;
+    const float* cbr = cb - kbase;  // the row's column terms
+    const TB tbr = tb.at(-kbase);
+    s_load_il(s_addr, xa);
+    tmem_ld_wait(xa);
+#pragma unroll
+    for (int k = 0; k < 4; k += 2) {
+      s_load_il(s_addr + 2 * CW * (k + 1), xb);
+      const int ka = 2 * CW * k + CW * hh;
+      exp_pack_store<true, kBucket, false, CW / 2>(xa, cbr + ka, tbr.at(ka), nullptr, ka, nvalid,
+                                                   scale_log2, m, rs2, p_addr + CW * k);
+      tmem_ld_wait(xb);
+      if (k + 2 < 4) s_load_il(s_addr + 2 * CW * (k + 2), xa);
+      const int kb = 2 * CW * (k + 1) + CW * hh;
+      exp_pack_store<true, kBucket, false, CW / 2>(xb, cbr + kb, tbr.at(kb), nullptr, kb, nvalid,
+                                                   scale_log2, m, rs2, p_addr + CW * (k + 1));
+      if (k + 2 < 4) tmem_ld_wait(xa);
+    }
+    tmem_wait_st();
+    float r0, r1, r2, r3;
+    f2_unpack(rs2[0], r0, r1);
+    f2_unpack(rs2[1], r2, r3);
+    return (r0 + r1) + (r2 + r3);
+  }
   uint32_t w1[kDense ? 16 : 1];
   s_load(s_addr, xa);
   tmem_ld_wait(xa);
@@ -1095,11 +1126,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
           ok = (j < it.nk && (it.nk - 1 - j) * BN + BN - 1 > mask_from)
                    ? step(j, std::true_type{})
                    : step(j, std::false_type{});
-      } else if constexpr (kBucket) {
-        // one copy of the tile code for every tile (faster for this form than a peeled
-        // first tile): an unmasked tile has nvalid = 128 and takes the visible-chunk
-        // branch throughout
-        for (int j = 0; ok && j < it.nt; ++j, ++g) ok = step(j, std::true_type{});
       } else {
         if (it.nt > 0) {
           ok = step(0, std::true_type{});

@@ -203,6 +203,32 @@ int genrank_embed_assemble(int B, int64_t T, const int32_t* seq_offsets, const i
   return launch_embed_fwd(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int genrank_embed_assemble_rmsnorm(int B, int64_t T, const int32_t* seq_offsets,
+                                   const int32_t* hist_len, const int32_t* item_ids,
+                                   const int32_t* action_ids, const int64_t* ts,
+                                   const void* item_tab, int64_t n_item, const void* action_tab,
+                                   int n_action, const void* pos_tab, int n_pos,
+                                   const void* ri_tab, int n_ri, const void* rt_tab, int n_rt,
+                                   int d, float* x_out, void* a_out, float eps, int32_t* pos,
+                                   int32_t* req_idx, int32_t* rt_bucket, int32_t* dev_err,
+                                   genrank_stream_t stream) {
+  if (B < 1 || T < 0 || !seq_offsets || !hist_len || !dev_err || d < 1 || !(eps >= 0.f))
+    return GENRANK_ERR_INVALID_ARG;
+  if (n_item < 1 || n_action < 1 || n_pos < 2 || n_ri < 2 || n_rt < 2)
+    return GENRANK_ERR_INVALID_ARG;
+  if (n_rt > 65 || d != 512) return GENRANK_ERR_UNSUPPORTED;
+  if (T > 0 && (!item_ids || !action_ids || !ts || !item_tab || !action_tab || !pos_tab ||
+                !ri_tab || !rt_tab || !x_out || !a_out || !pos || !req_idx || !rt_bucket))
+    return GENRANK_ERR_INVALID_ARG;
+  if (!aligned16(item_tab) || !aligned16(action_tab) || !aligned16(pos_tab) ||
+      !aligned16(ri_tab) || !aligned16(rt_tab) || !aligned16(x_out) || !aligned16(a_out))
+    return GENRANK_ERR_INVALID_ARG;
+  EmbedFwdArgs a{B, T, seq_offsets, hist_len, item_ids, action_ids, ts, item_tab, n_item,
+                 action_tab, n_action, pos_tab, n_pos, ri_tab, n_ri, rt_tab, n_rt, d, GENRANK_BF16,
+                 nullptr, pos, req_idx, rt_bucket, dev_err, x_out, a_out, eps};
+  return launch_embed_fwd(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int genrank_embed_assemble_bwd(int B, int64_t T, const int32_t* seq_offsets,
                                const int32_t* hist_len, const int32_t* item_ids,
                                const int32_t* action_ids, const int32_t* pos,

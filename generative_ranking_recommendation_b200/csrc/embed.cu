@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(256) k_token_meta(
 // rows with 16-byte vector loads, the row indices broadcast from their lanes by
 // shuffles, two tokens' loads in flight together.  The rows are summed in fp32 and
 // rounded once.  At most 64 registers per thread keep four blocks resident per SM.
-template <typename T>
+template <typename T, bool kNorm>
 __global__ void __launch_bounds__(256, 4) k_embed_fwd(
     int B, long long Ttok, const int32_t* __restrict__ off, const int32_t* __restrict__ hist_len,
     const int32_t* __restrict__ item_ids, const int32_t* __restrict__ action_ids,
@@ -128,7 +128,8 @@ __global__ void __launch_bounds__(256, 4) k_embed_fwd(
     int n_action, const T* __restrict__ pos_tab, const T* __restrict__ ri_tab,
     const T* __restrict__ rt_tab, int d, int n_pos, int n_ri, int n_rt,
     const int32_t* __restrict__ pos, const int32_t* __restrict__ req_idx,
-    const int32_t* __restrict__ rt_bucket, T* __restrict__ E, int tokens_per_warp, int32_t* err) {
+    const int32_t* __restrict__ rt_bucket, T* __restrict__ E, int tokens_per_warp, int32_t* err,
+    float* __restrict__ x_out = nullptr, T* __restrict__ a_out = nullptr, float eps = 0.f) {
   constexpr int V = Elem<T>::kPerVec;
   constexpr int U = 2;  // tokens whose row gathers are in flight together
   const int lane = threadIdx.x & 31;
@@ -171,6 +172,61 @@ __global__ void __launch_bounds__(256, 4) k_embed_fwd(
       }
     }
     const int nt = (int)min(32LL, tend - t0);
+    if constexpr (kNorm) {
+      // one token at a time: the lane's two 8-column vectors of the row (d = 512) are
+      // summed, rounded to the table type (E's value), written as the fp32 x row, and
+      // normalised with the row's sum of squares (the same lanes, order and
+      // reduction as the RMSNorm pass over E, so the result is the same bit for bit)
+      for (int k = 0; k < nt; ++k) {
+        const uint4* rw[5];
+        rw[0] = reinterpret_cast<const uint4*>(item_tab + __shfl_sync(0xffffffffu, it, k) * d);
+        rw[1] = reinterpret_cast<const uint4*>(action_tab +
+                                               (long long)__shfl_sync(0xffffffffu, a, k) * d);
+        rw[2] = reinterpret_cast<const uint4*>(pos_tab +
+                                               (long long)__shfl_sync(0xffffffffu, p, k) * d);
+        rw[3] = reinterpret_cast<const uint4*>(ri_tab +
+                                               (long long)__shfl_sync(0xffffffffu, r, k) * d);
+        rw[4] = reinterpret_cast<const uint4*>(rt_tab +
+                                               (long long)__shfl_sync(0xffffffffu, b, k) * d);
+        uint4 xv[2][5];
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+#pragma unroll
+          for (int c = 0; c < 5; ++c) xv[w][c] = __ldg(rw[c] + lane + 32 * w);
+        float f[2][V];
+        float ss = 0.f;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          float g[V];
+          Elem<T>::unpack(xv[w][0], f[w]);
+#pragma unroll
+          for (int c = 1; c < 5; ++c) {
+            Elem<T>::unpack(xv[w][c], g);
+#pragma unroll
+            for (int e = 0; e < V; ++e) f[w][e] += g[e];
+          }
+          Elem<T>::unpack(Elem<T>::pack(f[w]), f[w]);  // E's rounded value
+#pragma unroll
+          for (int e = 0; e < V; ++e) ss = fmaf(f[w][e], f[w][e], ss);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float rn = rsqrtf(ss / (float)d + eps);
+        const long long row = t0 + k;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int c0 = (lane + 32 * w) * V;
+          float4* xo = reinterpret_cast<float4*>(x_out + row * d + c0);
+#pragma unroll
+          for (int e = 0; e < V; e += 4)
+            xo[e / 4] = make_float4(f[w][e], f[w][e + 1], f[w][e + 2], f[w][e + 3]);
+          float h[V];
+#pragma unroll
+          for (int e = 0; e < V; ++e) h[e] = f[w][e] * rn;
+          *reinterpret_cast<uint4*>(a_out + row * d + c0) = Elem<T>::pack(h);
+        }
+      }
+    } else {
     // the warp gathers the tokens' rows U at a time, indices broadcast from their lanes
     for (int k = 0; k < nt; k += U) {
       const uint4* rows[U][5];
@@ -207,6 +263,7 @@ __global__ void __launch_bounds__(256, 4) k_embed_fwd(
           if (k + q < nt) reinterpret_cast<uint4*>(E + (t0 + k + q) * d)[v] = Elem<T>::pack(f);
         }
       }
+    }
     }
   }
 }
@@ -359,16 +416,23 @@ int launch_embed_fwd(const EmbedFwdArgs& a, cudaStream_t st) {
   int tpw = 32 * (int)max(1LL, (a.T + 32 * warps_target - 1) / (32 * warps_target));
   long long warps = (a.T + tpw - 1) / tpw;
   long long blocks = (warps + 7) / 8;
-  if (a.dtype == GENRANK_BF16) {
+  if (a.x_out) {  // bf16 tables, d = 512 (checked by the caller)
     using T = __nv_bfloat16;
-    k_embed_fwd<T><<<(unsigned)blocks, 256, 0, st>>>(
+    k_embed_fwd<T, true><<<(unsigned)blocks, 256, 0, st>>>(
+        a.B, a.T, a.off, a.hist_len, a.item_ids, a.action_ids, (const T*)a.item_tab, a.n_item,
+        (const T*)a.action_tab, a.n_action, (const T*)a.pos_tab, (const T*)a.ri_tab,
+        (const T*)a.rt_tab, a.d, a.n_pos, a.n_ri, a.n_rt, a.pos, a.req_idx, a.rt_bucket, nullptr,
+        tpw, a.err, a.x_out, (T*)a.a_out, a.eps);
+  } else if (a.dtype == GENRANK_BF16) {
+    using T = __nv_bfloat16;
+    k_embed_fwd<T, false><<<(unsigned)blocks, 256, 0, st>>>(
         a.B, a.T, a.off, a.hist_len, a.item_ids, a.action_ids, (const T*)a.item_tab, a.n_item,
         (const T*)a.action_tab, a.n_action, (const T*)a.pos_tab, (const T*)a.ri_tab,
         (const T*)a.rt_tab, a.d, a.n_pos, a.n_ri, a.n_rt, a.pos, a.req_idx, a.rt_bucket, (T*)a.E,
         tpw, a.err);
   } else {
     using T = float;
-    k_embed_fwd<T><<<(unsigned)blocks, 256, 0, st>>>(
+    k_embed_fwd<T, false><<<(unsigned)blocks, 256, 0, st>>>(
         a.B, a.T, a.off, a.hist_len, a.item_ids, a.action_ids, (const T*)a.item_tab, a.n_item,
         (const T*)a.action_tab, a.n_action, (const T*)a.pos_tab, (const T*)a.ri_tab,
         (const T*)a.rt_tab, a.d, a.n_pos, a.n_ri, a.n_rt, a.pos, a.req_idx, a.rt_bucket, (T*)a.E,

@@ -32,6 +32,11 @@ struct EmbedFwdArgs {
   int32_t* req_idx;
   int32_t* rt_bucket;
   int32_t* err;
+  // with x_out: instead of E, the fp32 copy of E's rows (x_out) and their RMSNorm in
+  // bf16 (a_out), the first block's input (bf16 tables, d = 512)
+  float* x_out = nullptr;
+  void* a_out = nullptr;
+  float eps = 0.f;
 };
 
 struct EmbedBwdArgs {

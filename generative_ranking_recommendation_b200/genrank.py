@@ -25,7 +25,8 @@ DERR = {
 # every entry point declared in include/genrank.h
 EXPORTS = (
     "genrank_status_string", "genrank_device_error_string", "genrank_check_error",
-    "genrank_alibi_slopes", "genrank_embed_assemble", "genrank_embed_assemble_bwd",
+    "genrank_alibi_slopes", "genrank_embed_assemble", "genrank_embed_assemble_rmsnorm",
+    "genrank_embed_assemble_bwd",
     "genrank_attn_fwd", "genrank_attn_bwd", "genrank_attn_workspace_size",
     "genrank_attn_fwd_static", "genrank_candidate_logits", "genrank_attn_fwd_cached",
     "genrank_attn_cached_workspace_size", "genrank_attn_fwd_bucketed",
@@ -64,6 +65,10 @@ def lib():
         L.genrank_embed_assemble.argtypes = [
             _I, _L, _P, _P, _P, _P, _P, _P, _L, _P, _I, _P, _I, _P, _I, _P, _I, _I, _I,
             _P, _P, _P, _P, _P, _P]
+        L.genrank_embed_assemble_rmsnorm.restype = _I
+        L.genrank_embed_assemble_rmsnorm.argtypes = [
+            _I, _L, _P, _P, _P, _P, _P, _P, _L, _P, _I, _P, _I, _P, _I, _P, _I, _I, _P, _P, _F,
+            _P, _P, _P, _P, _P]
         L.genrank_embed_assemble_bwd.restype = _I
         L.genrank_embed_assemble_bwd.argtypes = [
             _I, _L, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _L, _P, _I, _P, _I, _P, _I,
@@ -171,6 +176,23 @@ def embed_assemble(seq_offsets, hist_len, item_ids, action_ids, ts, item_tab, ac
         rt_tab.shape[0], d, _dtype_code(item_tab), _ptr(E), _ptr(pos), _ptr(req_idx),
         _ptr(rt_bucket), _ptr(dev_err), _stream(stream))
     _check(rc, "genrank_embed_assemble")
+
+
+def embed_assemble_rmsnorm(seq_offsets, hist_len, item_ids, action_ids, ts, item_tab, action_tab,
+                           pos_tab, ri_tab, rt_tab, x_out, a_out, pos, req_idx, rt_bucket, dev_err,
+                           eps=1e-6, stream=None):
+    """genrank_embed_assemble_rmsnorm: the gather-sum written as the fp32 residual rows
+    (x_out) and their RMSNorm in bf16 (a_out) instead of E."""
+    B = hist_len.numel()
+    T = item_ids.numel()
+    d = item_tab.shape[1]
+    rc = lib().genrank_embed_assemble_rmsnorm(
+        B, T, _ptr(seq_offsets), _ptr(hist_len), _ptr(item_ids), _ptr(action_ids), _ptr(ts),
+        _ptr(item_tab), item_tab.shape[0], _ptr(action_tab), action_tab.shape[0] - 1,
+        _ptr(pos_tab), pos_tab.shape[0], _ptr(ri_tab), ri_tab.shape[0], _ptr(rt_tab),
+        rt_tab.shape[0], d, _ptr(x_out), _ptr(a_out), float(eps), _ptr(pos), _ptr(req_idx),
+        _ptr(rt_bucket), _ptr(dev_err), _stream(stream))
+    _check(rc, "genrank_embed_assemble_rmsnorm")
 
 
 def embed_assemble_bwd(seq_offsets, hist_len, item_ids, action_ids, pos, req_idx, rt_bucket, dE,

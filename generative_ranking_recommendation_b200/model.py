@@ -189,16 +189,21 @@ class GenRankModel:
 
     def _forward_fused(self, db: DeviceBatch, attn_events=None) -> torch.Tensor:
         """The four-layer scoring step on the library's kernels end to end: embedding
-        assembly, RMSNorm, per layer the QKV projection, the attention, W_o with the
+        assembly with the first RMSNorm, per layer the QKV projection, the attention, W_o with the
         residual update and the next RMSNorm in its epilogue, W1 with SiLU in its
         epilogue and W2 with the residual update and the next RMSNorm; the last layer's
         W_o and FFN run on candidate rows only and its W2 epilogue applies the final
         RMSNorm and the head."""
-        E, (pos, _, _) = self.embed(db)
         T, d, dev = db.T, self.d, self.device
+        # the gather-sum writes the fp32 residual rows and their RMSNorm directly
         x = torch.empty((T, d), dtype=torch.float32, device=dev)
         a = torch.empty((T, d), dtype=self.dtype, device=dev)
-        G.rmsnorm(E, a, self.err, x_out=x, eps=RMS_EPS)
+        pos = torch.empty(T, dtype=torch.int32, device=dev)
+        req = torch.empty(T, dtype=torch.int32, device=dev)
+        rtb = torch.empty(T, dtype=torch.int32, device=dev)
+        G.embed_assemble_rmsnorm(db.seq_offsets, db.hist_len, db.item_ids, db.action_ids, db.ts,
+                                 self.item_tab, self.action_tab, self.pos_tab, self.ri_tab,
+                                 self.rt_tab, x, a, pos, req, rtb, self.err, eps=RMS_EPS)
         nl = len(self.layers)
         for li, W in enumerate(self.layers):
             qkv = self._linear(a, W["WqkvT"])

@@ -124,6 +124,26 @@ int genrank_embed_assemble(int B, int64_t T, const int32_t *seq_offsets, const i
                            void *E, int32_t *pos, int32_t *req_idx, int32_t *rt_bucket,
                            int32_t *dev_err, genrank_stream_t stream);
 
+/* Step a2 with the first block's pre-norm fused in: the same metadata and gather-sum
+ * as genrank_embed_assemble, but instead of E each token's row is written as
+ *   x_out [T, d] fp32  = E_i as genrank_embed_assemble rounds it (bf16), upcast
+ *   a_out [T, d] bf16  = bf16(x_out_i / sqrt(mean_j x_out_ij^2 + eps))
+ * which is bit for bit what genrank_rmsnorm(E, ..., x_out) gives after
+ * genrank_embed_assemble (the same lanes, summation order and rounding): the fp32
+ * residual stream and the normalised input of a pre-RMSNorm block, without E's
+ * round trip through memory.  bf16 tables and d = 512 only (GENRANK_ERR_UNSUPPORTED
+ * otherwise); x_out and a_out 16-byte aligned with row stride d; eps >= 0.  Other
+ * arguments and errors as genrank_embed_assemble. */
+int genrank_embed_assemble_rmsnorm(int B, int64_t T, const int32_t *seq_offsets,
+                                   const int32_t *hist_len, const int32_t *item_ids,
+                                   const int32_t *action_ids, const int64_t *ts,
+                                   const void *item_tab, int64_t n_item, const void *action_tab,
+                                   int n_action, const void *pos_tab, int n_pos,
+                                   const void *ri_tab, int n_ri, const void *rt_tab, int n_rt,
+                                   int d, float *x_out, void *a_out, float eps, int32_t *pos,
+                                   int32_t *req_idx, int32_t *rt_bucket, int32_t *dev_err,
+                                   genrank_stream_t stream);
+
 /* Step a5: table gradients of the embedding sum (training).  Each token's dE_i
  * is added to the five rows it read: d_item[x_i], d_action[a_i or M],
  * d_pos[pos_i], d_ri[req_idx_i], d_rt[rt_bucket_i].  pos/req_idx/rt_bucket are

@@ -172,3 +172,61 @@ def test_embed_bwd_parity(G, name):
     for got, w in pairs:
         # fp32 accumulation of O(T) terms of size O(1): allow a few ulps of the row sums
         assert np.max(np.abs(got - w)) <= 1e-4 * max(1.0, np.max(np.abs(w))), np.max(np.abs(got - w))
+
+
+def _run_fused(G, cfg, batch, tabs, eps=1e-6):
+    T, d = batch.T, cfg.d
+    x = torch.full((T, d), float("nan"), device="cuda")
+    a = torch.full((T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    meta = [torch.empty(T, dtype=torch.int32, device="cuda") for _ in range(3)]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    G.embed_assemble_rmsnorm(_dev(batch.seq_offsets), _dev(batch.hist_len), _dev(batch.item_ids),
+                             _dev(batch.action_ids), _dev(batch.ts), *tabs, x, a, *meta, err,
+                             eps=eps)
+    return x, a, meta, G.check_error(err)
+
+
+@pytest.mark.parametrize("users", [16, None])
+def test_embed_rmsnorm_equals_gather_sum_then_rmsnorm(G, users):
+    """The fused entry gives, bit for bit, the residual rows and normalised rows of the
+    gather-sum followed by the RMSNorm pass (the first block's input at c2 shapes)."""
+    cfg = CONFIGS["c2"]
+    batch = make_batch(cfg, users=list(range(users)) if users else None)
+    tabs = _tables(cfg, make_model(cfg))
+    E, meta, code = run_embed(G, cfg, batch, tabs)
+    assert code == 0
+    x2 = torch.empty((batch.T, cfg.d), device="cuda")
+    a2 = torch.empty((batch.T, cfg.d), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    G.rmsnorm(E, a2, err, x_out=x2, eps=1e-6)
+    assert G.check_error(err) == 0
+    x, a, meta_f, code_f = _run_fused(G, cfg, batch, tabs)
+    assert code_f == 0
+    assert torch.equal(x, x2)
+    assert torch.equal(a, a2)
+    for m1, m2 in zip(meta_f, meta):
+        assert torch.equal(m1, m2)
+
+
+def test_embed_rmsnorm_against_oracle(G):
+    """x_out is E (the five rows' sum, rounded once to bf16) and a_out its RMSNorm,
+    checked against the float64 oracle on a seeded sample of c2 users."""
+    cfg = CONFIGS["c2"]
+    batch = make_batch(cfg, users=list(range(8)))
+    model = make_model(cfg)
+    x, a, meta, code = _run_fused(G, cfg, batch, _tables(cfg, model))
+    assert code == 0
+    _compare(cfg, batch, model, x, meta)
+    Er, _ = ref.embed(batch, model, None)
+    want = Er / np.sqrt((Er * Er).mean(axis=1, keepdims=True) + 1e-6)
+    got = a.double().cpu().numpy()
+    assert ref.rel_to_max(got, want) <= 2e-2
+    err_r = np.abs(got - want).max(axis=1) / np.abs(want).max(axis=1)
+    assert np.max(err_r) <= 2e-2
+
+
+def test_embed_rmsnorm_rejects_other_widths(G):
+    cfg = CONFIGS["c1"]  # d = 256
+    batch = make_batch(cfg, users=list(range(2)))
+    with pytest.raises(G.GenRankError):
+        _run_fused(G, cfg, batch, _tables(cfg, make_model(cfg)))

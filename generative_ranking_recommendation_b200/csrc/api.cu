@@ -501,6 +501,45 @@ int genrank_attn_fwd_cached(int B, int64_t C, const int32_t* cand_offsets, int m
   return launch_attn_fwd_cached(c, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t genrank_attn_candidates_workspace_size(int B, int64_t T, int H, int dh, int max_seqlen) {
+  if (B < 1 || T < 0 || H < 1 || dh < 1 || max_seqlen < 0) return 0;
+  return attn_fwd_cached_workspace(B, T, T, H, max_seqlen);
+}
+
+int genrank_attn_fwd_candidates(int B, int64_t T, const int32_t* seq_offsets,
+                                const int32_t* hist_len, int max_seqlen, const void* q,
+                                const void* k, const void* v, int64_t tok_stride, int H, int dh,
+                                const int32_t* pos, const int64_t* ts, const float* slope_pos,
+                                const float* slope_time, float scale, int dtype, void* o,
+                                int64_t o_stride, float* lse, void* ws, size_t ws_bytes,
+                                int32_t* dev_err, genrank_stream_t stream) {
+  int rc = check_attn_common(B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh,
+                             pos, ts, slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  if (rc) return rc;
+  if (T > 0 && (!o || !aligned16(o))) return GENRANK_ERR_INVALID_ARG;
+  if (!use_tc(dtype, dh)) return GENRANK_ERR_UNSUPPORTED;
+  const size_t need = genrank_attn_candidates_workspace_size(B, T, H, dh, max_seqlen);
+  if (!ws || ws_bytes < need || !aligned16(ws)) return GENRANK_ERR_WORKSPACE;
+  if (T == 0) return GENRANK_OK;
+  CachedAttnArgs c;
+  memset(&c, 0, sizeof(c));
+  fill_attn(c.a, B, T, seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts,
+            slope_pos, slope_time, scale, dtype, o_stride, dev_err);
+  c.a.o = o;
+  c.a.lse = lse;
+  c.a.ws = ws;
+  c.a.ws_bytes = ws_bytes;
+  c.hist_off = nullptr;  // the jagged array: history keys are the users' own history rows
+  c.k_hist = k;
+  c.v_hist = v;
+  c.hist_stride = tok_stride;
+  c.Th = T;
+  c.pos_hist = pos;
+  c.ts_hist = ts;
+  c.max_cand = max_seqlen;
+  return launch_attn_fwd_cached(c, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int genrank_attn_bwd(int B, int64_t T, const int32_t* seq_offsets, const int32_t* hist_len,
                      int max_seqlen, const void* q, const void* k, const void* v,
                      int64_t tok_stride, int H, int dh, const int32_t* pos, const int64_t* ts,

@@ -321,6 +321,16 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue(const __grid_constan
 // (history: the cached positions and times; candidates: position n + 1 and their request
 // time) and check the orders the separable bias relies on; block B writes the records.
 GR_DEVICE bool cached_user(const CachedAttnArgs& c, int u, int& cs, int& n, int& m, int& hs) {
+  if (!c.hist_off) {  // one jagged token array: history, then candidates, per user
+    const long long s = c.a.off[u], e = c.a.off[u + 1];
+    if (s < 0 || e < s || e > c.a.T) return false;
+    const int L = (int)(e - s);
+    n = max(0, min(c.a.hist_len[u], L));
+    m = L - n;
+    hs = (int)s;
+    cs = (int)s + n;
+    return true;
+  }
   const long long cs_ = c.a.off[u], ce = c.a.off[u + 1];
   const long long hs_ = c.hist_off[u], he = c.hist_off[u + 1];
   if (cs_ < 0 || ce < cs_ || ce > c.a.T || hs_ < 0 || he < hs_ || he > c.Th) return false;

@@ -112,7 +112,10 @@ struct AttnArgs {
 // times [C], a.o / a.lse = outputs [C, H*dh] / [H, C]); the cache has Th rows.
 struct CachedAttnArgs {
   AttnArgs a;
-  const int32_t* hist_off;  // [B+1] rows of user u's history in the cache
+  // [B+1] rows of user u's history in the cache; null for one jagged token array (the
+  // full attention's layout): user u's history rows [off[u], off[u] + hist_len[u]) of
+  // the keys and values, its candidates the rest of [off[u], off[u+1])
+  const int32_t* hist_off;
   const void* k_hist;
   const void* v_hist;
   long long hist_stride;  // elements

@@ -28,6 +28,7 @@ EXPORTS = (
     "genrank_alibi_slopes", "genrank_embed_assemble", "genrank_embed_assemble_rmsnorm",
     "genrank_embed_assemble_bwd",
     "genrank_attn_fwd", "genrank_attn_bwd", "genrank_attn_workspace_size",
+    "genrank_attn_fwd_candidates", "genrank_attn_candidates_workspace_size",
     "genrank_attn_fwd_static", "genrank_candidate_logits", "genrank_attn_fwd_cached",
     "genrank_attn_cached_workspace_size", "genrank_attn_fwd_bucketed",
     "genrank_attn_bwd_bucketed", "genrank_attn_fwd_dense_bias", "genrank_linear",
@@ -77,6 +78,10 @@ def lib():
         L.genrank_attn_fwd.argtypes = [
             _I, _L, _P, _P, _I, _P, _P, _P, _L, _I, _I, _P, _P, _P, _P, _F, _I, _P, _L, _P,
             _P, _Z, _P, _P]
+        L.genrank_attn_fwd_candidates.restype = _I
+        L.genrank_attn_fwd_candidates.argtypes = L.genrank_attn_fwd.argtypes
+        L.genrank_attn_candidates_workspace_size.restype = _Z
+        L.genrank_attn_candidates_workspace_size.argtypes = [_I, _L, _I, _I, _I]
         L.genrank_attn_fwd_bucketed.restype = _I
         L.genrank_attn_fwd_bucketed.argtypes = L.genrank_attn_fwd.argtypes
         L.genrank_attn_bwd.restype = _I
@@ -234,6 +239,26 @@ def attn_fwd(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos,
         float(scale), _dtype_code(q), _ptr(o), int(o_stride), _ptr(lse), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream))
     _check(rc, "genrank_attn_fwd_bucketed" if bucketed else "genrank_attn_fwd")
+
+
+def attn_fwd_candidates(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts,
+                        slope_pos, slope_time, scale, o, o_stride, lse, ws, dev_err, T=None,
+                        stream=None):
+    """genrank_attn_fwd_candidates: genrank_attn_fwd's candidate rows only (history rows of
+    o and lse are left as they are); the same arguments."""
+    B = hist_len.numel()
+    T = o.shape[0] if T is None else T
+    sp, st = _host_floats(slope_pos), _host_floats(slope_time)
+    rc = lib().genrank_attn_fwd_candidates(
+        B, T, _ptr(seq_offsets), _ptr(hist_len), int(max_seqlen), _ptr(q), _ptr(k), _ptr(v),
+        int(tok_stride), H, dh, _ptr(pos), _ptr(ts), ctypes.cast(sp, _P), ctypes.cast(st, _P),
+        float(scale), _dtype_code(q), _ptr(o), int(o_stride), _ptr(lse), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream))
+    _check(rc, "genrank_attn_fwd_candidates")
+
+
+def attn_candidates_workspace_size(B, T, H, dh, max_seqlen) -> int:
+    return int(lib().genrank_attn_candidates_workspace_size(B, T, H, dh, max_seqlen))
 
 
 def attn_bwd(seq_offsets, hist_len, max_seqlen, q, k, v, tok_stride, H, dh, pos, ts, slope_pos,

@@ -111,9 +111,13 @@ class GenRankModel:
         self.fused_qkv = False
 
     # -------------------------------------------------------------------------------------
-    def workspace(self, db: DeviceBatch, bwd: bool) -> torch.Tensor:
-        n = G.attn_workspace_size(db.B, db.T, self.H, self.dh, db.max_seqlen, bwd)
-        key = bool(bwd)
+    def workspace(self, db: DeviceBatch, bwd, cand_only=False) -> torch.Tensor:
+        if cand_only:
+            n = G.attn_candidates_workspace_size(db.B, db.T, self.H, self.dh, db.max_seqlen)
+            key = "cand"
+        else:
+            n = G.attn_workspace_size(db.B, db.T, self.H, self.dh, db.max_seqlen, bwd)
+            key = bool(bwd)
         w = self._ws.get(key)
         if w is None or w.numel() < n:
             w = torch.empty(max(n, 256), dtype=torch.uint8, device=self.device)
@@ -131,13 +135,17 @@ class GenRankModel:
                          E, pos, req, rtb, self.err)
         return E, (pos, req, rtb)
 
-    def attention(self, db: DeviceBatch, qkv: torch.Tensor, pos: torch.Tensor, need_lse=False):
+    def attention(self, db: DeviceBatch, qkv: torch.Tensor, pos: torch.Tensor, need_lse=False,
+                  cand_only=False):
+        """O (and the LSE) of every token, or with ``cand_only`` of the candidate rows only
+        (the other rows of O are left unwritten)."""
         d = self.d
         o = torch.empty((db.T, d), dtype=qkv.dtype, device=self.device)
         lse = torch.empty((self.H, db.T), dtype=torch.float32, device=self.device) if need_lse else None
-        G.attn_fwd(db.seq_offsets, db.hist_len, db.max_seqlen, qkv, qkv[:, d:], qkv[:, 2 * d:],
-                   3 * d, self.H, self.dh, pos, db.ts, self.slope_pos, self.slope_time,
-                   self.scale, o, d, lse, self.workspace(db, False), self.err, T=db.T)
+        fn = G.attn_fwd_candidates if cand_only else G.attn_fwd
+        fn(db.seq_offsets, db.hist_len, db.max_seqlen, qkv, qkv[:, d:], qkv[:, 2 * d:], 3 * d,
+           self.H, self.dh, pos, db.ts, self.slope_pos, self.slope_time, self.scale, o, d, lse,
+           self.workspace(db, False, cand_only), self.err, T=db.T)
         return o, lse
 
     def attention_bwd(self, db, qkv, pos, o, lse, do):
@@ -208,7 +216,8 @@ class GenRankModel:
         for li, W in enumerate(self.layers):
             qkv = self._linear(a, W["WqkvT"])
             ev = self._event(attn_events)
-            o, _ = self.attention(db, qkv, pos)
+            # after the last attention only candidate rows reach the head
+            o, _ = self.attention(db, qkv, pos, cand_only=li == nl - 1)
             if ev is not None:
                 ev[1].record()
             if li == nl - 1:  # only candidate rows reach the head

@@ -313,6 +313,27 @@ int genrank_attn_fwd_cached(int B, int64_t C, const int32_t *cand_offsets, int m
 size_t genrank_attn_cached_workspace_size(int B, int64_t C, int64_t Th, int H, int dh,
                                           int max_cand);
 
+/* The candidate rows of genrank_attn_fwd only, on its own jagged layout: for every user
+ * u the rows [seq_offsets[u] + hist_len[u], seq_offsets[u+1]) of o (and those columns
+ * of lse) are written exactly as genrank_attn_fwd defines them; history rows of o and
+ * lse are left untouched.  This is candidate scoring with the history keys and values
+ * read in place from k and v (the cached kernel in the layout the full attention
+ * uses): a model whose next step reads only candidate rows (the last block before the
+ * head: only candidates reach the logits, huaxiaozhuan "GenRank [2025]" §1.3.1) skips
+ * the history rows' attention.  Arguments, layouts and errors as genrank_attn_fwd;
+ * bf16 with dh = 64 only (GENRANK_ERR_UNSUPPORTED otherwise); ws of at least
+ * genrank_attn_candidates_workspace_size(...) bytes, contents on entry do not matter. */
+int genrank_attn_fwd_candidates(int B, int64_t T, const int32_t *seq_offsets,
+                                const int32_t *hist_len, int max_seqlen, const void *q,
+                                const void *k, const void *v, int64_t tok_stride, int H, int dh,
+                                const int32_t *pos, const int64_t *ts, const float *slope_pos,
+                                const float *slope_time, float scale, int dtype, void *o,
+                                int64_t o_stride, float *lse, void *ws, size_t ws_bytes,
+                                int32_t *dev_err, genrank_stream_t stream);
+
+/* Bytes of workspace genrank_attn_fwd_candidates needs (0 if invalid). */
+size_t genrank_attn_candidates_workspace_size(int B, int64_t T, int H, int dh, int max_seqlen);
+
 /* genrank_attn_fwd for callers that cannot allocate device memory.
  * The paper has no counterpart of this call; it exists for deployment.  Some
  * callers cannot call cudaMalloc (or any allocator, torch's included) where they

@@ -159,3 +159,61 @@ def test_cached_device_error_flags(G):
     bad["hoff"] = c["hoff"].copy()
     bad["hoff"][3] = bad["hoff"][3] + 9  # offsets past the cache
     assert run_cached(G, cfg, bad)[2] & G.DERR["LAYOUT"]
+
+
+def run_candidates(G, cfg, batch, pos, qkv, poison=False):
+    """genrank_attn_fwd_candidates on the jagged token array; o and lse start as NaN so
+    that rows it must leave alone can be checked."""
+    T, H, dh = batch.T, cfg.H, cfg.dh
+    d = H * dh
+    q = _dev(qkv.reshape(T, 3 * d), torch.bfloat16)
+    o = torch.full((T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((H, T), float("nan"), dtype=torch.float32, device="cuda")
+    msl = int(np.max(np.diff(batch.seq_offsets)))
+    ws = torch.empty(G.attn_candidates_workspace_size(batch.B, T, H, dh, msl), dtype=torch.uint8,
+                     device="cuda")
+    if poison:
+        ws.fill_(0xFF)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sp, st = G.alibi_slopes(H)
+    G.attn_fwd_candidates(_dev(batch.seq_offsets), _dev(batch.hist_len), msl, q, q[:, d:],
+                          q[:, 2 * d:], 3 * d, H, dh, _dev(pos.astype(np.int32)), _dev(batch.ts),
+                          sp, st, 1.0 / math.sqrt(dh), o, d, lse, ws, err, T=T)
+    code = G.check_error(err)
+    return (o.float().cpu().numpy().astype(np.float64).reshape(T, H, dh),
+            lse.cpu().numpy().astype(np.float64), code)
+
+
+@pytest.mark.parametrize("poison", [False, True])
+def test_candidates_only_forward_edge_users(G, poison):
+    """Candidate rows of the full attention computed alone on the jagged layout (history
+    keys and values read in place): against the oracle, and the history rows of o and
+    lse left untouched; edge users as for the cached entry."""
+    cfg = CONFIGS["c1"].with_(B=len(USERS), H=2)
+    batch = make_batch(cfg, hist_override=[n for n, _ in USERS], m_override=[m for _, m in USERS])
+    pos, _, _ = ref.meta(batch)
+    qkv = make_qkv(cfg, batch.T, seed=54)
+    O, L, code = run_candidates(G, cfg, batch, pos, qkv, poison=poison)
+    assert code == 0
+    rows = ref.cand_rows(batch)
+    hist = np.setdiff1d(np.arange(batch.T), rows)
+    assert np.all(np.isnan(O[hist])) and np.all(np.isnan(L[:, hist]))
+    Or, Lr = ref.attn(qkv[:, 0], qkv[:, 1], qkv[:, 2], batch, pos)
+    _check(O[rows], L[:, rows], Or[rows], Lr[:, rows])
+
+
+def test_candidates_only_equals_full_forward(G):
+    """At c2 shapes (16 users, 480 history + 256 candidates, 8 heads) the candidate rows
+    agree with the full forward kernel's to within its bf16 rounding."""
+    from test_gpu_attention import run_fwd
+
+    cfg = CONFIGS["c2"]
+    batch = make_batch(cfg, users=list(range(16)))
+    pos, _, _ = ref.meta(batch)
+    qkv = make_qkv(cfg, batch.T, seed=55)
+    O, L, code = run_candidates(G, cfg, batch, pos, qkv)
+    assert code == 0
+    Of, Lf = run_fwd(G, cfg, batch, pos, qkv)
+    rows = ref.cand_rows(batch)
+    assert ref.rel_to_max(O[rows], Of[rows]) <= 1e-2
+    assert np.max(np.abs(L[:, rows] - Lf[:, rows])) <= 1e-3

@@ -238,10 +238,10 @@ class GenRankModel:
         """Candidate logits with the blocks as torch ops (the QKV projection optionally on
         the library's linear layer).
 
-        Every layer's attention runs over all tokens (history rows feed the next
-        layer's keys and values).  After the last attention only candidate rows
-        reach the head, so the last output projection, residual, FFN and final norm
-        run on candidate rows alone; with one block and no FFN the head is one fused
+        Every layer's attention but the last runs over all tokens (history rows feed
+        the next layer's keys and values); only candidate rows reach the head, so the
+        last attention (bf16, head dim 64) computes candidate rows alone, and the last
+        output projection, residual, FFN and final norm run on candidate rows alone; with one block and no FFN the head is one fused
         kernel, z = E . w_head + o . (W_o w_head) at candidate rows (the same sum
         regrouped).  ``attn_events``: optional list; a (start, end)
         pair of CUDA events recorded on the current stream around each attention
@@ -258,7 +258,10 @@ class GenRankModel:
                 a = E if li == 0 else x.to(self.dtype)
             qkv = self._linear(a, W["WqkvT"]) if fused_qkv else a @ W["Wqkv"]
             ev = self._event(attn_events)
-            o, _ = self.attention(db, qkv, pos)
+            # the last attention is needed at candidate rows only (the candidate-only
+            # kernel takes bf16 with head dim 64; other forms run the full attention)
+            cand_only = li == nl - 1 and self.dtype == torch.bfloat16 and self.dh == 64
+            o, _ = self.attention(db, qkv, pos, cand_only=cand_only)
             if ev is not None:
                 ev[1].record()
             if li == nl - 1 and x is None:

@@ -363,15 +363,16 @@ __global__ void __launch_bounds__(1024) k_embed_bwd(
         if (!col_ok || itq[q] < 0 || k + q >= nt) continue;
         red_add_v2(g_item + itq[q] * d + col, g0[q], g1[q]);
         if (kSmem) {
-          const int cl = 2 * lane;
-          atomicAdd(s_action + aq[q] * kBwdCols + cl, g0[q]);
-          atomicAdd(s_action + aq[q] * kBwdCols + cl + 1, g1[q]);
-          atomicAdd(s_pos + pq[q] * kBwdCols + cl, g0[q]);
-          atomicAdd(s_pos + pq[q] * kBwdCols + cl + 1, g1[q]);
-          atomicAdd(s_ri + rq[q] * kBwdCols + cl, g0[q]);
-          atomicAdd(s_ri + rq[q] * kBwdCols + cl + 1, g1[q]);
-          atomicAdd(s_rt + bq[q] * kBwdCols + cl, g0[q]);
-          atomicAdd(s_rt + bq[q] * kBwdCols + cl + 1, g1[q]);
+          // a slice row holds column 2l + k at k * 32 + l, so each of these adds covers
+          // 32 consecutive words (one per bank)
+          atomicAdd(s_action + aq[q] * kBwdCols + lane, g0[q]);
+          atomicAdd(s_action + aq[q] * kBwdCols + 32 + lane, g1[q]);
+          atomicAdd(s_pos + pq[q] * kBwdCols + lane, g0[q]);
+          atomicAdd(s_pos + pq[q] * kBwdCols + 32 + lane, g1[q]);
+          atomicAdd(s_ri + rq[q] * kBwdCols + lane, g0[q]);
+          atomicAdd(s_ri + rq[q] * kBwdCols + 32 + lane, g1[q]);
+          atomicAdd(s_rt + bq[q] * kBwdCols + lane, g0[q]);
+          atomicAdd(s_rt + bq[q] * kBwdCols + 32 + lane, g1[q]);
         } else {
           red_add_v2(g_action + (long long)aq[q] * d + col, g0[q], g1[q]);
           red_add_v2(g_pos + (long long)pq[q] * d + col, g0[q], g1[q]);
@@ -385,7 +386,8 @@ __global__ void __launch_bounds__(1024) k_embed_bwd(
     __syncthreads();
     for (int i = threadIdx.x; i < rows_small * kBwdCols; i += blockDim.x) {
       const float v = acc[i];
-      const int row = i / kBwdCols, c = c0 + i % kBwdCols;
+      const int j = i % kBwdCols;  // column 2 (j % 32) + j / 32 of the slice
+      const int row = i / kBwdCols, c = c0 + 2 * (j & 31) + (j >> 5);
       if (v == 0.f || c >= d) continue;
       float* dst;
       if (row < n_act_rows) dst = g_action + (long long)row * d;

@@ -9,8 +9,9 @@
 //   * A prologue kernel lists (user, 128-row query tile) work records sorted by the
 //     number of 128-key tiles they visit (longest first), and writes the ALiBi
 //     column term c_j = log2(e) (m_h p_j + m_t,h (t_j - t_0)) for every token and
-//     head into a 16-byte aligned scratch layout.  On visible pairs p_i >= p_j and
-//     t_i >= t_j, so the bias is c_j - c_i; c_i cancels in the softmax and only c_j
+//     head into a 16-byte aligned scratch layout (entries between users' segments are
+//     zeroed, so every term a key tile reads is finite).  On visible pairs p_i >= p_j
+//     and t_i >= t_j, so the bias is c_j - c_i; c_i cancels in the softmax and only c_j
 //     is added per element; the literal LSE subtracts c_i in the epilogue.
 //   * A persistent grid walks the records round-robin (one head per work item).  An
 //     item visits its history key tiles (history tile t: key tiles 0..t; candidate
@@ -28,7 +29,13 @@
 //     each SM sub-partition: bias, mask and exponentials in one pass per tile, with
 //     the offset fixed at the row's own column term (every visible key has
 //     c_j <= c_i); a tile whose row sum leaves the safe range is redone exactly and O
-//     rescaled in TMEM.
+//     rescaled in TMEM.  Only an item's first tile can need the row mask: it runs
+//     chunk by chunk (16 keys) with the two half-warps interleaved by chunks, so that
+//     both halves skip wholly masked chunks and only the chunk a row's mask cuts pays
+//     for it; the loop over the other tiles holds the plain code alone.
+//   * The same kernel scores candidates from a KV cache (or, reading the cache in
+//     place, the candidate rows of one jagged token array alone): records then hold
+//     candidate tiles only, whose key tiles are the user's history plus the diagonal.
 //   * Warps 10-13 (one row per thread) finish each item from its O buffer while the
 //     next item runs: O is normalised and written through shared memory as whole
 //     128-byte rows, and the literal LSE is stored.

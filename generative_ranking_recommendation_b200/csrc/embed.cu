@@ -120,6 +120,8 @@ __global__ void __launch_bounds__(256) k_token_meta(
 // rows with 16-byte vector loads, the row indices broadcast from their lanes by
 // shuffles, two tokens' loads in flight together.  The rows are summed in fp32 and
 // rounded once.  At most 64 registers per thread keep four blocks resident per SM.
+// kNorm (bf16, d = 512): instead of E, each row is written as its fp32 value and its
+// RMSNorm in bf16 (the first pre-norm block's input), one token at a time.
 template <typename T, bool kNorm>
 __global__ void __launch_bounds__(256, 4) k_embed_fwd(
     int B, long long Ttok, const int32_t* __restrict__ off, const int32_t* __restrict__ hist_len,

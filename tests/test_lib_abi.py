@@ -150,3 +150,44 @@ def test_backward_host_side_argument_checks(L):
     assert call(ws=None) == 3
     assert call(wsb=16) == 3
 
+
+
+def test_candidates_and_fused_embedding_host_checks(L):
+    """The candidate-only attention and the gather-sum with the first RMSNorm reject bad
+    arguments on the host; the candidate workspace covers the cached form's."""
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    sp = (ctypes.c_float * 4)(0.5, 0.25, 0.125, 0.0625)
+    st = (ctypes.c_float * 4)(*(x / 3600 for x in sp))
+
+    def cand(**kw):
+        a = dict(B=1, T=10, off=fake, hl=fake, msl=10, q=fake, k=fake, v=fake, stride=768, H=4,
+                 dh=64, pos=fake, ts=fake, scale=0.125, dtype=1, o=fake, ostride=256, lse=None,
+                 ws=fake, wsb=1 << 20, err=fake)
+        a.update(kw)
+        return L.genrank_attn_fwd_candidates(
+            a["B"], a["T"], a["off"], a["hl"], a["msl"], a["q"], a["k"], a["v"], a["stride"],
+            a["H"], a["dh"], a["pos"], a["ts"], ctypes.cast(sp, P), ctypes.cast(st, P),
+            a["scale"], a["dtype"], a["o"], a["ostride"], a["lse"], a["ws"], a["wsb"], a["err"],
+            None)
+
+    assert cand(B=0) == 1
+    assert cand(hl=None) == 1
+    assert cand(o=P(0x10008)) == 1
+    assert cand(dtype=0, stride=768, ostride=256) == 2  # fp32: the tensor-core kernel only
+    assert cand(ws=None) == 3
+    assert cand(wsb=16) == 3
+    n = L.genrank_attn_candidates_workspace_size(64, 100000, 16, 64, 1504)
+    assert n == L.genrank_attn_cached_workspace_size(64, 100000, 100000, 16, 64, 1504) > 0
+    assert L.genrank_attn_candidates_workspace_size(0, 10, 4, 64, 10) == 0
+
+    def emb(d=512, eps=1e-6, x=fake, a=fake, n_rt=64):
+        return L.genrank_embed_assemble_rmsnorm(1, 10, fake, fake, fake, fake, fake, fake, 100,
+                                                fake, 8, fake, 600, fake, 128, fake, n_rt, d, x,
+                                                a, eps, fake, fake, fake, fake, None)
+
+    assert emb(d=256) == 2  # the fused form takes d = 512 only
+    assert emb(eps=-1.0) == 1
+    assert emb(x=None) == 1
+    assert emb(a=P(0x10008)) == 1
+    assert emb(n_rt=80) == 2

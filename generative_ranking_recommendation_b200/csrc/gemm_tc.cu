@@ -53,9 +53,10 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, 0, 0);  // A K-major, Wt K-major
+// SM pair: one MMA of M = 256 rows (128 per CTA) x N = 256 over both SMs
+constexpr uint32_t kIdescPair = idesc_bf16_f32(2 * BM, BN, 0, 0);
 constexpr uint32_t kABytes = BM * BK * 2;                    // 16 KB
 constexpr uint32_t kBBytes = BN * BK * 2;                    // 32 KB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
 // res+rms: the two 256-column halves take turns in chunks of this many k-steps, so a
 // tile's A rows are read from DRAM once (the other half's read of the chunk hits L2) and
 // the first half still completes one chunk ahead of the second
@@ -75,9 +76,12 @@ constexpr int kXBufs = 4;             // res+rms: residual boxes in flight per e
 //     (one float per row and column half).
 // Then the barriers: full[S], empty[S], acc_full[2], acc_empty[2], done and, for res+rms,
 // one per residual box.
-template <bool kRes>
+//   SM pair: each CTA holds its 128 A rows and half of the 256 Wt rows of a k-step, 32 KB
+//     a stage, so six stages fit (four with the residual boxes).
+template <bool kRes, bool kPair>
 struct Layout {
-  static constexpr int kStages = kRes ? 3 : 4;
+  static constexpr uint32_t kStageBytes = kABytes + (kPair ? kBBytes / 2 : kBBytes);
+  static constexpr int kStages = kRes ? (kPair ? 4 : 3) : (kPair ? 6 : 4);
   static constexpr uint32_t kOffBox = kStages * kStageBytes;
   static constexpr uint32_t kXBytes = kRes ? kEpiWarps * kXBufs * kBoxBytes : 0;
   static constexpr uint32_t kOutBoxes = kRes ? 1 : 2;
@@ -88,8 +92,8 @@ struct Layout {
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmem = kOffMisc + 16 + 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(kStageBytes % 1024 == 0, "1024-byte aligned stages");
 };
-static_assert(kStageBytes % 1024 == 0, "1024-byte aligned stages");
 
 struct Params {
   CUtensorMap ta, tb;
@@ -145,12 +149,13 @@ GR_DEVICE void box_bf16x16(uint8_t* box, int r, int half, const float* v) {
                    pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
 }
 
-template <int kEpi>
+template <int kEpi, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__ Params P) {
   constexpr bool kRes = kEpi == kEpiResRms || kEpi == kEpiResRmsRel;
   constexpr bool kRel = kEpi == kEpiResRmsRel;
-  using L = Layout<kRes>;
+  using L = Layout<kRes, kPair>;
   constexpr int kStages = L::kStages;
+  constexpr uint32_t kStageBytes = L::kStageBytes;
   constexpr int kHalves = kRes ? 2 : 1;  // 256-column blocks per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -169,6 +174,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // rows per tile: 128, or 256 for an SM pair (CTA `rank` of the cluster holds rows
+  // [128 rank, 128 rank + 128) of each tile; the even CTA issues the MMAs)
+  constexpr int kTileRows = kPair ? 2 * BM : BM;
+  const int rank = kPair ? (int)cluster_ctarank() : 0;
+  const int first = kPair ? (int)cluster_idx() : (int)blockIdx.x;  // tiles first, +stride
+  const int stride = kPair ? (int)cluster_count() : (int)gridDim.x;
+  const int row_off = rank * BM;  // this CTA's first row within a tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -177,7 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kEpiWarps);  // one arrival per epilogue warp
+      // one arrival per epilogue warp (of both CTAs for a pair: the even CTA's barrier)
+      mbar_init(&acc_empty[b], kPair ? 2 * kEpiWarps : kEpiWarps);
     }
     mbar_init(done, 1);
     if (kRes)
@@ -195,14 +208,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     }
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc<kPair>(tmem_slot, kTmemCols);
+    tmem_relinquish<kPair>();
   }
   tc_fence_before();
-  __syncthreads();
+  // a pair: both CTAs' barriers are initialised before either signals the other's
+  if constexpr (kPair)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int m_tiles = (g.M + BM - 1) / BM;
+  const int m_tiles = (g.M + kTileRows - 1) / kTileRows;
   const int n_tiles = kRes ? 1 : g.N / BN;
   const int tiles = m_tiles * n_tiles;
   const int ksteps = g.K / BK;
@@ -211,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     // ------------------------------------------------------------------ TMA producer
     int it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+    for (int t = first; t < tiles && ok; t += stride) {
       const int mt = t / n_tiles, nt = t - mt * n_tiles;
       for (int k0 = 0; k0 < ksteps && ok; k0 += kChunkSteps) {
         const int k1 = min(ksteps, k0 + kChunkSteps);
@@ -224,34 +241,49 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
             }
             if (lane == 0) {
               uint8_t* sa = smem + st * kStageBytes;
-              mbar_expect_tx(&full[st], kStageBytes);
-              tma_load_2d(sa, &P.ta, &full[st], ks * BK, mt * BM);
-              tma_load_2d(sa + kABytes, &P.tb, &full[st], ks * BK, (nt + h) * BN);
+              if constexpr (kPair) {
+                // both CTAs' tiles complete on the even CTA's barrier, which expects both
+                const uint32_t fb = cluster_addr(&full[st], 0);
+                if (rank == 0) mbar_expect_tx(&full[st], 2 * kStageBytes);
+                tma_load_2d_pair(sa, &P.ta, fb, ks * BK, mt * kTileRows + row_off);
+                tma_load_2d_pair(sa + kABytes, &P.tb, fb, ks * BK,
+                                 (nt + h) * BN + rank * (BN / 2));
+              } else {
+                mbar_expect_tx(&full[st], kStageBytes);
+                tma_load_2d(sa, &P.ta, &full[st], ks * BK, mt * BM);
+                tma_load_2d(sa + kABytes, &P.tb, &full[st], ks * BK, (nt + h) * BN);
+              }
             }
           }
         }
       }
     }
-    // the copies issued last land before the CTA exits
+    // the copies issued last land before the CTA exits (the odd CTA of a pair: its stages
+    // have been read by the pair's MMAs, which waited for them)
     if (lane == 0)
-      for (int x = max(0, it - kStages); x < it; ++x) mbar_drain(&full[x % kStages], par(x / kStages));
+      for (int x = max(0, it - kStages); x < it; ++x) {
+        if (rank == 0)
+          mbar_drain(&full[x % kStages], par(x / kStages));
+        else
+          mbar_drain(&empty[x % kStages], par(x / kStages));
+      }
   } else if (warp == 0) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int it = 0, tc = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
+      for (int t = first; t < tiles && ok; t += stride, ++tc) {
         const int buf = kRes ? 0 : (tc & 1);
         const uint32_t ph_empty = kRes ? par(tc) ^ 1u : par(tc >> 1) ^ 1u;
         if (!kRes) {
-          if (!mbar_wait(&acc_empty[buf], ph_empty, abort_flag, g.err)) break;
+          if (!mbar_wait<kPair>(&acc_empty[buf], ph_empty, abort_flag, g.err)) break;
           tc_fence_after();
         }
         for (int k0 = 0; k0 < ksteps && ok; k0 += kChunkSteps) {
           const int k1 = min(ksteps, k0 + kChunkSteps);
           for (int h = 0; h < kHalves && ok; ++h) {
             if (kRes && k0 == 0) {  // each half's columns are released on their own
-              if (!mbar_wait(&acc_empty[h], ph_empty, abort_flag, g.err)) {
+              if (!mbar_wait<kPair>(&acc_empty[h], ph_empty, abort_flag, g.err)) {
                 ok = false;
                 break;
               }
@@ -270,16 +302,31 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
               for (int kk = 0; kk < BK / 16; ++kk) {
                 const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
                 const uint64_t bd = smem_desc_sw128(sa + kABytes + kk * 32, 16, 1024);
-                mma_bf16_ss(acc, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                if constexpr (kPair)
+                  mma_bf16_ss_pair(acc, ad, bd, kIdescPair, (ks > 0 || kk > 0) ? 1u : 0u);
+                else
+                  mma_bf16_ss(acc, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
               }
-              mma_commit(&empty[st]);  // the stage is free once these MMAs have read it
+              // the stage (both CTAs' copies of it) is free once these MMAs have read it
+              if constexpr (kPair)
+                mma_commit_pair(&empty[st], 0x3);
+              else
+                mma_commit(&empty[st]);
             }
-            if (ok && k1 == ksteps) mma_commit(&acc_full[kRes ? h : buf]);
+            if (ok && k1 == ksteps) {
+              if constexpr (kPair)
+                mma_commit_pair(&acc_full[kRes ? h : buf], 0x3);
+              else
+                mma_commit(&acc_full[kRes ? h : buf]);
+            }
           }
         }
       }
       // every MMA issued has completed before TMEM is freed
-      mma_commit(done);
+      if constexpr (kPair)
+        mma_commit_pair(done, 0x1);
+      else
+        mma_commit(done);
       mbar_drain(done, 0);
     }
     __syncwarp();
@@ -290,11 +337,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     const int ch = ew >> 2;  // which 128 columns of each 256-column block
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
     const int rloc = q * 32 + lane;  // row within the tile
-    const int box_row = q * 32;      // + mt * BM: the warp's first row in C
+    const int box_row = q * 32;      // + the CTA's first row of the tile: the warp's in C
     uint8_t* out = smem + L::kOffOut + ew * L::kOutBoxes * kBoxBytes;  // output boxes
+    // accumulator buffer b has been read by this warp (a pair: on the even CTA's barrier)
+    auto release_acc = [&](int b) {
+      if constexpr (kPair)
+        mbar_arrive_cluster(cluster_addr(&acc_empty[b], 0));
+      else
+        mbar_arrive(&acc_empty[b]);
+    };
     if (!kRes) {
       int tc = 0;
-      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
+      for (int t = first; t < tiles; t += stride, ++tc) {
         const int mt = t / n_tiles, nt = t - mt * n_tiles;
         const int buf = tc & 1;
         if (!wait_warp(&acc_full[buf], par(tc >> 1), abort_flag, g.err)) break;
@@ -304,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         // two boxes and stored by the TMA engine as whole lines; rows past M are clipped
         // by the tensor map
         const int gcol = nt * BN + ch * 128;
+        const int grow = mt * kTileRows + row_off + box_row;  // the warp's first row in C
 #pragma unroll 1
         for (int c = 0; c < 128; c += 32) {
           float v[32];
@@ -318,14 +373,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
           box_bf16x32(box, lane, v);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0 && mt * BM + box_row < g.M) {  // boxes wholly past M are skipped
-            tma_store_2d(&P.tc, box, gcol + c, mt * BM + box_row);
+          if (lane == 0 && grow < g.M) {  // boxes wholly past M are skipped
+            tma_store_2d(&P.tc, box, gcol + c, grow);
             bulk_commit();
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        if (lane == 0) release_acc(buf);
       }
     } else {
       // res+rms.  The warp's residual boxes (32 rows x 16 fp32 columns, 16 a tile: 8 per
@@ -337,16 +392,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       constexpr int kPerTile = kRel ? 32 : 16;
       uint8_t* xb = smem + L::kOffBox + ew * kXBufs * kBoxBytes;
       uint64_t* xw = xbar + ew * kXBufs;
-      const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+      const int my_tiles = first < tiles ? (tiles - 1 - first) / stride + 1 : 0;
       const int nbox = kPerTile * my_tiles;
       auto issue = [&](int n) {  // lane 0: load box n
-        const int t = blockIdx.x + (n / kPerTile) * gridDim.x;
+        const int t = first + (n / kPerTile) * stride;
         const int w = n % kPerTile;
         const int col = ((w >> 3) & 1) * BN + ch * 128 + (w & 7) * 16;
         const int b = n % kXBufs;
         mbar_expect_tx(&xw[b], kBoxBytes);
         tma_load_2d(xb + b * kBoxBytes, w < 16 ? (const void*)&P.txi : (const void*)&P.tx, &xw[b],
-                    col, t * BM + box_row);
+                    col, t * kTileRows + row_off + box_row);
       };
       int ld = 0;  // boxes whose loads were issued
       if (lane == 0)
@@ -367,11 +422,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
       // A failed (timed-out) wait skips the work but not the named barriers below, so the
       // other warp of the quadrant never waits for a partner that has left.
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
+      for (int t = first; t < tiles; t += stride, ++tc) {
         const int mt = t;
-        const long long row = (long long)mt * BM + rloc;
+        const int grow = mt * kTileRows + row_off + box_row;  // the warp's first row
+        const long long row = (long long)mt * kTileRows + row_off + rloc;
         const bool valid = row < g.M;
-        const bool rows_in = mt * BM + box_row < g.M;  // boxes wholly past M are skipped
+        const bool rows_in = grow < g.M;  // boxes wholly past M are skipped
         // pass 1 per half as soon as its MMAs are done: y = x_in + acc, kept in TMEM,
         // written to x_out through the output box, its squares summed
         float ss = 0.f;
@@ -420,14 +476,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0 && rows_in) {
-              tma_store_2d(&P.tx, out, c0 + c, mt * BM + box_row);
+              tma_store_2d(&P.tx, out, c0 + c, grow);
               bulk_commit();
             }
           }
           if (kRel && ok) {  // this half's accumulator columns go back to the MMAs
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[h]);
+            if (lane == 0) release_acc(h);
           }
         }
         // the row's sum of squares over both warps of this quadrant
@@ -485,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0 && rows_in) {
-                  tma_store_2d(&P.tc, out, c0 + c - 16, mt * BM + box_row);
+                  tma_store_2d(&P.tc, out, c0 + c - 16, grow);
                   bulk_commit();
                 }
               }
@@ -505,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
           if (!kRel) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[h]);
+            if (lane == 0) release_acc(h);
           }
         }
         if (g.w_head) {
@@ -528,9 +584,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   if (warp >= 2 && lane == 0) bulk_wait_all();  // the output stores have landed
   __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  // a pair: neither CTA leaves (or frees TMEM) while the other may still signal its
+  // barriers or the pair's MMAs read its shared memory
+  if constexpr (kPair)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 0) tmem_dealloc<kPair>(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -603,8 +664,6 @@ static bool make_map(CUtensorMap* m, const void* base, long long rows, int K, lo
          CUDA_SUCCESS;
 }
 
-static DeviceOnce gemm_smem_attr[4];
-
 // [rows][N] output (bf16 or fp32) with row stride ld elements, for TMA stores of 32-row
 // boxes of 64 bytes (32 bf16 or 16 fp32 columns) with the 64-byte swizzle.
 static bool make_store_map(CUtensorMap* m, void* base, long long rows, int N, long long ld,
@@ -622,12 +681,14 @@ static bool make_store_map(CUtensorMap* m, void* base, long long rows, int N, lo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int kEpi>
+template <int kEpi, bool kPair>
 static int launch_t(const GemmArgs& g, cudaStream_t st) {
+  constexpr bool kRes = kEpi >= kEpiResRms;
   Params p;
-  if (!make_map(&p.ta, g.a, g.M, g.K, g.lda, BM) || !make_map(&p.tb, g.w, g.N, g.K, g.ldw, BN))
+  if (!make_map(&p.ta, g.a, g.M, g.K, g.lda, BM) ||
+      !make_map(&p.tb, g.w, g.N, g.K, g.ldw, kPair ? BN / 2 : BN))
     return GENRANK_ERR_CUDA;
-  if (kEpi >= kEpiResRms) {
+  if (kRes) {
     if (!make_store_map(&p.tx, g.x_out, g.M, g.N, g.ldx, true) ||
         !make_store_map(&p.txi, const_cast<float*>(g.x_in), g.M, g.N, g.ldx, true) ||
         (g.a_out && !make_store_map(&p.tc, g.a_out, g.M, g.N, g.lda_out, false)))
@@ -636,15 +697,46 @@ static int launch_t(const GemmArgs& g, cudaStream_t st) {
     return GENRANK_ERR_CUDA;
   }
   p.g = g;
-  constexpr int kSmem = (int)Layout<kEpi >= kEpiResRms>::kSmem;
-  if (!set_smem_limit_once(gemm_smem_attr[kEpi], (const void*)k_gemm_tc<kEpi>, kSmem))
+  constexpr int kSmem = (int)Layout<kRes, kPair>::kSmem;
+  static DeviceOnce smem_attr;
+  if (!set_smem_limit_once(smem_attr, (const void*)k_gemm_tc<kEpi, kPair>, kSmem))
     return GENRANK_ERR_CUDA;
   const int sms = sm_count_current();
   if (sms <= 0) return GENRANK_ERR_CUDA;
+  constexpr int kTileRows = kPair ? 2 * BM : BM;
   const long long tiles =
-      (long long)((g.M + BM - 1) / BM) * (kEpi >= kEpiResRms ? 1 : g.N / BN);
-  const int grid = (int)(tiles < sms ? tiles : sms);
-  k_gemm_tc<kEpi><<<grid, kThreads, kSmem, st>>>(p);
+      (long long)((g.M + kTileRows - 1) / kTileRows) * (kRes ? 1 : g.N / BN);
+  if constexpr (!kPair) {
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    k_gemm_tc<kEpi, false><<<grid, kThreads, kSmem, st>>>(p);
+  } else {
+    // clusters of two CTAs (one per SM of a pair), as many as can be resident at once
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    static DeviceOnce pairs_once;
+    const int pairs = pairs_once.run([&](int) {
+      cudaLaunchConfig_t q = cfg;
+      q.gridDim = dim3(2 * (unsigned)(sms / 2));
+      int n = 0;
+      return cudaOccupancyMaxActiveClusters(&n, (const void*)k_gemm_tc<kEpi, true>, &q) ==
+                     cudaSuccess
+                 ? n
+                 : 0;
+    });
+    if (pairs <= 0) return GENRANK_ERR_CUDA;
+    cfg.gridDim = dim3(2 * (unsigned)(tiles < pairs ? tiles : pairs));
+    if (cudaLaunchKernelEx(&cfg, k_gemm_tc<kEpi, true>, p) != cudaSuccess)
+      return GENRANK_ERR_LAUNCH;
+  }
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
 }
 
@@ -654,10 +746,11 @@ int launch_gemm_tc(const GemmArgs& g, cudaStream_t st) {
   using namespace tg;
   if (g.M == 0) return GENRANK_OK;
   switch (g.epilogue) {
-    case kEpiStore: return launch_t<kEpiStore>(g, st);
-    case kEpiSilu: return launch_t<kEpiSilu>(g, st);
+    case kEpiStore: return launch_t<kEpiStore, true>(g, st);
+    case kEpiSilu: return launch_t<kEpiSilu, true>(g, st);
     case kEpiResRms:
-      return g.K >= kReleaseMinK ? launch_t<kEpiResRmsRel>(g, st) : launch_t<kEpiResRms>(g, st);
+      return g.K >= kReleaseMinK ? launch_t<kEpiResRmsRel, true>(g, st)
+                                 : launch_t<kEpiResRms, true>(g, st);
     default: return GENRANK_ERR_INVALID_ARG;
   }
 }

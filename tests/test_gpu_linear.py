@@ -50,7 +50,8 @@ def _rows_ok(got, want, tol=2e-2):
 
 
 @pytest.mark.parametrize("M,N,K,epi", [(1000, 1536, 512, 0), (129, 256, 64, 0),
-                                       (4097, 2048, 512, 1), (1, 512, 2048, 1)])
+                                       (4097, 2048, 512, 1), (1, 512, 2048, 1),
+                                       (255, 512, 128, 0), (257, 256, 192, 1)])
 def test_linear_parity(G, M, N, K, epi):
     A = _bf((M, K), 1, 1.0)
     Wt = _bf((N, K), 2, 1.0 / np.sqrt(K))
@@ -84,6 +85,23 @@ def test_linear_residual_rmsnorm_parity(G, M, K, head):
     _rows_ok(_np(a_out), _rms(xo))
     if head:
         assert ref.rel_to_max(z.double().cpu().numpy(), _rms(xo) @ w.double().cpu().numpy()) <= 2e-2
+
+
+@pytest.mark.parametrize("M,N,epi", [(20001, 1536, 0), (12345, 2048, 1)])
+def test_linear_many_tiles(G, M, N, epi):
+    """More 256-row tiles than SM pairs, so every pair runs several tiles through both
+    accumulator buffers and the operand ring wraps many times; ragged last tile."""
+    K = 512
+    A = _bf((M, K), 5, 1.0)
+    Wt = _bf((N, K), 6, 1.0 / np.sqrt(K))
+    C = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    G.linear(A, Wt, C, err, epilogue=epi)
+    assert G.check_error(err) == 0
+    want = _np(A) @ _np(Wt).T
+    if epi == 1:
+        want = want / (1.0 + np.exp(-want))
+    _rows_ok(_np(C), want)
 
 
 @pytest.mark.parametrize("M,K", [(50_000, 512), (40_001, 2048)])

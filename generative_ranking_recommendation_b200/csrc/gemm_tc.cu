@@ -16,12 +16,19 @@
 // so the residual stream is read and written once per update and the normalised
 // activations never take a separate pass.
 //
-// Design, one CTA per SM (persistent), 320 threads:
-//   * warp 1 issues TMA loads of 128 x 64 A tiles and 256 x 64 Wt tiles (128B swizzle,
-//     no multicast) into a ring of 48 KB stages (four; three for res+rms);
-//   * warp 0 (one thread) issues tcgen05.mma M = 128, N = 256, K = 16 (four per 64-wide
-//     k-step) into a TMEM accumulator.  The store and SiLU epilogues double-buffer the
-//     accumulator (2 x 256 columns) so a tile's epilogue overlaps the next tile's MMAs.
+// Design: persistent clusters of two CTAs, one per SM of an SM pair, 320 threads each.
+// A tile is 256 rows x 256 columns (x 512 for res+rms), computed by one tcgen05.mma of
+// M = 256 spanning both SMs (cta_group::2): each CTA holds its own 128 rows of A and half
+// of the 256 Wt rows, so an SM loads 32 KB of operands per 64-wide k-step instead of
+// 48 KB, and each CTA's TMEM receives its own 128 rows of the accumulator.
+//   * warp 1 of each CTA issues TMA loads of its 128 x 64 A tile and 128 x 64 Wt tile
+//     (128B swizzle, no multicast) into a ring of 32 KB stages (six; four for res+rms);
+//     both CTAs' loads complete on the even CTA's barrier;
+//   * warp 0 of the even CTA (one thread) issues the pair's MMAs, N = 256, K = 16 (four
+//     per k-step), and commits each stage's release and each accumulator's completion to
+//     the barriers of both CTAs.  The store and SiLU epilogues double-buffer the
+//     accumulator (2 x 256 columns) so a tile's epilogue overlaps the next tile's MMAs;
+//     the epilogue warps of both CTAs hand a buffer back on the even CTA's barrier.
 //     res+rms computes its row (d = 512) as two 256-column halves, into columns [0, 256)
 //     and [256, 512), taking turns every 16 k-steps (the A rows of a chunk are re-read
 //     from L2, not DRAM): the first half completes a chunk early and its residual pass
@@ -34,7 +41,7 @@
 //     through 2 KB shared-memory boxes (64-byte swizzle, so one-row-per-thread writes
 //     hit every bank) as TMA stores of whole lines; res+rms loads its residual rows the
 //     same way, four boxes ahead of use per warp.
-// Tiles are ordered with the N tiles of one M tile adjacent, so CTAs running them at the
+// Tiles are ordered with the N tiles of one M tile adjacent, so pairs running them at the
 // same time share the A tile in L2.  Every mbarrier wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -52,9 +59,9 @@ constexpr int BK = 64;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, 0, 0);  // A K-major, Wt K-major
-// SM pair: one MMA of M = 256 rows (128 per CTA) x N = 256 over both SMs
-constexpr uint32_t kIdescPair = idesc_bf16_f32(2 * BM, BN, 0, 0);
+// one MMA of M = 256 rows (128 per CTA of an SM pair) x N = 256; A and Wt K-major
+constexpr uint32_t kIdesc = idesc_bf16_f32(2 * BM, BN, 0, 0);
+constexpr int kTileRows = 2 * BM;  // rows per tile
 constexpr uint32_t kABytes = BM * BK * 2;                    // 16 KB
 constexpr uint32_t kBBytes = BN * BK * 2;                    // 32 KB
 // res+rms: the two 256-column halves take turns in chunks of this many k-steps, so a
@@ -69,19 +76,18 @@ constexpr int kReleaseMinK = 1024;
 constexpr uint32_t kBoxBytes = 2048;  // 32 rows x 64 bytes (32 bf16 or 16 fp32 columns)
 constexpr int kXBufs = 4;             // res+rms: residual boxes in flight per epilogue warp
 
-// Shared memory of each epilogue, after the operand stages:
-//   store / SiLU: four stages; two output boxes per epilogue warp (ping-pong).
-//   res+rms: three stages (room for the residual boxes); per epilogue warp kXBufs boxes
+// Shared memory of each CTA: the operand stages (its 128 A rows and 128 Wt rows of a
+// k-step, 32 KB), then per epilogue:
+//   store / SiLU: six stages; two output boxes per epilogue warp (ping-pong).
+//   res+rms: four stages (room for the residual boxes); per epilogue warp kXBufs boxes
 //     the residual rows are loaded into and one output box; then the row partial sums
 //     (one float per row and column half).
 // Then the barriers: full[S], empty[S], acc_full[2], acc_empty[2], done and, for res+rms,
-// one per residual box.
-//   SM pair: each CTA holds its 128 A rows and half of the 256 Wt rows of a k-step, 32 KB
-//     a stage, so six stages fit (four with the residual boxes).
-template <bool kRes, bool kPair>
+// one per residual box (full and acc_empty are used in the even CTA only).
+template <bool kRes>
 struct Layout {
-  static constexpr uint32_t kStageBytes = kABytes + (kPair ? kBBytes / 2 : kBBytes);
-  static constexpr int kStages = kRes ? (kPair ? 4 : 3) : (kPair ? 6 : 4);
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes / 2;
+  static constexpr int kStages = kRes ? 4 : 6;
   static constexpr uint32_t kOffBox = kStages * kStageBytes;
   static constexpr uint32_t kXBytes = kRes ? kEpiWarps * kXBufs * kBoxBytes : 0;
   static constexpr uint32_t kOutBoxes = kRes ? 1 : 2;
@@ -149,11 +155,11 @@ GR_DEVICE void box_bf16x16(uint8_t* box, int r, int half, const float* v) {
                    pack_bf16(v[8 * j + 4], v[8 * j + 5]), pack_bf16(v[8 * j + 6], v[8 * j + 7]));
 }
 
-template <int kEpi, bool kPair>
+template <int kEpi>
 __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__ Params P) {
   constexpr bool kRes = kEpi == kEpiResRms || kEpi == kEpiResRmsRel;
   constexpr bool kRel = kEpi == kEpiResRmsRel;
-  using L = Layout<kRes, kPair>;
+  using L = Layout<kRes>;
   constexpr int kStages = L::kStages;
   constexpr uint32_t kStageBytes = L::kStageBytes;
   constexpr int kHalves = kRes ? 2 : 1;  // 256-column blocks per tile
@@ -174,12 +180,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // rows per tile: 128, or 256 for an SM pair (CTA `rank` of the cluster holds rows
-  // [128 rank, 128 rank + 128) of each tile; the even CTA issues the MMAs)
-  constexpr int kTileRows = kPair ? 2 * BM : BM;
-  const int rank = kPair ? (int)cluster_ctarank() : 0;
-  const int first = kPair ? (int)cluster_idx() : (int)blockIdx.x;  // tiles first, +stride
-  const int stride = kPair ? (int)cluster_count() : (int)gridDim.x;
+  // CTA `rank` of the pair holds rows [128 rank, 128 rank + 128) of each tile; the even
+  // CTA issues the MMAs.  The pair runs tiles first, first + stride, ...
+  const int rank = (int)cluster_ctarank();
+  const int first = (int)cluster_idx();
+  const int stride = (int)cluster_count();
   const int row_off = rank * BM;  // this CTA's first row within a tile
 
   if (threadIdx.x == 0) {
@@ -189,8 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      // one arrival per epilogue warp (of both CTAs for a pair: the even CTA's barrier)
-      mbar_init(&acc_empty[b], kPair ? 2 * kEpiWarps : kEpiWarps);
+      // one arrival per epilogue warp of both CTAs (the even CTA's barrier is used)
+      mbar_init(&acc_empty[b], 2 * kEpiWarps);
     }
     mbar_init(done, 1);
     if (kRes)
@@ -208,15 +213,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     }
   }
   if (warp == 0) {
-    tmem_alloc<kPair>(tmem_slot, kTmemCols);
-    tmem_relinquish<kPair>();
+    tmem_alloc<true>(tmem_slot, kTmemCols);
+    tmem_relinquish<true>();
   }
   tc_fence_before();
-  // a pair: both CTAs' barriers are initialised before either signals the other's
-  if constexpr (kPair)
-    cluster_sync();
-  else
-    __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before either signals the other's
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int m_tiles = (g.M + kTileRows - 1) / kTileRows;
@@ -241,18 +242,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
             }
             if (lane == 0) {
               uint8_t* sa = smem + st * kStageBytes;
-              if constexpr (kPair) {
-                // both CTAs' tiles complete on the even CTA's barrier, which expects both
-                const uint32_t fb = cluster_addr(&full[st], 0);
-                if (rank == 0) mbar_expect_tx(&full[st], 2 * kStageBytes);
-                tma_load_2d_pair(sa, &P.ta, fb, ks * BK, mt * kTileRows + row_off);
-                tma_load_2d_pair(sa + kABytes, &P.tb, fb, ks * BK,
-                                 (nt + h) * BN + rank * (BN / 2));
-              } else {
-                mbar_expect_tx(&full[st], kStageBytes);
-                tma_load_2d(sa, &P.ta, &full[st], ks * BK, mt * BM);
-                tma_load_2d(sa + kABytes, &P.tb, &full[st], ks * BK, (nt + h) * BN);
-              }
+              // both CTAs' tiles complete on the even CTA's barrier, which expects both
+              const uint32_t fb = cluster_addr(&full[st], 0);
+              if (rank == 0) mbar_expect_tx(&full[st], 2 * kStageBytes);
+              tma_load_2d_pair(sa, &P.ta, fb, ks * BK, mt * kTileRows + row_off);
+              tma_load_2d_pair(sa + kABytes, &P.tb, fb, ks * BK, (nt + h) * BN + rank * (BN / 2));
             }
           }
         }
@@ -276,14 +270,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
         const int buf = kRes ? 0 : (tc & 1);
         const uint32_t ph_empty = kRes ? par(tc) ^ 1u : par(tc >> 1) ^ 1u;
         if (!kRes) {
-          if (!mbar_wait<kPair>(&acc_empty[buf], ph_empty, abort_flag, g.err)) break;
+          if (!mbar_wait<true>(&acc_empty[buf], ph_empty, abort_flag, g.err)) break;
           tc_fence_after();
         }
         for (int k0 = 0; k0 < ksteps && ok; k0 += kChunkSteps) {
           const int k1 = min(ksteps, k0 + kChunkSteps);
           for (int h = 0; h < kHalves && ok; ++h) {
             if (kRes && k0 == 0) {  // each half's columns are released on their own
-              if (!mbar_wait<kPair>(&acc_empty[h], ph_empty, abort_flag, g.err)) {
+              if (!mbar_wait<true>(&acc_empty[h], ph_empty, abort_flag, g.err)) {
                 ok = false;
                 break;
               }
@@ -302,31 +296,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
               for (int kk = 0; kk < BK / 16; ++kk) {
                 const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
                 const uint64_t bd = smem_desc_sw128(sa + kABytes + kk * 32, 16, 1024);
-                if constexpr (kPair)
-                  mma_bf16_ss_pair(acc, ad, bd, kIdescPair, (ks > 0 || kk > 0) ? 1u : 0u);
-                else
-                  mma_bf16_ss(acc, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                mma_bf16_ss_pair(acc, ad, bd, kIdesc, (ks > 0 || kk > 0) ? 1u : 0u);
               }
               // the stage (both CTAs' copies of it) is free once these MMAs have read it
-              if constexpr (kPair)
-                mma_commit_pair(&empty[st], 0x3);
-              else
-                mma_commit(&empty[st]);
+              mma_commit_pair(&empty[st], 0x3);
             }
-            if (ok && k1 == ksteps) {
-              if constexpr (kPair)
-                mma_commit_pair(&acc_full[kRes ? h : buf], 0x3);
-              else
-                mma_commit(&acc_full[kRes ? h : buf]);
-            }
+            if (ok && k1 == ksteps) mma_commit_pair(&acc_full[kRes ? h : buf], 0x3);
           }
         }
       }
       // every MMA issued has completed before TMEM is freed
-      if constexpr (kPair)
-        mma_commit_pair(done, 0x1);
-      else
-        mma_commit(done);
+      mma_commit_pair(done, 0x1);
       mbar_drain(done, 0);
     }
     __syncwarp();
@@ -339,13 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
     const int rloc = q * 32 + lane;  // row within the tile
     const int box_row = q * 32;      // + the CTA's first row of the tile: the warp's in C
     uint8_t* out = smem + L::kOffOut + ew * L::kOutBoxes * kBoxBytes;  // output boxes
-    // accumulator buffer b has been read by this warp (a pair: on the even CTA's barrier)
-    auto release_acc = [&](int b) {
-      if constexpr (kPair)
-        mbar_arrive_cluster(cluster_addr(&acc_empty[b], 0));
-      else
-        mbar_arrive(&acc_empty[b]);
-    };
+    // accumulator buffer b has been read by this warp (on the even CTA's barrier)
+    auto release_acc = [&](int b) { mbar_arrive_cluster(cluster_addr(&acc_empty[b], 0)); };
     if (!kRes) {
       int tc = 0;
       for (int t = first; t < tiles; t += stride, ++tc) {
@@ -584,14 +559,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_gemm_tc(const __grid_constant__
   if (warp >= 2 && lane == 0) bulk_wait_all();  // the output stores have landed
   __syncwarp();
   tc_fence_before();
-  // a pair: neither CTA leaves (or frees TMEM) while the other may still signal its
-  // barriers or the pair's MMAs read its shared memory
-  if constexpr (kPair)
-    cluster_sync();
-  else
-    __syncthreads();
+  // neither CTA leaves (or frees TMEM) while the other may still signal its barriers or
+  // the pair's MMAs read its shared memory
+  cluster_sync();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc<kPair>(tmem, kTmemCols);
+  if (warp == 0) tmem_dealloc<true>(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -681,12 +653,11 @@ static bool make_store_map(CUtensorMap* m, void* base, long long rows, int N, lo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int kEpi, bool kPair>
+template <int kEpi>
 static int launch_t(const GemmArgs& g, cudaStream_t st) {
   constexpr bool kRes = kEpi >= kEpiResRms;
   Params p;
-  if (!make_map(&p.ta, g.a, g.M, g.K, g.lda, BM) ||
-      !make_map(&p.tb, g.w, g.N, g.K, g.ldw, kPair ? BN / 2 : BN))
+  if (!make_map(&p.ta, g.a, g.M, g.K, g.lda, BM) || !make_map(&p.tb, g.w, g.N, g.K, g.ldw, BN / 2))
     return GENRANK_ERR_CUDA;
   if (kRes) {
     if (!make_store_map(&p.tx, g.x_out, g.M, g.N, g.ldx, true) ||
@@ -697,46 +668,38 @@ static int launch_t(const GemmArgs& g, cudaStream_t st) {
     return GENRANK_ERR_CUDA;
   }
   p.g = g;
-  constexpr int kSmem = (int)Layout<kRes, kPair>::kSmem;
+  constexpr int kSmem = (int)Layout<kRes>::kSmem;
   static DeviceOnce smem_attr;
-  if (!set_smem_limit_once(smem_attr, (const void*)k_gemm_tc<kEpi, kPair>, kSmem))
+  if (!set_smem_limit_once(smem_attr, (const void*)k_gemm_tc<kEpi>, kSmem))
     return GENRANK_ERR_CUDA;
   const int sms = sm_count_current();
   if (sms <= 0) return GENRANK_ERR_CUDA;
-  constexpr int kTileRows = kPair ? 2 * BM : BM;
   const long long tiles =
       (long long)((g.M + kTileRows - 1) / kTileRows) * (kRes ? 1 : g.N / BN);
-  if constexpr (!kPair) {
-    const int grid = (int)(tiles < sms ? tiles : sms);
-    k_gemm_tc<kEpi, false><<<grid, kThreads, kSmem, st>>>(p);
-  } else {
-    // clusters of two CTAs (one per SM of a pair), as many as can be resident at once
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmem;
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    static DeviceOnce pairs_once;
-    const int pairs = pairs_once.run([&](int) {
-      cudaLaunchConfig_t q = cfg;
-      q.gridDim = dim3(2 * (unsigned)(sms / 2));
-      int n = 0;
-      return cudaOccupancyMaxActiveClusters(&n, (const void*)k_gemm_tc<kEpi, true>, &q) ==
-                     cudaSuccess
-                 ? n
-                 : 0;
-    });
-    if (pairs <= 0) return GENRANK_ERR_CUDA;
-    cfg.gridDim = dim3(2 * (unsigned)(tiles < pairs ? tiles : pairs));
-    if (cudaLaunchKernelEx(&cfg, k_gemm_tc<kEpi, true>, p) != cudaSuccess)
-      return GENRANK_ERR_LAUNCH;
-  }
+  // clusters of two CTAs (one per SM of a pair), as many as can be resident at once
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static DeviceOnce pairs_once;
+  const int pairs = pairs_once.run([&](int) {
+    cudaLaunchConfig_t q = cfg;
+    q.gridDim = dim3(2 * (unsigned)(sms / 2));
+    int n = 0;
+    return cudaOccupancyMaxActiveClusters(&n, (const void*)k_gemm_tc<kEpi>, &q) == cudaSuccess
+               ? n
+               : 0;
+  });
+  if (pairs <= 0) return GENRANK_ERR_CUDA;
+  cfg.gridDim = dim3(2 * (unsigned)(tiles < pairs ? tiles : pairs));
+  if (cudaLaunchKernelEx(&cfg, k_gemm_tc<kEpi>, p) != cudaSuccess) return GENRANK_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
 }
 
@@ -746,11 +709,10 @@ int launch_gemm_tc(const GemmArgs& g, cudaStream_t st) {
   using namespace tg;
   if (g.M == 0) return GENRANK_OK;
   switch (g.epilogue) {
-    case kEpiStore: return launch_t<kEpiStore, true>(g, st);
-    case kEpiSilu: return launch_t<kEpiSilu, true>(g, st);
+    case kEpiStore: return launch_t<kEpiStore>(g, st);
+    case kEpiSilu: return launch_t<kEpiSilu>(g, st);
     case kEpiResRms:
-      return g.K >= kReleaseMinK ? launch_t<kEpiResRmsRel, true>(g, st)
-                                 : launch_t<kEpiResRms, true>(g, st);
+      return g.K >= kReleaseMinK ? launch_t<kEpiResRmsRel>(g, st) : launch_t<kEpiResRms>(g, st);
     default: return GENRANK_ERR_INVALID_ARG;
   }
 }

@@ -454,8 +454,21 @@ GR_DEVICE uint32_t par(int use) { return (uint32_t)(use & 1); }
 
 // Every lane waits (bounded), then the warp agrees, so that the warp stays
 // converged for the .sync.aligned tcgen05 instructions that follow.
+// A phase that has completed already (the usual case in the tile loop) is seen by a
+// non-blocking test; only a phase still open goes through the bounded wait.
+GR_DEVICE bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 GR_DEVICE bool wait_warp(uint64_t* bar, uint32_t ph, volatile int* abort_flag, int32_t* err) {
-  const bool ok = mbar_wait(bar, ph, abort_flag, err);
+  const bool ok = mbar_test(bar, ph) || mbar_wait(bar, ph, abort_flag, err);
   return __all_sync(0xffffffffu, ok);
 }
 

@@ -75,7 +75,7 @@ constexpr uint32_t kOffStage = kOffQTR + 2 * kCBBytes;       // O rows staged, 1
 constexpr uint32_t kOffML = kOffStage + BM * DH * 2;         // (m, l) per row, 2 buffers
 constexpr uint32_t kOffRec = kOffML + 2 * BM * 8;            // item record with each Q tile
 constexpr uint32_t kOffBar = kOffRec + 2 * 32;               // barriers
-constexpr uint32_t kNumBars = 17 + 3 * kStages;
+constexpr uint32_t kNumBars = 15 + 3 * kStages;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;        // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;        // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -129,8 +129,8 @@ struct CachedArgsHolder {
 };
 
 enum Bar {
-  kQFull = 0, kQEmpty = 2, kSFull = 4, kSFree = 6, kPFull = 8, kPFree = 10, kOFull = 12,
-  kOEmpty = 14, kDone = 16, kKFull = 17, kVFull = kKFull + kStages, kKVEmpty = kVFull + kStages
+  kQFull = 0, kQEmpty = 2, kSFull = 4, kPFull = 6, kPFree = 8, kOFull = 10, kOEmpty = 12,
+  kDone = 14, kKFull = 15, kVFull = kKFull + kStages, kKVEmpty = kVFull + kStages
 };
 static_assert(kKVEmpty + kStages <= (int)kNumBars, "barriers");
 
@@ -867,7 +867,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       mbar_init(&bars[kQFull + b], 1);
       mbar_init(&bars[kQEmpty + b], 1 + kSoftmaxWarps);  // last S commit + c_i reads
       mbar_init(&bars[kSFull + b], 1);
-      mbar_init(&bars[kSFree + b], kSoftmaxWarps);
       mbar_init(&bars[kPFull + b], kSoftmaxWarps);
       mbar_init(&bars[kPFree + b], 1);
       mbar_init(&bars[kOFull + b], 1 + kSoftmaxWarps);  // last P V commit + (m, l)
@@ -993,7 +992,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
       };
       auto issue_s = [&](const Cursor& t) -> bool {
         const int sb = t.g & 1, st = t.g % kStages, qb = t.qi & 1;
-        if (!mbar_wait(&bars[kSFree + sb], par(t.g >> 1) ^ 1u, abort_flag, a.err)) return false;
+        // the S buffer is free once the softmax has handed over the P it computed from it
+        if (!mbar_wait(&bars[kPFull + sb], par(t.g >> 1) ^ 1u, abort_flag, a.err)) return false;
         if (!mbar_wait(&bars[kKFull + st], par(t.g / kStages), abort_flag, a.err)) return false;
         tc_fence_after();
 #pragma unroll
@@ -1145,10 +1145,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
         if (!done) return false;
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bars[kSFree + sb]);
-          mbar_arrive(&bars[kPFull + sb]);
-        }
+        if (lane == 0) mbar_arrive(&bars[kPFull + sb]);  // P is ready and S has been read
         return true;
       };
       if constexpr (kDense) {  // one loop: peeling adds spills to this form's larger state

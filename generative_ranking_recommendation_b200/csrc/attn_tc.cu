@@ -57,9 +57,19 @@ constexpr int BN = 128;  // keys per tile
 constexpr int DH = 64;   // head dim
 constexpr int kThreads = 448;  // warp 0 MMA, 1 TMA, 2-9 softmax, 10-13 epilogue
 constexpr int kSoftmaxWarps = 8;  // barrier arrivals are one per warp
-constexpr int kStages = 5;     // K/V ring
+constexpr int kStages = 4;     // K/V ring
 constexpr uint32_t kTileBytes = BM * DH * 2;  // one Q, K or V tile (16 KB)
-constexpr uint32_t kCBBytes = BN * 4;         // column terms of one key tile
+constexpr uint32_t kCBBytes = BN * 4;         // fp32 terms (own column terms, key times) of a tile
+// The column term c_j enters S through the MMA: each key's row of the K tile is followed
+// by 16 more bf16 columns holding c_j / (scale log2 e) as three bf16 parts (the rest of
+// the 8-column row in memory zero, the next 8 columns read from the next key's row), and
+// each query row by 16 columns (1, 1, 1, 0, ...; zeros in the second 8), so that
+// S' = Q K^T + c_j / (scale log2 e) and x = S' scale log2 e - m.  The zeros meet the
+// next key's entry, which the prologue has written (every entry a key tile can read is
+// written on every call), so their products vanish.
+constexpr uint32_t kKABytes = BN * 16;        // one key tile's 8-column rows (2 KB)
+constexpr uint32_t kKAStride = kKABytes + 128;  // + a zeroed pad the last row's read reaches
+constexpr uint32_t kQABytes = 2 * BM * 16;    // the query side: 1, 1, 1 rows, then zeros
 constexpr float kOverflowSum = 1.2676506e30f;   // 2^100: a tile's row sum above this is redone
 constexpr float kUnderflowSum = 7.8886091e-31f;  // 2^-100: a first tile's row sum below this too
 
@@ -67,8 +77,9 @@ constexpr float kUnderflowSum = 7.8886091e-31f;  // 2^-100: a first tile's row s
 constexpr uint32_t kOffQ = 0;                                // 2 x 16 KB
 constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;           // kStages x 16 KB
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;     // kStages x 16 KB
-constexpr uint32_t kOffCB = kOffV + kStages * kTileBytes;    // kStages x 512 B
-constexpr uint32_t kOffQCB = kOffCB + kStages * kCBBytes;    // 2 x 512 B: the rows' own terms
+constexpr uint32_t kOffKA = kOffV + kStages * kTileBytes;    // kStages x (2 KB + pad)
+constexpr uint32_t kOffQA = kOffKA + kStages * kKAStride;    // 4 KB, written once
+constexpr uint32_t kOffQCB = kOffQA + kQABytes;              // 2 x 512 B: the rows' own terms
 constexpr uint32_t kOffTR = kOffQCB + 2 * kCBBytes;         // bucketed bias: key times, kStages x 512 B
 constexpr uint32_t kOffQTR = kOffTR + kStages * kCBBytes;    // bucketed bias: row times, 2 x 512 B
 constexpr uint32_t kOffStage = kOffQTR + 2 * kCBBytes;       // O rows staged, 16 KB
@@ -79,7 +90,9 @@ constexpr uint32_t kNumBars = 15 + 3 * kStages;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;        // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;        // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-static_assert(kOffStage % 16 == 0 && kOffTR % 16 == 0, "16-byte aligned bulk copies");
+static_assert(kOffStage % 16 == 0 && kOffTR % 16 == 0 && kOffKA % 128 == 0 &&
+                  kKAStride % 128 == 0 && kOffQA % 128 == 0,
+              "aligned bulk copies and MMA operands");
 
 // Bucketed time bias (the variant -m_p (p_i - p_j) - m_t bucket(t_i - t_j)):
 //   bucket(D) = min(62, floor(4 log2(D + 1))) for a gap of D >= 0 seconds.
@@ -103,6 +116,18 @@ constexpr uint32_t kColP = 256;  // two P buffers (bf16 pairs, 64 columns each)
 constexpr uint32_t kColO = 384;  // two O buffers (fp32, 64 columns each)
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);   // Q K-major, K K-major
+
+// Descriptor of a K-major operand without swizzle: core matrices of 8 rows x 16 bytes
+// (rows 16 bytes apart), sbo bytes between row groups, lbo bytes between the two 8-column
+// halves of a K = 16 slice.
+GR_DEVICE uint64_t smem_desc_plain(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100; layout type 0: no swizzle
+  return d;
+}
 constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, DH, 0, 1);  // P K-major (TMEM), V MN-major
 
 // scratch layout
@@ -121,6 +146,7 @@ struct Params {
   const int4* recs;      // [count][2] work records
   const int32_t* count;  // number of records
   const float* cbias;    // [H][Tp] column terms (log2 units)
+  const uint4* caug;     // [H][Tp] the same terms / (scale log2 e) as three bf16 parts
   long long Tp;
 };
 
@@ -189,6 +215,22 @@ __host__ __device__ inline long long scratch_tp_cached(long long T, int B) {
 // ------------------------------------------------------------------------------------------
 // prologue: work records (block B) and column terms (blocks 0..B-1)
 // ------------------------------------------------------------------------------------------
+// A column term c (log2 units) as the MMA adds it: q = c / (scale log2 e) split into
+// three bf16 parts (q - hi and q - hi - mid are exact in fp32, so the parts sum to q to
+// within about 2^-25 of it), in the first three of the entry's eight bf16 columns.
+GR_DEVICE uint4 cterm_parts(float c, float scale_log2) {
+  const float q = c / scale_log2;
+  const __nv_bfloat16 hi = __float2bfloat16_rn(q);
+  const float r1 = q - __bfloat162float(hi);
+  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+  return make_uint4((uint32_t)__bfloat16_as_ushort(hi) | ((uint32_t)__bfloat16_as_ushort(mid) << 16),
+                    (uint32_t)__bfloat16_as_ushort(lo), 0u, 0u);
+}
+GR_DEVICE void put_cterm(float* cbias, uint4* caug, long long at, float c, float scale_log2) {
+  cbias[at] = c;
+  caug[at] = cterm_parts(c, scale_log2);
+}
 constexpr int kMaxTileBuckets = 257;
 constexpr int kSchedThreads = 256;
 
@@ -230,12 +272,13 @@ GR_DEVICE int block_exclusive_scan(int v, int* excl, int* warp_sums) {
 __global__ void __launch_bounds__(kSchedThreads) k_prologue(const __grid_constant__ AttnArgs a,
                                                             int max_tiles, int4* recs,
                                                             int32_t* count, int32_t* uorder,
-                                                            float* cbias, int32_t* trel,
-                                                            long long Tp) {
+                                                            float* cbias, uint4* caug,
+                                                            int32_t* trel, long long Tp) {
   const int b = blockIdx.x;
   if (b < a.B) {
     const long long s = a.off[b], e = a.off[b + 1];
     if (s < 0 || e < s || e > a.T || !cbias) return;  // layout flagged by the schedule block
+    const float sl2 = a.scale * kLog2e;
     const int L = (int)(e - s);
     const long long base = seg_start(s, b);
     const long long t0 = L > 0 ? a.ts[s] : 0;
@@ -244,11 +287,13 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue(const __grid_constan
       const long long dtl = a.ts[s + i] - t0;
       if (trel) {
         trel[base + i] = (int)min(max(dtl, 0LL), (long long)kMaxRelTime - 1);
-        for (int h = 0; h < a.H; ++h) cbias[(long long)h * Tp + base + i] = kLog2e * (a.slope_pos[h] * p);
+        for (int h = 0; h < a.H; ++h)
+          put_cterm(cbias, caug, (long long)h * Tp + base + i, kLog2e * (a.slope_pos[h] * p), sl2);
       } else {
         const float dt = (float)dtl;
         for (int h = 0; h < a.H; ++h)
-          cbias[(long long)h * Tp + base + i] = kLog2e * (a.slope_pos[h] * p + a.slope_time[h] * dt);
+          put_cterm(cbias, caug, (long long)h * Tp + base + i,
+                    kLog2e * (a.slope_pos[h] * p + a.slope_time[h] * dt), sl2);
       }
     }
     // the entries up to the next user's segment (up to the end for the last user) are
@@ -257,7 +302,10 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue(const __grid_constan
     const long long next = b + 1 < a.B ? seg_start(e, b + 1) : Tp;
     for (long long i = base + L + threadIdx.x; i < next; i += blockDim.x) {
       if (trel) trel[i] = 0;
-      for (int h = 0; h < a.H; ++h) cbias[(long long)h * Tp + i] = 0.f;
+      for (int h = 0; h < a.H; ++h) {
+        cbias[(long long)h * Tp + i] = 0.f;
+        caug[(long long)h * Tp + i] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
     return;
   }
@@ -350,11 +398,12 @@ GR_DEVICE bool cached_user(const CachedAttnArgs& c, int u, int& cs, int& n, int&
 
 __global__ void __launch_bounds__(kSchedThreads) k_prologue_cached(
     const __grid_constant__ CachedArgsHolder ch, int max_tiles, int4* recs, int32_t* count,
-    int32_t* uorder, float* cbias, long long Tp) {
+    int32_t* uorder, float* cbias, uint4* caug, long long Tp) {
   const CachedAttnArgs& c = ch.c;
   const AttnArgs& a = c.a;
   const int b = blockIdx.x;
   if (b < a.B) {
+    const float sl2 = a.scale * kLog2e;
     int cs, n, m, hs;
     if (!cached_user(c, b, cs, n, m, hs)) return;  // flagged by the schedule block
     const int L = n + m;
@@ -378,7 +427,8 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue_cached(
       const float pf = (float)p, dt = (float)(t - t0);
       const long long at = base + (i < n ? i : n4 + (i - n));
       for (int h = 0; h < a.H; ++h)
-        cbias[(long long)h * Tp + at] = kLog2e * (a.slope_pos[h] * pf + a.slope_time[h] * dt);
+        put_cterm(cbias, caug, (long long)h * Tp + at,
+                  kLog2e * (a.slope_pos[h] * pf + a.slope_time[h] * dt), sl2);
     }
     // the padding after the history and the entries up to the next user's segment (up
     // to the end for the last user) are zeroed: the attention kernel relies on every
@@ -390,7 +440,10 @@ __global__ void __launch_bounds__(kSchedThreads) k_prologue_cached(
     }
     for (long long i = base + n + threadIdx.x; i < next; i += blockDim.x) {
       if (i >= base + n4 && i < base + n4 + m) continue;
-      for (int h = 0; h < a.H; ++h) cbias[(long long)h * Tp + i] = 0.f;
+      for (int h = 0; h < a.H; ++h) {
+        cbias[(long long)h * Tp + i] = 0.f;
+        caug[(long long)h * Tp + i] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
     return;
   }
@@ -537,11 +590,11 @@ GR_DEVICE void buckets4(const TB& tb, int c, uint64_t& b01, uint64_t& b23) {
   b23 = f2_sub(f2_pack(e[2], e[3]), base);
 }
 
-// x = s * scale + c_j (- m_t bucket for the bucketed bias) for CW columns (key kc0 + c of
-// the tile); keys at or beyond nvalid are masked.  Four independent running maxima
+// x = s * scale log2 e (- m_t bucket for the bucketed bias; s holds c_j already) for CW
+// columns (key kc0 + c of the tile); keys at or beyond nvalid are masked.  Four independent running maxima
 // shorten the chain.
 template <bool kMasked, bool kBucket, bool kDense>
-GR_DEVICE void row_max_chunk(const uint32_t (&s)[CW], const float* cb, const TB& tb,
+GR_DEVICE void row_max_chunk(const uint32_t (&s)[CW], const TB& tb,
                              const uint32_t* bw, int kc0, int nvalid, float scale_log2,
                              float (&mx4)[4]) {
 #pragma unroll
@@ -552,12 +605,8 @@ GR_DEVICE void row_max_chunk(const uint32_t (&s)[CW], const float* cb, const TB&
       bb[1] = kLog2e * bf16_hi(bw[c / 2]);
       bb[2] = kLog2e * bf16_lo(bw[c / 2 + 1]);
       bb[3] = kLog2e * bf16_hi(bw[c / 2 + 1]);
-    } else {
-      const float4 b4 = *reinterpret_cast<const float4*>(cb + c);
-      bb[0] = b4.x;
-      bb[1] = b4.y;
-      bb[2] = b4.z;
-      bb[3] = b4.w;
+    } else {  // the column term is in s already
+      bb[0] = bb[1] = bb[2] = bb[3] = 0.f;
     }
     if (kBucket) {
       uint64_t b01, b23;
@@ -580,11 +629,10 @@ GR_DEVICE void row_max_chunk(const uint32_t (&s)[CW], const float* cb, const TB&
 // bf16 pairs in pk.  The bias and scale arithmetic runs on column pairs (two-wide fp32
 // instructions).
 template <bool kMasked, bool kBucket, bool kDense>
-GR_DEVICE void exp_pack(const uint32_t (&s)[CW], const float* cb, const TB& tb,
+GR_DEVICE void exp_pack(const uint32_t (&s)[CW], const TB& tb,
                         const uint32_t* bw, int kc0, int nvalid, float scale_log2, float m_use,
                         uint64_t (&rs2)[2], uint32_t (&pk)[CW / 2]) {
   const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
-  const uint64_t m2 = f2_pack(m_use, m_use);
 #pragma unroll
   for (int c = 0; c < CW; c += 4) {
     uint64_t t01, t23;
@@ -592,10 +640,9 @@ GR_DEVICE void exp_pack(const uint32_t (&s)[CW], const float* cb, const TB& tb,
       const uint64_t l2e = f2_pack(kLog2e, kLog2e), nm2 = f2_pack(-m_use, -m_use);
       t01 = f2_fma(f2_pack(bf16_lo(bw[c / 2]), bf16_hi(bw[c / 2])), l2e, nm2);
       t23 = f2_fma(f2_pack(bf16_lo(bw[c / 2 + 1]), bf16_hi(bw[c / 2 + 1])), l2e, nm2);
-    } else {
-      const float4 b4 = *reinterpret_cast<const float4*>(cb + c);
-      t01 = f2_sub(f2_pack(b4.x, b4.y), m2);
-      t23 = f2_sub(f2_pack(b4.z, b4.w), m2);
+    } else {  // the column term is in s already
+      t01 = f2_pack(-m_use, -m_use);
+      t23 = t01;
     }
     if (kBucket) {
       uint64_t b01, b23;
@@ -628,12 +675,12 @@ GR_DEVICE void exp_pack(const uint32_t (&s)[CW], const float* cb, const TB& tb,
 // form keeps a select per key (its bias rows past a user's end are the caller's).  The
 // branches only compute, so the warp is converged again for the store.
 template <bool kMasked, bool kBucket, bool kDense, int kPOff = kHalf / 2>
-GR_DEVICE void exp_pack_store(uint32_t (&s)[CW], const float* cb, const TB& tb,
+GR_DEVICE void exp_pack_store(uint32_t (&s)[CW], const TB& tb,
                               const uint32_t* bw, int kc0, int nvalid, float scale_log2,
                               float m_use, uint64_t (&rs2)[2], uint32_t taddr) {
   uint32_t pk[CW / 2];
   if (kDense || !kMasked) {
-    exp_pack<kMasked, kBucket, kDense>(s, cb, tb, bw, kc0, nvalid, scale_log2, m_use, rs2, pk);
+    exp_pack<kMasked, kBucket, kDense>(s, tb, bw, kc0, nvalid, scale_log2, m_use, rs2, pk);
   } else if (kc0 >= nvalid) {
 #pragma unroll
     for (int k = 0; k < CW / 2; ++k) pk[k] = 0u;
@@ -643,15 +690,15 @@ GR_DEVICE void exp_pack_store(uint32_t (&s)[CW], const float* cb, const TB& tb,
       for (int e = 0; e < CW; ++e)
         if (kc0 + e >= nvalid) s[e] = 0xff800000u;  // -inf
     }
-    exp_pack<false, kBucket, kDense>(s, cb, tb, bw, kc0, nvalid, scale_log2, m_use, rs2, pk);
+    exp_pack<false, kBucket, kDense>(s, tb, bw, kc0, nvalid, scale_log2, m_use, rs2, pk);
   }
   p_store<kPOff>(taddr, pk);
 }
 
-// Maximum of x over this thread's half of the tile (S at s_addr, column terms of the
-// half at cb, first key kbase), CW columns at a time with the next chunk's load in flight.
+// Maximum of x over this thread's half of the tile (S at s_addr, first key kbase), CW
+// columns at a time with the next chunk's load in flight.
 template <bool kMasked, bool kBucket, bool kDense>
-GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, const TB& tb, const DB& db,
+GR_DEVICE float tile_max(uint32_t s_addr, const TB& tb, const DB& db,
                          int kbase, int nvalid, float scale_log2) {
   float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   uint32_t xa[CW], xb[CW];
@@ -670,11 +717,11 @@ GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, const TB& tb, const D
       }
     }
     s_load(s_addr + c0 + CW, xb);
-    row_max_chunk<kMasked, kBucket, kDense>(xa, cb + c0, tb.at(c0), bw, kbase + c0, nvalid,
+    row_max_chunk<kMasked, kBucket, kDense>(xa, tb.at(c0), bw, kbase + c0, nvalid,
                                             scale_log2, mx4);
     tmem_ld_wait(xb);
     if (c0 + 2 * CW < kHalf) s_load(s_addr + c0 + 2 * CW, xa);
-    row_max_chunk<kMasked, kBucket, kDense>(xb, cb + c0 + CW, tb.at(c0 + CW),
+    row_max_chunk<kMasked, kBucket, kDense>(xb, tb.at(c0 + CW),
                                             kDense ? bw + CW / 2 : bw, kbase + c0 + CW, nvalid,
                                             scale_log2, mx4);
     if (c0 + 2 * CW < kHalf) tmem_ld_wait(xa);
@@ -685,14 +732,13 @@ GR_DEVICE float tile_max(uint32_t s_addr, const float* cb, const TB& tb, const D
 // P = 2^(x - m) for this thread's half of the tile, written as bf16 pairs to the P
 // columns at p_addr; the stores have landed when it returns.  Returns the half's sum.
 template <bool kMasked, bool kBucket, bool kDense>
-GR_DEVICE float tile_exp(uint32_t s_addr, uint32_t p_addr, const float* cb, const TB& tb,
+GR_DEVICE float tile_exp(uint32_t s_addr, uint32_t p_addr, const TB& tb,
                          const DB& db, int kbase, int nvalid, float scale_log2, float m) {
   uint64_t rs2[2] = {0ull, 0ull};  // (+0, +0) pairs
   uint32_t xa[CW], xb[CW];
   if constexpr (kMasked && !kDense) {
     // the halves interleaved by chunks (see s_load_il); P lands in the same columns
     const int hh = kbase / kHalf;
-    const float* cbr = cb - kbase;  // the row's column terms
     const TB tbr = tb.at(-kbase);
     s_load_il(s_addr, xa);
     tmem_ld_wait(xa);
@@ -700,12 +746,12 @@ GR_DEVICE float tile_exp(uint32_t s_addr, uint32_t p_addr, const float* cb, cons
     for (int k = 0; k < 4; k += 2) {
       s_load_il(s_addr + 2 * CW * (k + 1), xb);
       const int ka = 2 * CW * k + CW * hh;
-      exp_pack_store<true, kBucket, false, CW / 2>(xa, cbr + ka, tbr.at(ka), nullptr, ka, nvalid,
+      exp_pack_store<true, kBucket, false, CW / 2>(xa, tbr.at(ka), nullptr, ka, nvalid,
                                                    scale_log2, m, rs2, p_addr + CW * k);
       tmem_ld_wait(xb);
       if (k + 2 < 4) s_load_il(s_addr + 2 * CW * (k + 2), xa);
       const int kb = 2 * CW * (k + 1) + CW * hh;
-      exp_pack_store<true, kBucket, false, CW / 2>(xb, cbr + kb, tbr.at(kb), nullptr, kb, nvalid,
+      exp_pack_store<true, kBucket, false, CW / 2>(xb, tbr.at(kb), nullptr, kb, nvalid,
                                                    scale_log2, m, rs2, p_addr + CW * (k + 1));
       if (k + 2 < 4) tmem_ld_wait(xa);
     }
@@ -730,11 +776,11 @@ GR_DEVICE float tile_exp(uint32_t s_addr, uint32_t p_addr, const float* cb, cons
       }
     }
     s_load(s_addr + c0 + CW, xb);
-    exp_pack_store<kMasked, kBucket, kDense>(xa, cb + c0, tb.at(c0), bw, kbase + c0, nvalid,
+    exp_pack_store<kMasked, kBucket, kDense>(xa, tb.at(c0), bw, kbase + c0, nvalid,
                                              scale_log2, m, rs2, p_addr + c0 / 2);
     tmem_ld_wait(xb);
     if (c0 + 2 * CW < kHalf) s_load(s_addr + c0 + 2 * CW, xa);
-    exp_pack_store<kMasked, kBucket, kDense>(xb, cb + c0 + CW, tb.at(c0 + CW),
+    exp_pack_store<kMasked, kBucket, kDense>(xb, tb.at(c0 + CW),
                                              kDense ? bw + CW / 2 : bw, kbase + c0 + CW, nvalid,
                                              scale_log2, m, rs2, p_addr + (c0 + CW) / 2);
     if (c0 + 2 * CW < kHalf) tmem_ld_wait(xa);
@@ -769,25 +815,25 @@ GR_DEVICE bool rescale_o(uint32_t o_addr, float alpha, uint64_t* prev_pv, uint32
 // offset max(m, tile max), rescaling O in TMEM.  Rows past the user's end never
 // redo (their output is not written).
 template <bool kMasked, bool kBucket, bool kDense>
-GR_DEVICE bool softmax_tile(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, const float* cb,
+GR_DEVICE bool softmax_tile(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr,
                             const TB& tb, const DB& bw, int kbase, int nvalid,
                             float scale_log2, bool first, bool row_ok, float& m, float& l,
                             uint64_t* prev_pv, uint32_t prev_ph, volatile int* abort_flag,
                             int32_t* err) {
-  float rs = tile_exp<kMasked, kBucket, kDense>(s_addr, p_addr, cb, tb, bw, kbase, nvalid,
+  float rs = tile_exp<kMasked, kBucket, kDense>(s_addr, p_addr, tb, bw, kbase, nvalid,
                                                 scale_log2, m);
   const float rs_row = rs + __shfl_xor_sync(0xffffffffu, rs, 16);
   const bool redo = row_ok && (!(rs_row <= kOverflowSum) || (first && rs_row < kUnderflowSum));
   if (__any_sync(0xffffffffu, redo)) {
     // every lane takes part in the .sync.aligned TMEM accesses; only redo rows move m
-    float mx = tile_max<kMasked, kBucket, kDense>(s_addr, cb, tb, bw, kbase, nvalid, scale_log2);
+    float mx = tile_max<kMasked, kBucket, kDense>(s_addr, tb, bw, kbase, nvalid, scale_log2);
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
     const float m_new = redo ? (first ? mx : fmaxf(m, mx)) : m;
     const float alpha = first ? 1.f : ex2(m - m_new);
     m = m_new;
     if (!first && !rescale_o(o_addr, alpha, prev_pv, prev_ph, abort_flag, err)) return false;
     l *= alpha;
-    rs = tile_exp<kMasked, kBucket, kDense>(s_addr, p_addr, cb, tb, bw, kbase, nvalid,
+    rs = tile_exp<kMasked, kBucket, kDense>(s_addr, p_addr, tb, bw, kbase, nvalid,
                                             scale_log2, m);
   }
   l = first ? rs : l + rs;
@@ -795,13 +841,13 @@ GR_DEVICE bool softmax_tile(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, c
 }
 
 // The diagonal tile: S = Q K^T over the item's own rows, of which a candidate row
-// keeps only its own key (position and time differences 0, so the bias is 0 and the
-// score is relative to c_i).  A warp's 16 rows have their own keys in one 16-key chunk
+// keeps only its own key (position and time differences 0, so the bias is 0: its S
+// holds c_i, and the score is relative to the offset).  A warp's 16 rows have their own keys in one 16-key chunk
 // of one half of the tile, so only that chunk is read (by the threads of that half) and
 // P is zero elsewhere.  The offset moves (O rescaled) only if the term would overflow,
 // or is set exactly on a first tile.
 GR_DEVICE bool softmax_diag(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, int rt, int h,
-                            bool cand_row, float rowcb, float scale_log2, bool first, float& m,
+                            bool cand_row, float scale_log2, bool first, float& m,
                             float& l, uint64_t* prev_pv, uint32_t prev_ph,
                             volatile int* abort_flag, int32_t* err, float diagb = 0.f) {
   const int r0 = rt & ~15;  // the warp's first row
@@ -814,7 +860,7 @@ GR_DEVICE bool softmax_diag(uint32_t s_addr, uint32_t p_addr, uint32_t o_addr, i
   float sv = 0.f;
 #pragma unroll
   for (int c = 0; c < 16; ++c) sv = e == c ? __uint_as_float(x[c]) : sv;
-  const float xm = mine ? fmaf(sv, scale_log2, rowcb + diagb) : -INFINITY;
+  const float xm = mine ? fmaf(sv, scale_log2, diagb) : -INFINITY;
   const float xr = fmaxf(xm, __shfl_xor_sync(0xffffffffu, xm, 16));  // the row's self score
   const bool move = xr > -INFINITY && (first || xr - m > 100.f);
   if (!first && __any_sync(0xffffffffu, move)) {
@@ -858,9 +904,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  const float* sCB = reinterpret_cast<const float*>(smem + kOffCB);
   float2* sML = reinterpret_cast<float2*>(smem + kOffML);  // [2][BM]: (m - c_i, l)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // the query side of the column-term MMA (rows 1, 1, 1, 0, ..., then 2 KB of zeros) and
+  // the pads after the key-side stages, read by the MMAs through the async proxy
+  if (!kDense) {
+    uint4* qa = reinterpret_cast<uint4*>(smem + kOffQA);
+    for (int i = threadIdx.x; i < (int)(kQABytes / 16); i += kThreads)
+      qa[i] = i < BM ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = threadIdx.x; i < kStages * 8; i += kThreads)
+      *reinterpret_cast<uint4*>(smem + kOffKA + (i >> 3) * kKAStride + kKABytes + (i & 7) * 16) =
+          make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < 2; ++b) {
@@ -918,8 +975,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
         ok = false;
         break;
       }
-      const float* cb_src = P.cbias + (long long)it.h * P.Tp + it.spad;  // history keys
-      const float* cbr_src = P.cbias + (long long)it.h * P.Tp + it.rb;   // query rows
+      const float* cbr_src = P.cbias + (long long)it.h * P.Tp + it.rb;  // query rows' c_i
+      const uint4* ka_src = P.caug + (long long)it.h * P.Tp + it.spad;  // history keys
+      const uint4* kar_src = P.caug + (long long)it.h * P.Tp + it.rb;   // the rows as keys
       const int32_t* tr_src = kBucket ? P.trel + it.spad : nullptr;
       if (lane == 0) {
         sRec[2 * qb] = make_int4(it.q0, it.n, it.L, it.nk);
@@ -946,12 +1004,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
           const int kv0 = hist ? (it.nk - 1 - j) * BN : it.q0;
           const int row = hist ? it.kb + kv0 : it.s + kv0;
           mbar_expect_tx(&bars[kKFull + st],
-                         kTileBytes + (kDense ? 0 : (kBucket ? 2 : 1) * kCBBytes));
+                         kTileBytes + (kDense ? 0 : kKABytes) + (kBucket ? kCBBytes : 0));
           tma_load_3d(smem + kOffK + st * kTileBytes, hist ? &P.tk : &P.tkc, &bars[kKFull + st],
                       0, it.h, row);
           if (!kDense)
-            bulk_load(smem + kOffCB + st * kCBBytes, hist ? cb_src + kv0 : cbr_src + kv0, kCBBytes,
-                      &bars[kKFull + st]);
+            bulk_load(smem + kOffKA + st * kKAStride, hist ? ka_src + kv0 : kar_src + kv0,
+                      kKABytes, &bars[kKFull + st]);
           if (kBucket)
             bulk_load(smem + kOffTR + st * kCBBytes, tr_src + kv0, kCBBytes, &bars[kKFull + st]);
           mbar_expect_tx(&bars[kVFull + st], kTileBytes);
@@ -982,7 +1040,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
     // before P_g V_g, so the softmax finds each S ready when it finishes the last one.
     if (lane == 0) {
       const uint32_t sQ = smem_u32(smem + kOffQ), sK = smem_u32(smem + kOffK),
-                     sV = smem_u32(smem + kOffV);
+                     sV = smem_u32(smem + kOffV), sQA = smem_u32(smem + kOffQA),
+                     sKA = smem_u32(smem + kOffKA);
       const int4* sRec = reinterpret_cast<const int4*>(smem + kOffRec);
       // number of tiles of the qi-th item (its Q tile has landed), or -1 at the end
       auto tiles = [&](int qi) -> int {
@@ -1001,6 +1060,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
           const uint64_t ad = smem_desc_sw128(sQ + qb * kTileBytes + k * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(sK + st * kTileBytes + k * 32, 16, 1024);
           mma_bf16_ss(tmem + kColS + sb * BN, ad, bd, kIdescS, k > 0 ? 1u : 0u);
+        }
+        if (!kDense) {  // + c_j / (scale log2 e): the query side's second 8 columns are zero
+          const uint64_t ad = smem_desc_plain(sQA, kQABytes / 2, 128);
+          const uint64_t bd = smem_desc_plain(sKA + st * kKAStride, 16, 128);
+          mma_bf16_ss(tmem + kColS + sb * BN, ad, bd, kIdescS, 1u);
         }
         mma_commit(&bars[kSFull + sb]);
         if (t.j == t.nt - 1) mma_commit(&bars[kQEmpty + qb]);
@@ -1112,9 +1176,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
           }
         }
         // S_g's commit also covers every MMA issued before it, P_{g-2} V_{g-2} included,
-        // so once S_g is here its P buffer is free as well
+        // so once S_g is here its P buffer is free as well; only the bucketed bias reads
+        // the key stage itself (the key times)
         if (!wait_warp(&bars[kSFull + sb], par(g >> 1), abort_flag, a.err) ||
-            !wait_warp(&bars[kKFull + st], par(g / kStages), abort_flag, a.err))
+            (kBucket && !wait_warp(&bars[kKFull + st], par(g / kStages), abort_flag, a.err)))
           return false;
         tc_fence_after();
         const uint32_t s_addr = lane_base + kColS + sb * BN;
@@ -1124,22 +1189,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_fwd_tc(const __grid_consta
         bool done;
         if (j < it.nk) {
           const int kv0 = (it.nk - 1 - j) * BN;  // most recent keys first
-          const float* cb = sCB + st * BN + kHalf * h;
           if (kBucket) tb.tr = sTR + st * BN + kHalf * h;
           if constexpr (kM) {
             // keys past the row's last visible key are masked (none on an unmasked tile)
             const int nvalid = max(0, min(BN, lim - kv0 + 1));
             done = softmax_tile<true, kBucket, kDense>(
-                s_addr, p_addr, o_addr, cb, tb, bw, kHalf * h, nvalid, scale_log2, j == 0,
+                s_addr, p_addr, o_addr, tb, bw, kHalf * h, nvalid, scale_log2, j == 0,
                 row_ok, m, l, prev_pv, prev_ph, abort_flag, a.err);
           } else {
             if (kv0 + BN - 1 > mask_from) flag(a.err, GENRANK_DERR_LAYOUT);  // not reachable
             done = softmax_tile<false, kBucket, kDense>(
-                s_addr, p_addr, o_addr, cb, tb, bw, kHalf * h, BN, scale_log2, j == 0,
+                s_addr, p_addr, o_addr, tb, bw, kHalf * h, BN, scale_log2, j == 0,
                 row_ok, m, l, prev_pv, prev_ph, abort_flag, a.err);
           }
         } else {
-          done = softmax_diag(s_addr, p_addr, o_addr, rt, h, cand_row, rowcb, scale_log2,
+          done = softmax_diag(s_addr, p_addr, o_addr, rt, h, cand_row, scale_log2,
                               j == 0, m, l, prev_pv, prev_ph, abort_flag, a.err, diagb);
         }
         if (!done) return false;
@@ -1291,9 +1355,11 @@ static size_t users_bytes(int B) { return ((size_t)B * 4 + 15) / 16 * 16; }
 
 size_t attn_fwd_tc_workspace(int B, long long T, int H, int max_seqlen) {
   using namespace tc;
-  // records, user order, column terms [H][Tp] and (bucketed bias) token times [Tp]
+  // records, user order, column terms [H][Tp], (bucketed bias) token times [Tp] and the
+  // column terms in the MMA's form [H][Tp] x 16 B
   return kHeaderBytes + recs_bytes(B, max_seqlen) + users_bytes(B) +
-         (size_t)(H + 1) * scratch_tp(T, B) * sizeof(float);
+         (size_t)(H + 1) * scratch_tp(T, B) * sizeof(float) +
+         (size_t)H * scratch_tp(T, B) * sizeof(uint4);
 }
 
 int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
@@ -1321,8 +1387,10 @@ int launch_attn_fwd_tc(const AttnArgs& a, cudaStream_t st) {
   const bool bucket = a.time_bias == kTimeBiasBucketed;
   int32_t* trel = bucket ? (int32_t*)(cbias + (size_t)a.H * p.Tp) : nullptr;
   p.trel = trel;
-  k_prologue<<<a.B + 1, kSchedThreads, 0, st>>>(a, max_tiles, recs, count, uorder, cbias, trel,
-                                                p.Tp);
+  uint4* caug = (uint4*)(cbias + (size_t)(a.H + 1) * p.Tp);
+  p.caug = caug;
+  k_prologue<<<a.B + 1, kSchedThreads, 0, st>>>(a, max_tiles, recs, count, uorder, cbias, caug,
+                                                trel, p.Tp);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   p.dbias = nullptr;
   p.Lpad = 0;
@@ -1350,12 +1418,13 @@ int launch_attn_fwd_dense(const AttnArgs& a, const void* bias, long long Lpad, c
   p.count = count;
   p.recs = recs;
   p.cbias = cbias;  // not read by the dense-bias kernel
+  p.caug = nullptr;
   p.Tp = scratch_tp(a.T, a.B);
   p.trel = nullptr;
   p.dbias = (const __nv_bfloat16*)bias;
   p.Lpad = Lpad;
   k_prologue<<<a.B + 1, kSchedThreads, 0, st>>>(a, max_tiles_of(a.max_seqlen), recs, count,
-                                                uorder, nullptr, nullptr, p.Tp);
+                                                uorder, nullptr, nullptr, nullptr, p.Tp);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   return launch_kernel(p, kDenseBiasMode, st);
 }
@@ -1363,7 +1432,7 @@ int launch_attn_fwd_dense(const AttnArgs& a, const void* bias, long long Lpad, c
 size_t attn_fwd_cached_workspace(int B, long long C, long long Th, int H, int max_cand) {
   using namespace tc;
   return kHeaderBytes + recs_bytes(B, max_cand) + users_bytes(B) +
-         (size_t)H * scratch_tp_cached(C + Th, B) * sizeof(float);
+         (size_t)H * scratch_tp_cached(C + Th, B) * (sizeof(float) + sizeof(uint4));
 }
 
 int launch_attn_fwd_cached(const CachedAttnArgs& c, cudaStream_t st) {
@@ -1394,9 +1463,11 @@ int launch_attn_fwd_cached(const CachedAttnArgs& c, cudaStream_t st) {
   p.recs = recs;
   p.cbias = cbias;
   p.Tp = scratch_tp_cached(a.T + c.Th, a.B);
+  uint4* caug = (uint4*)(cbias + (size_t)a.H * p.Tp);
+  p.caug = caug;
   CachedArgsHolder holder{c};
   k_prologue_cached<<<a.B + 1, kSchedThreads, 0, st>>>(holder, max_tiles_of(c.max_cand), recs,
-                                                       count, uorder, cbias, p.Tp);
+                                                       count, uorder, cbias, caug, p.Tp);
   if (cudaGetLastError() != cudaSuccess) return GENRANK_ERR_LAUNCH;
   p.trel = nullptr;
   p.dbias = nullptr;

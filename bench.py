@@ -702,11 +702,12 @@ def run_native(args, cfg, world, rank, local):
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         # per step: metadata scan + gather-sum (with the first RMSNorm on the fused
         # blocks), attention prologue + kernel per layer, on the fused blocks the four
-        # linear layers per layer (QKV, W_o, W1, W2), and for training the backward's five
+        # linear layers per layer (QKV, W_o, W1, W2) and the last layer's two candidate-row
+        # gathers, and for training the backward's five
         # kernels per layer plus the embedding backward; a one-block model without FFN
         # adds the fused candidate head
         "gpu_launches": args.steps * (2 + 2 * cfg.layers + (5 * cfg.layers + 1 if training else 0)
-                                      + (4 * cfg.layers if (gm.fused_blocks and not training)
+                                      + (4 * cfg.layers + 2 if (gm.fused_blocks and not training)
                                          else 0)
                                       + (0 if (cfg.ffn or cfg.layers > 1 or training) else 1)),
         "clocks": clocks,

@@ -280,6 +280,28 @@ int genrank_candidate_logits(int M, const int64_t* rows, int64_t T, int d, const
   return launch_cand_logits(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int genrank_gather_rows(int64_t M, const int64_t* rows, int64_t T, int64_t row_bytes,
+                        const void* src, int64_t src_stride, void* dst, int64_t dst_stride,
+                        int32_t* dev_err, genrank_stream_t stream) {
+  if (M < 0 || T < 0 || row_bytes <= 0 || row_bytes % 16 || !dev_err)
+    return GENRANK_ERR_INVALID_ARG;
+  if (M == 0) return GENRANK_OK;
+  if (!rows || !src || !dst || src_stride < row_bytes || dst_stride < row_bytes ||
+      src_stride % 16 || dst_stride % 16 || !aligned16(src) || !aligned16(dst))
+    return GENRANK_ERR_INVALID_ARG;
+  GatherRowsArgs a;
+  a.M = M;
+  a.rows = rows;
+  a.T = T;
+  a.row_bytes = row_bytes;
+  a.src = src;
+  a.src_stride = src_stride;
+  a.dst = dst;
+  a.dst_stride = dst_stride;
+  a.err = dev_err;
+  return launch_gather_rows(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t genrank_attn_workspace_size(int B, int64_t T, int H, int dh, int max_seqlen, int is_bwd) {
   if (B < 1 || T < 0 || H < 1 || dh < 1 || max_seqlen < 0) return 0;
   if (is_bwd) {

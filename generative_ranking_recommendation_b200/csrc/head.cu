@@ -1,6 +1,8 @@
-// Candidate logits of a one-block scorer without FFN: z = x . w + o . u at
-// candidate rows ("GenRank [2025]" chapter notes §1.3.1: the output lives at
-// candidate positions; u = W_o w_head is formed by the caller).
+// Candidate-side helpers ("GenRank [2025]" chapter notes §1.3.1: the loss and the
+// ranking output live at candidate positions):
+//   * the logits of a one-block scorer without FFN, z = x . w + o . u at candidate rows
+//     (u = W_o w_head is formed by the caller);
+//   * the gather of candidate rows that the last block's projections and FFN run on.
 #include "common.cuh"
 #include "host_util.h"
 #include "kernels.h"
@@ -61,6 +63,38 @@ int launch_cand_logits(const CandLogitsArgs& a, cudaStream_t st) {
     k_cand_logits<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
   else
     k_cand_logits<float><<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
+}
+
+// dst row k = src row rows[k], whole rows of row_bytes (a multiple of 16): one warp per
+// row, each lane moving 16-byte vectors.  A row index outside [0, T) is flagged and its
+// destination row zeroed.
+__global__ void __launch_bounds__(256) k_gather_rows(const GatherRowsArgs a) {
+  const int lane = threadIdx.x & 31;
+  const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+  const long long vecs = a.row_bytes / 16;
+  for (long long k = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); k < a.M;
+       k += nwarps) {
+    const long long row = a.rows[k];
+    uint4* d = reinterpret_cast<uint4*>(static_cast<uint8_t*>(a.dst) + k * a.dst_stride);
+    if (row < 0 || row >= a.T) {
+      if (lane == 0) flag(a.err, GENRANK_DERR_INDEX);
+      for (long long v = lane; v < vecs; v += 32) d[v] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const uint4* s =
+        reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.src) + row * a.src_stride);
+    for (long long v = lane; v < vecs; v += 32) d[v] = __ldg(s + v);
+  }
+}
+
+int launch_gather_rows(const GatherRowsArgs& a, cudaStream_t st) {
+  if (a.M == 0) return GENRANK_OK;
+  const int n = sm_count_current();
+  const int sms = n > 0 ? n : 148;  // only sizes the grid
+  const long long blocks = (a.M + 7) / 8;
+  const int grid = (int)(blocks < 16LL * sms ? blocks : 16LL * sms);
+  k_gather_rows<<<grid, 256, 0, st>>>(a);
   return cudaGetLastError() == cudaSuccess ? GENRANK_OK : GENRANK_ERR_LAUNCH;
 }
 

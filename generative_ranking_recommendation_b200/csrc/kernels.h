@@ -170,6 +170,19 @@ struct CandLogitsArgs {
 
 int launch_cand_logits(const CandLogitsArgs& a, cudaStream_t st);
 
+struct GatherRowsArgs {
+  long long M;
+  const int64_t* rows;
+  long long T;
+  long long row_bytes;   // a multiple of 16
+  const void* src;
+  long long src_stride;  // bytes
+  void* dst;
+  long long dst_stride;  // bytes
+  int32_t* err;
+};
+int launch_gather_rows(const GatherRowsArgs& a, cudaStream_t st);
+
 int launch_embed_fwd(const EmbedFwdArgs& a, cudaStream_t st);
 int launch_embed_bwd(const EmbedBwdArgs& a, cudaStream_t st);
 

@@ -32,7 +32,7 @@ EXPORTS = (
     "genrank_attn_fwd_static", "genrank_candidate_logits", "genrank_attn_fwd_cached",
     "genrank_attn_cached_workspace_size", "genrank_attn_fwd_bucketed",
     "genrank_attn_bwd_bucketed", "genrank_attn_fwd_dense_bias", "genrank_linear",
-    "genrank_linear_residual_rmsnorm", "genrank_rmsnorm",
+    "genrank_linear_residual_rmsnorm", "genrank_rmsnorm", "genrank_gather_rows",
 )
 EPI_STORE, EPI_SILU = 0, 1
 
@@ -108,6 +108,8 @@ def lib():
         L.genrank_candidate_logits.restype = _I
         L.genrank_candidate_logits.argtypes = [
             _I, _P, _L, _I, _P, _L, _P, _L, _I, _P, _P, _P, _P, _P]
+        L.genrank_gather_rows.restype = _I
+        L.genrank_gather_rows.argtypes = [_L, _P, _L, _L, _P, _L, _P, _L, _P, _P]
         L.genrank_attn_fwd_cached.restype = _I
         L.genrank_attn_fwd_cached.argtypes = [
             _I, _L, _P, _I, _P, _P, _P, _L, _L, _P, _P, _P, _L, _P, _P, _P, _I, _I, _P, _P, _F,
@@ -303,6 +305,21 @@ def candidate_logits(rows, x, o, w, u, z, dev_err, stream=None):
         int(x.stride(0)), _ptr(o), int(o.stride(0)), _dtype_code(x), _ptr(w), _ptr(u), _ptr(z),
         _ptr(dev_err), _stream(stream))
     _check(rc, "genrank_candidate_logits")
+
+
+def gather_rows(rows, src, dst, dev_err, stream=None):
+    """genrank_gather_rows: dst[k] = src[rows[k]] for 2-D tensors of one element type
+    whose rows are contiguous; dst has rows.numel() rows."""
+    if src.dtype != dst.dtype or src.dim() != 2 or dst.dim() != 2 or src.shape[1] != dst.shape[1]:
+        raise GenRankError("gather_rows: src and dst must be 2-D of one dtype and width")
+    if src.stride(1) != 1 or dst.stride(1) != 1 or dst.shape[0] != rows.numel():
+        raise GenRankError("gather_rows: contiguous rows, one dst row per index")
+    es = src.element_size()
+    rc = lib().genrank_gather_rows(
+        int(rows.numel()), _ptr(rows), int(src.shape[0]), int(src.shape[1]) * es, _ptr(src),
+        int(src.stride(0)) * es, _ptr(dst), int(dst.stride(0)) * es, _ptr(dev_err),
+        _stream(stream))
+    _check(rc, "genrank_gather_rows")
 
 
 def attn_cached_workspace_size(B, C, Th, H, dh, max_cand) -> int:

@@ -222,7 +222,11 @@ class GenRankModel:
                 ev[1].record()
             if li == nl - 1:  # only candidate rows reach the head
                 rows = db.cand_rows
-                o, x = o.index_select(0, rows), x.index_select(0, rows)
+                oc = torch.empty((rows.numel(), d), dtype=o.dtype, device=dev)
+                xc = torch.empty((rows.numel(), d), dtype=x.dtype, device=dev)
+                G.gather_rows(rows, o, oc, self.err)
+                G.gather_rows(rows, x, xc, self.err)
+                o, x = oc, xc
             a2 = torch.empty_like(o)
             G.linear_residual_rmsnorm(o, W["WoT"], x, x, a2, self.err, eps=RMS_EPS)
             u = self._linear(a2, W["W1T"], G.EPI_SILU)

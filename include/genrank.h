@@ -378,6 +378,20 @@ int genrank_candidate_logits(int M, const int64_t *rows, int64_t T, int d, const
                              const float *w, const float *u, float *z, int32_t *dev_err,
                              genrank_stream_t stream);
 
+/* The candidate rows of a token matrix, gathered into a dense one: only candidate rows
+ * reach the ranking output (huaxiaozhuan "GenRank [2025]" §1.3.1), so the last block's
+ * output projection, residual and FFN run on them alone.
+ *   dst [M] rows: dst row k = src row rows[k], row_bytes bytes each (a byte copy, so
+ *   any element type), src rows src_stride bytes apart, dst rows dst_stride apart.
+ * Arguments: M >= 0; rows [M] int64 in [0, T) (device); row_bytes > 0 and the strides
+ * multiples of 16, strides >= row_bytes; src, dst 16-byte aligned device pointers that
+ * do not overlap.  The caller owns every buffer.  A row outside [0, T) sets
+ * GENRANK_DERR_INDEX and zeroes its destination row.  Returns GENRANK_ERR_INVALID_ARG
+ * for invalid sizes or alignment, before any launch. */
+int genrank_gather_rows(int64_t M, const int64_t *rows, int64_t T, int64_t row_bytes,
+                        const void *src, int64_t src_stride, void *dst, int64_t dst_stride,
+                        int32_t *dev_err, genrank_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * The blocks around the attention, on tensor cores with fused epilogues.
  * huaxiaozhuan "GenRank [2025]" §1.4.1 and fun-rec §7.2.1: the action-oriented layout

@@ -109,6 +109,25 @@ def test_host_side_argument_checks_return_before_launch(L):
     assert r == 2  # 80 time buckets: beyond what the integer bucket supports
 
 
+def test_gather_rows_host_checks(L):
+    """The candidate-row gather rejects bad sizes and alignment on the host."""
+    P = ctypes.c_void_p
+    fake = P(0x10000)  # never dereferenced: every call below fails its host checks
+
+    def call(M=4, rows=fake, T=10, rb=1024, src=fake, ss=1024, dst=fake, ds=1024, err=fake):
+        return L.genrank_gather_rows(M, rows, T, rb, src, ss, dst, ds, err, None)
+
+    assert call(M=-1) == 1
+    assert call(rb=0) == 1
+    assert call(rb=24, ss=32, ds=32) == 1  # not a multiple of 16 bytes
+    assert call(ss=512) == 1  # src stride shorter than a row
+    assert call(ds=1040 + 8) == 1  # dst stride not a multiple of 16
+    assert call(src=P(0x10008)) == 1  # misaligned
+    assert call(rows=None) == 1
+    assert call(err=None) == 1
+    assert call(M=0, rows=None, src=None, dst=None) == 0  # nothing to do
+
+
 def test_backward_workspace_covers_its_regions(L):
     """The backward scratch holds the fp32 dQ accumulator [T, H, 64], three fp32 per-row
     arrays [H, T] (column term, log2 LSE, D) and an 8-byte record per token."""

@@ -680,7 +680,9 @@ def run_native(args, cfg, world, rank, local):
                     "peak_source": burst_src, "traffic": measured_traffic(cfg.name),
                     "algorithmic_flops_per_launch": flops, "avg_launch_ms": attn_avg_ms,
                     "note": "one layer's attention call (prologue + kernel) timed alone on its "
-                            "own graph; avg_launch_ms includes the prologue"}
+                            "own graph; avg_launch_ms includes the prologue.  On the fused "
+                            "four-layer step the W2 linear layer's kernel has about the same "
+                            "share of device time (its line is in kernels)"}
         emb_ms = float(np.mean(embed_ms))
         gbs = embed_bytes(T_avg, cfg.d, es) / (emb_ms / 1e3) / 1e9
         embed_line = {"kernel": "k_token_meta + k_embed_fwd (genrank_embed_assemble)",

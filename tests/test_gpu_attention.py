@@ -323,6 +323,26 @@ def test_bwd_c2_shapes(G):
     _check_grads(cfg, got, want, np.arange(batch.T), qkv, dO, batch, pos)
 
 
+def test_fwd_year_long_histories(G):
+    """Histories stretched to about a year: with the linear time slope the column terms
+    reach thousands of log2 units, and they enter the scores through the MMA as three
+    bf16 parts of c / (scale log2 e) summed in fp32 next to q.k.  The softmax of each
+    row still matches the oracle."""
+    cfg = CONFIGS["c1"].with_(B=6)
+    batch = make_batch(cfg, hist_override=[300, 20, 500, 129, 1, 64])
+    for u in range(batch.B):
+        s, e = batch.seq_offsets[u], batch.seq_offsets[u + 1]
+        t = batch.ts[s:e]
+        span = max(int(t[-1] - t[0]), 1)
+        batch.ts[s:e] = t[0] + (t - t[0]) * (31_536_000 // span)  # order kept
+    pos, _, _ = ref.meta(batch)
+    qkv = make_qkv(cfg, batch.T, seed=41)
+    O, L = run_fwd(G, cfg, batch, pos, qkv)
+    Or, Lr = ref.attn(qkv[:, 0], qkv[:, 1], qkv[:, 2], batch, pos)
+    assert np.all(np.isfinite(O)) and np.all(np.isfinite(L))
+    _check(cfg, O, L, Or, Lr, np.arange(batch.T))
+
+
 def test_fwd_older_keys_dominating_take_the_exact_path(G):
     """Keys are visited most recent first; when much older keys score far higher
     (beyond 2^100 in a row sum), the tile is recomputed with an exact offset."""

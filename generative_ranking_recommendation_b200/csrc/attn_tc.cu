@@ -10,23 +10,26 @@
 //     number of 128-key tiles they visit (longest first), and writes the ALiBi
 //     column term c_j = log2(e) (m_h p_j + m_t,h (t_j - t_0)) for every token and
 //     head into a 16-byte aligned scratch layout (entries between users' segments are
-//     zeroed, so every term a key tile reads is finite).  On visible pairs p_i >= p_j
-//     and t_i >= t_j, so the bias is c_j - c_i; c_i cancels in the softmax and only c_j
-//     is added per element; the literal LSE subtracts c_i in the epilogue.
+//     zeroed, so every term a key tile reads is finite), in fp32 and as three bf16 parts
+//     of c_j / (scale log2 e).  On visible pairs p_i >= p_j and t_i >= t_j, so the bias
+//     is c_j - c_i; c_i cancels in the softmax (it is the row's fixed offset), c_j is
+//     added by the MMA that forms S, and the literal LSE subtracts c_i in the epilogue.
 //   * A persistent grid walks the records round-robin (one head per work item).  An
 //     item visits its history key tiles (history tile t: key tiles 0..t; candidate
 //     rows: the history only; most recent keys first) and, when it holds candidate
 //     rows, one diagonal tile: its own rows as keys, of which only each candidate's
 //     own key (bias 0) is kept.  Key tiles a query tile never sees are never visited.
 //   * Warp 1 issues TMA loads (Q with the rows' own column terms, double-buffered;
-//     K, V and their column terms in a five-stage ring; 128B swizzle, no multicast).
-//   * Warp 0 (one thread) issues tcgen05.mma: S = Q K^T (128 x 128, fp32) into one
-//     of two TMEM buffers, the next S before the current P V, and O += P V (128 x 64,
+//     K, V and the keys' split column terms in a four-stage ring; 128B swizzle, no
+//     multicast).
+//   * Warp 0 (one thread) issues tcgen05.mma: S = Q K^T + c_j / (scale log2 e) (128 x
+//     128, fp32; a fifth K = 16 slice adds the split column terms) into one of two TMEM
+//     buffers, the next S before the current P V, and O += P V (128 x 64,
 //     fp32) into the item's TMEM O buffer (two, alternating by item), P (bf16 pairs)
 //     read from one of two TMEM P buffers.
 //   * Warps 2-9 stream the softmax with two threads per query row, each on one half
 //     of the key columns (TMEM access shape 16x32bx2), so two softmax warps share
-//     each SM sub-partition: bias, mask and exponentials in one pass per tile, with
+//     each SM sub-partition: offset, mask and exponentials in one pass per tile, with
 //     the offset fixed at the row's own column term (every visible key has
 //     c_j <= c_i); a tile whose row sum leaves the safe range is redone exactly and O
 //     rescaled in TMEM.  Only an item's first tile can need the row mask: it runs

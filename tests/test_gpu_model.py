@@ -114,3 +114,26 @@ def test_fused_blocks_match_torch_blocks(M, name):
     from generative_ranking_recommendation_b200 import genrank as G
 
     assert G.check_error(gm.err) == 0
+
+
+def test_train_step_gradient_tables_start_clean(M):
+    """The gradient tables are reused across steps, the previous step's item rows zeroed:
+    a second step's tables equal those of a model that ran only that step, and item rows
+    only the first batch touched are exactly zero."""
+    cfg = CONFIGS["c3"].with_(B=4, n_item=50_000)
+    model = make_model(cfg)
+    b1, b2 = make_batch(cfg, seed=101), make_batch(cfg, seed=202)
+    gm = M.GenRankModel(cfg, model, "cuda")
+    gm.train_step(M.DeviceBatch.from_batch(b1, "cuda"))
+    _, _, g2 = gm.train_step(M.DeviceBatch.from_batch(b2, "cuda"))
+    g2 = {k: v.cpu().numpy().astype(np.float64) for k, v in g2.items()}
+    fresh = M.GenRankModel(cfg, model, "cuda")
+    _, _, gf = fresh.train_step(M.DeviceBatch.from_batch(b2, "cuda"))
+    gf = {k: v.cpu().numpy().astype(np.float64) for k, v in gf.items()}
+    from generative_ranking_recommendation_b200 import genrank as G
+
+    assert G.check_error(gm.err) == 0 and G.check_error(fresh.err) == 0
+    for k in g2:  # equal up to the order of the atomic additions
+        assert ref.rel_to_max(g2[k], gf[k]) <= 1e-4, k
+    only1 = np.setdiff1d(np.unique(b1.item_ids), np.unique(b2.item_ids))
+    assert only1.size > 0 and not g2["item"][only1].any()

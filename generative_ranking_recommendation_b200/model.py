@@ -171,7 +171,8 @@ class GenRankModel:
 
     @staticmethod
     def rms(x):
-        return x * torch.rsqrt((x * x).mean(dim=-1, keepdim=True) + RMS_EPS)
+        # x / sqrt(mean(x^2) + eps), unit gain, as one torch kernel
+        return torch.nn.functional.rms_norm(x, (x.shape[-1],), eps=RMS_EPS)
 
     # -------------------------------------------------------------------------------------
     def _event(self, attn_events):

@@ -282,16 +282,16 @@ class GenRankModel:
             if li == nl - 1:
                 rows = db.cand_rows
                 base = x.index_select(0, rows)
-                h = base + (o.index_select(0, rows) @ W["Wo"]).float()
+                h = base + (o.index_select(0, rows) @ W["Wo"])
                 if ffn:
                     f = self.rms(h).to(self.dtype)
-                    h = h + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"]).float()
+                    h = h + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"])
                     h = self.rms(h)
                 return h @ self.w_head
-            x = x + (o @ W["Wo"]).float()
+            x = x + (o @ W["Wo"])  # the add promotes the bf16 product to fp32 exactly
             if ffn:
                 f = self.rms(x).to(self.dtype)
-                x = x + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"]).float()
+                x = x + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"])
         raise ValueError("a model needs at least one layer")
 
     # -------------------------------------------------------------------------------------
@@ -330,17 +330,17 @@ class GenRankModel:
             o = _Attn.apply(qkv)
             if li == nl - 1:  # only candidate rows reach the loss
                 rows = db.cand_rows
-                h = x.index_select(0, rows) + (o.index_select(0, rows) @ W["Wo"]).float()
+                h = x.index_select(0, rows) + (o.index_select(0, rows) @ W["Wo"])
                 if ffn:
                     f = self.rms(h).to(self.dtype)
-                    h = h + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"]).float()
+                    h = h + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"])
                     h = self.rms(h)
                 z = h @ self.w_head
                 break
-            x = x + (o @ W["Wo"]).float()
+            x = x + (o @ W["Wo"])  # the add promotes the bf16 product to fp32 exactly
             if ffn:
                 f = self.rms(x).to(self.dtype)
-                x = x + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"]).float()
+                x = x + (torch.nn.functional.silu(f @ W["W1"]) @ W["W2"])
         loss = torch.nn.functional.binary_cross_entropy_with_logits(z, db.labels)
         loss.backward()
         dE = Eg.grad.to(self.dtype).contiguous()
